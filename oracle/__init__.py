@@ -1,0 +1,209 @@
+"""CPU oracle for the top-1 sigmoid-gated MoE feed-forward layer.
+
+TEST INFRASTRUCTURE ONLY.  Only ``tests/``, ``__graft_entry__.smoke()`` and the
+``cpu_baseline`` / reference legs of ``bench.py`` may import this package.  The
+product path (the CUDA library and its Python binding) never imports, links or
+calls anything here, and this package imports nothing from the product.
+
+The arithmetic lives in ``oracle.c`` (plain C, fp64 accumulation, OpenMP over
+tokens); this module only compiles it with gcc and marshals numpy arrays.
+Inputs are numpy arrays in their storage dtype: float32, bf16 as uint16 bit
+patterns, E4M3 as uint8 codes.
+
+Every function is pinned by ``tests/test_oracle_pins.py`` to something other
+than itself (library matmuls on reductions of the layer, closed forms,
+invariants, numpy's argmax / stable argsort, torch's bf16 and float8 decoders).
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import subprocess
+import threading
+
+import numpy as np
+
+F32, BF16, E4M3 = 0, 1, 2
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+_SRC = os.path.join(_HERE, "oracle.c")
+_LIB = os.path.join(_HERE, "liboracle.so")
+_lock = threading.Lock()
+_lib = None
+
+
+def build(force: bool = False) -> str:
+    """Compile oracle.c into liboracle.so (gcc, OpenMP, no fast-math)."""
+    if (not force and os.path.exists(_LIB)
+            and os.path.getmtime(_LIB) >= os.path.getmtime(_SRC)):
+        return _LIB
+    tmp = _LIB + f".tmp{os.getpid()}"
+    cmd = ["gcc", "-O2", "-std=c11", "-fopenmp", "-fPIC", "-shared",
+           "-Wall", "-Wextra", "-o", tmp, _SRC, "-lm"]
+    subprocess.run(cmd, check=True)
+    os.replace(tmp, _LIB)
+    return _LIB
+
+
+def _load():
+    global _lib
+    with _lock:
+        if _lib is None:
+            build()
+            lib = ctypes.CDLL(_LIB)
+            vp, i32, f32p = ctypes.c_void_p, ctypes.c_int, ctypes.c_void_p
+            lib.oracle_bf16_to_double.restype = ctypes.c_double
+            lib.oracle_bf16_to_double.argtypes = [ctypes.c_uint16]
+            lib.oracle_e4m3_to_double.restype = ctypes.c_double
+            lib.oracle_e4m3_to_double.argtypes = [ctypes.c_uint8]
+            lib.oracle_route.restype = None
+            lib.oracle_route.argtypes = [i32, i32, i32, vp, i32, vp, i32, f32p,
+                                         vp, vp, vp]
+            lib.oracle_permutation.restype = None
+            lib.oracle_permutation.argtypes = [i32, i32, vp, vp, vp, vp]
+            lib.oracle_forward.restype = ctypes.c_int
+            lib.oracle_forward.argtypes = [i32, i32, i32, i32, i32,
+                                           vp, i32, vp, i32, f32p,
+                                           vp, vp, vp, vp, i32,
+                                           vp, vp, vp, vp,
+                                           i32, vp, vp, vp, vp]
+            lib.oracle_num_threads.restype = ctypes.c_int
+            lib.oracle_num_threads.argtypes = []
+            _lib = lib
+    return _lib
+
+
+def _dtype_code(a: np.ndarray) -> int:
+    if a.dtype == np.float32:
+        return F32
+    if a.dtype == np.uint16:
+        return BF16
+    if a.dtype == np.uint8:
+        return E4M3
+    raise TypeError(f"oracle: unsupported storage dtype {a.dtype}")
+
+
+def _ptr(a):
+    return None if a is None else a.ctypes.data
+
+
+def num_threads() -> int:
+    """OpenMP threads the oracle runs on (OMP_NUM_THREADS or all cores)."""
+    return int(_load().oracle_num_threads())
+
+
+def bf16_to_f64(bits: int) -> float:
+    return float(_load().oracle_bf16_to_double(int(bits)))
+
+
+def e4m3_to_f64(code: int) -> float:
+    return float(_load().oracle_e4m3_to_double(int(code)))
+
+
+def route(x: np.ndarray, Wr: np.ndarray, bias: np.ndarray | None = None):
+    """Router for all tokens: (idx int32[T], lmax f32[T], margin f32[T]).
+
+    x is [T, d], Wr is [d, E] (router weight, ``x @ Wr`` orientation); the
+    fp32 logits are the fp64 sums rounded once; the top-1 index takes the
+    lowest index on ties; margin is the winning logit minus the runner-up.
+    """
+    x = np.ascontiguousarray(x)
+    Wr = np.ascontiguousarray(Wr)
+    T, d = x.shape
+    d2, E = Wr.shape
+    assert d == d2
+    b = None if bias is None else np.ascontiguousarray(bias, dtype=np.float32)
+    idx = np.empty(T, np.int32)
+    lmax = np.empty(T, np.float32)
+    margin = np.empty(T, np.float32)
+    _load().oracle_route(T, d, E, _ptr(x), _dtype_code(x), _ptr(Wr),
+                         _dtype_code(Wr), _ptr(b), _ptr(idx), _ptr(lmax),
+                         _ptr(margin))
+    return idx, lmax, margin
+
+
+def permutation(idx: np.ndarray, E: int):
+    """(counts[E], offsets[E+1], perm[T]) with perm the stable expert order."""
+    idx = np.ascontiguousarray(idx, dtype=np.int32)
+    T = idx.shape[0]
+    counts = np.empty(E, np.int32)
+    offsets = np.empty(E + 1, np.int32)
+    perm = np.empty(T, np.int32)
+    _load().oracle_permutation(T, E, _ptr(idx), _ptr(counts), _ptr(offsets),
+                               _ptr(perm))
+    return counts, offsets, perm
+
+
+def forward(x, Wr, W_gate_up, W_down, Ws_gate_up, Ws_down, *, bias=None,
+            s_gate_up=None, s_down=None, ss_gate_up=None, ss_down=None,
+            tokens=None):
+    """Layer output in fp64 for ``tokens`` (all tokens when None).
+
+    W_gate_up / W_down are length-E lists of [d, 2F] / [F, d] arrays; entries
+    may be None for experts no selected token reaches.  For E4M3 weights the
+    per-output-column fp32 scales are required.  Returns
+    (out f64[n_sel, d], idx int32[n_sel], gate f64[n_sel]).
+    """
+    x = np.ascontiguousarray(x)
+    Wr = np.ascontiguousarray(Wr)
+    T, d = x.shape
+    E = Wr.shape[1]
+    assert len(W_gate_up) == E and len(W_down) == E
+    Ws_gate_up = np.ascontiguousarray(Ws_gate_up)
+    Ws_down = np.ascontiguousarray(Ws_down)
+    Fs = Ws_down.shape[0]
+    F = None
+    keep = []
+    gu_ptrs = (ctypes.c_void_p * E)()
+    dn_ptrs = (ctypes.c_void_p * E)()
+    w_code = _dtype_code(Ws_gate_up)
+    for e in range(E):
+        if W_gate_up[e] is not None:
+            a = np.ascontiguousarray(W_gate_up[e])
+            b = np.ascontiguousarray(W_down[e])
+            assert _dtype_code(a) == w_code and _dtype_code(b) == w_code
+            F = b.shape[0]
+            keep += [a, b]
+            gu_ptrs[e] = a.ctypes.data
+            dn_ptrs[e] = b.ctypes.data
+    if F is None:
+        F = Fs
+    sgu_ptrs = sdn_ptrs = None
+    if w_code == E4M3:
+        sgu_ptrs = (ctypes.c_void_p * E)()
+        sdn_ptrs = (ctypes.c_void_p * E)()
+        for e in range(E):
+            if s_gate_up is not None and s_gate_up[e] is not None:
+                a = np.ascontiguousarray(s_gate_up[e], dtype=np.float32)
+                b = np.ascontiguousarray(s_down[e], dtype=np.float32)
+                keep += [a, b]
+                sgu_ptrs[e] = a.ctypes.data
+                sdn_ptrs[e] = b.ctypes.data
+        ss_gate_up = np.ascontiguousarray(ss_gate_up, dtype=np.float32)
+        ss_down = np.ascontiguousarray(ss_down, dtype=np.float32)
+    else:
+        ss_gate_up = ss_down = None
+    bias = None if bias is None else np.ascontiguousarray(bias, dtype=np.float32)
+    if tokens is None:
+        sel = None
+        n_sel = T
+    else:
+        sel = np.ascontiguousarray(tokens, dtype=np.int32)
+        n_sel = sel.shape[0]
+    out = np.zeros((n_sel, d), np.float64)
+    sel_idx = np.empty(n_sel, np.int32)
+    sel_gate = np.empty(n_sel, np.float64)
+    rc = _load().oracle_forward(
+        T, d, E, F, Fs, _ptr(x), _dtype_code(x), _ptr(Wr), _dtype_code(Wr),
+        _ptr(bias), ctypes.cast(gu_ptrs, ctypes.c_void_p),
+        ctypes.cast(dn_ptrs, ctypes.c_void_p), _ptr(Ws_gate_up), _ptr(Ws_down),
+        w_code,
+        None if sgu_ptrs is None else ctypes.cast(sgu_ptrs, ctypes.c_void_p),
+        None if sdn_ptrs is None else ctypes.cast(sdn_ptrs, ctypes.c_void_p),
+        _ptr(ss_gate_up), _ptr(ss_down), n_sel, _ptr(sel), _ptr(out),
+        _ptr(sel_idx), _ptr(sel_gate))
+    del keep
+    if rc != 0:
+        raise ValueError("oracle.forward: a selected token routes to an expert "
+                         "whose weights were not supplied")
+    return out, sel_idx, sel_gate

@@ -1,0 +1,233 @@
+/*
+ * oracle.c -- plain, slow CPU oracle for the Llama-4 style top-1 sigmoid-gated
+ * mixture-of-experts feed-forward layer.
+ *
+ * TEST INFRASTRUCTURE ONLY.  Nothing on the product path links, loads or calls
+ * this file; only the test suite, the smoke check and the CPU-baseline leg of
+ * the benchmark do.  It shares no code, header, table or helper with the CUDA
+ * library.
+ *
+ * What it computes, token by token, in fp64 (every input widened exactly):
+ *
+ *   superteams.ai "Llama 4" glossary, section "Mixture of Experts: Why Total
+ *   and Active Parameters Diverge" (the routing sketch): the router produces
+ *   one score per expert, the single highest-scoring expert is selected, and
+ *   the layer returns the shared expert's output plus the selected expert's
+ *   output; the remaining experts do no work for that token.
+ *   KerasFormers "Llama 4" page, "What is unusual about the block": the
+ *   routed expert is applied to the input after it has been multiplied by a
+ *   sigmoid gate, so the routed expert sees sigmoid(winning logit) * x while
+ *   the shared expert sees the ungated x.
+ *   llm-architectures-explained "Llama 4 Maverick", field table rows
+ *   ffns.moe.gated / ffns.moe.d_expert / ffns.moe.d_shared: experts and the
+ *   shared expert are gated MLPs (SwiGLU) of width 8192.
+ *
+ * Readings where the pages are silent (each listed in the design notes):
+ *   - logits are formed in fp64 and rounded once to fp32; the argmax runs on
+ *     those fp32 values with a strict ">" so the lowest index wins a tie and a
+ *     NaN never wins;
+ *   - gate g = 1 / (1 + exp(-l*)) evaluated in fp64 on the fp32 logit;
+ *   - the fused gate/up weight is [d, 2F] with gate columns [0, F) and up
+ *     columns [F, 2F); the down weight is [F, d]; the router weight is [d, E];
+ *   - silu(z) = z / (1 + exp(-z));
+ *   - an optional fp32 router bias b[E] is added to the logits;
+ *   - FP8 weights are OCP E4M3 (bias 7, no infinities, S.1111.111 = NaN,
+ *     max 448) with one fp32 scale per output column; w = e4m3(q) * scale.
+ *
+ * Parity pins (tests/test_oracle_pins.py): E = 1 with the gate forced to 1
+ * reduces to two dense SwiGLU FFNs evaluated by a library matmul; a constant
+ * logit gives the sigmoid closed form and pins input (not output) gating;
+ * ties resolve to the lowest index like numpy.argmax; the permutation equals
+ * numpy's stable argsort; zero input gives exactly zero output; the E4M3 and
+ * bf16 decoders agree with torch's for every code.
+ */
+#include <math.h>
+#include <stdint.h>
+#include <stdlib.h>
+#include <string.h>
+#ifdef _OPENMP
+#include <omp.h>
+#endif
+
+enum { ORACLE_F32 = 0, ORACLE_BF16 = 1, ORACLE_E4M3 = 2 };
+
+/* bf16 is the upper half of an IEEE binary32; widening is exact. */
+double oracle_bf16_to_double(uint16_t b) {
+    uint32_t u = (uint32_t)b << 16;
+    float f;
+    memcpy(&f, &u, sizeof f);
+    return (double)f;
+}
+
+/* OCP 8-bit floating point, E4M3 variant: 1 sign, 4 exponent (bias 7),
+ * 3 mantissa bits; exponent field 0 is subnormal; S.1111.111 is NaN; there
+ * is no infinity. */
+double oracle_e4m3_to_double(uint8_t q) {
+    int sign = (q >> 7) & 1;
+    int e = (q >> 3) & 0xF;
+    int m = q & 0x7;
+    double v;
+    if (e == 0xF && m == 0x7) return NAN;
+    if (e == 0)
+        v = ldexp((double)m / 8.0, 1 - 7);
+    else
+        v = ldexp(1.0 + (double)m / 8.0, e - 7);
+    return sign ? -v : v;
+}
+
+static double load_elem(const void *p, int dtype, size_t i) {
+    switch (dtype) {
+    case ORACLE_F32: return (double)((const float *)p)[i];
+    case ORACLE_BF16: return oracle_bf16_to_double(((const uint16_t *)p)[i]);
+    case ORACLE_E4M3: return oracle_e4m3_to_double(((const uint8_t *)p)[i]);
+    default: return NAN;
+    }
+}
+
+/* A weight element of a [rows, cols] row-major matrix; for E4M3 the
+ * per-output-column scale is applied (dequantisation). */
+static double load_weight(const void *W, int dtype, const float *col_scale,
+                          size_t row, size_t cols, size_t col) {
+    double w = load_elem(W, dtype, row * cols + col);
+    if (dtype == ORACLE_E4M3) w *= (double)col_scale[col];
+    return w;
+}
+
+static double sigmoid(double z) { return 1.0 / (1.0 + exp(-z)); }
+static double silu(double z) { return z / (1.0 + exp(-z)); }
+
+/* Router for one token: fp32 logits, top-1 index (lowest index on ties),
+ * winning logit and the margin to the runner-up (+inf when E == 1). */
+static int route_token(int d, int E, const void *x_t, int x_dtype,
+                       const void *Wr, int wr_dtype, const float *bias,
+                       float *lmax_out, float *margin_out) {
+    int best = 0;
+    float lbest = -INFINITY, lsecond = -INFINITY;
+    for (int e = 0; e < E; ++e) {
+        double acc = 0.0;
+        for (int k = 0; k < d; ++k)
+            acc += load_elem(x_t, x_dtype, (size_t)k) *
+                   load_elem(Wr, wr_dtype, (size_t)k * (size_t)E + (size_t)e);
+        if (bias) acc += (double)bias[e];
+        float l = (float)acc;
+        if (l > lbest) {            /* strict: earlier index keeps a tie */
+            lsecond = lbest;
+            lbest = l;
+            best = e;
+        } else if (l > lsecond) {
+            lsecond = l;
+        }
+    }
+    if (lmax_out) *lmax_out = lbest;
+    if (margin_out) *margin_out = (E > 1) ? (float)((double)lbest - (double)lsecond) : INFINITY;
+    return best;
+}
+
+/* One SwiGLU FFN on one input row u[d]:
+ *   a = u . Wgu  (2Fw values), h_j = silu(a_j) * a_{Fw+j},  y += h . Wd.  */
+static void swiglu_ffn_accumulate(int d, int Fw, const double *u,
+                                  const void *Wgu, const void *Wd, int w_dtype,
+                                  const float *s_gu, const float *s_d,
+                                  double *a, double *h, double *y) {
+    size_t two_f = 2 * (size_t)Fw;
+    for (size_t j = 0; j < two_f; ++j) a[j] = 0.0;
+    for (int k = 0; k < d; ++k) {
+        double uk = u[k];
+        for (size_t j = 0; j < two_f; ++j)
+            a[j] += uk * load_weight(Wgu, w_dtype, s_gu, (size_t)k, two_f, j);
+    }
+    for (int j = 0; j < Fw; ++j) h[j] = silu(a[j]) * a[Fw + j];
+    for (int j = 0; j < Fw; ++j) {
+        double hj = h[j];
+        for (int n = 0; n < d; ++n)
+            y[n] += hj * load_weight(Wd, w_dtype, s_d, (size_t)j, (size_t)d, (size_t)n);
+    }
+}
+
+/* Routing for all T tokens. */
+void oracle_route(int T, int d, int E, const void *x, int x_dtype,
+                  const void *Wr, int wr_dtype, const float *bias,
+                  int32_t *idx, float *lmax, float *margin) {
+    size_t xs = (x_dtype == ORACLE_F32) ? 4 : 2;
+#pragma omp parallel for schedule(static)
+    for (int t = 0; t < T; ++t) {
+        const char *x_t = (const char *)x + (size_t)t * (size_t)d * xs;
+        idx[t] = route_token(d, E, x_t, x_dtype, Wr, wr_dtype, bias,
+                             lmax ? &lmax[t] : NULL, margin ? &margin[t] : NULL);
+    }
+}
+
+/* Per-expert counts, exclusive offsets and the stable permutation
+ * perm[p] = token at expert-sorted slot p (order by expert, then token). */
+void oracle_permutation(int T, int E, const int32_t *idx, int32_t *counts,
+                        int32_t *offsets, int32_t *perm) {
+    for (int e = 0; e < E; ++e) counts[e] = 0;
+    for (int t = 0; t < T; ++t) counts[idx[t]] += 1;
+    offsets[0] = 0;
+    for (int e = 0; e < E; ++e) offsets[e + 1] = offsets[e] + counts[e];
+    int32_t *fill = (int32_t *)malloc(sizeof(int32_t) * (size_t)(E > 0 ? E : 1));
+    for (int e = 0; e < E; ++e) fill[e] = offsets[e];
+    for (int t = 0; t < T; ++t) perm[fill[idx[t]]++] = t;
+    free(fill);
+}
+
+/* Full layer output for the tokens listed in sel[0..n_sel) (all tokens
+ * when sel == NULL, n_sel == T).  out is [n_sel, d] fp64.  W_gate_up[e] /
+ * W_down[e] may be NULL for experts that none of the selected tokens
+ * reaches; returns -1 if a needed expert is missing, 0 on success.
+ * sel_idx / sel_gate (optional) receive each selected token's expert and
+ * gate. */
+int oracle_forward(int T, int d, int E, int F, int Fs,
+                   const void *x, int x_dtype,
+                   const void *Wr, int wr_dtype, const float *bias,
+                   const void *const *W_gate_up, const void *const *W_down,
+                   const void *Ws_gate_up, const void *Ws_down, int w_dtype,
+                   const float *const *s_gate_up, const float *const *s_down,
+                   const float *ss_gate_up, const float *ss_down,
+                   int n_sel, const int32_t *sel, double *out,
+                   int32_t *sel_idx, double *sel_gate) {
+    size_t xs = (x_dtype == ORACLE_F32) ? 4 : 2;
+    int missing = 0;
+    (void)T;
+#pragma omp parallel for schedule(dynamic, 1) reduction(| : missing)
+    for (int i = 0; i < n_sel; ++i) {
+        int t = sel ? sel[i] : i;
+        const char *x_t = (const char *)x + (size_t)t * (size_t)d * xs;
+        int Fmax = F > Fs ? F : Fs;
+        double *u = (double *)malloc(sizeof(double) * (size_t)d);
+        double *a = (double *)malloc(sizeof(double) * 2 * (size_t)Fmax);
+        double *h = (double *)malloc(sizeof(double) * (size_t)Fmax);
+        double *y = out + (size_t)i * (size_t)d;
+        float lmax;
+        int e = route_token(d, E, x_t, x_dtype, Wr, wr_dtype, bias, &lmax, NULL);
+        double g = sigmoid((double)lmax);
+        if (sel_idx) sel_idx[i] = e;
+        if (sel_gate) sel_gate[i] = g;
+        for (int n = 0; n < d; ++n) y[n] = 0.0;
+        /* shared expert on the ungated input */
+        for (int k = 0; k < d; ++k) u[k] = load_elem(x_t, x_dtype, (size_t)k);
+        swiglu_ffn_accumulate(d, Fs, u, Ws_gate_up, Ws_down, w_dtype,
+                              ss_gate_up, ss_down, a, h, y);
+        /* routed expert on the sigmoid-gated input */
+        if (!W_gate_up[e] || !W_down[e]) {
+            missing |= 1;
+        } else {
+            for (int k = 0; k < d; ++k) u[k] = g * load_elem(x_t, x_dtype, (size_t)k);
+            swiglu_ffn_accumulate(d, F, u, W_gate_up[e], W_down[e], w_dtype,
+                                  s_gate_up ? s_gate_up[e] : NULL,
+                                  s_down ? s_down[e] : NULL, a, h, y);
+        }
+        free(u);
+        free(a);
+        free(h);
+    }
+    return missing ? -1 : 0;
+}
+
+int oracle_num_threads(void) {
+#ifdef _OPENMP
+    return omp_get_max_threads();
+#else
+    return 1;
+#endif
+}

@@ -1,0 +1,252 @@
+"""Pins of the CPU oracle to things other than itself.
+
+Each test reduces the layer to a case that the pages or the mathematics fix
+(a library matmul, a closed form, an invariant, numpy's argmax / stable
+argsort, torch's own dtype decoders), chosen so that a plausible slip in the
+oracle (dropped shared expert, gate on the output instead of the input,
+swapped gate/up halves, transposed down weight, wrong sigmoid sign, highest
+index on ties, wrong subnormal decode, per-row instead of per-column FP8
+scales) fails at least one of them.
+"""
+import numpy as np
+import pytest
+import torch
+from scipy.special import expit
+
+import oracle
+from sparse_moe_transformer_router_b200.workloads import quantize_e4m3_columns
+
+
+def _bf16_bits(a: np.ndarray) -> np.ndarray:
+    return torch.from_numpy(np.ascontiguousarray(a, np.float32)).to(torch.bfloat16) \
+        .view(torch.int16).numpy().view(np.uint16)
+
+
+def _bf16_f64(bits: np.ndarray) -> np.ndarray:
+    return torch.from_numpy(bits.view(np.int16)).view(torch.bfloat16).to(torch.float64).numpy()
+
+
+def _store(a: np.ndarray, dtype: str):
+    """(storage array for the oracle, exact fp64 values it represents)."""
+    if dtype == "f32":
+        s = np.ascontiguousarray(a, np.float32)
+        return s, s.astype(np.float64)
+    s = _bf16_bits(a)
+    return s, _bf16_f64(s)
+
+
+def _dense_swiglu(u, Wgu, Wd):
+    """Textbook SwiGLU FFN through library routines (torch fp64 matmul, F.silu)."""
+    u = torch.from_numpy(u)
+    Wgu = torch.from_numpy(Wgu)
+    Wd = torch.from_numpy(Wd)
+    F = Wd.shape[0]
+    a = u @ Wgu
+    h = torch.nn.functional.silu(a[:, :F]) * a[:, F:]
+    return (h @ Wd).numpy()
+
+
+def _layer(rng, T, d, E, F, Fs, dtype, wstd=0.2):
+    x, x64 = _store(rng.standard_normal((T, d)), dtype)
+    Wr, Wr64 = _store(rng.standard_normal((d, E)) * 0.3, dtype)
+    Wgu, Wd, Wgu64, Wd64 = [], [], [], []
+    for _ in range(E):
+        a, a64 = _store(rng.standard_normal((d, 2 * F)) * wstd, dtype)
+        b, b64 = _store(rng.standard_normal((F, d)) * wstd, dtype)
+        Wgu.append(a), Wd.append(b), Wgu64.append(a64), Wd64.append(b64)
+    Wsgu, Wsgu64 = _store(rng.standard_normal((d, 2 * Fs)) * wstd, dtype)
+    Wsd, Wsd64 = _store(rng.standard_normal((Fs, d)) * wstd, dtype)
+    return dict(x=x, x64=x64, Wr=Wr, Wr64=Wr64, Wgu=Wgu, Wd=Wd, Wgu64=Wgu64, Wd64=Wd64,
+                Wsgu=Wsgu, Wsgu64=Wsgu64, Wsd=Wsd, Wsd64=Wsd64)
+
+
+def test_bf16_decoder_matches_torch_for_every_code():
+    codes = np.arange(1 << 16, dtype=np.uint32).astype(np.uint16)
+    ref = _bf16_f64(codes)
+    got = np.array([oracle.bf16_to_f64(c) for c in codes])
+    nan = np.isnan(ref)
+    assert np.array_equal(nan, np.isnan(got))
+    assert np.array_equal(ref[~nan], got[~nan])
+
+
+def test_e4m3_decoder_matches_torch_for_every_code():
+    codes = np.arange(256, dtype=np.uint8)
+    ref = torch.from_numpy(codes).view(torch.float8_e4m3fn).to(torch.float64).numpy()
+    got = np.array([oracle.e4m3_to_f64(c) for c in codes])
+    nan = np.isnan(ref)
+    assert nan.sum() == 2  # S.1111.111 for both signs
+    assert np.array_equal(nan, np.isnan(got))
+    assert np.array_equal(ref[~nan], got[~nan])
+    assert got[0x7E] == 448.0 and got[0x01] == 2.0 ** -9
+
+
+@pytest.mark.parametrize("dtype", ["f32", "bf16"])
+def test_single_expert_with_saturated_gate_is_two_dense_ffns(dtype):
+    """E = 1 and router bias 100 force routing to expert 0 with
+    sigmoid(>= 100 - small) == 1.0 exactly in fp64, so the layer must equal
+    dense_swiglu(x; Wgu_0, Wd_0) + dense_swiglu(x; Ws_gu, Ws_d)."""
+    rng = np.random.default_rng(1)
+    T, d, F, Fs = 7, 48, 40, 24
+    L = _layer(rng, T, d, 1, F, Fs, dtype)
+    bias = np.array([100.0], np.float32)
+    out, idx, gate = oracle.forward(L["x"], L["Wr"], L["Wgu"], L["Wd"], L["Wsgu"], L["Wsd"], bias=bias)
+    assert np.all(idx == 0) and np.all(gate == 1.0)
+    ref = _dense_swiglu(L["x64"], L["Wgu64"][0], L["Wd64"][0]) + \
+        _dense_swiglu(L["x64"], L["Wsgu64"], L["Wsd64"])
+    scale = np.sqrt(np.mean(ref ** 2))
+    assert np.max(np.abs(out - ref)) <= 1e-12 * scale
+
+
+@pytest.mark.parametrize("c", [0.7, -1.3])
+def test_constant_logit_gives_sigmoid_gate_on_the_input(c):
+    """A zero router weight and a bias with a unique maximum c make every
+    logit constant: all tokens go to the arg-max expert with gate
+    sigmoid(c), and the routed FFN sees gate * x (not gate * FFN(x))."""
+    rng = np.random.default_rng(2)
+    T, d, E, F, Fs = 5, 32, 3, 24, 16
+    L = _layer(rng, T, d, E, F, Fs, "f32", wstd=0.5)
+    Wr0 = np.zeros((d, E), np.float32)
+    bias = np.array([c - 1.0, c, c - 0.5], np.float32)  # expert 1 wins
+    Wgu = [None, L["Wgu"][1], None]
+    Wd = [None, L["Wd"][1], None]
+    out, idx, gate = oracle.forward(L["x"], Wr0, Wgu, Wd, L["Wsgu"], L["Wsd"], bias=bias)
+    g = expit(np.float64(np.float32(c)))
+    assert np.all(idx == 1)
+    assert np.allclose(gate, g, rtol=0, atol=1e-15)
+    shared = _dense_swiglu(L["x64"], L["Wsgu64"], L["Wsd64"])
+    ref_in = shared + _dense_swiglu(g * L["x64"], L["Wgu64"][1], L["Wd64"][1])
+    ref_out = shared + g * _dense_swiglu(L["x64"], L["Wgu64"][1], L["Wd64"][1])
+    scale = np.sqrt(np.mean(ref_in ** 2))
+    assert np.max(np.abs(out - ref_in)) <= 1e-12 * scale
+    # the pin has power: gating the output instead would be far off
+    assert np.max(np.abs(ref_out - ref_in)) > 1e-3 * scale
+
+
+def test_argmax_takes_lowest_index_on_ties():
+    """One-hot tokens make the logits exact copies of router rows; rows with
+    duplicated maxima must resolve to the lowest index, as numpy.argmax does."""
+    d, E = 6, 5
+    Wr = np.array([[0.0, 2.0, 1.0, 2.0, 2.0],
+                   [3.0, 3.0, 3.0, 3.0, 3.0],
+                   [-1.0, -2.0, -1.0, -3.0, -1.0],
+                   [0.5, 0.25, 0.75, 0.75, 0.1],
+                   [0.0, 0.0, 0.0, 0.0, 1.0],
+                   [-5.0, -4.0, -4.0, -6.0, -4.0]], np.float32)
+    x = np.eye(d, dtype=np.float32)
+    idx, lmax, margin = oracle.route(x, Wr)
+    assert np.array_equal(idx, np.argmax(Wr, axis=1).astype(np.int32))
+    assert list(idx) == [1, 0, 0, 2, 4, 1]
+    assert np.array_equal(lmax, Wr.max(axis=1))
+    assert list(margin[:3]) == [0.0, 0.0, 0.0] and margin[4] == 1.0
+
+
+@pytest.mark.parametrize("dtype", ["f32", "bf16"])
+def test_router_equals_library_matmul_then_argmax(dtype):
+    rng = np.random.default_rng(3)
+    T, d, E = 257, 96, 16
+    x, x64 = _store(rng.standard_normal((T, d)), dtype)
+    Wr, Wr64 = _store(rng.standard_normal((d, E)) * 0.1, dtype)
+    bias = (rng.standard_normal(E) * 0.05).astype(np.float32)
+    idx, lmax, margin = oracle.route(x, Wr, bias)
+    logits = (x64 @ Wr64 + bias.astype(np.float64)).astype(np.float32)
+    assert np.array_equal(idx, np.argmax(logits, axis=1))
+    assert np.array_equal(lmax, logits.max(axis=1))
+    srt = np.sort(logits.astype(np.float64), axis=1)
+    assert np.allclose(margin, (srt[:, -1] - srt[:, -2]).astype(np.float32), rtol=0, atol=0)
+
+
+def test_permutation_is_the_stable_argsort():
+    rng = np.random.default_rng(4)
+    E, T = 12, 1000
+    idx = rng.integers(0, E, T).astype(np.int32)
+    idx[idx == 5] = 6          # expert 5 empty
+    idx[:40] = 11              # heavy tail expert
+    counts, offsets, perm = oracle.permutation(idx, E)
+    assert counts.sum() == T
+    assert np.array_equal(counts, np.bincount(idx, minlength=E))
+    assert np.array_equal(offsets, np.concatenate([[0], np.cumsum(np.bincount(idx, minlength=E))]))
+    assert np.array_equal(perm, np.argsort(idx, kind="stable"))
+    inv = np.empty(T, np.int64)
+    inv[perm] = np.arange(T)
+    assert np.array_equal(np.sort(perm), np.arange(T))
+    assert np.array_equal(perm[inv], np.arange(T))
+
+
+def test_zero_input_gives_exact_zero_output():
+    rng = np.random.default_rng(5)
+    T, d, E, F, Fs = 9, 32, 4, 16, 16
+    L = _layer(rng, T, d, E, F, Fs, "bf16")
+    x = np.zeros_like(L["x"])
+    out, idx, gate = oracle.forward(x, L["Wr"], L["Wgu"], L["Wd"], L["Wsgu"], L["Wsd"])
+    assert np.all(idx == 0)            # all logits 0: tie -> lowest index
+    assert np.all(gate == 0.5)
+    assert np.all(out == 0.0)
+
+
+def test_token_and_expert_relabelling_symmetries():
+    """Per-token independence: permuting tokens permutes outputs exactly.
+    Expert labels carry no meaning: relabelling experts (router columns and
+    weight lists together) leaves every output bit-identical."""
+    rng = np.random.default_rng(6)
+    T, d, E, F, Fs = 23, 40, 6, 24, 16
+    L = _layer(rng, T, d, E, F, Fs, "bf16")
+    bias = (rng.standard_normal(E) * 0.3).astype(np.float32)
+    out, idx, gate = oracle.forward(L["x"], L["Wr"], L["Wgu"], L["Wd"], L["Wsgu"], L["Wsd"], bias=bias)
+    pt = rng.permutation(T)
+    out_t, idx_t, _ = oracle.forward(L["x"][pt], L["Wr"], L["Wgu"], L["Wd"], L["Wsgu"], L["Wsd"], bias=bias)
+    assert np.array_equal(out_t, out[pt]) and np.array_equal(idx_t, idx[pt])
+    pe = rng.permutation(E)              # new expert j is old expert pe[j]
+    out_e, idx_e, gate_e = oracle.forward(
+        L["x"], np.ascontiguousarray(L["Wr"][:, pe]), [L["Wgu"][j] for j in pe],
+        [L["Wd"][j] for j in pe], L["Wsgu"], L["Wsd"], bias=bias[pe])
+    assert np.array_equal(out_e, out)
+    assert np.array_equal(pe[idx_e], idx)
+    assert np.array_equal(gate_e, gate)
+
+
+def test_fp8_weights_dequantise_per_output_column():
+    """E4M3 weights with per-output-column scales equal the dense layer on
+    the dequantised weights (torch's float8 decoder times the column scale)."""
+    rng = np.random.default_rng(7)
+    T, d, F, Fs = 6, 64, 32, 48
+    x, x64 = _store(rng.standard_normal((T, d)), "bf16")
+    Wr, _ = _store(rng.standard_normal((d, 1)), "bf16")
+
+    def q(shape):
+        w = torch.from_numpy(rng.standard_normal(shape) * 0.02).float()
+        w[:, 0] *= 50.0  # very different column ranges
+        qq, s = quantize_e4m3_columns(w)
+        deq = qq.to(torch.float64) * s.to(torch.float64)[None, :]
+        return qq.view(torch.uint8).numpy(), s.numpy(), deq.numpy()
+
+    gu, sgu, gu64 = q((d, 2 * F))
+    dn, sdn, dn64 = q((F, d))
+    sgu_s, ssgu, sgu64 = q((d, 2 * Fs))
+    sdn_s, ssdn, sdn64 = q((Fs, d))
+    out, idx, gate = oracle.forward(x, Wr, [gu], [dn], sgu_s, sdn_s, bias=np.array([100.0], np.float32),
+                                    s_gate_up=[sgu], s_down=[sdn], ss_gate_up=ssgu, ss_down=ssdn)
+    assert np.all(gate == 1.0)
+    ref = _dense_swiglu(x64, gu64, dn64) + _dense_swiglu(x64, sgu64, sdn64)
+    scale = np.sqrt(np.mean(ref ** 2))
+    assert np.max(np.abs(out - ref)) <= 1e-12 * scale
+
+
+def test_token_subset_equals_rows_of_full_run_and_missing_expert_raises():
+    rng = np.random.default_rng(8)
+    T, d, E, F, Fs = 17, 32, 4, 16, 24
+    L = _layer(rng, T, d, E, F, Fs, "f32")
+    full, idx, _ = oracle.forward(L["x"], L["Wr"], L["Wgu"], L["Wd"], L["Wsgu"], L["Wsd"])
+    sel = np.array([16, 0, 5, 5, 9], np.int32)
+    sub, sidx, _ = oracle.forward(L["x"], L["Wr"], L["Wgu"], L["Wd"], L["Wsgu"], L["Wsd"], tokens=sel)
+    assert np.array_equal(sub, full[sel]) and np.array_equal(sidx, idx[sel])
+    needed = set(idx[sel].tolist())
+    Wgu = [w if e in needed else None for e, w in enumerate(L["Wgu"])]
+    Wd = [w if e in needed else None for e, w in enumerate(L["Wd"])]
+    sub2, _, _ = oracle.forward(L["x"], L["Wr"], Wgu, Wd, L["Wsgu"], L["Wsd"], tokens=sel)
+    assert np.array_equal(sub2, sub)
+    missing = next(e for e in range(E) if e not in needed) if len(needed) < E else None
+    if missing is not None:
+        t = int(np.nonzero(idx == missing)[0][0]) if np.any(idx == missing) else None
+        if t is not None:
+            with pytest.raises(ValueError):
+                oracle.forward(L["x"], L["Wr"], Wgu, Wd, L["Wsgu"], L["Wsd"], tokens=np.array([t], np.int32))
