@@ -1,0 +1,179 @@
+/*
+ * l4moe.h -- C ABI of a B200 (sm_100a) implementation of the Llama-4 style
+ * mixture-of-experts feed-forward layer: top-1 routing with a sigmoid gate on
+ * the routed expert's input, a SwiGLU routed expert and an always-on SwiGLU
+ * shared expert whose outputs are summed.
+ *
+ * What the layer computes (per token t, input row x_t of width d):
+ *   - router logits l_e = x_t . W_router[:, e] (+ optional bias b_e), fp32;
+ *     superteams.ai "Llama 4" glossary, section "Mixture of Experts: Why
+ *     Total and Active Parameters Diverge" (routing sketch: one logit per
+ *     expert);
+ *   - the single expert e* with the largest logit (lowest index on ties),
+ *     same section (top-1 routing) and KerasFormers "Llama 4" API table
+ *     (num_experts_per_tok = 1);
+ *   - gate g = sigmoid(l_{e*}) applied to the routed expert's INPUT:
+ *     KerasFormers "Llama 4", section "What is unusual about the block";
+ *   - routed output  y_r = SwiGLU_{e*}(g * x_t), shared output
+ *     y_s = SwiGLU_shared(x_t), out_t = y_s + y_r: glossary routing sketch
+ *     (shared plus routed) and llm-architectures-explained "Llama 4
+ *     Maverick" field table (ffns.moe.* rows: gated experts of width 8192,
+ *     one shared expert of width 8192).
+ *   SwiGLU_W(u) = (silu(u . Wg) * (u . Wu)) . Wd with silu(z) = z/(1+e^-z).
+ *
+ * Layouts (all row-major, "x @ W" orientation, element = the dtype below):
+ *   x          [T, d]        W_router  [d, E]
+ *   W_gate_up  [d, 2F] per expert: gate columns [0, F), up columns [F, 2F)
+ *   W_down     [F, d]  per expert
+ *   Ws_gate_up [d, 2Fs], Ws_down [Fs, d]  (shared expert)
+ *   out        [T, d]
+ * Dtypes (l4moe_dtype):
+ *   L4MOE_F32       every tensor fp32 (tensor-core math in TF32, fp32 accumulate)
+ *   L4MOE_BF16      every tensor bf16 (bf16 MMA, fp32 accumulate)
+ *   L4MOE_FP8_E4M3  expert and shared weights OCP E4M3 with one fp32 scale per
+ *                   output column (l4moe_set_fp8_scales); x, W_router, out bf16.
+ *
+ * Ownership: the caller owns every tensor, the scale vectors, the bias and
+ * the stream.  The handle owns only its workspace (unless the caller supplies
+ * one) and a cache of TMA descriptors keyed by the weight pointer values.
+ * Pointers passed to l4moe_forward must stay valid until the work enqueued on
+ * the stream has finished.
+ *
+ * Errors: every entry point returns a status; argument errors are reported
+ * synchronously and launch nothing.  l4moe_forward never synchronises the
+ * stream; device-side faults of the kernels' own bounded waits are recorded
+ * in a device word that l4moe_check_device_status reads (it synchronises).
+ * l4moe_last_error gives a message for the last non-OK status of a handle.
+ *
+ * Requirements: d, F, Fs multiples of 64; 1 <= E <= 256; all tensor pointers
+ * 16-byte aligned.  One handle serves one stream at a time (the workspace is
+ * shared by the calls made with it).
+ */
+#ifndef L4MOE_H
+#define L4MOE_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define L4MOE_API __attribute__((visibility("default")))
+#else
+#define L4MOE_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+    L4MOE_OK = 0,
+    L4MOE_ERR_ARG = 1,          /* null / out-of-range argument                */
+    L4MOE_ERR_DTYPE = 2,        /* unknown dtype or missing FP8 scales         */
+    L4MOE_ERR_ALIGN = 3,        /* pointer not 16-byte aligned / bad multiple  */
+    L4MOE_ERR_CUDA = 4,         /* a CUDA runtime or driver call failed        */
+    L4MOE_ERR_WORKSPACE = 5,    /* workspace too small / allocation failed     */
+    L4MOE_ERR_TIMEOUT = 6,      /* a kernel's bounded wait ran out             */
+    L4MOE_ERR_UNSUPPORTED = 7   /* device is not sm_100 or feature unavailable */
+} l4moe_status;
+
+typedef enum {
+    L4MOE_F32 = 0,
+    L4MOE_BF16 = 1,
+    L4MOE_FP8_E4M3 = 2
+} l4moe_dtype;
+
+typedef struct {
+    int d_model;      /* d  : model width (KerasFormers "Llama 4": embed_dim)       */
+    int expert_ffn;   /* F  : routed expert width (Maverick table: d_expert)       */
+    int shared_ffn;   /* Fs : shared expert width (Maverick table: d_shared)       */
+    int num_experts;  /* E  : routed experts (16 Scout, 128 Maverick)              */
+    l4moe_dtype dtype;
+} l4moe_params;
+
+typedef struct l4moe_handle l4moe_handle;
+
+/* Validate the shapes and dtype and create a handle.  Host only; no device
+ * work and no allocation on the device.  *out receives the handle. */
+L4MOE_API l4moe_status l4moe_create(const l4moe_params *params, l4moe_handle **out);
+
+/* Free the handle, its own workspace and descriptor cache.  Waits for
+ * nothing: the caller must ensure no enqueued work still uses it. */
+L4MOE_API void l4moe_destroy(l4moe_handle *h);
+
+/* Bytes of device workspace l4moe_forward needs for up to max_tokens tokens
+ * (routing vectors, permutation, group tables, gated expert-ordered input,
+ * both hidden activations, host-path staging).  0 on a bad argument. */
+L4MOE_API size_t l4moe_workspace_size(const l4moe_handle *h, int max_tokens);
+
+/* Give the handle a caller-owned device workspace of `bytes` bytes (256-byte
+ * aligned) sized for max_tokens tokens.  Without this call, l4moe_forward
+ * allocates one itself (cudaMalloc) on first use or when T grows. */
+L4MOE_API l4moe_status l4moe_set_workspace(l4moe_handle *h, void *dev_ptr, size_t bytes, int max_tokens);
+
+/* Optional fp32 router bias b[E] (device pointer, NULL = none) added to the
+ * logits before the arg-max and the gate.  The pages' router has no bias;
+ * this exists to draw skewed expert loads. */
+L4MOE_API l4moe_status l4moe_set_router_bias(l4moe_handle *h, const float *bias_dev);
+
+/* FP8 weights only: per-output-column fp32 scales (device pointers).
+ * s_gate_up / s_down are HOST arrays of E device pointers to [2F] / [d]
+ * vectors; ss_gate_up [2Fs] and ss_down [d] are the shared expert's.  The
+ * dequantised weight is e4m3(q) * scale[column]. */
+L4MOE_API l4moe_status l4moe_set_fp8_scales(l4moe_handle *h, const float *const *s_gate_up,
+                                  const float *const *s_down, const float *ss_gate_up,
+                                  const float *ss_down);
+
+/* Enqueue one forward pass of the layer for T tokens on `stream` (a
+ * cudaStream_t, NULL = legacy default stream).  x, W_router, Ws_gate_up,
+ * Ws_down, out are device pointers; W_gate_up and W_down are HOST arrays of E
+ * device pointers (one weight matrix per expert).  out is fully written.  T = 0
+ * enqueues nothing and returns L4MOE_OK.  Asynchronous: no host sync. */
+L4MOE_API l4moe_status l4moe_forward(l4moe_handle *h, int T, const void *x, const void *W_router,
+                           const void *const *W_gate_up, const void *const *W_down,
+                           const void *Ws_gate_up, const void *Ws_down, void *out,
+                           void *stream);
+
+/* As l4moe_forward, but x_host and out_host are HOST buffers (pinned memory
+ * recommended): the call enqueues the host-to-device copy of x, the layer and
+ * the device-to-host copy of out on `stream`, using staging buffers inside
+ * the workspace.  Weights stay device pointers.  Asynchronous like
+ * l4moe_forward: out_host is valid after the stream has been synchronised. */
+L4MOE_API l4moe_status l4moe_forward_host(l4moe_handle *h, int T, const void *x_host, const void *W_router,
+                                const void *const *W_gate_up, const void *const *W_down,
+                                const void *Ws_gate_up, const void *Ws_down, void *out_host,
+                                void *stream);
+
+/* Device pointers (inside the workspace) to the routing of the last forward
+ * enqueued with this handle; valid once that work has run and until the next
+ * forward.  Any output pointer may be NULL.
+ *   idx[T] int32 expert per token; gate[T] fp32 sigmoid gate; lmax[T] fp32
+ *   winning logit; margin[T] fp32 winning minus runner-up logit;
+ *   counts[E] int32; offsets[E+1] int32 exclusive prefix of counts;
+ *   perm[T] int32 expert-ordered slot -> token (stable by token). */
+L4MOE_API l4moe_status l4moe_get_routing(const l4moe_handle *h, const int32_t **idx, const float **gate,
+                               const float **lmax, const float **margin, const int32_t **counts,
+                               const int32_t **offsets, const int32_t **perm);
+
+/* Synchronise `stream` and read the device error word of the handle's
+ * workspace: L4MOE_OK, L4MOE_ERR_TIMEOUT (a bounded wait ran out) or
+ * L4MOE_ERR_CUDA.  Clears the word. */
+L4MOE_API l4moe_status l4moe_check_device_status(l4moe_handle *h, void *stream);
+
+/* Number of kernels this handle has launched so far. */
+L4MOE_API uint64_t l4moe_launch_count(const l4moe_handle *h);
+
+/* Message for the handle's last non-OK status ("" if none); h may be NULL
+ * for errors of l4moe_create. */
+L4MOE_API const char *l4moe_last_error(const l4moe_handle *h);
+
+/* Static name of a status code. */
+L4MOE_API const char *l4moe_status_string(l4moe_status s);
+
+/* ABI version (major * 100 + minor). */
+L4MOE_API int l4moe_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* L4MOE_H */

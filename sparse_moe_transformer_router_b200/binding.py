@@ -1,0 +1,207 @@
+"""Thin ctypes binding over libl4moe.so (include/l4moe.h).
+
+Argument marshalling only: every step of the layer runs in the library's CUDA
+kernels.  torch is used for device memory and streams.  There is no fallback:
+if the compiled library is missing or the call fails, an exception is raised.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+
+import torch
+
+_PKG = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_PKG, "libl4moe.so")
+
+OK, ERR_ARG, ERR_DTYPE, ERR_ALIGN, ERR_CUDA, ERR_WORKSPACE, ERR_TIMEOUT, ERR_UNSUPPORTED = range(8)
+DTYPES = {"f32": 0, "bf16": 1, "fp8": 2}
+EXPORTED = ("l4moe_create", "l4moe_destroy", "l4moe_workspace_size", "l4moe_set_workspace",
+            "l4moe_set_router_bias", "l4moe_set_fp8_scales", "l4moe_forward",
+            "l4moe_forward_host", "l4moe_get_routing", "l4moe_check_device_status",
+            "l4moe_launch_count", "l4moe_last_error", "l4moe_status_string", "l4moe_version")
+
+_lib = None
+
+
+class L4MoEError(RuntimeError):
+    def __init__(self, status: int, message: str):
+        super().__init__(f"{message} (status {status})")
+        self.status = status
+
+
+class Params(ctypes.Structure):
+    _fields_ = [("d_model", ctypes.c_int), ("expert_ffn", ctypes.c_int),
+                ("shared_ffn", ctypes.c_int), ("num_experts", ctypes.c_int),
+                ("dtype", ctypes.c_int)]
+
+
+def load_library():
+    """Load libl4moe.so (raises if it has not been built)."""
+    global _lib
+    if _lib is not None:
+        return _lib
+    if not os.path.exists(LIB_PATH):
+        raise ImportError(f"{LIB_PATH} is missing: build it with "
+                          "`python -m sparse_moe_transformer_router_b200.build`")
+    lib = ctypes.CDLL(LIB_PATH)
+    vp, i32, sz = ctypes.c_void_p, ctypes.c_int, ctypes.c_size_t
+    pvp = ctypes.POINTER(ctypes.c_void_p)
+    lib.l4moe_create.argtypes = [ctypes.POINTER(Params), ctypes.POINTER(vp)]
+    lib.l4moe_destroy.argtypes = [vp]
+    lib.l4moe_destroy.restype = None
+    lib.l4moe_workspace_size.argtypes = [vp, i32]
+    lib.l4moe_workspace_size.restype = sz
+    lib.l4moe_set_workspace.argtypes = [vp, vp, sz, i32]
+    lib.l4moe_set_router_bias.argtypes = [vp, vp]
+    lib.l4moe_set_fp8_scales.argtypes = [vp, pvp, pvp, vp, vp]
+    fwd = [vp, i32, vp, vp, pvp, pvp, vp, vp, vp, vp]
+    lib.l4moe_forward.argtypes = fwd
+    lib.l4moe_forward_host.argtypes = fwd
+    lib.l4moe_get_routing.argtypes = [vp] + [pvp] * 7
+    lib.l4moe_check_device_status.argtypes = [vp, vp]
+    lib.l4moe_launch_count.argtypes = [vp]
+    lib.l4moe_launch_count.restype = ctypes.c_uint64
+    lib.l4moe_last_error.argtypes = [vp]
+    lib.l4moe_last_error.restype = ctypes.c_char_p
+    lib.l4moe_status_string.argtypes = [i32]
+    lib.l4moe_status_string.restype = ctypes.c_char_p
+    lib.l4moe_version.argtypes = []
+    for name in ("l4moe_create", "l4moe_set_workspace", "l4moe_set_router_bias",
+                 "l4moe_set_fp8_scales", "l4moe_forward", "l4moe_forward_host",
+                 "l4moe_get_routing", "l4moe_check_device_status", "l4moe_version"):
+        getattr(lib, name).restype = ctypes.c_int
+    _lib = lib
+    return lib
+
+
+def _ptr(t) -> int | None:
+    if t is None:
+        return None
+    if isinstance(t, int):
+        return t
+    if not t.is_contiguous():
+        raise ValueError("l4moe: tensors must be contiguous (row-major)")
+    return t.data_ptr()
+
+
+def _ptr_array(tensors):
+    arr = (ctypes.c_void_p * len(tensors))()
+    for i, t in enumerate(tensors):
+        arr[i] = _ptr(t)
+    return arr
+
+
+def _stream_handle(stream) -> int | None:
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    if isinstance(stream, int):
+        return stream
+    return stream.cuda_stream
+
+
+class _DevView:
+    """Zero-copy torch view of a device buffer (CUDA array interface)."""
+
+    def __init__(self, ptr, shape, typestr):
+        self.__cuda_array_interface__ = {"shape": tuple(shape), "typestr": typestr,
+                                         "data": (int(ptr), False), "version": 3, "strides": None}
+
+
+class L4MoE:
+    """One MoE feed-forward layer (d_model, expert_ffn, shared_ffn, num_experts, dtype)."""
+
+    def __init__(self, d_model: int, expert_ffn: int, shared_ffn: int, num_experts: int,
+                 dtype: str = "bf16"):
+        self._lib = load_library()
+        self.params = Params(d_model, expert_ffn, shared_ffn, num_experts, DTYPES[dtype])
+        self.d_model, self.expert_ffn, self.shared_ffn = d_model, expert_ffn, shared_ffn
+        self.num_experts, self.dtype = num_experts, dtype
+        h = ctypes.c_void_p()
+        st = self._lib.l4moe_create(ctypes.byref(self.params), ctypes.byref(h))
+        if st != OK:
+            raise L4MoEError(st, self._lib.l4moe_last_error(None).decode())
+        self._h = h
+        self._keep = []
+        self.last_T = 0
+
+    def close(self):
+        if getattr(self, "_h", None):
+            self._lib.l4moe_destroy(self._h)
+            self._h = None
+
+    def __del__(self):
+        try:
+            self.close()
+        except Exception:
+            pass
+
+    def _check(self, st: int):
+        if st != OK:
+            raise L4MoEError(st, self._lib.l4moe_last_error(self._h).decode())
+
+    def workspace_size(self, max_tokens: int) -> int:
+        return int(self._lib.l4moe_workspace_size(self._h, max_tokens))
+
+    def set_workspace(self, buf: torch.Tensor, max_tokens: int):
+        self._check(self._lib.l4moe_set_workspace(self._h, _ptr(buf), buf.numel() * buf.element_size(),
+                                                  max_tokens))
+        self._keep.append(buf)
+
+    def set_router_bias(self, bias: torch.Tensor | None):
+        self._check(self._lib.l4moe_set_router_bias(self._h, _ptr(bias)))
+        self._bias = bias
+
+    def set_fp8_scales(self, s_gate_up, s_down, ss_gate_up, ss_down):
+        a, b = _ptr_array(s_gate_up), _ptr_array(s_down)
+        self._check(self._lib.l4moe_set_fp8_scales(self._h, a, b, _ptr(ss_gate_up), _ptr(ss_down)))
+        self._scales = (list(s_gate_up), list(s_down), ss_gate_up, ss_down)
+
+    def _weights(self, W_gate_up, W_down):
+        key = (tuple(_ptr(w) for w in W_gate_up), tuple(_ptr(w) for w in W_down))
+        if getattr(self, "_wkey", None) != key:
+            self._wkey = key
+            self._warr = (_ptr_array(W_gate_up), _ptr_array(W_down))
+        return self._warr
+
+    def forward(self, x, W_router, W_gate_up, W_down, Ws_gate_up, Ws_down, out=None, stream=None):
+        T = x.shape[0]
+        if out is None:
+            out = torch.empty((T, self.d_model), dtype=x.dtype, device=x.device)
+        gu, dn = self._weights(W_gate_up, W_down)
+        self._check(self._lib.l4moe_forward(self._h, T, _ptr(x), _ptr(W_router), gu, dn,
+                                            _ptr(Ws_gate_up), _ptr(Ws_down), _ptr(out),
+                                            _stream_handle(stream)))
+        self.last_T = T
+        return out
+
+    def forward_host(self, x_host, W_router, W_gate_up, W_down, Ws_gate_up, Ws_down, out_host,
+                     stream=None):
+        T = x_host.shape[0]
+        gu, dn = self._weights(W_gate_up, W_down)
+        self._check(self._lib.l4moe_forward_host(self._h, T, _ptr(x_host), _ptr(W_router), gu, dn,
+                                                 _ptr(Ws_gate_up), _ptr(Ws_down), _ptr(out_host),
+                                                 _stream_handle(stream)))
+        self.last_T = T
+        return out_host
+
+    def routing(self):
+        """Zero-copy device views of the last forward's routing (valid until
+        the next forward on this handle)."""
+        ptrs = [ctypes.c_void_p() for _ in range(7)]
+        self._check(self._lib.l4moe_get_routing(self._h, *[ctypes.byref(p) for p in ptrs]))
+        T, E = self.last_T, self.num_experts
+        spec = [("idx", (T,), "<i4"), ("gate", (T,), "<f4"), ("lmax", (T,), "<f4"),
+                ("margin", (T,), "<f4"), ("counts", (E,), "<i4"), ("offsets", (E + 1,), "<i4"),
+                ("perm", (T,), "<i4")]
+        out = {}
+        for (name, shape, ts), p in zip(spec, ptrs):
+            out[name] = torch.as_tensor(_DevView(p.value, shape, ts), device="cuda")
+        return out
+
+    def check_device_status(self, stream=None):
+        self._check(self._lib.l4moe_check_device_status(self._h, _stream_handle(stream)))
+
+    @property
+    def launch_count(self) -> int:
+        return int(self._lib.l4moe_launch_count(self._h))

@@ -1,0 +1,559 @@
+// l4moe.cu -- host side of the C ABI declared in include/l4moe.h: argument
+// checks, workspace layout, TMA descriptor cache and the launch sequence
+//
+//   router -> permute (counts, scan, slots, work lists) -> copy of x into
+//   expert order -> grouped gate/up (shared expert + routed experts; gate and
+//   SwiGLU in the epilogue) -> grouped down (shared + routed contraction in
+//   one accumulator, un-permuted store)
+//
+// all enqueued on the caller's stream with no host synchronisation.
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+#include <algorithm>
+#include <cstdio>
+#include <cstring>
+#include <mutex>
+#include <string>
+#include <vector>
+
+#include "l4moe.h"
+#include "moe_gemm.cuh"
+#include "permute.cuh"
+#include "router.cuh"
+
+using namespace l4moe;
+
+namespace {
+
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
+                                  const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
+                                  const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                  CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+    static EncodeTiledFn fn = nullptr;
+    static std::once_flag once;
+    std::call_once(once, [] {
+        void* p = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) ==
+                cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<EncodeTiledFn>(p);
+    });
+    return fn;
+}
+
+// 2-D row-major tensor [outer, inner] with 128-byte swizzled boxes.
+bool encode_2d(CUtensorMap* m, CUtensorMapDataType dt, const void* base, uint64_t inner,
+               uint64_t outer, uint64_t row_bytes, uint32_t box_inner, uint32_t box_outer,
+               CUtensorMapSwizzle swz = CU_TENSOR_MAP_SWIZZLE_128B) {
+    EncodeTiledFn enc = encode_fn();
+    if (!enc) return false;
+    cuuint64_t dims[2] = {inner, outer};
+    cuuint64_t strides[1] = {row_bytes};
+    cuuint32_t box[2] = {box_inner, box_outer};
+    cuuint32_t estr[2] = {1, 1};
+    return enc(m, dt, 2, const_cast<void*>(base), dims, strides, box, estr,
+               CU_TENSOR_MAP_INTERLEAVE_NONE, swz,
+               CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+struct WsLayout {
+    size_t err, idx, gate, lmax, margin, inv, perm, gslot, counts, offsets, tab_gu, tab_dn, xg, hr,
+        hs, xin, xout, total;
+};
+
+size_t act_bytes(l4moe_dtype dt) { return dt == L4MOE_F32 ? 4 : 2; }
+size_t w_bytes(l4moe_dtype dt) { return dt == L4MOE_F32 ? 4 : (dt == L4MOE_BF16 ? 2 : 1); }
+
+WsLayout ws_layout(const l4moe_params& p, int T) {
+    WsLayout L{};
+    size_t off = 0;
+    auto take = [&](size_t bytes) {
+        const size_t o = off;
+        off += (bytes + 255) & ~size_t(255);
+        return o;
+    };
+    const size_t t = (size_t)std::max(T, 1), E = (size_t)p.num_experts, es = act_bytes(p.dtype);
+    L.err = take(256);
+    L.idx = take(4 * t);
+    L.gate = take(4 * t);
+    L.lmax = take(4 * t);
+    L.margin = take(4 * t);
+    L.inv = take(4 * t);
+    L.perm = take(4 * t);
+    L.gslot = take(4 * t);
+    L.counts = take(4 * E);
+    L.offsets = take(4 * (E + 1));
+    L.tab_gu = take(sizeof(GroupTable));
+    L.tab_dn = take(sizeof(GroupTable));
+    L.xg = take(t * p.d_model * es);
+    L.hr = take(t * p.expert_ffn * es);
+    L.hs = take(t * p.shared_ffn * es);
+    L.xin = take(t * p.d_model * es);
+    L.xout = take(t * p.d_model * es);
+    L.total = off;
+    return L;
+}
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+}  // namespace
+
+struct l4moe_handle {
+    l4moe_params p{};
+    int device = -1;
+    int sms = 0;
+    uint8_t* ws = nullptr;
+    size_t ws_bytes = 0;
+    int ws_tokens = 0;
+    bool ws_owned = false;
+    const float* bias = nullptr;
+    std::vector<const float*> s_gu, s_dn;
+    const float* ss_gu = nullptr;
+    const float* ss_dn = nullptr;
+    // TMA descriptors of the weights, keyed by pointer value
+    std::vector<const void*> key_gu, key_dn;
+    const void* key_sgu = nullptr;
+    const void* key_sdn = nullptr;
+    std::vector<CUtensorMap> h_maps;  // [2][E+1]: gate/up set then down set
+    CUtensorMap* d_maps = nullptr;
+    uint64_t launches = 0;
+    std::string err;
+    int last_T = 0;
+};
+
+namespace {
+
+thread_local std::string g_create_error;
+
+l4moe_status fail(l4moe_handle* h, l4moe_status s, const std::string& msg) {
+    if (h) h->err = msg;
+    else g_create_error = msg;
+    return s;
+}
+
+l4moe_status cuda_fail(l4moe_handle* h, cudaError_t e, const char* what) {
+    return fail(h, L4MOE_ERR_CUDA, std::string(what) + ": " + cudaGetErrorString(e));
+}
+
+l4moe_status ensure_workspace(l4moe_handle* h, int T) {
+    if (h->ws && T <= h->ws_tokens) return L4MOE_OK;
+    if (h->ws && !h->ws_owned)
+        return fail(h, L4MOE_ERR_WORKSPACE, "caller workspace is sized for fewer tokens than T");
+    if (h->ws_owned && h->ws) {
+        cudaFree(h->ws);  // implicit device sync; only when T grows
+        h->ws = nullptr;
+    }
+    const int cap = std::max(T, 256);
+    const WsLayout L = ws_layout(h->p, cap);
+    void* p = nullptr;
+    cudaError_t e = cudaMalloc(&p, L.total);
+    if (e != cudaSuccess) return cuda_fail(h, e, "workspace cudaMalloc");
+    e = cudaMemset(p, 0, 256);
+    if (e != cudaSuccess) return cuda_fail(h, e, "workspace cudaMemset");
+    h->ws = static_cast<uint8_t*>(p);
+    h->ws_bytes = L.total;
+    h->ws_tokens = cap;
+    h->ws_owned = true;
+    return L4MOE_OK;
+}
+
+// (Re)build the weight descriptors when any weight pointer changed.
+l4moe_status ensure_weight_maps(l4moe_handle* h, const void* const* Wgu, const void* const* Wdn,
+                                const void* Wsgu, const void* Wsdn, cudaStream_t st) {
+    const int E = h->p.num_experts;
+    bool same = h->d_maps && h->key_sgu == Wsgu && h->key_sdn == Wsdn;
+    for (int e = 0; same && e < E; ++e) same = h->key_gu[e] == Wgu[e] && h->key_dn[e] == Wdn[e];
+    if (same) return L4MOE_OK;
+    const int d = h->p.d_model, F = h->p.expert_ffn, Fs = h->p.shared_ffn;
+    const size_t wb = w_bytes(h->p.dtype);
+    CUtensorMapDataType dt = h->p.dtype == L4MOE_F32 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT32
+                             : h->p.dtype == L4MOE_BF16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16
+                                                        : CU_TENSOR_MAP_DATA_TYPE_UINT8;
+    const uint32_t bk = h->p.dtype == L4MOE_F32 ? 32 : 64;  // K rows per box
+    const uint32_t bw = (uint32_t)(128 / wb);               // features per box
+    // MN-major 32-bit operands need the 32-byte swizzle unit
+    const CUtensorMapSwizzle swz = h->p.dtype == L4MOE_F32 ? CU_TENSOR_MAP_SWIZZLE_128B_ATOM_32B
+                                                           : CU_TENSOR_MAP_SWIZZLE_128B;
+    h->h_maps.assign(2 * (E + 1), CUtensorMap{});
+    for (int e = 0; e <= E; ++e) {
+        const bool sh = (e == E);
+        const void* gu = sh ? Wsgu : Wgu[e];
+        const void* dn = sh ? Wsdn : Wdn[e];
+        const int f = sh ? Fs : F;
+        if (!encode_2d(&h->h_maps[e], dt, gu, 2ull * f, (uint64_t)d, 2ull * f * wb, bw, bk, swz) ||
+            !encode_2d(&h->h_maps[E + 1 + e], dt, dn, (uint64_t)d, (uint64_t)f, (uint64_t)d * wb, bw,
+                       bk, swz))
+            return fail(h, L4MOE_ERR_CUDA, "cuTensorMapEncodeTiled failed for a weight");
+    }
+    if (!h->d_maps) {
+        cudaError_t e = cudaMalloc(&h->d_maps, sizeof(CUtensorMap) * 2 * (E + 1));
+        if (e != cudaSuccess) return cuda_fail(h, e, "descriptor cudaMalloc");
+    }
+    // pageable source: returns once the bytes are staged, so h_maps may change later
+    cudaError_t e = cudaMemcpyAsync(h->d_maps, h->h_maps.data(), sizeof(CUtensorMap) * 2 * (E + 1),
+                                    cudaMemcpyHostToDevice, st);
+    if (e != cudaSuccess) return cuda_fail(h, e, "descriptor upload");
+    h->key_gu.assign(Wgu, Wgu + E);
+    h->key_dn.assign(Wdn, Wdn + E);
+    h->key_sgu = Wsgu;
+    h->key_sdn = Wsdn;
+    return L4MOE_OK;
+}
+
+template <typename K>
+void set_smem_attr(K kernel, size_t bytes) {
+    cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)bytes);
+}
+
+template <typename ET, int NT, int TPT, int NG>
+void launch_router_t(const void* x, const void* Wr, const float* bias, int T, int d, int E,
+                     int32_t* idx, float* gate, float* lmax, float* margin, cudaStream_t st) {
+    constexpr size_t smem = router_smem_bytes<NT, TPT, NG>();
+    static std::once_flag once;
+    std::call_once(once, [] { set_smem_attr(router_kernel<ET, NT, TPT, NG>, smem); });
+    const int TT = NT / TPT;
+    const int wr_vec = (E % Vec16<ET>::N) == 0 ? 1 : 0;
+    router_kernel<ET, NT, TPT, NG><<<(T + TT - 1) / TT, NT, smem, st>>>(
+        static_cast<const ET*>(x), static_cast<const ET*>(Wr), bias, T, d, E, wr_vec, idx, gate,
+        lmax, margin);
+}
+
+template <typename ET>
+void launch_router(const void* x, const void* Wr, const float* bias, int T, int d, int E,
+                   int32_t* idx, float* gate, float* lmax, float* margin, cudaStream_t st) {
+    const int EG = (E + 3) / 4;
+    if (EG <= 1) launch_router_t<ET, 128, 1, 1>(x, Wr, bias, T, d, E, idx, gate, lmax, margin, st);
+    else if (EG <= 2) launch_router_t<ET, 128, 2, 1>(x, Wr, bias, T, d, E, idx, gate, lmax, margin, st);
+    else if (EG <= 4) launch_router_t<ET, 128, 4, 1>(x, Wr, bias, T, d, E, idx, gate, lmax, margin, st);
+    else if (EG <= 8) launch_router_t<ET, 128, 8, 1>(x, Wr, bias, T, d, E, idx, gate, lmax, margin, st);
+    else if (EG <= 16) launch_router_t<ET, 256, 8, 2>(x, Wr, bias, T, d, E, idx, gate, lmax, margin, st);
+    else if (EG <= 32) launch_router_t<ET, 256, 8, 4>(x, Wr, bias, T, d, E, idx, gate, lmax, margin, st);
+    else launch_router_t<ET, 256, 8, 8>(x, Wr, bias, T, d, E, idx, gate, lmax, margin, st);
+}
+
+template <int MODE, typename ET>
+void launch_gemm(int grid, const CUtensorMap& b_routed, const CUtensorMap& b_shared,
+                 const GemmArgs& a, cudaStream_t st) {
+    using Cfg = GemmCfg<MODE, ET>;
+    static std::once_flag once;
+    std::call_once(once, [] { set_smem_attr(moe_gemm_kernel<MODE, ET>, Cfg::SMEM_BYTES); });
+    moe_gemm_kernel<MODE, ET><<<grid, 192, Cfg::SMEM_BYTES, st>>>(b_routed, b_shared, a);
+}
+
+template <typename ET>
+l4moe_status run_layer(l4moe_handle* h, int T, const void* x, const void* Wr,
+                       const void* const* Wgu, const void* const* Wdn, const void* Wsgu,
+                       const void* Wsdn, void* out, cudaStream_t st) {
+    const l4moe_params& p = h->p;
+    const int d = p.d_model, F = p.expert_ffn, Fs = p.shared_ffn, E = p.num_experts;
+    const WsLayout L = ws_layout(p, h->ws_tokens);
+    uint8_t* w = h->ws;
+    unsigned* err = reinterpret_cast<unsigned*>(w + L.err);
+    int32_t* idx = reinterpret_cast<int32_t*>(w + L.idx);
+    float* gate = reinterpret_cast<float*>(w + L.gate);
+    float* lmax = reinterpret_cast<float*>(w + L.lmax);
+    float* margin = reinterpret_cast<float*>(w + L.margin);
+    int32_t* inv = reinterpret_cast<int32_t*>(w + L.inv);
+    int32_t* perm = reinterpret_cast<int32_t*>(w + L.perm);
+    float* gslot = reinterpret_cast<float*>(w + L.gslot);
+    int32_t* counts = reinterpret_cast<int32_t*>(w + L.counts);
+    int32_t* offsets = reinterpret_cast<int32_t*>(w + L.offsets);
+    GroupTable* tab_gu = reinterpret_cast<GroupTable*>(w + L.tab_gu);
+    GroupTable* tab_dn = reinterpret_cast<GroupTable*>(w + L.tab_dn);
+    ET* xg = reinterpret_cast<ET*>(w + L.xg);
+    ET* hr = reinterpret_cast<ET*>(w + L.hr);
+    ET* hs = reinterpret_cast<ET*>(w + L.hs);
+
+    // per-call activation descriptors (K-major rows, boxes of 128 B x 64 rows)
+    const CUtensorMapDataType adt =
+        sizeof(ET) == 4 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT32 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16;
+    const uint32_t bk = (uint32_t)(128 / sizeof(ET));
+    CUtensorMap m_xg, m_x, m_hr, m_hs;
+    if (!encode_2d(&m_xg, adt, xg, d, T, (uint64_t)d * sizeof(ET), bk, 64) ||
+        !encode_2d(&m_x, adt, x, d, T, (uint64_t)d * sizeof(ET), bk, 64) ||
+        !encode_2d(&m_hr, adt, hr, F, T, (uint64_t)F * sizeof(ET), bk, 64) ||
+        !encode_2d(&m_hs, adt, hs, Fs, T, (uint64_t)Fs * sizeof(ET), bk, 64))
+        return fail(h, L4MOE_ERR_CUDA, "cuTensorMapEncodeTiled failed for an activation");
+
+    cudaError_t e;
+#define L4MOE_CHECK_LAUNCH(what)                                  \
+    do {                                                          \
+        ++h->launches;                                            \
+        if ((e = cudaGetLastError()) != cudaSuccess) return cuda_fail(h, e, what); \
+    } while (0)
+
+    launch_router<ET>(x, Wr, h->bias, T, d, E, idx, gate, lmax, margin, st);
+    L4MOE_CHECK_LAUNCH("router launch");
+
+    const int fb_gu_r = (F + kFeatTile - 1) / kFeatTile;
+    const int fb_gu_s = (Fs + kFeatTile - 1) / kFeatTile;
+    const int fb_dn = (d + kFeatTile - 1) / kFeatTile;
+    const size_t psmem = sizeof(int) * (34 * (size_t)E + 1);
+    permute_kernel<<<1, 1024, psmem, st>>>(idx, T, E, fb_gu_r, fb_gu_s, fb_dn, counts, offsets,
+                                           perm, inv, tab_gu, tab_dn, err);
+    L4MOE_CHECK_LAUNCH("permute launch");
+
+    const int sc_blocks = std::min((T + 7) / 8, h->sms * 8);
+    permute_rows_kernel<ET><<<sc_blocks, 256, 0, st>>>(static_cast<const ET*>(x), gate, inv, T, d,
+                                                        xg, gslot);
+    L4MOE_CHECK_LAUNCH("row permutation launch");
+
+    const int tb = (T + kTokTile - 1) / kTokTile;
+    auto grid_for = [&](long long tiles) { return (int)std::max(1LL, std::min<long long>(h->sms, tiles)); };
+
+    GemmArgs gu{};
+    gu.table = tab_gu;
+    gu.a_maps = h->d_maps;
+    gu.num_experts = E;
+    gu.k_routed = d;
+    gu.k_shared = d;
+    gu.k_pre = 0;
+    gu.m_routed = F;
+    gu.m_shared = Fs;
+    gu.up_routed = F;
+    gu.up_shared = Fs;
+    gu.out_routed = hr;          // routed hidden rows in slot order
+    gu.ld_routed = F;
+    gu.out_shared = hs;          // shared hidden rows, also stored in slot order
+    gu.ld_shared = Fs;
+    gu.rowmap_routed = nullptr;
+    gu.rowmap_shared = inv;
+    gu.colscale_routed = gslot;  // sigmoid gate of each routed slot
+    gu.err = err;
+    launch_gemm<MODE_GATEUP, ET>(
+        grid_for((long long)fb_gu_s * tb + (long long)fb_gu_r * (tb + std::min(E, T))), m_xg, m_x,
+        gu, st);
+    L4MOE_CHECK_LAUNCH("gate/up launch");
+
+    GemmArgs dn{};
+    dn.table = tab_dn;
+    dn.a_maps = h->d_maps + (E + 1);
+    dn.num_experts = E;
+    dn.k_routed = F;
+    dn.k_shared = 0;
+    dn.k_pre = Fs;               // shared expert's down contraction first
+    dn.m_routed = d;
+    dn.m_shared = d;
+    dn.out_routed = out;
+    dn.ld_routed = d;
+    dn.out_shared = out;
+    dn.ld_shared = d;
+    dn.rowmap_routed = perm;     // slot -> token: un-permute on store
+    dn.rowmap_shared = nullptr;
+    dn.colscale_routed = nullptr;
+    dn.err = err;
+    launch_gemm<MODE_DOWN, ET>(grid_for((long long)fb_dn * (tb + std::min(E, T))), m_hr, m_hs, dn, st);
+    L4MOE_CHECK_LAUNCH("down launch");
+#undef L4MOE_CHECK_LAUNCH
+    h->last_T = T;
+    return L4MOE_OK;
+}
+
+l4moe_status check_forward_args(l4moe_handle* h, int T, const void* x, const void* Wr,
+                                const void* const* Wgu, const void* const* Wdn, const void* Wsgu,
+                                const void* Wsdn, const void* out) {
+    if (!h) return L4MOE_ERR_ARG;
+    if (T < 0) return fail(h, L4MOE_ERR_ARG, "T must be >= 0");
+    if (!x || !Wr || !Wgu || !Wdn || !Wsgu || !Wsdn || !out)
+        return fail(h, L4MOE_ERR_ARG, "null tensor pointer");
+    const void* ptrs[] = {x, Wr, Wsgu, Wsdn, out};
+    for (const void* q : ptrs)
+        if (!aligned16(q)) return fail(h, L4MOE_ERR_ALIGN, "tensor pointer not 16-byte aligned");
+    for (int e = 0; e < h->p.num_experts; ++e) {
+        if (!Wgu[e] || !Wdn[e]) return fail(h, L4MOE_ERR_ARG, "null expert weight pointer");
+        if (!aligned16(Wgu[e]) || !aligned16(Wdn[e]))
+            return fail(h, L4MOE_ERR_ALIGN, "expert weight pointer not 16-byte aligned");
+    }
+    if (h->p.dtype == L4MOE_FP8_E4M3 && (h->s_gu.empty() || !h->ss_gu || !h->ss_dn))
+        return fail(h, L4MOE_ERR_DTYPE, "FP8 weights need l4moe_set_fp8_scales first");
+    return L4MOE_OK;
+}
+
+l4moe_status forward_impl(l4moe_handle* h, int T, const void* x, const void* Wr,
+                          const void* const* Wgu, const void* const* Wdn, const void* Wsgu,
+                          const void* Wsdn, void* out, cudaStream_t st) {
+    l4moe_status s;
+    if ((s = ensure_workspace(h, T)) != L4MOE_OK) return s;
+    if ((s = ensure_weight_maps(h, Wgu, Wdn, Wsgu, Wsdn, st)) != L4MOE_OK) return s;
+    switch (h->p.dtype) {
+    case L4MOE_F32: return run_layer<float>(h, T, x, Wr, Wgu, Wdn, Wsgu, Wsdn, out, st);
+    case L4MOE_BF16: return run_layer<__nv_bfloat16>(h, T, x, Wr, Wgu, Wdn, Wsgu, Wsdn, out, st);
+    default: return fail(h, L4MOE_ERR_UNSUPPORTED, "FP8 weight path not built in this library");
+    }
+}
+
+}  // namespace
+
+extern "C" {
+
+int l4moe_version(void) { return 100; }
+
+const char* l4moe_status_string(l4moe_status s) {
+    switch (s) {
+    case L4MOE_OK: return "L4MOE_OK";
+    case L4MOE_ERR_ARG: return "L4MOE_ERR_ARG";
+    case L4MOE_ERR_DTYPE: return "L4MOE_ERR_DTYPE";
+    case L4MOE_ERR_ALIGN: return "L4MOE_ERR_ALIGN";
+    case L4MOE_ERR_CUDA: return "L4MOE_ERR_CUDA";
+    case L4MOE_ERR_WORKSPACE: return "L4MOE_ERR_WORKSPACE";
+    case L4MOE_ERR_TIMEOUT: return "L4MOE_ERR_TIMEOUT";
+    case L4MOE_ERR_UNSUPPORTED: return "L4MOE_ERR_UNSUPPORTED";
+    }
+    return "L4MOE_ERR_UNKNOWN";
+}
+
+l4moe_status l4moe_create(const l4moe_params* params, l4moe_handle** out) {
+    if (!params || !out) return fail(nullptr, L4MOE_ERR_ARG, "null params or out");
+    *out = nullptr;
+    const l4moe_params& p = *params;
+    if (p.dtype != L4MOE_F32 && p.dtype != L4MOE_BF16 && p.dtype != L4MOE_FP8_E4M3)
+        return fail(nullptr, L4MOE_ERR_DTYPE, "unknown dtype");
+    if (p.d_model <= 0 || p.expert_ffn <= 0 || p.shared_ffn <= 0 || p.num_experts < 1 ||
+        p.num_experts > 256)
+        return fail(nullptr, L4MOE_ERR_ARG, "shape out of range (need d, F, Fs > 0 and 1 <= E <= 256)");
+    if (p.d_model % 64 || p.expert_ffn % 64 || p.shared_ffn % 64)
+        return fail(nullptr, L4MOE_ERR_ALIGN, "d_model, expert_ffn and shared_ffn must be multiples of 64");
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return fail(nullptr, L4MOE_ERR_CUDA, std::string("cudaGetDevice: ") + cudaGetErrorString(e));
+    int major = 0, minor = 0, sms = 0;
+    cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev);
+    cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, dev);
+    cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+    if (major != 10 || minor != 0)
+        return fail(nullptr, L4MOE_ERR_UNSUPPORTED, "this library is built for sm_100a (B200) only");
+    if (!encode_fn()) return fail(nullptr, L4MOE_ERR_UNSUPPORTED, "cuTensorMapEncodeTiled unavailable");
+    l4moe_handle* h = new l4moe_handle();
+    h->p = p;
+    h->device = dev;
+    h->sms = sms;
+    *out = h;
+    return L4MOE_OK;
+}
+
+void l4moe_destroy(l4moe_handle* h) {
+    if (!h) return;
+    if (h->ws_owned && h->ws) cudaFree(h->ws);
+    if (h->d_maps) cudaFree(h->d_maps);
+    delete h;
+}
+
+size_t l4moe_workspace_size(const l4moe_handle* h, int max_tokens) {
+    if (!h || max_tokens < 0) return 0;
+    return ws_layout(h->p, max_tokens).total;
+}
+
+l4moe_status l4moe_set_workspace(l4moe_handle* h, void* dev_ptr, size_t bytes, int max_tokens) {
+    if (!h) return L4MOE_ERR_ARG;
+    if (!dev_ptr || max_tokens < 1) return fail(h, L4MOE_ERR_ARG, "null workspace or max_tokens < 1");
+    if (reinterpret_cast<uintptr_t>(dev_ptr) & 255u)
+        return fail(h, L4MOE_ERR_ALIGN, "workspace must be 256-byte aligned");
+    if (bytes < ws_layout(h->p, max_tokens).total)
+        return fail(h, L4MOE_ERR_WORKSPACE, "workspace smaller than l4moe_workspace_size");
+    if (h->ws_owned && h->ws) cudaFree(h->ws);
+    h->ws = static_cast<uint8_t*>(dev_ptr);
+    h->ws_bytes = bytes;
+    h->ws_tokens = max_tokens;
+    h->ws_owned = false;
+    cudaError_t e = cudaMemset(h->ws, 0, 256);
+    if (e != cudaSuccess) return cuda_fail(h, e, "workspace cudaMemset");
+    return L4MOE_OK;
+}
+
+l4moe_status l4moe_set_router_bias(l4moe_handle* h, const float* bias_dev) {
+    if (!h) return L4MOE_ERR_ARG;
+    if (bias_dev && (reinterpret_cast<uintptr_t>(bias_dev) & 3u))
+        return fail(h, L4MOE_ERR_ALIGN, "bias must be 4-byte aligned");
+    h->bias = bias_dev;
+    return L4MOE_OK;
+}
+
+l4moe_status l4moe_set_fp8_scales(l4moe_handle* h, const float* const* s_gate_up,
+                                  const float* const* s_down, const float* ss_gate_up,
+                                  const float* ss_down) {
+    if (!h) return L4MOE_ERR_ARG;
+    if (h->p.dtype != L4MOE_FP8_E4M3) return fail(h, L4MOE_ERR_DTYPE, "scales apply to FP8 weights only");
+    if (!s_gate_up || !s_down || !ss_gate_up || !ss_down) return fail(h, L4MOE_ERR_ARG, "null scale pointer");
+    const int E = h->p.num_experts;
+    for (int e = 0; e < E; ++e)
+        if (!s_gate_up[e] || !s_down[e]) return fail(h, L4MOE_ERR_ARG, "null expert scale pointer");
+    h->s_gu.assign(s_gate_up, s_gate_up + E);
+    h->s_dn.assign(s_down, s_down + E);
+    h->ss_gu = ss_gate_up;
+    h->ss_dn = ss_down;
+    return L4MOE_OK;
+}
+
+l4moe_status l4moe_forward(l4moe_handle* h, int T, const void* x, const void* W_router,
+                           const void* const* W_gate_up, const void* const* W_down,
+                           const void* Ws_gate_up, const void* Ws_down, void* out, void* stream) {
+    l4moe_status s = check_forward_args(h, T, x, W_router, W_gate_up, W_down, Ws_gate_up, Ws_down, out);
+    if (s != L4MOE_OK || T == 0) return s;
+    return forward_impl(h, T, x, W_router, W_gate_up, W_down, Ws_gate_up, Ws_down, out,
+                        static_cast<cudaStream_t>(stream));
+}
+
+l4moe_status l4moe_forward_host(l4moe_handle* h, int T, const void* x_host, const void* W_router,
+                                const void* const* W_gate_up, const void* const* W_down,
+                                const void* Ws_gate_up, const void* Ws_down, void* out_host,
+                                void* stream) {
+    l4moe_status s =
+        check_forward_args(h, T, x_host, W_router, W_gate_up, W_down, Ws_gate_up, Ws_down, out_host);
+    if (s != L4MOE_OK || T == 0) return s;
+    if ((s = ensure_workspace(h, T)) != L4MOE_OK) return s;
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    const WsLayout L = ws_layout(h->p, h->ws_tokens);
+    void* xin = h->ws + L.xin;
+    void* xout = h->ws + L.xout;
+    const size_t bytes = (size_t)T * h->p.d_model * act_bytes(h->p.dtype);
+    cudaError_t e = cudaMemcpyAsync(xin, x_host, bytes, cudaMemcpyHostToDevice, st);
+    if (e != cudaSuccess) return cuda_fail(h, e, "input host-to-device copy");
+    if ((s = forward_impl(h, T, xin, W_router, W_gate_up, W_down, Ws_gate_up, Ws_down, xout, st)) != L4MOE_OK)
+        return s;
+    e = cudaMemcpyAsync(out_host, xout, bytes, cudaMemcpyDeviceToHost, st);
+    if (e != cudaSuccess) return cuda_fail(h, e, "output device-to-host copy");
+    return L4MOE_OK;
+}
+
+l4moe_status l4moe_get_routing(const l4moe_handle* h, const int32_t** idx, const float** gate,
+                               const float** lmax, const float** margin, const int32_t** counts,
+                               const int32_t** offsets, const int32_t** perm) {
+    if (!h || !h->ws) return L4MOE_ERR_ARG;
+    const WsLayout L = ws_layout(h->p, h->ws_tokens);
+    if (idx) *idx = reinterpret_cast<const int32_t*>(h->ws + L.idx);
+    if (gate) *gate = reinterpret_cast<const float*>(h->ws + L.gate);
+    if (lmax) *lmax = reinterpret_cast<const float*>(h->ws + L.lmax);
+    if (margin) *margin = reinterpret_cast<const float*>(h->ws + L.margin);
+    if (counts) *counts = reinterpret_cast<const int32_t*>(h->ws + L.counts);
+    if (offsets) *offsets = reinterpret_cast<const int32_t*>(h->ws + L.offsets);
+    if (perm) *perm = reinterpret_cast<const int32_t*>(h->ws + L.perm);
+    return L4MOE_OK;
+}
+
+l4moe_status l4moe_check_device_status(l4moe_handle* h, void* stream) {
+    if (!h) return L4MOE_ERR_ARG;
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    cudaError_t e = cudaStreamSynchronize(st);
+    if (e != cudaSuccess) return cuda_fail(h, e, "stream synchronize");
+    if (!h->ws) return L4MOE_OK;
+    unsigned word = 0;
+    e = cudaMemcpy(&word, h->ws + ws_layout(h->p, h->ws_tokens).err, sizeof(word), cudaMemcpyDeviceToHost);
+    if (e != cudaSuccess) return cuda_fail(h, e, "error word read");
+    if (word == 0) return L4MOE_OK;
+    cudaMemset(h->ws + ws_layout(h->p, h->ws_tokens).err, 0, sizeof(word));
+    char msg[160];
+    snprintf(msg, sizeof msg, "device error word 0x%x (1: producer wait, 2: MMA wait, 4: epilogue wait, 8: bad expert index)", word);
+    return fail(h, (word & 7u) ? L4MOE_ERR_TIMEOUT : L4MOE_ERR_ARG, msg);
+}
+
+uint64_t l4moe_launch_count(const l4moe_handle* h) { return h ? h->launches : 0; }
+
+const char* l4moe_last_error(const l4moe_handle* h) {
+    return h ? h->err.c_str() : g_create_error.c_str();
+}
+
+}  // extern "C"

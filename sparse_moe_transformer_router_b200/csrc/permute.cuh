@@ -1,0 +1,205 @@
+// permute.cuh -- token dispatch: per-expert histogram, exclusive scan,
+// stable slot assignment, and the copy of the input rows into expert order.
+//
+// superteams.ai "Llama 4" glossary, routing sketch: each token is handed to
+// the one expert its router picked.  On the GPU the tokens of each expert are
+// gathered into a contiguous block of rows (expert-ordered "slots") so the
+// experts run as a grouped GEMM.  The order inside an expert is by token
+// index (stable), so slot = offsets[e] + #{t' < t : idx[t'] == e}.
+#pragma once
+#include <cuda_bf16.h>
+#include <cstdint>
+
+#include "ptx.cuh"
+
+namespace l4moe {
+
+// One GEMM launch's work list: the non-empty groups (a routed expert or the
+// shared expert), the rows each group owns in its activation matrix, and the
+// first tile of each group in the launch's linear tile order.  Tiles of a
+// group are (feature block) x (token block); group g holds
+// ceil(rows/kTokTile) * feature_blocks tiles.
+constexpr int kMaxGroups = 257;  // 256 routed experts + the shared expert
+constexpr int kTokTile = 256;    // tokens per GEMM tile (MMA N, swap-AB)
+constexpr int kFeatTile = 128;   // output features per GEMM tile (MMA M)
+
+struct GroupTable {
+    int num_groups;
+    int total_tiles;
+    int pad0, pad1;
+    int rows[kMaxGroups];
+    int row0[kMaxGroups];
+    int expert[kMaxGroups];       // 0..E-1 routed, E = shared
+    int tile_start[kMaxGroups + 1];
+};
+
+__device__ __forceinline__ int warp_incl_scan(int v) {
+    const int lane = threadIdx.x & 31;
+#pragma unroll
+    for (int off = 1; off < 32; off <<= 1) {
+        const int o = __shfl_up_sync(0xffffffffu, v, off);
+        if (lane >= off) v += o;
+    }
+    return v;
+}
+
+// Warp 0 writes one table from candidate groups [0, G): candidate g has
+// rows(g), row0(g), expert(g), feature blocks fb(g).  Empty groups are left
+// out.
+template <typename RowsF, typename Row0F, typename ExpF, typename FbF>
+__device__ void build_table(GroupTable* tab, int G, RowsF rows_of, Row0F row0_of, ExpF exp_of,
+                            FbF fb_of) {
+    const int lane = threadIdx.x & 31;
+    int n_base = 0, t_base = 0;
+    for (int base = 0; base < G; base += 32) {
+        const int g = base + lane;
+        int rows = 0, tiles = 0;
+        if (g < G) {
+            rows = rows_of(g);
+            tiles = rows > 0 ? ((rows + kTokTile - 1) / kTokTile) * fb_of(g) : 0;
+        }
+        const int flag = tiles > 0 ? 1 : 0;
+        const int fi = warp_incl_scan(flag);
+        const int ti = warp_incl_scan(tiles);
+        if (flag) {
+            const int pos = n_base + fi - 1;
+            tab->rows[pos] = rows;
+            tab->row0[pos] = row0_of(g);
+            tab->expert[pos] = exp_of(g);
+            tab->tile_start[pos] = t_base + ti - tiles;
+        }
+        n_base += __shfl_sync(0xffffffffu, fi, 31);
+        t_base += __shfl_sync(0xffffffffu, ti, 31);
+    }
+    if (lane == 0) {
+        tab->num_groups = n_base;
+        tab->total_tiles = t_base;
+        tab->tile_start[n_base] = t_base;
+    }
+}
+
+// Single CTA of 1024 threads.  Writes counts[E], offsets[E+1], perm[T]
+// (slot -> token), inv[T] (token -> slot) and two work lists:
+//   tab_gu : shared expert (rows T) then the routed experts, gate/up GEMM
+//   tab_dn : routed experts (rows = their slots), down GEMM with the shared
+//            expert's K segment fused in front
+// smem: wcnt[32][E] + running[E] ints.
+__global__ void __launch_bounds__(1024) permute_kernel(const int32_t* __restrict__ idx, int T,
+                                                       int E, int fb_gu_routed, int fb_gu_shared,
+                                                       int fb_down, int32_t* __restrict__ counts,
+                                                       int32_t* __restrict__ offsets,
+                                                       int32_t* __restrict__ perm,
+                                                       int32_t* __restrict__ inv,
+                                                       GroupTable* tab_gu, GroupTable* tab_dn,
+                                                       unsigned* err) {
+    extern __shared__ int psm[];
+    int* wcnt = psm;              // [32][E]
+    int* running = psm + 32 * E;  // [E]
+    int* soff = running + E;      // [E + 1]
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+
+    for (int e = tid; e < E; e += 1024) running[e] = 0;
+    __syncthreads();
+    for (int c0 = 0; c0 < T; c0 += 1024) {
+        for (int i = tid; i < 32 * E; i += 1024) wcnt[i] = 0;
+        __syncthreads();
+        const int t = c0 + tid;
+        int e = -1;
+        if (t < T) {
+            e = idx[t];
+            if (e < 0 || e >= E) {
+                atomicOr(err, DEV_ERR_BAD_INDEX);
+                e = -1;
+            }
+        }
+        const unsigned same = __match_any_sync(0xffffffffu, e);
+        const int lane_rank = __popc(same & ((1u << lane) - 1u));
+        if (e >= 0 && lane_rank == 0) wcnt[warp * E + e] = __popc(same);
+        __syncthreads();
+        for (int x = tid; x < E; x += 1024) {  // prefix over warps, per expert
+            int acc = running[x];
+            for (int w = 0; w < 32; ++w) {
+                const int v = wcnt[w * E + x];
+                wcnt[w * E + x] = acc;
+                acc += v;
+            }
+            running[x] = acc;
+        }
+        __syncthreads();
+        if (e >= 0) inv[t] = wcnt[warp * E + e] + lane_rank;  // rank inside expert
+        __syncthreads();
+    }
+    // exclusive scan of the counts (warp 0, up to 8 experts per lane)
+    if (warp == 0) {
+        int local[8];
+        int sum = 0;
+#pragma unroll
+        for (int j = 0; j < 8; ++j) {
+            const int e = lane * 8 + j;
+            local[j] = (e < E) ? running[e] : 0;
+            sum += local[j];
+        }
+        const int incl = warp_incl_scan(sum);
+        int acc = incl - sum;
+#pragma unroll
+        for (int j = 0; j < 8; ++j) {
+            const int e = lane * 8 + j;
+            if (e < E) {
+                soff[e] = acc;
+                offsets[e] = acc;
+                counts[e] = local[j];
+            }
+            acc += local[j];
+        }
+        if (lane == 31) {
+            soff[E] = incl;
+            offsets[E] = incl;
+        }
+    }
+    __syncthreads();
+    for (int t = tid; t < T; t += 1024) {
+        const int e = idx[t];
+        if (e >= 0 && e < E) {
+            const int slot = soff[e] + inv[t];
+            inv[t] = slot;
+            perm[slot] = t;
+        }
+    }
+    if (warp == 0) {
+        // gate/up: candidate 0 is the shared expert, 1..E the routed experts
+        build_table(
+            tab_gu, E + 1, [&](int g) { return g == 0 ? T : running[g - 1]; },
+            [&](int g) { return g == 0 ? 0 : soff[g - 1]; },
+            [&](int g) { return g == 0 ? E : g - 1; },
+            [&](int g) { return g == 0 ? fb_gu_shared : fb_gu_routed; });
+        build_table(
+            tab_dn, E, [&](int g) { return running[g]; }, [&](int g) { return soff[g]; },
+            [&](int g) { return g; }, [&](int) { return fb_down; });
+    }
+}
+
+// Expert-ordered copy of the input rows, xp[inv[t]] = x[t] (exact), and the
+// gate of each slot, gate_slot[inv[t]] = gate[t].  The sigmoid gate scales
+// the routed expert's input, which is linear in the gate/up contraction, so
+// it is applied to the fp32 accumulator in the GEMM epilogue instead of
+// rounding g * x to the activation type here.
+// One warp per token row, 16-byte vectors; d % (16 / sizeof(ET)) == 0.
+template <typename ET>
+__global__ void __launch_bounds__(256) permute_rows_kernel(const ET* __restrict__ x,
+                                                           const float* __restrict__ gate,
+                                                           const int32_t* __restrict__ inv,
+                                                           int T, int d, ET* __restrict__ xp,
+                                                           float* __restrict__ gate_slot) {
+    const int lane = threadIdx.x & 31;
+    const int warps = (gridDim.x * blockDim.x) >> 5;
+    for (int t = (blockIdx.x * blockDim.x + threadIdx.x) >> 5; t < T; t += warps) {
+        const int slot = inv[t];
+        if (lane == 0) gate_slot[slot] = gate[t];
+        const uint4* s = reinterpret_cast<const uint4*>(x + (size_t)t * d);
+        uint4* o = reinterpret_cast<uint4*>(xp + (size_t)slot * d);
+        const int nv = d * (int)sizeof(ET) / 16;
+        for (int i = lane; i < nv; i += 32) o[i] = s[i];
+    }
+}
+
+}  // namespace l4moe

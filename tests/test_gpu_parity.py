@@ -1,0 +1,124 @@
+"""CUDA path (through the C ABI) against the CPU oracle on the same seeded
+inputs: small layers element by element (several tiles, ragged tails, empty
+experts, degenerate routings), and the full-size workloads on sampled tokens
+plus full routing."""
+import numpy as np
+import pytest
+import torch
+
+from parity_util import (check_outputs, check_routing, make_layer, oracle_routing, run_gpu,
+                         sample_tokens)
+from sparse_moe_transformer_router_b200.workloads import (CONFIGS, DECODE_TOKENS, LayerConfig,
+                                                          generate)
+
+pytestmark = pytest.mark.gpu
+
+SMALL = {
+    # tiny fp32 workload: T=64, d=128, E=4, F=Fs=256
+    "tiny_f32": CONFIGS["tiny_f32"],
+    # several feature tiles (F = 384 -> 3), ragged token tiles per expert
+    "bf16_ragged": LayerConfig("bf16_ragged", 300, 256, 8, 384, 256, "bf16", wr_std=0.1),
+    # d not a multiple of the 128-feature tile; 3 token tiles per expert
+    "bf16_two_experts": LayerConfig("bf16_two_experts", 1100, 192, 2, 128, 192, "bf16", wr_std=0.1),
+    "f32_ragged": LayerConfig("f32_ragged", 300, 256, 8, 384, 256, "f32", wr_std=0.1),
+    # skewed loads with idle experts (router bias)
+    "bf16_zipf": LayerConfig("bf16_zipf", 512, 128, 16, 128, 128, "bf16", router="zipf", n_dead=4,
+                             wr_std=0.05),
+    "bf16_T1": LayerConfig("bf16_T1", 1, 256, 8, 256, 256, "bf16", wr_std=0.1),
+    "bf16_E1": LayerConfig("bf16_E1", 70, 128, 1, 128, 128, "bf16"),
+    "bf16_E256": LayerConfig("bf16_E256", 600, 128, 256, 64, 64, "bf16", wr_std=0.1),
+}
+
+
+@pytest.mark.parametrize("name", list(SMALL))
+def test_small_layer_matches_oracle(name):
+    cfg = SMALL[name]
+    inp = generate(cfg, seed=0, device="cuda")
+    layer = make_layer(inp)
+    out, r = run_gpu(layer, inp)
+    rep = check_routing(inp, r)
+    ratio = check_outputs(inp, out, None, rep["same"])
+    print(f"{name}: max|err|/rms = {ratio:.3e}, excluded {rep['excluded']}, flipped {rep['flipped']}")
+
+
+def test_zero_input_gives_zero_output_and_expert_zero():
+    cfg = LayerConfig("zero", 200, 128, 6, 128, 128, "bf16")
+    inp = generate(cfg, seed=1, device="cuda")
+    inp.x.zero_()
+    layer = make_layer(inp)
+    out, r = run_gpu(layer, inp)
+    assert torch.all(r["idx"] == 0)
+    assert torch.all(r["gate"] == 0.5)
+    assert torch.all(out == 0)
+
+
+def test_all_tokens_to_one_expert_and_saturated_gate():
+    cfg = LayerConfig("one_expert", 700, 128, 8, 128, 256, "bf16", wr_std=0.02)
+    inp = generate(cfg, seed=2, device="cuda")
+    bias = torch.full((8,), -50.0, device="cuda")
+    bias[5] = 60.0
+    inp.bias = bias
+    layer = make_layer(inp)
+    out, r = run_gpu(layer, inp)
+    assert torch.all(r["idx"] == 5)
+    assert torch.all(r["gate"] == 1.0)
+    assert r["counts"].cpu().tolist() == [0, 0, 0, 0, 0, 700, 0, 0]
+    rep = check_routing(inp, r)
+    check_outputs(inp, out, None, rep["same"])
+
+
+def test_repeatable_and_host_path_identical():
+    cfg = SMALL["bf16_ragged"]
+    inp = generate(cfg, seed=3, device="cuda")
+    layer = make_layer(inp)
+    out1, _ = run_gpu(layer, inp)
+    out2, _ = run_gpu(layer, inp)
+    assert torch.equal(out1, out2)
+    x_host = inp.x.cpu().pin_memory()
+    out_host = torch.empty_like(x_host).pin_memory()
+    layer.forward_host(x_host, inp.W_router, inp.W_gate_up, inp.W_down, inp.Ws_gate_up,
+                       inp.Ws_down, out_host)
+    torch.cuda.synchronize()
+    layer.check_device_status()
+    assert torch.equal(out_host, out1.cpu())
+
+
+def test_weight_pointer_change_rebuilds_descriptors():
+    cfg = LayerConfig("swap", 256, 128, 4, 128, 128, "bf16", wr_std=0.1)
+    a = generate(cfg, seed=4, device="cuda")
+    b = generate(cfg, seed=5, device="cuda")
+    b.x, b.W_router = a.x, a.W_router  # same routing input, different experts
+    layer = make_layer(a)
+    out_a, _ = run_gpu(layer, a)
+    out_b, r = run_gpu(layer, b)
+    rep = check_routing(b, r)
+    check_outputs(b, out_b, None, rep["same"])
+    assert not torch.equal(out_a, out_b)
+
+
+def _full_size(cfg, seed=0):
+    inp = generate(cfg, seed=seed, device="cuda")
+    layer = make_layer(inp)
+    out, r = run_gpu(layer, inp)
+    ora = oracle_routing(inp)
+    rep = check_routing(inp, r, ora)
+    toks = sample_tokens(r, rep, cfg.T, seed=seed)
+    ratio = check_outputs(inp, out, toks, rep["same"], rep["o_idx"])
+    print(f"{cfg.name}: {len(toks)} sampled tokens, max|err|/rms = {ratio:.3e}, "
+          f"excluded {rep['excluded']}, flipped {rep['flipped']}, "
+          f"experts with tokens {int(np.count_nonzero(rep['counts']))}")
+    del inp, layer
+    torch.cuda.empty_cache()
+
+
+def test_full_size_scout_prefill():
+    _full_size(CONFIGS["scout_prefill_bf16"])
+
+
+def test_full_size_maverick_prefill_zipf():
+    _full_size(CONFIGS["maverick_prefill_bf16"])
+
+
+@pytest.mark.parametrize("T", DECODE_TOKENS)
+def test_full_size_maverick_decode(T):
+    _full_size(CONFIGS["maverick_decode_bf16"].with_tokens(T))
