@@ -1,0 +1,411 @@
+"""Benchmark of the MoE feed-forward layer on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME] [--impl b200|reference]
+
+One step = one full forward of the layer (router, permutation, grouped
+gate/up, grouped down) over one batch of T synthetic tokens already resident
+in HBM.  The default workload is the Scout-shaped prefill layer (T = 4096,
+d_model 5120, 16 experts, expert and shared SwiGLU width 8192, bf16).  The
+metric is layer tokens/s; the JSON line also carries TFLOP/s on active FLOPs,
+the layer's roofline fraction, the dominant kernel's roofline (its events
+timed live on the launching stream), the end-to-end number through the
+host-buffer C-ABI call (input copy in, output copy out, every step), the
+oracle timed on the host cores, and the SM clocks sampled during the timed
+region.
+
+N > 1 (torchrun, one process per GPU): every rank runs its own replica on its
+own batch (tokens are independent, so the layer shards by tokens with no data
+exchange); value = all ranks' tokens / max-over-ranks time (weak scaling).
+
+--impl reference times the CPU oracle, as it stands, on the host cores on a
+bounded sample of the same workload (rank 0 only).
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import re
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+import numpy as np
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+from sparse_moe_transformer_router_b200 import accounting  # noqa: E402
+from sparse_moe_transformer_router_b200.workloads import CONFIGS, generate, to_storage_numpy  # noqa: E402
+
+DEFAULT_WORKLOAD = "scout_prefill_bf16"
+METRIC = "moe_layer_tokens_per_s"
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+
+
+def dist_env():
+    return int(os.environ.get("RANK", 0)), int(os.environ.get("WORLD_SIZE", 1)), \
+        int(os.environ.get("LOCAL_RANK", 0))
+
+
+def load_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            d = json.load(f)
+        return d, "measured"
+    return dict(FALLBACK_PEAKS), "fallback"
+
+
+class ClockSampler:
+    """nvidia-smi clock / throttle-reason samples during the timed region."""
+
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, device_index: int):
+        self.dev = device_index
+        self.proc = None
+        self.path = None
+
+    def start(self):
+        fd, self.path = tempfile.mkstemp(suffix=".csv")
+        os.close(fd)
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.dev), f"--query-gpu={self.FIELDS}",
+                 "--format=csv,noheader,nounits", "-lms", "100"],
+                stdout=open(self.path, "w"), stderr=subprocess.DEVNULL)
+        except (FileNotFoundError, OSError):
+            self.proc = None
+
+    def stop(self) -> dict:
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+        rows = []
+        with open(self.path) as f:
+            for line in f:
+                parts = [p.strip() for p in line.split(",")]
+                if len(parts) >= 9:
+                    rows.append(parts)
+        os.unlink(self.path)
+        if not rows:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": [], "samples": 0}
+        sm = [float(r[1]) for r in rows if r[1].replace(".", "").isdigit()]
+        mx = [float(r[2]) for r in rows if r[2].replace(".", "").isdigit()]
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({n for r in rows for n, v in zip(names, r[5:9]) if v.lower() == "active"})
+        return {"sm_mhz": statistics.median(sm) if sm else None,
+                "sm_max_mhz": max(mx) if mx else None, "reasons": reasons, "samples": len(rows)}
+
+
+def kernel_flops_bytes(cfg, counts):
+    """Algorithmic FLOPs / bytes per launch of each kernel."""
+    T, d, E, F, Fs = cfg.T, cfg.d_model, cfg.num_experts, cfg.expert_ffn, cfg.shared_ffn
+    a = accounting.ACT_BYTES[cfg.dtype]
+    w = accounting.W_BYTES[cfg.dtype]
+    touched = int(np.count_nonzero(counts))
+    return {
+        "router": {"flops": 2 * T * d * E, "bytes": T * d * a + d * E * a + T * 16},
+        "permute": {"flops": 0, "bytes": T * 4 * 4},
+        "row_copy": {"flops": 0, "bytes": 2 * T * d * a + T * 12},
+        "gemm_gate_up": {"flops": 4 * T * d * (F + Fs),
+                         "bytes": (touched * 2 * d * F + 2 * d * Fs) * w + 2 * T * d * a + T * (F + Fs) * a},
+        "gemm_down": {"flops": 2 * T * d * (F + Fs),
+                      "bytes": (touched * F * d + Fs * d) * w + T * (F + Fs) * a + T * d * a},
+    }
+
+
+def profile_traffic(kernel: str, workload: str):
+    """DRAM bytes per launch from the committed ncu summary of this kernel,
+    if the kernel sources are unchanged since it was taken (else None)."""
+    path = os.path.join(ROOT, "profiles", f"{kernel}__{workload}.md")
+    if not os.path.exists(path):
+        return None
+    text = open(path).read()
+    m_b = re.search(r"dram_bytes_per_launch:\s*([0-9.eE+]+)", text)
+    m_h = re.search(r"sources_sha256:\s*([0-9a-f]+)", text)
+    if not m_b or not m_h or m_h.group(1) != kernel_sources_sha():
+        return None
+    return float(m_b.group(1))
+
+
+def kernel_sources_sha() -> str:
+    h = hashlib.sha256()
+    csrc = os.path.join(ROOT, "sparse_moe_transformer_router_b200", "csrc")
+    for name in sorted(os.listdir(csrc)):
+        with open(os.path.join(csrc, name), "rb") as f:
+            h.update(name.encode())
+            h.update(f.read())
+    return h.hexdigest()[:16]
+
+
+def cpu_baseline(inp, budget_s: float = 15.0) -> dict:
+    """The oracle, as it stands, on the host cores: full-layer outputs for a
+    bounded sample of the workload's tokens; tokens/s."""
+    import oracle
+    cfg = inp.cfg
+    threads = oracle.num_threads()
+    x = to_storage_numpy(inp.x)
+    Wr = to_storage_numpy(inp.W_router)
+    bias = None if inp.bias is None else inp.bias.cpu().numpy()
+    Ws_gu = to_storage_numpy(inp.Ws_gate_up)
+    Ws_dn = to_storage_numpy(inp.Ws_down)
+    idx, _, _ = oracle.route(x, Wr, bias)
+
+    def run(n):
+        sel = np.arange(n, dtype=np.int32) * max(1, cfg.T // max(n, 1))
+        sel = sel[sel < cfg.T]
+        need = set(int(e) for e in idx[sel])
+        Wgu = [to_storage_numpy(inp.W_gate_up[e]) if e in need else None for e in range(cfg.num_experts)]
+        Wdn = [to_storage_numpy(inp.W_down[e]) if e in need else None for e in range(cfg.num_experts)]
+        kw = {}
+        if cfg.dtype == "fp8":
+            kw = dict(s_gate_up=[inp.s_gate_up[e].cpu().numpy() if e in need else None for e in range(cfg.num_experts)],
+                      s_down=[inp.s_down[e].cpu().numpy() if e in need else None for e in range(cfg.num_experts)],
+                      ss_gate_up=inp.ss_gate_up.cpu().numpy(), ss_down=inp.ss_down.cpu().numpy())
+        t0 = time.perf_counter()
+        oracle.forward(x, Wr, Wgu, Wdn, Ws_gu, Ws_dn, bias=bias, tokens=sel, **kw)
+        return len(sel), time.perf_counter() - t0
+
+    n, dt = run(max(1, threads))                      # calibration sample
+    per_tok = dt / n
+    n2 = int(max(1, min(cfg.T, budget_s / per_tok)))
+    n2 = max(threads, (n2 // max(1, threads)) * threads) if n2 >= threads else n2
+    n2 = min(n2, cfg.T)
+    n2, dt2 = run(n2)
+    return {"value": n2 / dt2, "unit": "tokens/s", "cores": threads, "kind": "oracle",
+            "sample": f"full-layer outputs (router + shared + routed SwiGLU, fp64) for {n2} of the "
+                      f"{cfg.T} tokens, evenly spaced, {dt2:.1f} s"}
+
+
+def run_reference(args, rank, world):
+    if rank != 0:
+        return
+    cfg = CONFIGS[args.workload]
+    dev = "cuda" if torch.cuda.is_available() else "cpu"
+    inp = generate(cfg, seed=0, device=dev)
+    per_step_budget = max(2.0, min(20.0, 120.0 / max(1, args.steps + args.warmup)))
+    for _ in range(args.warmup):
+        cpu_baseline(inp, budget_s=per_step_budget / 4)
+    vals, samples = [], []
+    cb = None
+    for _ in range(args.steps):
+        cb = cpu_baseline(inp, budget_s=per_step_budget)
+        vals.append(cb["value"])
+        samples.append(cb["sample"])
+    value = float(np.median(vals))
+    ms = cfg.T / value * 1e3
+    line = {"metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "f64", "data": "synthetic", "impl": "reference",
+            "config": config_dict(cfg, world),
+            "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": cb["cores"], "kind": "oracle",
+                             "sample": samples[-1] + "; value = median over steps; ms_per_step = T / value"},
+            "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+
+
+def config_dict(cfg, world):
+    return {"workload": cfg.name, "T": cfg.T, "d_model": cfg.d_model, "experts": cfg.num_experts,
+            "expert_ffn": cfg.expert_ffn, "shared_ffn": cfg.shared_ffn, "top_k": 1,
+            "router": cfg.router, "parallelism": f"replicas{world}" if world > 1 else "single",
+            "l2": "inputs larger than L2: every step streams all touched expert weights "
+                  "(GBs) through a 126 MB L2; no explicit flush"}
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=50)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--workload", default=DEFAULT_WORKLOAD, choices=sorted(CONFIGS))
+    ap.add_argument("--tokens", type=int, default=0, help="override T (decode sweeps)")
+    ap.add_argument("--experts", type=int, default=0,
+                    help="override E (smaller profiling captures)")
+    ap.add_argument("--impl", default="b200", choices=["b200", "reference"])
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--e2e-steps", type=int, default=0)
+    args = ap.parse_args()
+    args.warmup = max(args.warmup, 3)
+    rank, world, local = dist_env()
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        torch.cuda.set_device(local)
+        dist.init_process_group("nccl" if args.impl == "b200" else "gloo",
+                                timeout=datetime.timedelta(seconds=300))
+    if args.tokens:
+        CONFIGS[args.workload] = CONFIGS[args.workload].with_tokens(args.tokens)
+    if args.experts:
+        from dataclasses import replace
+        c = CONFIGS[args.workload]
+        CONFIGS[args.workload] = replace(c, num_experts=args.experts, name=f"{c.name}@E{args.experts}",
+                                         n_dead=min(c.n_dead, args.experts // 4))
+    if args.impl == "reference":
+        run_reference(args, rank, world)
+        if world > 1:
+            import torch.distributed as dist
+            dist.destroy_process_group()
+        return
+    run_b200(args, rank, world, local)
+
+
+def run_b200(args, rank, world, local):
+    from sparse_moe_transformer_router_b200.binding import L4MoE
+    torch.cuda.set_device(local)
+    cfg = CONFIGS[args.workload]
+    inp = generate(cfg, seed=rank, device="cuda")
+    layer = L4MoE(cfg.d_model, cfg.expert_ffn, cfg.shared_ffn, cfg.num_experts, cfg.dtype)
+    if inp.bias is not None:
+        layer.set_router_bias(inp.bias)
+    if cfg.dtype == "fp8":
+        layer.set_fp8_scales(inp.s_gate_up, inp.s_down, inp.ss_gate_up, inp.ss_down)
+    out = torch.empty((cfg.T, cfg.d_model), dtype=inp.x.dtype, device="cuda")
+    fwd = lambda: layer.forward(inp.x, inp.W_router, inp.W_gate_up, inp.W_down,  # noqa: E731
+                                inp.Ws_gate_up, inp.Ws_down, out=out)
+    stream = torch.cuda.current_stream()
+
+    def barrier():
+        if world > 1:
+            import torch.distributed as dist
+            dist.barrier()
+
+    def max_over_ranks(v: float) -> float:
+        if world == 1:
+            return v
+        import torch.distributed as dist
+        t = torch.tensor([v], device="cuda", dtype=torch.float64)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        return float(t.item())
+
+    for _ in range(args.warmup):
+        fwd()
+    torch.cuda.synchronize()
+    layer.check_device_status()
+    counts = layer.routing()["counts"].cpu().numpy()
+    layer.read_timing()  # drop anything recorded so far
+
+    # ---------------------------------------------------------------- timed
+    sampler = ClockSampler(local)
+    sampler.start()
+    layer.set_timing(True)
+    launches0 = layer.launch_count
+    barrier()
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(args.steps):
+        fwd()
+    e1.record(stream)
+    torch.cuda.synchronize()
+    barrier()
+    clocks = sampler.stop()
+    layer.set_timing(False)
+    launches = layer.launch_count - launches0
+    t_ms = max_over_ranks(e0.elapsed_time(e1))
+    ktimes = layer.read_timing()
+    layer.check_device_status()
+
+    ms_step = t_ms / args.steps
+    value = world * cfg.T * args.steps / (t_ms / 1e3)
+
+    # ------------------------------------------------------------- e2e (host buffers)
+    x_host = inp.x.cpu().pin_memory()
+    out_host = torch.empty_like(x_host).pin_memory()
+    e2e_steps = args.e2e_steps or max(3, min(args.steps, 20))
+    fwd_h = lambda: layer.forward_host(x_host, inp.W_router, inp.W_gate_up, inp.W_down,  # noqa: E731
+                                       inp.Ws_gate_up, inp.Ws_down, out_host)
+    for _ in range(2):
+        fwd_h()
+    torch.cuda.synchronize()
+    barrier()
+    h0, h1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    h0.record(stream)
+    for _ in range(e2e_steps):
+        fwd_h()
+    h1.record(stream)
+    torch.cuda.synchronize()
+    barrier()
+    th_ms = max_over_ranks(h0.elapsed_time(h1))
+    layer.check_device_status()
+    io_bytes = cfg.T * cfg.d_model * inp.x.element_size()
+    e2e = {"value": world * cfg.T * e2e_steps / (th_ms / 1e3), "unit": "tokens/s",
+           "h2d_bytes_per_step": io_bytes, "d2h_bytes_per_step": io_bytes,
+           "ms_per_step": th_ms / e2e_steps,
+           "path": "l4moe_forward_host: pinned host x -> device, layer, device -> pinned host out"}
+
+    if rank != 0:
+        if world > 1:
+            import torch.distributed as dist
+            dist.destroy_process_group()
+        return
+
+    # ---------------------------------------------------------------- roofline
+    peaks, peak_src = load_peaks()
+    kfb = kernel_flops_bytes(cfg, counts)
+    per_kernel = {}
+    for name, (ms, n) in ktimes.items():
+        if n:
+            avg = ms / n
+            per_kernel[name] = {"avg_us": avg * 1e3, "share": None, "launches": n,
+                                "tflops": kfb[name]["flops"] / (avg / 1e3) / 1e12,
+                                "gbs": kfb[name]["bytes"] / (avg / 1e3) / 1e9}
+    tot = sum(v["avg_us"] for v in per_kernel.values())
+    for v in per_kernel.values():
+        v["share"] = v["avg_us"] / tot if tot else None
+    dom = max(per_kernel, key=lambda k: per_kernel[k]["avg_us"])
+    long_region = t_ms > 1000.0
+    tensor_peak = peaks.get("bf16_tflops_sustained" if long_region else "bf16_tflops")
+    hbm = peaks["hbm_gbs"]
+    f, b = kfb[dom]["flops"], kfb[dom]["bytes"]
+    t_tensor = f / (tensor_peak * 1e12) if f else 0.0
+    t_hbm = b / (hbm * 1e9)
+    bound = "tensor" if t_tensor >= t_hbm else "hbm"
+    avg_s = per_kernel[dom]["avg_us"] / 1e6
+    if bound == "tensor":
+        achieved, peak, unit = f / avg_s / 1e12, tensor_peak, "TFLOP/s"
+    else:
+        achieved, peak, unit = b / avg_s / 1e9, hbm, "GB/s"
+    traffic = profile_traffic(dom, cfg.name)
+    roofline = {"kernel": dom, "bound": bound, "achieved": achieved, "peak": peak, "unit": unit,
+                "frac": achieved / peak, "traffic": traffic,
+                "peak_source": f"{peak_src} ({'sustained' if (bound == 'tensor' and long_region) else 'burst'})"
+                if bound == "tensor" else f"{peak_src} hbm_gbs",
+                "algorithmic_per_launch": {"flops": f, "bytes": b}}
+    # whole layer against its own roof
+    flops = accounting.layer_flops(cfg.T, cfg.d_model, cfg.num_experts, cfg.expert_ffn, cfg.shared_ffn)
+    lbytes = accounting.layer_bytes(cfg.T, cfg.d_model, cfg.num_experts, cfg.expert_ffn, cfg.shared_ffn,
+                                    cfg.dtype, accounting.experts_touched(counts))
+    t_roof = max(flops / (tensor_peak * 1e12), lbytes / (hbm * 1e9))
+    layer_roof = {"bound": "tensor" if flops / (tensor_peak * 1e12) >= lbytes / (hbm * 1e9) else "hbm",
+                  "frac": t_roof / (ms_step / 1e3), "tflops_active": flops / (ms_step / 1e3) / 1e12,
+                  "gbs_algorithmic": lbytes / (ms_step / 1e3) / 1e9,
+                  "flops_per_step": flops, "bytes_per_step": lbytes}
+
+    line = {"metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "bf16" if cfg.dtype != "f32" else "f32",
+            "data": "synthetic (seeded N(0,1) inputs, N(0,0.02) weights, random-init)",
+            "config": config_dict(cfg, world), "roofline": roofline, "layer_roofline": layer_roof,
+            "kernels": per_kernel, "e2e": e2e, "gpu_launches": launches, "clocks": clocks,
+            "experts_touched": accounting.experts_touched(counts)}
+    if cfg.dtype == "fp8":
+        line["dtype"] = "bf16 (E4M3 weights widened exactly to bf16)"
+    if world == 1 and not args.no_cpu_baseline:
+        line["cpu_baseline"] = cpu_baseline(inp)
+    print(json.dumps(line), flush=True)
+
+
+if __name__ == "__main__":
+    main()

@@ -19,7 +19,9 @@ DTYPES = {"f32": 0, "bf16": 1, "fp8": 2}
 EXPORTED = ("l4moe_create", "l4moe_destroy", "l4moe_workspace_size", "l4moe_set_workspace",
             "l4moe_set_router_bias", "l4moe_set_fp8_scales", "l4moe_forward",
             "l4moe_forward_host", "l4moe_get_routing", "l4moe_check_device_status",
-            "l4moe_launch_count", "l4moe_last_error", "l4moe_status_string", "l4moe_version")
+            "l4moe_launch_count", "l4moe_last_error", "l4moe_status_string", "l4moe_version",
+            "l4moe_set_timing", "l4moe_read_timing", "l4moe_kernel_name")
+NUM_KERNELS = 5
 
 _lib = None
 
@@ -67,9 +69,15 @@ def load_library():
     lib.l4moe_status_string.argtypes = [i32]
     lib.l4moe_status_string.restype = ctypes.c_char_p
     lib.l4moe_version.argtypes = []
+    lib.l4moe_set_timing.argtypes = [vp, i32]
+    lib.l4moe_read_timing.argtypes = [vp, ctypes.POINTER(ctypes.c_double),
+                                      ctypes.POINTER(ctypes.c_uint64)]
+    lib.l4moe_kernel_name.argtypes = [i32]
+    lib.l4moe_kernel_name.restype = ctypes.c_char_p
     for name in ("l4moe_create", "l4moe_set_workspace", "l4moe_set_router_bias",
                  "l4moe_set_fp8_scales", "l4moe_forward", "l4moe_forward_host",
-                 "l4moe_get_routing", "l4moe_check_device_status", "l4moe_version"):
+                 "l4moe_get_routing", "l4moe_check_device_status", "l4moe_version",
+                 "l4moe_set_timing", "l4moe_read_timing"):
         getattr(lib, name).restype = ctypes.c_int
     _lib = lib
     return lib
@@ -201,6 +209,17 @@ class L4MoE:
 
     def check_device_status(self, stream=None):
         self._check(self._lib.l4moe_check_device_status(self._h, _stream_handle(stream)))
+
+    def set_timing(self, enable: bool):
+        self._check(self._lib.l4moe_set_timing(self._h, 1 if enable else 0))
+
+    def read_timing(self) -> dict:
+        """{kernel name: (total ms, launches)} recorded since the last read."""
+        ms = (ctypes.c_double * NUM_KERNELS)()
+        n = (ctypes.c_uint64 * NUM_KERNELS)()
+        self._check(self._lib.l4moe_read_timing(self._h, ms, n))
+        return {self._lib.l4moe_kernel_name(i).decode(): (ms[i], int(n[i]))
+                for i in range(NUM_KERNELS)}
 
     @property
     def launch_count(self) -> int:

@@ -123,6 +123,10 @@ struct l4moe_handle {
     uint64_t launches = 0;
     std::string err;
     int last_T = 0;
+    // per-kernel event timing (l4moe_set_timing)
+    bool timing = false;
+    std::vector<cudaEvent_t> ev_pool;             // recycled events
+    std::vector<std::pair<int, std::pair<cudaEvent_t, cudaEvent_t>>> ev_pending;
 };
 
 namespace {
@@ -138,6 +142,34 @@ l4moe_status fail(l4moe_handle* h, l4moe_status s, const std::string& msg) {
 l4moe_status cuda_fail(l4moe_handle* h, cudaError_t e, const char* what) {
     return fail(h, L4MOE_ERR_CUDA, std::string(what) + ": " + cudaGetErrorString(e));
 }
+
+cudaEvent_t take_event(l4moe_handle* h) {
+    if (!h->ev_pool.empty()) {
+        cudaEvent_t e = h->ev_pool.back();
+        h->ev_pool.pop_back();
+        return e;
+    }
+    cudaEvent_t e = nullptr;
+    if (cudaEventCreate(&e) != cudaSuccess) return nullptr;
+    return e;
+}
+
+// Event pair around one launch when timing is enabled.
+struct LaunchTimer {
+    l4moe_handle* h;
+    int slot;
+    cudaStream_t st;
+    cudaEvent_t a = nullptr, b = nullptr;
+    LaunchTimer(l4moe_handle* h_, int slot_, cudaStream_t st_) : h(h_), slot(slot_), st(st_) {
+        if (h->timing && (a = take_event(h)) != nullptr) cudaEventRecord(a, st);
+    }
+    void stop() {
+        if (a && (b = take_event(h)) != nullptr) {
+            cudaEventRecord(b, st);
+            h->ev_pending.push_back({slot, {a, b}});
+        }
+    }
+};
 
 l4moe_status ensure_workspace(l4moe_handle* h, int T) {
     if (h->ws && T <= h->ws_tokens) return L4MOE_OK;
@@ -286,20 +318,26 @@ l4moe_status run_layer(l4moe_handle* h, int T, const void* x, const void* Wr,
         if ((e = cudaGetLastError()) != cudaSuccess) return cuda_fail(h, e, what); \
     } while (0)
 
+    LaunchTimer t_router(h, 0, st);
     launch_router<ET>(x, Wr, h->bias, T, d, E, idx, gate, lmax, margin, st);
+    t_router.stop();
     L4MOE_CHECK_LAUNCH("router launch");
 
     const int fb_gu_r = (F + kFeatTile - 1) / kFeatTile;
     const int fb_gu_s = (Fs + kFeatTile - 1) / kFeatTile;
     const int fb_dn = (d + kFeatTile - 1) / kFeatTile;
     const size_t psmem = sizeof(int) * (34 * (size_t)E + 1);
+    LaunchTimer t_perm(h, 1, st);
     permute_kernel<<<1, 1024, psmem, st>>>(idx, T, E, fb_gu_r, fb_gu_s, fb_dn, counts, offsets,
                                            perm, inv, tab_gu, tab_dn, err);
+    t_perm.stop();
     L4MOE_CHECK_LAUNCH("permute launch");
 
     const int sc_blocks = std::min((T + 7) / 8, h->sms * 8);
+    LaunchTimer t_rows(h, 2, st);
     permute_rows_kernel<ET><<<sc_blocks, 256, 0, st>>>(static_cast<const ET*>(x), gate, inv, T, d,
                                                         xg, gslot);
+    t_rows.stop();
     L4MOE_CHECK_LAUNCH("row permutation launch");
 
     const int tb = (T + kTokTile - 1) / kTokTile;
@@ -324,9 +362,11 @@ l4moe_status run_layer(l4moe_handle* h, int T, const void* x, const void* Wr,
     gu.rowmap_shared = inv;
     gu.colscale_routed = gslot;  // sigmoid gate of each routed slot
     gu.err = err;
+    LaunchTimer t_gu(h, 3, st);
     launch_gemm<MODE_GATEUP, ET>(
         grid_for((long long)fb_gu_s * tb + (long long)fb_gu_r * (tb + std::min(E, T))), m_xg, m_x,
         gu, st);
+    t_gu.stop();
     L4MOE_CHECK_LAUNCH("gate/up launch");
 
     GemmArgs dn{};
@@ -346,7 +386,9 @@ l4moe_status run_layer(l4moe_handle* h, int T, const void* x, const void* Wr,
     dn.rowmap_shared = nullptr;
     dn.colscale_routed = nullptr;
     dn.err = err;
+    LaunchTimer t_dn(h, 4, st);
     launch_gemm<MODE_DOWN, ET>(grid_for((long long)fb_dn * (tb + std::min(E, T))), m_hr, m_hs, dn, st);
+    t_dn.stop();
     L4MOE_CHECK_LAUNCH("down launch");
 #undef L4MOE_CHECK_LAUNCH
     h->last_T = T;
@@ -437,6 +479,11 @@ l4moe_status l4moe_create(const l4moe_params* params, l4moe_handle** out) {
 
 void l4moe_destroy(l4moe_handle* h) {
     if (!h) return;
+    for (cudaEvent_t e : h->ev_pool) cudaEventDestroy(e);
+    for (auto& p : h->ev_pending) {
+        cudaEventDestroy(p.second.first);
+        cudaEventDestroy(p.second.second);
+    }
     if (h->ws_owned && h->ws) cudaFree(h->ws);
     if (h->d_maps) cudaFree(h->d_maps);
     delete h;
@@ -548,6 +595,36 @@ l4moe_status l4moe_check_device_status(l4moe_handle* h, void* stream) {
     char msg[160];
     snprintf(msg, sizeof msg, "device error word 0x%x (1: producer wait, 2: MMA wait, 4: epilogue wait, 8: bad expert index)", word);
     return fail(h, (word & 7u) ? L4MOE_ERR_TIMEOUT : L4MOE_ERR_ARG, msg);
+}
+
+l4moe_status l4moe_set_timing(l4moe_handle* h, int enable) {
+    if (!h) return L4MOE_ERR_ARG;
+    h->timing = enable != 0;
+    return L4MOE_OK;
+}
+
+l4moe_status l4moe_read_timing(l4moe_handle* h, double* ms, uint64_t* launches) {
+    if (!h || !ms || !launches) return L4MOE_ERR_ARG;
+    if (h->ev_pending.empty()) return L4MOE_OK;
+    cudaError_t e = cudaEventSynchronize(h->ev_pending.back().second.second);
+    if (e != cudaSuccess) return cuda_fail(h, e, "timing event synchronize");
+    for (auto& p : h->ev_pending) {
+        float t = 0.f;
+        e = cudaEventElapsedTime(&t, p.second.first, p.second.second);
+        if (e != cudaSuccess) return cuda_fail(h, e, "timing elapsed time");
+        ms[p.first] += t;
+        launches[p.first] += 1;
+        h->ev_pool.push_back(p.second.first);
+        h->ev_pool.push_back(p.second.second);
+    }
+    h->ev_pending.clear();
+    return L4MOE_OK;
+}
+
+const char* l4moe_kernel_name(int slot) {
+    static const char* names[L4MOE_NUM_KERNELS] = {"router", "permute", "row_copy", "gemm_gate_up",
+                                                   "gemm_down"};
+    return (slot >= 0 && slot < L4MOE_NUM_KERNELS) ? names[slot] : "";
 }
 
 uint64_t l4moe_launch_count(const l4moe_handle* h) { return h ? h->launches : 0; }
