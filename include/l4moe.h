@@ -143,6 +143,37 @@ L4MOE_API l4moe_status l4moe_forward_host(l4moe_handle *h, int T, const void *x_
                                 const void *Ws_gate_up, const void *Ws_down, void *out_host,
                                 void *stream);
 
+/* Allocation-free forward (no counterpart in the pages; an interface for
+ * callers that cannot allocate device memory).  Some callers may not call
+ * cudaMalloc at all: code running while a CUDA graph is being captured,
+ * inside another framework's allocator or memory-pool callbacks, or under a
+ * hard memory budget where every byte is pre-reserved.  l4moe_forward
+ * allocates its workspace (and a descriptor table) on first use; this entry
+ * point instead uses one fixed scratch area compiled into the library, a
+ * file-scope device array of L4MOE_STATIC_WORKSPACE_BYTES bytes that every
+ * GPU loading the library holds until the process exits.  It calls no
+ * cudaMalloc, cudaFree or other allocating routine.
+ *
+ * Arguments and results are those of l4moe_forward (the caller still owns
+ * x, the weights and out).  The first call on each device resolves the
+ * scratch array's device address (cudaGetSymbolAddress, with that device
+ * current) and caches it; make that first call before any stream capture.
+ * Fails with L4MOE_ERR_WORKSPACE, launching nothing, when T tokens of this
+ * layer do not fit in the scratch area: it holds the workspace of
+ * l4moe_workspace_size(h, T) bytes (rounded up to 256) plus 2(E+1) TMA
+ * descriptors of 128 bytes, e.g. about 500 tokens at d_model 5120 and
+ * F = Fs = 8192.  Every call, from any handle, shares the one array: calls
+ * whose work overlaps on the GPU (other streams, other threads) race and
+ * corrupt each other; serialise them.  The array keeps the last call's
+ * contents; the call clears the device error word itself.  Per-kernel
+ * timing is not recorded for these calls, and l4moe_get_routing /
+ * l4moe_check_device_status keep referring to the handle's own workspace. */
+#define L4MOE_STATIC_WORKSPACE_BYTES (32u << 20)
+L4MOE_API l4moe_status l4moe_forward_static(l4moe_handle *h, int T, const void *x, const void *W_router,
+                                  const void *const *W_gate_up, const void *const *W_down,
+                                  const void *Ws_gate_up, const void *Ws_down, void *out,
+                                  void *stream);
+
 /* Device pointers (inside the workspace) to the routing of the last forward
  * enqueued with this handle; valid once that work has run and until the next
  * forward.  Any output pointer may be NULL.

@@ -20,7 +20,9 @@ EXPORTED = ("l4moe_create", "l4moe_destroy", "l4moe_workspace_size", "l4moe_set_
             "l4moe_set_router_bias", "l4moe_set_fp8_scales", "l4moe_forward",
             "l4moe_forward_host", "l4moe_get_routing", "l4moe_check_device_status",
             "l4moe_launch_count", "l4moe_last_error", "l4moe_status_string", "l4moe_version",
-            "l4moe_set_timing", "l4moe_read_timing", "l4moe_kernel_name")
+            "l4moe_set_timing", "l4moe_read_timing", "l4moe_kernel_name",
+            "l4moe_forward_static")
+STATIC_WORKSPACE_BYTES = 32 << 20
 NUM_KERNELS = 5
 
 _lib = None
@@ -60,6 +62,7 @@ def load_library():
     fwd = [vp, i32, vp, vp, pvp, pvp, vp, vp, vp, vp]
     lib.l4moe_forward.argtypes = fwd
     lib.l4moe_forward_host.argtypes = fwd
+    lib.l4moe_forward_static.argtypes = fwd
     lib.l4moe_get_routing.argtypes = [vp] + [pvp] * 7
     lib.l4moe_check_device_status.argtypes = [vp, vp]
     lib.l4moe_launch_count.argtypes = [vp]
@@ -77,7 +80,7 @@ def load_library():
     for name in ("l4moe_create", "l4moe_set_workspace", "l4moe_set_router_bias",
                  "l4moe_set_fp8_scales", "l4moe_forward", "l4moe_forward_host",
                  "l4moe_get_routing", "l4moe_check_device_status", "l4moe_version",
-                 "l4moe_set_timing", "l4moe_read_timing"):
+                 "l4moe_set_timing", "l4moe_read_timing", "l4moe_forward_static"):
         getattr(lib, name).restype = ctypes.c_int
     _lib = lib
     return lib
@@ -181,6 +184,17 @@ class L4MoE:
                                             _ptr(Ws_gate_up), _ptr(Ws_down), _ptr(out),
                                             _stream_handle(stream)))
         self.last_T = T
+        return out
+
+    def forward_static(self, x, W_router, W_gate_up, W_down, Ws_gate_up, Ws_down, out, stream=None):
+        """l4moe_forward_static: the same layer with the library's fixed device
+        scratch array instead of an allocated workspace (no device allocation
+        in the call; `out` must be supplied)."""
+        T = x.shape[0]
+        gu, dn = self._weights(W_gate_up, W_down)
+        self._check(self._lib.l4moe_forward_static(self._h, T, _ptr(x), _ptr(W_router), gu, dn,
+                                                   _ptr(Ws_gate_up), _ptr(Ws_down), _ptr(out),
+                                                   _stream_handle(stream)))
         return out
 
     def forward_host(self, x_host, W_router, W_gate_up, W_down, Ws_gate_up, Ws_down, out_host,

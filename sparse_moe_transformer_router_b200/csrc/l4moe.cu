@@ -119,6 +119,9 @@ struct l4moe_handle {
     const void* key_sgu = nullptr;
     const void* key_sdn = nullptr;
     std::vector<CUtensorMap> h_maps;  // [2][E+1]: gate/up set then down set
+    std::vector<const void*> hkey_gu, hkey_dn;  // weights h_maps was encoded for
+    const void* hkey_sgu = nullptr;
+    const void* hkey_sdn = nullptr;
     CUtensorMap* d_maps = nullptr;
     uint64_t launches = 0;
     std::string err;
@@ -193,12 +196,13 @@ l4moe_status ensure_workspace(l4moe_handle* h, int T) {
     return L4MOE_OK;
 }
 
-// (Re)build the weight descriptors when any weight pointer changed.
-l4moe_status ensure_weight_maps(l4moe_handle* h, const void* const* Wgu, const void* const* Wdn,
-                                const void* Wsgu, const void* Wsdn, cudaStream_t st) {
+// Encode the weight descriptors on the host (h->h_maps) unless they already
+// describe these pointers.
+l4moe_status encode_weight_maps(l4moe_handle* h, const void* const* Wgu, const void* const* Wdn,
+                                const void* Wsgu, const void* Wsdn) {
     const int E = h->p.num_experts;
-    bool same = h->d_maps && h->key_sgu == Wsgu && h->key_sdn == Wsdn;
-    for (int e = 0; same && e < E; ++e) same = h->key_gu[e] == Wgu[e] && h->key_dn[e] == Wdn[e];
+    bool same = !h->h_maps.empty() && h->hkey_sgu == Wsgu && h->hkey_sdn == Wsdn;
+    for (int e = 0; same && e < E; ++e) same = h->hkey_gu[e] == Wgu[e] && h->hkey_dn[e] == Wdn[e];
     if (same) return L4MOE_OK;
     const int d = h->p.d_model, F = h->p.expert_ffn, Fs = h->p.shared_ffn;
     const size_t wb = w_bytes(h->p.dtype);
@@ -211,6 +215,7 @@ l4moe_status ensure_weight_maps(l4moe_handle* h, const void* const* Wgu, const v
     const CUtensorMapSwizzle swz = h->p.dtype == L4MOE_F32 ? CU_TENSOR_MAP_SWIZZLE_128B_ATOM_32B
                                                            : CU_TENSOR_MAP_SWIZZLE_128B;
     h->h_maps.assign(2 * (E + 1), CUtensorMap{});
+    h->hkey_gu.clear();
     for (int e = 0; e <= E; ++e) {
         const bool sh = (e == E);
         const void* gu = sh ? Wsgu : Wgu[e];
@@ -218,9 +223,27 @@ l4moe_status ensure_weight_maps(l4moe_handle* h, const void* const* Wgu, const v
         const int f = sh ? Fs : F;
         if (!encode_2d(&h->h_maps[e], dt, gu, 2ull * f, (uint64_t)d, 2ull * f * wb, bw, bk, swz) ||
             !encode_2d(&h->h_maps[E + 1 + e], dt, dn, (uint64_t)d, (uint64_t)f, (uint64_t)d * wb, bw,
-                       bk, swz))
+                       bk, swz)) {
+            h->h_maps.clear();
             return fail(h, L4MOE_ERR_CUDA, "cuTensorMapEncodeTiled failed for a weight");
+        }
     }
+    h->hkey_gu.assign(Wgu, Wgu + E);
+    h->hkey_dn.assign(Wdn, Wdn + E);
+    h->hkey_sgu = Wsgu;
+    h->hkey_sdn = Wsdn;
+    return L4MOE_OK;
+}
+
+// (Re)build and upload the weight descriptors when any weight pointer changed.
+l4moe_status ensure_weight_maps(l4moe_handle* h, const void* const* Wgu, const void* const* Wdn,
+                                const void* Wsgu, const void* Wsdn, cudaStream_t st) {
+    const int E = h->p.num_experts;
+    bool same = h->d_maps && h->key_sgu == Wsgu && h->key_sdn == Wsdn;
+    for (int e = 0; same && e < E; ++e) same = h->key_gu[e] == Wgu[e] && h->key_dn[e] == Wdn[e];
+    if (same) return L4MOE_OK;
+    l4moe_status s = encode_weight_maps(h, Wgu, Wdn, Wsgu, Wsdn);
+    if (s != L4MOE_OK) return s;
     if (!h->d_maps) {
         cudaError_t e = cudaMalloc(&h->d_maps, sizeof(CUtensorMap) * 2 * (E + 1));
         if (e != cudaSuccess) return cuda_fail(h, e, "descriptor cudaMalloc");
@@ -276,14 +299,16 @@ void launch_gemm(int grid, const CUtensorMap& b_routed, const CUtensorMap& b_sha
     moe_gemm_kernel<MODE, ET><<<grid, 192, Cfg::SMEM_BYTES, st>>>(b_routed, b_shared, a);
 }
 
+// The launch sequence of one forward.  w / ws_tokens: the workspace and the
+// token count its layout was made for; maps: device array of the 2(E+1)
+// weight descriptors.
 template <typename ET>
-l4moe_status run_layer(l4moe_handle* h, int T, const void* x, const void* Wr,
-                       const void* const* Wgu, const void* const* Wdn, const void* Wsgu,
-                       const void* Wsdn, void* out, cudaStream_t st) {
+l4moe_status run_layer(l4moe_handle* h, int T, const void* x, const void* Wr, const void* Wsgu,
+                       const void* Wsdn, void* out, cudaStream_t st, uint8_t* w, int ws_tokens,
+                       const CUtensorMap* maps) {
     const l4moe_params& p = h->p;
     const int d = p.d_model, F = p.expert_ffn, Fs = p.shared_ffn, E = p.num_experts;
-    const WsLayout L = ws_layout(p, h->ws_tokens);
-    uint8_t* w = h->ws;
+    const WsLayout L = ws_layout(p, ws_tokens);
     unsigned* err = reinterpret_cast<unsigned*>(w + L.err);
     int32_t* idx = reinterpret_cast<int32_t*>(w + L.idx);
     float* gate = reinterpret_cast<float*>(w + L.gate);
@@ -345,7 +370,7 @@ l4moe_status run_layer(l4moe_handle* h, int T, const void* x, const void* Wr,
 
     GemmArgs gu{};
     gu.table = tab_gu;
-    gu.a_maps = h->d_maps;
+    gu.a_maps = maps;
     gu.num_experts = E;
     gu.k_routed = d;
     gu.k_shared = d;
@@ -371,7 +396,7 @@ l4moe_status run_layer(l4moe_handle* h, int T, const void* x, const void* Wr,
 
     GemmArgs dn{};
     dn.table = tab_dn;
-    dn.a_maps = h->d_maps + (E + 1);
+    dn.a_maps = maps + (E + 1);
     dn.num_experts = E;
     dn.k_routed = F;
     dn.k_shared = 0;
@@ -422,15 +447,84 @@ l4moe_status forward_impl(l4moe_handle* h, int T, const void* x, const void* Wr,
     if ((s = ensure_workspace(h, T)) != L4MOE_OK) return s;
     if ((s = ensure_weight_maps(h, Wgu, Wdn, Wsgu, Wsdn, st)) != L4MOE_OK) return s;
     switch (h->p.dtype) {
-    case L4MOE_F32: return run_layer<float>(h, T, x, Wr, Wgu, Wdn, Wsgu, Wsdn, out, st);
-    case L4MOE_BF16: return run_layer<__nv_bfloat16>(h, T, x, Wr, Wgu, Wdn, Wsgu, Wsdn, out, st);
+    case L4MOE_F32:
+        return run_layer<float>(h, T, x, Wr, Wsgu, Wsdn, out, st, h->ws, h->ws_tokens, h->d_maps);
+    case L4MOE_BF16:
+        return run_layer<__nv_bfloat16>(h, T, x, Wr, Wsgu, Wsdn, out, st, h->ws, h->ws_tokens,
+                                        h->d_maps);
     default: return fail(h, L4MOE_ERR_UNSUPPORTED, "FP8 weight path not built in this library");
     }
+}
+
+// ------------------------------------------------------------------------
+// Allocation-free forward: workspace and weight descriptors in a fixed
+// device array of this file, never in cudaMalloc'd memory.
+static __device__ __align__(256) uint8_t g_static_ws[L4MOE_STATIC_WORKSPACE_BYTES];
+
+constexpr int kMaxDevices = 64;
+std::mutex g_static_mu;
+uint8_t* g_static_addr[kMaxDevices] = {};
+
+// Device address of g_static_ws on the current device, resolved once per
+// device (the host-side symbol is only a stand-in, not a device address).
+l4moe_status static_workspace(l4moe_handle* h, uint8_t** out) {
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return cuda_fail(h, e, "cudaGetDevice");
+    if (dev < 0 || dev >= kMaxDevices) return fail(h, L4MOE_ERR_UNSUPPORTED, "device index out of range");
+    std::lock_guard<std::mutex> lock(g_static_mu);
+    if (!g_static_addr[dev]) {
+        void* ptr = nullptr;
+        e = cudaGetSymbolAddress(&ptr, g_static_ws);
+        if (e != cudaSuccess || !ptr) return cuda_fail(h, e, "cudaGetSymbolAddress(static workspace)");
+        g_static_addr[dev] = static_cast<uint8_t*>(ptr);
+    }
+    *out = g_static_addr[dev];
+    return L4MOE_OK;
 }
 
 }  // namespace
 
 extern "C" {
+
+l4moe_status l4moe_forward_static(l4moe_handle* h, int T, const void* x, const void* W_router,
+                                  const void* const* W_gate_up, const void* const* W_down,
+                                  const void* Ws_gate_up, const void* Ws_down, void* out,
+                                  void* stream) {
+    l4moe_status s = check_forward_args(h, T, x, W_router, W_gate_up, W_down, Ws_gate_up, Ws_down, out);
+    if (s != L4MOE_OK || T == 0) return s;
+    if (h->p.dtype != L4MOE_F32 && h->p.dtype != L4MOE_BF16)
+        return fail(h, L4MOE_ERR_UNSUPPORTED, "FP8 weight path not built in this library");
+    const int E = h->p.num_experts;
+    const size_t ws_bytes = (ws_layout(h->p, T).total + 255) & ~size_t(255);
+    const size_t maps_bytes = sizeof(CUtensorMap) * 2 * (E + 1);
+    if (ws_bytes + maps_bytes > L4MOE_STATIC_WORKSPACE_BYTES) {
+        char msg[200];
+        snprintf(msg, sizeof msg,
+                 "T = %d needs %zu bytes of static workspace; the library's static array holds %u",
+                 T, ws_bytes + maps_bytes, (unsigned)L4MOE_STATIC_WORKSPACE_BYTES);
+        return fail(h, L4MOE_ERR_WORKSPACE, msg);
+    }
+    uint8_t* base = nullptr;
+    if ((s = static_workspace(h, &base)) != L4MOE_OK) return s;
+    if ((s = encode_weight_maps(h, W_gate_up, W_down, Ws_gate_up, Ws_down)) != L4MOE_OK) return s;
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    CUtensorMap* maps = reinterpret_cast<CUtensorMap*>(base + ws_bytes);
+    // every call shares the array: upload this call's descriptors and clear
+    // the error word (the only state a forward expects to start at zero)
+    cudaError_t e = cudaMemcpyAsync(maps, h->h_maps.data(), maps_bytes, cudaMemcpyHostToDevice, st);
+    if (e != cudaSuccess) return cuda_fail(h, e, "static descriptor upload");
+    e = cudaMemsetAsync(base + ws_layout(h->p, T).err, 0, sizeof(unsigned), st);
+    if (e != cudaSuccess) return cuda_fail(h, e, "static error word clear");
+    const bool timing = h->timing;  // event timing would create events: off here
+    h->timing = false;
+    if (h->p.dtype == L4MOE_F32)
+        s = run_layer<float>(h, T, x, W_router, Ws_gate_up, Ws_down, out, st, base, T, maps);
+    else
+        s = run_layer<__nv_bfloat16>(h, T, x, W_router, Ws_gate_up, Ws_down, out, st, base, T, maps);
+    h->timing = timing;
+    return s;
+}
 
 int l4moe_version(void) { return 100; }
 

@@ -1,0 +1,55 @@
+"""The allocation-free entry point, l4moe_forward_static.
+
+It exists for callers that may not allocate device memory while they run the
+layer (work recorded under CUDA-graph stream capture, code inside another
+framework's allocator callbacks, or a process whose device memory is fully
+reserved up front).  It runs the same kernels as l4moe_forward but keeps its
+workspace in the library's fixed device array.  This file runs last so that a
+run stopping at the first failure has already run every other test.
+"""
+import numpy as np
+import pytest
+import torch
+
+from parity_util import OUT_UNIT_ROUNDOFF, TOL, make_layer
+from sparse_moe_transformer_router_b200.binding import ERR_WORKSPACE, L4MoEError
+from sparse_moe_transformer_router_b200.workloads import LayerConfig, generate
+
+pytestmark = pytest.mark.gpu
+
+
+def _assert_close(out: torch.Tensor, ref: torch.Tensor, dtype: str):
+    o = out.double().cpu().numpy()
+    r = ref.double().cpu().numpy()
+    assert np.all(np.isfinite(o))
+    rms = float(np.sqrt(np.mean(r ** 2)))
+    bound = TOL[dtype] * rms + OUT_UNIT_ROUNDOFF[dtype] * np.abs(r)
+    assert np.all(np.abs(o - r) <= bound)
+
+
+@pytest.mark.parametrize("dtype", ["bf16", "f32"])
+def test_static_forward_matches_allocating_forward_on_two_calls(dtype):
+    cfg = LayerConfig(f"noalloc_{dtype}", 300, 256, 8, 384, 256, dtype, wr_std=0.1)
+    inp = generate(cfg, seed=11, device="cuda")
+    layer = make_layer(inp)
+    args = (inp.x, inp.W_router, inp.W_gate_up, inp.W_down, inp.Ws_gate_up, inp.Ws_down)
+    ref = layer.forward(*args)
+    torch.cuda.synchronize()
+    for _ in range(2):  # the shared scratch array keeps the previous call's contents
+        out = torch.full_like(ref, float("nan"))
+        layer.forward_static(*args, out)
+        torch.cuda.synchronize()
+        _assert_close(out, ref, dtype)
+
+
+def test_static_forward_rejects_batches_beyond_its_array():
+    cfg = LayerConfig("noalloc_big", 64, 256, 8, 384, 256, "bf16", wr_std=0.1)
+    inp = generate(cfg, seed=12, device="cuda")
+    layer = make_layer(inp)
+    x_big = torch.zeros((20000, cfg.d_model), dtype=torch.bfloat16, device="cuda")
+    out = torch.empty_like(x_big)
+    with pytest.raises(L4MoEError) as ei:
+        layer.forward_static(x_big, inp.W_router, inp.W_gate_up, inp.W_down, inp.Ws_gate_up,
+                             inp.Ws_down, out)
+    assert ei.value.status == ERR_WORKSPACE
+    assert "static" in str(ei.value)
