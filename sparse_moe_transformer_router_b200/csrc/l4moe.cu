@@ -344,13 +344,26 @@ l4moe_status run_layer(l4moe_handle* h, int T, const void* x, const void* Wr, co
     } while (0)
 
     LaunchTimer t_router(h, 0, st);
-    launch_router<ET>(x, Wr, h->bias, T, d, E, idx, gate, lmax, margin, st);
+    if (sizeof(ET) == 2 && E % 8 == 0) {
+        // tensor-core router: W_router [d, E] as the MN-major operand
+        CUtensorMap m_wr;
+        if (!encode_2d(&m_wr, adt, Wr, (uint64_t)E, (uint64_t)d, (uint64_t)E * sizeof(ET), 64, 64))
+            return fail(h, L4MOE_ERR_CUDA, "cuTensorMapEncodeTiled failed for the router weight");
+        static std::once_flag once;
+        std::call_once(once, [] { set_smem_attr(router_mma_kernel, rmma::SMEM_BYTES); });
+        router_mma_kernel<<<(T + 127) / 128, 128, rmma::SMEM_BYTES, st>>>(
+            m_x, m_wr, h->bias, T, d, E, idx, gate, lmax, margin, err);
+    } else {
+        launch_router<ET>(x, Wr, h->bias, T, d, E, idx, gate, lmax, margin, st);
+    }
     t_router.stop();
     L4MOE_CHECK_LAUNCH("router launch");
 
-    const int fb_gu_r = (F + kFeatTile - 1) / kFeatTile;
-    const int fb_gu_s = (Fs + kFeatTile - 1) / kFeatTile;
-    const int fb_dn = (d + kFeatTile - 1) / kFeatTile;
+    // feature blocks per pair tile: 128 features for gate/up, 256 for down
+    const int fpg = pair_features<MODE_GATEUP>(), fpd = pair_features<MODE_DOWN>();
+    const int fb_gu_r = (F + fpg - 1) / fpg;
+    const int fb_gu_s = (Fs + fpg - 1) / fpg;
+    const int fb_dn = (d + fpd - 1) / fpd;
     const size_t psmem = sizeof(int) * (34 * (size_t)E + 1);
     LaunchTimer t_perm(h, 1, st);
     permute_kernel<<<1, 1024, psmem, st>>>(idx, T, E, fb_gu_r, fb_gu_s, fb_dn, counts, offsets,
@@ -366,7 +379,10 @@ l4moe_status run_layer(l4moe_handle* h, int T, const void* x, const void* Wr, co
     L4MOE_CHECK_LAUNCH("row permutation launch");
 
     const int tb = (T + kTokTile - 1) / kTokTile;
-    auto grid_for = [&](long long tiles) { return (int)std::max(1LL, std::min<long long>(h->sms, tiles)); };
+    // CTA pairs: two CTAs (one cluster) per tile, at most one pair per two SMs
+    auto grid_for = [&](long long tiles) {
+        return 2 * (int)std::max(1LL, std::min<long long>(h->sms / 2, tiles));
+    };
 
     GemmArgs gu{};
     gu.table = tab_gu;

@@ -1,6 +1,6 @@
 // moe_gemm.cuh -- persistent grouped GEMM on the 5th-generation tensor cores
-// (tcgen05 + TMEM accumulators + TMA-fed shared-memory pipeline) for the
-// three contractions of the layer:
+// (tcgen05 on CTA pairs, TMEM accumulators, TMA-fed shared-memory pipeline)
+// for the two contractions of the layer:
 //
 //   gate/up  : a = g * (x . W_gate_up)  then h = silu(a[:F]) * a[F:]
 //              (SwiGLU), for the shared expert (g = 1) and every routed
@@ -17,21 +17,33 @@
 // sketch: the layer output is the shared expert's output plus the routed
 // expert's.
 //
-// Orientation ("swap-AB"): the weight is the MMA A operand (M = 128 output
-// features, read MN-major straight from the row-major [K, N] weight) and the
-// activations are the B operand (N = up to 256 tokens, K-major rows).  A
+// Orientation ("swap-AB"): the weight is the MMA A operand (output features
+// as M, read MN-major straight from the row-major [K, N] weight) and the
+// activations are the B operand (tokens as N, up to 256, K-major rows).  A
 // group's token count is only padded to a multiple of 16, so ragged experts
-// (and decode, T <= 128) waste little tensor work.  For gate/up a tile holds
-// the gate block and the matching up block of 128 features each, as two TMEM
-// accumulators, so the SwiGLU is computed in the epilogue from registers.
+// (and decode, T <= 128) waste little tensor work.
 //
-// Roles (192 threads): warp 0 lane 0 issues TMA loads into a STAGES-deep ring
-// of shared-memory stages; warp 1 owns TMEM (alloc/dealloc) and lane 0
-// issues the MMAs and commits; warps 2..5 are the epilogue (warp w reads TMEM
-// lanes 32*(w%4) .. +31).  Every mbarrier wait is bounded; on a timeout a
-// role records a bit in the error word and returns, the producer drains its
-// in-flight copies, the MMA thread waits for its issued MMAs, and TMEM is
-// freed before exit.
+// CTA pairs (cluster of 2, cta_group::2): one MMA computes M = 256 rows x N
+// tokens; each CTA loads its own 128 A rows and its own half of the N tokens
+// into its shared memory and holds its 128 rows x N columns of the fp32
+// accumulator in its TMEM.  Per SM that halves the token operand each tile
+// streams through L2 compared with a single-CTA 128-row tile.
+//   down   : pair tile = 256 output features (128 per CTA).
+//   gate/up: pair tile = 128 features; each CTA's 128 A rows are the gate
+//            rows (64 features) followed by the up rows of the same 64
+//            features, so TMEM lane r holds gate and lane r + 64 holds up;
+//            the epilogue pairs them through a small shared-memory exchange.
+// Accumulators are double-buffered (2 x 256 TMEM columns) so the epilogue of
+// one tile overlaps the MMAs of the next.
+//
+// Roles (192 threads per CTA): warp 0 lane 0 issues TMA loads into a
+// STAGES-deep ring (both CTAs; completion counted on the leader's barrier);
+// warp 1 allocates TMEM (both CTAs) and, in the leader CTA only, lane 0
+// issues the MMAs and commits to both CTAs' barriers; warps 2..5 are the
+// epilogue (warp w reads TMEM lanes 32*(w%4) .. +31) and release the
+// accumulator to the leader.  Every mbarrier wait is bounded: on a timeout a
+// role records a bit in the error word and returns; the leader drains the
+// copies and MMAs in flight before the pair synchronises and frees TMEM.
 #pragma once
 #include <cuda_bf16.h>
 #include <cstdint>
@@ -82,25 +94,29 @@ struct GemmArgs {
     unsigned* err;
 };
 
+// Output features covered by one pair tile.
+template <int MODE>
+__host__ __device__ constexpr int pair_features() { return MODE == MODE_GATEUP ? 128 : 256; }
+
 template <int MODE, typename ET>
 struct GemmCfg {
     using C = ElemCfg<ET>;
-    static constexpr int A_OPS = (MODE == MODE_GATEUP) ? 2 : 1;
-    static constexpr int A_OP_BYTES = kFeatTile * 128;               // 128 features x 128 B of K
-    static constexpr int A_BOX_FEATS = 128 / C::BYTES;               // features per A box
-    static constexpr int A_BOXES = kFeatTile / A_BOX_FEATS;          // boxes per A operand
-    static constexpr int A_BOX_BYTES = C::BK * 128;                  // BK rows x 128 B
+    static constexpr int A_BYTES = 128 * 128;                // 128 A rows x 128 B of K
+    static constexpr int A_BOX_FEATS = 128 / C::BYTES;       // features per A box (one 128 B slab)
+    static constexpr int A_BOXES = 128 / A_BOX_FEATS;        // boxes per CTA A tile
+    static constexpr int A_BOX_BYTES = C::BK * 128;          // BK rows x 128 B
     static constexpr int B_BOX_ROWS = 64;
     static constexpr int B_BOX_BYTES = B_BOX_ROWS * 128;
-    static constexpr int B_BYTES = kTokTile * 128;
-    static constexpr int STAGE_BYTES = A_OPS * A_OP_BYTES + B_BYTES;
-    static constexpr int STAGES = (MODE == MODE_GATEUP) ? 3 : 4;
-    static constexpr int ACC_BUFS = (MODE == MODE_GATEUP) ? 1 : 2;  // 512 TMEM columns either way
+    static constexpr int B_BYTES = (kTokTile / 2) * 128;     // this CTA's half of the tokens
+    static constexpr int STAGE_BYTES = A_BYTES + B_BYTES;    // 32 KB
+    static constexpr int STAGES = 6;
+    static constexpr int ACC_BUFS = 2;
     static constexpr int TMEM_COLS = 512;
-    static constexpr int NUM_BARS = 2 * STAGES + 2 * 2 + 1;
-    static constexpr size_t SMEM_BYTES =
-        1024 /*alignment slack*/ + (size_t)STAGES * STAGE_BYTES + NUM_BARS * 8 + 16 +
-        sizeof(GroupTable);
+    static constexpr int XLD = 17;                           // exchange row stride (floats)
+    static constexpr int XCH_BYTES = (MODE == MODE_GATEUP) ? 2 * 2 * 32 * XLD * 4 : 0;
+    static constexpr int NUM_BARS = 2 * STAGES + 2 * ACC_BUFS + 1;
+    static constexpr size_t SMEM_BYTES = 1024 /*alignment slack*/ + (size_t)STAGES * STAGE_BYTES +
+                                         XCH_BYTES + NUM_BARS * 8 + 16 + sizeof(GroupTable);
 };
 
 struct TileInfo {
@@ -108,6 +124,7 @@ struct TileInfo {
     bool shared;
 };
 
+template <int MODE>
 __device__ __forceinline__ TileInfo decode_tile(const GroupTable& tab, const GemmArgs& a, int L) {
     int lo = 0, hi = tab.num_groups - 1;
     while (lo < hi) {
@@ -126,7 +143,7 @@ __device__ __forceinline__ TileInfo decode_tile(const GroupTable& tab, const Gem
     ti.row0 = tab.row0[g] + tb * kTokTile;
     ti.n_valid = min(kTokTile, rows - tb * kTokTile);
     ti.n_mma = (ti.n_valid + 15) & ~15;
-    ti.f0 = fb * kFeatTile;
+    ti.f0 = fb * pair_features<MODE>();
     ti.k_pre = ti.shared ? 0 : a.k_pre;
     ti.K = ti.k_pre + (ti.shared ? a.k_shared : a.k_routed);
     ti.M = ti.shared ? a.m_shared : a.m_routed;
@@ -134,13 +151,13 @@ __device__ __forceinline__ TileInfo decode_tile(const GroupTable& tab, const Gem
     return ti;
 }
 
-__device__ __forceinline__ float silu_f(float z) { return z / (1.0f + __expf(-z)); }
+__device__ __forceinline__ float silu_f(float z) { return __fdividef(z, 1.0f + __expf(-z)); }
 
 __device__ __forceinline__ void store_elem(float* p, float v) { *p = v; }
 __device__ __forceinline__ void store_elem(__nv_bfloat16* p, float v) { *p = __float2bfloat16_rn(v); }
 
 template <int MODE, typename ET>
-__global__ void __launch_bounds__(192, 1)
+__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(192, 1)
     moe_gemm_kernel(const __grid_constant__ CUtensorMap b_routed,
                     const __grid_constant__ CUtensorMap b_shared, const GemmArgs args) {
     using Cfg = GemmCfg<MODE, ET>;
@@ -148,75 +165,89 @@ __global__ void __launch_bounds__(192, 1)
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>(
         (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
-    uint64_t* bars = reinterpret_cast<uint64_t*>(smem + (size_t)Cfg::STAGES * Cfg::STAGE_BYTES);
-    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + Cfg::NUM_BARS);
-    GroupTable* tab = reinterpret_cast<GroupTable*>(tmem_slot + 4);
+    float* xch = reinterpret_cast<float*>(smem + (size_t)Cfg::STAGES * Cfg::STAGE_BYTES);
+    uint64_t* bars = reinterpret_cast<uint64_t*>(smem + (size_t)Cfg::STAGES * Cfg::STAGE_BYTES +
+                                                 Cfg::XCH_BYTES);
+    uint32_t* misc = reinterpret_cast<uint32_t*>(bars + Cfg::NUM_BARS);  // [0] TMEM base, [1] abort
+    GroupTable* tab = reinterpret_cast<GroupTable*>(misc + 4);
 
     const int warp = threadIdx.x >> 5;
     const int lane = threadIdx.x & 31;
+    const uint32_t rank = cluster_ctarank();  // 0: leader (issues the MMAs), 1: peer
+    const bool leader = rank == 0;
     const uint32_t stage0 = smem_u32(smem);
     const uint32_t bar0 = smem_u32(bars);
     auto full_bar = [&](int s) { return bar0 + 8u * s; };
     auto empty_bar = [&](int s) { return bar0 + 8u * (Cfg::STAGES + s); };
     auto tfull_bar = [&](int b) { return bar0 + 8u * (2 * Cfg::STAGES + b); };
-    auto tempty_bar = [&](int b) { return bar0 + 8u * (2 * Cfg::STAGES + 2 + b); };
-    const uint32_t drain_bar = bar0 + 8u * (2 * Cfg::STAGES + 4);
+    auto tempty_bar = [&](int b) { return bar0 + 8u * (2 * Cfg::STAGES + Cfg::ACC_BUFS + b); };
+    const uint32_t drain_bar = bar0 + 8u * (2 * Cfg::STAGES + 2 * Cfg::ACC_BUFS);
 
-    // work list -> shared memory
-    {
+    {   // work list -> shared memory
         const int* src = reinterpret_cast<const int*>(args.table);
         int* dst = reinterpret_cast<int*>(tab);
         for (int i = threadIdx.x; i < (int)(sizeof(GroupTable) / 4); i += blockDim.x) dst[i] = src[i];
     }
     if (threadIdx.x == 0) {
         for (int s = 0; s < Cfg::STAGES; ++s) {
-            mbar_init(full_bar(s), 1);
-            mbar_init(empty_bar(s), 1);
+            mbar_init(full_bar(s), 1);   // leader: one expect_tx arrival for both CTAs' bytes
+            mbar_init(empty_bar(s), 1);  // one multicast commit per use
         }
-        for (int b = 0; b < 2; ++b) {
+        for (int b = 0; b < Cfg::ACC_BUFS; ++b) {
             mbar_init(tfull_bar(b), 1);
-            mbar_init(tempty_bar(b), 4);
+            mbar_init(tempty_bar(b), 8);  // leader: 4 epilogue warps of each CTA
         }
         mbar_init(drain_bar, 1);
+        misc[1] = 0;
         fence_barrier_init();
     }
     if (warp == 0 && lane == 0) {
         tma_prefetch_desc(&b_routed);
         tma_prefetch_desc(&b_shared);
     }
+    cluster_sync();  // barriers of both CTAs initialised before any remote use
     if (warp == 1) {
-        tmem_alloc(smem_u32(tmem_slot), Cfg::TMEM_COLS);
-        tmem_relinquish();
+        tmem_alloc_pair(smem_u32(misc), Cfg::TMEM_COLS);
+        tmem_relinquish_pair();
     }
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
-    const uint32_t tmem_base = *tmem_slot;
+    const uint32_t tmem_base = misc[0];
     const int total = tab->total_tiles;
+    const int pair = blockIdx.x >> 1;
+    const int npairs = gridDim.x >> 1;
 
     if (warp == 0) {
         if (lane == 0) {
             // ------------------------------------------------ TMA producer
             int stage = 0;
             uint32_t phase = 0;
-            uint32_t used = 0, last_par = 0;  // per-stage: issued at least once / parity
-            for (int L = blockIdx.x; L < total; L += gridDim.x) {
-                const TileInfo ti = decode_tile(*tab, args, L);
+            uint32_t used = 0, last_par = 0;  // per stage: issued at least once / its parity
+            bool aborted = false;
+            for (int L = pair; L < total && !aborted; L += npairs) {
+                const TileInfo ti = decode_tile<MODE>(*tab, args, L);
                 const CUtensorMap* amap_main = args.a_maps + ti.expert;
                 const CUtensorMap* amap_pre = args.a_maps + args.num_experts;
                 const void* bmap_main = ti.shared ? (const void*)&b_shared : (const void*)&b_routed;
                 const int nkb = ti.K / C::BK;
                 const int nkb_pre = ti.k_pre / C::BK;
-                const int nbb = (ti.n_mma + Cfg::B_BOX_ROWS - 1) / Cfg::B_BOX_ROWS;
-                const uint32_t tx =
-                    Cfg::A_OPS * Cfg::A_OP_BYTES + (uint32_t)nbb * Cfg::B_BOX_BYTES;
-                bool ok = true;
+                const int half = ti.n_mma >> 1;  // tokens per CTA
+                const int nbb = (half + Cfg::B_BOX_ROWS - 1) / Cfg::B_BOX_ROWS;
+                const uint32_t tx_cta = Cfg::A_BYTES + (uint32_t)nbb * Cfg::B_BOX_BYTES;
+                const int brow = ti.row0 + (int)rank * half;
+                // this CTA's A columns: gate/up -> [gate 64 | up 64] of features
+                // f0 + 64*rank; down -> 128 features f0 + 128*rank
+                const int acol0 =
+                    (MODE == MODE_GATEUP) ? ti.f0 + 64 * (int)rank : ti.f0 + 128 * (int)rank;
                 for (int kb = 0; kb < nkb; ++kb) {
                     if (!mbar_wait(empty_bar(stage), phase ^ 1u, args.err, DEV_ERR_TIMEOUT_PRODUCER)) {
-                        ok = false;
+                        aborted = true;
                         break;
                     }
-                    mbar_arrive_expect_tx(full_bar(stage), tx);
+                    const uint32_t fb_local = full_bar(stage);
+                    const uint32_t fb_leader = mapa_shared(fb_local, 0);
+                    if (leader) mbar_arrive_expect_tx(fb_local, 2 * tx_cta);
                     const uint32_t sb = stage0 + (uint32_t)stage * Cfg::STAGE_BYTES;
                     // leading shared-expert segment (down only), then the tile's own weights
                     const bool pre = kb < nkb_pre;
@@ -224,17 +255,20 @@ __global__ void __launch_bounds__(192, 1)
                     const void* bmap = pre ? (const void*)&b_shared : bmap_main;
                     const int k = (pre ? kb : kb - nkb_pre) * C::BK;
 #pragma unroll
-                    for (int op = 0; op < Cfg::A_OPS; ++op) {
-                        const int col0 = (op == 0 ? 0 : ti.up_off) + ti.f0;
-#pragma unroll
-                        for (int bx = 0; bx < Cfg::A_BOXES; ++bx)
-                            tma_load_2d(sb + op * Cfg::A_OP_BYTES + bx * Cfg::A_BOX_BYTES, amap,
-                                        full_bar(stage), col0 + bx * Cfg::A_BOX_FEATS, k);
+                    for (int bx = 0; bx < Cfg::A_BOXES; ++bx) {
+                        int col;
+                        if constexpr (MODE == MODE_GATEUP) {
+                            const int j = bx * Cfg::A_BOX_FEATS;  // 0..127 within [gate 64 | up 64]
+                            col = (j < 64 ? 0 : ti.up_off - 64) + acol0 + j;
+                        } else {
+                            col = acol0 + bx * Cfg::A_BOX_FEATS;
+                        }
+                        tma_load_2d_pair(sb + bx * Cfg::A_BOX_BYTES, amap, fb_leader, col, k);
                     }
-                    const uint32_t bb = sb + Cfg::A_OPS * Cfg::A_OP_BYTES;
+                    const uint32_t bb = sb + Cfg::A_BYTES;
                     for (int j = 0; j < nbb; ++j)
-                        tma_load_2d(bb + j * Cfg::B_BOX_BYTES, bmap, full_bar(stage), k,
-                                    ti.row0 + j * Cfg::B_BOX_ROWS);
+                        tma_load_2d_pair(bb + j * Cfg::B_BOX_BYTES, bmap, fb_leader, k,
+                                         brow + j * Cfg::B_BOX_ROWS);
                     used |= 1u << stage;
                     last_par = (last_par & ~(1u << stage)) | (phase << stage);
                     if (++stage == Cfg::STAGES) {
@@ -242,25 +276,30 @@ __global__ void __launch_bounds__(192, 1)
                         phase ^= 1u;
                     }
                 }
-                if (!ok) break;
             }
-            // drain: every issued copy must land before the CTA may exit
-            for (int s = 0; s < Cfg::STAGES; ++s)
-                if (used & (1u << s))
-                    mbar_wait(full_bar(s), (last_par >> s) & 1u, args.err, DEV_ERR_TIMEOUT_PRODUCER);
+            if (leader) {
+                // the leader's full barriers count both CTAs' bytes: wait for
+                // every issued copy before the pair may exit
+                for (int s = 0; s < Cfg::STAGES; ++s)
+                    if (used & (1u << s))
+                        mbar_wait(full_bar(s), (last_par >> s) & 1u, args.err, DEV_ERR_TIMEOUT_PRODUCER);
+            } else if (aborted) {
+                __nanosleep(100000);  // let this CTA's own copies land before exit
+            }
         }
     } else if (warp == 1) {
-        if (lane == 0) {
-            // ------------------------------------------------ MMA issuer
+        if (lane == 0 && leader) {
+            // ------------------------------------------------ MMA issuer (leader)
             int stage = 0;
             uint32_t phase = 0;
             int acc = 0;
             uint32_t acc_phase = 0;
-            for (int L = blockIdx.x; L < total; L += gridDim.x) {
-                const TileInfo ti = decode_tile(*tab, args, L);
-                if (!mbar_wait(tempty_bar(acc), acc_phase ^ 1u, args.err, DEV_ERR_TIMEOUT_MMA)) break;
+            for (int L = pair; L < total; L += npairs) {
+                const TileInfo ti = decode_tile<MODE>(*tab, args, L);
+                if (!mbar_wait_cluster(tempty_bar(acc), acc_phase ^ 1u, args.err, DEV_ERR_TIMEOUT_MMA))
+                    break;
                 tc_fence_after();
-                const uint32_t idesc = make_idesc(C::FMT, 1u, 0u, (uint32_t)ti.n_mma, 128u);
+                const uint32_t idesc = make_idesc(C::FMT, 1u, 0u, (uint32_t)ti.n_mma, 256u);
                 const uint32_t d_tmem = tmem_base + (uint32_t)acc * 256u;
                 const int nkb = ti.K / C::BK;
                 bool ok = true;
@@ -271,53 +310,53 @@ __global__ void __launch_bounds__(192, 1)
                     }
                     tc_fence_after();
                     const uint32_t sb = stage0 + (uint32_t)stage * Cfg::STAGE_BYTES;
-                    const uint32_t bb = sb + Cfg::A_OPS * Cfg::A_OP_BYTES;
+                    const uint32_t bb = sb + Cfg::A_BYTES;
 #pragma unroll
                     for (int kk = 0; kk < C::BK / C::MMA_K; ++kk) {
                         const uint64_t bdesc = smem_desc(bb + kk * 32, 16, 1024, 2);
-#pragma unroll
-                        for (int op = 0; op < Cfg::A_OPS; ++op) {
-                            const uint64_t adesc =
-                                smem_desc(sb + op * Cfg::A_OP_BYTES + kk * C::MMA_K * 128,
-                                          Cfg::A_BOX_BYTES, C::A_SBO, C::A_LAYOUT);
-                            const uint32_t accum = (kb | kk) != 0 ? 1u : 0u;
-                            if constexpr (C::FMT == 1)
-                                mma_bf16(d_tmem + op * 256u, adesc, bdesc, idesc, accum);
-                            else
-                                mma_tf32(d_tmem + op * 256u, adesc, bdesc, idesc, accum);
-                        }
+                        const uint64_t adesc = smem_desc(sb + kk * C::MMA_K * 128, Cfg::A_BOX_BYTES,
+                                                         C::A_SBO, C::A_LAYOUT);
+                        const uint32_t accum = (kb | kk) != 0 ? 1u : 0u;
+                        if constexpr (C::FMT == 1)
+                            mma_bf16_pair(d_tmem, adesc, bdesc, idesc, accum);
+                        else
+                            mma_tf32_pair(d_tmem, adesc, bdesc, idesc, accum);
                     }
-                    mma_commit(empty_bar(stage));
+                    mma_commit_pair_mc(empty_bar(stage), 0x3);  // frees the stage in both CTAs
                     if (++stage == Cfg::STAGES) {
                         stage = 0;
                         phase ^= 1u;
                     }
                 }
                 if (!ok) break;
-                mma_commit(tfull_bar(acc));
+                mma_commit_pair_mc(tfull_bar(acc), 0x3);  // accumulator ready in both CTAs
                 if (++acc == Cfg::ACC_BUFS) {
                     acc = 0;
                     acc_phase ^= 1u;
                 }
             }
-            // every issued MMA must finish before TMEM is released
-            mma_commit(drain_bar);
+            // every issued MMA must finish before the pair releases TMEM
+            mma_commit_pair(drain_bar);
             mbar_wait(drain_bar, 0, args.err, DEV_ERR_TIMEOUT_MMA);
         }
     } else {
         // ---------------------------------------------------- epilogue
-        const int q = warp & 3;            // TMEM lane quarter of this warp
-        const int row = q * 32 + lane;     // feature within the tile
+        const int q = warp & 3;  // TMEM lane quarter of this warp
         int acc = 0;
         uint32_t acc_phase = 0;
-        for (int L = blockIdx.x; L < total; L += gridDim.x) {
-            const TileInfo ti = decode_tile(*tab, args, L);
-            // warp-uniform outcome: the TMEM loads below are .sync.aligned
+        volatile uint32_t* abort_flag = misc + 1;
+        for (int L = pair; L < total; L += npairs) {
+            const TileInfo ti = decode_tile<MODE>(*tab, args, L);
             const bool ok = mbar_wait(tfull_bar(acc), acc_phase, args.err, DEV_ERR_TIMEOUT_EPILOGUE);
-            if (!__all_sync(0xffffffffu, ok)) break;
+            if constexpr (MODE == MODE_GATEUP) {
+                // the 4 warps meet at named barriers below: leave together or not at all
+                if (!__all_sync(0xffffffffu, ok) && lane == 0) *abort_flag = 1u;
+                named_bar_sync(1, 128);
+                if (*abort_flag) break;
+            } else {
+                if (!__all_sync(0xffffffffu, ok)) break;
+            }
             tc_fence_after();
-            const int f = ti.f0 + row;
-            const bool fvalid = f < ti.M;
             const uint32_t tb = tmem_base + ((uint32_t)(q * 32) << 16) + (uint32_t)acc * 256u;
             ET* outp = reinterpret_cast<ET*>(ti.shared ? args.out_shared : args.out_routed);
             const long long ld = ti.shared ? args.ld_shared : args.ld_routed;
@@ -331,19 +370,38 @@ __global__ void __launch_bounds__(192, 1)
                 const float my_scale = (cval && colscale) ? colscale[ti.row0 + c + lane] : 1.0f;
                 float v[32];
                 tmem_ld_32x32(tb + (uint32_t)c, v);
+                tmem_wait_ld();
                 if constexpr (MODE == MODE_GATEUP) {
-                    float u[32];
-                    tmem_ld_32x32(tb + 256u + (uint32_t)c, u);
-                    tmem_wait_ld();
+                    // lanes 0-63: gate rows, 64-127: up rows of the same 64 features.
+                    // Gate warps (q 0,1) finish columns c..c+15, up warps (q 2,3)
+                    // columns c+16..c+31; each hands the other half over.
+                    const bool gate_warp = q < 2;
+                    const int pq = q & 1;  // feature quarter of the pair
+                    float* xg = xch + (0 * 2 + pq) * 32 * Cfg::XLD;  // gate values, cols 16..31
+                    float* xu = xch + (1 * 2 + pq) * 32 * Cfg::XLD;  // up values, cols 0..15
 #pragma unroll
-                    for (int i = 0; i < 32; ++i) {
-                        const int orow = __shfl_sync(0xffffffffu, my_row, i);
-                        const float g = __shfl_sync(0xffffffffu, my_scale, i);
-                        if (fvalid && c + i < ti.n_valid)
-                            store_elem(outp + (size_t)orow * ld + f, silu_f(g * v[i]) * (g * u[i]));
+                    for (int i = 0; i < 16; ++i) {
+                        if (gate_warp) xg[lane * Cfg::XLD + i] = v[16 + i];
+                        else xu[lane * Cfg::XLD + i] = v[i];
                     }
+                    named_bar_sync(1, 128);
+                    const int f = ti.f0 + 64 * (int)rank + 32 * pq + lane;
+                    const bool fvalid = f < ti.M;
+                    const int cb = gate_warp ? 0 : 16;
+#pragma unroll
+                    for (int i = 0; i < 16; ++i) {
+                        const int col = cb + i;
+                        const int orow = __shfl_sync(0xffffffffu, my_row, col);
+                        const float g = __shfl_sync(0xffffffffu, my_scale, col);
+                        const float gv = gate_warp ? v[i] : xg[lane * Cfg::XLD + i];
+                        const float uv = gate_warp ? xu[lane * Cfg::XLD + i] : v[16 + i];
+                        if (fvalid && c + col < ti.n_valid)
+                            store_elem(outp + (size_t)orow * ld + f, silu_f(g * gv) * (g * uv));
+                    }
+                    named_bar_sync(1, 128);  // exchange buffer free for the next chunk
                 } else {
-                    tmem_wait_ld();
+                    const int f = ti.f0 + 128 * (int)rank + 32 * q + lane;
+                    const bool fvalid = f < ti.M;
 #pragma unroll
                     for (int i = 0; i < 32; ++i) {
                         const int orow = __shfl_sync(0xffffffffu, my_row, i);
@@ -354,7 +412,7 @@ __global__ void __launch_bounds__(192, 1)
             }
             tc_fence_before();
             __syncwarp();
-            if (lane == 0) mbar_arrive(tempty_bar(acc));
+            if (lane == 0) mbar_arrive_remote(mapa_shared(tempty_bar(acc), 0));  // to the leader
             if (++acc == Cfg::ACC_BUFS) {
                 acc = 0;
                 acc_phase ^= 1u;
@@ -363,10 +421,11 @@ __global__ void __launch_bounds__(192, 1)
     }
 
     tc_fence_before();
-    __syncthreads();
+    __syncwarp();
+    cluster_sync();  // no CTA of the pair leaves while the other may still use its memory
     if (warp == 1) {
         tc_fence_after();
-        tmem_dealloc(tmem_base, Cfg::TMEM_COLS);
+        tmem_dealloc_pair(tmem_base, Cfg::TMEM_COLS);
     }
 }
 

@@ -17,6 +17,8 @@
 #include <cuda_bf16.h>
 #include <cstdint>
 
+#include "ptx.cuh"
+
 namespace l4moe {
 
 __device__ __forceinline__ float to_f32(float v) { return v; }
@@ -173,6 +175,147 @@ __global__ void __launch_bounds__(NT) router_kernel(const ET* __restrict__ x,
         lmax[t] = best;
         margin[t] = best - second;
         gate[t] = 1.0f / (1.0f + expf(-best));
+    }
+}
+
+// ---------------------------------------------------------------------------
+// Tensor-core router for bf16 layers with E % 8 == 0 (E <= 256): one CTA per
+// 128-token tile computes the fp32 logits of all E experts with tcgen05 (M =
+// 128 tokens, N = E rounded up to 16, K = d; x rows are the K-major A
+// operand, W_router [d, E] the MN-major B operand), then each of 128 threads
+// owns one token's logits in TMEM and applies the same arg-max / runner-up /
+// sigmoid rule as the CUDA-core router above.  Warp 0 lane 0 issues the TMA
+// loads, warp 1 lane 0 the MMAs; all four warps run the epilogue.
+namespace rmma {
+constexpr int STAGES = 4;
+constexpr int A_BYTES = 128 * 128;     // 128 tokens x 64 K (bf16)
+constexpr int B_BOX_BYTES = 64 * 128;  // 64 K rows x 64 experts (bf16)
+constexpr int MAX_B_BOXES = 4;         // E <= 256
+constexpr int STAGE_BYTES = A_BYTES + MAX_B_BOXES * B_BOX_BYTES;
+constexpr size_t SMEM_BYTES = 1024 + (size_t)STAGES * STAGE_BYTES + (2 * STAGES + 1) * 8 + 16;
+}  // namespace rmma
+
+__global__ void __launch_bounds__(128, 1)
+    router_mma_kernel(const __grid_constant__ CUtensorMap x_map, const __grid_constant__ CUtensorMap wr_map,
+                      const float* __restrict__ bias, int T, int d, int E, int32_t* __restrict__ idx,
+                      float* __restrict__ gate, float* __restrict__ lmax,
+                      float* __restrict__ margin, unsigned* err) {
+    extern __shared__ uint8_t rsmem_raw[];
+    uint8_t* smem = reinterpret_cast<uint8_t*>(
+        (reinterpret_cast<uintptr_t>(rsmem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
+    uint64_t* bars = reinterpret_cast<uint64_t*>(smem + (size_t)rmma::STAGES * rmma::STAGE_BYTES);
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 2 * rmma::STAGES + 1);
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const uint32_t stage0 = smem_u32(smem), bar0 = smem_u32(bars);
+    auto full_bar = [&](int s) { return bar0 + 8u * s; };
+    auto empty_bar = [&](int s) { return bar0 + 8u * (rmma::STAGES + s); };
+    const uint32_t done_bar = bar0 + 8u * (2 * rmma::STAGES);
+    const int n_pad = (E + 15) & ~15;
+    const int nbb = (E + 63) / 64;
+    uint32_t ncols = 32;
+    while ((int)ncols < n_pad) ncols <<= 1;
+
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < rmma::STAGES; ++s) {
+            mbar_init(full_bar(s), 1);
+            mbar_init(empty_bar(s), 1);
+        }
+        mbar_init(done_bar, 1);
+        fence_barrier_init();
+    }
+    if (warp == 1) {
+        tmem_alloc(smem_u32(tmem_slot), ncols);
+        tmem_relinquish();
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem_base = *tmem_slot;
+    const int t0 = blockIdx.x * 128;
+    const int nkb = d / 64;
+
+    if (warp == 0 && lane == 0) {
+        int stage = 0;
+        uint32_t phase = 0, used = 0, last_par = 0;
+        for (int kb = 0; kb < nkb; ++kb) {
+            if (!mbar_wait(empty_bar(stage), phase ^ 1u, err, DEV_ERR_TIMEOUT_PRODUCER)) break;
+            mbar_arrive_expect_tx(full_bar(stage), rmma::A_BYTES + nbb * rmma::B_BOX_BYTES);
+            const uint32_t sb = stage0 + (uint32_t)stage * rmma::STAGE_BYTES;
+            tma_load_2d(sb, &x_map, full_bar(stage), kb * 64, t0);
+            tma_load_2d(sb + 64 * 128, &x_map, full_bar(stage), kb * 64, t0 + 64);
+            for (int j = 0; j < nbb; ++j)
+                tma_load_2d(sb + rmma::A_BYTES + j * rmma::B_BOX_BYTES, &wr_map, full_bar(stage), 64 * j,
+                            kb * 64);
+            used |= 1u << stage;
+            last_par = (last_par & ~(1u << stage)) | (phase << stage);
+            if (++stage == rmma::STAGES) {
+                stage = 0;
+                phase ^= 1u;
+            }
+        }
+        for (int s = 0; s < rmma::STAGES; ++s)  // drain copies in flight
+            if (used & (1u << s)) mbar_wait(full_bar(s), (last_par >> s) & 1u, err, DEV_ERR_TIMEOUT_PRODUCER);
+    } else if (warp == 1 && lane == 0) {
+        int stage = 0;
+        uint32_t phase = 0;
+        const uint32_t idesc = make_idesc(1u, 0u, 1u, (uint32_t)n_pad, 128u);
+        for (int kb = 0; kb < nkb; ++kb) {
+            if (!mbar_wait(full_bar(stage), phase, err, DEV_ERR_TIMEOUT_MMA)) break;
+            tc_fence_after();
+            const uint32_t sb = stage0 + (uint32_t)stage * rmma::STAGE_BYTES;
+#pragma unroll
+            for (int kk = 0; kk < 4; ++kk) {
+                const uint64_t adesc = smem_desc(sb + kk * 32, 16, 1024, 2);
+                const uint64_t bdesc = smem_desc(sb + rmma::A_BYTES + kk * 2048, rmma::B_BOX_BYTES, 1024, 2);
+                mma_bf16(tmem_base, adesc, bdesc, idesc, (kb | kk) != 0 ? 1u : 0u);
+            }
+            mma_commit(empty_bar(stage));
+            if (++stage == rmma::STAGES) {
+                stage = 0;
+                phase ^= 1u;
+            }
+        }
+        mma_commit(done_bar);  // logits complete (or every issued MMA finished)
+    }
+    __syncwarp();
+    // epilogue: thread = token row (TMEM lane 32*warp + lane)
+    const bool ok = mbar_wait(done_bar, 0, err, DEV_ERR_TIMEOUT_EPILOGUE);
+    if (__all_sync(0xffffffffu, ok)) {
+        tc_fence_after();
+        float best = -INFINITY, second = -INFINITY;
+        int bi = 0;
+        for (int c = 0; c < n_pad; c += 32) {
+            float v[32];
+            tmem_ld_32x32(tmem_base + ((uint32_t)(32 * warp) << 16) + (uint32_t)c, v);
+            tmem_wait_ld();
+#pragma unroll
+            for (int i = 0; i < 32; ++i) {
+                const int e = c + i;
+                if (e < E) {
+                    const float l = v[i] + (bias ? bias[e] : 0.f);
+                    if (l > best) {
+                        second = best;
+                        best = l;
+                        bi = e;
+                    } else if (l > second) {
+                        second = l;
+                    }
+                }
+            }
+        }
+        const int t = t0 + 32 * warp + lane;
+        if (t < T) {
+            idx[t] = bi;
+            lmax[t] = best;
+            margin[t] = best - second;
+            gate[t] = 1.0f / (1.0f + expf(-best));
+        }
+    }
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 1) {
+        tc_fence_after();
+        tmem_dealloc(tmem_base, ncols);
     }
 }
 
