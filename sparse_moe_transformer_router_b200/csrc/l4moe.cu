@@ -114,6 +114,8 @@ struct l4moe_handle {
     std::vector<const float*> s_gu, s_dn;
     const float* ss_gu = nullptr;
     const float* ss_dn = nullptr;
+    const float** d_scales = nullptr;  // device [2][E+1] scale pointers (gate/up, down)
+    bool scales_dirty = false;
     // TMA descriptors of the weights, keyed by pointer value
     std::vector<const void*> key_gu, key_dn;
     const void* key_sgu = nullptr;
@@ -209,11 +211,15 @@ l4moe_status encode_weight_maps(l4moe_handle* h, const void* const* Wgu, const v
     CUtensorMapDataType dt = h->p.dtype == L4MOE_F32 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT32
                              : h->p.dtype == L4MOE_BF16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16
                                                         : CU_TENSOR_MAP_DATA_TYPE_UINT8;
+    const bool fp8 = h->p.dtype == L4MOE_FP8_E4M3;
     const uint32_t bk = h->p.dtype == L4MOE_F32 ? 32 : 64;  // K rows per box
-    const uint32_t bw = (uint32_t)(128 / wb);               // features per box
+    // features per box: one 128-byte swizzled slab; E4M3 weights are staged
+    // raw (64-feature boxes, unswizzled) and widened in shared memory
+    const uint32_t bw = fp8 ? 64u : (uint32_t)(128 / wb);
     // MN-major 32-bit operands need the 32-byte swizzle unit
-    const CUtensorMapSwizzle swz = h->p.dtype == L4MOE_F32 ? CU_TENSOR_MAP_SWIZZLE_128B_ATOM_32B
-                                                           : CU_TENSOR_MAP_SWIZZLE_128B;
+    const CUtensorMapSwizzle swz = fp8 ? CU_TENSOR_MAP_SWIZZLE_NONE
+                                   : h->p.dtype == L4MOE_F32 ? CU_TENSOR_MAP_SWIZZLE_128B_ATOM_32B
+                                                             : CU_TENSOR_MAP_SWIZZLE_128B;
     h->h_maps.assign(2 * (E + 1), CUtensorMap{});
     h->hkey_gu.clear();
     for (int e = 0; e <= E; ++e) {
@@ -290,19 +296,19 @@ void launch_router(const void* x, const void* Wr, const float* bias, int T, int 
     else launch_router_t<ET, 256, 8, 8>(x, Wr, bias, T, d, E, idx, gate, lmax, margin, st);
 }
 
-template <int MODE, typename ET>
+template <int MODE, typename ET, bool FP8W>
 void launch_gemm(int grid, const CUtensorMap& b_routed, const CUtensorMap& b_shared,
                  const GemmArgs& a, cudaStream_t st) {
-    using Cfg = GemmCfg<MODE, ET>;
+    using Cfg = GemmCfg<MODE, ET, FP8W>;
     static std::once_flag once;
-    std::call_once(once, [] { set_smem_attr(moe_gemm_kernel<MODE, ET>, Cfg::SMEM_BYTES); });
-    moe_gemm_kernel<MODE, ET><<<grid, 192, Cfg::SMEM_BYTES, st>>>(b_routed, b_shared, a);
+    std::call_once(once, [] { set_smem_attr(moe_gemm_kernel<MODE, ET, FP8W>, Cfg::SMEM_BYTES); });
+    moe_gemm_kernel<MODE, ET, FP8W><<<grid, Cfg::THREADS, Cfg::SMEM_BYTES, st>>>(b_routed, b_shared, a);
 }
 
 // The launch sequence of one forward.  w / ws_tokens: the workspace and the
 // token count its layout was made for; maps: device array of the 2(E+1)
 // weight descriptors.
-template <typename ET>
+template <typename ET, bool FP8W = false>
 l4moe_status run_layer(l4moe_handle* h, int T, const void* x, const void* Wr, const void* Wsgu,
                        const void* Wsdn, void* out, cudaStream_t st, uint8_t* w, int ws_tokens,
                        const CUtensorMap* maps) {
@@ -402,9 +408,10 @@ l4moe_status run_layer(l4moe_handle* h, int T, const void* x, const void* Wr, co
     gu.rowmap_routed = nullptr;
     gu.rowmap_shared = inv;
     gu.colscale_routed = gslot;  // sigmoid gate of each routed slot
+    gu.wscale = FP8W ? h->d_scales : nullptr;
     gu.err = err;
     LaunchTimer t_gu(h, 3, st);
-    launch_gemm<MODE_GATEUP, ET>(
+    launch_gemm<MODE_GATEUP, ET, FP8W>(
         grid_for((long long)fb_gu_s * tb + (long long)fb_gu_r * (tb + std::min(E, T))), m_xg, m_x,
         gu, st);
     t_gu.stop();
@@ -426,13 +433,39 @@ l4moe_status run_layer(l4moe_handle* h, int T, const void* x, const void* Wr, co
     dn.rowmap_routed = perm;     // slot -> token: un-permute on store
     dn.rowmap_shared = nullptr;
     dn.colscale_routed = nullptr;
+    dn.wscale = FP8W ? h->d_scales + (E + 1) : nullptr;
     dn.err = err;
     LaunchTimer t_dn(h, 4, st);
-    launch_gemm<MODE_DOWN, ET>(grid_for((long long)fb_dn * (tb + std::min(E, T))), m_hr, m_hs, dn, st);
+    launch_gemm<MODE_DOWN, ET, FP8W>(grid_for((long long)fb_dn * (tb + std::min(E, T))), m_hr, m_hs, dn, st);
     t_dn.stop();
     L4MOE_CHECK_LAUNCH("down launch");
 #undef L4MOE_CHECK_LAUNCH
     h->last_T = T;
+    return L4MOE_OK;
+}
+
+// Device table of the per-column scale vectors of the E4M3 weights:
+// [gate/up of experts 0..E-1, shared gate/up, down of experts 0..E-1, shared down].
+l4moe_status ensure_scales(l4moe_handle* h, cudaStream_t st) {
+    const int E = h->p.num_experts;
+    if (!h->d_scales) {
+        cudaError_t e = cudaMalloc(&h->d_scales, sizeof(float*) * 2 * (E + 1));
+        if (e != cudaSuccess) return cuda_fail(h, e, "scale table cudaMalloc");
+        h->scales_dirty = true;
+    }
+    if (!h->scales_dirty) return L4MOE_OK;
+    std::vector<const float*> tab(2 * (E + 1));
+    for (int e = 0; e < E; ++e) {
+        tab[e] = h->s_gu[e];
+        tab[E + 1 + e] = h->s_dn[e];
+    }
+    tab[E] = h->ss_gu;
+    tab[2 * E + 1] = h->ss_dn;
+    // pageable source: staged before the call returns
+    cudaError_t e = cudaMemcpyAsync(h->d_scales, tab.data(), sizeof(float*) * tab.size(),
+                                    cudaMemcpyHostToDevice, st);
+    if (e != cudaSuccess) return cuda_fail(h, e, "scale table upload");
+    h->scales_dirty = false;
     return L4MOE_OK;
 }
 
@@ -462,14 +495,18 @@ l4moe_status forward_impl(l4moe_handle* h, int T, const void* x, const void* Wr,
     l4moe_status s;
     if ((s = ensure_workspace(h, T)) != L4MOE_OK) return s;
     if ((s = ensure_weight_maps(h, Wgu, Wdn, Wsgu, Wsdn, st)) != L4MOE_OK) return s;
+    if (h->p.dtype == L4MOE_FP8_E4M3 && (s = ensure_scales(h, st)) != L4MOE_OK) return s;
     switch (h->p.dtype) {
     case L4MOE_F32:
         return run_layer<float>(h, T, x, Wr, Wsgu, Wsdn, out, st, h->ws, h->ws_tokens, h->d_maps);
     case L4MOE_BF16:
         return run_layer<__nv_bfloat16>(h, T, x, Wr, Wsgu, Wsdn, out, st, h->ws, h->ws_tokens,
                                         h->d_maps);
-    default: return fail(h, L4MOE_ERR_UNSUPPORTED, "FP8 weight path not built in this library");
+    case L4MOE_FP8_E4M3:
+        return run_layer<__nv_bfloat16, true>(h, T, x, Wr, Wsgu, Wsdn, out, st, h->ws, h->ws_tokens,
+                                              h->d_maps);
     }
+    return fail(h, L4MOE_ERR_DTYPE, "unknown dtype");
 }
 
 // ------------------------------------------------------------------------
@@ -596,6 +633,7 @@ void l4moe_destroy(l4moe_handle* h) {
     }
     if (h->ws_owned && h->ws) cudaFree(h->ws);
     if (h->d_maps) cudaFree(h->d_maps);
+    if (h->d_scales) cudaFree(h->d_scales);
     delete h;
 }
 
@@ -642,6 +680,7 @@ l4moe_status l4moe_set_fp8_scales(l4moe_handle* h, const float* const* s_gate_up
     h->s_dn.assign(s_down, s_down + E);
     h->ss_gu = ss_gate_up;
     h->ss_dn = ss_down;
+    h->scales_dirty = true;
     return L4MOE_OK;
 }
 

@@ -36,7 +36,14 @@
 // Accumulators are double-buffered (2 x 256 TMEM columns) so the epilogue of
 // one tile overlaps the MMAs of the next.
 //
-// Roles (192 threads per CTA): warp 0 lane 0 issues TMA loads into a
+// E4M3 weights (FP8W): TMA brings the raw 8-bit A tile (64 K rows x 2 slabs
+// of 64 features) into a raw ring; four converter warps widen it to bf16,
+// multiplying each value by its output column's fp32 scale (one bf16
+// rounding of q * scale), write the swizzled MN-major operand layout, fence
+// to the async proxy and report to the leader; the MMA waits for the token
+// tile and for both CTAs' converted weights.
+//
+// Roles (192 threads per CTA, 320 with E4M3 weights): warp 0 lane 0 issues TMA loads into a
 // STAGES-deep ring (both CTAs; completion counted on the leader's barrier);
 // warp 1 allocates TMEM (both CTAs) and, in the leader CTA only, lane 0
 // issues the MMAs and commits to both CTAs' barriers; warps 2..5 are the
@@ -46,6 +53,7 @@
 // copies and MMAs in flight before the pair synchronises and frees TMEM.
 #pragma once
 #include <cuda_bf16.h>
+#include <cuda_fp8.h>
 #include <cstdint>
 
 #include "permute.cuh"
@@ -91,6 +99,8 @@ struct GemmArgs {
     const int32_t* rowmap_routed;  // down: output row of a slot (perm), else null
     const int32_t* rowmap_shared;  // gate/up: slot of a token (inv), else null
     const float* colscale_routed;  // gate/up: sigmoid gate of each slot, else null
+    const float* const* wscale;    // E4M3 weights: per-column scale vector of each of the
+                                   // E + 1 weight matrices of this launch, else null
     unsigned* err;
 };
 
@@ -98,7 +108,7 @@ struct GemmArgs {
 template <int MODE>
 __host__ __device__ constexpr int pair_features() { return MODE == MODE_GATEUP ? 128 : 256; }
 
-template <int MODE, typename ET>
+template <int MODE, typename ET, bool FP8W>
 struct GemmCfg {
     using C = ElemCfg<ET>;
     static constexpr int A_BYTES = 128 * 128;                // 128 A rows x 128 B of K
@@ -108,13 +118,15 @@ struct GemmCfg {
     static constexpr int B_BOX_ROWS = 64;
     static constexpr int B_BOX_BYTES = B_BOX_ROWS * 128;
     static constexpr int B_BYTES = (kTokTile / 2) * 128;     // this CTA's half of the tokens
-    static constexpr int STAGE_BYTES = A_BYTES + B_BYTES;    // 32 KB
-    static constexpr int STAGES = 6;
+    static constexpr int RAW_BYTES = FP8W ? 2 * 64 * 64 : 0; // 2 slabs x 64 K rows x 64 features
+    static constexpr int STAGE_BYTES = A_BYTES + B_BYTES + RAW_BYTES;
+    static constexpr int STAGES = FP8W ? 5 : 6;
     static constexpr int ACC_BUFS = 2;
     static constexpr int TMEM_COLS = 512;
+    static constexpr int THREADS = FP8W ? 320 : 192;
     static constexpr int XLD = 17;                           // exchange row stride (floats)
     static constexpr int XCH_BYTES = (MODE == MODE_GATEUP) ? 2 * 2 * 32 * XLD * 4 : 0;
-    static constexpr int NUM_BARS = 2 * STAGES + 2 * ACC_BUFS + 1;
+    static constexpr int NUM_BARS = 2 * STAGES + 2 * ACC_BUFS + 1 + (FP8W ? 2 * STAGES : 0);
     static constexpr size_t SMEM_BYTES = 1024 /*alignment slack*/ + (size_t)STAGES * STAGE_BYTES +
                                          XCH_BYTES + NUM_BARS * 8 + 16 + sizeof(GroupTable);
 };
@@ -153,14 +165,37 @@ __device__ __forceinline__ TileInfo decode_tile(const GroupTable& tab, const Gem
 
 __device__ __forceinline__ float silu_f(float z) { return __fdividef(z, 1.0f + __expf(-z)); }
 
+// 8 E4M3 codes (little-endian in a uint2) -> 8 bf16 values of code * scale.
+__device__ __forceinline__ uint4 e4m3x8_scaled_to_bf16(uint2 raw, const float (&sc)[8]) {
+    const uint32_t w[2] = {raw.x, raw.y};
+    uint32_t o[4];
+#pragma unroll
+    for (int h = 0; h < 2; ++h) {
+#pragma unroll
+        for (int p = 0; p < 2; ++p) {
+            const __nv_fp8x2_storage_t two = (__nv_fp8x2_storage_t)((w[h] >> (16 * p)) & 0xffffu);
+            const __half2_raw hr = __nv_cvt_fp8x2_to_halfraw2(two, __NV_E4M3);
+            const float2 f = __half22float2(*reinterpret_cast<const __half2*>(&hr));
+            const int i = 4 * h + 2 * p;
+            const __nv_bfloat162 b = __floats2bfloat162_rn(f.x * sc[i], f.y * sc[i + 1]);
+            o[2 * h + p] = *reinterpret_cast<const uint32_t*>(&b);
+        }
+    }
+    return make_uint4(o[0], o[1], o[2], o[3]);
+}
+
+__device__ __forceinline__ void fence_proxy_async_smem() {
+    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+}
+
 __device__ __forceinline__ void store_elem(float* p, float v) { *p = v; }
 __device__ __forceinline__ void store_elem(__nv_bfloat16* p, float v) { *p = __float2bfloat16_rn(v); }
 
-template <int MODE, typename ET>
-__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(192, 1)
+template <int MODE, typename ET, bool FP8W>
+__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(GemmCfg<MODE, ET, FP8W>::THREADS, 1)
     moe_gemm_kernel(const __grid_constant__ CUtensorMap b_routed,
                     const __grid_constant__ CUtensorMap b_shared, const GemmArgs args) {
-    using Cfg = GemmCfg<MODE, ET>;
+    using Cfg = GemmCfg<MODE, ET, FP8W>;
     using C = ElemCfg<ET>;
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>(
@@ -182,6 +217,11 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(192, 1)
     auto tfull_bar = [&](int b) { return bar0 + 8u * (2 * Cfg::STAGES + b); };
     auto tempty_bar = [&](int b) { return bar0 + 8u * (2 * Cfg::STAGES + Cfg::ACC_BUFS + b); };
     const uint32_t drain_bar = bar0 + 8u * (2 * Cfg::STAGES + 2 * Cfg::ACC_BUFS);
+    // E4M3 weights: raw tile landed (local) / both CTAs' converted tile ready (leader)
+    auto rawfull_bar = [&](int s) { return bar0 + 8u * (2 * Cfg::STAGES + 2 * Cfg::ACC_BUFS + 1 + s); };
+    auto conv_bar = [&](int s) {
+        return bar0 + 8u * (3 * Cfg::STAGES + 2 * Cfg::ACC_BUFS + 1 + s);
+    };
 
     {   // work list -> shared memory
         const int* src = reinterpret_cast<const int*>(args.table);
@@ -198,6 +238,12 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(192, 1)
             mbar_init(tempty_bar(b), 8);  // leader: 4 epilogue warps of each CTA
         }
         mbar_init(drain_bar, 1);
+        if constexpr (FP8W) {
+            for (int s = 0; s < Cfg::STAGES; ++s) {
+                mbar_init(rawfull_bar(s), 1);
+                mbar_init(conv_bar(s), 8);  // leader: 4 converter warps of each CTA
+            }
+        }
         misc[1] = 0;
         fence_barrier_init();
     }
@@ -234,7 +280,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(192, 1)
                 const int nkb_pre = ti.k_pre / C::BK;
                 const int half = ti.n_mma >> 1;  // tokens per CTA
                 const int nbb = (half + Cfg::B_BOX_ROWS - 1) / Cfg::B_BOX_ROWS;
-                const uint32_t tx_cta = Cfg::A_BYTES + (uint32_t)nbb * Cfg::B_BOX_BYTES;
+                const uint32_t tx_cta = (FP8W ? 0u : (uint32_t)Cfg::A_BYTES) + (uint32_t)nbb * Cfg::B_BOX_BYTES;
                 const int brow = ti.row0 + (int)rank * half;
                 // this CTA's A columns: gate/up -> [gate 64 | up 64] of features
                 // f0 + 64*rank; down -> 128 features f0 + 128*rank
@@ -254,16 +300,29 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(192, 1)
                     const CUtensorMap* amap = pre ? amap_pre : amap_main;
                     const void* bmap = pre ? (const void*)&b_shared : bmap_main;
                     const int k = (pre ? kb : kb - nkb_pre) * C::BK;
+                    if constexpr (FP8W) {
+                        // raw 8-bit weights: two 64-feature slabs, signalled locally
+                        const uint32_t rb = sb + Cfg::A_BYTES + Cfg::B_BYTES;
+                        mbar_arrive_expect_tx(rawfull_bar(stage), Cfg::RAW_BYTES);
 #pragma unroll
-                    for (int bx = 0; bx < Cfg::A_BOXES; ++bx) {
-                        int col;
-                        if constexpr (MODE == MODE_GATEUP) {
-                            const int j = bx * Cfg::A_BOX_FEATS;  // 0..127 within [gate 64 | up 64]
-                            col = (j < 64 ? 0 : ti.up_off - 64) + acol0 + j;
-                        } else {
-                            col = acol0 + bx * Cfg::A_BOX_FEATS;
+                        for (int j = 0; j < 2; ++j) {
+                            const int col = (MODE == MODE_GATEUP)
+                                                ? (j == 0 ? acol0 : ti.up_off + acol0)
+                                                : acol0 + 64 * j;
+                            tma_load_2d(rb + j * 4096, amap, rawfull_bar(stage), col, k);
                         }
-                        tma_load_2d_pair(sb + bx * Cfg::A_BOX_BYTES, amap, fb_leader, col, k);
+                    } else {
+#pragma unroll
+                        for (int bx = 0; bx < Cfg::A_BOXES; ++bx) {
+                            int col;
+                            if constexpr (MODE == MODE_GATEUP) {
+                                const int j = bx * Cfg::A_BOX_FEATS;  // 0..127 within [gate 64 | up 64]
+                                col = (j < 64 ? 0 : ti.up_off - 64) + acol0 + j;
+                            } else {
+                                col = acol0 + bx * Cfg::A_BOX_FEATS;
+                            }
+                            tma_load_2d_pair(sb + bx * Cfg::A_BOX_BYTES, amap, fb_leader, col, k);
+                        }
                     }
                     const uint32_t bb = sb + Cfg::A_BYTES;
                     for (int j = 0; j < nbb; ++j)
@@ -276,6 +335,11 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(192, 1)
                         phase ^= 1u;
                     }
                 }
+            }
+            if constexpr (FP8W) {  // raw weight copies are counted on this CTA's barriers
+                for (int s = 0; s < Cfg::STAGES; ++s)
+                    if (used & (1u << s))
+                        mbar_wait(rawfull_bar(s), (last_par >> s) & 1u, args.err, DEV_ERR_TIMEOUT_PRODUCER);
             }
             if (leader) {
                 // the leader's full barriers count both CTAs' bytes: wait for
@@ -308,6 +372,12 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(192, 1)
                         ok = false;
                         break;
                     }
+                    if constexpr (FP8W) {
+                        if (!mbar_wait_cluster(conv_bar(stage), phase, args.err, DEV_ERR_TIMEOUT_MMA)) {
+                            ok = false;
+                            break;
+                        }
+                    }
                     tc_fence_after();
                     const uint32_t sb = stage0 + (uint32_t)stage * Cfg::STAGE_BYTES;
                     const uint32_t bb = sb + Cfg::A_BYTES;
@@ -338,6 +408,60 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(192, 1)
             // every issued MMA must finish before the pair releases TMEM
             mma_commit_pair(drain_bar);
             mbar_wait(drain_bar, 0, args.err, DEV_ERR_TIMEOUT_MMA);
+        }
+    } else if (FP8W && warp >= 6) {
+        // ---------------------------------------------------- E4M3 converters
+        const int ct = threadIdx.x - 192;  // 0..127
+        const int c8 = ct & 7;             // 8-feature chunk of each slab this thread owns
+        int stage = 0;
+        uint32_t phase = 0;
+        bool ok = true;
+        for (int L = pair; L < total && ok; L += npairs) {
+            const TileInfo ti = decode_tile<MODE>(*tab, args, L);
+            const int nkb = ti.K / C::BK;
+            const int nkb_pre = ti.k_pre / C::BK;
+            const int acol0 = (MODE == MODE_GATEUP) ? ti.f0 + 64 * (int)rank : ti.f0 + 128 * (int)rank;
+            float sc[2][8];
+            int seg = -1;
+            for (int kb = 0; kb < nkb; ++kb) {
+                const int want = kb < nkb_pre ? 0 : 1;
+                if (want != seg) {  // this segment's per-column scales for my 2 x 8 features
+                    seg = want;
+                    const float* sv = args.wscale[seg == 0 ? args.num_experts : ti.expert];
+#pragma unroll
+                    for (int j = 0; j < 2; ++j) {
+                        const int col = ((MODE == MODE_GATEUP) ? (j == 0 ? acol0 : ti.up_off + acol0)
+                                                               : acol0 + 64 * j) + 8 * c8;
+                        const int mcol = (MODE == MODE_GATEUP) ? (j == 0 ? ti.M : ti.up_off + ti.M)
+                                                               : ti.M;  // columns of this weight
+#pragma unroll
+                        for (int i = 0; i < 8; ++i) sc[j][i] = (col + i < mcol) ? sv[col + i] : 0.f;
+                    }
+                }
+                const bool got = mbar_wait(rawfull_bar(stage), phase, args.err, DEV_ERR_TIMEOUT_PRODUCER);
+                if (!__all_sync(0xffffffffu, got)) {
+                    ok = false;
+                    break;
+                }
+                const uint8_t* sbp = smem + (size_t)stage * Cfg::STAGE_BYTES;
+                const uint8_t* raw = sbp + Cfg::A_BYTES + Cfg::B_BYTES;
+                uint8_t* a = const_cast<uint8_t*>(sbp);
+#pragma unroll
+                for (int i = 0; i < 8; ++i) {
+                    // unit u = ct + 128 i: slab u / 512 = i / 4 (ct < 128), K row (u / 8) % 64
+                    const int j = i >> 2, kr = ((ct >> 3) + 16 * i) & 63;
+                    const uint2 q8 = *reinterpret_cast<const uint2*>(raw + j * 4096 + kr * 64 + c8 * 8);
+                    *reinterpret_cast<uint4*>(a + j * 8192 + kr * 128 + ((c8 ^ (kr & 7)) << 4)) =
+                        e4m3x8_scaled_to_bf16(q8, sc[j]);
+                }
+                fence_proxy_async_smem();  // generic-proxy writes -> tensor-core reads
+                __syncwarp();
+                if (lane == 0) mbar_arrive_remote(mapa_shared(conv_bar(stage), 0));
+                if (++stage == Cfg::STAGES) {
+                    stage = 0;
+                    phase ^= 1u;
+                }
+            }
         }
     } else {
         // ---------------------------------------------------- epilogue

@@ -27,6 +27,11 @@ SMALL = {
     "bf16_T1": LayerConfig("bf16_T1", 1, 256, 8, 256, 256, "bf16", wr_std=0.1),
     "bf16_E1": LayerConfig("bf16_E1", 70, 128, 1, 128, 128, "bf16"),
     "bf16_E256": LayerConfig("bf16_E256", 600, 128, 256, 64, 64, "bf16", wr_std=0.1),
+    # E4M3 weights with per-output-column scales, bf16 activations
+    "fp8_ragged": LayerConfig("fp8_ragged", 300, 256, 8, 384, 256, "fp8", wr_std=0.1),
+    "fp8_zipf": LayerConfig("fp8_zipf", 700, 192, 16, 128, 320, "fp8", router="zipf", n_dead=4,
+                            wr_std=0.05),
+    "fp8_T1": LayerConfig("fp8_T1", 1, 256, 8, 256, 256, "fp8", wr_std=0.1),
 }
 
 
@@ -122,3 +127,7 @@ def test_full_size_maverick_prefill_zipf():
 @pytest.mark.parametrize("T", DECODE_TOKENS)
 def test_full_size_maverick_decode(T):
     _full_size(CONFIGS["maverick_decode_bf16"].with_tokens(T))
+
+
+def test_full_size_maverick_fp8_zipf():
+    _full_size(CONFIGS["maverick_fp8"])
