@@ -37,13 +37,13 @@
 // one tile overlaps the MMAs of the next.
 //
 // E4M3 weights (FP8W): TMA brings the raw 8-bit A tile (64 K rows x 2 slabs
-// of 64 features) into a raw ring; four converter warps widen it to bf16,
+// of 64 features) into a raw ring; eight converter warps widen it to bf16,
 // multiplying each value by its output column's fp32 scale (one bf16
 // rounding of q * scale), write the swizzled MN-major operand layout, fence
 // to the async proxy and report to the leader; the MMA waits for the token
 // tile and for both CTAs' converted weights.
 //
-// Roles (192 threads per CTA, 320 with E4M3 weights): warp 0 lane 0 issues TMA loads into a
+// Roles (192 threads per CTA, 448 with E4M3 weights): warp 0 lane 0 issues TMA loads into a
 // STAGES-deep ring (both CTAs; completion counted on the leader's barrier);
 // warp 1 allocates TMEM (both CTAs) and, in the leader CTA only, lane 0
 // issues the MMAs and commits to both CTAs' barriers; warps 2..5 are the
@@ -53,7 +53,6 @@
 // copies and MMAs in flight before the pair synchronises and frees TMEM.
 #pragma once
 #include <cuda_bf16.h>
-#include <cuda_fp8.h>
 #include <cstdint>
 
 #include "permute.cuh"
@@ -123,7 +122,8 @@ struct GemmCfg {
     static constexpr int STAGES = FP8W ? 5 : 6;
     static constexpr int ACC_BUFS = 2;
     static constexpr int TMEM_COLS = 512;
-    static constexpr int THREADS = FP8W ? 320 : 192;
+    static constexpr int CONV_WARPS = FP8W ? 8 : 0;         // E4M3 widening warps (6..13)
+    static constexpr int THREADS = 192 + 32 * CONV_WARPS;
     static constexpr int XLD = 17;                           // exchange row stride (floats)
     static constexpr int XCH_BYTES = (MODE == MODE_GATEUP) ? 2 * 2 * 32 * XLD * 4 : 0;
     static constexpr int NUM_BARS = 2 * STAGES + 2 * ACC_BUFS + 1 + (FP8W ? 2 * STAGES : 0);
@@ -166,20 +166,31 @@ __device__ __forceinline__ TileInfo decode_tile(const GroupTable& tab, const Gem
 __device__ __forceinline__ float silu_f(float z) { return __fdividef(z, 1.0f + __expf(-z)); }
 
 // 8 E4M3 codes (little-endian in a uint2) -> 8 bf16 values of code * scale.
+// Integer/FMA-pipe widening (the conversion pipe runs at a quarter of their
+// rate): a byte permute puts code i in bits 31..24; an arithmetic shift by 4
+// spreads its sign over bits 31..27 and the mask keeps the sign (bit 31) and
+// the 7 exponent/mantissa bits at 26..20.  Read as fp32 that is exactly
+// code * 2^-120 for every finite code, subnormals included (the E4M3 bias
+// is 7, fp32's 127); the product with 2^120 is exact, the product with the
+// scale is rounded once in fp32 and the pair is packed to bf16 (nearest even).
+__device__ __forceinline__ float e4m3_byte_to_f32(uint32_t w, uint32_t sel) {
+    const uint32_t t = __byte_perm(w, 0u, sel);  // code << 24
+    return __uint_as_float((uint32_t)((int32_t)t >> 4) & 0x87F00000u) * 0x1p120f;
+}
+
 __device__ __forceinline__ uint4 e4m3x8_scaled_to_bf16(uint2 raw, const float (&sc)[8]) {
     const uint32_t w[2] = {raw.x, raw.y};
     uint32_t o[4];
 #pragma unroll
     for (int h = 0; h < 2; ++h) {
-#pragma unroll
-        for (int p = 0; p < 2; ++p) {
-            const __nv_fp8x2_storage_t two = (__nv_fp8x2_storage_t)((w[h] >> (16 * p)) & 0xffffu);
-            const __half2_raw hr = __nv_cvt_fp8x2_to_halfraw2(two, __NV_E4M3);
-            const float2 f = __half22float2(*reinterpret_cast<const __half2*>(&hr));
-            const int i = 4 * h + 2 * p;
-            const __nv_bfloat162 b = __floats2bfloat162_rn(f.x * sc[i], f.y * sc[i + 1]);
-            o[2 * h + p] = *reinterpret_cast<const uint32_t*>(&b);
-        }
+        const float f0 = e4m3_byte_to_f32(w[h], 0x0444u) * sc[4 * h + 0];
+        const float f1 = e4m3_byte_to_f32(w[h], 0x1444u) * sc[4 * h + 1];
+        const float f2 = e4m3_byte_to_f32(w[h], 0x2444u) * sc[4 * h + 2];
+        const float f3 = e4m3_byte_to_f32(w[h], 0x3444u) * sc[4 * h + 3];
+        const __nv_bfloat162 b01 = __floats2bfloat162_rn(f0, f1);
+        const __nv_bfloat162 b23 = __floats2bfloat162_rn(f2, f3);
+        o[2 * h] = *reinterpret_cast<const uint32_t*>(&b01);
+        o[2 * h + 1] = *reinterpret_cast<const uint32_t*>(&b23);
     }
     return make_uint4(o[0], o[1], o[2], o[3]);
 }
@@ -241,7 +252,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(GemmCfg<MODE, ET, FP
         if constexpr (FP8W) {
             for (int s = 0; s < Cfg::STAGES; ++s) {
                 mbar_init(rawfull_bar(s), 1);
-                mbar_init(conv_bar(s), 8);  // leader: 4 converter warps of each CTA
+                mbar_init(conv_bar(s), 2 * Cfg::CONV_WARPS);  // leader: converter warps of both CTAs
             }
         }
         misc[1] = 0;
@@ -373,7 +384,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(GemmCfg<MODE, ET, FP
                         break;
                     }
                     if constexpr (FP8W) {
-                        if (!mbar_wait_cluster(conv_bar(stage), phase, args.err, DEV_ERR_TIMEOUT_MMA)) {
+                        if (!mbar_wait(conv_bar(stage), phase, args.err, DEV_ERR_TIMEOUT_MMA)) {
                             ok = false;
                             break;
                         }
@@ -411,8 +422,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(GemmCfg<MODE, ET, FP
         }
     } else if (FP8W && warp >= 6) {
         // ---------------------------------------------------- E4M3 converters
-        const int ct = threadIdx.x - 192;  // 0..127
-        const int c8 = ct & 7;             // 8-feature chunk of each slab this thread owns
+        constexpr int NCT = 32 * (Cfg::CONV_WARPS > 0 ? Cfg::CONV_WARPS : 8);  // converter threads
+        static_assert(NCT == 256, "each converter thread owns 4 units: slab i / 2");
+        const int ct = threadIdx.x - 192;           // 0 .. NCT-1
+        const int c8 = ct & 7;                      // 8-feature chunk of each slab this thread owns
         int stage = 0;
         uint32_t phase = 0;
         bool ok = true;
@@ -447,9 +460,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(GemmCfg<MODE, ET, FP
                 const uint8_t* raw = sbp + Cfg::A_BYTES + Cfg::B_BYTES;
                 uint8_t* a = const_cast<uint8_t*>(sbp);
 #pragma unroll
-                for (int i = 0; i < 8; ++i) {
-                    // unit u = ct + 128 i: slab u / 512 = i / 4 (ct < 128), K row (u / 8) % 64
-                    const int j = i >> 2, kr = ((ct >> 3) + 16 * i) & 63;
+                for (int i = 0; i < 1024 / NCT; ++i) {
+                    // unit u = ct + NCT i (of 2 slabs x 64 K rows x 8 chunks):
+                    // slab u / 512, K row (u / 8) % 64, chunk c8
+                    const int j = (i * NCT) >> 9, kr = ((ct >> 3) + (NCT / 8) * i) & 63;
                     const uint2 q8 = *reinterpret_cast<const uint2*>(raw + j * 4096 + kr * 64 + c8 * 8);
                     *reinterpret_cast<uint4*>(a + j * 8192 + kr * 128 + ((c8 ^ (kr & 7)) << 4)) =
                         e4m3x8_scaled_to_bf16(q8, sc[j]);
