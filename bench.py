@@ -79,7 +79,7 @@ class ClockSampler:
         try:
             self.proc = subprocess.Popen(
                 ["nvidia-smi", "-i", str(self.dev), f"--query-gpu={self.FIELDS}",
-                 "--format=csv,noheader,nounits", "-lms", "100"],
+                 "--format=csv,noheader,nounits", "-lms", "20"],
                 stdout=open(self.path, "w"), stderr=subprocess.DEVNULL)
         except (FileNotFoundError, OSError):
             self.proc = None
@@ -227,7 +227,7 @@ def config_dict(cfg, world):
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=50)
+    ap.add_argument("--steps", type=int, default=100)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--workload", default=DEFAULT_WORKLOAD, choices=sorted(CONFIGS))
     ap.add_argument("--tokens", type=int, default=0, help="override T (decode sweeps)")
@@ -310,7 +310,6 @@ def run_b200(args, rank, world, local):
     e1.record(stream)
     torch.cuda.synchronize()
     barrier()
-    clocks = sampler.stop()
     layer.set_timing(False)
     launches = layer.launch_count - launches0
     t_ms = max_over_ranks(e0.elapsed_time(e1))
@@ -334,16 +333,21 @@ def run_b200(args, rank, world, local):
     h0.record(stream)
     for _ in range(e2e_steps):
         fwd_h()
+    layer.join_host(stream)  # the end event waits for the last output copy
     h1.record(stream)
     torch.cuda.synchronize()
     barrier()
     th_ms = max_over_ranks(h0.elapsed_time(h1))
+    clocks = sampler.stop()  # samples span the device-timed and the end-to-end regions
     layer.check_device_status()
     io_bytes = cfg.T * cfg.d_model * inp.x.element_size()
     e2e = {"value": world * cfg.T * e2e_steps / (th_ms / 1e3), "unit": "tokens/s",
            "h2d_bytes_per_step": io_bytes, "d2h_bytes_per_step": io_bytes,
            "ms_per_step": th_ms / e2e_steps,
-           "path": "l4moe_forward_host: pinned host x -> device, layer, device -> pinned host out"}
+           "path": "l4moe_forward_host per step: pinned host x -> device (copy-in stream), layer "
+                   "(caller stream), device -> pinned host out (copy-out stream); consecutive "
+                   "steps overlap their copies with each other's compute; the timed region "
+                   "ends after the last output copy"}
 
     if rank != 0:
         if world > 1:

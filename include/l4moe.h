@@ -134,10 +134,14 @@ L4MOE_API l4moe_status l4moe_forward(l4moe_handle *h, int T, const void *x, cons
                            void *stream);
 
 /* As l4moe_forward, but x_host and out_host are HOST buffers (pinned memory
- * recommended): the call enqueues the host-to-device copy of x, the layer and
- * the device-to-host copy of out on `stream`, using staging buffers inside
- * the workspace.  Weights stay device pointers.  Asynchronous like
- * l4moe_forward: out_host is valid after the stream has been synchronised. */
+ * recommended).  The input copy runs on a copy-in stream of the handle into
+ * one of two staging slots of the workspace, the layer runs on `stream`, and
+ * the output copy runs on a copy-out stream; events order them, so the
+ * copies of consecutive calls overlap each other's layer computation.  Weights
+ * stay device pointers.  Asynchronous: x_host must not change and out_host is
+ * not complete until the call's output copy has finished -- make a stream
+ * wait for it with l4moe_join_host, or call l4moe_check_device_status (which
+ * synchronises).  The input copy does not wait for earlier work on `stream`. */
 L4MOE_API l4moe_status l4moe_forward_host(l4moe_handle *h, int T, const void *x_host, const void *W_router,
                                 const void *const *W_gate_up, const void *const *W_down,
                                 const void *Ws_gate_up, const void *Ws_down, void *out_host,
@@ -159,10 +163,11 @@ L4MOE_API l4moe_status l4moe_forward_host(l4moe_handle *h, int T, const void *x_
  * scratch array's device address (cudaGetSymbolAddress, with that device
  * current) and caches it; make that first call before any stream capture.
  * Fails with L4MOE_ERR_WORKSPACE, launching nothing, when T tokens of this
- * layer do not fit in the scratch area: it holds the workspace of
- * l4moe_workspace_size(h, T) bytes (rounded up to 256) plus 2(E+1) TMA
- * descriptors of 128 bytes, e.g. about 500 tokens at d_model 5120 and
- * F = Fs = 8192.  Every call, from any handle, shares the one array: calls
+ * layer do not fit in the scratch area: it holds the device part of the
+ * workspace (l4moe_workspace_size without the host-path staging slots,
+ * rounded up to 256 bytes) plus 2(E+1) TMA descriptors of 128 bytes, e.g.
+ * about 390 tokens at d_model 5120 and F = Fs = 8192.  Every call, from any
+ * handle, shares the one array: calls
  * whose work overlaps on the GPU (other streams, other threads) race and
  * corrupt each other; serialise them.  The array keeps the last call's
  * contents; the call clears the device error word itself.  Per-kernel
@@ -173,6 +178,10 @@ L4MOE_API l4moe_status l4moe_forward_static(l4moe_handle *h, int T, const void *
                                   const void *const *W_gate_up, const void *const *W_down,
                                   const void *Ws_gate_up, const void *Ws_down, void *out,
                                   void *stream);
+
+/* Make `stream` wait (on the device, no host sync) until the output copies of
+ * every l4moe_forward_host call enqueued so far have completed. */
+L4MOE_API l4moe_status l4moe_join_host(l4moe_handle *h, void *stream);
 
 /* Device pointers (inside the workspace) to the routing of the last forward
  * enqueued with this handle; valid once that work has run and until the next
@@ -185,9 +194,9 @@ L4MOE_API l4moe_status l4moe_get_routing(const l4moe_handle *h, const int32_t **
                                const float **lmax, const float **margin, const int32_t **counts,
                                const int32_t **offsets, const int32_t **perm);
 
-/* Synchronise `stream` and read the device error word of the handle's
- * workspace: L4MOE_OK, L4MOE_ERR_TIMEOUT (a bounded wait ran out) or
- * L4MOE_ERR_CUDA.  Clears the word. */
+/* Synchronise `stream` (and the handle's copy-out stream) and read the device
+ * error word of the handle's workspace: L4MOE_OK, L4MOE_ERR_TIMEOUT (a
+ * bounded wait ran out) or L4MOE_ERR_CUDA.  Clears the word. */
 L4MOE_API l4moe_status l4moe_check_device_status(l4moe_handle *h, void *stream);
 
 /* Per-kernel timing.  While enabled, l4moe_forward records a CUDA event

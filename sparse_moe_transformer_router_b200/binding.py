@@ -21,7 +21,7 @@ EXPORTED = ("l4moe_create", "l4moe_destroy", "l4moe_workspace_size", "l4moe_set_
             "l4moe_forward_host", "l4moe_get_routing", "l4moe_check_device_status",
             "l4moe_launch_count", "l4moe_last_error", "l4moe_status_string", "l4moe_version",
             "l4moe_set_timing", "l4moe_read_timing", "l4moe_kernel_name",
-            "l4moe_forward_static")
+            "l4moe_forward_static", "l4moe_join_host")
 STATIC_WORKSPACE_BYTES = 32 << 20
 NUM_KERNELS = 5
 
@@ -63,6 +63,7 @@ def load_library():
     lib.l4moe_forward.argtypes = fwd
     lib.l4moe_forward_host.argtypes = fwd
     lib.l4moe_forward_static.argtypes = fwd
+    lib.l4moe_join_host.argtypes = [vp, vp]
     lib.l4moe_get_routing.argtypes = [vp] + [pvp] * 7
     lib.l4moe_check_device_status.argtypes = [vp, vp]
     lib.l4moe_launch_count.argtypes = [vp]
@@ -80,7 +81,8 @@ def load_library():
     for name in ("l4moe_create", "l4moe_set_workspace", "l4moe_set_router_bias",
                  "l4moe_set_fp8_scales", "l4moe_forward", "l4moe_forward_host",
                  "l4moe_get_routing", "l4moe_check_device_status", "l4moe_version",
-                 "l4moe_set_timing", "l4moe_read_timing", "l4moe_forward_static"):
+                 "l4moe_set_timing", "l4moe_read_timing", "l4moe_forward_static",
+                 "l4moe_join_host"):
         getattr(lib, name).restype = ctypes.c_int
     _lib = lib
     return lib
@@ -206,6 +208,10 @@ class L4MoE:
                                                  _stream_handle(stream)))
         self.last_T = T
         return out_host
+
+    def join_host(self, stream=None):
+        """Make `stream` wait for the output copies of all forward_host calls."""
+        self._check(self._lib.l4moe_join_host(self._h, _stream_handle(stream)))
 
     def routing(self):
         """Zero-copy device views of the last forward's routing (valid until

@@ -60,15 +60,65 @@ bool encode_2d(CUtensorMap* m, CUtensorMapDataType dt, const void* base, uint64_
                CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+// Split-K is used for batches of at most this many tokens, into at most
+// kMaxSplit k-ranges (tiles too few to fill the GPU, e.g. decode).
+constexpr size_t kSplitMaxTokens = 64;
+constexpr int kMaxSplit = 8;
+// The expert-split router (one token tile) also splits K into this many slices.
+constexpr int kRouterKSplit = 8;
+
 struct WsLayout {
     size_t err, idx, gate, lmax, margin, inv, perm, gslot, counts, offsets, tab_gu, tab_dn, xg, hr,
-        hs, xin, xout, total;
+        hs, part, logits, xin, xout;
+    size_t device_total;  // everything l4moe_forward uses
+    size_t total;         // plus the host-path staging slots (last)
 };
 
 size_t act_bytes(l4moe_dtype dt) { return dt == L4MOE_F32 ? 4 : 2; }
 size_t w_bytes(l4moe_dtype dt) { return dt == L4MOE_F32 ? 4 : (dt == L4MOE_BF16 ? 2 : 1); }
 
-WsLayout ws_layout(const l4moe_params& p, int T) {
+// Split-K plan of one forward of T tokens: how many k-ranges the gate/up and
+// the down launches use.  Only batches of at most kSplitMaxTokens split; the
+// aim is about four waves of CTA pairs with at least 8 k-blocks per range.
+struct SplitPlan {
+    int s_gu, s_dn;
+};
+
+SplitPlan split_plan(const l4moe_params& p, int T, int sms) {
+    const int d = p.d_model, F = p.expert_ffn, Fs = p.shared_ffn, E = p.num_experts;
+    const int kblk = (int)(128 / act_bytes(p.dtype));  // K elements per k-block
+    const int fb_gu_r = (F + 127) / 128, fb_gu_s = (Fs + 127) / 128, fb_dn = (d + 255) / 256;
+    auto pick = [&](long long tiles, int nkb) {
+        if ((size_t)T > kSplitMaxTokens || tiles <= 0) return 1;
+        const long long want = 4LL * (sms / 2);
+        long long sp = (want + tiles - 1) / tiles;
+        sp = std::min<long long>(sp, kMaxSplit);
+        sp = std::min<long long>(sp, std::max(1, nkb / 8));
+        return (int)std::max(1LL, sp);
+    };
+    const long long eg = std::min(E, T);  // non-empty routed experts (one token tile each)
+    SplitPlan sp;
+    sp.s_gu = pick((long long)fb_gu_s + fb_gu_r * eg, d / kblk);
+    sp.s_dn = pick((long long)fb_dn * (eg + 1), std::min(F, Fs) / kblk);
+    return sp;
+}
+
+// fp32 partial floats any forward of at most T tokens needs: split gate/up
+// results, and the down's shared + routed results (times its splits).
+size_t part_floats(const l4moe_params& p, int T, int sms) {
+    size_t need = 0;
+    auto add = [&](int t) {
+        const SplitPlan sp = split_plan(p, t, sms);
+        if (sp.s_gu > 1)
+            need = std::max<size_t>(need, (size_t)sp.s_gu * t * (2ull * p.expert_ffn + 2ull * p.shared_ffn));
+        need = std::max<size_t>(need, 2ull * sp.s_dn * t * p.d_model);
+    };
+    for (int t = 1; t <= std::min<int>(T, (int)kSplitMaxTokens); ++t) add(t);
+    add(std::max(T, 1));
+    return need;
+}
+
+WsLayout ws_layout(const l4moe_params& p, int T, int sms) {
     WsLayout L{};
     size_t off = 0;
     auto take = [&](size_t bytes) {
@@ -92,8 +142,11 @@ WsLayout ws_layout(const l4moe_params& p, int T) {
     L.xg = take(t * p.d_model * es);
     L.hr = take(t * p.expert_ffn * es);
     L.hs = take(t * p.shared_ffn * es);
-    L.xin = take(t * p.d_model * es);
-    L.xout = take(t * p.d_model * es);
+    L.part = take(sizeof(float) * part_floats(p, (int)t, sms));
+    L.logits = take(sizeof(float) * kRouterKSplit * std::min<size_t>(t, 128) * E);  // split router
+    L.device_total = off;
+    L.xin = take(2 * t * p.d_model * es);   // host path: two input staging slots
+    L.xout = take(2 * t * p.d_model * es);  // and two output staging slots
     L.total = off;
     return L;
 }
@@ -128,6 +181,12 @@ struct l4moe_handle {
     uint64_t launches = 0;
     std::string err;
     int last_T = 0;
+    // host path (l4moe_forward_host): copy streams and per-slot events so
+    // consecutive calls overlap their copies with each other's compute
+    cudaStream_t s_in = nullptr, s_out = nullptr;
+    cudaEvent_t ev_h2d[2] = {}, ev_comp[2] = {}, ev_d2h[2] = {};
+    bool slot_used[2] = {false, false};
+    int host_slot = 0;
     // per-kernel event timing (l4moe_set_timing)
     bool timing = false;
     std::vector<cudaEvent_t> ev_pool;             // recycled events
@@ -185,7 +244,7 @@ l4moe_status ensure_workspace(l4moe_handle* h, int T) {
         h->ws = nullptr;
     }
     const int cap = std::max(T, 256);
-    const WsLayout L = ws_layout(h->p, cap);
+    const WsLayout L = ws_layout(h->p, cap, h->sms);
     void* p = nullptr;
     cudaError_t e = cudaMalloc(&p, L.total);
     if (e != cudaSuccess) return cuda_fail(h, e, "workspace cudaMalloc");
@@ -314,7 +373,7 @@ l4moe_status run_layer(l4moe_handle* h, int T, const void* x, const void* Wr, co
                        const CUtensorMap* maps) {
     const l4moe_params& p = h->p;
     const int d = p.d_model, F = p.expert_ffn, Fs = p.shared_ffn, E = p.num_experts;
-    const WsLayout L = ws_layout(p, ws_tokens);
+    const WsLayout L = ws_layout(p, ws_tokens, h->sms);
     unsigned* err = reinterpret_cast<unsigned*>(w + L.err);
     int32_t* idx = reinterpret_cast<int32_t*>(w + L.idx);
     float* gate = reinterpret_cast<float*>(w + L.gate);
@@ -350,6 +409,10 @@ l4moe_status run_layer(l4moe_handle* h, int T, const void* x, const void* Wr, co
     } while (0)
 
     LaunchTimer t_router(h, 0, st);
+    // one token tile and many experts: split the router over 16-expert chunks
+    const bool split_router = sizeof(ET) == 2 && E % 16 == 0 && E >= 32 && T <= 128;
+    float* logits = split_router ? reinterpret_cast<float*>(w + L.logits) : nullptr;
+    int router_logit_splits = 1;
     if (sizeof(ET) == 2 && E % 8 == 0) {
         // tensor-core router: W_router [d, E] as the MN-major operand
         CUtensorMap m_wr;
@@ -357,8 +420,11 @@ l4moe_status run_layer(l4moe_handle* h, int T, const void* x, const void* Wr, co
             return fail(h, L4MOE_ERR_CUDA, "cuTensorMapEncodeTiled failed for the router weight");
         static std::once_flag once;
         std::call_once(once, [] { set_smem_attr(router_mma_kernel, rmma::SMEM_BYTES); });
-        router_mma_kernel<<<(T + 127) / 128, 128, rmma::SMEM_BYTES, st>>>(
-            m_x, m_wr, h->bias, T, d, E, idx, gate, lmax, margin, err);
+        const int n_chunk = split_router ? 16 : E;
+        const int kslices = split_router ? std::min(kRouterKSplit, std::max(1, d / 256)) : 1;
+        router_logit_splits = kslices;
+        router_mma_kernel<<<dim3((T + 127) / 128, E / n_chunk, kslices), 128, rmma::SMEM_BYTES, st>>>(
+            m_x, m_wr, h->bias, T, d, E, n_chunk, logits, idx, gate, lmax, margin, err);
     } else {
         launch_router<ET>(x, Wr, h->bias, T, d, E, idx, gate, lmax, margin, st);
     }
@@ -370,10 +436,14 @@ l4moe_status run_layer(l4moe_handle* h, int T, const void* x, const void* Wr, co
     const int fb_gu_r = (F + fpg - 1) / fpg;
     const int fb_gu_s = (Fs + fpg - 1) / fpg;
     const int fb_dn = (d + fpd - 1) / fpd;
+    // split-K k-ranges when a small batch leaves too few tiles
+    const SplitPlan plan = split_plan(p, T, h->sms);
+    const int s_gu = plan.s_gu, s_dn = plan.s_dn;
     const size_t psmem = sizeof(int) * (34 * (size_t)E + 1);
     LaunchTimer t_perm(h, 1, st);
-    permute_kernel<<<1, 1024, psmem, st>>>(idx, T, E, fb_gu_r, fb_gu_s, fb_dn, counts, offsets,
-                                           perm, inv, tab_gu, tab_dn, err);
+    permute_kernel<<<1, 1024, psmem, st>>>(logits, router_logit_splits, gate, lmax, margin, idx, T, E,
+                                           fb_gu_r * s_gu, fb_gu_s * s_gu, fb_dn * s_dn, counts,
+                                           offsets, perm, inv, tab_gu, tab_dn, err);
     t_perm.stop();
     L4MOE_CHECK_LAUNCH("permute launch");
 
@@ -396,7 +466,6 @@ l4moe_status run_layer(l4moe_handle* h, int T, const void* x, const void* Wr, co
     gu.num_experts = E;
     gu.k_routed = d;
     gu.k_shared = d;
-    gu.k_pre = 0;
     gu.m_routed = F;
     gu.m_shared = Fs;
     gu.up_routed = F;
@@ -409,11 +478,27 @@ l4moe_status run_layer(l4moe_handle* h, int T, const void* x, const void* Wr, co
     gu.rowmap_shared = inv;
     gu.colscale_routed = gslot;  // sigmoid gate of each routed slot
     gu.wscale = FP8W ? h->d_scales : nullptr;
+    float* part = reinterpret_cast<float*>(w + L.part);
+    gu.ksplit = s_gu;
+    gu.partial_out = s_gu > 1 ? 1 : 0;
+    gu.part_routed = part;
+    gu.ld_part_routed = 2LL * F;
+    gu.part_stride_routed = (long long)T * 2 * F;
+    gu.part_shared = part + (size_t)s_gu * T * 2 * F;
+    gu.ld_part_shared = 2LL * Fs;
+    gu.part_stride_shared = (long long)T * 2 * Fs;
     gu.err = err;
     LaunchTimer t_gu(h, 3, st);
     launch_gemm<MODE_GATEUP, ET, FP8W>(
-        grid_for((long long)fb_gu_s * tb + (long long)fb_gu_r * (tb + std::min(E, T))), m_xg, m_x,
-        gu, st);
+        grid_for(s_gu * ((long long)fb_gu_s * tb + (long long)fb_gu_r * (tb + std::min(E, T)))),
+        m_xg, m_x, gu, st);
+    if (s_gu > 1) {
+        const long long n = (long long)T * (F + Fs);
+        gateup_finish_kernel<ET><<<(int)std::min<long long>((n + 255) / 256, 4LL * h->sms), 256, 0, st>>>(
+            gu.part_routed, gu.ld_part_routed, gu.part_stride_routed, gu.part_shared, gu.ld_part_shared,
+            gu.part_stride_shared, s_gu, T, F, Fs, gslot, hr, hs);
+        ++h->launches;
+    }
     t_gu.stop();
     L4MOE_CHECK_LAUNCH("gate/up launch");
 
@@ -422,8 +507,7 @@ l4moe_status run_layer(l4moe_handle* h, int T, const void* x, const void* Wr, co
     dn.a_maps = maps + (E + 1);
     dn.num_experts = E;
     dn.k_routed = F;
-    dn.k_shared = 0;
-    dn.k_pre = Fs;               // shared expert's down contraction first
+    dn.k_shared = Fs;
     dn.m_routed = d;
     dn.m_shared = d;
     dn.out_routed = out;
@@ -431,12 +515,28 @@ l4moe_status run_layer(l4moe_handle* h, int T, const void* x, const void* Wr, co
     dn.out_shared = out;
     dn.ld_shared = d;
     dn.rowmap_routed = perm;     // slot -> token: un-permute on store
-    dn.rowmap_shared = nullptr;
+    dn.rowmap_shared = perm;     // the shared rows are slots too (H_s in slot order)
     dn.colscale_routed = nullptr;
     dn.wscale = FP8W ? h->d_scales + (E + 1) : nullptr;
+    dn.ksplit = s_dn;
+    dn.partial_out = 1;
+    // partial slots: [0, s_dn) routed, [s_dn, 2 s_dn) shared
+    dn.part_routed = part;
+    dn.ld_part_routed = d;
+    dn.part_stride_routed = (long long)T * d;
+    dn.part_shared = part + (size_t)s_dn * T * d;
+    dn.ld_part_shared = d;
+    dn.part_stride_shared = (long long)T * d;
     dn.err = err;
     LaunchTimer t_dn(h, 4, st);
-    launch_gemm<MODE_DOWN, ET, FP8W>(grid_for((long long)fb_dn * (tb + std::min(E, T))), m_hr, m_hs, dn, st);
+    launch_gemm<MODE_DOWN, ET, FP8W>(grid_for(s_dn * (long long)fb_dn * (2 * tb + std::min(E, T))),
+                                     m_hr, m_hs, dn, st);
+    {
+        const long long n = (long long)T * d;
+        down_finish_kernel<ET><<<(int)std::min<long long>((n / 4 + 255) / 256, 4LL * h->sms), 256, 0, st>>>(
+            part, dn.part_stride_routed, 2 * s_dn, n, static_cast<ET*>(out));
+        ++h->launches;
+    }
     t_dn.stop();
     L4MOE_CHECK_LAUNCH("down launch");
 #undef L4MOE_CHECK_LAUNCH
@@ -549,7 +649,7 @@ l4moe_status l4moe_forward_static(l4moe_handle* h, int T, const void* x, const v
     if (h->p.dtype != L4MOE_F32 && h->p.dtype != L4MOE_BF16)
         return fail(h, L4MOE_ERR_UNSUPPORTED, "FP8 weight path not built in this library");
     const int E = h->p.num_experts;
-    const size_t ws_bytes = (ws_layout(h->p, T).total + 255) & ~size_t(255);
+    const size_t ws_bytes = (ws_layout(h->p, T, h->sms).device_total + 255) & ~size_t(255);
     const size_t maps_bytes = sizeof(CUtensorMap) * 2 * (E + 1);
     if (ws_bytes + maps_bytes > L4MOE_STATIC_WORKSPACE_BYTES) {
         char msg[200];
@@ -567,7 +667,7 @@ l4moe_status l4moe_forward_static(l4moe_handle* h, int T, const void* x, const v
     // the error word (the only state a forward expects to start at zero)
     cudaError_t e = cudaMemcpyAsync(maps, h->h_maps.data(), maps_bytes, cudaMemcpyHostToDevice, st);
     if (e != cudaSuccess) return cuda_fail(h, e, "static descriptor upload");
-    e = cudaMemsetAsync(base + ws_layout(h->p, T).err, 0, sizeof(unsigned), st);
+    e = cudaMemsetAsync(base + ws_layout(h->p, T, h->sms).err, 0, sizeof(unsigned), st);
     if (e != cudaSuccess) return cuda_fail(h, e, "static error word clear");
     const bool timing = h->timing;  // event timing would create events: off here
     h->timing = false;
@@ -627,6 +727,13 @@ l4moe_status l4moe_create(const l4moe_params* params, l4moe_handle** out) {
 void l4moe_destroy(l4moe_handle* h) {
     if (!h) return;
     for (cudaEvent_t e : h->ev_pool) cudaEventDestroy(e);
+    for (int b = 0; b < 2; ++b) {
+        if (h->ev_h2d[b]) cudaEventDestroy(h->ev_h2d[b]);
+        if (h->ev_comp[b]) cudaEventDestroy(h->ev_comp[b]);
+        if (h->ev_d2h[b]) cudaEventDestroy(h->ev_d2h[b]);
+    }
+    if (h->s_in) cudaStreamDestroy(h->s_in);
+    if (h->s_out) cudaStreamDestroy(h->s_out);
     for (auto& p : h->ev_pending) {
         cudaEventDestroy(p.second.first);
         cudaEventDestroy(p.second.second);
@@ -639,7 +746,7 @@ void l4moe_destroy(l4moe_handle* h) {
 
 size_t l4moe_workspace_size(const l4moe_handle* h, int max_tokens) {
     if (!h || max_tokens < 0) return 0;
-    return ws_layout(h->p, max_tokens).total;
+    return ws_layout(h->p, max_tokens, h->sms).total;
 }
 
 l4moe_status l4moe_set_workspace(l4moe_handle* h, void* dev_ptr, size_t bytes, int max_tokens) {
@@ -647,7 +754,7 @@ l4moe_status l4moe_set_workspace(l4moe_handle* h, void* dev_ptr, size_t bytes, i
     if (!dev_ptr || max_tokens < 1) return fail(h, L4MOE_ERR_ARG, "null workspace or max_tokens < 1");
     if (reinterpret_cast<uintptr_t>(dev_ptr) & 255u)
         return fail(h, L4MOE_ERR_ALIGN, "workspace must be 256-byte aligned");
-    if (bytes < ws_layout(h->p, max_tokens).total)
+    if (bytes < ws_layout(h->p, max_tokens, h->sms).total)
         return fail(h, L4MOE_ERR_WORKSPACE, "workspace smaller than l4moe_workspace_size");
     if (h->ws_owned && h->ws) cudaFree(h->ws);
     h->ws = static_cast<uint8_t*>(dev_ptr);
@@ -701,17 +808,57 @@ l4moe_status l4moe_forward_host(l4moe_handle* h, int T, const void* x_host, cons
         check_forward_args(h, T, x_host, W_router, W_gate_up, W_down, Ws_gate_up, Ws_down, out_host);
     if (s != L4MOE_OK || T == 0) return s;
     if ((s = ensure_workspace(h, T)) != L4MOE_OK) return s;
+    cudaError_t e;
+    if (!h->s_in) {
+        if ((e = cudaStreamCreateWithFlags(&h->s_in, cudaStreamNonBlocking)) != cudaSuccess ||
+            (e = cudaStreamCreateWithFlags(&h->s_out, cudaStreamNonBlocking)) != cudaSuccess)
+            return cuda_fail(h, e, "copy stream creation");
+        for (int b = 0; b < 2; ++b)
+            if ((e = cudaEventCreateWithFlags(&h->ev_h2d[b], cudaEventDisableTiming)) != cudaSuccess ||
+                (e = cudaEventCreateWithFlags(&h->ev_comp[b], cudaEventDisableTiming)) != cudaSuccess ||
+                (e = cudaEventCreateWithFlags(&h->ev_d2h[b], cudaEventDisableTiming)) != cudaSuccess)
+                return cuda_fail(h, e, "copy event creation");
+    }
     cudaStream_t st = static_cast<cudaStream_t>(stream);
-    const WsLayout L = ws_layout(h->p, h->ws_tokens);
-    void* xin = h->ws + L.xin;
-    void* xout = h->ws + L.xout;
+    const WsLayout L = ws_layout(h->p, h->ws_tokens, h->sms);
+    const size_t slab = (size_t)h->ws_tokens * h->p.d_model * act_bytes(h->p.dtype);
+    const int b = h->host_slot;
+    h->host_slot ^= 1;
+    void* xin = h->ws + L.xin + b * slab;
+    void* xout = h->ws + L.xout + b * slab;
     const size_t bytes = (size_t)T * h->p.d_model * act_bytes(h->p.dtype);
-    cudaError_t e = cudaMemcpyAsync(xin, x_host, bytes, cudaMemcpyHostToDevice, st);
-    if (e != cudaSuccess) return cuda_fail(h, e, "input host-to-device copy");
+    // input copy on the copy-in stream, once the compute that last read this slot is done
+    if (h->slot_used[b] && (e = cudaStreamWaitEvent(h->s_in, h->ev_comp[b], 0)) != cudaSuccess)
+        return cuda_fail(h, e, "copy-in wait");
+    if ((e = cudaMemcpyAsync(xin, x_host, bytes, cudaMemcpyHostToDevice, h->s_in)) != cudaSuccess)
+        return cuda_fail(h, e, "input host-to-device copy");
+    if ((e = cudaEventRecord(h->ev_h2d[b], h->s_in)) != cudaSuccess) return cuda_fail(h, e, "event record");
+    // the layer on the caller's stream: after this input, and after the
+    // output copy that last read this slot's output buffer
+    if ((e = cudaStreamWaitEvent(st, h->ev_h2d[b], 0)) != cudaSuccess) return cuda_fail(h, e, "compute wait");
+    if (h->slot_used[b] && (e = cudaStreamWaitEvent(st, h->ev_d2h[b], 0)) != cudaSuccess)
+        return cuda_fail(h, e, "compute wait");
     if ((s = forward_impl(h, T, xin, W_router, W_gate_up, W_down, Ws_gate_up, Ws_down, xout, st)) != L4MOE_OK)
         return s;
-    e = cudaMemcpyAsync(out_host, xout, bytes, cudaMemcpyDeviceToHost, st);
-    if (e != cudaSuccess) return cuda_fail(h, e, "output device-to-host copy");
+    if ((e = cudaEventRecord(h->ev_comp[b], st)) != cudaSuccess) return cuda_fail(h, e, "event record");
+    // output copy on the copy-out stream
+    if ((e = cudaStreamWaitEvent(h->s_out, h->ev_comp[b], 0)) != cudaSuccess)
+        return cuda_fail(h, e, "copy-out wait");
+    if ((e = cudaMemcpyAsync(out_host, xout, bytes, cudaMemcpyDeviceToHost, h->s_out)) != cudaSuccess)
+        return cuda_fail(h, e, "output device-to-host copy");
+    if ((e = cudaEventRecord(h->ev_d2h[b], h->s_out)) != cudaSuccess) return cuda_fail(h, e, "event record");
+    h->slot_used[b] = true;
+    return L4MOE_OK;
+}
+
+l4moe_status l4moe_join_host(l4moe_handle* h, void* stream) {
+    if (!h) return L4MOE_ERR_ARG;
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    for (int b = 0; b < 2; ++b)
+        if (h->slot_used[b]) {
+            cudaError_t e = cudaStreamWaitEvent(st, h->ev_d2h[b], 0);
+            if (e != cudaSuccess) return cuda_fail(h, e, "join wait");
+        }
     return L4MOE_OK;
 }
 
@@ -719,7 +866,7 @@ l4moe_status l4moe_get_routing(const l4moe_handle* h, const int32_t** idx, const
                                const float** lmax, const float** margin, const int32_t** counts,
                                const int32_t** offsets, const int32_t** perm) {
     if (!h || !h->ws) return L4MOE_ERR_ARG;
-    const WsLayout L = ws_layout(h->p, h->ws_tokens);
+    const WsLayout L = ws_layout(h->p, h->ws_tokens, h->sms);
     if (idx) *idx = reinterpret_cast<const int32_t*>(h->ws + L.idx);
     if (gate) *gate = reinterpret_cast<const float*>(h->ws + L.gate);
     if (lmax) *lmax = reinterpret_cast<const float*>(h->ws + L.lmax);
@@ -734,13 +881,14 @@ l4moe_status l4moe_check_device_status(l4moe_handle* h, void* stream) {
     if (!h) return L4MOE_ERR_ARG;
     cudaStream_t st = static_cast<cudaStream_t>(stream);
     cudaError_t e = cudaStreamSynchronize(st);
+    if (e == cudaSuccess && h->s_out) e = cudaStreamSynchronize(h->s_out);
     if (e != cudaSuccess) return cuda_fail(h, e, "stream synchronize");
     if (!h->ws) return L4MOE_OK;
     unsigned word = 0;
-    e = cudaMemcpy(&word, h->ws + ws_layout(h->p, h->ws_tokens).err, sizeof(word), cudaMemcpyDeviceToHost);
+    e = cudaMemcpy(&word, h->ws + ws_layout(h->p, h->ws_tokens, h->sms).err, sizeof(word), cudaMemcpyDeviceToHost);
     if (e != cudaSuccess) return cuda_fail(h, e, "error word read");
     if (word == 0) return L4MOE_OK;
-    cudaMemset(h->ws + ws_layout(h->p, h->ws_tokens).err, 0, sizeof(word));
+    cudaMemset(h->ws + ws_layout(h->p, h->ws_tokens, h->sms).err, 0, sizeof(word));
     char msg[160];
     snprintf(msg, sizeof msg, "device error word 0x%x (1: producer wait, 2: MMA wait, 4: epilogue wait, 8: bad expert index)", word);
     return fail(h, (word & 7u) ? L4MOE_ERR_TIMEOUT : L4MOE_ERR_ARG, msg);

@@ -7,9 +7,10 @@
 //              expert (x rows in expert order, g = the token's sigmoid gate,
 //              applied to the fp32 accumulator: the gate scales the input
 //              and the contraction is linear in it) in one launch
-//   down     : out[token] = h_shared . Ws_down + h_routed . W_down[e], both
-//              contractions accumulated into one TMEM tile (a shared K segment
-//              then the routed one), so the sum is rounded once
+//   down     : y = h . W_down for the shared expert (all tokens) and every
+//              routed expert in one launch; each tile stores its fp32 result
+//              un-permuted to the token's row of a partial buffer, and a
+//              finish kernel writes out = rn(y_shared + y_routed), one rounding
 //
 // llm-architectures-explained "Llama 4 Maverick", field table rows
 // ffns.moe.gated / d_expert / d_shared: every expert and the shared expert is
@@ -87,19 +88,29 @@ struct GemmArgs {
     const GroupTable* table;
     const CUtensorMap* a_maps;  // weights, [E + 1]: routed experts then the shared expert
     int num_experts;            // E (expert index E = shared)
-    int k_routed, k_shared;     // main K segment per class (gate/up: d, d; down: F)
-    int k_pre;                  // down: leading K segment over the shared expert (Fs), else 0
+    int k_routed, k_shared;     // reduction length per class (gate/up: d, d; down: F, Fs)
     int m_routed, m_shared;     // output features per class (F / Fs, or d)
     int up_routed, up_shared;   // gate/up: column offset of the "up" half (F / Fs)
     void* out_routed;
     long long ld_routed;
     void* out_shared;
     long long ld_shared;
-    const int32_t* rowmap_routed;  // down: output row of a slot (perm), else null
-    const int32_t* rowmap_shared;  // gate/up: slot of a token (inv), else null
+    const int32_t* rowmap_routed;  // down: output row (token) of a slot (perm), else null
+    const int32_t* rowmap_shared;  // gate/up: slot of a token (inv); down: perm
     const float* colscale_routed;  // gate/up: sigmoid gate of each slot, else null
     const float* const* wscale;    // E4M3 weights: per-column scale vector of each of the
                                    // E + 1 weight matrices of this launch, else null
+    // fp32 partial output (always for down; for gate/up when split): each
+    // tile covers k-block range s of ksplit (split-K when tiles are few, e.g.
+    // decode) and stores its fp32 result; a finish kernel sums the partials
+    int ksplit;                    // 1 = no split
+    int partial_out;               // store fp32 partials instead of the epilogue's output
+    float* part_routed;            // [ksplit][rows][ld_part_routed] fp32, or null
+    long long ld_part_routed;
+    float* part_shared;            // gate/up only: shared expert partials
+    long long ld_part_shared;
+    long long part_stride_routed;  // elements between splits
+    long long part_stride_shared;
     unsigned* err;
 };
 
@@ -132,11 +143,12 @@ struct GemmCfg {
 };
 
 struct TileInfo {
-    int expert, row0, n_valid, n_mma, f0, K, k_pre, M, up_off;
+    int expert, row0, n_valid, n_mma, f0, K, M, up_off;
+    int split, kb0, kb1;  // k-block range [kb0, kb1) of this tile's split
     bool shared;
 };
 
-template <int MODE>
+template <int MODE, int ElemCfgBK>
 __device__ __forceinline__ TileInfo decode_tile(const GroupTable& tab, const GemmArgs& a, int L) {
     int lo = 0, hi = tab.num_groups - 1;
     while (lo < hi) {
@@ -148,18 +160,23 @@ __device__ __forceinline__ TileInfo decode_tile(const GroupTable& tab, const Gem
     const int rows = tab.rows[g];
     const int ntb = (rows + kTokTile - 1) / kTokTile;
     const int tb = local % ntb;
-    const int fb = local / ntb;
+    const int rest = local / ntb;
+    const int split = rest % a.ksplit;
+    const int fb = rest / a.ksplit;
     TileInfo ti;
+    ti.split = split;
     ti.expert = tab.expert[g];
     ti.shared = (ti.expert == a.num_experts);
     ti.row0 = tab.row0[g] + tb * kTokTile;
     ti.n_valid = min(kTokTile, rows - tb * kTokTile);
     ti.n_mma = (ti.n_valid + 15) & ~15;
     ti.f0 = fb * pair_features<MODE>();
-    ti.k_pre = ti.shared ? 0 : a.k_pre;
-    ti.K = ti.k_pre + (ti.shared ? a.k_shared : a.k_routed);
+    ti.K = ti.shared ? a.k_shared : a.k_routed;
     ti.M = ti.shared ? a.m_shared : a.m_routed;
     ti.up_off = ti.shared ? a.up_shared : a.up_routed;
+    const int nkb = ti.K / ElemCfgBK;
+    ti.kb0 = (int)(((long long)nkb * split) / a.ksplit);
+    ti.kb1 = (int)(((long long)nkb * (split + 1)) / a.ksplit);
     return ti;
 }
 
@@ -283,12 +300,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(GemmCfg<MODE, ET, FP
             uint32_t used = 0, last_par = 0;  // per stage: issued at least once / its parity
             bool aborted = false;
             for (int L = pair; L < total && !aborted; L += npairs) {
-                const TileInfo ti = decode_tile<MODE>(*tab, args, L);
-                const CUtensorMap* amap_main = args.a_maps + ti.expert;
-                const CUtensorMap* amap_pre = args.a_maps + args.num_experts;
-                const void* bmap_main = ti.shared ? (const void*)&b_shared : (const void*)&b_routed;
-                const int nkb = ti.K / C::BK;
-                const int nkb_pre = ti.k_pre / C::BK;
+                const TileInfo ti = decode_tile<MODE, C::BK>(*tab, args, L);
+                const CUtensorMap* amap = args.a_maps + ti.expert;
+                const void* bmap = ti.shared ? (const void*)&b_shared : (const void*)&b_routed;
                 const int half = ti.n_mma >> 1;  // tokens per CTA
                 const int nbb = (half + Cfg::B_BOX_ROWS - 1) / Cfg::B_BOX_ROWS;
                 const uint32_t tx_cta = (FP8W ? 0u : (uint32_t)Cfg::A_BYTES) + (uint32_t)nbb * Cfg::B_BOX_BYTES;
@@ -297,7 +311,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(GemmCfg<MODE, ET, FP
                 // f0 + 64*rank; down -> 128 features f0 + 128*rank
                 const int acol0 =
                     (MODE == MODE_GATEUP) ? ti.f0 + 64 * (int)rank : ti.f0 + 128 * (int)rank;
-                for (int kb = 0; kb < nkb; ++kb) {
+                for (int kb = ti.kb0; kb < ti.kb1; ++kb) {
                     if (!mbar_wait(empty_bar(stage), phase ^ 1u, args.err, DEV_ERR_TIMEOUT_PRODUCER)) {
                         aborted = true;
                         break;
@@ -306,11 +320,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(GemmCfg<MODE, ET, FP
                     const uint32_t fb_leader = mapa_shared(fb_local, 0);
                     if (leader) mbar_arrive_expect_tx(fb_local, 2 * tx_cta);
                     const uint32_t sb = stage0 + (uint32_t)stage * Cfg::STAGE_BYTES;
-                    // leading shared-expert segment (down only), then the tile's own weights
-                    const bool pre = kb < nkb_pre;
-                    const CUtensorMap* amap = pre ? amap_pre : amap_main;
-                    const void* bmap = pre ? (const void*)&b_shared : bmap_main;
-                    const int k = (pre ? kb : kb - nkb_pre) * C::BK;
+                    const int k = kb * C::BK;
                     if constexpr (FP8W) {
                         // raw 8-bit weights: two 64-feature slabs, signalled locally
                         const uint32_t rb = sb + Cfg::A_BYTES + Cfg::B_BYTES;
@@ -370,15 +380,14 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(GemmCfg<MODE, ET, FP
             int acc = 0;
             uint32_t acc_phase = 0;
             for (int L = pair; L < total; L += npairs) {
-                const TileInfo ti = decode_tile<MODE>(*tab, args, L);
+                const TileInfo ti = decode_tile<MODE, C::BK>(*tab, args, L);
                 if (!mbar_wait_cluster(tempty_bar(acc), acc_phase ^ 1u, args.err, DEV_ERR_TIMEOUT_MMA))
                     break;
                 tc_fence_after();
                 const uint32_t idesc = make_idesc(C::FMT, 1u, 0u, (uint32_t)ti.n_mma, 256u);
                 const uint32_t d_tmem = tmem_base + (uint32_t)acc * 256u;
-                const int nkb = ti.K / C::BK;
                 bool ok = true;
-                for (int kb = 0; kb < nkb; ++kb) {
+                for (int kb = ti.kb0; kb < ti.kb1; ++kb) {
                     if (!mbar_wait(full_bar(stage), phase, args.err, DEV_ERR_TIMEOUT_MMA)) {
                         ok = false;
                         break;
@@ -397,7 +406,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(GemmCfg<MODE, ET, FP
                         const uint64_t bdesc = smem_desc(bb + kk * 32, 16, 1024, 2);
                         const uint64_t adesc = smem_desc(sb + kk * C::MMA_K * 128, Cfg::A_BOX_BYTES,
                                                          C::A_SBO, C::A_LAYOUT);
-                        const uint32_t accum = (kb | kk) != 0 ? 1u : 0u;
+                        const uint32_t accum = (kb != ti.kb0 || kk != 0) ? 1u : 0u;
                         if constexpr (C::FMT == 1)
                             mma_bf16_pair(d_tmem, adesc, bdesc, idesc, accum);
                         else
@@ -430,27 +439,23 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(GemmCfg<MODE, ET, FP
         uint32_t phase = 0;
         bool ok = true;
         for (int L = pair; L < total && ok; L += npairs) {
-            const TileInfo ti = decode_tile<MODE>(*tab, args, L);
-            const int nkb = ti.K / C::BK;
-            const int nkb_pre = ti.k_pre / C::BK;
+            const TileInfo ti = decode_tile<MODE, C::BK>(*tab, args, L);
             const int acol0 = (MODE == MODE_GATEUP) ? ti.f0 + 64 * (int)rank : ti.f0 + 128 * (int)rank;
+            // this tile's per-column scales for my 2 x 8 features
             float sc[2][8];
-            int seg = -1;
-            for (int kb = 0; kb < nkb; ++kb) {
-                const int want = kb < nkb_pre ? 0 : 1;
-                if (want != seg) {  // this segment's per-column scales for my 2 x 8 features
-                    seg = want;
-                    const float* sv = args.wscale[seg == 0 ? args.num_experts : ti.expert];
+            {
+                const float* sv = args.wscale[ti.expert];
 #pragma unroll
-                    for (int j = 0; j < 2; ++j) {
-                        const int col = ((MODE == MODE_GATEUP) ? (j == 0 ? acol0 : ti.up_off + acol0)
-                                                               : acol0 + 64 * j) + 8 * c8;
-                        const int mcol = (MODE == MODE_GATEUP) ? (j == 0 ? ti.M : ti.up_off + ti.M)
-                                                               : ti.M;  // columns of this weight
+                for (int j = 0; j < 2; ++j) {
+                    const int col = ((MODE == MODE_GATEUP) ? (j == 0 ? acol0 : ti.up_off + acol0)
+                                                           : acol0 + 64 * j) + 8 * c8;
+                    const int mcol = (MODE == MODE_GATEUP) ? (j == 0 ? ti.M : ti.up_off + ti.M)
+                                                           : ti.M;  // columns of this weight
 #pragma unroll
-                        for (int i = 0; i < 8; ++i) sc[j][i] = (col + i < mcol) ? sv[col + i] : 0.f;
-                    }
+                    for (int i = 0; i < 8; ++i) sc[j][i] = (col + i < mcol) ? sv[col + i] : 0.f;
                 }
+            }
+            for (int kb = ti.kb0; kb < ti.kb1; ++kb) {
                 const bool got = mbar_wait(rawfull_bar(stage), phase, args.err, DEV_ERR_TIMEOUT_PRODUCER);
                 if (!__all_sync(0xffffffffu, got)) {
                     ok = false;
@@ -484,7 +489,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(GemmCfg<MODE, ET, FP
         uint32_t acc_phase = 0;
         volatile uint32_t* abort_flag = misc + 1;
         for (int L = pair; L < total; L += npairs) {
-            const TileInfo ti = decode_tile<MODE>(*tab, args, L);
+            const TileInfo ti = decode_tile<MODE, C::BK>(*tab, args, L);
             const bool ok = mbar_wait(tfull_bar(acc), acc_phase, args.err, DEV_ERR_TIMEOUT_EPILOGUE);
             if constexpr (MODE == MODE_GATEUP) {
                 // the 4 warps meet at named barriers below: leave together or not at all
@@ -500,6 +505,45 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(GemmCfg<MODE, ET, FP
             const long long ld = ti.shared ? args.ld_shared : args.ld_routed;
             const int32_t* rowmap = ti.shared ? args.rowmap_shared : args.rowmap_routed;
             const float* colscale = ti.shared ? nullptr : args.colscale_routed;
+            if (args.partial_out) {
+                // split-K: store this split's fp32 partial; row = slot (gate/up) or
+                // token (down), column = the weight column of this TMEM lane
+                float* pbase = ti.shared ? args.part_shared : args.part_routed;
+                const long long pld = ti.shared ? args.ld_part_shared : args.ld_part_routed;
+                const long long pst = ti.shared ? args.part_stride_shared : args.part_stride_routed;
+                float* pp = pbase + pst * ti.split;
+                int col, fcheck;
+                if constexpr (MODE == MODE_GATEUP) {
+                    const int r = q * 32 + lane;                      // 0..127: [gate 64 | up 64]
+                    fcheck = ti.f0 + 64 * (int)rank + (r & 63);       // feature
+                    col = (r < 64 ? 0 : ti.up_off) + fcheck;
+                } else {
+                    fcheck = ti.f0 + 128 * (int)rank + q * 32 + lane;
+                    col = fcheck;
+                }
+                const bool fvalid = fcheck < ti.M;
+                for (int c = 0; c < ti.n_valid; c += 32) {
+                    const bool cval = c + lane < ti.n_valid;
+                    const int my_row =
+                        cval ? (rowmap ? rowmap[ti.row0 + c + lane] : ti.row0 + c + lane) : 0;
+                    float v[32];
+                    tmem_ld_32x32(tb + (uint32_t)c, v);
+                    tmem_wait_ld();
+#pragma unroll
+                    for (int i = 0; i < 32; ++i) {
+                        const int orow = __shfl_sync(0xffffffffu, my_row, i);
+                        if (fvalid && c + i < ti.n_valid) pp[(size_t)orow * pld + col] = v[i];
+                    }
+                }
+                tc_fence_before();
+                __syncwarp();
+                if (lane == 0) mbar_arrive_remote(mapa_shared(tempty_bar(acc), 0));
+                if (++acc == Cfg::ACC_BUFS) {
+                    acc = 0;
+                    acc_phase ^= 1u;
+                }
+                continue;
+            }
             for (int c = 0; c < ti.n_valid; c += 32) {
                 // output row (token or slot) and scale of each of the 32 columns, one per lane
                 const bool cval = c + lane < ti.n_valid;
@@ -564,6 +608,60 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(GemmCfg<MODE, ET, FP
     if (warp == 1) {
         tc_fence_after();
         tmem_dealloc_pair(tmem_base, Cfg::TMEM_COLS);
+    }
+}
+
+// Split-K finish of the gate/up contraction: h = silu(g * sum_s a_gate) *
+// (g * sum_s a_up) over the splits in order, for the routed slots (g = the
+// slot's sigmoid gate) and the shared rows (g = 1).  One thread per output.
+template <typename ET>
+__global__ void __launch_bounds__(256) gateup_finish_kernel(
+    const float* __restrict__ part_r, long long ld_r, long long stride_r, const float* __restrict__ part_s,
+    long long ld_s, long long stride_s, int ksplit, int T, int F, int Fs,
+    const float* __restrict__ gslot, ET* __restrict__ hr, ET* __restrict__ hs) {
+    const long long n_r = (long long)T * F, n = n_r + (long long)T * Fs;
+    for (long long i = blockIdx.x * (long long)blockDim.x + threadIdx.x; i < n;
+         i += (long long)gridDim.x * blockDim.x) {
+        const bool shared = i >= n_r;
+        const long long j = shared ? i - n_r : i;
+        const int w = shared ? Fs : F;
+        const int row = (int)(j / w), f = (int)(j % w);
+        const float* p = shared ? part_s : part_r;
+        const long long ld = shared ? ld_s : ld_r, st = shared ? stride_s : stride_r;
+        float ag = 0.f, au = 0.f;
+        for (int s = 0; s < ksplit; ++s) {
+            ag += p[st * s + (long long)row * ld + f];
+            au += p[st * s + (long long)row * ld + w + f];
+        }
+        const float g = shared ? 1.0f : gslot[row];
+        store_elem((shared ? hs : hr) + (long long)row * w + f, silu_f(g * ag) * (g * au));
+    }
+}
+
+// Finish of the down contraction: out = rn(sum of the partials in order)
+// (shared and routed results, times the split-K ranges).  n % 4 == 0; four
+// outputs per thread with 16-byte loads.
+template <typename ET>
+__global__ void __launch_bounds__(256) down_finish_kernel(const float* __restrict__ part, long long stride,
+                                                          int nparts, long long n, ET* __restrict__ out) {
+    const long long n4 = n >> 2;
+    for (long long i = blockIdx.x * (long long)blockDim.x + threadIdx.x; i < n4;
+         i += (long long)gridDim.x * blockDim.x) {
+        float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+        for (int s = 0; s < nparts; ++s) {
+            const float4 v = reinterpret_cast<const float4*>(part + stride * s)[i];
+            acc.x += v.x, acc.y += v.y, acc.z += v.z, acc.w += v.w;
+        }
+        if constexpr (sizeof(ET) == 2) {
+            const __nv_bfloat162 lo = __floats2bfloat162_rn(acc.x, acc.y);
+            const __nv_bfloat162 hi = __floats2bfloat162_rn(acc.z, acc.w);
+            uint2 pk;
+            pk.x = *reinterpret_cast<const uint32_t*>(&lo);
+            pk.y = *reinterpret_cast<const uint32_t*>(&hi);
+            reinterpret_cast<uint2*>(out)[i] = pk;
+        } else {
+            reinterpret_cast<float4*>(out)[i] = acc;
+        }
     }
 }
 

@@ -81,10 +81,21 @@ __device__ void build_table(GroupTable* tab, int G, RowsF rows_of, Row0F row0_of
 // Single CTA of 1024 threads.  Writes counts[E], offsets[E+1], perm[T]
 // (slot -> token), inv[T] (token -> slot) and two work lists:
 //   tab_gu : shared expert (rows T) then the routed experts, gate/up GEMM
-//   tab_dn : routed experts (rows = their slots), down GEMM with the shared
-//            expert's K segment fused in front
+//   tab_dn : shared expert (rows = all T slots) then the routed experts,
+//            down GEMM (the two contractions meet in fp32 partials)
 // smem: wcnt[32][E] + running[E] ints.
-__global__ void __launch_bounds__(1024) permute_kernel(const int32_t* __restrict__ idx, int T,
+//
+// logits != null (expert-split router): first finish the routing here -- per
+// token, sum the router's logit_splits partial logits [split][T][E] in
+// order, then the arg-max over the E biased fp32 logits (lowest index on ties,
+// NaN never wins), the runner-up margin and the sigmoid gate -- writing idx,
+// gate, lmax and margin.
+__global__ void __launch_bounds__(1024) permute_kernel(const float* __restrict__ logits,
+                                                       int logit_splits,
+                                                       float* __restrict__ gate,
+                                                       float* __restrict__ lmax,
+                                                       float* __restrict__ margin,
+                                                       int32_t* __restrict__ idx, int T,
                                                        int E, int fb_gu_routed, int fb_gu_shared,
                                                        int fb_down, int32_t* __restrict__ counts,
                                                        int32_t* __restrict__ offsets,
@@ -98,6 +109,46 @@ __global__ void __launch_bounds__(1024) permute_kernel(const int32_t* __restrict
     int* soff = running + E;      // [E + 1]
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
 
+    if (logits) {
+        // one warp per token: lane owns experts lane, lane+32, ... (ascending
+        // inside the lane); the warp then keeps the larger value, lower index
+        for (int t = warp; t < T; t += 32) {
+            float best = -INFINITY, second = -INFINITY;
+            int bi = 0x7fffffff;
+            for (int e = lane; e < E; e += 32) {
+                float l = 0.f;  // the router's K-split partials, summed in order
+                for (int s = 0; s < logit_splits; ++s) l += logits[((size_t)s * T + t) * E + e];
+                if (l > best) {
+                    second = best;
+                    best = l;
+                    bi = e;
+                } else if (l > second) {
+                    second = l;
+                }
+            }
+            if (bi == 0x7fffffff) bi = lane;  // no finite winner in this lane
+#pragma unroll
+            for (int off = 16; off > 0; off >>= 1) {
+                const float ob = __shfl_xor_sync(0xffffffffu, best, off);
+                const float os = __shfl_xor_sync(0xffffffffu, second, off);
+                const int oi = __shfl_xor_sync(0xffffffffu, bi, off);
+                if (ob > best || (ob == best && oi < bi)) {
+                    second = fmaxf(os, best);
+                    best = ob;
+                    bi = oi;
+                } else {
+                    second = fmaxf(second, ob);
+                }
+            }
+            if (lane == 0) {
+                idx[t] = bi;
+                lmax[t] = best;
+                margin[t] = best - second;
+                gate[t] = 1.0f / (1.0f + expf(-best));
+            }
+        }
+        __syncthreads();
+    }
     for (int e = tid; e < E; e += 1024) running[e] = 0;
     __syncthreads();
     for (int c0 = 0; c0 < T; c0 += 1024) {
@@ -173,8 +224,9 @@ __global__ void __launch_bounds__(1024) permute_kernel(const int32_t* __restrict
             [&](int g) { return g == 0 ? E : g - 1; },
             [&](int g) { return g == 0 ? fb_gu_shared : fb_gu_routed; });
         build_table(
-            tab_dn, E, [&](int g) { return running[g]; }, [&](int g) { return soff[g]; },
-            [&](int g) { return g; }, [&](int) { return fb_down; });
+            tab_dn, E + 1, [&](int g) { return g == 0 ? T : running[g - 1]; },
+            [&](int g) { return g == 0 ? 0 : soff[g - 1]; },
+            [&](int g) { return g == 0 ? E : g - 1; }, [&](int) { return fb_down; });
     }
 }
 

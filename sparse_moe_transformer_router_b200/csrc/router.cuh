@@ -195,9 +195,16 @@ constexpr int STAGE_BYTES = A_BYTES + MAX_B_BOXES * B_BOX_BYTES;
 constexpr size_t SMEM_BYTES = 1024 + (size_t)STAGES * STAGE_BYTES + (2 * STAGES + 1) * 8 + 16;
 }  // namespace rmma
 
+// Expert-split mode (logits != null, for batches of one token tile): CTA
+// (y, z) computes experts [y*n_chunk, (y+1)*n_chunk) over K slice z of
+// gridDim.z and stores the fp32 partial logits to logits[z][T][E] (the bias
+// in slice 0); the sum over slices and the arg-max then run in the
+// permutation kernel.  This spreads the router weight stream over
+// (E / n_chunk) x slices SMs instead of one.
 __global__ void __launch_bounds__(128, 1)
     router_mma_kernel(const __grid_constant__ CUtensorMap x_map, const __grid_constant__ CUtensorMap wr_map,
-                      const float* __restrict__ bias, int T, int d, int E, int32_t* __restrict__ idx,
+                      const float* __restrict__ bias, int T, int d, int E, int n_chunk,
+                      float* __restrict__ logits, int32_t* __restrict__ idx,
                       float* __restrict__ gate, float* __restrict__ lmax,
                       float* __restrict__ margin, unsigned* err) {
     extern __shared__ uint8_t rsmem_raw[];
@@ -210,8 +217,10 @@ __global__ void __launch_bounds__(128, 1)
     auto full_bar = [&](int s) { return bar0 + 8u * s; };
     auto empty_bar = [&](int s) { return bar0 + 8u * (rmma::STAGES + s); };
     const uint32_t done_bar = bar0 + 8u * (2 * rmma::STAGES);
-    const int n_pad = (E + 15) & ~15;
-    const int nbb = (E + 63) / 64;
+    const int e0 = blockIdx.y * n_chunk;        // first expert of this CTA
+    const int ne = min(n_chunk, E - e0);         // experts of this CTA
+    const int n_pad = (ne + 15) & ~15;
+    const int nbb = (ne + 63) / 64;
     uint32_t ncols = 32;
     while ((int)ncols < n_pad) ncols <<= 1;
 
@@ -232,7 +241,10 @@ __global__ void __launch_bounds__(128, 1)
     tc_fence_after();
     const uint32_t tmem_base = *tmem_slot;
     const int t0 = blockIdx.x * 128;
-    const int nkb = d / 64;
+    const int nkb_all = d / 64;
+    const int kb_begin = (int)(((long long)nkb_all * blockIdx.z) / gridDim.z);
+    const int kb_end = (int)(((long long)nkb_all * (blockIdx.z + 1)) / gridDim.z);
+    const int nkb = kb_end - kb_begin;
 
     if (warp == 0 && lane == 0) {
         int stage = 0;
@@ -241,11 +253,12 @@ __global__ void __launch_bounds__(128, 1)
             if (!mbar_wait(empty_bar(stage), phase ^ 1u, err, DEV_ERR_TIMEOUT_PRODUCER)) break;
             mbar_arrive_expect_tx(full_bar(stage), rmma::A_BYTES + nbb * rmma::B_BOX_BYTES);
             const uint32_t sb = stage0 + (uint32_t)stage * rmma::STAGE_BYTES;
-            tma_load_2d(sb, &x_map, full_bar(stage), kb * 64, t0);
-            tma_load_2d(sb + 64 * 128, &x_map, full_bar(stage), kb * 64, t0 + 64);
+            const int kg = (kb_begin + kb) * 64;
+            tma_load_2d(sb, &x_map, full_bar(stage), kg, t0);
+            tma_load_2d(sb + 64 * 128, &x_map, full_bar(stage), kg, t0 + 64);
             for (int j = 0; j < nbb; ++j)
-                tma_load_2d(sb + rmma::A_BYTES + j * rmma::B_BOX_BYTES, &wr_map, full_bar(stage), 64 * j,
-                            kb * 64);
+                tma_load_2d(sb + rmma::A_BYTES + j * rmma::B_BOX_BYTES, &wr_map, full_bar(stage), e0 + 64 * j,
+                            kg);
             used |= 1u << stage;
             last_par = (last_par & ~(1u << stage)) | (phase << stage);
             if (++stage == rmma::STAGES) {
@@ -282,9 +295,24 @@ __global__ void __launch_bounds__(128, 1)
     const bool ok = mbar_wait(done_bar, 0, err, DEV_ERR_TIMEOUT_EPILOGUE);
     if (__all_sync(0xffffffffu, ok)) {
         tc_fence_after();
+        const int t = t0 + 32 * warp + lane;
+        if (logits) {
+            for (int c = 0; c < n_pad; c += 32) {
+                float v[32];
+                tmem_ld_32x32(tmem_base + ((uint32_t)(32 * warp) << 16) + (uint32_t)c, v);
+                tmem_wait_ld();
+#pragma unroll
+                for (int i = 0; i < 32; ++i) {
+                    const int e = c + i;
+                    if (e < ne && t < T)
+                        logits[((size_t)blockIdx.z * T + t) * E + e0 + e] =
+                            v[i] + ((bias && blockIdx.z == 0) ? bias[e0 + e] : 0.f);
+                }
+            }
+        }
         float best = -INFINITY, second = -INFINITY;
         int bi = 0;
-        for (int c = 0; c < n_pad; c += 32) {
+        for (int c = 0; !logits && c < n_pad; c += 32) {
             float v[32];
             tmem_ld_32x32(tmem_base + ((uint32_t)(32 * warp) << 16) + (uint32_t)c, v);
             tmem_wait_ld();
@@ -303,8 +331,7 @@ __global__ void __launch_bounds__(128, 1)
                 }
             }
         }
-        const int t = t0 + 32 * warp + lane;
-        if (t < T) {
+        if (!logits && t < T) {
             idx[t] = bi;
             lmax[t] = best;
             margin[t] = best - second;

@@ -32,6 +32,13 @@ SMALL = {
     "fp8_zipf": LayerConfig("fp8_zipf", 700, 192, 16, 128, 320, "fp8", router="zipf", n_dead=4,
                             wr_std=0.05),
     "fp8_T1": LayerConfig("fp8_T1", 1, 256, 8, 256, 256, "fp8", wr_std=0.1),
+    # few tiles: split-K partials + finish kernels; T <= 128 with E % 16 == 0:
+    # expert-split router with the arg-max in the permutation kernel
+    "bf16_splitk": LayerConfig("bf16_splitk", 2, 1024, 8, 1024, 1024, "bf16", wr_std=0.03),
+    "f32_splitk": LayerConfig("f32_splitk", 3, 1024, 8, 1024, 512, "f32", wr_std=0.03),
+    "fp8_splitk": LayerConfig("fp8_splitk", 2, 1024, 8, 1024, 1024, "fp8", wr_std=0.03),
+    "bf16_router_split": LayerConfig("bf16_router_split", 1, 1024, 64, 512, 512, "bf16", wr_std=0.03),
+    "bf16_T40_E32": LayerConfig("bf16_T40_E32", 40, 512, 32, 512, 768, "bf16", wr_std=0.05),
 }
 
 
@@ -80,12 +87,15 @@ def test_repeatable_and_host_path_identical():
     out2, _ = run_gpu(layer, inp)
     assert torch.equal(out1, out2)
     x_host = inp.x.cpu().pin_memory()
-    out_host = torch.empty_like(x_host).pin_memory()
-    layer.forward_host(x_host, inp.W_router, inp.W_gate_up, inp.W_down, inp.Ws_gate_up,
-                       inp.Ws_down, out_host)
-    torch.cuda.synchronize()
+    outs = [torch.empty_like(x_host).pin_memory() for _ in range(3)]
+    for o in outs:  # pipelined calls: slots are reused while earlier copies may be in flight
+        layer.forward_host(x_host, inp.W_router, inp.W_gate_up, inp.W_down, inp.Ws_gate_up,
+                           inp.Ws_down, o)
+    layer.join_host()
+    torch.cuda.current_stream().synchronize()
+    for o in outs:
+        assert torch.equal(o, out1.cpu())
     layer.check_device_status()
-    assert torch.equal(out_host, out1.cpu())
 
 
 def test_weight_pointer_change_rebuilds_descriptors():
