@@ -189,6 +189,28 @@ def cpu_baseline(inp, budget_s: float = 15.0) -> dict:
                       f"{cfg.T} tokens, evenly spaced, {dt2:.1f} s"}
 
 
+def rank_barrier(world: int):
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+
+
+def rank_max(v: float, world: int, device: str) -> float:
+    """The slowest rank's time (every rank takes part, every rank gets it)."""
+    if world == 1:
+        return v
+    import torch.distributed as dist
+    t = torch.tensor([v], device=device, dtype=torch.float64)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def replica_throughput(world: int, tokens_per_rank: int, steps: int, t_ms: float) -> float:
+    """Weak scaling: every rank processed its own batch each step; the job's
+    throughput is all ranks' tokens over the slowest rank's time."""
+    return world * tokens_per_rank * steps / (t_ms / 1e3)
+
+
 def run_reference(args, rank, world):
     if rank != 0:
         return
@@ -242,7 +264,8 @@ def main():
     if world > 1:
         import datetime
         import torch.distributed as dist
-        torch.cuda.set_device(local)
+        if torch.cuda.is_available():
+            torch.cuda.set_device(local)
         dist.init_process_group("nccl" if args.impl == "b200" else "gloo",
                                 timeout=datetime.timedelta(seconds=300))
     if args.tokens:
@@ -275,19 +298,8 @@ def run_b200(args, rank, world, local):
     fwd = lambda: layer.forward(inp.x, inp.W_router, inp.W_gate_up, inp.W_down,  # noqa: E731
                                 inp.Ws_gate_up, inp.Ws_down, out=out)
     stream = torch.cuda.current_stream()
-
-    def barrier():
-        if world > 1:
-            import torch.distributed as dist
-            dist.barrier()
-
-    def max_over_ranks(v: float) -> float:
-        if world == 1:
-            return v
-        import torch.distributed as dist
-        t = torch.tensor([v], device="cuda", dtype=torch.float64)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        return float(t.item())
+    barrier = lambda: rank_barrier(world)  # noqa: E731
+    max_over_ranks = lambda v: rank_max(v, world, "cuda")  # noqa: E731
 
     for _ in range(args.warmup):
         fwd()
@@ -317,7 +329,7 @@ def run_b200(args, rank, world, local):
     layer.check_device_status()
 
     ms_step = t_ms / args.steps
-    value = world * cfg.T * args.steps / (t_ms / 1e3)
+    value = replica_throughput(world, cfg.T, args.steps, t_ms)
 
     # ------------------------------------------------------------- e2e (host buffers)
     x_host = inp.x.cpu().pin_memory()
@@ -341,7 +353,7 @@ def run_b200(args, rank, world, local):
     clocks = sampler.stop()  # samples span the device-timed and the end-to-end regions
     layer.check_device_status()
     io_bytes = cfg.T * cfg.d_model * inp.x.element_size()
-    e2e = {"value": world * cfg.T * e2e_steps / (th_ms / 1e3), "unit": "tokens/s",
+    e2e = {"value": replica_throughput(world, cfg.T, e2e_steps, th_ms), "unit": "tokens/s",
            "h2d_bytes_per_step": io_bytes, "d2h_bytes_per_step": io_bytes,
            "ms_per_step": th_ms / e2e_steps,
            "path": "l4moe_forward_host per step: pinned host x -> device (copy-in stream), layer "
