@@ -63,7 +63,7 @@ bool encode_2d(CUtensorMap* m, CUtensorMapDataType dt, const void* base, uint64_
 // Split-K is used for batches of at most this many tokens, into at most
 // kMaxSplit k-ranges (tiles too few to fill the GPU, e.g. decode).
 constexpr size_t kSplitMaxTokens = 64;
-constexpr int kMaxSplit = 8;
+constexpr int kMaxSplit = 16;
 // The expert-split router (one token tile) also splits K into this many slices.
 constexpr int kRouterKSplit = 8;
 
@@ -78,8 +78,8 @@ size_t act_bytes(l4moe_dtype dt) { return dt == L4MOE_F32 ? 4 : 2; }
 size_t w_bytes(l4moe_dtype dt) { return dt == L4MOE_F32 ? 4 : (dt == L4MOE_BF16 ? 2 : 1); }
 
 // Split-K plan of one forward of T tokens: how many k-ranges the gate/up and
-// the down launches use.  Only batches of at most kSplitMaxTokens split; the
-// aim is about four waves of CTA pairs with at least 8 k-blocks per range.
+// the down launches use.  Only batches of at most kSplitMaxTokens split, into
+// ranges of at least 8 k-blocks.
 struct SplitPlan {
     int s_gu, s_dn;
 };
@@ -88,17 +88,33 @@ SplitPlan split_plan(const l4moe_params& p, int T, int sms) {
     const int d = p.d_model, F = p.expert_ffn, Fs = p.shared_ffn, E = p.num_experts;
     const int kblk = (int)(128 / act_bytes(p.dtype));  // K elements per k-block
     const int fb_gu_r = (F + 127) / 128, fb_gu_s = (Fs + 127) / 128, fb_dn = (d + 255) / 256;
+    // Tiles are striped over the CTA pairs, so the launch lasts ceil(units /
+    // pairs) tile times: take the split count that fills the last wave best
+    // (fewer splits unless more fill it clearly better).  On decode batches of
+    // a Maverick-shaped layer a split gate/up launch (partials plus a finish
+    // kernel) was slower than the unsplit one whenever at least half of the
+    // pairs had a tile, so gate/up splits only below that.
+    const long long pairs = std::max(1, sms / 2);
     auto pick = [&](long long tiles, int nkb) {
         if ((size_t)T > kSplitMaxTokens || tiles <= 0) return 1;
-        const long long want = 4LL * (sms / 2);
-        long long sp = (want + tiles - 1) / tiles;
-        sp = std::min<long long>(sp, kMaxSplit);
-        sp = std::min<long long>(sp, std::max(1, nkb / 8));
-        return (int)std::max(1LL, sp);
+        const int max_sp = std::min(kMaxSplit, std::max(1, nkb / 8));
+        int best = 1;
+        double best_fill = 0.0;
+        for (int sp = 1; sp <= max_sp; ++sp) {
+            const long long units = tiles * sp;
+            const long long waves = (units + pairs - 1) / pairs;
+            const double fill = (double)units / (double)(waves * pairs);
+            if (fill > best_fill + 0.02) {
+                best = sp;
+                best_fill = fill;
+            }
+        }
+        return best;
     };
     const long long eg = std::min(E, T);  // non-empty routed experts (one token tile each)
     SplitPlan sp;
-    sp.s_gu = pick((long long)fb_gu_s + fb_gu_r * eg, d / kblk);
+    const long long gu_tiles = (long long)fb_gu_s + fb_gu_r * eg;
+    sp.s_gu = 2 * gu_tiles < pairs ? pick(gu_tiles, d / kblk) : 1;
     sp.s_dn = pick((long long)fb_dn * (eg + 1), std::min(F, Fs) / kblk);
     return sp;
 }
@@ -356,12 +372,11 @@ void launch_router(const void* x, const void* Wr, const float* bias, int T, int 
 }
 
 template <int MODE, typename ET, bool FP8W>
-void launch_gemm(int grid, const CUtensorMap& b_routed, const CUtensorMap& b_shared,
-                 const GemmArgs& a, cudaStream_t st) {
+void launch_gemm(int grid, const BMaps& bm, const GemmArgs& a, cudaStream_t st) {
     using Cfg = GemmCfg<MODE, ET, FP8W>;
     static std::once_flag once;
     std::call_once(once, [] { set_smem_attr(moe_gemm_kernel<MODE, ET, FP8W>, Cfg::SMEM_BYTES); });
-    moe_gemm_kernel<MODE, ET, FP8W><<<grid, Cfg::THREADS, Cfg::SMEM_BYTES, st>>>(b_routed, b_shared, a);
+    moe_gemm_kernel<MODE, ET, FP8W><<<grid, Cfg::THREADS, Cfg::SMEM_BYTES, st>>>(bm, a);
 }
 
 // The launch sequence of one forward.  w / ws_tokens: the workspace and the
@@ -390,15 +405,23 @@ l4moe_status run_layer(l4moe_handle* h, int T, const void* x, const void* Wr, co
     ET* hr = reinterpret_cast<ET*>(w + L.hr);
     ET* hs = reinterpret_cast<ET*>(w + L.hs);
 
-    // per-call activation descriptors (K-major rows, boxes of 128 B x 64 rows)
+    // per-call activation descriptors (K-major rows of 128 B): the router's
+    // x (64-row boxes) and the GEMMs' token operands (full- and small-tile
+    // boxes: gate/up reads x in expert order and x, down reads H_r and H_s)
     const CUtensorMapDataType adt =
         sizeof(ET) == 4 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT32 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16;
     const uint32_t bk = (uint32_t)(128 / sizeof(ET));
-    CUtensorMap m_xg, m_x, m_hr, m_hs;
-    if (!encode_2d(&m_xg, adt, xg, d, T, (uint64_t)d * sizeof(ET), bk, 64) ||
-        !encode_2d(&m_x, adt, x, d, T, (uint64_t)d * sizeof(ET), bk, 64) ||
-        !encode_2d(&m_hr, adt, hr, F, T, (uint64_t)F * sizeof(ET), bk, 64) ||
-        !encode_2d(&m_hs, adt, hs, Fs, T, (uint64_t)Fs * sizeof(ET), bk, 64))
+    using GCfg = GemmCfg<MODE_GATEUP, ET, FP8W>;
+    constexpr uint32_t rb = GCfg::B_BOX_ROWS, rs = GCfg::B_SMALL_ROWS;
+    CUtensorMap m_x;
+    BMaps bm_gu, bm_dn;
+    auto act = [&](CUtensorMap* m, const void* base, int width, uint32_t rows) {
+        return encode_2d(m, adt, base, (uint64_t)width, (uint64_t)T, (uint64_t)width * sizeof(ET), bk, rows);
+    };
+    if (!act(&m_x, x, d, 64) || !act(&bm_gu.routed, xg, d, rb) || !act(&bm_gu.routed_small, xg, d, rs) ||
+        !act(&bm_gu.shared, x, d, rb) || !act(&bm_gu.shared_small, x, d, rs) ||
+        !act(&bm_dn.routed, hr, F, rb) || !act(&bm_dn.routed_small, hr, F, rs) ||
+        !act(&bm_dn.shared, hs, Fs, rb) || !act(&bm_dn.shared_small, hs, Fs, rs))
         return fail(h, L4MOE_ERR_CUDA, "cuTensorMapEncodeTiled failed for an activation");
 
     cudaError_t e;
@@ -491,7 +514,7 @@ l4moe_status run_layer(l4moe_handle* h, int T, const void* x, const void* Wr, co
     LaunchTimer t_gu(h, 3, st);
     launch_gemm<MODE_GATEUP, ET, FP8W>(
         grid_for(s_gu * ((long long)fb_gu_s * tb + (long long)fb_gu_r * (tb + std::min(E, T)))),
-        m_xg, m_x, gu, st);
+        bm_gu, gu, st);
     if (s_gu > 1) {
         const long long n = (long long)T * (F + Fs);
         gateup_finish_kernel<ET><<<(int)std::min<long long>((n + 255) / 256, 4LL * h->sms), 256, 0, st>>>(
@@ -530,7 +553,7 @@ l4moe_status run_layer(l4moe_handle* h, int T, const void* x, const void* Wr, co
     dn.err = err;
     LaunchTimer t_dn(h, 4, st);
     launch_gemm<MODE_DOWN, ET, FP8W>(grid_for(s_dn * (long long)fb_dn * (2 * tb + std::min(E, T))),
-                                     m_hr, m_hs, dn, st);
+                                     bm_dn, dn, st);
     {
         const long long n = (long long)T * d;
         down_finish_kernel<ET><<<(int)std::min<long long>((n / 4 + 255) / 256, 4LL * h->sms), 256, 0, st>>>(

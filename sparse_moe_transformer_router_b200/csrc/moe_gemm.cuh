@@ -125,8 +125,10 @@ struct GemmCfg {
     static constexpr int A_BOX_FEATS = 128 / C::BYTES;       // features per A box (one 128 B slab)
     static constexpr int A_BOXES = 128 / A_BOX_FEATS;        // boxes per CTA A tile
     static constexpr int A_BOX_BYTES = C::BK * 128;          // BK rows x 128 B
-    static constexpr int B_BOX_ROWS = 64;
+    static constexpr int B_BOX_ROWS = 128;                   // token rows per full-tile box
     static constexpr int B_BOX_BYTES = B_BOX_ROWS * 128;
+    static constexpr int B_SMALL_ROWS = 32;                  // token rows per small-tile box
+    static constexpr int B_SMALL_BYTES = B_SMALL_ROWS * 128;
     static constexpr int B_BYTES = (kTokTile / 2) * 128;     // this CTA's half of the tokens
     static constexpr int RAW_BYTES = FP8W ? 2 * 64 * 64 : 0; // 2 slabs x 64 K rows x 64 features
     static constexpr int STAGE_BYTES = A_BYTES + B_BYTES + RAW_BYTES;
@@ -148,8 +150,13 @@ struct TileInfo {
     bool shared;
 };
 
-template <int MODE, int ElemCfgBK>
-__device__ __forceinline__ TileInfo decode_tile(const GroupTable& tab, const GemmArgs& a, int L) {
+// Activation bytes a band of token tiles may keep in L2 (each of the two
+// dies caches what its SMs read, so this stays well under half of L2).
+constexpr long long kBandBytes = 24ll << 20;
+
+template <int MODE, int ElemCfgBK, int ElemBytes>
+__device__ __forceinline__ TileInfo decode_tile(const GroupTable& tab, const GemmArgs& a, int pos) {
+    const int L = tile_at(pos, tab.heavy_tiles, tab.total_tiles);
     int lo = 0, hi = tab.num_groups - 1;
     while (lo < hi) {
         const int mid = (lo + hi + 1) >> 1;
@@ -159,19 +166,28 @@ __device__ __forceinline__ TileInfo decode_tile(const GroupTable& tab, const Gem
     const int local = L - tab.tile_start[g];
     const int rows = tab.rows[g];
     const int ntb = (rows + kTokTile - 1) / kTokTile;
-    const int tb = local % ntb;
-    const int rest = local / ntb;
-    const int split = rest % a.ksplit;
-    const int fb = rest / a.ksplit;
     TileInfo ti;
-    ti.split = split;
     ti.expert = tab.expert[g];
     ti.shared = (ti.expert == a.num_experts);
+    ti.K = ti.shared ? a.k_shared : a.k_routed;
+    // Token tiles go in bands of `band` tiles whose activation rows (the B
+    // operand, about kBandBytes) stay in L2 while the band sweeps every
+    // feature block; inside a band the token tile varies fastest, so the
+    // tiles that share a weight tile run side by side.
+    const int band = max(1, (int)(kBandBytes / ((long long)kTokTile * ti.K * ElemBytes)));
+    const int fbk = (tab.tile_start[g + 1] - tab.tile_start[g]) / ntb;  // feature blocks x splits
+    const int b = local / (band * fbk);
+    const int nb = min(band, ntb - b * band);  // token tiles in this band (the last may be short)
+    const int rem = local - b * band * fbk;
+    const int tb = b * band + rem % nb;
+    const int rest = rem / nb;
+    const int split = rest % a.ksplit;
+    const int fb = rest / a.ksplit;
+    ti.split = split;
     ti.row0 = tab.row0[g] + tb * kTokTile;
     ti.n_valid = min(kTokTile, rows - tb * kTokTile);
     ti.n_mma = (ti.n_valid + 15) & ~15;
     ti.f0 = fb * pair_features<MODE>();
-    ti.K = ti.shared ? a.k_shared : a.k_routed;
     ti.M = ti.shared ? a.m_shared : a.m_routed;
     ti.up_off = ti.shared ? a.up_shared : a.up_routed;
     const int nkb = ti.K / ElemCfgBK;
@@ -219,10 +235,18 @@ __device__ __forceinline__ void fence_proxy_async_smem() {
 __device__ __forceinline__ void store_elem(float* p, float v) { *p = v; }
 __device__ __forceinline__ void store_elem(__nv_bfloat16* p, float v) { *p = __float2bfloat16_rn(v); }
 
+// Token-operand (B) descriptors of the routed and the shared rows, with
+// 128-row boxes for tiles of more than 64 tokens per CTA and 32-row boxes
+// for the others.  A box always lands whole (zero-filled past the matrix), so
+// the box size sets the bytes a small tile moves; one big box instead of
+// several small ones keeps the TMA unit's per-box cost off the full tiles.
+struct BMaps {
+    CUtensorMap routed, shared, routed_small, shared_small;
+};
+
 template <int MODE, typename ET, bool FP8W>
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(GemmCfg<MODE, ET, FP8W>::THREADS, 1)
-    moe_gemm_kernel(const __grid_constant__ CUtensorMap b_routed,
-                    const __grid_constant__ CUtensorMap b_shared, const GemmArgs args) {
+    moe_gemm_kernel(const __grid_constant__ BMaps bm, const GemmArgs args) {
     using Cfg = GemmCfg<MODE, ET, FP8W>;
     using C = ElemCfg<ET>;
     extern __shared__ uint8_t smem_raw[];
@@ -276,8 +300,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(GemmCfg<MODE, ET, FP
         fence_barrier_init();
     }
     if (warp == 0 && lane == 0) {
-        tma_prefetch_desc(&b_routed);
-        tma_prefetch_desc(&b_shared);
+        tma_prefetch_desc(&bm.routed);
+        tma_prefetch_desc(&bm.shared);
+        tma_prefetch_desc(&bm.routed_small);
+        tma_prefetch_desc(&bm.shared_small);
     }
     cluster_sync();  // barriers of both CTAs initialised before any remote use
     if (warp == 1) {
@@ -300,12 +326,16 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(GemmCfg<MODE, ET, FP
             uint32_t used = 0, last_par = 0;  // per stage: issued at least once / its parity
             bool aborted = false;
             for (int L = pair; L < total && !aborted; L += npairs) {
-                const TileInfo ti = decode_tile<MODE, C::BK>(*tab, args, L);
+                const TileInfo ti = decode_tile<MODE, C::BK, C::BYTES>(*tab, args, L);
                 const CUtensorMap* amap = args.a_maps + ti.expert;
-                const void* bmap = ti.shared ? (const void*)&b_shared : (const void*)&b_routed;
                 const int half = ti.n_mma >> 1;  // tokens per CTA
-                const int nbb = (half + Cfg::B_BOX_ROWS - 1) / Cfg::B_BOX_ROWS;
-                const uint32_t tx_cta = (FP8W ? 0u : (uint32_t)Cfg::A_BYTES) + (uint32_t)nbb * Cfg::B_BOX_BYTES;
+                const bool big = half > 2 * Cfg::B_SMALL_ROWS;
+                const void* bmap = ti.shared ? (big ? (const void*)&bm.shared : (const void*)&bm.shared_small)
+                                             : (big ? (const void*)&bm.routed : (const void*)&bm.routed_small);
+                const int brows = big ? Cfg::B_BOX_ROWS : Cfg::B_SMALL_ROWS;
+                const int nbb = (half + brows - 1) / brows;
+                const uint32_t tx_cta =
+                    (FP8W ? 0u : (uint32_t)Cfg::A_BYTES) + (uint32_t)(nbb * brows * 128);
                 const int brow = ti.row0 + (int)rank * half;
                 // this CTA's A columns: gate/up -> [gate 64 | up 64] of features
                 // f0 + 64*rank; down -> 128 features f0 + 128*rank
@@ -347,8 +377,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(GemmCfg<MODE, ET, FP
                     }
                     const uint32_t bb = sb + Cfg::A_BYTES;
                     for (int j = 0; j < nbb; ++j)
-                        tma_load_2d_pair(bb + j * Cfg::B_BOX_BYTES, bmap, fb_leader, k,
-                                         brow + j * Cfg::B_BOX_ROWS);
+                        tma_load_2d_pair(bb + (uint32_t)(j * brows * 128), bmap, fb_leader, k,
+                                         brow + j * brows);
                     used |= 1u << stage;
                     last_par = (last_par & ~(1u << stage)) | (phase << stage);
                     if (++stage == Cfg::STAGES) {
@@ -380,7 +410,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(GemmCfg<MODE, ET, FP
             int acc = 0;
             uint32_t acc_phase = 0;
             for (int L = pair; L < total; L += npairs) {
-                const TileInfo ti = decode_tile<MODE, C::BK>(*tab, args, L);
+                const TileInfo ti = decode_tile<MODE, C::BK, C::BYTES>(*tab, args, L);
                 if (!mbar_wait_cluster(tempty_bar(acc), acc_phase ^ 1u, args.err, DEV_ERR_TIMEOUT_MMA))
                     break;
                 tc_fence_after();
@@ -439,7 +469,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(GemmCfg<MODE, ET, FP
         uint32_t phase = 0;
         bool ok = true;
         for (int L = pair; L < total && ok; L += npairs) {
-            const TileInfo ti = decode_tile<MODE, C::BK>(*tab, args, L);
+            const TileInfo ti = decode_tile<MODE, C::BK, C::BYTES>(*tab, args, L);
             const int acol0 = (MODE == MODE_GATEUP) ? ti.f0 + 64 * (int)rank : ti.f0 + 128 * (int)rank;
             // this tile's per-column scales for my 2 x 8 features
             float sc[2][8];
@@ -489,7 +519,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(GemmCfg<MODE, ET, FP
         uint32_t acc_phase = 0;
         volatile uint32_t* abort_flag = misc + 1;
         for (int L = pair; L < total; L += npairs) {
-            const TileInfo ti = decode_tile<MODE, C::BK>(*tab, args, L);
+            const TileInfo ti = decode_tile<MODE, C::BK, C::BYTES>(*tab, args, L);
             const bool ok = mbar_wait(tfull_bar(acc), acc_phase, args.err, DEV_ERR_TIMEOUT_EPILOGUE);
             if constexpr (MODE == MODE_GATEUP) {
                 // the 4 warps meet at named barriers below: leave together or not at all

@@ -21,12 +21,19 @@ namespace l4moe {
 // ceil(rows/kTokTile) * feature_blocks tiles.
 constexpr int kMaxGroups = 257;  // 256 routed experts + the shared expert
 constexpr int kTokTile = 256;    // tokens per GEMM tile (MMA N, swap-AB)
-constexpr int kFeatTile = 128;   // output features per GEMM tile (MMA M)
+
+// Groups are listed in two runs: first the "heavy" groups (at least
+// kHeavyRows rows: enough tokens per weight tile that the tensor cores, not
+// the weight stream, bound them), then the light ones.  The GEMM interleaves
+// the two runs' tiles evenly (see tile_at), so compute-bound and
+// weight-stream-bound tiles run side by side instead of in separate phases.
+constexpr int kHeavyRows = 192;
 
 struct GroupTable {
     int num_groups;
     int total_tiles;
-    int pad0, pad1;
+    int heavy_tiles;  // tiles of the leading heavy run: tile_start[first light group]
+    int pad0;
     int rows[kMaxGroups];
     int row0[kMaxGroups];
     int expert[kMaxGroups];       // 0..E-1 routed, E = shared
@@ -45,37 +52,51 @@ __device__ __forceinline__ int warp_incl_scan(int v) {
 
 // Warp 0 writes one table from candidate groups [0, G): candidate g has
 // rows(g), row0(g), expert(g), feature blocks fb(g).  Empty groups are left
-// out.
+// out; heavy groups come first, each run in candidate order.
 template <typename RowsF, typename Row0F, typename ExpF, typename FbF>
 __device__ void build_table(GroupTable* tab, int G, RowsF rows_of, Row0F row0_of, ExpF exp_of,
                             FbF fb_of) {
     const int lane = threadIdx.x & 31;
     int n_base = 0, t_base = 0;
-    for (int base = 0; base < G; base += 32) {
-        const int g = base + lane;
-        int rows = 0, tiles = 0;
-        if (g < G) {
-            rows = rows_of(g);
-            tiles = rows > 0 ? ((rows + kTokTile - 1) / kTokTile) * fb_of(g) : 0;
+    for (int run = 0; run < 2; ++run) {  // 0: heavy groups, 1: light groups
+        for (int base = 0; base < G; base += 32) {
+            const int g = base + lane;
+            int rows = 0, tiles = 0;
+            if (g < G) {
+                rows = rows_of(g);
+                const bool in_run = (rows >= kHeavyRows) == (run == 0);
+                tiles = (rows > 0 && in_run) ? ((rows + kTokTile - 1) / kTokTile) * fb_of(g) : 0;
+            }
+            const int flag = tiles > 0 ? 1 : 0;
+            const int fi = warp_incl_scan(flag);
+            const int ti = warp_incl_scan(tiles);
+            if (flag) {
+                const int pos = n_base + fi - 1;
+                tab->rows[pos] = rows;
+                tab->row0[pos] = row0_of(g);
+                tab->expert[pos] = exp_of(g);
+                tab->tile_start[pos] = t_base + ti - tiles;
+            }
+            n_base += __shfl_sync(0xffffffffu, fi, 31);
+            t_base += __shfl_sync(0xffffffffu, ti, 31);
         }
-        const int flag = tiles > 0 ? 1 : 0;
-        const int fi = warp_incl_scan(flag);
-        const int ti = warp_incl_scan(tiles);
-        if (flag) {
-            const int pos = n_base + fi - 1;
-            tab->rows[pos] = rows;
-            tab->row0[pos] = row0_of(g);
-            tab->expert[pos] = exp_of(g);
-            tab->tile_start[pos] = t_base + ti - tiles;
-        }
-        n_base += __shfl_sync(0xffffffffu, fi, 31);
-        t_base += __shfl_sync(0xffffffffu, ti, 31);
+        if (run == 0 && lane == 0) tab->heavy_tiles = t_base;
     }
     if (lane == 0) {
         tab->num_groups = n_base;
         tab->total_tiles = t_base;
         tab->tile_start[n_base] = t_base;
     }
+}
+
+// Launch position L (0 .. total-1) -> tile number in the table's order.  The
+// heavy run's H tiles take the positions where floor((L+1) H / N) steps up,
+// spread as evenly as integers allow, the light run's tiles the others; both
+// runs keep their own order, so tiles that share a weight tile stay close.
+__host__ __device__ __forceinline__ int tile_at(int L, int heavy, int total) {
+    const long long h1 = ((long long)(L + 1) * heavy) / total;
+    const long long h0 = ((long long)L * heavy) / total;
+    return h1 > h0 ? (int)(h1 - 1) : heavy + (L - (int)h1);
 }
 
 // Single CTA of 1024 threads.  Writes counts[E], offsets[E+1], perm[T]
