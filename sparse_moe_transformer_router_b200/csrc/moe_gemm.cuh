@@ -198,34 +198,25 @@ __device__ __forceinline__ TileInfo decode_tile(const GroupTable& tab, const Gem
 
 __device__ __forceinline__ float silu_f(float z) { return __fdividef(z, 1.0f + __expf(-z)); }
 
-// 8 E4M3 codes (little-endian in a uint2) -> 8 bf16 values of code * scale.
-// Integer/FMA-pipe widening (the conversion pipe runs at a quarter of their
-// rate): a byte permute puts code i in bits 31..24; an arithmetic shift by 4
-// spreads its sign over bits 31..27 and the mask keeps the sign (bit 31) and
-// the 7 exponent/mantissa bits at 26..20.  Read as fp32 that is exactly
-// code * 2^-120 for every finite code, subnormals included (the E4M3 bias
-// is 7, fp32's 127); the product with 2^120 is exact, the product with the
-// scale is rounded once in fp32 and the pair is packed to bf16 (nearest even).
-__device__ __forceinline__ float e4m3_byte_to_f32(uint32_t w, uint32_t sel) {
-    const uint32_t t = __byte_perm(w, 0u, sel);  // code << 24
-    return __uint_as_float((uint32_t)((int32_t)t >> 4) & 0x87F00000u) * 0x1p120f;
+// 2 E4M3 codes -> 2 bf16, exactly (bf16 has the wider exponent and
+// mantissa).  A byte permute puts code i in bits 15..8 of 16-bit lane i; the
+// sign stays at bit 15 and the 7 exponent/mantissa bits move to 10..4, which
+// read as bf16 is code * 2^-120 (the E4M3 exponent bias is 7, bf16's 127),
+// subnormal codes becoming bf16 subnormals.  One packed bf16 multiply by
+// 2^120 restores the value (exact: a power of two, results in range).  The
+// per-column scale is applied to the fp32 accumulator in the epilogue.
+__device__ __forceinline__ uint32_t e4m3x2_to_bf16x2(uint32_t w, uint32_t sel) {
+    const uint32_t t = __byte_perm(w, 0u, sel);  // code_i << 8 in lane i
+    const uint32_t bits = (t & 0x80008000u) | ((t >> 4) & 0x07F007F0u);
+    uint32_t r;
+    asm("mul.rn.bf16x2 %0, %1, %2;" : "=r"(r) : "r"(bits), "r"(0x7B807B80u));  // 2^120 in each lane
+    return r;
 }
 
-__device__ __forceinline__ uint4 e4m3x8_scaled_to_bf16(uint2 raw, const float (&sc)[8]) {
-    const uint32_t w[2] = {raw.x, raw.y};
-    uint32_t o[4];
-#pragma unroll
-    for (int h = 0; h < 2; ++h) {
-        const float f0 = e4m3_byte_to_f32(w[h], 0x0444u) * sc[4 * h + 0];
-        const float f1 = e4m3_byte_to_f32(w[h], 0x1444u) * sc[4 * h + 1];
-        const float f2 = e4m3_byte_to_f32(w[h], 0x2444u) * sc[4 * h + 2];
-        const float f3 = e4m3_byte_to_f32(w[h], 0x3444u) * sc[4 * h + 3];
-        const __nv_bfloat162 b01 = __floats2bfloat162_rn(f0, f1);
-        const __nv_bfloat162 b23 = __floats2bfloat162_rn(f2, f3);
-        o[2 * h] = *reinterpret_cast<const uint32_t*>(&b01);
-        o[2 * h + 1] = *reinterpret_cast<const uint32_t*>(&b23);
-    }
-    return make_uint4(o[0], o[1], o[2], o[3]);
+// 8 E4M3 codes (little-endian in a uint2) -> 8 bf16 values.
+__device__ __forceinline__ uint4 e4m3x8_to_bf16(uint2 raw) {
+    return make_uint4(e4m3x2_to_bf16x2(raw.x, 0x1404u), e4m3x2_to_bf16x2(raw.x, 0x3424u),
+                      e4m3x2_to_bf16x2(raw.y, 0x1404u), e4m3x2_to_bf16x2(raw.y, 0x3424u));
 }
 
 __device__ __forceinline__ void fence_proxy_async_smem() {
@@ -470,21 +461,6 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(GemmCfg<MODE, ET, FP
         bool ok = true;
         for (int L = pair; L < total && ok; L += npairs) {
             const TileInfo ti = decode_tile<MODE, C::BK, C::BYTES>(*tab, args, L);
-            const int acol0 = (MODE == MODE_GATEUP) ? ti.f0 + 64 * (int)rank : ti.f0 + 128 * (int)rank;
-            // this tile's per-column scales for my 2 x 8 features
-            float sc[2][8];
-            {
-                const float* sv = args.wscale[ti.expert];
-#pragma unroll
-                for (int j = 0; j < 2; ++j) {
-                    const int col = ((MODE == MODE_GATEUP) ? (j == 0 ? acol0 : ti.up_off + acol0)
-                                                           : acol0 + 64 * j) + 8 * c8;
-                    const int mcol = (MODE == MODE_GATEUP) ? (j == 0 ? ti.M : ti.up_off + ti.M)
-                                                           : ti.M;  // columns of this weight
-#pragma unroll
-                    for (int i = 0; i < 8; ++i) sc[j][i] = (col + i < mcol) ? sv[col + i] : 0.f;
-                }
-            }
             for (int kb = ti.kb0; kb < ti.kb1; ++kb) {
                 const bool got = mbar_wait(rawfull_bar(stage), phase, args.err, DEV_ERR_TIMEOUT_PRODUCER);
                 if (!__all_sync(0xffffffffu, got)) {
@@ -501,7 +477,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(GemmCfg<MODE, ET, FP
                     const int j = (i * NCT) >> 9, kr = ((ct >> 3) + (NCT / 8) * i) & 63;
                     const uint2 q8 = *reinterpret_cast<const uint2*>(raw + j * 4096 + kr * 64 + c8 * 8);
                     *reinterpret_cast<uint4*>(a + j * 8192 + kr * 128 + ((c8 ^ (kr & 7)) << 4)) =
-                        e4m3x8_scaled_to_bf16(q8, sc[j]);
+                        e4m3x8_to_bf16(q8);
                 }
                 fence_proxy_async_smem();  // generic-proxy writes -> tensor-core reads
                 __syncwarp();
@@ -535,6 +511,16 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(GemmCfg<MODE, ET, FP
             const long long ld = ti.shared ? args.ld_shared : args.ld_routed;
             const int32_t* rowmap = ti.shared ? args.rowmap_shared : args.rowmap_routed;
             const float* colscale = ti.shared ? nullptr : args.colscale_routed;
+            // E4M3 weights: the scale of this TMEM lane's weight column (lane =
+            // row of the A tile: gate/up [gate 64 | up 64] features, down 128)
+            float wsc = 1.0f;
+            if constexpr (FP8W) {
+                const int r = q * 32 + lane;
+                const int f = (MODE == MODE_GATEUP) ? ti.f0 + 64 * (int)rank + (r & 63)
+                                                    : ti.f0 + 128 * (int)rank + r;
+                const int wcol = (MODE == MODE_GATEUP && r >= 64) ? ti.up_off + f : f;
+                wsc = f < ti.M ? args.wscale[ti.expert][wcol] : 0.0f;
+            }
             if (args.partial_out) {
                 // split-K: store this split's fp32 partial; row = slot (gate/up) or
                 // token (down), column = the weight column of this TMEM lane
@@ -559,6 +545,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(GemmCfg<MODE, ET, FP
                     float v[32];
                     tmem_ld_32x32(tb + (uint32_t)c, v);
                     tmem_wait_ld();
+                    if constexpr (FP8W) {
+#pragma unroll
+                        for (int i = 0; i < 32; ++i) v[i] *= wsc;
+                    }
 #pragma unroll
                     for (int i = 0; i < 32; ++i) {
                         const int orow = __shfl_sync(0xffffffffu, my_row, i);
@@ -583,6 +573,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(GemmCfg<MODE, ET, FP
                 float v[32];
                 tmem_ld_32x32(tb + (uint32_t)c, v);
                 tmem_wait_ld();
+                if constexpr (FP8W) {
+#pragma unroll
+                    for (int i = 0; i < 32; ++i) v[i] *= wsc;
+                }
                 if constexpr (MODE == MODE_GATEUP) {
                     // lanes 0-63: gate rows, 64-127: up rows of the same 64 features.
                     // Gate warps (q 0,1) finish columns c..c+15, up warps (q 2,3)

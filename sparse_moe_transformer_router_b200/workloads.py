@@ -185,6 +185,40 @@ def generate(cfg: LayerConfig, seed: int = 0, device="cpu", experts=None) -> Lay
                        ss_gu if fp8 else None, ss_dn if fp8 else None)
 
 
+# E4M3 code sets for layers that exercise the weight widening: every finite
+# code (0x7F / 0xFF are NaN), and the zero and subnormal codes (exponent
+# field 0) alone.
+E4M3_FINITE_CODES = tuple(c for c in range(256) if c & 0x7F != 0x7F)
+E4M3_SUBNORMAL_CODES = tuple(range(0x00, 0x08)) + tuple(range(0x80, 0x88))
+
+
+def with_e4m3_codes(inp: LayerInputs, codes, scale: float, seed: int) -> LayerInputs:
+    """Replace an E4M3 layer's expert and shared weights by codes drawn
+    uniformly (seeded) from ``codes`` and set every column scale to ``scale``."""
+    assert inp.cfg.dtype == "fp8"
+    table = torch.tensor(codes, dtype=torch.uint8)
+
+    def draw(w, name, e):
+        if w is None:
+            return None
+        g = torch.Generator().manual_seed(_seed(seed, "codes:" + name, e))
+        i = torch.randint(0, table.numel(), tuple(w.shape), generator=g)
+        return table[i].view(torch.float8_e4m3fn).to(w.device)
+
+    def full(s):
+        return None if s is None else torch.full_like(s, scale)
+
+    inp.W_gate_up = [draw(w, "W_gate_up", e) for e, w in enumerate(inp.W_gate_up)]
+    inp.W_down = [draw(w, "W_down", e) for e, w in enumerate(inp.W_down)]
+    inp.Ws_gate_up = draw(inp.Ws_gate_up, "Ws_gate_up", -1)
+    inp.Ws_down = draw(inp.Ws_down, "Ws_down", -1)
+    inp.s_gate_up = [full(s) for s in inp.s_gate_up]
+    inp.s_down = [full(s) for s in inp.s_down]
+    inp.ss_gate_up = full(inp.ss_gate_up)
+    inp.ss_down = full(inp.ss_down)
+    return inp
+
+
 def to_storage_numpy(t: torch.Tensor | None) -> np.ndarray | None:
     """Host copy in storage form: float32 as is, bf16 as uint16 bit patterns,
     float8_e4m3fn as uint8 codes (marshalling only, no arithmetic)."""

@@ -8,8 +8,9 @@ import torch
 
 from parity_util import (check_outputs, check_routing, make_layer, oracle_routing, run_gpu,
                          sample_tokens)
-from sparse_moe_transformer_router_b200.workloads import (CONFIGS, DECODE_TOKENS, LayerConfig,
-                                                          generate)
+from sparse_moe_transformer_router_b200.workloads import (CONFIGS, DECODE_TOKENS,
+                                                          E4M3_FINITE_CODES, E4M3_SUBNORMAL_CODES,
+                                                          LayerConfig, generate, with_e4m3_codes)
 
 pytestmark = pytest.mark.gpu
 
@@ -51,6 +52,23 @@ def test_small_layer_matches_oracle(name):
     rep = check_routing(inp, r)
     ratio = check_outputs(inp, out, None, rep["same"])
     print(f"{name}: max|err|/rms = {ratio:.3e}, excluded {rep['excluded']}, flipped {rep['flipped']}")
+
+
+@pytest.mark.parametrize("codes,scale", [(E4M3_FINITE_CODES, 4e-4), (E4M3_SUBNORMAL_CODES, 20.0)],
+                         ids=["all_finite_codes", "subnormal_codes"])
+def test_e4m3_widening_is_exact_for_every_code(codes, scale):
+    """Weights drawn from every finite E4M3 code (or from the zero and
+    subnormal codes alone) with one column scale: the widening to bf16 is
+    exact and the scale meets the fp32 accumulator, so the layer meets the
+    bf16 tolerance, not just the E4M3 one (a flushed or mis-mapped code
+    class would break it)."""
+    cfg = LayerConfig("fp8_codes", 300, 256, 4, 256, 192, "fp8", wr_std=0.1)
+    inp = with_e4m3_codes(generate(cfg, seed=7, device="cuda"), codes, scale, seed=7)
+    layer = make_layer(inp)
+    out, r = run_gpu(layer, inp)
+    rep = check_routing(inp, r)
+    ratio = check_outputs(inp, out, None, rep["same"], tol=2e-2)
+    print(f"max|err|/rms = {ratio:.3e}")
 
 
 def test_zero_input_gives_zero_output_and_expert_zero():
