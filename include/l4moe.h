@@ -199,16 +199,20 @@ L4MOE_API l4moe_status l4moe_get_routing(const l4moe_handle *h, const int32_t **
  * bounded wait ran out) or L4MOE_ERR_CUDA.  Clears the word. */
 L4MOE_API l4moe_status l4moe_check_device_status(l4moe_handle *h, void *stream);
 
-/* Per-kernel timing.  While enabled, l4moe_forward records a CUDA event
- * before and after each kernel it launches, on the caller's stream, so the
- * durations are those of the real launches in place.  Kernel slots:
- * 0 router, 1 permute, 2 row copy, 3 gate/up GEMM, 4 down GEMM
- * (L4MOE_NUM_KERNELS).  l4moe_read_timing synchronises on the last recorded
+/* Per-kernel timing.  `mask` selects kernel slots (bit i = slot i; 0 turns
+ * timing off; L4MOE_TIME_ALL every slot; anything else: L4MOE_ERR_ARG).
+ * For each selected slot l4moe_forward records a CUDA event before and
+ * after the kernel(s) of that slot, on the caller's stream, so the durations
+ * are those of the real launches in place (every event pair adds a little
+ * to the step, so time only what is needed).  Kernel slots: 0 router,
+ * 1 permute, 2 row copy, 3 gate/up GEMM (+ its split-K finish), 4 down GEMM
+ * + finish (L4MOE_NUM_KERNELS).  l4moe_read_timing synchronises on the last recorded
  * event, adds every recorded pair to ms[slot] and launches[slot] (arrays of
  * at least L4MOE_NUM_KERNELS entries, accumulated into), and recycles the
  * events.  Returns L4MOE_ERR_CUDA if an event call fails. */
 #define L4MOE_NUM_KERNELS 5
-L4MOE_API l4moe_status l4moe_set_timing(l4moe_handle *h, int enable);
+#define L4MOE_TIME_ALL ((1 << L4MOE_NUM_KERNELS) - 1)
+L4MOE_API l4moe_status l4moe_set_timing(l4moe_handle *h, int mask);
 L4MOE_API l4moe_status l4moe_read_timing(l4moe_handle *h, double *ms, uint64_t *launches);
 L4MOE_API const char *l4moe_kernel_name(int slot);
 

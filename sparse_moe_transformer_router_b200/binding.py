@@ -230,8 +230,16 @@ class L4MoE:
     def check_device_status(self, stream=None):
         self._check(self._lib.l4moe_check_device_status(self._h, _stream_handle(stream)))
 
-    def set_timing(self, enable: bool):
-        self._check(self._lib.l4moe_set_timing(self._h, 1 if enable else 0))
+    def set_timing(self, kernels=True):
+        """Time every kernel (True), none (False), or the named kernels."""
+        if kernels is True:
+            mask = (1 << NUM_KERNELS) - 1
+        elif kernels is False or kernels is None:
+            mask = 0
+        else:
+            names = [self._lib.l4moe_kernel_name(i).decode() for i in range(NUM_KERNELS)]
+            mask = sum(1 << names.index(k) for k in kernels)
+        self._check(self._lib.l4moe_set_timing(self._h, mask))
 
     def read_timing(self) -> dict:
         """{kernel name: (total ms, launches)} recorded since the last read."""

@@ -203,8 +203,8 @@ struct l4moe_handle {
     cudaEvent_t ev_h2d[2] = {}, ev_comp[2] = {}, ev_d2h[2] = {};
     bool slot_used[2] = {false, false};
     int host_slot = 0;
-    // per-kernel event timing (l4moe_set_timing)
-    bool timing = false;
+    // per-kernel event timing (l4moe_set_timing): bit i times kernel slot i
+    unsigned timing = 0;
     std::vector<cudaEvent_t> ev_pool;             // recycled events
     std::vector<std::pair<int, std::pair<cudaEvent_t, cudaEvent_t>>> ev_pending;
 };
@@ -241,7 +241,7 @@ struct LaunchTimer {
     cudaStream_t st;
     cudaEvent_t a = nullptr, b = nullptr;
     LaunchTimer(l4moe_handle* h_, int slot_, cudaStream_t st_) : h(h_), slot(slot_), st(st_) {
-        if (h->timing && (a = take_event(h)) != nullptr) cudaEventRecord(a, st);
+        if ((h->timing >> slot_ & 1u) && (a = take_event(h)) != nullptr) cudaEventRecord(a, st);
     }
     void stop() {
         if (a && (b = take_event(h)) != nullptr) {
@@ -692,8 +692,8 @@ l4moe_status l4moe_forward_static(l4moe_handle* h, int T, const void* x, const v
     if (e != cudaSuccess) return cuda_fail(h, e, "static descriptor upload");
     e = cudaMemsetAsync(base + ws_layout(h->p, T, h->sms).err, 0, sizeof(unsigned), st);
     if (e != cudaSuccess) return cuda_fail(h, e, "static error word clear");
-    const bool timing = h->timing;  // event timing would create events: off here
-    h->timing = false;
+    const unsigned timing = h->timing;  // event timing would create events: off here
+    h->timing = 0;
     if (h->p.dtype == L4MOE_F32)
         s = run_layer<float>(h, T, x, W_router, Ws_gate_up, Ws_down, out, st, base, T, maps);
     else
@@ -917,9 +917,9 @@ l4moe_status l4moe_check_device_status(l4moe_handle* h, void* stream) {
     return fail(h, (word & 7u) ? L4MOE_ERR_TIMEOUT : L4MOE_ERR_ARG, msg);
 }
 
-l4moe_status l4moe_set_timing(l4moe_handle* h, int enable) {
-    if (!h) return L4MOE_ERR_ARG;
-    h->timing = enable != 0;
+l4moe_status l4moe_set_timing(l4moe_handle* h, int mask) {
+    if (!h || mask < 0 || mask >= (1 << L4MOE_NUM_KERNELS)) return L4MOE_ERR_ARG;
+    h->timing = (unsigned)mask;
     return L4MOE_OK;
 }
 
