@@ -15,6 +15,7 @@
 #include <cstring>
 #include <mutex>
 #include <string>
+#include <utility>
 #include <vector>
 
 #include "l4moe.h"
@@ -234,6 +235,27 @@ cudaEvent_t take_event(l4moe_handle* h) {
     return e;
 }
 
+// Every kernel goes out with programmatic stream serialisation: it may begin
+// launching while the previous kernel of the stream finishes, and waits for
+// it (pdl_enter) before touching memory, which hides the launch gaps of the
+// short kernels of a small batch.  Launch errors are left for
+// cudaGetLastError, like a <<<>>> launch.
+template <typename... KArgs, typename... Args>
+void launch_k(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t st,
+              Args&&... args) {
+    cudaLaunchConfig_t cfg{};
+    cfg.gridDim = grid;
+    cfg.blockDim = block;
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = st;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    cudaLaunchKernelEx(&cfg, kernel, std::forward<Args>(args)...);
+}
+
 // Event pair around one launch when timing is enabled.
 struct LaunchTimer {
     l4moe_handle* h;
@@ -353,9 +375,9 @@ void launch_router_t(const void* x, const void* Wr, const float* bias, int T, in
     std::call_once(once, [] { set_smem_attr(router_kernel<ET, NT, TPT, NG>, smem); });
     const int TT = NT / TPT;
     const int wr_vec = (E % Vec16<ET>::N) == 0 ? 1 : 0;
-    router_kernel<ET, NT, TPT, NG><<<(T + TT - 1) / TT, NT, smem, st>>>(
-        static_cast<const ET*>(x), static_cast<const ET*>(Wr), bias, T, d, E, wr_vec, idx, gate,
-        lmax, margin);
+    launch_k(router_kernel<ET, NT, TPT, NG>, dim3((T + TT - 1) / TT), dim3(NT), smem, st,
+             static_cast<const ET*>(x), static_cast<const ET*>(Wr), bias, T, d, E, wr_vec, idx, gate,
+             lmax, margin);
 }
 
 template <typename ET>
@@ -376,7 +398,7 @@ void launch_gemm(int grid, const BMaps& bm, const GemmArgs& a, cudaStream_t st) 
     using Cfg = GemmCfg<MODE, ET, FP8W>;
     static std::once_flag once;
     std::call_once(once, [] { set_smem_attr(moe_gemm_kernel<MODE, ET, FP8W>, Cfg::SMEM_BYTES); });
-    moe_gemm_kernel<MODE, ET, FP8W><<<grid, Cfg::THREADS, Cfg::SMEM_BYTES, st>>>(bm, a);
+    launch_k(moe_gemm_kernel<MODE, ET, FP8W>, dim3(grid), dim3(Cfg::THREADS), Cfg::SMEM_BYTES, st, bm, a);
 }
 
 // The launch sequence of one forward.  w / ws_tokens: the workspace and the
@@ -446,8 +468,9 @@ l4moe_status run_layer(l4moe_handle* h, int T, const void* x, const void* Wr, co
         const int n_chunk = split_router ? 16 : E;
         const int kslices = split_router ? std::min(kRouterKSplit, std::max(1, d / 256)) : 1;
         router_logit_splits = kslices;
-        router_mma_kernel<<<dim3((T + 127) / 128, E / n_chunk, kslices), 128, rmma::SMEM_BYTES, st>>>(
-            m_x, m_wr, h->bias, T, d, E, n_chunk, logits, idx, gate, lmax, margin, err);
+        launch_k(router_mma_kernel, dim3((T + 127) / 128, E / n_chunk, kslices), dim3(128),
+                 rmma::SMEM_BYTES, st, m_x, m_wr, (const float*)h->bias, T, d, E, n_chunk, logits, idx,
+                 gate, lmax, margin, err);
     } else {
         launch_router<ET>(x, Wr, h->bias, T, d, E, idx, gate, lmax, margin, st);
     }
@@ -464,16 +487,16 @@ l4moe_status run_layer(l4moe_handle* h, int T, const void* x, const void* Wr, co
     const int s_gu = plan.s_gu, s_dn = plan.s_dn;
     const size_t psmem = sizeof(int) * (34 * (size_t)E + 1);
     LaunchTimer t_perm(h, 1, st);
-    permute_kernel<<<1, 1024, psmem, st>>>(logits, router_logit_splits, gate, lmax, margin, idx, T, E,
-                                           fb_gu_r * s_gu, fb_gu_s * s_gu, fb_dn * s_dn, counts,
-                                           offsets, perm, inv, tab_gu, tab_dn, err);
+    launch_k(permute_kernel, dim3(1), dim3(1024), psmem, st, (const float*)logits, router_logit_splits,
+             gate, lmax, margin, idx, T, E, fb_gu_r * s_gu, fb_gu_s * s_gu, fb_dn * s_dn, counts, offsets,
+             perm, inv, tab_gu, tab_dn, err);
     t_perm.stop();
     L4MOE_CHECK_LAUNCH("permute launch");
 
     const int sc_blocks = std::min((T + 7) / 8, h->sms * 8);
     LaunchTimer t_rows(h, 2, st);
-    permute_rows_kernel<ET><<<sc_blocks, 256, 0, st>>>(static_cast<const ET*>(x), gate, inv, T, d,
-                                                        xg, gslot);
+    launch_k(permute_rows_kernel<ET>, dim3(sc_blocks), dim3(256), 0, st, static_cast<const ET*>(x),
+             (const float*)gate, (const int32_t*)inv, T, d, xg, gslot);
     t_rows.stop();
     L4MOE_CHECK_LAUNCH("row permutation launch");
 
@@ -517,9 +540,10 @@ l4moe_status run_layer(l4moe_handle* h, int T, const void* x, const void* Wr, co
         bm_gu, gu, st);
     if (s_gu > 1) {
         const long long n = (long long)T * (F + Fs);
-        gateup_finish_kernel<ET><<<(int)std::min<long long>((n + 255) / 256, 4LL * h->sms), 256, 0, st>>>(
-            gu.part_routed, gu.ld_part_routed, gu.part_stride_routed, gu.part_shared, gu.ld_part_shared,
-            gu.part_stride_shared, s_gu, T, F, Fs, gslot, hr, hs);
+        launch_k(gateup_finish_kernel<ET>, dim3((int)std::min<long long>((n + 255) / 256, 4LL * h->sms)),
+                 dim3(256), 0, st, (const float*)gu.part_routed, gu.ld_part_routed, gu.part_stride_routed,
+                 (const float*)gu.part_shared, gu.ld_part_shared, gu.part_stride_shared, s_gu, T, F, Fs,
+                 (const float*)gslot, hr, hs);
         ++h->launches;
     }
     t_gu.stop();
@@ -556,8 +580,9 @@ l4moe_status run_layer(l4moe_handle* h, int T, const void* x, const void* Wr, co
                                      bm_dn, dn, st);
     {
         const long long n = (long long)T * d;
-        down_finish_kernel<ET><<<(int)std::min<long long>((n / 4 + 255) / 256, 4LL * h->sms), 256, 0, st>>>(
-            part, dn.part_stride_routed, 2 * s_dn, n, static_cast<ET*>(out));
+        launch_k(down_finish_kernel<ET>, dim3((int)std::min<long long>((n / 4 + 255) / 256, 4LL * h->sms)),
+                 dim3(256), 0, st, (const float*)part, dn.part_stride_routed, 2 * s_dn, n,
+                 static_cast<ET*>(out));
         ++h->launches;
     }
     t_dn.stop();

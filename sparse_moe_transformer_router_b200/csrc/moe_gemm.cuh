@@ -238,6 +238,7 @@ struct BMaps {
 template <int MODE, typename ET, bool FP8W>
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(GemmCfg<MODE, ET, FP8W>::THREADS, 1)
     moe_gemm_kernel(const __grid_constant__ BMaps bm, const GemmArgs args) {
+    pdl_enter();
     using Cfg = GemmCfg<MODE, ET, FP8W>;
     using C = ElemCfg<ET>;
     extern __shared__ uint8_t smem_raw[];
@@ -643,6 +644,7 @@ __global__ void __launch_bounds__(256) gateup_finish_kernel(
     const float* __restrict__ part_r, long long ld_r, long long stride_r, const float* __restrict__ part_s,
     long long ld_s, long long stride_s, int ksplit, int T, int F, int Fs,
     const float* __restrict__ gslot, ET* __restrict__ hr, ET* __restrict__ hs) {
+    pdl_enter();
     const long long n_r = (long long)T * F, n = n_r + (long long)T * Fs;
     for (long long i = blockIdx.x * (long long)blockDim.x + threadIdx.x; i < n;
          i += (long long)gridDim.x * blockDim.x) {
@@ -668,6 +670,7 @@ __global__ void __launch_bounds__(256) gateup_finish_kernel(
 template <typename ET>
 __global__ void __launch_bounds__(256) down_finish_kernel(const float* __restrict__ part, long long stride,
                                                           int nparts, long long n, ET* __restrict__ out) {
+    pdl_enter();
     const long long n4 = n >> 2;
     for (long long i = blockIdx.x * (long long)blockDim.x + threadIdx.x; i < n4;
          i += (long long)gridDim.x * blockDim.x) {

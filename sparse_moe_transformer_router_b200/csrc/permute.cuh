@@ -124,6 +124,7 @@ __global__ void __launch_bounds__(1024) permute_kernel(const float* __restrict__
                                                        int32_t* __restrict__ inv,
                                                        GroupTable* tab_gu, GroupTable* tab_dn,
                                                        unsigned* err) {
+    pdl_enter();
     extern __shared__ int psm[];
     int* wcnt = psm;              // [32][E]
     int* running = psm + 32 * E;  // [E]
@@ -263,6 +264,7 @@ __global__ void __launch_bounds__(256) permute_rows_kernel(const ET* __restrict_
                                                            const int32_t* __restrict__ inv,
                                                            int T, int d, ET* __restrict__ xp,
                                                            float* __restrict__ gate_slot) {
+    pdl_enter();
     const int lane = threadIdx.x & 31;
     const int warps = (gridDim.x * blockDim.x) >> 5;
     for (int t = (blockIdx.x * blockDim.x + threadIdx.x) >> 5; t < T; t += warps) {

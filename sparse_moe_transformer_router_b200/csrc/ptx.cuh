@@ -100,6 +100,17 @@ __device__ __forceinline__ bool mbar_wait_cluster(uint32_t bar, uint32_t parity,
     return true;
 }
 
+// ---------------------------------------------------------------- launches
+// Programmatic dependent launch: wait until the previous kernel of the stream
+// has finished and its writes are visible, then let the next kernel start
+// launching (its blocks run up to their own wait).  Every kernel of the layer
+// calls this first, before any global memory access, so the chain stays
+// ordered.  Both instructions are no-ops without the launch attribute.
+__device__ __forceinline__ void pdl_enter() {
+    asm volatile("griddepcontrol.wait;" ::: "memory");
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+
 // ---------------------------------------------------------------- clusters
 __device__ __forceinline__ uint32_t cluster_ctarank() {
     uint32_t r;

@@ -67,6 +67,7 @@ __global__ void __launch_bounds__(NT) router_kernel(const ET* __restrict__ x,
                                                     float* __restrict__ gate,
                                                     float* __restrict__ lmax,
                                                     float* __restrict__ margin) {
+    pdl_enter();
     constexpr int TT = NT / TPT;
     constexpr int EPAD = 4 * TPT * NG;
     constexpr int XLD = kRouterKC + 1;
@@ -207,6 +208,7 @@ __global__ void __launch_bounds__(128, 1)
                       float* __restrict__ logits, int32_t* __restrict__ idx,
                       float* __restrict__ gate, float* __restrict__ lmax,
                       float* __restrict__ margin, unsigned* err) {
+    pdl_enter();
     extern __shared__ uint8_t rsmem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>(
         (reinterpret_cast<uintptr_t>(rsmem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
