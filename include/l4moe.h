@@ -32,6 +32,10 @@
  *   L4MOE_BF16      every tensor bf16 (bf16 MMA, fp32 accumulate)
  *   L4MOE_FP8_E4M3  expert and shared weights OCP E4M3 with one fp32 scale per
  *                   output column (l4moe_set_fp8_scales); x, W_router, out bf16.
+ *                   The expert contractions run in f16 (kind::f16 MMA, fp32
+ *                   accumulate): weights widened exactly, x and the hidden
+ *                   rows held in f16 (exact for bf16 values of magnitude in
+ *                   [2^-14, 65504]), the column scale applied in fp32.
  *
  * Ownership: the caller owns every tensor, the scale vectors, the bias and
  * the stream.  The handle owns only its workspace (unless the caller supplies
@@ -166,7 +170,8 @@ L4MOE_API l4moe_status l4moe_forward_host(l4moe_handle *h, int T, const void *x_
  * layer do not fit in the scratch area: it holds the device part of the
  * workspace (l4moe_workspace_size without the host-path staging slots,
  * rounded up to 256 bytes) plus 2(E+1) TMA descriptors of 128 bytes, e.g.
- * about 390 tokens at d_model 5120 and F = Fs = 8192.  Every call, from any
+ * about 390 tokens at d_model 5120 and F = Fs = 8192 in bf16 (E4M3 layers
+ * also keep x in f16 there: about 350 tokens).  Every call, from any
  * handle, shares the one array: calls
  * whose work overlaps on the GPU (other streams, other threads) race and
  * corrupt each other; serialise them.  The array keeps the last call's

@@ -70,7 +70,7 @@ constexpr int kRouterKSplit = 8;
 
 struct WsLayout {
     size_t err, idx, gate, lmax, margin, inv, perm, gslot, counts, offsets, tab_gu, tab_dn, xg, hr,
-        hs, part, logits, xin, xout;
+        hs, x16, part, logits, xin, xout;
     size_t device_total;  // everything l4moe_forward uses
     size_t total;         // plus the host-path staging slots (last)
 };
@@ -159,6 +159,8 @@ WsLayout ws_layout(const l4moe_params& p, int T, int sms) {
     L.xg = take(t * p.d_model * es);
     L.hr = take(t * p.expert_ffn * es);
     L.hs = take(t * p.shared_ffn * es);
+    // E4M3 layers: x in f16, token order (the shared expert's operand)
+    L.x16 = take(p.dtype == L4MOE_FP8_E4M3 ? t * p.d_model * 2 : 0);
     L.part = take(sizeof(float) * part_floats(p, (int)t, sms));
     L.logits = take(sizeof(float) * kRouterKSplit * std::min<size_t>(t, 128) * E);  // split router
     L.device_total = off;
@@ -423,27 +425,37 @@ l4moe_status run_layer(l4moe_handle* h, int T, const void* x, const void* Wr, co
     int32_t* offsets = reinterpret_cast<int32_t*>(w + L.offsets);
     GroupTable* tab_gu = reinterpret_cast<GroupTable*>(w + L.tab_gu);
     GroupTable* tab_dn = reinterpret_cast<GroupTable*>(w + L.tab_dn);
-    ET* xg = reinterpret_cast<ET*>(w + L.xg);
-    ET* hr = reinterpret_cast<ET*>(w + L.hr);
-    ET* hs = reinterpret_cast<ET*>(w + L.hs);
+    // the GEMMs' activation type: the layer's, or f16 for E4M3 weights
+    // (widened exactly to f16; kind::f16 wants both operands of one type)
+    using GT = typename GemmAct<ET, FP8W>::type;
+    GT* xg = reinterpret_cast<GT*>(w + L.xg);
+    GT* hr = reinterpret_cast<GT*>(w + L.hr);
+    GT* hs = reinterpret_cast<GT*>(w + L.hs);
+    GT* x16 = reinterpret_cast<GT*>(w + L.x16);
 
     // per-call activation descriptors (K-major rows of 128 B): the router's
     // x (64-row boxes) and the GEMMs' token operands (full- and small-tile
     // boxes: gate/up reads x in expert order and x, down reads H_r and H_s)
-    const CUtensorMapDataType adt =
-        sizeof(ET) == 4 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT32 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16;
+    auto tmap_type = [](size_t bytes, bool f16) {
+        return bytes == 4 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT32
+                          : f16 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT16 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16;
+    };
+    const CUtensorMapDataType adt = tmap_type(sizeof(ET), false);
+    const CUtensorMapDataType gdt = tmap_type(sizeof(GT), FP8W);
     const uint32_t bk = (uint32_t)(128 / sizeof(ET));
     using GCfg = GemmCfg<MODE_GATEUP, ET, FP8W>;
     constexpr uint32_t rb = GCfg::B_BOX_ROWS, rs = GCfg::B_SMALL_ROWS;
     CUtensorMap m_x;
     BMaps bm_gu, bm_dn;
-    auto act = [&](CUtensorMap* m, const void* base, int width, uint32_t rows) {
-        return encode_2d(m, adt, base, (uint64_t)width, (uint64_t)T, (uint64_t)width * sizeof(ET), bk, rows);
+    auto act = [&](CUtensorMap* m, CUtensorMapDataType dt, const void* base, int width, uint32_t rows) {
+        return encode_2d(m, dt, base, (uint64_t)width, (uint64_t)T, (uint64_t)width * sizeof(ET), bk, rows);
     };
-    if (!act(&m_x, x, d, 64) || !act(&bm_gu.routed, xg, d, rb) || !act(&bm_gu.routed_small, xg, d, rs) ||
-        !act(&bm_gu.shared, x, d, rb) || !act(&bm_gu.shared_small, x, d, rs) ||
-        !act(&bm_dn.routed, hr, F, rb) || !act(&bm_dn.routed_small, hr, F, rs) ||
-        !act(&bm_dn.shared, hs, Fs, rb) || !act(&bm_dn.shared_small, hs, Fs, rs))
+    const void* xs = FP8W ? (const void*)x16 : x;  // the shared expert's operand
+    if (!act(&m_x, adt, x, d, 64) || !act(&bm_gu.routed, gdt, xg, d, rb) ||
+        !act(&bm_gu.routed_small, gdt, xg, d, rs) || !act(&bm_gu.shared, gdt, xs, d, rb) ||
+        !act(&bm_gu.shared_small, gdt, xs, d, rs) || !act(&bm_dn.routed, gdt, hr, F, rb) ||
+        !act(&bm_dn.routed_small, gdt, hr, F, rs) || !act(&bm_dn.shared, gdt, hs, Fs, rb) ||
+        !act(&bm_dn.shared_small, gdt, hs, Fs, rs))
         return fail(h, L4MOE_ERR_CUDA, "cuTensorMapEncodeTiled failed for an activation");
 
     cudaError_t e;
@@ -495,8 +507,8 @@ l4moe_status run_layer(l4moe_handle* h, int T, const void* x, const void* Wr, co
 
     const int sc_blocks = std::min((T + 7) / 8, h->sms * 8);
     LaunchTimer t_rows(h, 2, st);
-    launch_k(permute_rows_kernel<ET>, dim3(sc_blocks), dim3(256), 0, st, static_cast<const ET*>(x),
-             (const float*)gate, (const int32_t*)inv, T, d, xg, gslot);
+    launch_k(permute_rows_kernel<ET, GT>, dim3(sc_blocks), dim3(256), 0, st, static_cast<const ET*>(x),
+             (const float*)gate, (const int32_t*)inv, T, d, xg, gslot, FP8W ? x16 : (GT*)nullptr);
     t_rows.stop();
     L4MOE_CHECK_LAUNCH("row permutation launch");
 
@@ -540,7 +552,7 @@ l4moe_status run_layer(l4moe_handle* h, int T, const void* x, const void* Wr, co
         bm_gu, gu, st);
     if (s_gu > 1) {
         const long long n = (long long)T * (F + Fs);
-        launch_k(gateup_finish_kernel<ET>, dim3((int)std::min<long long>((n + 255) / 256, 4LL * h->sms)),
+        launch_k(gateup_finish_kernel<GT>, dim3((int)std::min<long long>((n + 255) / 256, 4LL * h->sms)),
                  dim3(256), 0, st, (const float*)gu.part_routed, gu.ld_part_routed, gu.part_stride_routed,
                  (const float*)gu.part_shared, gu.ld_part_shared, gu.part_stride_shared, s_gu, T, F, Fs,
                  (const float*)gslot, hr, hs);

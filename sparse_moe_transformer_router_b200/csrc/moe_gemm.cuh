@@ -54,6 +54,7 @@
 // copies and MMAs in flight before the pair synchronises and frees TMEM.
 #pragma once
 #include <cuda_bf16.h>
+#include <cuda_fp16.h>
 #include <cstdint>
 
 #include "permute.cuh"
@@ -198,26 +199,33 @@ __device__ __forceinline__ TileInfo decode_tile(const GroupTable& tab, const Gem
 
 __device__ __forceinline__ float silu_f(float z) { return __fdividef(z, 1.0f + __expf(-z)); }
 
-// 2 E4M3 codes -> 2 bf16, exactly (bf16 has the wider exponent and
-// mantissa).  A byte permute puts code i in bits 15..8 of 16-bit lane i; the
-// sign stays at bit 15 and the 7 exponent/mantissa bits move to 10..4, which
-// read as bf16 is code * 2^-120 (the E4M3 exponent bias is 7, bf16's 127),
-// subnormal codes becoming bf16 subnormals.  One packed bf16 multiply by
-// 2^120 restores the value (exact: a power of two, results in range).  The
+// 8 E4M3 codes (little-endian in a uint2) -> 8 f16 values, exactly (every
+// E4M3 value, subnormals included, is an f16 value), with the hardware
+// conversion (two codes per instruction, element order kept).  The
 // per-column scale is applied to the fp32 accumulator in the epilogue.
-__device__ __forceinline__ uint32_t e4m3x2_to_bf16x2(uint32_t w, uint32_t sel) {
-    const uint32_t t = __byte_perm(w, 0u, sel);  // code_i << 8 in lane i
-    const uint32_t bits = (t & 0x80008000u) | ((t >> 4) & 0x07F007F0u);
+__device__ __forceinline__ uint32_t e4m3x2_to_f16x2(uint32_t two_codes) {
     uint32_t r;
-    asm("mul.rn.bf16x2 %0, %1, %2;" : "=r"(r) : "r"(bits), "r"(0x7B807B80u));  // 2^120 in each lane
+    asm("{\n\t.reg .b16 c;\n\tcvt.u16.u32 c, %1;\n\tcvt.rn.f16x2.e4m3x2 %0, c;\n\t}"
+        : "=r"(r)
+        : "r"(two_codes));
     return r;
 }
 
-// 8 E4M3 codes (little-endian in a uint2) -> 8 bf16 values.
-__device__ __forceinline__ uint4 e4m3x8_to_bf16(uint2 raw) {
-    return make_uint4(e4m3x2_to_bf16x2(raw.x, 0x1404u), e4m3x2_to_bf16x2(raw.x, 0x3424u),
-                      e4m3x2_to_bf16x2(raw.y, 0x1404u), e4m3x2_to_bf16x2(raw.y, 0x3424u));
+__device__ __forceinline__ uint4 e4m3x8_to_f16(uint2 raw) {
+    return make_uint4(e4m3x2_to_f16x2(raw.x & 0xFFFFu), e4m3x2_to_f16x2(raw.x >> 16),
+                      e4m3x2_to_f16x2(raw.y & 0xFFFFu), e4m3x2_to_f16x2(raw.y >> 16));
 }
+
+// The contractions' activation (token operand and hidden) type: the layer's
+// own, or f16 for E4M3 weights (kind::f16 takes both operands in one type).
+template <typename ET, bool FP8W>
+struct GemmAct {
+    using type = ET;
+};
+template <>
+struct GemmAct<__nv_bfloat16, true> {
+    using type = __half;
+};
 
 __device__ __forceinline__ void fence_proxy_async_smem() {
     asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
@@ -225,6 +233,7 @@ __device__ __forceinline__ void fence_proxy_async_smem() {
 
 __device__ __forceinline__ void store_elem(float* p, float v) { *p = v; }
 __device__ __forceinline__ void store_elem(__nv_bfloat16* p, float v) { *p = __float2bfloat16_rn(v); }
+__device__ __forceinline__ void store_elem(__half* p, float v) { *p = __float2half_rn(v); }
 
 // Token-operand (B) descriptors of the routed and the shared rows, with
 // 128-row boxes for tiles of more than 64 tokens per CTA and 32-row boxes
@@ -406,7 +415,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(GemmCfg<MODE, ET, FP
                 if (!mbar_wait_cluster(tempty_bar(acc), acc_phase ^ 1u, args.err, DEV_ERR_TIMEOUT_MMA))
                     break;
                 tc_fence_after();
-                const uint32_t idesc = make_idesc(C::FMT, 1u, 0u, (uint32_t)ti.n_mma, 256u);
+                // E4M3 layers: both operands f16 (format 0), else the layer's type
+                const uint32_t idesc = make_idesc(FP8W ? 0u : C::FMT, 1u, 0u, (uint32_t)ti.n_mma, 256u);
                 const uint32_t d_tmem = tmem_base + (uint32_t)acc * 256u;
                 bool ok = true;
                 for (int kb = ti.kb0; kb < ti.kb1; ++kb) {
@@ -478,7 +488,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(GemmCfg<MODE, ET, FP
                     const int j = (i * NCT) >> 9, kr = ((ct >> 3) + (NCT / 8) * i) & 63;
                     const uint2 q8 = *reinterpret_cast<const uint2*>(raw + j * 4096 + kr * 64 + c8 * 8);
                     *reinterpret_cast<uint4*>(a + j * 8192 + kr * 128 + ((c8 ^ (kr & 7)) << 4)) =
-                        e4m3x8_to_bf16(q8);
+                        e4m3x8_to_f16(q8);
                 }
                 fence_proxy_async_smem();  // generic-proxy writes -> tensor-core reads
                 __syncwarp();
@@ -508,7 +518,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(GemmCfg<MODE, ET, FP
             }
             tc_fence_after();
             const uint32_t tb = tmem_base + ((uint32_t)(q * 32) << 16) + (uint32_t)acc * 256u;
-            ET* outp = reinterpret_cast<ET*>(ti.shared ? args.out_shared : args.out_routed);
+            using OT = typename GemmAct<ET, FP8W>::type;  // hidden rows (gate/up's output)
+            OT* outp = reinterpret_cast<OT*>(ti.shared ? args.out_shared : args.out_routed);
             const long long ld = ti.shared ? args.ld_shared : args.ld_routed;
             const int32_t* rowmap = ti.shared ? args.rowmap_shared : args.rowmap_routed;
             const float* colscale = ti.shared ? nullptr : args.colscale_routed;

@@ -8,6 +8,7 @@
 // index (stable), so slot = offsets[e] + #{t' < t : idx[t'] == e}.
 #pragma once
 #include <cuda_bf16.h>
+#include <cuda_fp16.h>
 #include <cstdint>
 
 #include "ptx.cuh"
@@ -252,19 +253,36 @@ __global__ void __launch_bounds__(1024) permute_kernel(const float* __restrict__
     }
 }
 
-// Expert-ordered copy of the input rows, xp[inv[t]] = x[t] (exact), and the
-// gate of each slot, gate_slot[inv[t]] = gate[t].  The sigmoid gate scales
-// the routed expert's input, which is linear in the gate/up contraction, so
-// it is applied to the fp32 accumulator in the GEMM epilogue instead of
-// rounding g * x to the activation type here.
-// One warp per token row, 16-byte vectors; d % (16 / sizeof(ET)) == 0.
-template <typename ET>
-__global__ void __launch_bounds__(256) permute_rows_kernel(const ET* __restrict__ x,
+// Expert-ordered copy of the input rows, xp[inv[t]] = x[t], and the gate of
+// each slot, gate_slot[inv[t]] = gate[t].  The sigmoid gate scales the
+// routed expert's input, which is linear in the gate/up contraction, so it
+// is applied to the fp32 accumulator in the GEMM epilogue instead of
+// rounding g * x to the activation type here.  OT = IT copies exactly; for
+// E4M3 layers IT = bf16, OT = f16 (the contractions' operand type) and
+// x_tok (if not null) also receives the f16 rows in token order.
+// One warp per token row, 16-byte vectors; d % 8 == 0.
+__device__ __forceinline__ uint4 cvt_row_vec(uint4 v, __nv_bfloat16, __half) {
+    uint32_t w[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+        const float2 f = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&w[i]));
+        const __half2 hv = __floats2half2_rn(f.x, f.y);
+        w[i] = *reinterpret_cast<const uint32_t*>(&hv);
+    }
+    return make_uint4(w[0], w[1], w[2], w[3]);
+}
+template <typename T>
+__device__ __forceinline__ uint4 cvt_row_vec(uint4 v, T, T) { return v; }
+
+template <typename IT, typename OT>
+__global__ void __launch_bounds__(256) permute_rows_kernel(const IT* __restrict__ x,
                                                            const float* __restrict__ gate,
                                                            const int32_t* __restrict__ inv,
-                                                           int T, int d, ET* __restrict__ xp,
-                                                           float* __restrict__ gate_slot) {
+                                                           int T, int d, OT* __restrict__ xp,
+                                                           float* __restrict__ gate_slot,
+                                                           OT* __restrict__ x_tok) {
     pdl_enter();
+    static_assert(sizeof(IT) == sizeof(OT), "row copy keeps the element size");
     const int lane = threadIdx.x & 31;
     const int warps = (gridDim.x * blockDim.x) >> 5;
     for (int t = (blockIdx.x * blockDim.x + threadIdx.x) >> 5; t < T; t += warps) {
@@ -272,8 +290,13 @@ __global__ void __launch_bounds__(256) permute_rows_kernel(const ET* __restrict_
         if (lane == 0) gate_slot[slot] = gate[t];
         const uint4* s = reinterpret_cast<const uint4*>(x + (size_t)t * d);
         uint4* o = reinterpret_cast<uint4*>(xp + (size_t)slot * d);
-        const int nv = d * (int)sizeof(ET) / 16;
-        for (int i = lane; i < nv; i += 32) o[i] = s[i];
+        uint4* ot = x_tok ? reinterpret_cast<uint4*>(x_tok + (size_t)t * d) : nullptr;
+        const int nv = d * (int)sizeof(IT) / 16;
+        for (int i = lane; i < nv; i += 32) {
+            const uint4 v = cvt_row_vec(s[i], IT{}, OT{});
+            o[i] = v;
+            if (ot) ot[i] = v;
+        }
     }
 }
 
