@@ -242,20 +242,34 @@ cudaEvent_t take_event(l4moe_handle* h) {
 // it (pdl_enter) before touching memory, which hides the launch gaps of the
 // short kernels of a small batch.  Launch errors are left for
 // cudaGetLastError, like a <<<>>> launch.
+// cluster_z > 0 also launches the grid as clusters of (1, 1, cluster_z).
 template <typename... KArgs, typename... Args>
-void launch_k(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t st,
-              Args&&... args) {
+void launch_kc(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t st,
+               unsigned cluster_z, Args&&... args) {
     cudaLaunchConfig_t cfg{};
     cfg.gridDim = grid;
     cfg.blockDim = block;
     cfg.dynamicSmemBytes = smem;
     cfg.stream = st;
-    cudaLaunchAttribute attr[1];
+    cudaLaunchAttribute attr[2];
     attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
     attr[0].val.programmaticStreamSerializationAllowed = 1;
-    cfg.attrs = attr;
     cfg.numAttrs = 1;
+    if (cluster_z > 0) {
+        attr[1].id = cudaLaunchAttributeClusterDimension;
+        attr[1].val.clusterDim.x = 1;
+        attr[1].val.clusterDim.y = 1;
+        attr[1].val.clusterDim.z = cluster_z;
+        cfg.numAttrs = 2;
+    }
+    cfg.attrs = attr;
     cudaLaunchKernelEx(&cfg, kernel, std::forward<Args>(args)...);
+}
+
+template <typename... KArgs, typename... Args>
+void launch_k(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t st,
+              Args&&... args) {
+    launch_kc(kernel, grid, block, smem, st, 0u, std::forward<Args>(args)...);
 }
 
 // Event pair around one launch when timing is enabled.
@@ -478,11 +492,19 @@ l4moe_status run_layer(l4moe_handle* h, int T, const void* x, const void* Wr, co
         static std::once_flag once;
         std::call_once(once, [] { set_smem_attr(router_mma_kernel, rmma::SMEM_BYTES); });
         const int n_chunk = split_router ? 16 : E;
-        const int kslices = split_router ? std::min(kRouterKSplit, std::max(1, d / 256)) : 1;
-        router_logit_splits = kslices;
-        launch_k(router_mma_kernel, dim3((T + 127) / 128, E / n_chunk, kslices), dim3(128),
-                 rmma::SMEM_BYTES, st, m_x, m_wr, (const float*)h->bias, T, d, E, n_chunk, logits, idx,
-                 gate, lmax, margin, err);
+        const int tiles = (T + 127) / 128;
+        int kslices;
+        if (split_router) {
+            kslices = std::min(kRouterKSplit, std::max(1, d / 256));
+            router_logit_splits = kslices;
+        } else {
+            // few token tiles: K slices per tile (at most 4 and the SMs'
+            // worth), reduced inside a cluster of the slices
+            kslices = std::max(1, std::min({4, h->sms / tiles, d / 256}));
+        }
+        launch_kc(router_mma_kernel, dim3(tiles, E / n_chunk, kslices), dim3(128), rmma::SMEM_BYTES, st,
+                  split_router || kslices == 1 ? 0u : (unsigned)kslices, m_x, m_wr, (const float*)h->bias,
+                  T, d, E, n_chunk, logits, idx, gate, lmax, margin, err);
     } else {
         launch_router<ET>(x, Wr, h->bias, T, d, E, idx, gate, lmax, margin, st);
     }

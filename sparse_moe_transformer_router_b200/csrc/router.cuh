@@ -196,6 +196,15 @@ constexpr int STAGE_BYTES = A_BYTES + MAX_B_BOXES * B_BOX_BYTES;
 constexpr size_t SMEM_BYTES = 1024 + (size_t)STAGES * STAGE_BYTES + (2 * STAGES + 1) * 8 + 16;
 }  // namespace rmma
 
+// Cluster K-split mode (logits == null, gridDim.z = S > 1, launched as
+// clusters of (1, 1, S)): CTA z of a cluster computes the partial logits of
+// the same 128 tokens over K slice z and keeps them in its shared memory;
+// after a cluster barrier rank 0 adds ranks 1..S-1's partials to its own in
+// slice order (deterministic) and runs the arg-max epilogue.  This spreads
+// the x stream of a batch of few token tiles over S times more SMs.
+// Each CTA's partial (fp32, column-major [n_pad][128], at most 128 KB for
+// E = 256) reuses its own operand stages.
+//
 // Expert-split mode (logits != null, for batches of one token tile): CTA
 // (y, z) computes experts [y*n_chunk, (y+1)*n_chunk) over K slice z of
 // gridDim.z and stores the fp32 partial logits to logits[z][T][E] (the bias
@@ -295,7 +304,25 @@ __global__ void __launch_bounds__(128, 1)
     __syncwarp();
     // epilogue: thread = token row (TMEM lane 32*warp + lane)
     const bool ok = mbar_wait(done_bar, 0, err, DEV_ERR_TIMEOUT_EPILOGUE);
-    if (__all_sync(0xffffffffu, ok)) {
+    const bool kreduce = !logits && gridDim.z > 1;
+    const uint32_t crank = kreduce ? cluster_ctarank() : 0u;
+    float* red = reinterpret_cast<float*>(smem);  // this CTA's partial, [n_pad][128] (column-major)
+    if (kreduce) {
+        // every CTA reaches both cluster barriers, whatever its waits gave
+        if (crank != 0 && __all_sync(0xffffffffu, ok)) {
+            tc_fence_after();
+            for (int c = 0; c < n_pad; c += 32) {
+                float v[32];
+                tmem_ld_32x32(tmem_base + ((uint32_t)(32 * warp) << 16) + (uint32_t)c, v);
+                tmem_wait_ld();
+#pragma unroll
+                for (int i = 0; i < 32; ++i)
+                    if (c + i < n_pad) red[(c + i) * 128 + 32 * warp + lane] = v[i];
+            }
+        }
+        cluster_sync();  // partials of ranks 1..S-1 complete in their shared memory
+    }
+    if ((!kreduce || crank == 0) && __all_sync(0xffffffffu, ok)) {
         tc_fence_after();
         const int t = t0 + 32 * warp + lane;
         if (logits) {
@@ -318,6 +345,13 @@ __global__ void __launch_bounds__(128, 1)
             float v[32];
             tmem_ld_32x32(tmem_base + ((uint32_t)(32 * warp) << 16) + (uint32_t)c, v);
             tmem_wait_ld();
+            for (uint32_t z = 1; kreduce && z < gridDim.z; ++z) {  // slices in order
+                // a warp reads 32 consecutive rows of a column: 128 B per load
+                const uint32_t base = mapa_shared(smem_u32(red + c * 128 + 32 * warp + lane), z);
+#pragma unroll
+                for (int i = 0; i < 32; ++i)
+                    if (c + i < n_pad) v[i] += ld_shared_cluster_f32(base + 512u * i);
+            }
 #pragma unroll
             for (int i = 0; i < 32; ++i) {
                 const int e = c + i;
@@ -340,6 +374,7 @@ __global__ void __launch_bounds__(128, 1)
             gate[t] = 1.0f / (1.0f + expf(-best));
         }
     }
+    if (kreduce) cluster_sync();  // rank 0 done reading the others' shared memory
     tc_fence_before();
     __syncthreads();
     if (warp == 1) {

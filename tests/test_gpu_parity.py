@@ -40,6 +40,10 @@ SMALL = {
     "fp8_splitk": LayerConfig("fp8_splitk", 2, 1024, 8, 1024, 1024, "fp8", wr_std=0.03),
     "bf16_router_split": LayerConfig("bf16_router_split", 1, 1024, 64, 512, 512, "bf16", wr_std=0.03),
     "bf16_T40_E32": LayerConfig("bf16_T40_E32", 40, 512, 32, 512, 768, "bf16", wr_std=0.05),
+    # few token tiles and E < 32: the router splits K into 4 slices per token
+    # tile and reduces them inside a cluster (ragged last tile)
+    "bf16_router_kslices": LayerConfig("bf16_router_kslices", 700, 1024, 16, 256, 256, "bf16",
+                                       wr_std=0.03),
 }
 
 
