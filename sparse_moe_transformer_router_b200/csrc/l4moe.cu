@@ -65,7 +65,8 @@ bool encode_2d(CUtensorMap* m, CUtensorMapDataType dt, const void* base, uint64_
 // kMaxSplit k-ranges (tiles too few to fill the GPU, e.g. decode).
 constexpr size_t kSplitMaxTokens = 64;
 constexpr int kMaxSplit = 16;
-// The expert-split router (one token tile) also splits K into this many slices.
+// The expert-split router (one token tile) also splits K into this many
+// slices, one cluster of CTAs per 16-expert chunk.
 constexpr int kRouterKSplit = 8;
 
 struct WsLayout {
@@ -162,7 +163,7 @@ WsLayout ws_layout(const l4moe_params& p, int T, int sms) {
     // E4M3 layers: x in f16, token order (the shared expert's operand)
     L.x16 = take(p.dtype == L4MOE_FP8_E4M3 ? t * p.d_model * 2 : 0);
     L.part = take(sizeof(float) * part_floats(p, (int)t, sms));
-    L.logits = take(sizeof(float) * kRouterKSplit * std::min<size_t>(t, 128) * E);  // split router
+    L.logits = take(sizeof(float) * std::min<size_t>(t, 128) * E);  // expert-split router
     L.device_total = off;
     L.xin = take(2 * t * p.d_model * es);   // host path: two input staging slots
     L.xout = take(2 * t * p.d_model * es);  // and two output staging slots
@@ -483,7 +484,6 @@ l4moe_status run_layer(l4moe_handle* h, int T, const void* x, const void* Wr, co
     // one token tile and many experts: split the router over 16-expert chunks
     const bool split_router = sizeof(ET) == 2 && E % 16 == 0 && E >= 32 && T <= 128;
     float* logits = split_router ? reinterpret_cast<float*>(w + L.logits) : nullptr;
-    int router_logit_splits = 1;
     if (sizeof(ET) == 2 && E % 8 == 0) {
         // tensor-core router: W_router [d, E] as the MN-major operand
         CUtensorMap m_wr;
@@ -496,14 +496,13 @@ l4moe_status run_layer(l4moe_handle* h, int T, const void* x, const void* Wr, co
         int kslices;
         if (split_router) {
             kslices = std::min(kRouterKSplit, std::max(1, d / 256));
-            router_logit_splits = kslices;
         } else {
             // few token tiles: K slices per tile (at most 4 and the SMs'
             // worth), reduced inside a cluster of the slices
             kslices = std::max(1, std::min({4, h->sms / tiles, d / 256}));
         }
         launch_kc(router_mma_kernel, dim3(tiles, E / n_chunk, kslices), dim3(128), rmma::SMEM_BYTES, st,
-                  split_router || kslices == 1 ? 0u : (unsigned)kslices, m_x, m_wr, (const float*)h->bias,
+                  kslices == 1 ? 0u : (unsigned)kslices, m_x, m_wr, (const float*)h->bias,
                   T, d, E, n_chunk, logits, idx, gate, lmax, margin, err);
     } else {
         launch_router<ET>(x, Wr, h->bias, T, d, E, idx, gate, lmax, margin, st);
@@ -521,7 +520,7 @@ l4moe_status run_layer(l4moe_handle* h, int T, const void* x, const void* Wr, co
     const int s_gu = plan.s_gu, s_dn = plan.s_dn;
     const size_t psmem = sizeof(int) * (34 * (size_t)E + 1);
     LaunchTimer t_perm(h, 1, st);
-    launch_k(permute_kernel, dim3(1), dim3(1024), psmem, st, (const float*)logits, router_logit_splits,
+    launch_k(permute_kernel, dim3(1), dim3(1024), psmem, st, (const float*)logits,
              gate, lmax, margin, idx, T, E, fb_gu_r * s_gu, fb_gu_s * s_gu, fb_dn * s_dn, counts, offsets,
              perm, inv, tab_gu, tab_dn, err);
     t_perm.stop();

@@ -107,13 +107,11 @@ __host__ __device__ __forceinline__ int tile_at(int L, int heavy, int total) {
 //            down GEMM (the two contractions meet in fp32 partials)
 // smem: wcnt[32][E] + running[E] ints.
 //
-// logits != null (expert-split router): first finish the routing here -- per
-// token, sum the router's logit_splits partial logits [split][T][E] in
-// order, then the arg-max over the E biased fp32 logits (lowest index on ties,
-// NaN never wins), the runner-up margin and the sigmoid gate -- writing idx,
-// gate, lmax and margin.
+// logits != null (expert-split router, logits [T][E] biased fp32): first
+// finish the routing here -- per token, the arg-max over the E logits
+// (lowest index on ties, NaN never wins), the runner-up margin and the
+// sigmoid gate -- writing idx, gate, lmax and margin.
 __global__ void __launch_bounds__(1024) permute_kernel(const float* __restrict__ logits,
-                                                       int logit_splits,
                                                        float* __restrict__ gate,
                                                        float* __restrict__ lmax,
                                                        float* __restrict__ margin,
@@ -139,8 +137,7 @@ __global__ void __launch_bounds__(1024) permute_kernel(const float* __restrict__
             float best = -INFINITY, second = -INFINITY;
             int bi = 0x7fffffff;
             for (int e = lane; e < E; e += 32) {
-                float l = 0.f;  // the router's K-split partials, summed in order
-                for (int s = 0; s < logit_splits; ++s) l += logits[((size_t)s * T + t) * E + e];
+                const float l = logits[(size_t)t * E + e];
                 if (l > best) {
                     second = best;
                     best = l;

@@ -196,8 +196,8 @@ constexpr int STAGE_BYTES = A_BYTES + MAX_B_BOXES * B_BOX_BYTES;
 constexpr size_t SMEM_BYTES = 1024 + (size_t)STAGES * STAGE_BYTES + (2 * STAGES + 1) * 8 + 16;
 }  // namespace rmma
 
-// Cluster K-split mode (logits == null, gridDim.z = S > 1, launched as
-// clusters of (1, 1, S)): CTA z of a cluster computes the partial logits of
+// Cluster K-split (gridDim.z = S > 1, launched as clusters of (1, 1, S)):
+// CTA z of a cluster computes the partial logits of
 // the same 128 tokens over K slice z and keeps them in its shared memory;
 // after a cluster barrier rank 0 adds ranks 1..S-1's partials to its own in
 // slice order (deterministic) and runs the arg-max epilogue.  This spreads
@@ -207,9 +207,9 @@ constexpr size_t SMEM_BYTES = 1024 + (size_t)STAGES * STAGE_BYTES + (2 * STAGES 
 //
 // Expert-split mode (logits != null, for batches of one token tile): CTA
 // (y, z) computes experts [y*n_chunk, (y+1)*n_chunk) over K slice z of
-// gridDim.z and stores the fp32 partial logits to logits[z][T][E] (the bias
-// in slice 0); the sum over slices and the arg-max then run in the
-// permutation kernel.  This spreads the router weight stream over
+// gridDim.z; the slices meet in rank 0 of their cluster as above, which
+// stores the biased fp32 logits to logits[T][E]; the arg-max then runs in
+// the permutation kernel.  This spreads the router weight stream over
 // (E / n_chunk) x slices SMs instead of one.
 __global__ void __launch_bounds__(128, 1)
     router_mma_kernel(const __grid_constant__ CUtensorMap x_map, const __grid_constant__ CUtensorMap wr_map,
@@ -304,7 +304,7 @@ __global__ void __launch_bounds__(128, 1)
     __syncwarp();
     // epilogue: thread = token row (TMEM lane 32*warp + lane)
     const bool ok = mbar_wait(done_bar, 0, err, DEV_ERR_TIMEOUT_EPILOGUE);
-    const bool kreduce = !logits && gridDim.z > 1;
+    const bool kreduce = gridDim.z > 1;  // K slices: always launched as clusters along z
     const uint32_t crank = kreduce ? cluster_ctarank() : 0u;
     float* red = reinterpret_cast<float*>(smem);  // this CTA's partial, [n_pad][128] (column-major)
     if (kreduce) {
@@ -330,12 +330,16 @@ __global__ void __launch_bounds__(128, 1)
                 float v[32];
                 tmem_ld_32x32(tmem_base + ((uint32_t)(32 * warp) << 16) + (uint32_t)c, v);
                 tmem_wait_ld();
+                for (uint32_t z = 1; kreduce && z < gridDim.z; ++z) {  // slices in order
+                    const uint32_t base = mapa_shared(smem_u32(red + c * 128 + 32 * warp + lane), z);
+#pragma unroll
+                    for (int i = 0; i < 32; ++i)
+                        if (c + i < n_pad) v[i] += ld_shared_cluster_f32(base + 512u * i);
+                }
 #pragma unroll
                 for (int i = 0; i < 32; ++i) {
                     const int e = c + i;
-                    if (e < ne && t < T)
-                        logits[((size_t)blockIdx.z * T + t) * E + e0 + e] =
-                            v[i] + ((bias && blockIdx.z == 0) ? bias[e0 + e] : 0.f);
+                    if (e < ne && t < T) logits[(size_t)t * E + e0 + e] = v[i] + (bias ? bias[e0 + e] : 0.f);
                 }
             }
         }
