@@ -3,10 +3,12 @@
 //
 //   router -> permute (counts, scan, slots, work lists) -> copy of x into
 //   expert order -> grouped gate/up (shared expert + routed experts; gate and
-//   SwiGLU in the epilogue) -> grouped down (shared + routed contraction in
-//   one accumulator, un-permuted store)
+//   SwiGLU in the epilogue; + a finish kernel when split over K) -> grouped
+//   down (shared and routed results as fp32 partials, un-permuted) -> finish
+//   (sum, one rounding)
 //
-// all enqueued on the caller's stream with no host synchronisation.
+// all enqueued on the caller's stream with no host synchronisation, each
+// kernel launched with programmatic stream serialisation.
 #include <cuda.h>
 #include <cuda_runtime.h>
 

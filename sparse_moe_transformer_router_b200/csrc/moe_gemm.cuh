@@ -38,11 +38,21 @@
 // one tile overlaps the MMAs of the next.
 //
 // E4M3 weights (FP8W): TMA brings the raw 8-bit A tile (64 K rows x 2 slabs
-// of 64 features) into a raw ring; eight converter warps widen it to bf16,
-// multiplying each value by its output column's fp32 scale (one bf16
-// rounding of q * scale), write the swizzled MN-major operand layout, fence
-// to the async proxy and report to the leader; the MMA waits for the token
-// tile and for both CTAs' converted weights.
+// of 64 features) into a raw ring; eight converter warps widen it exactly to
+// f16, write the swizzled MN-major operand layout, fence to the async proxy
+// and report to the leader; the MMA (kind::f16, both operands f16: these
+// layers keep their token operand and hidden rows in f16) waits for the
+// token tile and for both CTAs' converted weights, and the epilogue
+// multiplies each accumulator row by its weight column's fp32 scale.
+//
+// Tiles: a group's tiles are (feature block) x (token tile) x (k range), the
+// token tiles of one feature block adjacent so that they share the weight
+// tile through L2, in bands whose token rows stay in L2 while the band
+// sweeps the feature blocks; compute-bound and weight-bound groups are
+// interleaved (tile_at); CTA pairs take tiles in stripes.  The token operand
+// arrives as one 128-row box per k-block for tiles of more than 64 tokens
+// per CTA (measured: a box's issue cost dominated with 64-row boxes), else
+// as 32-row boxes.
 //
 // Roles (192 threads per CTA, 448 with E4M3 weights): warp 0 lane 0 issues TMA loads into a
 // STAGES-deep ring (both CTAs; completion counted on the leader's barrier);
@@ -127,9 +137,7 @@ struct GemmCfg {
     static constexpr int A_BOXES = 128 / A_BOX_FEATS;        // boxes per CTA A tile
     static constexpr int A_BOX_BYTES = C::BK * 128;          // BK rows x 128 B
     static constexpr int B_BOX_ROWS = 128;                   // token rows per full-tile box
-    static constexpr int B_BOX_BYTES = B_BOX_ROWS * 128;
     static constexpr int B_SMALL_ROWS = 32;                  // token rows per small-tile box
-    static constexpr int B_SMALL_BYTES = B_SMALL_ROWS * 128;
     static constexpr int B_BYTES = (kTokTile / 2) * 128;     // this CTA's half of the tokens
     static constexpr int RAW_BYTES = FP8W ? 2 * 64 * 64 : 0; // 2 slabs x 64 K rows x 64 features
     static constexpr int STAGE_BYTES = A_BYTES + B_BYTES + RAW_BYTES;

@@ -6,6 +6,9 @@
 // section "What is unusual about the block": the chosen expert is reached
 // through a sigmoid gate on its input.
 //
+// Two routers: the tensor-core one further down (bf16 layers, E % 8 == 0)
+// and this CUDA-core one for the others (fp32 layers, other E).
+//
 // One CTA handles TT = NT / TPT tokens; TPT threads share a token and each
 // owns NG groups of 4 consecutive experts.  x and W_router are staged through
 // shared memory in K chunks of 64 and converted to fp32; each thread keeps
