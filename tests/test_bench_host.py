@@ -1,0 +1,60 @@
+"""Host-side logic of bench.py that needs no GPU: the per-kernel FLOP split,
+the parsing of committed ncu summaries, the weak-scaling value and the
+oracle's timed CPU sample."""
+import os
+import sys
+
+import numpy as np
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+sys.path.insert(0, ROOT)
+
+import bench  # noqa: E402
+from sparse_moe_transformer_router_b200 import accounting  # noqa: E402
+from sparse_moe_transformer_router_b200.workloads import CONFIGS, generate  # noqa: E402
+
+
+@pytest.mark.parametrize("name", ["scout_prefill_bf16", "maverick_prefill_bf16", "maverick_fp8"])
+def test_kernel_flops_add_up_to_the_layer(name):
+    cfg = CONFIGS[name]
+    counts = np.full(cfg.num_experts, cfg.T // cfg.num_experts)
+    k = bench.kernel_flops_bytes(cfg, counts)
+    total = sum(v["flops"] for v in k.values())
+    assert total == accounting.layer_flops(cfg.T, cfg.d_model, cfg.num_experts, cfg.expert_ffn,
+                                           cfg.shared_ffn)
+    # the weights each GEMM streams: touched routed experts plus the shared one
+    w = accounting.W_BYTES[cfg.dtype]
+    assert k["gemm_down"]["bytes"] >= (cfg.num_experts * cfg.expert_ffn + cfg.shared_ffn) * cfg.d_model * w
+
+
+def test_profile_traffic_needs_the_current_kernel_hash(tmp_path, monkeypatch):
+    (tmp_path / "profiles").mkdir()
+    path = tmp_path / "profiles" / "gemm_gate_up__w.md"
+    sha = bench.kernel_sources_sha()
+    path.write_text(f"# x\n\ndram_bytes_per_launch: 1234500000\nsources_sha256: {sha}\n")
+    monkeypatch.setattr(bench, "ROOT", str(tmp_path))
+    # the hash covers the kernel headers under ROOT: point it at the real ones
+    monkeypatch.setattr(bench, "kernel_sources_sha", lambda: sha)
+    assert bench.profile_traffic("gemm_gate_up", "w") == 1234500000.0
+    path.write_text("dram_bytes_per_launch: 1234500000\nsources_sha256: 0000000000000000\n")
+    assert bench.profile_traffic("gemm_gate_up", "w") is None   # kernels changed since
+    assert bench.profile_traffic("gemm_down", "w") is None      # no summary at all
+
+
+def test_kernel_hash_covers_only_device_code():
+    sha = bench.kernel_sources_sha()
+    assert len(sha) == 16 and int(sha, 16) >= 0
+
+
+def test_weak_scaling_value():
+    # two ranks, 4096 tokens each, 10 steps in 20 ms on the slowest rank
+    assert bench.replica_throughput(2, 4096, 10, 20.0) == pytest.approx(2 * 4096 * 10 / 0.020)
+
+
+def test_cpu_baseline_times_the_oracle_on_a_bounded_sample():
+    cfg = CONFIGS["tiny_f32"]
+    inp = generate(cfg, seed=0)
+    cb = bench.cpu_baseline(inp, budget_s=0.5)
+    assert cb["kind"] == "oracle" and cb["unit"] == "tokens/s" and cb["value"] > 0
+    assert cb["cores"] >= 1 and "of the 64 tokens" in cb["sample"]

@@ -120,6 +120,24 @@ def test_repeatable_and_host_path_identical():
     layer.check_device_status()
 
 
+def test_kernel_timing_records_only_the_selected_kernels():
+    from sparse_moe_transformer_router_b200.binding import ERR_ARG, L4MoEError
+    cfg = SMALL["bf16_ragged"]
+    inp = generate(cfg, seed=3, device="cuda")
+    layer = make_layer(inp)
+    run_gpu(layer, inp)
+    layer.read_timing()
+    layer.set_timing(["gemm_gate_up"])
+    run_gpu(layer, inp)
+    layer.set_timing(False)
+    t = layer.read_timing()
+    assert t["gemm_gate_up"][1] == 1 and t["gemm_gate_up"][0] > 0
+    assert all(n == 0 for k, (ms, n) in t.items() if k != "gemm_gate_up")
+    with pytest.raises(L4MoEError) as ei:
+        layer._check(layer._lib.l4moe_set_timing(layer._h, 1 << 5))  # no such kernel slot
+    assert ei.value.status == ERR_ARG
+
+
 def test_weight_pointer_change_rebuilds_descriptors():
     cfg = LayerConfig("swap", 256, 128, 4, 128, 128, "bf16", wr_std=0.1)
     a = generate(cfg, seed=4, device="cuda")
