@@ -169,7 +169,8 @@ L4MOE_API l4moe_status l4moe_forward_host(l4moe_handle *h, int T, const void *x_
  * Fails with L4MOE_ERR_WORKSPACE, launching nothing, when T tokens of this
  * layer do not fit in the scratch area: it holds the device part of the
  * workspace (l4moe_workspace_size without the host-path staging slots,
- * rounded up to 256 bytes) plus 2(E+1) TMA descriptors of 128 bytes, e.g.
+ * rounded up to 256 bytes) plus 2(E+1) TMA descriptors of 128 bytes (and,
+ * for E4M3 weights, the 2(E+1) scale-vector pointers), e.g.
  * about 390 tokens at d_model 5120 and F = Fs = 8192 in bf16 (E4M3 layers
  * also keep x in f16 there: about 350 tokens).  Every call, from any
  * handle, shares the one array: calls

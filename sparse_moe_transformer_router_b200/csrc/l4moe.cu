@@ -426,7 +426,7 @@ void launch_gemm(int grid, const BMaps& bm, const GemmArgs& a, cudaStream_t st) 
 template <typename ET, bool FP8W = false>
 l4moe_status run_layer(l4moe_handle* h, int T, const void* x, const void* Wr, const void* Wsgu,
                        const void* Wsdn, void* out, cudaStream_t st, uint8_t* w, int ws_tokens,
-                       const CUtensorMap* maps) {
+                       const CUtensorMap* maps, const float* const* scales = nullptr) {
     const l4moe_params& p = h->p;
     const int d = p.d_model, F = p.expert_ffn, Fs = p.shared_ffn, E = p.num_experts;
     const WsLayout L = ws_layout(p, ws_tokens, h->sms);
@@ -558,7 +558,7 @@ l4moe_status run_layer(l4moe_handle* h, int T, const void* x, const void* Wr, co
     gu.rowmap_routed = nullptr;
     gu.rowmap_shared = inv;
     gu.colscale_routed = gslot;  // sigmoid gate of each routed slot
-    gu.wscale = FP8W ? h->d_scales : nullptr;
+    gu.wscale = FP8W ? scales : nullptr;
     float* part = reinterpret_cast<float*>(w + L.part);
     gu.ksplit = s_gu;
     gu.partial_out = s_gu > 1 ? 1 : 0;
@@ -599,7 +599,7 @@ l4moe_status run_layer(l4moe_handle* h, int T, const void* x, const void* Wr, co
     dn.rowmap_routed = perm;     // slot -> token: un-permute on store
     dn.rowmap_shared = perm;     // the shared rows are slots too (H_s in slot order)
     dn.colscale_routed = nullptr;
-    dn.wscale = FP8W ? h->d_scales + (E + 1) : nullptr;
+    dn.wscale = FP8W ? scales + (E + 1) : nullptr;
     dn.ksplit = s_dn;
     dn.partial_out = 1;
     // partial slots: [0, s_dn) routed, [s_dn, 2 s_dn) shared
@@ -629,6 +629,20 @@ l4moe_status run_layer(l4moe_handle* h, int T, const void* x, const void* Wr, co
 
 // Device table of the per-column scale vectors of the E4M3 weights:
 // [gate/up of experts 0..E-1, shared gate/up, down of experts 0..E-1, shared down].
+// The E4M3 column-scale pointers in the kernels' order: gate/up of experts
+// 0..E-1, the shared gate/up, then the same for down.
+std::vector<const float*> scale_table(const l4moe_handle* h) {
+    const int E = h->p.num_experts;
+    std::vector<const float*> tab(2 * (E + 1));
+    for (int e = 0; e < E; ++e) {
+        tab[e] = h->s_gu[e];
+        tab[E + 1 + e] = h->s_dn[e];
+    }
+    tab[E] = h->ss_gu;
+    tab[2 * E + 1] = h->ss_dn;
+    return tab;
+}
+
 l4moe_status ensure_scales(l4moe_handle* h, cudaStream_t st) {
     const int E = h->p.num_experts;
     if (!h->d_scales) {
@@ -637,13 +651,7 @@ l4moe_status ensure_scales(l4moe_handle* h, cudaStream_t st) {
         h->scales_dirty = true;
     }
     if (!h->scales_dirty) return L4MOE_OK;
-    std::vector<const float*> tab(2 * (E + 1));
-    for (int e = 0; e < E; ++e) {
-        tab[e] = h->s_gu[e];
-        tab[E + 1 + e] = h->s_dn[e];
-    }
-    tab[E] = h->ss_gu;
-    tab[2 * E + 1] = h->ss_dn;
+    const std::vector<const float*> tab = scale_table(h);
     // pageable source: staged before the call returns
     cudaError_t e = cudaMemcpyAsync(h->d_scales, tab.data(), sizeof(float*) * tab.size(),
                                     cudaMemcpyHostToDevice, st);
@@ -687,7 +695,7 @@ l4moe_status forward_impl(l4moe_handle* h, int T, const void* x, const void* Wr,
                                         h->d_maps);
     case L4MOE_FP8_E4M3:
         return run_layer<__nv_bfloat16, true>(h, T, x, Wr, Wsgu, Wsdn, out, st, h->ws, h->ws_tokens,
-                                              h->d_maps);
+                                              h->d_maps, h->d_scales);
     }
     return fail(h, L4MOE_ERR_DTYPE, "unknown dtype");
 }
@@ -729,16 +737,16 @@ l4moe_status l4moe_forward_static(l4moe_handle* h, int T, const void* x, const v
                                   void* stream) {
     l4moe_status s = check_forward_args(h, T, x, W_router, W_gate_up, W_down, Ws_gate_up, Ws_down, out);
     if (s != L4MOE_OK || T == 0) return s;
-    if (h->p.dtype != L4MOE_F32 && h->p.dtype != L4MOE_BF16)
-        return fail(h, L4MOE_ERR_UNSUPPORTED, "FP8 weight path not built in this library");
     const int E = h->p.num_experts;
+    const bool fp8 = h->p.dtype == L4MOE_FP8_E4M3;
     const size_t ws_bytes = (ws_layout(h->p, T, h->sms).device_total + 255) & ~size_t(255);
     const size_t maps_bytes = sizeof(CUtensorMap) * 2 * (E + 1);
-    if (ws_bytes + maps_bytes > L4MOE_STATIC_WORKSPACE_BYTES) {
+    const size_t scales_bytes = fp8 ? sizeof(float*) * 2 * (E + 1) : 0;
+    if (ws_bytes + maps_bytes + scales_bytes > L4MOE_STATIC_WORKSPACE_BYTES) {
         char msg[200];
         snprintf(msg, sizeof msg,
                  "T = %d needs %zu bytes of static workspace; the library's static array holds %u",
-                 T, ws_bytes + maps_bytes, (unsigned)L4MOE_STATIC_WORKSPACE_BYTES);
+                 T, ws_bytes + maps_bytes + scales_bytes, (unsigned)L4MOE_STATIC_WORKSPACE_BYTES);
         return fail(h, L4MOE_ERR_WORKSPACE, msg);
     }
     uint8_t* base = nullptr;
@@ -752,10 +760,21 @@ l4moe_status l4moe_forward_static(l4moe_handle* h, int T, const void* x, const v
     if (e != cudaSuccess) return cuda_fail(h, e, "static descriptor upload");
     e = cudaMemsetAsync(base + ws_layout(h->p, T, h->sms).err, 0, sizeof(unsigned), st);
     if (e != cudaSuccess) return cuda_fail(h, e, "static error word clear");
+    const float* const* scales = nullptr;
+    if (fp8) {  // the E4M3 scale-pointer table follows the descriptors
+        const std::vector<const float*> tab = scale_table(h);
+        scales = reinterpret_cast<const float* const*>(base + ws_bytes + maps_bytes);
+        e = cudaMemcpyAsync(const_cast<const float**>(scales), tab.data(), scales_bytes,
+                            cudaMemcpyHostToDevice, st);
+        if (e != cudaSuccess) return cuda_fail(h, e, "static scale table upload");
+    }
     const unsigned timing = h->timing;  // event timing would create events: off here
     h->timing = 0;
     if (h->p.dtype == L4MOE_F32)
         s = run_layer<float>(h, T, x, W_router, Ws_gate_up, Ws_down, out, st, base, T, maps);
+    else if (fp8)
+        s = run_layer<__nv_bfloat16, true>(h, T, x, W_router, Ws_gate_up, Ws_down, out, st, base, T, maps,
+                                           scales);
     else
         s = run_layer<__nv_bfloat16>(h, T, x, W_router, Ws_gate_up, Ws_down, out, st, base, T, maps);
     h->timing = timing;

@@ -27,7 +27,7 @@ def _assert_close(out: torch.Tensor, ref: torch.Tensor, dtype: str):
     assert np.all(np.abs(o - r) <= bound)
 
 
-@pytest.mark.parametrize("dtype", ["bf16", "f32"])
+@pytest.mark.parametrize("dtype", ["bf16", "f32", "fp8"])
 def test_static_forward_matches_allocating_forward_on_two_calls(dtype):
     cfg = LayerConfig(f"noalloc_{dtype}", 300, 256, 8, 384, 256, dtype, wr_std=0.1)
     inp = generate(cfg, seed=11, device="cuda")
@@ -53,3 +53,25 @@ def test_static_forward_rejects_batches_beyond_its_array():
                              inp.Ws_down, out)
     assert ei.value.status == ERR_WORKSPACE
     assert "static" in str(ei.value)
+
+
+def test_static_forward_replays_inside_a_cuda_graph():
+    """The use it exists for: record the layer once under stream capture,
+    replay it, including after the input values change in place."""
+    cfg = LayerConfig("noalloc_graph", 200, 256, 8, 384, 256, "bf16", wr_std=0.1)
+    inp = generate(cfg, seed=13, device="cuda")
+    layer = make_layer(inp)
+    args = (inp.x, inp.W_router, inp.W_gate_up, inp.W_down, inp.Ws_gate_up, inp.Ws_down)
+    out = torch.empty((cfg.T, cfg.d_model), dtype=inp.x.dtype, device="cuda")
+    layer.forward_static(*args, out)  # first call outside capture
+    torch.cuda.synchronize()
+    graph = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(graph):
+        layer.forward_static(*args, out)
+    for flip in (1.0, -0.5):
+        inp.x.mul_(flip)
+        ref = layer.forward(*args)
+        out.fill_(float("nan"))
+        graph.replay()
+        torch.cuda.synchronize()
+        _assert_close(out, ref, "bf16")
