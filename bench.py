@@ -197,7 +197,8 @@ def cpu_baseline(inp, budget_s: float = 15.0, host: HostLayer | None = None) -> 
     def run(n):
         sel = np.arange(n, dtype=np.int32) * max(1, cfg.T // max(n, 1))
         sel = sel[sel < cfg.T]
-        Wgu, Wdn, kw = h.expert_args(set(int(e) for e in h.idx[sel]))
+        need = set(int(e) for e in h.idx[sel]) if cfg.num_experts > 0 else set()
+        Wgu, Wdn, kw = h.expert_args(need)
         t0 = time.perf_counter()
         oracle.forward(h.x, h.Wr, Wgu, Wdn, h.Ws_gu, h.Ws_dn, bias=h.bias, tokens=sel, **kw)
         return len(sel), time.perf_counter() - t0

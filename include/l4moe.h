@@ -20,6 +20,9 @@
  *     Maverick" field table (ffns.moe.* rows: gated experts of width 8192,
  *     one shared expert of width 8192).
  *   SwiGLU_W(u) = (silu(u . Wg) * (u . Wu)) . Wd with silu(z) = z/(1+e^-z).
+ * With E = 0 the layer is the dense SwiGLU feed-forward of the layers
+ * without experts (the Maverick field table's dense width 16384 as Fs):
+ * W_router, W_gate_up and W_down are unused (may be NULL) and F may be 0.
  *
  * Layouts (all row-major, "x @ W" orientation, element = the dtype below):
  *   x          [T, d]        W_router  [d, E]
@@ -49,7 +52,7 @@
  * in a device word that l4moe_check_device_status reads (it synchronises).
  * l4moe_last_error gives a message for the last non-OK status of a handle.
  *
- * Requirements: d, F, Fs multiples of 64; 1 <= E <= 256; all tensor pointers
+ * Requirements: d, F, Fs multiples of 64; 0 <= E <= 256 (F > 0 when E > 0); all tensor pointers
  * 16-byte aligned.  One handle serves one stream at a time (the workspace is
  * shared by the calls made with it).
  */
@@ -90,7 +93,8 @@ typedef struct {
     int d_model;      /* d  : model width (KerasFormers "Llama 4": embed_dim)       */
     int expert_ffn;   /* F  : routed expert width (Maverick table: d_expert)       */
     int shared_ffn;   /* Fs : shared expert width (Maverick table: d_shared)       */
-    int num_experts;  /* E  : routed experts (16 Scout, 128 Maverick)              */
+    int num_experts;  /* E  : routed experts (16 Scout, 128 Maverick); 0 = a dense
+                         feed-forward layer: out = SwiGLU_shared(x) alone          */
     l4moe_dtype dtype;
 } l4moe_params;
 

@@ -22,6 +22,10 @@
  *   ffns.moe.gated / ffns.moe.d_expert / ffns.moe.d_shared: experts and the
  *   shared expert are gated MLPs (SwiGLU) of width 8192.
  *
+ * With E = 0 the layer is the shared SwiGLU alone: the dense feed-forward of
+ * the layers without experts (llm-architectures-explained "Llama 4
+ * Maverick", field table: d_ffn 16384 for the dense layers).
+ *
  * Readings where the pages are silent (each listed in the design notes):
  *   - logits are formed in fp64 and rounded once to fp32; the argmax runs on
  *     those fp32 values with a strict ">" so the lowest index wins a tie and a
@@ -198,16 +202,25 @@ int oracle_forward(int T, int d, int E, int F, int Fs,
         double *a = (double *)malloc(sizeof(double) * 2 * (size_t)Fmax);
         double *h = (double *)malloc(sizeof(double) * (size_t)Fmax);
         double *y = out + (size_t)i * (size_t)d;
+        for (int n = 0; n < d; ++n) y[n] = 0.0;
+        /* shared expert on the ungated input (with E == 0 the whole layer:
+         * the dense SwiGLU feed-forward of the layers without experts) */
+        for (int k = 0; k < d; ++k) u[k] = load_elem(x_t, x_dtype, (size_t)k);
+        swiglu_ffn_accumulate(d, Fs, u, Ws_gate_up, Ws_down, w_dtype,
+                              ss_gate_up, ss_down, a, h, y);
+        if (E == 0) {
+            if (sel_idx) sel_idx[i] = -1;
+            if (sel_gate) sel_gate[i] = 0.0;
+            free(u);
+            free(a);
+            free(h);
+            continue;
+        }
         float lmax;
         int e = route_token(d, E, x_t, x_dtype, Wr, wr_dtype, bias, &lmax, NULL);
         double g = sigmoid((double)lmax);
         if (sel_idx) sel_idx[i] = e;
         if (sel_gate) sel_gate[i] = g;
-        for (int n = 0; n < d; ++n) y[n] = 0.0;
-        /* shared expert on the ungated input */
-        for (int k = 0; k < d; ++k) u[k] = load_elem(x_t, x_dtype, (size_t)k);
-        swiglu_ffn_accumulate(d, Fs, u, Ws_gate_up, Ws_down, w_dtype,
-                              ss_gate_up, ss_down, a, h, y);
         /* routed expert on the sigmoid-gated input */
         if (!W_gate_up[e] || !W_down[e]) {
             missing |= 1;

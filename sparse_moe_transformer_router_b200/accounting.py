@@ -11,6 +11,7 @@ the test suite checks.
 Algorithmic bytes count each touched weight byte once (experts that receive no
 token are not read), the input read, the output write, and one write plus one
 read of the gated expert-ordered input and of the two hidden activations.
+With E = 0 (a dense feed-forward layer) only the shared SwiGLU counts.
 """
 from __future__ import annotations
 
@@ -35,7 +36,8 @@ def layer_bytes(T: int, d: int, E: int, F: int, Fs: int, dtype: str, experts_tou
         weights += (experts_touched * (2 * F + d) + (2 * Fs + d)) * 4
     router = d * E * a
     acts = T * d * a * 2                 # x read, out write
-    acts += T * d * a * 2                # gated expert-ordered input: write + read
+    if E > 0:
+        acts += T * d * a * 2            # gated expert-ordered input: write + read
     acts += T * (F + Fs) * a * 2         # hidden activations: write + read
     return weights + router + acts
 

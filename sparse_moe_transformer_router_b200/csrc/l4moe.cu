@@ -468,10 +468,14 @@ l4moe_status run_layer(l4moe_handle* h, int T, const void* x, const void* Wr, co
         return encode_2d(m, dt, base, (uint64_t)width, (uint64_t)T, (uint64_t)width * sizeof(ET), bk, rows);
     };
     const void* xs = FP8W ? (const void*)x16 : x;  // the shared expert's operand
+    // without experts (F may be 0) the routed hidden descriptors are never
+    // read: give them the shared hidden rows to describe
+    const void* hrm = F > 0 ? (const void*)hr : (const void*)hs;
+    const int Fr = F > 0 ? F : Fs;
     if (!act(&m_x, adt, x, d, 64) || !act(&bm_gu.routed, gdt, xg, d, rb) ||
         !act(&bm_gu.routed_small, gdt, xg, d, rs) || !act(&bm_gu.shared, gdt, xs, d, rb) ||
-        !act(&bm_gu.shared_small, gdt, xs, d, rs) || !act(&bm_dn.routed, gdt, hr, F, rb) ||
-        !act(&bm_dn.routed_small, gdt, hr, F, rs) || !act(&bm_dn.shared, gdt, hs, Fs, rb) ||
+        !act(&bm_gu.shared_small, gdt, xs, d, rs) || !act(&bm_dn.routed, gdt, hrm, Fr, rb) ||
+        !act(&bm_dn.routed_small, gdt, hrm, Fr, rs) || !act(&bm_dn.shared, gdt, hs, Fs, rb) ||
         !act(&bm_dn.shared_small, gdt, hs, Fs, rs))
         return fail(h, L4MOE_ERR_CUDA, "cuTensorMapEncodeTiled failed for an activation");
 
@@ -482,36 +486,6 @@ l4moe_status run_layer(l4moe_handle* h, int T, const void* x, const void* Wr, co
         if ((e = cudaGetLastError()) != cudaSuccess) return cuda_fail(h, e, what); \
     } while (0)
 
-    LaunchTimer t_router(h, 0, st);
-    // one token tile and many experts: split the router over 16-expert chunks
-    const bool split_router = sizeof(ET) == 2 && E % 16 == 0 && E >= 32 && T <= 128;
-    float* logits = split_router ? reinterpret_cast<float*>(w + L.logits) : nullptr;
-    if (sizeof(ET) == 2 && E % 8 == 0) {
-        // tensor-core router: W_router [d, E] as the MN-major operand
-        CUtensorMap m_wr;
-        if (!encode_2d(&m_wr, adt, Wr, (uint64_t)E, (uint64_t)d, (uint64_t)E * sizeof(ET), 64, 64))
-            return fail(h, L4MOE_ERR_CUDA, "cuTensorMapEncodeTiled failed for the router weight");
-        static std::once_flag once;
-        std::call_once(once, [] { set_smem_attr(router_mma_kernel, rmma::SMEM_BYTES); });
-        const int n_chunk = split_router ? 16 : E;
-        const int tiles = (T + 127) / 128;
-        int kslices;
-        if (split_router) {
-            kslices = std::min(kRouterKSplit, std::max(1, d / 256));
-        } else {
-            // few token tiles: K slices per tile (at most 4 and the SMs'
-            // worth), reduced inside a cluster of the slices
-            kslices = std::max(1, std::min({4, h->sms / tiles, d / 256}));
-        }
-        launch_kc(router_mma_kernel, dim3(tiles, E / n_chunk, kslices), dim3(128), rmma::SMEM_BYTES, st,
-                  kslices == 1 ? 0u : (unsigned)kslices, m_x, m_wr, (const float*)h->bias,
-                  T, d, E, n_chunk, logits, idx, gate, lmax, margin, err);
-    } else {
-        launch_router<ET>(x, Wr, h->bias, T, d, E, idx, gate, lmax, margin, st);
-    }
-    t_router.stop();
-    L4MOE_CHECK_LAUNCH("router launch");
-
     // feature blocks per pair tile: 128 features for gate/up, 256 for down
     const int fpg = pair_features<MODE_GATEUP>(), fpd = pair_features<MODE_DOWN>();
     const int fb_gu_r = (F + fpg - 1) / fpg;
@@ -520,20 +494,67 @@ l4moe_status run_layer(l4moe_handle* h, int T, const void* x, const void* Wr, co
     // split-K k-ranges when a small batch leaves too few tiles
     const SplitPlan plan = split_plan(p, T, h->sms);
     const int s_gu = plan.s_gu, s_dn = plan.s_dn;
-    const size_t psmem = sizeof(int) * (34 * (size_t)E + 1);
-    LaunchTimer t_perm(h, 1, st);
-    launch_k(permute_kernel, dim3(1), dim3(1024), psmem, st, (const float*)logits,
-             gate, lmax, margin, idx, T, E, fb_gu_r * s_gu, fb_gu_s * s_gu, fb_dn * s_dn, counts, offsets,
-             perm, inv, tab_gu, tab_dn, err);
-    t_perm.stop();
-    L4MOE_CHECK_LAUNCH("permute launch");
+    if (E > 0) {
+        LaunchTimer t_router(h, 0, st);
+        // one token tile and many experts: split the router over 16-expert chunks
+        const bool split_router = sizeof(ET) == 2 && E % 16 == 0 && E >= 32 && T <= 128;
+        float* logits = split_router ? reinterpret_cast<float*>(w + L.logits) : nullptr;
+        if (sizeof(ET) == 2 && E % 8 == 0) {
+            // tensor-core router: W_router [d, E] as the MN-major operand
+            CUtensorMap m_wr;
+            if (!encode_2d(&m_wr, adt, Wr, (uint64_t)E, (uint64_t)d, (uint64_t)E * sizeof(ET), 64, 64))
+                return fail(h, L4MOE_ERR_CUDA, "cuTensorMapEncodeTiled failed for the router weight");
+            static std::once_flag once;
+            std::call_once(once, [] { set_smem_attr(router_mma_kernel, rmma::SMEM_BYTES); });
+            const int n_chunk = split_router ? 16 : E;
+            const int tiles = (T + 127) / 128;
+            int kslices;
+            if (split_router) {
+                kslices = std::min(kRouterKSplit, std::max(1, d / 256));
+            } else {
+                // few token tiles: K slices per tile (at most 4 and the SMs'
+                // worth), reduced inside a cluster of the slices
+                kslices = std::max(1, std::min({4, h->sms / tiles, d / 256}));
+            }
+            launch_kc(router_mma_kernel, dim3(tiles, E / n_chunk, kslices), dim3(128), rmma::SMEM_BYTES, st,
+                      kslices == 1 ? 0u : (unsigned)kslices, m_x, m_wr, (const float*)h->bias,
+                      T, d, E, n_chunk, logits, idx, gate, lmax, margin, err);
+        } else {
+            launch_router<ET>(x, Wr, h->bias, T, d, E, idx, gate, lmax, margin, st);
+        }
+        t_router.stop();
+        L4MOE_CHECK_LAUNCH("router launch");
 
-    const int sc_blocks = std::min((T + 7) / 8, h->sms * 8);
-    LaunchTimer t_rows(h, 2, st);
-    launch_k(permute_rows_kernel<ET, GT>, dim3(sc_blocks), dim3(256), 0, st, static_cast<const ET*>(x),
-             (const float*)gate, (const int32_t*)inv, T, d, xg, gslot, FP8W ? x16 : (GT*)nullptr);
-    t_rows.stop();
-    L4MOE_CHECK_LAUNCH("row permutation launch");
+        const size_t psmem = sizeof(int) * (34 * (size_t)E + 1);
+        LaunchTimer t_perm(h, 1, st);
+        launch_k(permute_kernel, dim3(1), dim3(1024), psmem, st, (const float*)logits,
+                 gate, lmax, margin, idx, T, E, fb_gu_r * s_gu, fb_gu_s * s_gu, fb_dn * s_dn, counts, offsets,
+                 perm, inv, tab_gu, tab_dn, err);
+        t_perm.stop();
+        L4MOE_CHECK_LAUNCH("permute launch");
+
+        const int sc_blocks = std::min((T + 7) / 8, h->sms * 8);
+        LaunchTimer t_rows(h, 2, st);
+        launch_k(permute_rows_kernel<ET, GT>, dim3(sc_blocks), dim3(256), 0, st, static_cast<const ET*>(x),
+                 (const float*)gate, (const int32_t*)inv, T, d, xg, gslot, FP8W ? x16 : (GT*)nullptr);
+        t_rows.stop();
+        L4MOE_CHECK_LAUNCH("row permutation launch");
+    } else {
+        // no experts (a dense feed-forward layer): the shared SwiGLU over the
+        // tokens in order; the work lists hold that one group
+        LaunchTimer t_perm(h, 1, st);
+        launch_k(dense_table_kernel, dim3(1), dim3(32), 0, st, tab_gu, tab_dn, T, fb_gu_s * s_gu, fb_dn * s_dn);
+        t_perm.stop();
+        L4MOE_CHECK_LAUNCH("work list launch");
+        if (FP8W) {  // the f16 copy of x the contractions of E4M3 layers read
+            const int sc_blocks = std::min((T + 7) / 8, h->sms * 8);
+            LaunchTimer t_rows(h, 2, st);
+            launch_k(permute_rows_kernel<ET, GT>, dim3(sc_blocks), dim3(256), 0, st, static_cast<const ET*>(x),
+                     (const float*)nullptr, (const int32_t*)nullptr, T, d, x16, (float*)nullptr, (GT*)nullptr);
+            t_rows.stop();
+            L4MOE_CHECK_LAUNCH("row conversion launch");
+        }
+    }
 
     const int tb = (T + kTokTile - 1) / kTokTile;
     // CTA pairs: two CTAs (one cluster) per tile, at most one pair per two SMs
@@ -556,7 +577,7 @@ l4moe_status run_layer(l4moe_handle* h, int T, const void* x, const void* Wr, co
     gu.out_shared = hs;          // shared hidden rows, also stored in slot order
     gu.ld_shared = Fs;
     gu.rowmap_routed = nullptr;
-    gu.rowmap_shared = inv;
+    gu.rowmap_shared = E > 0 ? inv : nullptr;
     gu.colscale_routed = gslot;  // sigmoid gate of each routed slot
     gu.wscale = FP8W ? scales : nullptr;
     float* part = reinterpret_cast<float*>(w + L.part);
@@ -597,7 +618,7 @@ l4moe_status run_layer(l4moe_handle* h, int T, const void* x, const void* Wr, co
     dn.out_shared = out;
     dn.ld_shared = d;
     dn.rowmap_routed = perm;     // slot -> token: un-permute on store
-    dn.rowmap_shared = perm;     // the shared rows are slots too (H_s in slot order)
+    dn.rowmap_shared = E > 0 ? perm : nullptr;  // H_s in slot order (token order without experts)
     dn.colscale_routed = nullptr;
     dn.wscale = FP8W ? scales + (E + 1) : nullptr;
     dn.ksplit = s_dn;
@@ -615,9 +636,10 @@ l4moe_status run_layer(l4moe_handle* h, int T, const void* x, const void* Wr, co
                                      bm_dn, dn, st);
     {
         const long long n = (long long)T * d;
+        // the routed planes then the shared ones; without experts only the shared
         launch_k(down_finish_kernel<ET>, dim3((int)std::min<long long>((n / 4 + 255) / 256, 4LL * h->sms)),
-                 dim3(256), 0, st, (const float*)part, dn.part_stride_routed, 2 * s_dn, n,
-                 static_cast<ET*>(out));
+                 dim3(256), 0, st, (const float*)(E > 0 ? part : dn.part_shared), dn.part_stride_routed,
+                 E > 0 ? 2 * s_dn : s_dn, n, static_cast<ET*>(out));
         ++h->launches;
     }
     t_dn.stop();
@@ -665,9 +687,10 @@ l4moe_status check_forward_args(l4moe_handle* h, int T, const void* x, const voi
                                 const void* Wsdn, const void* out) {
     if (!h) return L4MOE_ERR_ARG;
     if (T < 0) return fail(h, L4MOE_ERR_ARG, "T must be >= 0");
-    if (!x || !Wr || !Wgu || !Wdn || !Wsgu || !Wsdn || !out)
+    const bool experts = h->p.num_experts > 0;  // without experts W_router, W_gate_up, W_down are unused
+    if (!x || !Wsgu || !Wsdn || !out || (experts && (!Wr || !Wgu || !Wdn)))
         return fail(h, L4MOE_ERR_ARG, "null tensor pointer");
-    const void* ptrs[] = {x, Wr, Wsgu, Wsdn, out};
+    const void* ptrs[] = {x, experts ? Wr : x, Wsgu, Wsdn, out};
     for (const void* q : ptrs)
         if (!aligned16(q)) return fail(h, L4MOE_ERR_ALIGN, "tensor pointer not 16-byte aligned");
     for (int e = 0; e < h->p.num_experts; ++e) {
@@ -675,7 +698,7 @@ l4moe_status check_forward_args(l4moe_handle* h, int T, const void* x, const voi
         if (!aligned16(Wgu[e]) || !aligned16(Wdn[e]))
             return fail(h, L4MOE_ERR_ALIGN, "expert weight pointer not 16-byte aligned");
     }
-    if (h->p.dtype == L4MOE_FP8_E4M3 && (h->s_gu.empty() || !h->ss_gu || !h->ss_dn))
+    if (h->p.dtype == L4MOE_FP8_E4M3 && !h->ss_gu)
         return fail(h, L4MOE_ERR_DTYPE, "FP8 weights need l4moe_set_fp8_scales first");
     return L4MOE_OK;
 }
@@ -803,9 +826,10 @@ l4moe_status l4moe_create(const l4moe_params* params, l4moe_handle** out) {
     const l4moe_params& p = *params;
     if (p.dtype != L4MOE_F32 && p.dtype != L4MOE_BF16 && p.dtype != L4MOE_FP8_E4M3)
         return fail(nullptr, L4MOE_ERR_DTYPE, "unknown dtype");
-    if (p.d_model <= 0 || p.expert_ffn <= 0 || p.shared_ffn <= 0 || p.num_experts < 1 ||
-        p.num_experts > 256)
-        return fail(nullptr, L4MOE_ERR_ARG, "shape out of range (need d, F, Fs > 0 and 1 <= E <= 256)");
+    if (p.d_model <= 0 || p.shared_ffn <= 0 || p.num_experts < 0 || p.num_experts > 256 ||
+        p.expert_ffn < 0 || (p.num_experts > 0 && p.expert_ffn == 0))
+        return fail(nullptr, L4MOE_ERR_ARG,
+                    "shape out of range (need d, Fs > 0, 0 <= E <= 256, F > 0 when E > 0)");
     if (p.d_model % 64 || p.expert_ffn % 64 || p.shared_ffn % 64)
         return fail(nullptr, L4MOE_ERR_ALIGN, "d_model, expert_ffn and shared_ffn must be multiples of 64");
     int dev = 0;
@@ -881,12 +905,13 @@ l4moe_status l4moe_set_fp8_scales(l4moe_handle* h, const float* const* s_gate_up
                                   const float* ss_down) {
     if (!h) return L4MOE_ERR_ARG;
     if (h->p.dtype != L4MOE_FP8_E4M3) return fail(h, L4MOE_ERR_DTYPE, "scales apply to FP8 weights only");
-    if (!s_gate_up || !s_down || !ss_gate_up || !ss_down) return fail(h, L4MOE_ERR_ARG, "null scale pointer");
     const int E = h->p.num_experts;
+    if (!ss_gate_up || !ss_down || (E > 0 && (!s_gate_up || !s_down)))
+        return fail(h, L4MOE_ERR_ARG, "null scale pointer");
     for (int e = 0; e < E; ++e)
         if (!s_gate_up[e] || !s_down[e]) return fail(h, L4MOE_ERR_ARG, "null expert scale pointer");
-    h->s_gu.assign(s_gate_up, s_gate_up + E);
-    h->s_dn.assign(s_down, s_down + E);
+    h->s_gu.assign(s_gate_up, s_gate_up + (E > 0 ? E : 0));
+    h->s_dn.assign(s_down, s_down + (E > 0 ? E : 0));
     h->ss_gu = ss_gate_up;
     h->ss_dn = ss_down;
     h->scales_dirty = true;

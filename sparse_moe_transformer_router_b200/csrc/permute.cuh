@@ -90,6 +90,29 @@ __device__ void build_table(GroupTable* tab, int G, RowsF rows_of, Row0F row0_of
     }
 }
 
+// Work lists of a layer without experts: one group (the shared SwiGLU, as
+// expert 0 == num_experts) over the T tokens in order.  One warp.
+__global__ void dense_table_kernel(GroupTable* tab_gu, GroupTable* tab_dn, int T, int fb_gu, int fb_dn) {
+    pdl_enter();
+    const int lane = threadIdx.x & 31;
+    if (threadIdx.x >= 32) return;
+    const int tb = (T + kTokTile - 1) / kTokTile;
+    for (int w = 0; w < 2; ++w) {
+        GroupTable* tab = w == 0 ? tab_gu : tab_dn;
+        const int tiles = tb * (w == 0 ? fb_gu : fb_dn);
+        if (lane == 0) {
+            tab->num_groups = T > 0 ? 1 : 0;
+            tab->total_tiles = tiles;
+            tab->heavy_tiles = T >= kHeavyRows ? tiles : 0;
+            tab->rows[0] = T;
+            tab->row0[0] = 0;
+            tab->expert[0] = 0;
+            tab->tile_start[0] = 0;
+            tab->tile_start[1] = tiles;
+        }
+    }
+}
+
 // Launch position L (0 .. total-1) -> tile number in the table's order.  The
 // heavy run's H tiles take the positions where floor((L+1) H / N) steps up,
 // spread as evenly as integers allow, the light run's tiles the others; both
@@ -256,7 +279,8 @@ __global__ void __launch_bounds__(1024) permute_kernel(const float* __restrict__
 // is applied to the fp32 accumulator in the GEMM epilogue instead of
 // rounding g * x to the activation type here.  OT = IT copies exactly; for
 // E4M3 layers IT = bf16, OT = f16 (the contractions' operand type) and
-// x_tok (if not null) also receives the f16 rows in token order.
+// x_tok (if not null) also receives the f16 rows in token order.  inv ==
+// null keeps token order (and gate / gate_slot are then unused).
 // One warp per token row, 16-byte vectors; d % 8 == 0.
 __device__ __forceinline__ uint4 cvt_row_vec(uint4 v, __nv_bfloat16, __half) {
     uint32_t w[4] = {v.x, v.y, v.z, v.w};
@@ -283,8 +307,8 @@ __global__ void __launch_bounds__(256) permute_rows_kernel(const IT* __restrict_
     const int lane = threadIdx.x & 31;
     const int warps = (gridDim.x * blockDim.x) >> 5;
     for (int t = (blockIdx.x * blockDim.x + threadIdx.x) >> 5; t < T; t += warps) {
-        const int slot = inv[t];
-        if (lane == 0) gate_slot[slot] = gate[t];
+        const int slot = inv ? inv[t] : t;
+        if (lane == 0 && gate_slot) gate_slot[slot] = gate[t];
         const uint4* s = reinterpret_cast<const uint4*>(x + (size_t)t * d);
         uint4* o = reinterpret_cast<uint4*>(xp + (size_t)slot * d);
         uint4* ot = x_tok ? reinterpret_cast<uint4*>(x_tok + (size_t)t * d) : nullptr;

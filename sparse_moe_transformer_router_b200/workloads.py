@@ -49,7 +49,8 @@ class LayerConfig:
 # The five workloads.  Sizes, dtypes and distributions: tiny fp32 layer; a
 # Scout-shaped prefill layer (16 experts); a Maverick-shaped prefill layer
 # (128 experts, Zipf(1.1) loads, 10 experts idle); Maverick-shaped decode
-# (T in {1, 8, 32, 128}, uniform routing); Maverick with E4M3 weights.
+# (T in {1, 8, 32, 128}, uniform routing); Maverick with E4M3 weights.  Plus
+# Maverick's dense feed-forward layer (no experts, width 16384).
 CONFIGS = {
     "tiny_f32": LayerConfig("tiny_f32", 64, 128, 4, 256, 256, "f32", wr_std=0.1),
     "scout_prefill_bf16": LayerConfig("scout_prefill_bf16", 4096, 5120, 16, 8192, 8192, "bf16"),
@@ -58,6 +59,8 @@ CONFIGS = {
     "maverick_decode_bf16": LayerConfig("maverick_decode_bf16", 128, 5120, 128, 8192, 8192, "bf16"),
     "maverick_fp8": LayerConfig("maverick_fp8", 16384, 5120, 128, 8192, 8192, "fp8",
                                 router="zipf", n_dead=10),
+    # the layers without experts: one SwiGLU feed-forward of width 16384
+    "maverick_dense_bf16": LayerConfig("maverick_dense_bf16", 8192, 5120, 0, 0, 16384, "bf16"),
 }
 DECODE_TOKENS = (1, 8, 32, 128)
 

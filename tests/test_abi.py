@@ -48,7 +48,9 @@ def _create(lib, d, F, Fs, E, dtype):
 @pytest.mark.parametrize("args,status", [
     ((5120, 8192, 8192, 16, 7), binding.ERR_DTYPE),       # unknown dtype
     ((0, 8192, 8192, 16, 1), binding.ERR_ARG),            # d = 0
-    ((5120, 8192, 8192, 0, 1), binding.ERR_ARG),          # E = 0
+    ((5120, 8192, 8192, -1, 1), binding.ERR_ARG),         # E < 0
+    ((5120, 0, 8192, 16, 1), binding.ERR_ARG),            # experts need F > 0
+    ((5120, 8192, 0, 0, 1), binding.ERR_ARG),             # Fs = 0
     ((5120, 8192, 8192, 257, 1), binding.ERR_ARG),        # E > 256
     ((5100, 8192, 8192, 16, 1), binding.ERR_ALIGN),       # d not a multiple of 64
     ((5120, 8200, 8192, 16, 1), binding.ERR_ALIGN),       # F not a multiple of 64

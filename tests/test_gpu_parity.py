@@ -75,6 +75,41 @@ def test_e4m3_widening_is_exact_for_every_code(codes, scale):
     print(f"max|err|/rms = {ratio:.3e}")
 
 
+DENSE = {
+    # no experts: the layer is one SwiGLU feed-forward (ragged token and
+    # feature tiles, fp32, E4M3 weights, a single token)
+    "dense_bf16": LayerConfig("dense_bf16", 300, 256, 0, 0, 384, "bf16"),
+    "dense_f32": LayerConfig("dense_f32", 130, 128, 0, 0, 192, "f32"),
+    "dense_fp8": LayerConfig("dense_fp8", 300, 256, 0, 0, 320, "fp8"),
+    "dense_T1": LayerConfig("dense_T1", 1, 1024, 0, 0, 1024, "bf16"),
+}
+
+
+def _dense_forward(inp):
+    layer = make_layer(inp)
+    out = layer.forward(inp.x, None, [], [], inp.Ws_gate_up, inp.Ws_down)
+    torch.cuda.synchronize()
+    layer.check_device_status()
+    return out
+
+
+@pytest.mark.parametrize("name", list(DENSE))
+def test_dense_layer_matches_oracle(name):
+    inp = generate(DENSE[name], seed=0, device="cuda")
+    ratio = check_outputs(inp, _dense_forward(inp), None)
+    print(f"{name}: max|err|/rms = {ratio:.3e}")
+
+
+def test_full_size_maverick_dense_layer():
+    cfg = CONFIGS["maverick_dense_bf16"]
+    inp = generate(cfg, seed=0, device="cuda")
+    out = _dense_forward(inp)
+    toks = np.unique(np.concatenate([np.linspace(0, cfg.T - 1, 24).astype(np.int32),
+                                     np.array([255, 256, 4095, 4096], np.int32)]))
+    ratio = check_outputs(inp, out, toks)
+    print(f"{cfg.name}: {len(toks)} sampled tokens, max|err|/rms = {ratio:.3e}")
+
+
 def test_zero_input_gives_zero_output_and_expert_zero():
     cfg = LayerConfig("zero", 200, 128, 6, 128, 128, "bf16")
     inp = generate(cfg, seed=1, device="cuda")

@@ -250,3 +250,15 @@ def test_token_subset_equals_rows_of_full_run_and_missing_expert_raises():
         if t is not None:
             with pytest.raises(ValueError):
                 oracle.forward(L["x"], L["Wr"], Wgu, Wd, L["Wsgu"], L["Wsd"], tokens=np.array([t], np.int32))
+
+
+@pytest.mark.parametrize("dtype", ["f32", "bf16"])
+def test_dense_layer_without_experts_is_one_swiglu_ffn(dtype):
+    """E = 0 (the layers without experts): the output is the shared SwiGLU
+    feed-forward alone, as a library matmul evaluates it."""
+    rng = np.random.default_rng(11)
+    L = _layer(rng, 9, 24, 0, 8, 40, dtype)
+    out, idx, gate = oracle.forward(L["x"], L["Wr"], [], [], L["Wsgu"], L["Wsd"])
+    ref = _dense_swiglu(L["x64"], L["Wsgu64"], L["Wsd64"])
+    np.testing.assert_allclose(out, ref, rtol=1e-12, atol=1e-12)
+    assert np.all(idx == -1)
