@@ -62,7 +62,10 @@ def _load():
             lib.oracle_permutation.restype = None
             lib.oracle_permutation.argtypes = [i32, i32, vp, vp, vp, vp]
             lib.oracle_forward.restype = ctypes.c_int
-            lib.oracle_forward.argtypes = [i32, i32, i32, i32, i32,
+            lib.oracle_route_topk.restype = None
+            lib.oracle_route_topk.argtypes = [i32, i32, i32, i32, vp, i32, vp, i32, f32p,
+                                              vp, vp, vp]
+            lib.oracle_forward.argtypes = [i32, i32, i32, i32, i32, i32,
                                            vp, i32, vp, i32, f32p,
                                            vp, vp, vp, vp, i32,
                                            vp, vp, vp, vp,
@@ -122,6 +125,25 @@ def route(x: np.ndarray, Wr: np.ndarray, bias: np.ndarray | None = None):
     return idx, lmax, margin
 
 
+def route_topk(x: np.ndarray, Wr: np.ndarray, k: int, bias: np.ndarray | None = None):
+    """Top-k router for all tokens: (idx int32[T, k], logits f32[T, k],
+    margin f32[T]): the k largest fp32 logits in descending order, ties to
+    the lower index; margin is the k-th selected logit minus the largest one
+    left out (+inf when k == E)."""
+    x = np.ascontiguousarray(x)
+    Wr = np.ascontiguousarray(Wr)
+    T, d = x.shape
+    d2, E = Wr.shape
+    assert d == d2 and 1 <= k <= E
+    b = None if bias is None else np.ascontiguousarray(bias, dtype=np.float32)
+    idx = np.empty((T, k), np.int32)
+    lsel = np.empty((T, k), np.float32)
+    margin = np.empty(T, np.float32)
+    _load().oracle_route_topk(T, d, E, k, _ptr(x), _dtype_code(x), _ptr(Wr), _dtype_code(Wr),
+                              _ptr(b), _ptr(idx), _ptr(lsel), _ptr(margin))
+    return idx, lsel, margin
+
+
 def permutation(idx: np.ndarray, E: int):
     """(counts[E], offsets[E+1], perm[T]) with perm the stable expert order."""
     idx = np.ascontiguousarray(idx, dtype=np.int32)
@@ -136,13 +158,16 @@ def permutation(idx: np.ndarray, E: int):
 
 def forward(x, Wr, W_gate_up, W_down, Ws_gate_up, Ws_down, *, bias=None,
             s_gate_up=None, s_down=None, ss_gate_up=None, ss_down=None,
-            tokens=None):
+            tokens=None, k=1):
     """Layer output in fp64 for ``tokens`` (all tokens when None).
 
     W_gate_up / W_down are length-E lists of [d, 2F] / [F, d] arrays; entries
     may be None for experts no selected token reaches.  For E4M3 weights the
-    per-output-column fp32 scales are required.  Returns
-    (out f64[n_sel, d], idx int32[n_sel], gate f64[n_sel]).
+    per-output-column fp32 scales are required.  k > 1: each token runs its
+    k highest-scoring experts, each on the input gated by the sigmoid of its
+    own logit, and their outputs add to the shared expert's.  Returns
+    (out f64[n_sel, d], idx int32[n_sel], gate f64[n_sel]), or [n_sel, k]
+    index and gate arrays for k > 1.
     """
     x = np.ascontiguousarray(x)
     Wr = np.ascontiguousarray(Wr)
@@ -190,11 +215,12 @@ def forward(x, Wr, W_gate_up, W_down, Ws_gate_up, Ws_down, *, bias=None,
     else:
         sel = np.ascontiguousarray(tokens, dtype=np.int32)
         n_sel = sel.shape[0]
+    assert 1 <= k <= max(E, 1) and k <= 8
     out = np.zeros((n_sel, d), np.float64)
-    sel_idx = np.empty(n_sel, np.int32)
-    sel_gate = np.empty(n_sel, np.float64)
+    sel_idx = np.empty(n_sel * k, np.int32)
+    sel_gate = np.empty(n_sel * k, np.float64)
     rc = _load().oracle_forward(
-        T, d, E, F, Fs, _ptr(x), _dtype_code(x), _ptr(Wr), _dtype_code(Wr),
+        T, d, E, k, F, Fs, _ptr(x), _dtype_code(x), _ptr(Wr), _dtype_code(Wr),
         _ptr(bias), ctypes.cast(gu_ptrs, ctypes.c_void_p),
         ctypes.cast(dn_ptrs, ctypes.c_void_p), _ptr(Ws_gate_up), _ptr(Ws_down),
         w_code,
@@ -206,4 +232,7 @@ def forward(x, Wr, W_gate_up, W_down, Ws_gate_up, Ws_down, *, bias=None,
     if rc != 0:
         raise ValueError("oracle.forward: a selected token routes to an expert "
                          "whose weights were not supplied")
+    if k > 1:
+        sel_idx = sel_idx.reshape(n_sel, k)
+        sel_gate = sel_gate.reshape(n_sel, k)
     return out, sel_idx, sel_gate

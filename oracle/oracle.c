@@ -127,6 +127,47 @@ static int route_token(int d, int E, const void *x_t, int x_dtype,
     return best;
 }
 
+/* Top-k router for one token (k >= 1): the k largest fp32 logits, in
+ * descending order, each pass taking the lowest index among the remaining
+ * maxima (strict ">" in ascending order; NaN never wins); margin = k-th
+ * selected logit minus the largest logit left out (+inf when k == E). */
+static void route_token_topk(int d, int E, int k, const void *x_t, int x_dtype,
+                             const void *Wr, int wr_dtype, const float *bias,
+                             int32_t *sel, float *lsel, float *margin_out) {
+    float *l = (float *)malloc(sizeof(float) * (size_t)E);
+    char *taken = (char *)calloc((size_t)E, 1);
+    for (int e = 0; e < E; ++e) {
+        double acc = 0.0;
+        for (int kk = 0; kk < d; ++kk)
+            acc += load_elem(x_t, x_dtype, (size_t)kk) *
+                   load_elem(Wr, wr_dtype, (size_t)kk * (size_t)E + (size_t)e);
+        if (bias) acc += (double)bias[e];
+        l[e] = (float)acc;
+    }
+    for (int j = 0; j < k; ++j) {
+        int best = -1;
+        float lb = -INFINITY;
+        for (int e = 0; e < E; ++e) {
+            if (taken[e] || l[e] != l[e]) continue;      /* NaN never wins */
+            if (best < 0 || l[e] > lb) {                 /* ties keep the lower index */
+                best = e;
+                lb = l[e];
+            }
+        }
+        for (int e = 0; best < 0 && e < E; ++e)          /* only NaN logits left */
+            if (!taken[e]) best = e;
+        taken[best] = 1;
+        sel[j] = best;
+        lsel[j] = l[best];
+    }
+    float rest = -INFINITY;
+    for (int e = 0; e < E; ++e)
+        if (!taken[e] && l[e] > rest) rest = l[e];
+    if (margin_out) *margin_out = (k < E) ? (float)((double)lsel[k - 1] - (double)rest) : INFINITY;
+    free(l);
+    free(taken);
+}
+
 /* One SwiGLU FFN on one input row u[d]:
  *   a = u . Wgu  (2Fw values), h_j = silu(a_j) * a_{Fw+j},  y += h . Wd.  */
 static void swiglu_ffn_accumulate(int d, int Fw, const double *u,
@@ -161,6 +202,19 @@ void oracle_route(int T, int d, int E, const void *x, int x_dtype,
     }
 }
 
+/* Top-k routing for all T tokens: idx / lsel [T][k], margin [T]. */
+void oracle_route_topk(int T, int d, int E, int k, const void *x, int x_dtype,
+                       const void *Wr, int wr_dtype, const float *bias,
+                       int32_t *idx, float *lsel, float *margin) {
+    size_t xs = (x_dtype == ORACLE_F32) ? 4 : 2;
+#pragma omp parallel for schedule(static)
+    for (int t = 0; t < T; ++t) {
+        const char *x_t = (const char *)x + (size_t)t * (size_t)d * xs;
+        route_token_topk(d, E, k, x_t, x_dtype, Wr, wr_dtype, bias, idx + (size_t)t * k,
+                         lsel + (size_t)t * k, margin ? &margin[t] : NULL);
+    }
+}
+
 /* Per-expert counts, exclusive offsets and the stable permutation
  * perm[p] = token at expert-sorted slot p (order by expert, then token). */
 void oracle_permutation(int T, int E, const int32_t *idx, int32_t *counts,
@@ -181,7 +235,7 @@ void oracle_permutation(int T, int E, const int32_t *idx, int32_t *counts,
  * reaches; returns -1 if a needed expert is missing, 0 on success.
  * sel_idx / sel_gate (optional) receive each selected token's expert and
  * gate. */
-int oracle_forward(int T, int d, int E, int F, int Fs,
+int oracle_forward(int T, int d, int E, int k, int F, int Fs,
                    const void *x, int x_dtype,
                    const void *Wr, int wr_dtype, const float *bias,
                    const void *const *W_gate_up, const void *const *W_down,
@@ -216,16 +270,24 @@ int oracle_forward(int T, int d, int E, int F, int Fs,
             free(h);
             continue;
         }
-        float lmax;
-        int e = route_token(d, E, x_t, x_dtype, Wr, wr_dtype, bias, &lmax, NULL);
-        double g = sigmoid((double)lmax);
-        if (sel_idx) sel_idx[i] = e;
-        if (sel_gate) sel_gate[i] = g;
-        /* routed expert on the sigmoid-gated input */
-        if (!W_gate_up[e] || !W_down[e]) {
-            missing |= 1;
+        int32_t sel_e[8];
+        float sel_l[8];
+        if (k == 1) {
+            sel_e[0] = route_token(d, E, x_t, x_dtype, Wr, wr_dtype, bias, &sel_l[0], NULL);
         } else {
-            for (int k = 0; k < d; ++k) u[k] = g * load_elem(x_t, x_dtype, (size_t)k);
+            route_token_topk(d, E, k, x_t, x_dtype, Wr, wr_dtype, bias, sel_e, sel_l, NULL);
+        }
+        /* each selected expert on the input gated by its own sigmoid */
+        for (int j = 0; j < k; ++j) {
+            int e = sel_e[j];
+            double g = sigmoid((double)sel_l[j]);
+            if (sel_idx) sel_idx[(size_t)i * k + j] = e;
+            if (sel_gate) sel_gate[(size_t)i * k + j] = g;
+            if (!W_gate_up[e] || !W_down[e]) {
+                missing |= 1;
+                continue;
+            }
+            for (int kk = 0; kk < d; ++kk) u[kk] = g * load_elem(x_t, x_dtype, (size_t)kk);
             swiglu_ffn_accumulate(d, F, u, W_gate_up[e], W_down[e], w_dtype,
                                   s_gate_up ? s_gate_up[e] : NULL,
                                   s_down ? s_down[e] : NULL, a, h, y);

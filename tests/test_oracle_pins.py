@@ -262,3 +262,56 @@ def test_dense_layer_without_experts_is_one_swiglu_ffn(dtype):
     ref = _dense_swiglu(L["x64"], L["Wsgu64"], L["Wsd64"])
     np.testing.assert_allclose(out, ref, rtol=1e-12, atol=1e-12)
     assert np.all(idx == -1)
+
+
+def test_topk_takes_the_k_largest_lowest_index_first_on_ties():
+    """One-hot tokens expose router rows as logits: the top-k list is the
+    row sorted by (value descending, index ascending), as numpy's stable
+    lexsort orders it; the margin is the k-th value minus the next one."""
+    d, E = 6, 5
+    Wr = np.array([[0.0, 2.0, 1.0, 2.0, 2.0],
+                   [3.0, 3.0, 3.0, 3.0, 3.0],
+                   [-1.0, -2.0, -1.0, -3.0, -1.0],
+                   [0.5, 0.25, 0.75, 0.75, 0.1],
+                   [0.0, 0.0, 0.0, 0.0, 1.0],
+                   [-5.0, -4.0, -4.0, -6.0, -4.0]], np.float32)
+    x = np.eye(d, dtype=np.float32)
+    for k in (1, 2, 3, 5):
+        idx, lsel, margin = oracle.route_topk(x, Wr, k)
+        order = np.stack([np.lexsort((np.arange(E), -row)) for row in Wr])[:, :k]
+        assert np.array_equal(idx, order.astype(np.int32))
+        assert np.array_equal(lsel, np.take_along_axis(Wr, order, axis=1))
+        if k < E:
+            nxt = np.take_along_axis(Wr, np.stack([np.lexsort((np.arange(E), -r)) for r in Wr])[:, k:k + 1],
+                                     axis=1)[:, 0]
+            assert np.array_equal(margin, lsel[:, -1] - nxt)
+        else:
+            assert np.all(np.isinf(margin))
+    idx1, lmax1, _ = oracle.route(x, Wr)
+    assert np.array_equal(oracle.route_topk(x, Wr, 1)[0][:, 0], idx1)
+
+
+@pytest.mark.parametrize("dtype", ["f32", "bf16"])
+def test_topk_with_every_expert_sums_each_gated_by_its_own_sigmoid(dtype):
+    """k = E: every expert runs, each on sigmoid(its logit) * x, and their
+    outputs add to the shared expert's -- library matmuls, expert by expert."""
+    rng = np.random.default_rng(12)
+    T, d, E, F, Fs = 5, 32, 3, 16, 24
+    L = _layer(rng, T, d, E, F, Fs, dtype)
+    out, idx, gate = oracle.forward(L["x"], L["Wr"], L["Wgu"], L["Wd"], L["Wsgu"], L["Wsd"], k=E)
+    logits = (L["x64"] @ L["Wr64"]).astype(np.float32).astype(np.float64)
+    ref = _dense_swiglu(L["x64"], L["Wsgu64"], L["Wsd64"])
+    for e in range(E):
+        g = expit(logits[:, e])[:, None]
+        ref = ref + _dense_swiglu(g * L["x64"], L["Wgu64"][e], L["Wd64"][e])
+    scale = np.sqrt(np.mean(ref ** 2))
+    assert np.max(np.abs(out - ref)) <= 1e-12 * scale
+    assert np.array_equal(np.sort(idx, axis=1), np.tile(np.arange(E), (T, 1)))
+
+
+def test_topk_of_one_is_the_top1_layer():
+    rng = np.random.default_rng(13)
+    L = _layer(rng, 11, 32, 6, 16, 16, "bf16")
+    a = oracle.forward(L["x"], L["Wr"], L["Wgu"], L["Wd"], L["Wsgu"], L["Wsd"])
+    b = oracle.forward(L["x"], L["Wr"], L["Wgu"], L["Wd"], L["Wsgu"], L["Wsd"], k=1)
+    assert np.array_equal(a[0], b[0]) and np.array_equal(a[1], b[1])
