@@ -123,6 +123,19 @@ L4MOE_API l4moe_status l4moe_set_workspace(l4moe_handle *h, void *dev_ptr, size_
  * this exists to draw skewed expert loads. */
 L4MOE_API l4moe_status l4moe_set_router_bias(l4moe_handle *h, const float *bias_dev);
 
+/* Experts per token (default 1, the Llama-4 layer).  k > 1: each token runs
+ * its k highest-scoring experts (descending fp32 logit, lower index first on
+ * equal values, NaN never selected), each on the input gated by the sigmoid
+ * of its own logit, and their outputs add to the shared expert's (the
+ * "experts per token" of a token-choice router, torchtune MoE
+ * documentation).  1 <= k <= min(4, E); k > 1 needs bf16 or E4M3 weights and
+ * E % 8 == 0 (else L4MOE_ERR_UNSUPPORTED).  The routing arrays of
+ * l4moe_get_routing then hold T * k entries (entry t * k + j: token t's j-th
+ * expert; margin stays [T]: the k-th logit minus the next one).  Changing k
+ * frees a workspace the handle allocated (it synchronises the device) and
+ * fails with L4MOE_ERR_WORKSPACE when a caller's workspace is too small. */
+L4MOE_API l4moe_status l4moe_set_top_k(l4moe_handle *h, int k);
+
 /* FP8 weights only: per-output-column fp32 scales (device pointers).
  * s_gate_up / s_down are HOST arrays of E device pointers to [2F] / [d]
  * vectors; ss_gate_up [2Fs] and ss_down [d] are the shared expert's.  The
@@ -199,7 +212,9 @@ L4MOE_API l4moe_status l4moe_join_host(l4moe_handle *h, void *stream);
  *   idx[T] int32 expert per token; gate[T] fp32 sigmoid gate; lmax[T] fp32
  *   winning logit; margin[T] fp32 winning minus runner-up logit;
  *   counts[E] int32; offsets[E+1] int32 exclusive prefix of counts;
- *   perm[T] int32 expert-ordered slot -> token (stable by token). */
+ *   perm[T] int32 expert-ordered slot -> token (stable by token).
+ * With top_k = k > 1, idx, gate, lmax and perm hold T * k entries (entry
+ * t * k + j is token t's j-th expert; perm maps a slot to its entry). */
 L4MOE_API l4moe_status l4moe_get_routing(const l4moe_handle *h, const int32_t **idx, const float **gate,
                                const float **lmax, const float **margin, const int32_t **counts,
                                const int32_t **offsets, const int32_t **perm);

@@ -21,7 +21,7 @@ EXPORTED = ("l4moe_create", "l4moe_destroy", "l4moe_workspace_size", "l4moe_set_
             "l4moe_forward_host", "l4moe_get_routing", "l4moe_check_device_status",
             "l4moe_launch_count", "l4moe_last_error", "l4moe_status_string", "l4moe_version",
             "l4moe_set_timing", "l4moe_read_timing", "l4moe_kernel_name",
-            "l4moe_forward_static", "l4moe_join_host")
+            "l4moe_forward_static", "l4moe_join_host", "l4moe_set_top_k")
 STATIC_WORKSPACE_BYTES = 32 << 20
 NUM_KERNELS = 5
 
@@ -74,6 +74,7 @@ def load_library():
     lib.l4moe_status_string.restype = ctypes.c_char_p
     lib.l4moe_version.argtypes = []
     lib.l4moe_set_timing.argtypes = [vp, i32]
+    lib.l4moe_set_top_k.argtypes = [vp, i32]
     lib.l4moe_read_timing.argtypes = [vp, ctypes.POINTER(ctypes.c_double),
                                       ctypes.POINTER(ctypes.c_uint64)]
     lib.l4moe_kernel_name.argtypes = [i32]
@@ -213,15 +214,22 @@ class L4MoE:
         """Make `stream` wait for the output copies of all forward_host calls."""
         self._check(self._lib.l4moe_join_host(self._h, _stream_handle(stream)))
 
+    def set_top_k(self, k: int):
+        """Experts per token (l4moe_set_top_k)."""
+        self._check(self._lib.l4moe_set_top_k(self._h, int(k)))
+        self.top_k = int(k)
+
     def routing(self):
         """Zero-copy device views of the last forward's routing (valid until
-        the next forward on this handle)."""
+        the next forward on this handle); with top_k = k > 1, idx / gate /
+        lmax / perm hold T * k entries (entry t * k + j: token t's j-th)."""
         ptrs = [ctypes.c_void_p() for _ in range(7)]
         self._check(self._lib.l4moe_get_routing(self._h, *[ctypes.byref(p) for p in ptrs]))
         T, E = self.last_T, self.num_experts
-        spec = [("idx", (T,), "<i4"), ("gate", (T,), "<f4"), ("lmax", (T,), "<f4"),
+        Tv = T * getattr(self, "top_k", 1)
+        spec = [("idx", (Tv,), "<i4"), ("gate", (Tv,), "<f4"), ("lmax", (Tv,), "<f4"),
                 ("margin", (T,), "<f4"), ("counts", (E,), "<i4"), ("offsets", (E + 1,), "<i4"),
-                ("perm", (T,), "<i4")]
+                ("perm", (Tv,), "<i4")]
         out = {}
         for (name, shape, ts), p in zip(spec, ptrs):
             out[name] = torch.as_tensor(_DevView(p.value, shape, ts), device="cuda")

@@ -88,7 +88,7 @@ struct SplitPlan {
     int s_gu, s_dn;
 };
 
-SplitPlan split_plan(const l4moe_params& p, int T, int sms) {
+SplitPlan split_plan(const l4moe_params& p, int T, int sms, int k = 1) {
     const int d = p.d_model, F = p.expert_ffn, Fs = p.shared_ffn, E = p.num_experts;
     const int kblk = (int)(128 / act_bytes(p.dtype));  // K elements per k-block
     const int fb_gu_r = (F + 127) / 128, fb_gu_s = (Fs + 127) / 128, fb_dn = (d + 255) / 256;
@@ -115,7 +115,7 @@ SplitPlan split_plan(const l4moe_params& p, int T, int sms) {
         }
         return best;
     };
-    const long long eg = std::min(E, T);  // non-empty routed experts (one token tile each)
+    const long long eg = std::min<long long>(E, (long long)T * k);  // non-empty routed experts
     SplitPlan sp;
     const long long gu_tiles = (long long)fb_gu_s + fb_gu_r * eg;
     sp.s_gu = 2 * gu_tiles < pairs ? pick(gu_tiles, d / kblk) : 1;
@@ -125,20 +125,23 @@ SplitPlan split_plan(const l4moe_params& p, int T, int sms) {
 
 // fp32 partial floats any forward of at most T tokens needs: split gate/up
 // results, and the down's shared + routed results (times its splits).
-size_t part_floats(const l4moe_params& p, int T, int sms) {
+size_t part_floats(const l4moe_params& p, int T, int sms, int k) {
     size_t need = 0;
-    auto add = [&](int t) {
-        const SplitPlan sp = split_plan(p, t, sms);
+    auto add = [&](int t) {  // t tokens: t * k routed entries, t shared rows
+        const SplitPlan sp = split_plan(p, t, sms, k);
+        const size_t tv = (size_t)t * k;
         if (sp.s_gu > 1)
-            need = std::max<size_t>(need, (size_t)sp.s_gu * t * (2ull * p.expert_ffn + 2ull * p.shared_ffn));
-        need = std::max<size_t>(need, 2ull * sp.s_dn * t * p.d_model);
+            need = std::max<size_t>(need, (size_t)sp.s_gu * (tv * 2ull * p.expert_ffn + (size_t)t * 2ull * p.shared_ffn));
+        need = std::max<size_t>(need, (size_t)sp.s_dn * (tv + t) * p.d_model);
     };
     for (int t = 1; t <= std::min<int>(T, (int)kSplitMaxTokens); ++t) add(t);
     add(std::max(T, 1));
     return need;
 }
 
-WsLayout ws_layout(const l4moe_params& p, int T, int sms) {
+// k: selected experts per token (l4moe_set_top_k); the routed rows are the
+// T * k token entries.
+WsLayout ws_layout(const l4moe_params& p, int T, int sms, int k) {
     WsLayout L{};
     size_t off = 0;
     auto take = [&](size_t bytes) {
@@ -147,24 +150,25 @@ WsLayout ws_layout(const l4moe_params& p, int T, int sms) {
         return o;
     };
     const size_t t = (size_t)std::max(T, 1), E = (size_t)p.num_experts, es = act_bytes(p.dtype);
+    const size_t tv = t * (size_t)k;
     L.err = take(256);
-    L.idx = take(4 * t);
-    L.gate = take(4 * t);
-    L.lmax = take(4 * t);
+    L.idx = take(4 * tv);
+    L.gate = take(4 * tv);
+    L.lmax = take(4 * tv);
     L.margin = take(4 * t);
-    L.inv = take(4 * t);
-    L.perm = take(4 * t);
-    L.gslot = take(4 * t);
+    L.inv = take(4 * tv);
+    L.perm = take(4 * tv);
+    L.gslot = take(4 * tv);
     L.counts = take(4 * E);
     L.offsets = take(4 * (E + 1));
     L.tab_gu = take(sizeof(GroupTable));
     L.tab_dn = take(sizeof(GroupTable));
-    L.xg = take(t * p.d_model * es);
-    L.hr = take(t * p.expert_ffn * es);
+    L.xg = take(tv * p.d_model * es);
+    L.hr = take(tv * p.expert_ffn * es);
     L.hs = take(t * p.shared_ffn * es);
     // E4M3 layers: x in f16, token order (the shared expert's operand)
     L.x16 = take(p.dtype == L4MOE_FP8_E4M3 ? t * p.d_model * 2 : 0);
-    L.part = take(sizeof(float) * part_floats(p, (int)t, sms));
+    L.part = take(sizeof(float) * part_floats(p, (int)t, sms, k));
     L.logits = take(sizeof(float) * std::min<size_t>(t, 128) * E);  // expert-split router
     L.device_total = off;
     L.xin = take(2 * t * p.d_model * es);   // host path: two input staging slots
@@ -184,6 +188,7 @@ struct l4moe_handle {
     uint8_t* ws = nullptr;
     size_t ws_bytes = 0;
     int ws_tokens = 0;
+    int top_k = 1;  // selected experts per token (l4moe_set_top_k)
     bool ws_owned = false;
     const float* bias = nullptr;
     std::vector<const float*> s_gu, s_dn;
@@ -301,7 +306,7 @@ l4moe_status ensure_workspace(l4moe_handle* h, int T) {
         h->ws = nullptr;
     }
     const int cap = std::max(T, 256);
-    const WsLayout L = ws_layout(h->p, cap, h->sms);
+    const WsLayout L = ws_layout(h->p, cap, h->sms, h->top_k);
     void* p = nullptr;
     cudaError_t e = cudaMalloc(&p, L.total);
     if (e != cudaSuccess) return cuda_fail(h, e, "workspace cudaMalloc");
@@ -429,7 +434,7 @@ l4moe_status run_layer(l4moe_handle* h, int T, const void* x, const void* Wr, co
                        const CUtensorMap* maps, const float* const* scales = nullptr) {
     const l4moe_params& p = h->p;
     const int d = p.d_model, F = p.expert_ffn, Fs = p.shared_ffn, E = p.num_experts;
-    const WsLayout L = ws_layout(p, ws_tokens, h->sms);
+    const WsLayout L = ws_layout(p, ws_tokens, h->sms, h->top_k);
     unsigned* err = reinterpret_cast<unsigned*>(w + L.err);
     int32_t* idx = reinterpret_cast<int32_t*>(w + L.idx);
     float* gate = reinterpret_cast<float*>(w + L.gate);
@@ -464,18 +469,29 @@ l4moe_status run_layer(l4moe_handle* h, int T, const void* x, const void* Wr, co
     constexpr uint32_t rb = GCfg::B_BOX_ROWS, rs = GCfg::B_SMALL_ROWS;
     CUtensorMap m_x;
     BMaps bm_gu, bm_dn;
+    // rows: T token rows (x, the shared hidden rows), or T * k entries for
+    // the routed rows (x in expert order, the routed hidden rows)
+    const int k = h->top_k;
+    const int Tv = T * k;
+    auto act_n = [&](CUtensorMap* m, CUtensorMapDataType dt, const void* base, int width, int nrows,
+                     uint32_t rows) {
+        return encode_2d(m, dt, base, (uint64_t)width, (uint64_t)nrows, (uint64_t)width * sizeof(ET), bk, rows);
+    };
     auto act = [&](CUtensorMap* m, CUtensorMapDataType dt, const void* base, int width, uint32_t rows) {
-        return encode_2d(m, dt, base, (uint64_t)width, (uint64_t)T, (uint64_t)width * sizeof(ET), bk, rows);
+        return act_n(m, dt, base, width, T, rows);
+    };
+    auto act_r = [&](CUtensorMap* m, CUtensorMapDataType dt, const void* base, int width, uint32_t rows) {
+        return act_n(m, dt, base, width, Tv, rows);
     };
     const void* xs = FP8W ? (const void*)x16 : x;  // the shared expert's operand
     // without experts (F may be 0) the routed hidden descriptors are never
     // read: give them the shared hidden rows to describe
     const void* hrm = F > 0 ? (const void*)hr : (const void*)hs;
     const int Fr = F > 0 ? F : Fs;
-    if (!act(&m_x, adt, x, d, 64) || !act(&bm_gu.routed, gdt, xg, d, rb) ||
-        !act(&bm_gu.routed_small, gdt, xg, d, rs) || !act(&bm_gu.shared, gdt, xs, d, rb) ||
-        !act(&bm_gu.shared_small, gdt, xs, d, rs) || !act(&bm_dn.routed, gdt, hrm, Fr, rb) ||
-        !act(&bm_dn.routed_small, gdt, hrm, Fr, rs) || !act(&bm_dn.shared, gdt, hs, Fs, rb) ||
+    if (!act(&m_x, adt, x, d, 64) || !act_r(&bm_gu.routed, gdt, xg, d, rb) ||
+        !act_r(&bm_gu.routed_small, gdt, xg, d, rs) || !act(&bm_gu.shared, gdt, xs, d, rb) ||
+        !act(&bm_gu.shared_small, gdt, xs, d, rs) || !act_r(&bm_dn.routed, gdt, hrm, Fr, rb) ||
+        !act_r(&bm_dn.routed_small, gdt, hrm, Fr, rs) || !act(&bm_dn.shared, gdt, hs, Fs, rb) ||
         !act(&bm_dn.shared_small, gdt, hs, Fs, rs))
         return fail(h, L4MOE_ERR_CUDA, "cuTensorMapEncodeTiled failed for an activation");
 
@@ -492,7 +508,7 @@ l4moe_status run_layer(l4moe_handle* h, int T, const void* x, const void* Wr, co
     const int fb_gu_s = (Fs + fpg - 1) / fpg;
     const int fb_dn = (d + fpd - 1) / fpd;
     // split-K k-ranges when a small batch leaves too few tiles
-    const SplitPlan plan = split_plan(p, T, h->sms);
+    const SplitPlan plan = split_plan(p, T, h->sms, h->top_k);
     const int s_gu = plan.s_gu, s_dn = plan.s_dn;
     if (E > 0) {
         LaunchTimer t_router(h, 0, st);
@@ -518,7 +534,7 @@ l4moe_status run_layer(l4moe_handle* h, int T, const void* x, const void* Wr, co
             }
             launch_kc(router_mma_kernel, dim3(tiles, E / n_chunk, kslices), dim3(128), rmma::SMEM_BYTES, st,
                       kslices == 1 ? 0u : (unsigned)kslices, m_x, m_wr, (const float*)h->bias,
-                      T, d, E, n_chunk, logits, idx, gate, lmax, margin, err);
+                      T, d, E, n_chunk, logits, idx, gate, lmax, margin, err, k);
         } else {
             launch_router<ET>(x, Wr, h->bias, T, d, E, idx, gate, lmax, margin, st);
         }
@@ -528,15 +544,15 @@ l4moe_status run_layer(l4moe_handle* h, int T, const void* x, const void* Wr, co
         const size_t psmem = sizeof(int) * (34 * (size_t)E + 1);
         LaunchTimer t_perm(h, 1, st);
         launch_k(permute_kernel, dim3(1), dim3(1024), psmem, st, (const float*)logits,
-                 gate, lmax, margin, idx, T, E, fb_gu_r * s_gu, fb_gu_s * s_gu, fb_dn * s_dn, counts, offsets,
+                 gate, lmax, margin, idx, T, k, E, fb_gu_r * s_gu, fb_gu_s * s_gu, fb_dn * s_dn, counts, offsets,
                  perm, inv, tab_gu, tab_dn, err);
         t_perm.stop();
         L4MOE_CHECK_LAUNCH("permute launch");
 
-        const int sc_blocks = std::min((T + 7) / 8, h->sms * 8);
+        const int sc_blocks = std::min((Tv + 7) / 8, h->sms * 8);
         LaunchTimer t_rows(h, 2, st);
         launch_k(permute_rows_kernel<ET, GT>, dim3(sc_blocks), dim3(256), 0, st, static_cast<const ET*>(x),
-                 (const float*)gate, (const int32_t*)inv, T, d, xg, gslot, FP8W ? x16 : (GT*)nullptr);
+                 (const float*)gate, (const int32_t*)inv, T, k, d, xg, gslot, FP8W ? x16 : (GT*)nullptr);
         t_rows.stop();
         L4MOE_CHECK_LAUNCH("row permutation launch");
     } else {
@@ -550,13 +566,14 @@ l4moe_status run_layer(l4moe_handle* h, int T, const void* x, const void* Wr, co
             const int sc_blocks = std::min((T + 7) / 8, h->sms * 8);
             LaunchTimer t_rows(h, 2, st);
             launch_k(permute_rows_kernel<ET, GT>, dim3(sc_blocks), dim3(256), 0, st, static_cast<const ET*>(x),
-                     (const float*)nullptr, (const int32_t*)nullptr, T, d, x16, (float*)nullptr, (GT*)nullptr);
+                     (const float*)nullptr, (const int32_t*)nullptr, T, 1, d, x16, (float*)nullptr, (GT*)nullptr);
             t_rows.stop();
             L4MOE_CHECK_LAUNCH("row conversion launch");
         }
     }
 
-    const int tb = (T + kTokTile - 1) / kTokTile;
+    const int tb = (T + kTokTile - 1) / kTokTile;     // shared token tiles
+    const int tbv = (Tv + kTokTile - 1) / kTokTile;   // routed entry tiles (bound)
     // CTA pairs: two CTAs (one cluster) per tile, at most one pair per two SMs
     auto grid_for = [&](long long tiles) {
         return 2 * (int)std::max(1LL, std::min<long long>(h->sms / 2, tiles));
@@ -577,7 +594,7 @@ l4moe_status run_layer(l4moe_handle* h, int T, const void* x, const void* Wr, co
     gu.out_shared = hs;          // shared hidden rows, also stored in slot order
     gu.ld_shared = Fs;
     gu.rowmap_routed = nullptr;
-    gu.rowmap_shared = E > 0 ? inv : nullptr;
+    gu.rowmap_shared = nullptr;  // shared hidden rows in token order
     gu.colscale_routed = gslot;  // sigmoid gate of each routed slot
     gu.wscale = FP8W ? scales : nullptr;
     float* part = reinterpret_cast<float*>(w + L.part);
@@ -585,20 +602,20 @@ l4moe_status run_layer(l4moe_handle* h, int T, const void* x, const void* Wr, co
     gu.partial_out = s_gu > 1 ? 1 : 0;
     gu.part_routed = part;
     gu.ld_part_routed = 2LL * F;
-    gu.part_stride_routed = (long long)T * 2 * F;
-    gu.part_shared = part + (size_t)s_gu * T * 2 * F;
+    gu.part_stride_routed = (long long)Tv * 2 * F;
+    gu.part_shared = part + (size_t)s_gu * Tv * 2 * F;
     gu.ld_part_shared = 2LL * Fs;
     gu.part_stride_shared = (long long)T * 2 * Fs;
     gu.err = err;
     LaunchTimer t_gu(h, 3, st);
     launch_gemm<MODE_GATEUP, ET, FP8W>(
-        grid_for(s_gu * ((long long)fb_gu_s * tb + (long long)fb_gu_r * (tb + std::min(E, T)))),
+        grid_for(s_gu * ((long long)fb_gu_s * tb + (long long)fb_gu_r * (tbv + std::min(E, Tv)))),
         bm_gu, gu, st);
     if (s_gu > 1) {
-        const long long n = (long long)T * (F + Fs);
+        const long long n = (long long)Tv * F + (long long)T * Fs;
         launch_k(gateup_finish_kernel<GT>, dim3((int)std::min<long long>((n + 255) / 256, 4LL * h->sms)),
                  dim3(256), 0, st, (const float*)gu.part_routed, gu.ld_part_routed, gu.part_stride_routed,
-                 (const float*)gu.part_shared, gu.ld_part_shared, gu.part_stride_shared, s_gu, T, F, Fs,
+                 (const float*)gu.part_shared, gu.ld_part_shared, gu.part_stride_shared, s_gu, Tv, T, F, Fs,
                  (const float*)gslot, hr, hs);
         ++h->launches;
     }
@@ -618,7 +635,7 @@ l4moe_status run_layer(l4moe_handle* h, int T, const void* x, const void* Wr, co
     dn.out_shared = out;
     dn.ld_shared = d;
     dn.rowmap_routed = perm;     // slot -> token: un-permute on store
-    dn.rowmap_shared = E > 0 ? perm : nullptr;  // H_s in slot order (token order without experts)
+    dn.rowmap_shared = nullptr;  // shared rows are tokens
     dn.colscale_routed = nullptr;
     dn.wscale = FP8W ? scales + (E + 1) : nullptr;
     dn.ksplit = s_dn;
@@ -626,20 +643,20 @@ l4moe_status run_layer(l4moe_handle* h, int T, const void* x, const void* Wr, co
     // partial slots: [0, s_dn) routed, [s_dn, 2 s_dn) shared
     dn.part_routed = part;
     dn.ld_part_routed = d;
-    dn.part_stride_routed = (long long)T * d;
-    dn.part_shared = part + (size_t)s_dn * T * d;
+    dn.part_stride_routed = (long long)Tv * d;  // routed rows: the T * k entries
+    dn.part_shared = part + (size_t)s_dn * Tv * d;
     dn.ld_part_shared = d;
     dn.part_stride_shared = (long long)T * d;
     dn.err = err;
     LaunchTimer t_dn(h, 4, st);
-    launch_gemm<MODE_DOWN, ET, FP8W>(grid_for(s_dn * (long long)fb_dn * (2 * tb + std::min(E, T))),
+    launch_gemm<MODE_DOWN, ET, FP8W>(grid_for(s_dn * (long long)fb_dn * (tb + tbv + std::min(E, Tv))),
                                      bm_dn, dn, st);
     {
         const long long n = (long long)T * d;
         // the routed planes then the shared ones; without experts only the shared
         launch_k(down_finish_kernel<ET>, dim3((int)std::min<long long>((n / 4 + 255) / 256, 4LL * h->sms)),
-                 dim3(256), 0, st, (const float*)(E > 0 ? part : dn.part_shared), dn.part_stride_routed,
-                 E > 0 ? 2 * s_dn : s_dn, n, static_cast<ET*>(out));
+                 dim3(256), 0, st, (const float*)part, dn.part_stride_routed, E > 0 ? s_dn : 0,
+                 (const float*)dn.part_shared, dn.part_stride_shared, s_dn, k, d, n, static_cast<ET*>(out));
         ++h->launches;
     }
     t_dn.stop();
@@ -762,7 +779,7 @@ l4moe_status l4moe_forward_static(l4moe_handle* h, int T, const void* x, const v
     if (s != L4MOE_OK || T == 0) return s;
     const int E = h->p.num_experts;
     const bool fp8 = h->p.dtype == L4MOE_FP8_E4M3;
-    const size_t ws_bytes = (ws_layout(h->p, T, h->sms).device_total + 255) & ~size_t(255);
+    const size_t ws_bytes = (ws_layout(h->p, T, h->sms, h->top_k).device_total + 255) & ~size_t(255);
     const size_t maps_bytes = sizeof(CUtensorMap) * 2 * (E + 1);
     const size_t scales_bytes = fp8 ? sizeof(float*) * 2 * (E + 1) : 0;
     if (ws_bytes + maps_bytes + scales_bytes > L4MOE_STATIC_WORKSPACE_BYTES) {
@@ -781,7 +798,7 @@ l4moe_status l4moe_forward_static(l4moe_handle* h, int T, const void* x, const v
     // the error word (the only state a forward expects to start at zero)
     cudaError_t e = cudaMemcpyAsync(maps, h->h_maps.data(), maps_bytes, cudaMemcpyHostToDevice, st);
     if (e != cudaSuccess) return cuda_fail(h, e, "static descriptor upload");
-    e = cudaMemsetAsync(base + ws_layout(h->p, T, h->sms).err, 0, sizeof(unsigned), st);
+    e = cudaMemsetAsync(base + ws_layout(h->p, T, h->sms, h->top_k).err, 0, sizeof(unsigned), st);
     if (e != cudaSuccess) return cuda_fail(h, e, "static error word clear");
     const float* const* scales = nullptr;
     if (fp8) {  // the E4M3 scale-pointer table follows the descriptors
@@ -872,7 +889,28 @@ void l4moe_destroy(l4moe_handle* h) {
 
 size_t l4moe_workspace_size(const l4moe_handle* h, int max_tokens) {
     if (!h || max_tokens < 0) return 0;
-    return ws_layout(h->p, max_tokens, h->sms).total;
+    return ws_layout(h->p, max_tokens, h->sms, h->top_k).total;
+}
+
+l4moe_status l4moe_set_top_k(l4moe_handle* h, int k) {
+    if (!h) return L4MOE_ERR_ARG;
+    const int E = h->p.num_experts;
+    if (k < 1 || k > kMaxTopK || (E > 0 && k > E) || (E == 0 && k != 1))
+        return fail(h, L4MOE_ERR_ARG, "top_k must be in [1, min(4, E)]");
+    if (k > 1 && (h->p.dtype == L4MOE_F32 || E % 8 != 0))
+        return fail(h, L4MOE_ERR_UNSUPPORTED,
+                    "top_k > 1 takes the tensor-core router: bf16 or E4M3 weights and E % 8 == 0");
+    if (k == h->top_k) return L4MOE_OK;
+    if (h->ws && !h->ws_owned && h->ws_bytes < ws_layout(h->p, h->ws_tokens, h->sms, k).total)
+        return fail(h, L4MOE_ERR_WORKSPACE, "the caller's workspace is too small for this top_k");
+    if (h->ws && h->ws_owned) {  // re-laid out (and re-sized) by the next forward
+        cudaError_t e = cudaFree(h->ws);  // synchronises: work in flight is done
+        h->ws = nullptr;
+        h->ws_tokens = 0;
+        if (e != cudaSuccess) return cuda_fail(h, e, "workspace cudaFree");
+    }
+    h->top_k = k;
+    return L4MOE_OK;
 }
 
 l4moe_status l4moe_set_workspace(l4moe_handle* h, void* dev_ptr, size_t bytes, int max_tokens) {
@@ -880,7 +918,7 @@ l4moe_status l4moe_set_workspace(l4moe_handle* h, void* dev_ptr, size_t bytes, i
     if (!dev_ptr || max_tokens < 1) return fail(h, L4MOE_ERR_ARG, "null workspace or max_tokens < 1");
     if (reinterpret_cast<uintptr_t>(dev_ptr) & 255u)
         return fail(h, L4MOE_ERR_ALIGN, "workspace must be 256-byte aligned");
-    if (bytes < ws_layout(h->p, max_tokens, h->sms).total)
+    if (bytes < ws_layout(h->p, max_tokens, h->sms, h->top_k).total)
         return fail(h, L4MOE_ERR_WORKSPACE, "workspace smaller than l4moe_workspace_size");
     if (h->ws_owned && h->ws) cudaFree(h->ws);
     h->ws = static_cast<uint8_t*>(dev_ptr);
@@ -947,7 +985,7 @@ l4moe_status l4moe_forward_host(l4moe_handle* h, int T, const void* x_host, cons
                 return cuda_fail(h, e, "copy event creation");
     }
     cudaStream_t st = static_cast<cudaStream_t>(stream);
-    const WsLayout L = ws_layout(h->p, h->ws_tokens, h->sms);
+    const WsLayout L = ws_layout(h->p, h->ws_tokens, h->sms, h->top_k);
     const size_t slab = (size_t)h->ws_tokens * h->p.d_model * act_bytes(h->p.dtype);
     const int b = h->host_slot;
     h->host_slot ^= 1;
@@ -993,7 +1031,7 @@ l4moe_status l4moe_get_routing(const l4moe_handle* h, const int32_t** idx, const
                                const float** lmax, const float** margin, const int32_t** counts,
                                const int32_t** offsets, const int32_t** perm) {
     if (!h || !h->ws) return L4MOE_ERR_ARG;
-    const WsLayout L = ws_layout(h->p, h->ws_tokens, h->sms);
+    const WsLayout L = ws_layout(h->p, h->ws_tokens, h->sms, h->top_k);
     if (idx) *idx = reinterpret_cast<const int32_t*>(h->ws + L.idx);
     if (gate) *gate = reinterpret_cast<const float*>(h->ws + L.gate);
     if (lmax) *lmax = reinterpret_cast<const float*>(h->ws + L.lmax);
@@ -1012,10 +1050,10 @@ l4moe_status l4moe_check_device_status(l4moe_handle* h, void* stream) {
     if (e != cudaSuccess) return cuda_fail(h, e, "stream synchronize");
     if (!h->ws) return L4MOE_OK;
     unsigned word = 0;
-    e = cudaMemcpy(&word, h->ws + ws_layout(h->p, h->ws_tokens, h->sms).err, sizeof(word), cudaMemcpyDeviceToHost);
+    e = cudaMemcpy(&word, h->ws + ws_layout(h->p, h->ws_tokens, h->sms, h->top_k).err, sizeof(word), cudaMemcpyDeviceToHost);
     if (e != cudaSuccess) return cuda_fail(h, e, "error word read");
     if (word == 0) return L4MOE_OK;
-    cudaMemset(h->ws + ws_layout(h->p, h->ws_tokens, h->sms).err, 0, sizeof(word));
+    cudaMemset(h->ws + ws_layout(h->p, h->ws_tokens, h->sms, h->top_k).err, 0, sizeof(word));
     char msg[160];
     snprintf(msg, sizeof msg, "device error word 0x%x (1: producer wait, 2: MMA wait, 4: epilogue wait, 8: bad expert index)", word);
     return fail(h, (word & 7u) ? L4MOE_ERR_TIMEOUT : L4MOE_ERR_ARG, msg);

@@ -661,10 +661,11 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(GemmCfg<MODE, ET, FP
 template <typename ET>
 __global__ void __launch_bounds__(256) gateup_finish_kernel(
     const float* __restrict__ part_r, long long ld_r, long long stride_r, const float* __restrict__ part_s,
-    long long ld_s, long long stride_s, int ksplit, int T, int F, int Fs,
+    long long ld_s, long long stride_s, int ksplit, int Tr, int T, int F, int Fs,
     const float* __restrict__ gslot, ET* __restrict__ hr, ET* __restrict__ hs) {
     pdl_enter();
-    const long long n_r = (long long)T * F, n = n_r + (long long)T * Fs;
+    // Tr routed rows (token entries), T shared rows
+    const long long n_r = (long long)Tr * F, n = n_r + (long long)T * Fs;
     for (long long i = blockIdx.x * (long long)blockDim.x + threadIdx.x; i < n;
          i += (long long)gridDim.x * blockDim.x) {
         const bool shared = i >= n_r;
@@ -683,19 +684,30 @@ __global__ void __launch_bounds__(256) gateup_finish_kernel(
     }
 }
 
-// Finish of the down contraction: out = rn(sum of the partials in order)
-// (shared and routed results, times the split-K ranges).  n % 4 == 0; four
-// outputs per thread with 16-byte loads.
+// Down finish: out[t] = rn(sum over splits s and selected experts j of the
+// routed partial of entry t * k + j, then sum over s of the shared partial)
+// -- one rounding, a fixed order.  Partials: routed [splits_r][T * k][d],
+// shared [splits_s][T][d] (fp32, rows un-permuted to entries / tokens).
+// Four outputs per thread; d % 4 == 0.
 template <typename ET>
-__global__ void __launch_bounds__(256) down_finish_kernel(const float* __restrict__ part, long long stride,
-                                                          int nparts, long long n, ET* __restrict__ out) {
+__global__ void __launch_bounds__(256) down_finish_kernel(const float* __restrict__ part_r, long long stride_r,
+                                                          int splits_r, const float* __restrict__ part_s,
+                                                          long long stride_s, int splits_s, int k, int d,
+                                                          long long n, ET* __restrict__ out) {
     pdl_enter();
     const long long n4 = n >> 2;
+    const int d4 = d >> 2;
     for (long long i = blockIdx.x * (long long)blockDim.x + threadIdx.x; i < n4;
          i += (long long)gridDim.x * blockDim.x) {
+        const long long t = i / d4, c4 = i % d4;
         float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
-        for (int s = 0; s < nparts; ++s) {
-            const float4 v = reinterpret_cast<const float4*>(part + stride * s)[i];
+        for (int s = 0; s < splits_r; ++s)
+            for (int j = 0; j < k; ++j) {
+                const float4 v = reinterpret_cast<const float4*>(part_r + stride_r * s)[(t * k + j) * d4 + c4];
+                acc.x += v.x, acc.y += v.y, acc.z += v.z, acc.w += v.w;
+            }
+        for (int s = 0; s < splits_s; ++s) {
+            const float4 v = reinterpret_cast<const float4*>(part_s + stride_s * s)[i];
             acc.x += v.x, acc.y += v.y, acc.z += v.z, acc.w += v.w;
         }
         if constexpr (sizeof(ET) == 2) {

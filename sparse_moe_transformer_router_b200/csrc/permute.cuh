@@ -12,6 +12,7 @@
 #include <cstdint>
 
 #include "ptx.cuh"
+#include "topk.cuh"
 
 namespace l4moe {
 
@@ -126,19 +127,24 @@ __host__ __device__ __forceinline__ int tile_at(int L, int heavy, int total) {
 // Single CTA of 1024 threads.  Writes counts[E], offsets[E+1], perm[T]
 // (slot -> token), inv[T] (token -> slot) and two work lists:
 //   tab_gu : shared expert (rows T) then the routed experts, gate/up GEMM
-//   tab_dn : shared expert (rows = all T slots) then the routed experts,
+//   tab_dn : shared expert (rows T, token order) then the routed experts,
 //            down GEMM (the two contractions meet in fp32 partials)
 // smem: wcnt[32][E] + running[E] ints.
 //
+// Top-k (k >= 1): each token owns k entries n = t * k + j (its j-th
+// selected expert), and the routed rows are these T * k entries: idx, gate,
+// inv are [T * k], perm maps a slot to its entry, and the routed groups'
+// rows add up to T * k while the shared expert keeps its T token rows.
+//
 // logits != null (expert-split router, logits [T][E] biased fp32): first
-// finish the routing here -- per token, the arg-max over the E logits
-// (lowest index on ties, NaN never wins), the runner-up margin and the
-// sigmoid gate -- writing idx, gate, lmax and margin.
+// finish the routing here -- per token, the k largest of the E logits
+// (lower index first on ties, NaN never selected), the margin of the k-th
+// to the next one and the sigmoid gates -- writing idx, gate, lmax, margin.
 __global__ void __launch_bounds__(1024) permute_kernel(const float* __restrict__ logits,
                                                        float* __restrict__ gate,
                                                        float* __restrict__ lmax,
                                                        float* __restrict__ margin,
-                                                       int32_t* __restrict__ idx, int T,
+                                                       int32_t* __restrict__ idx, int T, int k,
                                                        int E, int fb_gu_routed, int fb_gu_shared,
                                                        int fb_down, int32_t* __restrict__ counts,
                                                        int32_t* __restrict__ offsets,
@@ -155,51 +161,60 @@ __global__ void __launch_bounds__(1024) permute_kernel(const float* __restrict__
 
     if (logits) {
         // one warp per token: lane owns experts lane, lane+32, ... (ascending
-        // inside the lane); the warp then keeps the larger value, lower index
+        // inside the lane, so each lane's list is in selection order); the
+        // warp then takes k + 1 heads, each the first by (value, then index)
         for (int t = warp; t < T; t += 32) {
-            float best = -INFINITY, second = -INFINITY;
-            int bi = 0x7fffffff;
-            for (int e = lane; e < E; e += 32) {
-                const float l = logits[(size_t)t * E + e];
-                if (l > best) {
-                    second = best;
-                    best = l;
-                    bi = e;
-                } else if (l > second) {
-                    second = l;
-                }
-            }
-            if (bi == 0x7fffffff) bi = lane;  // no finite winner in this lane
+            TopK tk;
+            tk.init();
+            for (int e = lane; e < E; e += 32) tk.offer(logits[(size_t)t * E + e], e);
+            TopK out;
+            out.init();
+            int pos = 0;  // entries of this lane's list already taken
 #pragma unroll
-            for (int off = 16; off > 0; off >>= 1) {
-                const float ob = __shfl_xor_sync(0xffffffffu, best, off);
-                const float os = __shfl_xor_sync(0xffffffffu, second, off);
-                const int oi = __shfl_xor_sync(0xffffffffu, bi, off);
-                if (ob > best || (ob == best && oi < bi)) {
-                    second = fmaxf(os, best);
-                    best = ob;
-                    bi = oi;
-                } else {
-                    second = fmaxf(second, ob);
+            for (int j = 0; j <= kMaxTopK; ++j) {
+                float hv = tk.value(pos);
+                int hi = pos <= kMaxTopK ? tk.index(pos) : -1;
+                int hl = lane;
+#pragma unroll
+                for (int off = 16; off > 0; off >>= 1) {
+                    const float ov = __shfl_xor_sync(0xffffffffu, hv, off);
+                    const int oi = __shfl_xor_sync(0xffffffffu, hi, off);
+                    const int ol = __shfl_xor_sync(0xffffffffu, hl, off);
+                    if (topk_before(ov, oi, hv, hi)) {
+                        hv = ov;
+                        hi = oi;
+                        hl = ol;
+                    }
                 }
+                out.v[j] = hv;
+                out.i[j] = hi;
+                if (hl == lane && hi >= 0) ++pos;
             }
             if (lane == 0) {
-                idx[t] = bi;
-                lmax[t] = best;
-                margin[t] = best - second;
-                gate[t] = 1.0f / (1.0f + expf(-best));
+                out.fill_empty(k);
+#pragma unroll
+                for (int j = 0; j < kMaxTopK; ++j) {
+                    if (j < k) {
+                        const size_t n = (size_t)t * k + j;
+                        idx[n] = out.i[j];
+                        lmax[n] = out.v[j];
+                        gate[n] = 1.0f / (1.0f + expf(-out.v[j]));
+                    }
+                }
+                margin[t] = out.value(k - 1) - out.value(k);
             }
         }
         __syncthreads();
     }
+    const int Tv = T * k;  // entries: token t's j-th expert is entry t * k + j
     for (int e = tid; e < E; e += 1024) running[e] = 0;
     __syncthreads();
-    for (int c0 = 0; c0 < T; c0 += 1024) {
+    for (int c0 = 0; c0 < Tv; c0 += 1024) {
         for (int i = tid; i < 32 * E; i += 1024) wcnt[i] = 0;
         __syncthreads();
         const int t = c0 + tid;
         int e = -1;
-        if (t < T) {
+        if (t < Tv) {
             e = idx[t];
             if (e < 0 || e >= E) {
                 atomicOr(err, DEV_ERR_BAD_INDEX);
@@ -251,7 +266,7 @@ __global__ void __launch_bounds__(1024) permute_kernel(const float* __restrict__
         }
     }
     __syncthreads();
-    for (int t = tid; t < T; t += 1024) {
+    for (int t = tid; t < Tv; t += 1024) {
         const int e = idx[t];
         if (e >= 0 && e < E) {
             const int slot = soff[e] + inv[t];
@@ -273,8 +288,8 @@ __global__ void __launch_bounds__(1024) permute_kernel(const float* __restrict__
     }
 }
 
-// Expert-ordered copy of the input rows, xp[inv[t]] = x[t], and the gate of
-// each slot, gate_slot[inv[t]] = gate[t].  The sigmoid gate scales the
+// Expert-ordered copy of the input rows, xp[inv[n]] = x[n / k] for each
+// entry n, and the gate of each slot, gate_slot[inv[n]] = gate[n].  The sigmoid gate scales the
 // routed expert's input, which is linear in the gate/up contraction, so it
 // is applied to the fp32 accumulator in the GEMM epilogue instead of
 // rounding g * x to the activation type here.  OT = IT copies exactly; for
@@ -299,19 +314,21 @@ template <typename IT, typename OT>
 __global__ void __launch_bounds__(256) permute_rows_kernel(const IT* __restrict__ x,
                                                            const float* __restrict__ gate,
                                                            const int32_t* __restrict__ inv,
-                                                           int T, int d, OT* __restrict__ xp,
+                                                           int T, int k, int d, OT* __restrict__ xp,
                                                            float* __restrict__ gate_slot,
                                                            OT* __restrict__ x_tok) {
     pdl_enter();
     static_assert(sizeof(IT) == sizeof(OT), "row copy keeps the element size");
     const int lane = threadIdx.x & 31;
     const int warps = (gridDim.x * blockDim.x) >> 5;
-    for (int t = (blockIdx.x * blockDim.x + threadIdx.x) >> 5; t < T; t += warps) {
-        const int slot = inv ? inv[t] : t;
-        if (lane == 0 && gate_slot) gate_slot[slot] = gate[t];
+    // one warp per entry n = t * k + j (token t's j-th expert)
+    for (int n = (blockIdx.x * blockDim.x + threadIdx.x) >> 5; n < T * k; n += warps) {
+        const int t = n / k;
+        const int slot = inv ? inv[n] : n;
+        if (lane == 0 && gate_slot) gate_slot[slot] = gate[n];
         const uint4* s = reinterpret_cast<const uint4*>(x + (size_t)t * d);
         uint4* o = reinterpret_cast<uint4*>(xp + (size_t)slot * d);
-        uint4* ot = x_tok ? reinterpret_cast<uint4*>(x_tok + (size_t)t * d) : nullptr;
+        uint4* ot = (x_tok && n % k == 0) ? reinterpret_cast<uint4*>(x_tok + (size_t)t * d) : nullptr;
         const int nv = d * (int)sizeof(IT) / 16;
         for (int i = lane; i < nv; i += 32) {
             const uint4 v = cvt_row_vec(s[i], IT{}, OT{});

@@ -21,6 +21,7 @@
 #include <cstdint>
 
 #include "ptx.cuh"
+#include "topk.cuh"
 
 namespace l4moe {
 
@@ -183,7 +184,9 @@ __global__ void __launch_bounds__(NT) router_kernel(const ET* __restrict__ x,
 }
 
 // ---------------------------------------------------------------------------
-// Tensor-core router for bf16 layers with E % 8 == 0 (E <= 256): one CTA per
+// Tensor-core router for bf16 layers with E % 8 == 0 (E <= 256), top-k
+// (k = topk <= kMaxTopK; idx, gate, lmax hold [T][k], margin [T] is the k-th
+// selected logit minus the next one): one CTA per
 // 128-token tile computes the fp32 logits of all E experts with tcgen05 (M =
 // 128 tokens, N = E rounded up to 16, K = d; x rows are the K-major A
 // operand, W_router [d, E] the MN-major B operand), then each of 128 threads
@@ -219,7 +222,7 @@ __global__ void __launch_bounds__(128, 1)
                       const float* __restrict__ bias, int T, int d, int E, int n_chunk,
                       float* __restrict__ logits, int32_t* __restrict__ idx,
                       float* __restrict__ gate, float* __restrict__ lmax,
-                      float* __restrict__ margin, unsigned* err) {
+                      float* __restrict__ margin, unsigned* err, int topk) {
     pdl_enter();
     extern __shared__ uint8_t rsmem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>(
@@ -346,8 +349,8 @@ __global__ void __launch_bounds__(128, 1)
                 }
             }
         }
-        float best = -INFINITY, second = -INFINITY;
-        int bi = 0;
+        TopK tk;
+        tk.init();
         for (int c = 0; !logits && c < n_pad; c += 32) {
             float v[32];
             tmem_ld_32x32(tmem_base + ((uint32_t)(32 * warp) << 16) + (uint32_t)c, v);
@@ -362,23 +365,21 @@ __global__ void __launch_bounds__(128, 1)
 #pragma unroll
             for (int i = 0; i < 32; ++i) {
                 const int e = c + i;
-                if (e < E) {
-                    const float l = v[i] + (bias ? bias[e] : 0.f);
-                    if (l > best) {
-                        second = best;
-                        best = l;
-                        bi = e;
-                    } else if (l > second) {
-                        second = l;
-                    }
-                }
+                if (e < E) tk.offer(v[i] + (bias ? bias[e] : 0.f), e);
             }
         }
         if (!logits && t < T) {
-            idx[t] = bi;
-            lmax[t] = best;
-            margin[t] = best - second;
-            gate[t] = 1.0f / (1.0f + expf(-best));
+            tk.fill_empty(topk);
+#pragma unroll
+            for (int j = 0; j < kMaxTopK; ++j) {
+                if (j < topk) {
+                    const size_t n = (size_t)t * topk + j;
+                    idx[n] = tk.i[j];
+                    lmax[n] = tk.v[j];
+                    gate[n] = 1.0f / (1.0f + expf(-tk.v[j]));
+                }
+            }
+            margin[t] = tk.value(topk - 1) - tk.value(topk);  // k-th against the next one
         }
     }
     if (kreduce) cluster_sync();  // rank 0 done reading the others' shared memory

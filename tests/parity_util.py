@@ -86,8 +86,39 @@ def check_routing(inp: LayerInputs, r: dict, ora=None) -> dict:
             "counts": counts, "same": same, "o_idx": o_idx}
 
 
+def check_routing_topk(inp: LayerInputs, r: dict, k: int) -> dict:
+    """Top-k routing against the oracle's: the selected sets per token (the
+    order of near-equal selected logits may differ from the oracle's fp64
+    rounding, and the layer's output does not depend on it), each selected
+    expert's gate, and the permutation of the CUDA entries (exact)."""
+    E, T = inp.cfg.num_experts, inp.cfg.T
+    x = to_storage_numpy(inp.x)
+    Wr = to_storage_numpy(inp.W_router)
+    b = None if inp.bias is None else inp.bias.detach().cpu().numpy()
+    o_idx, o_lsel, o_margin = oracle.route_topk(x, Wr, k, b)
+    g_idx = r["idx"].cpu().numpy().reshape(T, k)
+    g_gate = r["gate"].cpu().numpy().reshape(T, k).astype(np.float64)
+    keep = o_margin >= MARGIN_EXCLUDE
+    same = np.all(np.sort(g_idx, axis=1) == np.sort(o_idx, axis=1), axis=1)
+    bad = np.nonzero(~same & keep)[0]
+    assert bad.size == 0, f"selected experts differ on {bad.size} tokens, e.g. {bad[:8]}"
+    assert np.all((g_idx >= 0) & (g_idx < E))
+    assert np.all(np.sort(g_idx, axis=1)[:, 1:] != np.sort(g_idx, axis=1)[:, :-1])  # distinct
+    o_gate = 1.0 / (1.0 + np.exp(-o_lsel.astype(np.float64)))
+    og = np.take_along_axis(o_gate, np.argsort(o_idx, axis=1), axis=1)
+    gg = np.take_along_axis(g_gate, np.argsort(g_idx, axis=1), axis=1)
+    assert np.max(np.abs(og[same] - gg[same]), initial=0.0) <= 1e-5
+    counts, offsets, perm = oracle.permutation(g_idx.reshape(-1), E)
+    assert np.array_equal(r["counts"].cpu().numpy(), counts)
+    assert np.array_equal(r["offsets"].cpu().numpy(), offsets)
+    assert np.array_equal(r["perm"].cpu().numpy(), perm)
+    assert counts.sum() == T * k
+    return {"excluded": int(np.count_nonzero(~keep)), "flipped": int(np.count_nonzero(~same)),
+            "counts": counts, "same": same, "o_idx": o_idx}
+
+
 def check_outputs(inp: LayerInputs, out: torch.Tensor, tokens, same_mask=None, o_idx=None,
-                  tol: float | None = None) -> float:
+                  tol: float | None = None, k: int = 1) -> float:
     """Oracle outputs for `tokens` (None = all) against the CUDA output rows.
     Tokens whose routing flipped on a near-tie are skipped.  Asserts the
     per-element bound (tol defaults to the dtype's); returns
@@ -99,7 +130,7 @@ def check_outputs(inp: LayerInputs, out: torch.Tensor, tokens, same_mask=None, o
     tokens = np.asarray(tokens, dtype=np.int32)
     if same_mask is not None:
         tokens = tokens[same_mask[tokens]]
-    need = set(range(c.num_experts)) if o_idx is None else set(int(e) for e in o_idx[tokens])
+    need = set(range(c.num_experts)) if o_idx is None else set(int(e) for e in np.asarray(o_idx)[tokens].ravel())
     x = to_storage_numpy(inp.x)
     Wr = to_storage_numpy(inp.W_router)
     b = None if inp.bias is None else inp.bias.detach().cpu().numpy()
@@ -111,7 +142,7 @@ def check_outputs(inp: LayerInputs, out: torch.Tensor, tokens, same_mask=None, o
                   s_down=[inp.s_down[e].cpu().numpy() if e in need else None for e in range(c.num_experts)],
                   ss_gate_up=inp.ss_gate_up.cpu().numpy(), ss_down=inp.ss_down.cpu().numpy())
     ref, _, _ = oracle.forward(x, Wr, Wgu, Wdn, to_storage_numpy(inp.Ws_gate_up),
-                               to_storage_numpy(inp.Ws_down), bias=b, tokens=tokens, **kw)
+                               to_storage_numpy(inp.Ws_down), bias=b, tokens=tokens, k=k, **kw)
     got = out[torch.as_tensor(tokens, device=out.device, dtype=torch.long)].float().cpu().numpy().astype(np.float64)
     rms = float(np.sqrt(np.mean(ref ** 2)))
     err = np.abs(got - ref)

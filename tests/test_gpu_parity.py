@@ -6,8 +6,8 @@ import numpy as np
 import pytest
 import torch
 
-from parity_util import (check_outputs, check_routing, make_layer, oracle_routing, run_gpu,
-                         sample_tokens)
+from parity_util import (check_outputs, check_routing, check_routing_topk, make_layer,
+                         oracle_routing, run_gpu, sample_tokens)
 from sparse_moe_transformer_router_b200.workloads import (CONFIGS, DECODE_TOKENS,
                                                           E4M3_FINITE_CODES, E4M3_SUBNORMAL_CODES,
                                                           LayerConfig, generate, with_e4m3_codes)
@@ -73,6 +73,53 @@ def test_e4m3_widening_is_exact_for_every_code(codes, scale):
     rep = check_routing(inp, r)
     ratio = check_outputs(inp, out, None, rep["same"], tol=2e-2)
     print(f"max|err|/rms = {ratio:.3e}")
+
+
+TOPK = {
+    # k experts per token: tensor-core router with the top-k epilogue
+    "bf16_k2": (LayerConfig("bf16_k2", 300, 256, 8, 384, 256, "bf16", wr_std=0.1), 2),
+    "bf16_k4_zipf": (LayerConfig("bf16_k4_zipf", 500, 128, 16, 128, 128, "bf16", router="zipf", n_dead=4,
+                                 wr_std=0.05), 4),
+    "fp8_k2": (LayerConfig("fp8_k2", 300, 256, 8, 384, 256, "fp8", wr_std=0.1), 2),
+    # K slices reduced in a cluster before the top-k epilogue
+    "bf16_k2_kslices": (LayerConfig("bf16_k2_kslices", 700, 1024, 16, 256, 256, "bf16", wr_std=0.03), 2),
+    # one token tile with E >= 32: expert-split router, top-k in the permutation
+    "bf16_k3_split_router": (LayerConfig("bf16_k3_sr", 40, 512, 32, 256, 384, "bf16", wr_std=0.05), 3),
+    "bf16_k2_T1": (LayerConfig("bf16_k2_T1", 1, 1024, 64, 512, 512, "bf16", wr_std=0.03), 2),
+}
+
+
+@pytest.mark.parametrize("name", list(TOPK))
+def test_topk_layer_matches_oracle(name):
+    cfg, k = TOPK[name]
+    inp = generate(cfg, seed=0, device="cuda")
+    layer = make_layer(inp)
+    layer.set_top_k(k)
+    out, r = run_gpu(layer, inp)
+    rep = check_routing_topk(inp, r, k)
+    ratio = check_outputs(inp, out, None, rep["same"], rep["o_idx"], k=k)
+    print(f"{name}: k={k} max|err|/rms = {ratio:.3e}, excluded {rep['excluded']}, flipped {rep['flipped']}")
+
+
+def test_top_k_bounds():
+    from sparse_moe_transformer_router_b200.binding import ERR_ARG, ERR_UNSUPPORTED, L4MoEError
+    inp = generate(TOPK["bf16_k2"][0], seed=0, device="cuda")
+    layer = make_layer(inp)
+    for bad in (0, 5, 9):
+        with pytest.raises(L4MoEError) as ei:
+            layer.set_top_k(bad)
+        assert ei.value.status == ERR_ARG
+    f32 = make_layer(generate(SMALL["f32_ragged"], seed=0, device="cuda"))
+    with pytest.raises(L4MoEError) as ei:
+        f32.set_top_k(2)
+    assert ei.value.status == ERR_UNSUPPORTED
+    # back to one expert per token after a top-2 forward
+    layer.set_top_k(2)
+    run_gpu(layer, inp)
+    layer.set_top_k(1)
+    out, r = run_gpu(layer, inp)
+    rep = check_routing(inp, r)
+    check_outputs(inp, out, None, rep["same"])
 
 
 DENSE = {
