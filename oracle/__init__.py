@@ -8,7 +8,7 @@ calls anything here, and this package imports nothing from the product.
 The arithmetic lives in ``oracle.c`` (plain C, fp64 accumulation, OpenMP over
 tokens); this module only compiles it with gcc and marshals numpy arrays.
 Inputs are numpy arrays in their storage dtype: float32, bf16 as uint16 bit
-patterns, E4M3 as uint8 codes.
+patterns, E4M3 as uint8 codes, int8 weights as int8.
 
 Every function is pinned by ``tests/test_oracle_pins.py`` to something other
 than itself (library matmuls on reductions of the layer, closed forms,
@@ -23,7 +23,7 @@ import threading
 
 import numpy as np
 
-F32, BF16, E4M3 = 0, 1, 2
+F32, BF16, E4M3, INT8 = 0, 1, 2, 3
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
 _SRC = os.path.join(_HERE, "oracle.c")
@@ -83,6 +83,8 @@ def _dtype_code(a: np.ndarray) -> int:
         return BF16
     if a.dtype == np.uint8:
         return E4M3
+    if a.dtype == np.int8:
+        return INT8
     raise TypeError(f"oracle: unsupported storage dtype {a.dtype}")
 
 
@@ -162,8 +164,8 @@ def forward(x, Wr, W_gate_up, W_down, Ws_gate_up, Ws_down, *, bias=None,
     """Layer output in fp64 for ``tokens`` (all tokens when None).
 
     W_gate_up / W_down are length-E lists of [d, 2F] / [F, d] arrays; entries
-    may be None for experts no selected token reaches.  For E4M3 weights the
-    per-output-column fp32 scales are required.  k > 1: each token runs its
+    may be None for experts no selected token reaches.  For E4M3 and int8
+    weights the per-output-column fp32 scales are required.  k > 1: each token runs its
     k highest-scoring experts, each on the input gated by the sigmoid of its
     own logit, and their outputs add to the shared expert's.  Returns
     (out f64[n_sel, d], idx int32[n_sel], gate f64[n_sel]), or [n_sel, k]
@@ -194,7 +196,7 @@ def forward(x, Wr, W_gate_up, W_down, Ws_gate_up, Ws_down, *, bias=None,
     if F is None:
         F = Fs
     sgu_ptrs = sdn_ptrs = None
-    if w_code == E4M3:
+    if w_code in (E4M3, INT8):
         sgu_ptrs = (ctypes.c_void_p * E)()
         sdn_ptrs = (ctypes.c_void_p * E)()
         for e in range(E):

@@ -37,6 +37,9 @@
  *   - an optional fp32 router bias b[E] is added to the logits;
  *   - FP8 weights are OCP E4M3 (bias 7, no infinities, S.1111.111 = NaN,
  *     max 448) with one fp32 scale per output column; w = e4m3(q) * scale.
+ *   - int8 weights (KerasFormers "Llama 4" page, "Lower memory": weight-only
+ *     int8 loading) are two's-complement integers with one fp32 scale per
+ *     output column, symmetric (no zero point); w = q * scale.
  *
  * Parity pins (tests/test_oracle_pins.py): E = 1 with the gate forced to 1
  * reduces to two dense SwiGLU FFNs evaluated by a library matmul; a constant
@@ -53,7 +56,7 @@
 #include <omp.h>
 #endif
 
-enum { ORACLE_F32 = 0, ORACLE_BF16 = 1, ORACLE_E4M3 = 2 };
+enum { ORACLE_F32 = 0, ORACLE_BF16 = 1, ORACLE_E4M3 = 2, ORACLE_INT8 = 3 };
 
 /* bf16 is the upper half of an IEEE binary32; widening is exact. */
 double oracle_bf16_to_double(uint16_t b) {
@@ -84,16 +87,17 @@ static double load_elem(const void *p, int dtype, size_t i) {
     case ORACLE_F32: return (double)((const float *)p)[i];
     case ORACLE_BF16: return oracle_bf16_to_double(((const uint16_t *)p)[i]);
     case ORACLE_E4M3: return oracle_e4m3_to_double(((const uint8_t *)p)[i]);
+    case ORACLE_INT8: return (double)((const int8_t *)p)[i];
     default: return NAN;
     }
 }
 
-/* A weight element of a [rows, cols] row-major matrix; for E4M3 the
- * per-output-column scale is applied (dequantisation). */
+/* A weight element of a [rows, cols] row-major matrix; for E4M3 and int8
+ * the per-output-column scale is applied (dequantisation). */
 static double load_weight(const void *W, int dtype, const float *col_scale,
                           size_t row, size_t cols, size_t col) {
     double w = load_elem(W, dtype, row * cols + col);
-    if (dtype == ORACLE_E4M3) w *= (double)col_scale[col];
+    if (dtype == ORACLE_E4M3 || dtype == ORACLE_INT8) w *= (double)col_scale[col];
     return w;
 }
 

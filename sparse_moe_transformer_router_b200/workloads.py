@@ -24,6 +24,7 @@ import numpy as np
 import torch
 
 E4M3_MAX = 448.0
+INT8_MAX = 127.0
 
 
 @dataclass(frozen=True)
@@ -34,7 +35,7 @@ class LayerConfig:
     num_experts: int
     expert_ffn: int
     shared_ffn: int
-    dtype: str            # "f32" | "bf16" | "fp8" (E4M3 weights, bf16 activations)
+    dtype: str            # "f32" | "bf16" | "fp8" / "int8" (E4M3 / int8 weights, bf16 activations)
     router: str = "plain"  # "plain": no bias; "zipf": per-expert bias for Zipf loads
     x_std: float = 1.0
     w_std: float = 0.02
@@ -61,6 +62,9 @@ CONFIGS = {
                                 router="zipf", n_dead=10),
     # the layers without experts: one SwiGLU feed-forward of width 16384
     "maverick_dense_bf16": LayerConfig("maverick_dense_bf16", 8192, 5120, 0, 0, 16384, "bf16"),
+    # weight-only int8 experts (per-output-column scales), Maverick-shaped
+    "maverick_int8": LayerConfig("maverick_int8", 16384, 5120, 128, 8192, 8192, "int8",
+                                 router="zipf", n_dead=10),
 }
 DECODE_TOKENS = (1, 8, 32, 128)
 
@@ -100,6 +104,16 @@ def quantize_e4m3_columns(w: torch.Tensor):
     amax = w.abs().amax(dim=0)
     scale = torch.where(amax > 0, amax / E4M3_MAX, torch.ones_like(amax))
     q = (w / scale).clamp_(-E4M3_MAX, E4M3_MAX).to(torch.float8_e4m3fn)
+    return q, scale.to(torch.float32)
+
+
+def quantize_int8_columns(w: torch.Tensor):
+    """Per-output-column symmetric int8 quantisation of an fp32 [K, N] weight:
+    scale[n] = max_k |w[k, n]| / 127, q = round(w / scale) (to nearest even),
+    clamped to [-127, 127].  Returns (q int8 [K, N], scale f32 [N])."""
+    amax = w.abs().amax(dim=0)
+    scale = torch.where(amax > 0, amax / INT8_MAX, torch.ones_like(amax))
+    q = torch.round(w / scale).clamp_(-INT8_MAX, INT8_MAX).to(torch.int8)
     return q, scale.to(torch.float32)
 
 
@@ -167,6 +181,8 @@ def generate(cfg: LayerConfig, seed: int = 0, device="cpu", experts=None) -> Lay
         w = _normal(shape, cfg.w_std, seed, name, e, device)
         if cfg.dtype == "fp8":
             return quantize_e4m3_columns(w)
+        if cfg.dtype == "int8":
+            return quantize_int8_columns(w)
         return w.to(act), None
 
     W_gu, W_dn, s_gu, s_dn = [], [], [], []
@@ -182,10 +198,10 @@ def generate(cfg: LayerConfig, seed: int = 0, device="cpu", experts=None) -> Lay
         s_dn.append(sb)
     Ws_gu, ss_gu = weight((d, 2 * Fs), "Ws_gate_up", -1)
     Ws_dn, ss_dn = weight((Fs, d), "Ws_down", -1)
-    fp8 = cfg.dtype == "fp8"
+    scaled = cfg.dtype in ("fp8", "int8")
     return LayerInputs(cfg, x, Wr, bias, W_gu, W_dn, Ws_gu, Ws_dn,
-                       s_gu if fp8 else None, s_dn if fp8 else None,
-                       ss_gu if fp8 else None, ss_dn if fp8 else None)
+                       s_gu if scaled else None, s_dn if scaled else None,
+                       ss_gu if scaled else None, ss_dn if scaled else None)
 
 
 # E4M3 code sets for layers that exercise the weight widening: every finite
@@ -195,18 +211,23 @@ E4M3_FINITE_CODES = tuple(c for c in range(256) if c & 0x7F != 0x7F)
 E4M3_SUBNORMAL_CODES = tuple(range(0x00, 0x08)) + tuple(range(0x80, 0x88))
 
 
-def with_e4m3_codes(inp: LayerInputs, codes, scale: float, seed: int) -> LayerInputs:
-    """Replace an E4M3 layer's expert and shared weights by codes drawn
-    uniformly (seeded) from ``codes`` and set every column scale to ``scale``."""
-    assert inp.cfg.dtype == "fp8"
-    table = torch.tensor(codes, dtype=torch.uint8)
+INT8_CODES = tuple(range(-128, 128))
+
+
+def with_weight_codes(inp: LayerInputs, codes, scale: float, seed: int) -> LayerInputs:
+    """Replace an E4M3 (or int8) layer's expert and shared weights by codes
+    drawn uniformly (seeded) from ``codes`` and set every column scale to
+    ``scale``."""
+    assert inp.cfg.dtype in ("fp8", "int8")
+    int8 = inp.cfg.dtype == "int8"
+    table = torch.tensor(codes, dtype=torch.int8 if int8 else torch.uint8)
 
     def draw(w, name, e):
         if w is None:
             return None
         g = torch.Generator().manual_seed(_seed(seed, "codes:" + name, e))
         i = torch.randint(0, table.numel(), tuple(w.shape), generator=g)
-        return table[i].view(torch.float8_e4m3fn).to(w.device)
+        return (table[i] if int8 else table[i].view(torch.float8_e4m3fn)).to(w.device)
 
     def full(s):
         return None if s is None else torch.full_like(s, scale)
@@ -224,7 +245,7 @@ def with_e4m3_codes(inp: LayerInputs, codes, scale: float, seed: int) -> LayerIn
 
 def to_storage_numpy(t: torch.Tensor | None) -> np.ndarray | None:
     """Host copy in storage form: float32 as is, bf16 as uint16 bit patterns,
-    float8_e4m3fn as uint8 codes (marshalling only, no arithmetic)."""
+    float8_e4m3fn as uint8 codes, int8 as int8 (marshalling only, no arithmetic)."""
     if t is None:
         return None
     t = t.detach().contiguous().cpu()
@@ -234,6 +255,6 @@ def to_storage_numpy(t: torch.Tensor | None) -> np.ndarray | None:
         return t.view(torch.int16).numpy().view(np.uint16)
     if t.dtype == torch.float8_e4m3fn:
         return t.view(torch.uint8).numpy()
-    if t.dtype in (torch.int32, torch.int64):
+    if t.dtype in (torch.int8, torch.int32, torch.int64):
         return t.numpy()
     raise TypeError(f"no storage mapping for {t.dtype}")

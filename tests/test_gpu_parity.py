@@ -10,7 +10,7 @@ from parity_util import (check_outputs, check_routing, check_routing_topk, make_
                          oracle_routing, run_gpu, sample_tokens)
 from sparse_moe_transformer_router_b200.workloads import (CONFIGS, DECODE_TOKENS,
                                                           E4M3_FINITE_CODES, E4M3_SUBNORMAL_CODES,
-                                                          LayerConfig, generate, with_e4m3_codes)
+                                                          LayerConfig, generate, with_weight_codes)
 
 pytestmark = pytest.mark.gpu
 
@@ -67,7 +67,7 @@ def test_e4m3_widening_is_exact_for_every_code(codes, scale):
     bf16 tolerance, not just the E4M3 one (a flushed or mis-mapped code
     class would break it)."""
     cfg = LayerConfig("fp8_codes", 300, 256, 4, 256, 192, "fp8", wr_std=0.1)
-    inp = with_e4m3_codes(generate(cfg, seed=7, device="cuda"), codes, scale, seed=7)
+    inp = with_weight_codes(generate(cfg, seed=7, device="cuda"), codes, scale, seed=7)
     layer = make_layer(inp)
     out, r = run_gpu(layer, inp)
     rep = check_routing(inp, r)

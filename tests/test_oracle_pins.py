@@ -315,3 +315,57 @@ def test_topk_of_one_is_the_top1_layer():
     a = oracle.forward(L["x"], L["Wr"], L["Wgu"], L["Wd"], L["Wsgu"], L["Wsd"])
     b = oracle.forward(L["x"], L["Wr"], L["Wgu"], L["Wd"], L["Wsgu"], L["Wsd"], k=1)
     assert np.array_equal(a[0], b[0]) and np.array_equal(a[1], b[1])
+
+
+def test_int8_weights_dequantise_per_output_column():
+    """int8 weights with per-output-column scales equal the dense layer on
+    the dequantised weights (torch's int8 values times the column scale)."""
+    from sparse_moe_transformer_router_b200.workloads import quantize_int8_columns
+    rng = np.random.default_rng(17)
+    T, d, F, Fs = 6, 64, 32, 48
+    x, x64 = _store(rng.standard_normal((T, d)), "bf16")
+    Wr, _ = _store(rng.standard_normal((d, 1)), "bf16")
+
+    def q(shape):
+        w = torch.from_numpy(rng.standard_normal(shape) * 0.02).float()
+        w[:, 0] *= 50.0  # very different column ranges
+        qq, s = quantize_int8_columns(w)
+        deq = qq.to(torch.float64) * s.to(torch.float64)[None, :]
+        return qq.numpy(), s.numpy(), deq.numpy()
+
+    gu, sgu, gu64 = q((d, 2 * F))
+    dn, sdn, dn64 = q((F, d))
+    sgu_s, ssgu, sgu64 = q((d, 2 * Fs))
+    sdn_s, ssdn, sdn64 = q((Fs, d))
+    out, idx, gate = oracle.forward(x, Wr, [gu], [dn], sgu_s, sdn_s, bias=np.array([100.0], np.float32),
+                                    s_gate_up=[sgu], s_down=[sdn], ss_gate_up=ssgu, ss_down=ssdn)
+    assert np.all(gate == 1.0)
+    ref = _dense_swiglu(x64, gu64, dn64) + _dense_swiglu(x64, sgu64, sdn64)
+    scale = np.sqrt(np.mean(ref ** 2))
+    assert np.max(np.abs(out - ref)) <= 1e-12 * scale
+
+
+def test_int8_codes_with_unit_scales_equal_the_bf16_layer():
+    """Every int8 code (-128 included) with unit column scales is the same
+    layer as bf16 weights holding those integers (exact in bf16): a code read
+    as unsigned, or with a sign slip, breaks the equality."""
+    rng = np.random.default_rng(18)
+    T, d, E, F, Fs = 9, 64, 3, 32, 48
+    x, _ = _store(rng.standard_normal((T, d)), "bf16")
+    Wr, _ = _store(rng.standard_normal((d, E)), "bf16")
+
+    def codes(shape):
+        q = rng.integers(-128, 128, size=shape).astype(np.int8)
+        q.flat[:256] = np.arange(-128, 128, dtype=np.int8)
+        return q, _bf16_bits(q.astype(np.float32) / 64.0)
+
+    gu = [codes((d, 2 * F)) for _ in range(E)]
+    dn = [codes((F, d)) for _ in range(E)]
+    sgu, sdn = codes((d, 2 * Fs)), codes((Fs, d))
+    ones = lambda n: np.ones(n, np.float32) / 64.0
+    o8, i8, g8 = oracle.forward(x, Wr, [a for a, _ in gu], [a for a, _ in dn], sgu[0], sdn[0],
+                                s_gate_up=[ones(2 * F)] * E, s_down=[ones(d)] * E,
+                                ss_gate_up=ones(2 * Fs), ss_down=ones(d))
+    ob, ib, gb = oracle.forward(x, Wr, [b for _, b in gu], [b for _, b in dn], sgu[1], sdn[1])
+    assert np.array_equal(i8, ib) and np.array_equal(g8, gb)
+    assert np.array_equal(o8, ob)
