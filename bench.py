@@ -171,13 +171,13 @@ class HostLayer:
             if e not in self._gu:
                 self._gu[e] = to_storage_numpy(inp.W_gate_up[e])
                 self._dn[e] = to_storage_numpy(inp.W_down[e])
-                if inp.cfg.dtype == "fp8":
+                if inp.cfg.dtype in ("fp8", "int8"):
                     self._sgu[e] = inp.s_gate_up[e].cpu().numpy()
                     self._sdn[e] = inp.s_down[e].cpu().numpy()
         Wgu = [self._gu.get(e) if e in need else None for e in range(E)]
         Wdn = [self._dn.get(e) if e in need else None for e in range(E)]
         kw = {}
-        if inp.cfg.dtype == "fp8":
+        if inp.cfg.dtype in ("fp8", "int8"):
             kw = dict(s_gate_up=[self._sgu.get(e) if e in need else None for e in range(E)],
                       s_down=[self._sdn.get(e) if e in need else None for e in range(E)],
                       ss_gate_up=inp.ss_gate_up.cpu().numpy(), ss_down=inp.ss_down.cpu().numpy())
@@ -318,8 +318,8 @@ def run_b200(args, rank, world, local):
     layer = L4MoE(cfg.d_model, cfg.expert_ffn, cfg.shared_ffn, cfg.num_experts, cfg.dtype)
     if inp.bias is not None:
         layer.set_router_bias(inp.bias)
-    if cfg.dtype == "fp8":
-        layer.set_fp8_scales(inp.s_gate_up, inp.s_down, inp.ss_gate_up, inp.ss_down)
+    if cfg.dtype in ("fp8", "int8"):
+        layer.set_weight_scales(inp.s_gate_up, inp.s_down, inp.ss_gate_up, inp.ss_down)
     out = torch.empty((cfg.T, cfg.d_model), dtype=inp.x.dtype, device="cuda")
     fwd = lambda: layer.forward(inp.x, inp.W_router, inp.W_gate_up, inp.W_down,  # noqa: E731
                                 inp.Ws_gate_up, inp.Ws_down, out=out)
@@ -458,8 +458,9 @@ def run_b200(args, rank, world, local):
                             f"the dominant kernel ({dom}) is timed inside the timed region",
             "e2e": e2e, "gpu_launches": launches, "clocks": clocks,
             "experts_touched": accounting.experts_touched(counts)}
-    if cfg.dtype == "fp8":
-        line["dtype"] = "bf16 (E4M3 weights widened exactly to bf16)"
+    if cfg.dtype in ("fp8", "int8"):
+        wname = "E4M3" if cfg.dtype == "fp8" else "int8"
+        line["dtype"] = f"f16 ({wname} weights widened exactly to f16, fp32 accumulate; bf16 in and out)"
     if world == 1 and not args.no_cpu_baseline:
         line["cpu_baseline"] = cpu_baseline(inp)
     print(json.dumps(line), flush=True)

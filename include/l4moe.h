@@ -34,11 +34,15 @@
  *   L4MOE_F32       every tensor fp32 (tensor-core math in TF32, fp32 accumulate)
  *   L4MOE_BF16      every tensor bf16 (bf16 MMA, fp32 accumulate)
  *   L4MOE_FP8_E4M3  expert and shared weights OCP E4M3 with one fp32 scale per
- *                   output column (l4moe_set_fp8_scales); x, W_router, out bf16.
+ *                   output column (l4moe_set_weight_scales); x, W_router, out bf16.
  *                   The expert contractions run in f16 (kind::f16 MMA, fp32
  *                   accumulate): weights widened exactly, x and the hidden
  *                   rows held in f16 (exact for bf16 values of magnitude in
  *                   [2^-14, 65504]), the column scale applied in fp32.
+ *   L4MOE_INT8      expert and shared weights int8 (two's complement, symmetric:
+ *                   no zero point) with one fp32 scale per output column, the
+ *                   weight-only int8 of KerasFormers "Llama 4", "Lower memory";
+ *                   otherwise as L4MOE_FP8_E4M3 (every int8 value is exact in f16).
  *
  * Ownership: the caller owns every tensor, the scale vectors, the bias and
  * the stream.  The handle owns only its workspace (unless the caller supplies
@@ -75,7 +79,7 @@ extern "C" {
 typedef enum {
     L4MOE_OK = 0,
     L4MOE_ERR_ARG = 1,          /* null / out-of-range argument                */
-    L4MOE_ERR_DTYPE = 2,        /* unknown dtype or missing FP8 scales         */
+    L4MOE_ERR_DTYPE = 2,        /* unknown dtype or missing 8-bit weight scales */
     L4MOE_ERR_ALIGN = 3,        /* pointer not 16-byte aligned / bad multiple  */
     L4MOE_ERR_CUDA = 4,         /* a CUDA runtime or driver call failed        */
     L4MOE_ERR_WORKSPACE = 5,    /* workspace too small / allocation failed     */
@@ -86,7 +90,8 @@ typedef enum {
 typedef enum {
     L4MOE_F32 = 0,
     L4MOE_BF16 = 1,
-    L4MOE_FP8_E4M3 = 2
+    L4MOE_FP8_E4M3 = 2,
+    L4MOE_INT8 = 3
 } l4moe_dtype;
 
 typedef struct {
@@ -128,7 +133,7 @@ L4MOE_API l4moe_status l4moe_set_router_bias(l4moe_handle *h, const float *bias_
  * equal values, NaN never selected), each on the input gated by the sigmoid
  * of its own logit, and their outputs add to the shared expert's (the
  * "experts per token" of a token-choice router, torchtune MoE
- * documentation).  1 <= k <= min(4, E); k > 1 needs bf16 or E4M3 weights and
+ * documentation).  1 <= k <= min(4, E); k > 1 needs bf16, E4M3 or int8 weights and
  * E % 8 == 0 (else L4MOE_ERR_UNSUPPORTED).  The routing arrays of
  * l4moe_get_routing then hold T * k entries (entry t * k + j: token t's j-th
  * expert; margin stays [T]: the k-th logit minus the next one).  Changing k
@@ -136,10 +141,17 @@ L4MOE_API l4moe_status l4moe_set_router_bias(l4moe_handle *h, const float *bias_
  * fails with L4MOE_ERR_WORKSPACE when a caller's workspace is too small. */
 L4MOE_API l4moe_status l4moe_set_top_k(l4moe_handle *h, int k);
 
-/* FP8 weights only: per-output-column fp32 scales (device pointers).
- * s_gate_up / s_down are HOST arrays of E device pointers to [2F] / [d]
- * vectors; ss_gate_up [2Fs] and ss_down [d] are the shared expert's.  The
- * dequantised weight is e4m3(q) * scale[column]. */
+/* E4M3 or int8 weights only: per-output-column fp32 scales (device
+ * pointers).  s_gate_up / s_down are HOST arrays of E device pointers to
+ * [2F] / [d] vectors; ss_gate_up [2Fs] and ss_down [d] are the shared
+ * expert's.  The dequantised weight is e4m3(q) * scale[column] or
+ * q * scale[column].  The pointers are kept, not copied: the vectors must
+ * stay valid while the handle runs forwards.  L4MOE_ERR_DTYPE for other
+ * dtypes, L4MOE_ERR_ARG for a NULL pointer. */
+L4MOE_API l4moe_status l4moe_set_weight_scales(l4moe_handle *h, const float *const *s_gate_up,
+                                     const float *const *s_down, const float *ss_gate_up,
+                                     const float *ss_down);
+/* The same call under its E4M3-era name. */
 L4MOE_API l4moe_status l4moe_set_fp8_scales(l4moe_handle *h, const float *const *s_gate_up,
                                   const float *const *s_down, const float *ss_gate_up,
                                   const float *ss_down);
@@ -187,7 +199,7 @@ L4MOE_API l4moe_status l4moe_forward_host(l4moe_handle *h, int T, const void *x_
  * layer do not fit in the scratch area: it holds the device part of the
  * workspace (l4moe_workspace_size without the host-path staging slots,
  * rounded up to 256 bytes) plus 2(E+1) TMA descriptors of 128 bytes (and,
- * for E4M3 weights, the 2(E+1) scale-vector pointers), e.g.
+ * for 8-bit weights, the 2(E+1) scale-vector pointers), e.g.
  * about 390 tokens at d_model 5120 and F = Fs = 8192 in bf16 (E4M3 layers
  * also keep x in f16 there: about 350 tokens).  Every call, from any
  * handle, shares the one array: calls

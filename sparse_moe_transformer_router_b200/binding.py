@@ -15,13 +15,14 @@ _PKG = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(_PKG, "libl4moe.so")
 
 OK, ERR_ARG, ERR_DTYPE, ERR_ALIGN, ERR_CUDA, ERR_WORKSPACE, ERR_TIMEOUT, ERR_UNSUPPORTED = range(8)
-DTYPES = {"f32": 0, "bf16": 1, "fp8": 2}
+DTYPES = {"f32": 0, "bf16": 1, "fp8": 2, "int8": 3}
 EXPORTED = ("l4moe_create", "l4moe_destroy", "l4moe_workspace_size", "l4moe_set_workspace",
             "l4moe_set_router_bias", "l4moe_set_fp8_scales", "l4moe_forward",
             "l4moe_forward_host", "l4moe_get_routing", "l4moe_check_device_status",
             "l4moe_launch_count", "l4moe_last_error", "l4moe_status_string", "l4moe_version",
             "l4moe_set_timing", "l4moe_read_timing", "l4moe_kernel_name",
-            "l4moe_forward_static", "l4moe_join_host", "l4moe_set_top_k")
+            "l4moe_forward_static", "l4moe_join_host", "l4moe_set_top_k",
+            "l4moe_set_weight_scales")
 STATIC_WORKSPACE_BYTES = 32 << 20
 NUM_KERNELS = 5
 
@@ -59,6 +60,7 @@ def load_library():
     lib.l4moe_set_workspace.argtypes = [vp, vp, sz, i32]
     lib.l4moe_set_router_bias.argtypes = [vp, vp]
     lib.l4moe_set_fp8_scales.argtypes = [vp, pvp, pvp, vp, vp]
+    lib.l4moe_set_weight_scales.argtypes = [vp, pvp, pvp, vp, vp]
     fwd = [vp, i32, vp, vp, pvp, pvp, vp, vp, vp, vp]
     lib.l4moe_forward.argtypes = fwd
     lib.l4moe_forward_host.argtypes = fwd
@@ -83,7 +85,7 @@ def load_library():
                  "l4moe_set_fp8_scales", "l4moe_forward", "l4moe_forward_host",
                  "l4moe_get_routing", "l4moe_check_device_status", "l4moe_version",
                  "l4moe_set_timing", "l4moe_read_timing", "l4moe_forward_static",
-                 "l4moe_join_host"):
+                 "l4moe_join_host", "l4moe_set_top_k", "l4moe_set_weight_scales"):
         getattr(lib, name).restype = ctypes.c_int
     _lib = lib
     return lib
@@ -166,10 +168,13 @@ class L4MoE:
         self._check(self._lib.l4moe_set_router_bias(self._h, _ptr(bias)))
         self._bias = bias
 
-    def set_fp8_scales(self, s_gate_up, s_down, ss_gate_up, ss_down):
+    def set_weight_scales(self, s_gate_up, s_down, ss_gate_up, ss_down):
+        """Per-output-column fp32 scales of E4M3 or int8 weights (device tensors)."""
         a, b = _ptr_array(s_gate_up), _ptr_array(s_down)
-        self._check(self._lib.l4moe_set_fp8_scales(self._h, a, b, _ptr(ss_gate_up), _ptr(ss_down)))
+        self._check(self._lib.l4moe_set_weight_scales(self._h, a, b, _ptr(ss_gate_up), _ptr(ss_down)))
         self._scales = (list(s_gate_up), list(s_down), ss_gate_up, ss_down)
+
+    set_fp8_scales = set_weight_scales
 
     def _weights(self, W_gate_up, W_down):
         key = (tuple(_ptr(w) for w in W_gate_up), tuple(_ptr(w) for w in W_down))

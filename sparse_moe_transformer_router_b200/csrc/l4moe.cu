@@ -80,6 +80,8 @@ struct WsLayout {
 
 size_t act_bytes(l4moe_dtype dt) { return dt == L4MOE_F32 ? 4 : 2; }
 size_t w_bytes(l4moe_dtype dt) { return dt == L4MOE_F32 ? 4 : (dt == L4MOE_BF16 ? 2 : 1); }
+// 8-bit weight codes (E4M3 or int8) with per-output-column scales
+bool coded8(l4moe_dtype dt) { return dt == L4MOE_FP8_E4M3 || dt == L4MOE_INT8; }
 
 // Split-K plan of one forward of T tokens: how many k-ranges the gate/up and
 // the down launches use.  Only batches of at most kSplitMaxTokens split, into
@@ -166,8 +168,8 @@ WsLayout ws_layout(const l4moe_params& p, int T, int sms, int k) {
     L.xg = take(tv * p.d_model * es);
     L.hr = take(tv * p.expert_ffn * es);
     L.hs = take(t * p.shared_ffn * es);
-    // E4M3 layers: x in f16, token order (the shared expert's operand)
-    L.x16 = take(p.dtype == L4MOE_FP8_E4M3 ? t * p.d_model * 2 : 0);
+    // 8-bit weight layers: x in f16, token order (the shared expert's operand)
+    L.x16 = take(coded8(p.dtype) ? t * p.d_model * 2 : 0);
     L.part = take(sizeof(float) * part_floats(p, (int)t, sms, k));
     L.logits = take(sizeof(float) * std::min<size_t>(t, 128) * E);  // expert-split router
     L.device_total = off;
@@ -332,9 +334,9 @@ l4moe_status encode_weight_maps(l4moe_handle* h, const void* const* Wgu, const v
     CUtensorMapDataType dt = h->p.dtype == L4MOE_F32 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT32
                              : h->p.dtype == L4MOE_BF16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16
                                                         : CU_TENSOR_MAP_DATA_TYPE_UINT8;
-    const bool fp8 = h->p.dtype == L4MOE_FP8_E4M3;
+    const bool fp8 = coded8(h->p.dtype);
     const uint32_t bk = h->p.dtype == L4MOE_F32 ? 32 : 64;  // K rows per box
-    // features per box: one 128-byte swizzled slab; E4M3 weights are staged
+    // features per box: one 128-byte swizzled slab; 8-bit weights are staged
     // raw (64-feature boxes, unswizzled) and widened in shared memory
     const uint32_t bw = fp8 ? 64u : (uint32_t)(128 / wb);
     // MN-major 32-bit operands need the 32-byte swizzle unit
@@ -417,21 +419,24 @@ void launch_router(const void* x, const void* Wr, const float* bias, int T, int 
     else launch_router_t<ET, 256, 8, 8>(x, Wr, bias, T, d, E, idx, gate, lmax, margin, st);
 }
 
-template <int MODE, typename ET, bool FP8W>
+template <int MODE, typename ET, int WQ>
 void launch_gemm(int grid, const BMaps& bm, const GemmArgs& a, cudaStream_t st) {
-    using Cfg = GemmCfg<MODE, ET, FP8W>;
+    using Cfg = GemmCfg<MODE, ET, WQ != kWqNone>;
     static std::once_flag once;
-    std::call_once(once, [] { set_smem_attr(moe_gemm_kernel<MODE, ET, FP8W>, Cfg::SMEM_BYTES); });
-    launch_k(moe_gemm_kernel<MODE, ET, FP8W>, dim3(grid), dim3(Cfg::THREADS), Cfg::SMEM_BYTES, st, bm, a);
+    std::call_once(once, [] { set_smem_attr(moe_gemm_kernel<MODE, ET, WQ>, Cfg::SMEM_BYTES); });
+    launch_k(moe_gemm_kernel<MODE, ET, WQ>, dim3(grid), dim3(Cfg::THREADS), Cfg::SMEM_BYTES, st, bm, a);
 }
 
 // The launch sequence of one forward.  w / ws_tokens: the workspace and the
 // token count its layout was made for; maps: device array of the 2(E+1)
 // weight descriptors.
-template <typename ET, bool FP8W = false>
+// WQ: the weights' storage (kWqNone: the layer's type; kWqE4M3 / kWqInt8:
+// 8-bit codes with per-column scales, widened to f16 in the GEMMs).
+template <typename ET, int WQ = kWqNone>
 l4moe_status run_layer(l4moe_handle* h, int T, const void* x, const void* Wr, const void* Wsgu,
                        const void* Wsdn, void* out, cudaStream_t st, uint8_t* w, int ws_tokens,
                        const CUtensorMap* maps, const float* const* scales = nullptr) {
+    constexpr bool FP8W = WQ != kWqNone;  // 8-bit weight codes (E4M3 or int8)
     const l4moe_params& p = h->p;
     const int d = p.d_model, F = p.expert_ffn, Fs = p.shared_ffn, E = p.num_experts;
     const WsLayout L = ws_layout(p, ws_tokens, h->sms, h->top_k);
@@ -447,7 +452,7 @@ l4moe_status run_layer(l4moe_handle* h, int T, const void* x, const void* Wr, co
     int32_t* offsets = reinterpret_cast<int32_t*>(w + L.offsets);
     GroupTable* tab_gu = reinterpret_cast<GroupTable*>(w + L.tab_gu);
     GroupTable* tab_dn = reinterpret_cast<GroupTable*>(w + L.tab_dn);
-    // the GEMMs' activation type: the layer's, or f16 for E4M3 weights
+    // the GEMMs' activation type: the layer's, or f16 for 8-bit weights
     // (widened exactly to f16; kind::f16 wants both operands of one type)
     using GT = typename GemmAct<ET, FP8W>::type;
     GT* xg = reinterpret_cast<GT*>(w + L.xg);
@@ -562,7 +567,7 @@ l4moe_status run_layer(l4moe_handle* h, int T, const void* x, const void* Wr, co
         launch_k(dense_table_kernel, dim3(1), dim3(32), 0, st, tab_gu, tab_dn, T, fb_gu_s * s_gu, fb_dn * s_dn);
         t_perm.stop();
         L4MOE_CHECK_LAUNCH("work list launch");
-        if (FP8W) {  // the f16 copy of x the contractions of E4M3 layers read
+        if (FP8W) {  // the f16 copy of x the contractions of 8-bit weight layers read
             const int sc_blocks = std::min((T + 7) / 8, h->sms * 8);
             LaunchTimer t_rows(h, 2, st);
             launch_k(permute_rows_kernel<ET, GT>, dim3(sc_blocks), dim3(256), 0, st, static_cast<const ET*>(x),
@@ -608,7 +613,7 @@ l4moe_status run_layer(l4moe_handle* h, int T, const void* x, const void* Wr, co
     gu.part_stride_shared = (long long)T * 2 * Fs;
     gu.err = err;
     LaunchTimer t_gu(h, 3, st);
-    launch_gemm<MODE_GATEUP, ET, FP8W>(
+    launch_gemm<MODE_GATEUP, ET, WQ>(
         grid_for(s_gu * ((long long)fb_gu_s * tb + (long long)fb_gu_r * (tbv + std::min(E, Tv)))),
         bm_gu, gu, st);
     if (s_gu > 1) {
@@ -649,7 +654,7 @@ l4moe_status run_layer(l4moe_handle* h, int T, const void* x, const void* Wr, co
     dn.part_stride_shared = (long long)T * d;
     dn.err = err;
     LaunchTimer t_dn(h, 4, st);
-    launch_gemm<MODE_DOWN, ET, FP8W>(grid_for(s_dn * (long long)fb_dn * (tb + tbv + std::min(E, Tv))),
+    launch_gemm<MODE_DOWN, ET, WQ>(grid_for(s_dn * (long long)fb_dn * (tb + tbv + std::min(E, Tv))),
                                      bm_dn, dn, st);
     {
         const long long n = (long long)T * d;
@@ -666,9 +671,9 @@ l4moe_status run_layer(l4moe_handle* h, int T, const void* x, const void* Wr, co
     return L4MOE_OK;
 }
 
-// Device table of the per-column scale vectors of the E4M3 weights:
+// Device table of the per-column scale vectors of the 8-bit weights:
 // [gate/up of experts 0..E-1, shared gate/up, down of experts 0..E-1, shared down].
-// The E4M3 column-scale pointers in the kernels' order: gate/up of experts
+// The column-scale pointers of 8-bit weights in the kernels' order: gate/up of experts
 // 0..E-1, the shared gate/up, then the same for down.
 std::vector<const float*> scale_table(const l4moe_handle* h) {
     const int E = h->p.num_experts;
@@ -715,8 +720,8 @@ l4moe_status check_forward_args(l4moe_handle* h, int T, const void* x, const voi
         if (!aligned16(Wgu[e]) || !aligned16(Wdn[e]))
             return fail(h, L4MOE_ERR_ALIGN, "expert weight pointer not 16-byte aligned");
     }
-    if (h->p.dtype == L4MOE_FP8_E4M3 && !h->ss_gu)
-        return fail(h, L4MOE_ERR_DTYPE, "FP8 weights need l4moe_set_fp8_scales first");
+    if (coded8(h->p.dtype) && !h->ss_gu)
+        return fail(h, L4MOE_ERR_DTYPE, "8-bit weights need l4moe_set_weight_scales first");
     return L4MOE_OK;
 }
 
@@ -726,7 +731,7 @@ l4moe_status forward_impl(l4moe_handle* h, int T, const void* x, const void* Wr,
     l4moe_status s;
     if ((s = ensure_workspace(h, T)) != L4MOE_OK) return s;
     if ((s = ensure_weight_maps(h, Wgu, Wdn, Wsgu, Wsdn, st)) != L4MOE_OK) return s;
-    if (h->p.dtype == L4MOE_FP8_E4M3 && (s = ensure_scales(h, st)) != L4MOE_OK) return s;
+    if (coded8(h->p.dtype) && (s = ensure_scales(h, st)) != L4MOE_OK) return s;
     switch (h->p.dtype) {
     case L4MOE_F32:
         return run_layer<float>(h, T, x, Wr, Wsgu, Wsdn, out, st, h->ws, h->ws_tokens, h->d_maps);
@@ -734,8 +739,11 @@ l4moe_status forward_impl(l4moe_handle* h, int T, const void* x, const void* Wr,
         return run_layer<__nv_bfloat16>(h, T, x, Wr, Wsgu, Wsdn, out, st, h->ws, h->ws_tokens,
                                         h->d_maps);
     case L4MOE_FP8_E4M3:
-        return run_layer<__nv_bfloat16, true>(h, T, x, Wr, Wsgu, Wsdn, out, st, h->ws, h->ws_tokens,
-                                              h->d_maps, h->d_scales);
+        return run_layer<__nv_bfloat16, kWqE4M3>(h, T, x, Wr, Wsgu, Wsdn, out, st, h->ws, h->ws_tokens,
+                                                 h->d_maps, h->d_scales);
+    case L4MOE_INT8:
+        return run_layer<__nv_bfloat16, kWqInt8>(h, T, x, Wr, Wsgu, Wsdn, out, st, h->ws, h->ws_tokens,
+                                                 h->d_maps, h->d_scales);
     }
     return fail(h, L4MOE_ERR_DTYPE, "unknown dtype");
 }
@@ -778,7 +786,7 @@ l4moe_status l4moe_forward_static(l4moe_handle* h, int T, const void* x, const v
     l4moe_status s = check_forward_args(h, T, x, W_router, W_gate_up, W_down, Ws_gate_up, Ws_down, out);
     if (s != L4MOE_OK || T == 0) return s;
     const int E = h->p.num_experts;
-    const bool fp8 = h->p.dtype == L4MOE_FP8_E4M3;
+    const bool fp8 = coded8(h->p.dtype);
     const size_t ws_bytes = (ws_layout(h->p, T, h->sms, h->top_k).device_total + 255) & ~size_t(255);
     const size_t maps_bytes = sizeof(CUtensorMap) * 2 * (E + 1);
     const size_t scales_bytes = fp8 ? sizeof(float*) * 2 * (E + 1) : 0;
@@ -801,7 +809,7 @@ l4moe_status l4moe_forward_static(l4moe_handle* h, int T, const void* x, const v
     e = cudaMemsetAsync(base + ws_layout(h->p, T, h->sms, h->top_k).err, 0, sizeof(unsigned), st);
     if (e != cudaSuccess) return cuda_fail(h, e, "static error word clear");
     const float* const* scales = nullptr;
-    if (fp8) {  // the E4M3 scale-pointer table follows the descriptors
+    if (fp8) {  // the scale-pointer table of 8-bit weights follows the descriptors
         const std::vector<const float*> tab = scale_table(h);
         scales = reinterpret_cast<const float* const*>(base + ws_bytes + maps_bytes);
         e = cudaMemcpyAsync(const_cast<const float**>(scales), tab.data(), scales_bytes,
@@ -812,9 +820,12 @@ l4moe_status l4moe_forward_static(l4moe_handle* h, int T, const void* x, const v
     h->timing = 0;
     if (h->p.dtype == L4MOE_F32)
         s = run_layer<float>(h, T, x, W_router, Ws_gate_up, Ws_down, out, st, base, T, maps);
-    else if (fp8)
-        s = run_layer<__nv_bfloat16, true>(h, T, x, W_router, Ws_gate_up, Ws_down, out, st, base, T, maps,
-                                           scales);
+    else if (h->p.dtype == L4MOE_FP8_E4M3)
+        s = run_layer<__nv_bfloat16, kWqE4M3>(h, T, x, W_router, Ws_gate_up, Ws_down, out, st, base, T, maps,
+                                              scales);
+    else if (h->p.dtype == L4MOE_INT8)
+        s = run_layer<__nv_bfloat16, kWqInt8>(h, T, x, W_router, Ws_gate_up, Ws_down, out, st, base, T, maps,
+                                              scales);
     else
         s = run_layer<__nv_bfloat16>(h, T, x, W_router, Ws_gate_up, Ws_down, out, st, base, T, maps);
     h->timing = timing;
@@ -841,7 +852,7 @@ l4moe_status l4moe_create(const l4moe_params* params, l4moe_handle** out) {
     if (!params || !out) return fail(nullptr, L4MOE_ERR_ARG, "null params or out");
     *out = nullptr;
     const l4moe_params& p = *params;
-    if (p.dtype != L4MOE_F32 && p.dtype != L4MOE_BF16 && p.dtype != L4MOE_FP8_E4M3)
+    if (p.dtype != L4MOE_F32 && p.dtype != L4MOE_BF16 && p.dtype != L4MOE_FP8_E4M3 && p.dtype != L4MOE_INT8)
         return fail(nullptr, L4MOE_ERR_DTYPE, "unknown dtype");
     if (p.d_model <= 0 || p.shared_ffn <= 0 || p.num_experts < 0 || p.num_experts > 256 ||
         p.expert_ffn < 0 || (p.num_experts > 0 && p.expert_ffn == 0))
@@ -899,7 +910,7 @@ l4moe_status l4moe_set_top_k(l4moe_handle* h, int k) {
         return fail(h, L4MOE_ERR_ARG, "top_k must be in [1, min(4, E)]");
     if (k > 1 && (h->p.dtype == L4MOE_F32 || E % 8 != 0))
         return fail(h, L4MOE_ERR_UNSUPPORTED,
-                    "top_k > 1 takes the tensor-core router: bf16 or E4M3 weights and E % 8 == 0");
+                    "top_k > 1 takes the tensor-core router: bf16, E4M3 or int8 weights and E % 8 == 0");
     if (k == h->top_k) return L4MOE_OK;
     if (h->ws && !h->ws_owned && h->ws_bytes < ws_layout(h->p, h->ws_tokens, h->sms, k).total)
         return fail(h, L4MOE_ERR_WORKSPACE, "the caller's workspace is too small for this top_k");
@@ -938,11 +949,11 @@ l4moe_status l4moe_set_router_bias(l4moe_handle* h, const float* bias_dev) {
     return L4MOE_OK;
 }
 
-l4moe_status l4moe_set_fp8_scales(l4moe_handle* h, const float* const* s_gate_up,
-                                  const float* const* s_down, const float* ss_gate_up,
-                                  const float* ss_down) {
+l4moe_status l4moe_set_weight_scales(l4moe_handle* h, const float* const* s_gate_up,
+                                     const float* const* s_down, const float* ss_gate_up,
+                                     const float* ss_down) {
     if (!h) return L4MOE_ERR_ARG;
-    if (h->p.dtype != L4MOE_FP8_E4M3) return fail(h, L4MOE_ERR_DTYPE, "scales apply to FP8 weights only");
+    if (!coded8(h->p.dtype)) return fail(h, L4MOE_ERR_DTYPE, "scales apply to E4M3 or int8 weights only");
     const int E = h->p.num_experts;
     if (!ss_gate_up || !ss_down || (E > 0 && (!s_gate_up || !s_down)))
         return fail(h, L4MOE_ERR_ARG, "null scale pointer");
@@ -954,6 +965,12 @@ l4moe_status l4moe_set_fp8_scales(l4moe_handle* h, const float* const* s_gate_up
     h->ss_dn = ss_down;
     h->scales_dirty = true;
     return L4MOE_OK;
+}
+
+l4moe_status l4moe_set_fp8_scales(l4moe_handle* h, const float* const* s_gate_up,
+                                  const float* const* s_down, const float* ss_gate_up,
+                                  const float* ss_down) {
+    return l4moe_set_weight_scales(h, s_gate_up, s_down, ss_gate_up, ss_down);
 }
 
 l4moe_status l4moe_forward(l4moe_handle* h, int T, const void* x, const void* W_router,

@@ -224,6 +224,30 @@ __device__ __forceinline__ uint4 e4m3x8_to_f16(uint2 raw) {
                       e4m3x2_to_f16x2(raw.y & 0xFFFFu), e4m3x2_to_f16x2(raw.y >> 16));
 }
 
+// 8 int8 codes (little-endian in a uint2) -> 8 f16 values, exactly.  With
+// the code biased to u = q + 128 in [0, 255] (flipping bit 7), the f16 whose
+// high byte is 0x64 and low byte is u has exponent 10 and value 1024 + u (u
+// fills the low mantissa bits); subtracting 1152 = 1024 + 128 leaves q, and
+// both values and the difference are integers below 2^11, so every step is
+// exact.  Two bytes per byte permutation and per f16x2 subtraction.
+__device__ __forceinline__ uint32_t i8x2_to_f16x2(uint32_t biased4, uint32_t sel) {
+    uint32_t h, r;
+    asm("prmt.b32 %0, %1, %2, %3;" : "=r"(h) : "r"(biased4), "r"(0x64646464u), "r"(sel));
+    asm("sub.rn.f16x2 %0, %1, %2;" : "=r"(r) : "r"(h), "r"(0x64806480u));
+    return r;
+}
+
+__device__ __forceinline__ uint4 int8x8_to_f16(uint2 raw) {
+    const uint32_t lo = raw.x ^ 0x80808080u, hi = raw.y ^ 0x80808080u;
+    // byte selectors: (code byte, 0x64, code byte, 0x64) from the low / high pair
+    return make_uint4(i8x2_to_f16x2(lo, 0x4140u), i8x2_to_f16x2(lo, 0x4342u),
+                      i8x2_to_f16x2(hi, 0x4140u), i8x2_to_f16x2(hi, 0x4342u));
+}
+
+// Weight storage of a GEMM: the layer's own type, or 8-bit codes widened in
+// shared memory (E4M3 floats or int8 integers, per-column scales).
+enum : int { kWqNone = 0, kWqE4M3 = 1, kWqInt8 = 2 };
+
 // The contractions' activation (token operand and hidden) type: the layer's
 // own, or f16 for E4M3 weights (kind::f16 takes both operands in one type).
 template <typename ET, bool FP8W>
@@ -252,10 +276,11 @@ struct BMaps {
     CUtensorMap routed, shared, routed_small, shared_small;
 };
 
-template <int MODE, typename ET, bool FP8W>
-__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(GemmCfg<MODE, ET, FP8W>::THREADS, 1)
+template <int MODE, typename ET, int WQ>
+__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(GemmCfg<MODE, ET, WQ != kWqNone>::THREADS, 1)
     moe_gemm_kernel(const __grid_constant__ BMaps bm, const GemmArgs args) {
     pdl_enter();
+    constexpr bool FP8W = WQ != kWqNone;  // 8-bit weight codes with converter warps
     using Cfg = GemmCfg<MODE, ET, FP8W>;
     using C = ElemCfg<ET>;
     extern __shared__ uint8_t smem_raw[];
@@ -470,7 +495,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(GemmCfg<MODE, ET, FP
             mbar_wait(drain_bar, 0, args.err, DEV_ERR_TIMEOUT_MMA);
         }
     } else if (FP8W && warp >= 6) {
-        // ---------------------------------------------------- E4M3 converters
+        // --------------------------------------- weight-code converters (E4M3, int8)
         constexpr int NCT = 32 * (Cfg::CONV_WARPS > 0 ? Cfg::CONV_WARPS : 8);  // converter threads
         static_assert(NCT == 256, "each converter thread owns 4 units: slab i / 2");
         const int ct = threadIdx.x - 192;           // 0 .. NCT-1
@@ -495,8 +520,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(GemmCfg<MODE, ET, FP
                     // slab u / 512, K row (u / 8) % 64, chunk c8
                     const int j = (i * NCT) >> 9, kr = ((ct >> 3) + (NCT / 8) * i) & 63;
                     const uint2 q8 = *reinterpret_cast<const uint2*>(raw + j * 4096 + kr * 64 + c8 * 8);
-                    *reinterpret_cast<uint4*>(a + j * 8192 + kr * 128 + ((c8 ^ (kr & 7)) << 4)) =
-                        e4m3x8_to_f16(q8);
+                    uint4 h8;
+                    if constexpr (WQ == kWqInt8) h8 = int8x8_to_f16(q8);
+                    else h8 = e4m3x8_to_f16(q8);
+                    *reinterpret_cast<uint4*>(a + j * 8192 + kr * 128 + ((c8 ^ (kr & 7)) << 4)) = h8;
                 }
                 fence_proxy_async_smem();  // generic-proxy writes -> tensor-core reads
                 __syncwarp();

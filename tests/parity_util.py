@@ -25,8 +25,8 @@ from sparse_moe_transformer_router_b200.binding import L4MoE
 from sparse_moe_transformer_router_b200.workloads import LayerInputs, to_storage_numpy
 
 MARGIN_EXCLUDE = 1e-4
-TOL = {"f32": 2e-2, "bf16": 2e-2, "fp8": 6e-2}
-OUT_UNIT_ROUNDOFF = {"f32": 2.0 ** -24, "bf16": 2.0 ** -8, "fp8": 2.0 ** -8}
+TOL = {"f32": 2e-2, "bf16": 2e-2, "fp8": 6e-2, "int8": 6e-2}
+OUT_UNIT_ROUNDOFF = {"f32": 2.0 ** -24, "bf16": 2.0 ** -8, "fp8": 2.0 ** -8, "int8": 2.0 ** -8}
 
 
 def make_layer(inp: LayerInputs) -> L4MoE:
@@ -34,8 +34,8 @@ def make_layer(inp: LayerInputs) -> L4MoE:
     layer = L4MoE(c.d_model, c.expert_ffn, c.shared_ffn, c.num_experts, c.dtype)
     if inp.bias is not None:
         layer.set_router_bias(inp.bias)
-    if c.dtype == "fp8":
-        layer.set_fp8_scales(inp.s_gate_up, inp.s_down, inp.ss_gate_up, inp.ss_down)
+    if c.dtype in ("fp8", "int8"):
+        layer.set_weight_scales(inp.s_gate_up, inp.s_down, inp.ss_gate_up, inp.ss_down)
     return layer
 
 
@@ -137,7 +137,7 @@ def check_outputs(inp: LayerInputs, out: torch.Tensor, tokens, same_mask=None, o
     Wgu = [to_storage_numpy(inp.W_gate_up[e]) if e in need else None for e in range(c.num_experts)]
     Wdn = [to_storage_numpy(inp.W_down[e]) if e in need else None for e in range(c.num_experts)]
     kw = {}
-    if c.dtype == "fp8":
+    if c.dtype in ("fp8", "int8"):
         kw = dict(s_gate_up=[inp.s_gate_up[e].cpu().numpy() if e in need else None for e in range(c.num_experts)],
                   s_down=[inp.s_down[e].cpu().numpy() if e in need else None for e in range(c.num_experts)],
                   ss_gate_up=inp.ss_gate_up.cpu().numpy(), ss_down=inp.ss_down.cpu().numpy())

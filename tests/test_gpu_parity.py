@@ -10,7 +10,8 @@ from parity_util import (check_outputs, check_routing, check_routing_topk, make_
                          oracle_routing, run_gpu, sample_tokens)
 from sparse_moe_transformer_router_b200.workloads import (CONFIGS, DECODE_TOKENS,
                                                           E4M3_FINITE_CODES, E4M3_SUBNORMAL_CODES,
-                                                          LayerConfig, generate, with_weight_codes)
+                                                          INT8_CODES, LayerConfig, generate,
+                                                          with_weight_codes)
 
 pytestmark = pytest.mark.gpu
 
@@ -33,11 +34,17 @@ SMALL = {
     "fp8_zipf": LayerConfig("fp8_zipf", 700, 192, 16, 128, 320, "fp8", router="zipf", n_dead=4,
                             wr_std=0.05),
     "fp8_T1": LayerConfig("fp8_T1", 1, 256, 8, 256, 256, "fp8", wr_std=0.1),
+    # int8 weights with per-output-column scales, bf16 activations
+    "int8_ragged": LayerConfig("int8_ragged", 300, 256, 8, 384, 256, "int8", wr_std=0.1),
+    "int8_zipf": LayerConfig("int8_zipf", 700, 192, 16, 128, 320, "int8", router="zipf", n_dead=4,
+                             wr_std=0.05),
+    "int8_T1": LayerConfig("int8_T1", 1, 256, 8, 256, 256, "int8", wr_std=0.1),
     # few tiles: split-K partials + finish kernels; T <= 128 with E % 16 == 0:
     # expert-split router with the arg-max in the permutation kernel
     "bf16_splitk": LayerConfig("bf16_splitk", 2, 1024, 8, 1024, 1024, "bf16", wr_std=0.03),
     "f32_splitk": LayerConfig("f32_splitk", 3, 1024, 8, 1024, 512, "f32", wr_std=0.03),
     "fp8_splitk": LayerConfig("fp8_splitk", 2, 1024, 8, 1024, 1024, "fp8", wr_std=0.03),
+    "int8_splitk": LayerConfig("int8_splitk", 2, 1024, 8, 1024, 1024, "int8", wr_std=0.03),
     "bf16_router_split": LayerConfig("bf16_router_split", 1, 1024, 64, 512, 512, "bf16", wr_std=0.03),
     "bf16_T40_E32": LayerConfig("bf16_T40_E32", 40, 512, 32, 512, 768, "bf16", wr_std=0.05),
     # few token tiles and E < 32: the router splits K into 4 slices per token
@@ -58,15 +65,17 @@ def test_small_layer_matches_oracle(name):
     print(f"{name}: max|err|/rms = {ratio:.3e}, excluded {rep['excluded']}, flipped {rep['flipped']}")
 
 
-@pytest.mark.parametrize("codes,scale", [(E4M3_FINITE_CODES, 4e-4), (E4M3_SUBNORMAL_CODES, 20.0)],
-                         ids=["all_finite_codes", "subnormal_codes"])
-def test_e4m3_widening_is_exact_for_every_code(codes, scale):
+@pytest.mark.parametrize("dtype,codes,scale", [("fp8", E4M3_FINITE_CODES, 4e-4),
+                                               ("fp8", E4M3_SUBNORMAL_CODES, 20.0),
+                                               ("int8", INT8_CODES, 1.5e-3)],
+                         ids=["e4m3_all_finite_codes", "e4m3_subnormal_codes", "int8_all_codes"])
+def test_weight_widening_is_exact_for_every_code(dtype, codes, scale):
     """Weights drawn from every finite E4M3 code (or from the zero and
-    subnormal codes alone) with one column scale: the widening to bf16 is
-    exact and the scale meets the fp32 accumulator, so the layer meets the
-    bf16 tolerance, not just the E4M3 one (a flushed or mis-mapped code
-    class would break it)."""
-    cfg = LayerConfig("fp8_codes", 300, 256, 4, 256, 192, "fp8", wr_std=0.1)
+    subnormal codes alone), or from every int8 code, with one column scale:
+    the widening to f16 is exact and the scale meets the fp32 accumulator, so
+    the layer meets the bf16 tolerance, not just the 8-bit one (a flushed or
+    mis-mapped code class would break it)."""
+    cfg = LayerConfig(f"{dtype}_codes", 300, 256, 4, 256, 192, dtype, wr_std=0.1)
     inp = with_weight_codes(generate(cfg, seed=7, device="cuda"), codes, scale, seed=7)
     layer = make_layer(inp)
     out, r = run_gpu(layer, inp)
@@ -81,6 +90,7 @@ TOPK = {
     "bf16_k4_zipf": (LayerConfig("bf16_k4_zipf", 500, 128, 16, 128, 128, "bf16", router="zipf", n_dead=4,
                                  wr_std=0.05), 4),
     "fp8_k2": (LayerConfig("fp8_k2", 300, 256, 8, 384, 256, "fp8", wr_std=0.1), 2),
+    "int8_k2": (LayerConfig("int8_k2", 300, 256, 8, 384, 256, "int8", wr_std=0.1), 2),
     # K slices reduced in a cluster before the top-k epilogue
     "bf16_k2_kslices": (LayerConfig("bf16_k2_kslices", 700, 1024, 16, 256, 256, "bf16", wr_std=0.03), 2),
     # one token tile with E >= 32: expert-split router, top-k in the permutation
@@ -128,6 +138,7 @@ DENSE = {
     "dense_bf16": LayerConfig("dense_bf16", 300, 256, 0, 0, 384, "bf16"),
     "dense_f32": LayerConfig("dense_f32", 130, 128, 0, 0, 192, "f32"),
     "dense_fp8": LayerConfig("dense_fp8", 300, 256, 0, 0, 320, "fp8"),
+    "dense_int8": LayerConfig("dense_int8", 300, 256, 0, 0, 320, "int8"),
     "dense_T1": LayerConfig("dense_T1", 1, 1024, 0, 0, 1024, "bf16"),
 }
 
@@ -263,3 +274,7 @@ def test_full_size_maverick_decode(T):
 
 def test_full_size_maverick_fp8_zipf():
     _full_size(CONFIGS["maverick_fp8"])
+
+
+def test_full_size_maverick_int8_zipf():
+    _full_size(CONFIGS["maverick_int8"])

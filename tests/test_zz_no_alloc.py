@@ -27,7 +27,7 @@ def _assert_close(out: torch.Tensor, ref: torch.Tensor, dtype: str):
     assert np.all(np.abs(o - r) <= bound)
 
 
-@pytest.mark.parametrize("dtype", ["bf16", "f32", "fp8"])
+@pytest.mark.parametrize("dtype", ["bf16", "f32", "fp8", "int8"])
 def test_static_forward_matches_allocating_forward_on_two_calls(dtype):
     cfg = LayerConfig(f"noalloc_{dtype}", 300, 256, 8, 384, 256, dtype, wr_std=0.1)
     inp = generate(cfg, seed=11, device="cuda")
