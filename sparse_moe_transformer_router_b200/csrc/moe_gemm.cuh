@@ -726,13 +726,21 @@ __global__ void __launch_bounds__(256) down_finish_kernel(const float* __restric
     const int d4 = d >> 2;
     for (long long i = blockIdx.x * (long long)blockDim.x + threadIdx.x; i < n4;
          i += (long long)gridDim.x * blockDim.x) {
-        const long long t = i / d4, c4 = i % d4;
         float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
-        for (int s = 0; s < splits_r; ++s)
-            for (int j = 0; j < k; ++j) {
-                const float4 v = reinterpret_cast<const float4*>(part_r + stride_r * s)[(t * k + j) * d4 + c4];
+        if (k == 1) {  // routed row t is entry t: the same index as the output
+            for (int s = 0; s < splits_r; ++s) {
+                const float4 v = reinterpret_cast<const float4*>(part_r + stride_r * s)[i];
                 acc.x += v.x, acc.y += v.y, acc.z += v.z, acc.w += v.w;
             }
+        } else {
+            const long long t = i / d4, c4 = i - t * d4;
+            for (int s = 0; s < splits_r; ++s)
+                for (int j = 0; j < k; ++j) {
+                    const float4 v =
+                        reinterpret_cast<const float4*>(part_r + stride_r * s)[(t * k + j) * d4 + c4];
+                    acc.x += v.x, acc.y += v.y, acc.z += v.z, acc.w += v.w;
+                }
+        }
         for (int s = 0; s < splits_s; ++s) {
             const float4 v = reinterpret_cast<const float4*>(part_s + stride_s * s)[i];
             acc.x += v.x, acc.y += v.y, acc.z += v.z, acc.w += v.w;

@@ -186,8 +186,7 @@ __global__ void __launch_bounds__(1024) permute_kernel(const float* __restrict__
                         hl = ol;
                     }
                 }
-                out.v[j] = hv;
-                out.i[j] = hi;
+                out.set(j, hv, hi);
                 if (hl == lane && hi >= 0) ++pos;
             }
             if (lane == 0) {
@@ -196,9 +195,9 @@ __global__ void __launch_bounds__(1024) permute_kernel(const float* __restrict__
                 for (int j = 0; j < kMaxTopK; ++j) {
                     if (j < k) {
                         const size_t n = (size_t)t * k + j;
-                        idx[n] = out.i[j];
-                        lmax[n] = out.v[j];
-                        gate[n] = 1.0f / (1.0f + expf(-out.v[j]));
+                        idx[n] = out.index(j);
+                        lmax[n] = out.value(j);
+                        gate[n] = 1.0f / (1.0f + expf(-out.value(j)));
                     }
                 }
                 margin[t] = out.value(k - 1) - out.value(k);

@@ -374,9 +374,9 @@ __global__ void __launch_bounds__(128, 1)
             for (int j = 0; j < kMaxTopK; ++j) {
                 if (j < topk) {
                     const size_t n = (size_t)t * topk + j;
-                    idx[n] = tk.i[j];
-                    lmax[n] = tk.v[j];
-                    gate[n] = 1.0f / (1.0f + expf(-tk.v[j]));
+                    idx[n] = tk.index(j);
+                    lmax[n] = tk.value(j);
+                    gate[n] = 1.0f / (1.0f + expf(-tk.value(j)));
                 }
             }
             margin[t] = tk.value(topk - 1) - tk.value(topk);  // k-th against the next one
