@@ -106,7 +106,9 @@ typedef struct {
 typedef struct l4moe_handle l4moe_handle;
 
 /* Validate the shapes and dtype and create a handle.  Host only; no device
- * work and no allocation on the device.  *out receives the handle. */
+ * work and no allocation on the device.  *out receives the handle.  The
+ * handle belongs to the CUDA device current at this call: its forwards must
+ * run with that device current (L4MOE_ERR_ARG otherwise). */
 L4MOE_API l4moe_status l4moe_create(const l4moe_params *params, l4moe_handle **out);
 
 /* Free the handle, its own workspace and descriptor cache.  Waits for

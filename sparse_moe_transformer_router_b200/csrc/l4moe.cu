@@ -13,6 +13,7 @@
 #include <cuda_runtime.h>
 
 #include <algorithm>
+#include <atomic>
 #include <cstdio>
 #include <cstring>
 #include <mutex>
@@ -393,12 +394,29 @@ void set_smem_attr(K kernel, size_t bytes) {
     cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)bytes);
 }
 
+// Raise a kernel's dynamic shared-memory limit once per device: the
+// attribute belongs to the kernel's instance in each device's context, so a
+// process that runs layers on several GPUs sets it on each.  `done` holds
+// one bit per device index (devices 64 and up set it on every call).
+template <typename K>
+void ensure_smem_attr(std::atomic<uint64_t>& done, K kernel, size_t bytes) {
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) {
+        set_smem_attr(kernel, bytes);
+        return;
+    }
+    const uint64_t bit = 1ull << dev;
+    if (done.load(std::memory_order_acquire) & bit) return;
+    set_smem_attr(kernel, bytes);
+    done.fetch_or(bit, std::memory_order_acq_rel);
+}
+
 template <typename ET, int NT, int TPT, int NG>
 void launch_router_t(const void* x, const void* Wr, const float* bias, int T, int d, int E,
                      int32_t* idx, float* gate, float* lmax, float* margin, cudaStream_t st) {
     constexpr size_t smem = router_smem_bytes<NT, TPT, NG>();
-    static std::once_flag once;
-    std::call_once(once, [] { set_smem_attr(router_kernel<ET, NT, TPT, NG>, smem); });
+    static std::atomic<uint64_t> attr_done{0};
+    ensure_smem_attr(attr_done, router_kernel<ET, NT, TPT, NG>, smem);
     const int TT = NT / TPT;
     const int wr_vec = (E % Vec16<ET>::N) == 0 ? 1 : 0;
     launch_k(router_kernel<ET, NT, TPT, NG>, dim3((T + TT - 1) / TT), dim3(NT), smem, st,
@@ -422,8 +440,8 @@ void launch_router(const void* x, const void* Wr, const float* bias, int T, int 
 template <int MODE, typename ET, int WQ>
 void launch_gemm(int grid, const BMaps& bm, const GemmArgs& a, cudaStream_t st) {
     using Cfg = GemmCfg<MODE, ET, WQ != kWqNone>;
-    static std::once_flag once;
-    std::call_once(once, [] { set_smem_attr(moe_gemm_kernel<MODE, ET, WQ>, Cfg::SMEM_BYTES); });
+    static std::atomic<uint64_t> attr_done{0};
+    ensure_smem_attr(attr_done, moe_gemm_kernel<MODE, ET, WQ>, Cfg::SMEM_BYTES);
     launch_k(moe_gemm_kernel<MODE, ET, WQ>, dim3(grid), dim3(Cfg::THREADS), Cfg::SMEM_BYTES, st, bm, a);
 }
 
@@ -525,8 +543,8 @@ l4moe_status run_layer(l4moe_handle* h, int T, const void* x, const void* Wr, co
             CUtensorMap m_wr;
             if (!encode_2d(&m_wr, adt, Wr, (uint64_t)E, (uint64_t)d, (uint64_t)E * sizeof(ET), 64, 64))
                 return fail(h, L4MOE_ERR_CUDA, "cuTensorMapEncodeTiled failed for the router weight");
-            static std::once_flag once;
-            std::call_once(once, [] { set_smem_attr(router_mma_kernel, rmma::SMEM_BYTES); });
+            static std::atomic<uint64_t> attr_done{0};
+            ensure_smem_attr(attr_done, router_mma_kernel, rmma::SMEM_BYTES);
             const int n_chunk = split_router ? 16 : E;
             const int tiles = (T + 127) / 128;
             int kslices;
@@ -709,6 +727,9 @@ l4moe_status check_forward_args(l4moe_handle* h, int T, const void* x, const voi
                                 const void* Wsdn, const void* out) {
     if (!h) return L4MOE_ERR_ARG;
     if (T < 0) return fail(h, L4MOE_ERR_ARG, "T must be >= 0");
+    int cur = -1;  // the workspace and descriptors live on the handle's device
+    if (cudaGetDevice(&cur) != cudaSuccess || cur != h->device)
+        return fail(h, L4MOE_ERR_ARG, "the current CUDA device is not the handle's (the one current at l4moe_create)");
     const bool experts = h->p.num_experts > 0;  // without experts W_router, W_gate_up, W_down are unused
     if (!x || !Wsgu || !Wsdn || !out || (experts && (!Wr || !Wgu || !Wdn)))
         return fail(h, L4MOE_ERR_ARG, "null tensor pointer");
