@@ -164,7 +164,7 @@ struct TileInfo {
 constexpr long long kBandBytes = 24ll << 20;
 
 template <int MODE, int ElemCfgBK, int ElemBytes>
-__device__ __forceinline__ TileInfo decode_tile(const GroupTable& tab, const GemmArgs& a, int pos) {
+__host__ __device__ __forceinline__ TileInfo decode_tile(const GroupTable& tab, const GemmArgs& a, int pos) {
     const int L = tile_at(pos, tab.heavy_tiles, tab.total_tiles);
     int lo = 0, hi = tab.num_groups - 1;
     while (lo < hi) {
