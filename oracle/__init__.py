@@ -8,7 +8,8 @@ calls anything here, and this package imports nothing from the product.
 The arithmetic lives in ``oracle.c`` (plain C, fp64 accumulation, OpenMP over
 tokens); this module only compiles it with gcc and marshals numpy arrays.
 Inputs are numpy arrays in their storage dtype: float32, bf16 as uint16 bit
-patterns, E4M3 as uint8 codes, int8 weights as int8.
+patterns, E4M3 as uint8 codes, int8 weights as int8, int4 weights as packed
+bytes viewed with ``INT4X2``.
 
 Every function is pinned by ``tests/test_oracle_pins.py`` to something other
 than itself (library matmuls on reductions of the layer, closed forms,
@@ -23,7 +24,17 @@ import threading
 
 import numpy as np
 
-F32, BF16, E4M3, INT8 = 0, 1, 2, 3
+F32, BF16, E4M3, INT8, INT4 = 0, 1, 2, 3, 4
+
+# int4 weights: a [K, N] matrix stored as [K, N / 2] bytes (two's-complement
+# nibbles, the even column in the low nibble), viewed with this one-byte
+# record dtype so that it is told apart from E4M3 codes.
+INT4X2 = np.dtype([("int4x2", np.uint8)])
+
+
+def as_int4x2(packed: np.ndarray) -> np.ndarray:
+    """View packed int4 bytes (uint8 [K, N / 2]) as the oracle's int4 storage."""
+    return np.ascontiguousarray(packed, dtype=np.uint8).view(INT4X2)
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
 _SRC = os.path.join(_HERE, "oracle.c")
@@ -85,6 +96,8 @@ def _dtype_code(a: np.ndarray) -> int:
         return E4M3
     if a.dtype == np.int8:
         return INT8
+    if a.dtype == INT4X2:
+        return INT4
     raise TypeError(f"oracle: unsupported storage dtype {a.dtype}")
 
 
@@ -164,8 +177,9 @@ def forward(x, Wr, W_gate_up, W_down, Ws_gate_up, Ws_down, *, bias=None,
     """Layer output in fp64 for ``tokens`` (all tokens when None).
 
     W_gate_up / W_down are length-E lists of [d, 2F] / [F, d] arrays; entries
-    may be None for experts no selected token reaches.  For E4M3 and int8
-    weights the per-output-column fp32 scales are required.  k > 1: each token runs its
+    may be None for experts no selected token reaches (int4 weights: packed
+    [d, F] / [F, d / 2] byte arrays viewed as ``INT4X2``).  For E4M3, int8 and
+    int4 weights the per-output-column fp32 scales are required.  k > 1: each token runs its
     k highest-scoring experts, each on the input gated by the sigmoid of its
     own logit, and their outputs add to the shared expert's.  Returns
     (out f64[n_sel, d], idx int32[n_sel], gate f64[n_sel]), or [n_sel, k]
@@ -196,7 +210,7 @@ def forward(x, Wr, W_gate_up, W_down, Ws_gate_up, Ws_down, *, bias=None,
     if F is None:
         F = Fs
     sgu_ptrs = sdn_ptrs = None
-    if w_code in (E4M3, INT8):
+    if w_code in (E4M3, INT8, INT4):
         sgu_ptrs = (ctypes.c_void_p * E)()
         sdn_ptrs = (ctypes.c_void_p * E)()
         for e in range(E):

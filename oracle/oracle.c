@@ -40,6 +40,11 @@
  *   - int8 weights (KerasFormers "Llama 4" page, "Lower memory": weight-only
  *     int8 loading) are two's-complement integers with one fp32 scale per
  *     output column, symmetric (no zero point); w = q * scale.
+ *   - int4 weights (superteams.ai glossary, "The Llama 4 Herd": Scout fits on
+ *     one H100 quantized to int4; aibase model card, "Quantization": on-the-fly
+ *     int4) are two's-complement 4-bit integers packed two per byte along the
+ *     output (column) dimension, the even column in the low nibble, with one
+ *     fp32 scale per output column; w = q * scale.
  *
  * Parity pins (tests/test_oracle_pins.py): E = 1 with the gate forced to 1
  * reduces to two dense SwiGLU FFNs evaluated by a library matmul; a constant
@@ -56,7 +61,7 @@
 #include <omp.h>
 #endif
 
-enum { ORACLE_F32 = 0, ORACLE_BF16 = 1, ORACLE_E4M3 = 2, ORACLE_INT8 = 3 };
+enum { ORACLE_F32 = 0, ORACLE_BF16 = 1, ORACLE_E4M3 = 2, ORACLE_INT8 = 3, ORACLE_INT4 = 4 };
 
 /* bf16 is the upper half of an IEEE binary32; widening is exact. */
 double oracle_bf16_to_double(uint16_t b) {
@@ -88,16 +93,23 @@ static double load_elem(const void *p, int dtype, size_t i) {
     case ORACLE_BF16: return oracle_bf16_to_double(((const uint16_t *)p)[i]);
     case ORACLE_E4M3: return oracle_e4m3_to_double(((const uint8_t *)p)[i]);
     case ORACLE_INT8: return (double)((const int8_t *)p)[i];
+    case ORACLE_INT4: { /* element i is nibble i: byte i / 2, low nibble first */
+        const uint8_t b = ((const uint8_t *)p)[i >> 1];
+        const int q = (i & 1) ? (b >> 4) : (b & 0xF);
+        return (double)(q >= 8 ? q - 16 : q);
+    }
     default: return NAN;
     }
 }
 
-/* A weight element of a [rows, cols] row-major matrix; for E4M3 and int8
- * the per-output-column scale is applied (dequantisation). */
+/* A weight element of a [rows, cols] row-major matrix (int4: cols even,
+ * packed along the row, so element (row, col) is nibble row * cols + col);
+ * for E4M3, int8 and int4 the per-output-column scale is applied
+ * (dequantisation). */
 static double load_weight(const void *W, int dtype, const float *col_scale,
                           size_t row, size_t cols, size_t col) {
     double w = load_elem(W, dtype, row * cols + col);
-    if (dtype == ORACLE_E4M3 || dtype == ORACLE_INT8) w *= (double)col_scale[col];
+    if (dtype == ORACLE_E4M3 || dtype == ORACLE_INT8 || dtype == ORACLE_INT4) w *= (double)col_scale[col];
     return w;
 }
 

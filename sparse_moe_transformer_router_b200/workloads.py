@@ -25,6 +25,7 @@ import torch
 
 E4M3_MAX = 448.0
 INT8_MAX = 127.0
+INT4_MAX = 7.0
 
 
 @dataclass(frozen=True)
@@ -115,6 +116,31 @@ def quantize_int8_columns(w: torch.Tensor):
     scale = torch.where(amax > 0, amax / INT8_MAX, torch.ones_like(amax))
     q = torch.round(w / scale).clamp_(-INT8_MAX, INT8_MAX).to(torch.int8)
     return q, scale.to(torch.float32)
+
+
+def int4_codes_columns(w: torch.Tensor):
+    """Per-output-column symmetric int4 codes of an fp32 [K, N] weight:
+    scale[n] = max_k |w[k, n]| / 7, q = round(w / scale) (to nearest even),
+    clamped to [-7, 7].  Returns (q int8 [K, N], scale f32 [N]), unpacked."""
+    amax = w.abs().amax(dim=0)
+    scale = torch.where(amax > 0, amax / INT4_MAX, torch.ones_like(amax))
+    q = torch.round(w / scale).clamp_(-INT4_MAX, INT4_MAX).to(torch.int8)
+    return q, scale.to(torch.float32)
+
+
+def pack_int4(q: torch.Tensor) -> torch.Tensor:
+    """int4 storage of integer codes q in [-8, 7], [K, N] with N even: two
+    two's-complement nibbles per byte along the row, the even column in the
+    low nibble.  Returns uint8 [K, N / 2]."""
+    assert q.shape[-1] % 2 == 0
+    n = (q.to(torch.int16) & 0xF).to(torch.uint8)
+    return n[..., 0::2] | (n[..., 1::2] << 4)
+
+
+def quantize_int4_columns(w: torch.Tensor):
+    """int4_codes_columns, packed: (uint8 [K, N / 2], scale f32 [N])."""
+    q, scale = int4_codes_columns(w)
+    return pack_int4(q), scale
 
 
 @functools.lru_cache(maxsize=16)

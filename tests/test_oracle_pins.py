@@ -369,3 +369,61 @@ def test_int8_codes_with_unit_scales_equal_the_bf16_layer():
     ob, ib, gb = oracle.forward(x, Wr, [b for _, b in gu], [b for _, b in dn], sgu[1], sdn[1])
     assert np.array_equal(i8, ib) and np.array_equal(g8, gb)
     assert np.array_equal(o8, ob)
+
+
+def test_int4_codes_equal_the_int8_layer_with_the_same_integers():
+    """int4 weights (every code from -8 to 7, packed two per byte along the
+    output columns) with per-column scales equal the int8 layer holding the
+    same integers and scales: a swapped nibble order, a missing sign
+    extension or a packing along the wrong axis breaks the equality."""
+    from sparse_moe_transformer_router_b200.workloads import pack_int4
+    rng = np.random.default_rng(19)
+    T, d, E, F, Fs = 9, 64, 3, 32, 48
+    x, _ = _store(rng.standard_normal((T, d)), "bf16")
+    Wr, _ = _store(rng.standard_normal((d, E)), "bf16")
+
+    def codes(shape):
+        q = rng.integers(-8, 8, size=shape).astype(np.int8)
+        q.flat[:16] = np.arange(-8, 8, dtype=np.int8)
+        s = (rng.random(shape[1]) * 0.05 + 0.01).astype(np.float32)
+        return q, oracle.as_int4x2(pack_int4(torch.from_numpy(q)).numpy()), s
+
+    gu = [codes((d, 2 * F)) for _ in range(E)]
+    dn = [codes((F, d)) for _ in range(E)]
+    sgu, sdn = codes((d, 2 * Fs)), codes((Fs, d))
+    scales = dict(s_gate_up=[g[2] for g in gu], s_down=[g[2] for g in dn], ss_gate_up=sgu[2], ss_down=sdn[2])
+    o4, i4, g4 = oracle.forward(x, Wr, [g[1] for g in gu], [g[1] for g in dn], sgu[1], sdn[1], **scales)
+    o8, i8, g8 = oracle.forward(x, Wr, [g[0] for g in gu], [g[0] for g in dn], sgu[0], sdn[0], **scales)
+    assert np.array_equal(i4, i8) and np.array_equal(g4, g8)
+    assert np.array_equal(o4, o8)
+    assert np.any(o4 != 0)
+
+
+def test_int4_quantised_weights_equal_their_codes_in_the_int8_layer():
+    """The int4 workload's quantiser (per-column scale max|w| / 7, codes in
+    [-7, 7]) fed packed to the oracle gives exactly the int8 layer on the
+    unpacked codes; and at k = E with a saturated gate, the library
+    evaluation of the dequantised weights."""
+    from sparse_moe_transformer_router_b200.workloads import int4_codes_columns, pack_int4
+    rng = np.random.default_rng(20)
+    T, d, F, Fs = 5, 64, 32, 48
+    x, x64 = _store(rng.standard_normal((T, d)), "bf16")
+    Wr, _ = _store(rng.standard_normal((d, 1)), "bf16")
+
+    def q(shape):
+        w = torch.from_numpy(rng.standard_normal(shape) * 0.02).float()
+        w[:, 1] *= 30.0
+        qq, s = int4_codes_columns(w)
+        assert int(qq.abs().max()) <= 7
+        deq = qq.to(torch.float64) * s.to(torch.float64)[None, :]
+        return qq.numpy(), oracle.as_int4x2(pack_int4(qq).numpy()), s.numpy(), deq.numpy()
+
+    gu, dn, sgu, sdn = q((d, 2 * F)), q((F, d)), q((d, 2 * Fs)), q((Fs, d))
+    kw = dict(bias=np.array([100.0], np.float32), s_gate_up=[gu[2]], s_down=[dn[2]], ss_gate_up=sgu[2],
+              ss_down=sdn[2])
+    o4, _, g4 = oracle.forward(x, Wr, [gu[1]], [dn[1]], sgu[1], sdn[1], **kw)
+    o8, _, _ = oracle.forward(x, Wr, [gu[0]], [dn[0]], sgu[0], sdn[0], **kw)
+    assert np.array_equal(o4, o8)
+    assert np.all(g4 == 1.0)
+    ref = _dense_swiglu(x64, gu[3], dn[3]) + _dense_swiglu(x64, sgu[3], sdn[3])
+    assert np.max(np.abs(o4 - ref)) <= 1e-12 * np.sqrt(np.mean(ref ** 2))
