@@ -135,16 +135,29 @@ def profile_traffic(kernel: str, workload: str):
     text = open(path).read()
     m_b = re.search(r"dram_bytes_per_launch:\s*([0-9.eE+]+)", text)
     m_h = re.search(r"sources_sha256:\s*([0-9a-f]+)", text)
-    if not m_b or not m_h or m_h.group(1) != kernel_sources_sha():
+    if not m_b or not m_h or m_h.group(1) != kernel_sources_sha(kernel):
         return None
     return float(m_b.group(1))
 
 
-def kernel_sources_sha() -> str:
-    """Hash of the device-code headers (every kernel lives in a .cuh file)."""
+# The headers each profiled kernel is compiled from (its own code and every
+# header it includes); a committed ncu summary stays valid while they hash
+# to the value it records.  Kernels not listed hash every device header.
+KERNEL_HEADERS = {
+    "gemm_gate_up": ("moe_gemm.cuh", "ptx.cuh", "schedule.cuh"),
+    "gemm_down": ("moe_gemm.cuh", "ptx.cuh", "schedule.cuh"),
+}
+
+
+def kernel_sources_sha(kernel: str | None = None) -> str:
+    """Hash of the device-code headers a kernel is built from (every kernel
+    lives in a .cuh file); all of them when the kernel is not listed."""
     h = hashlib.sha256()
     csrc = os.path.join(ROOT, "sparse_moe_transformer_router_b200", "csrc")
-    for name in sorted(n for n in os.listdir(csrc) if n.endswith(".cuh")):
+    names = KERNEL_HEADERS.get(kernel) if kernel else None
+    if names is None:
+        names = [n for n in os.listdir(csrc) if n.endswith(".cuh")]
+    for name in sorted(names):
         with open(os.path.join(csrc, name), "rb") as f:
             h.update(name.encode())
             h.update(f.read())

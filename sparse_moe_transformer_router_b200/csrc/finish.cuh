@@ -1,0 +1,90 @@
+// finish.cuh -- the kernels that close a GEMM launch made of fp32 partials:
+// the split-K sum of the gate/up contraction (with the gate and SwiGLU), and
+// the down projection's sum of the routed and shared partials, rounded once.
+#pragma once
+#include <cuda_bf16.h>
+#include <cuda_fp16.h>
+#include <cstdint>
+
+#include "moe_gemm.cuh"
+#include "ptx.cuh"
+
+namespace l4moe {
+
+// Split-K finish of the gate/up contraction: h = silu(g * sum_s a_gate) *
+// (g * sum_s a_up) over the splits in order, for the routed slots (g = the
+// slot's sigmoid gate) and the shared rows (g = 1).  One thread per output.
+template <typename ET>
+__global__ void __launch_bounds__(256) gateup_finish_kernel(
+    const float* __restrict__ part_r, long long ld_r, long long stride_r, const float* __restrict__ part_s,
+    long long ld_s, long long stride_s, int ksplit, int Tr, int T, int F, int Fs,
+    const float* __restrict__ gslot, ET* __restrict__ hr, ET* __restrict__ hs) {
+    pdl_enter();
+    // Tr routed rows (token entries), T shared rows
+    const long long n_r = (long long)Tr * F, n = n_r + (long long)T * Fs;
+    for (long long i = blockIdx.x * (long long)blockDim.x + threadIdx.x; i < n;
+         i += (long long)gridDim.x * blockDim.x) {
+        const bool shared = i >= n_r;
+        const long long j = shared ? i - n_r : i;
+        const int w = shared ? Fs : F;
+        const int row = (int)(j / w), f = (int)(j % w);
+        const float* p = shared ? part_s : part_r;
+        const long long ld = shared ? ld_s : ld_r, st = shared ? stride_s : stride_r;
+        float ag = 0.f, au = 0.f;
+        for (int s = 0; s < ksplit; ++s) {
+            ag += p[st * s + (long long)row * ld + f];
+            au += p[st * s + (long long)row * ld + w + f];
+        }
+        const float g = shared ? 1.0f : gslot[row];
+        store_elem((shared ? hs : hr) + (long long)row * w + f, silu_f(g * ag) * (g * au));
+    }
+}
+
+// Down finish: out[t] = rn(sum over splits s and selected experts j of the
+// routed partial of entry t * k + j, then sum over s of the shared partial)
+// -- one rounding, a fixed order.  Partials: routed [splits_r][T * k][d],
+// shared [splits_s][T][d] (fp32, rows un-permuted to entries / tokens).
+// Four outputs per thread; d % 4 == 0.
+template <typename ET>
+__global__ void __launch_bounds__(256) down_finish_kernel(const float* __restrict__ part_r, long long stride_r,
+                                                          int splits_r, const float* __restrict__ part_s,
+                                                          long long stride_s, int splits_s, int k, int d,
+                                                          long long n, ET* __restrict__ out) {
+    pdl_enter();
+    const long long n4 = n >> 2;
+    const int d4 = d >> 2;
+    for (long long i = blockIdx.x * (long long)blockDim.x + threadIdx.x; i < n4;
+         i += (long long)gridDim.x * blockDim.x) {
+        float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+        if (k == 1) {  // routed row t is entry t: the same index as the output
+            for (int s = 0; s < splits_r; ++s) {
+                const float4 v = reinterpret_cast<const float4*>(part_r + stride_r * s)[i];
+                acc.x += v.x, acc.y += v.y, acc.z += v.z, acc.w += v.w;
+            }
+        } else {
+            const long long t = i / d4, c4 = i - t * d4;
+            for (int s = 0; s < splits_r; ++s)
+                for (int j = 0; j < k; ++j) {
+                    const float4 v =
+                        reinterpret_cast<const float4*>(part_r + stride_r * s)[(t * k + j) * d4 + c4];
+                    acc.x += v.x, acc.y += v.y, acc.z += v.z, acc.w += v.w;
+                }
+        }
+        for (int s = 0; s < splits_s; ++s) {
+            const float4 v = reinterpret_cast<const float4*>(part_s + stride_s * s)[i];
+            acc.x += v.x, acc.y += v.y, acc.z += v.z, acc.w += v.w;
+        }
+        if constexpr (sizeof(ET) == 2) {
+            const __nv_bfloat162 lo = __floats2bfloat162_rn(acc.x, acc.y);
+            const __nv_bfloat162 hi = __floats2bfloat162_rn(acc.z, acc.w);
+            uint2 pk;
+            pk.x = *reinterpret_cast<const uint32_t*>(&lo);
+            pk.y = *reinterpret_cast<const uint32_t*>(&hi);
+            reinterpret_cast<uint2*>(out)[i] = pk;
+        } else {
+            reinterpret_cast<float4*>(out)[i] = acc;
+        }
+    }
+}
+
+}  // namespace l4moe

@@ -22,6 +22,7 @@
 #include <vector>
 
 #include "l4moe.h"
+#include "finish.cuh"
 #include "moe_gemm.cuh"
 #include "permute.cuh"
 #include "router.cuh"

@@ -35,7 +35,7 @@ def test_profile_traffic_needs_the_current_kernel_hash(tmp_path, monkeypatch):
     path.write_text(f"# x\n\ndram_bytes_per_launch: 1234500000\nsources_sha256: {sha}\n")
     monkeypatch.setattr(bench, "ROOT", str(tmp_path))
     # the hash covers the kernel headers under ROOT: point it at the real ones
-    monkeypatch.setattr(bench, "kernel_sources_sha", lambda: sha)
+    monkeypatch.setattr(bench, "kernel_sources_sha", lambda kernel=None: sha)
     assert bench.profile_traffic("gemm_gate_up", "w") == 1234500000.0
     path.write_text("dram_bytes_per_launch: 1234500000\nsources_sha256: 0000000000000000\n")
     assert bench.profile_traffic("gemm_gate_up", "w") is None   # kernels changed since
@@ -45,6 +45,26 @@ def test_profile_traffic_needs_the_current_kernel_hash(tmp_path, monkeypatch):
 def test_kernel_hash_covers_only_device_code():
     sha = bench.kernel_sources_sha()
     assert len(sha) == 16 and int(sha, 16) >= 0
+
+
+def test_gemm_hash_covers_exactly_the_headers_the_gemm_includes():
+    """A profiled kernel's hash lists its header and everything that header
+    includes (so an edit there invalidates the committed counters), and no
+    header the kernel does not include."""
+    import re
+    csrc = os.path.join(ROOT, "sparse_moe_transformer_router_b200", "csrc")
+
+    def closure(name, seen):
+        if name in seen:
+            return seen
+        seen.add(name)
+        for inc in re.findall(r'#include "([^"]+)"', open(os.path.join(csrc, name)).read()):
+            closure(inc, seen)
+        return seen
+
+    for kernel in ("gemm_gate_up", "gemm_down"):
+        assert set(bench.KERNEL_HEADERS[kernel]) == closure("moe_gemm.cuh", set())
+        assert bench.kernel_sources_sha(kernel) != bench.kernel_sources_sha()
 
 
 def test_weak_scaling_value():
