@@ -116,6 +116,27 @@ def _stream_handle(stream) -> int | None:
     return stream.cuda_stream
 
 
+_ACT_DTYPE = {"f32": torch.float32, "bf16": torch.bfloat16, "fp8": torch.bfloat16, "int8": torch.bfloat16}
+_W_DTYPE = {"f32": torch.float32, "bf16": torch.bfloat16, "fp8": torch.float8_e4m3fn, "int8": torch.int8}
+
+
+def _expect(t, name, shape, dtype):
+    """Shape / dtype check of one argument (the C ABI sees raw pointers, so a
+    wrong shape would make the kernels read past a buffer)."""
+    if t is None:
+        raise ValueError(f"l4moe: {name} is required")
+    if tuple(t.shape) != tuple(shape):
+        raise ValueError(f"l4moe: {name} has shape {tuple(t.shape)}, expected {tuple(shape)}")
+    if t.dtype != dtype:
+        raise ValueError(f"l4moe: {name} has dtype {t.dtype}, expected {dtype}")
+
+
+def _where(t, name, host=False):
+    """Device check of one argument (after every shape and dtype check)."""
+    if host == t.is_cuda:
+        raise ValueError(f"l4moe: {name} must be a {'host' if host else 'CUDA'} tensor")
+
+
 class _DevView:
     """Zero-copy torch view of a device buffer (CUDA array interface)."""
 
@@ -176,18 +197,49 @@ class L4MoE:
 
     set_fp8_scales = set_weight_scales
 
-    def _weights(self, W_gate_up, W_down):
-        key = (tuple(_ptr(w) for w in W_gate_up), tuple(_ptr(w) for w in W_down))
+    def _weights(self, W_gate_up, W_down, Ws_gate_up, Ws_down):
+        """Pointer arrays of the expert weights; shapes and dtypes are checked
+        whenever the set of weight tensors changes."""
+        key = (tuple(_ptr(w) for w in W_gate_up), tuple(_ptr(w) for w in W_down), _ptr(Ws_gate_up),
+               _ptr(Ws_down))
         if getattr(self, "_wkey", None) != key:
+            d, F, Fs, E = self.d_model, self.expert_ffn, self.shared_ffn, self.num_experts
+            wdt = _W_DTYPE[self.dtype]
+            if len(W_gate_up) != E or len(W_down) != E:
+                raise ValueError(f"l4moe: expected {E} expert weights, got {len(W_gate_up)} / {len(W_down)}")
+            named = [(W_gate_up[e], f"W_gate_up[{e}]", (d, 2 * F)) for e in range(E)]
+            named += [(W_down[e], f"W_down[{e}]", (F, d)) for e in range(E)]
+            named += [(Ws_gate_up, "Ws_gate_up", (d, 2 * Fs)), (Ws_down, "Ws_down", (Fs, d))]
+            for t, name, shape in named:
+                _expect(t, name, shape, wdt)
+            for t, name, _ in named:
+                _where(t, name)
             self._wkey = key
             self._warr = (_ptr_array(W_gate_up), _ptr_array(W_down))
         return self._warr
 
-    def forward(self, x, W_router, W_gate_up, W_down, Ws_gate_up, Ws_down, out=None, stream=None):
+    def _check_io(self, x, W_router, out, host=False):
+        if x.dim() != 2:
+            raise ValueError(f"l4moe: x must be [T, d_model], got shape {tuple(x.shape)}")
         T = x.shape[0]
+        act = _ACT_DTYPE[self.dtype]
+        _expect(x, "x", (T, self.d_model), act)
+        if self.num_experts > 0:
+            _expect(W_router, "W_router", (self.d_model, self.num_experts), act)
+        if out is not None:
+            _expect(out, "out", (T, self.d_model), act)
+        _where(x, "x", host)
+        if self.num_experts > 0:
+            _where(W_router, "W_router")
+        if out is not None:
+            _where(out, "out", host)
+        return T
+
+    def forward(self, x, W_router, W_gate_up, W_down, Ws_gate_up, Ws_down, out=None, stream=None):
+        T = self._check_io(x, W_router, out)
         if out is None:
             out = torch.empty((T, self.d_model), dtype=x.dtype, device=x.device)
-        gu, dn = self._weights(W_gate_up, W_down)
+        gu, dn = self._weights(W_gate_up, W_down, Ws_gate_up, Ws_down)
         self._check(self._lib.l4moe_forward(self._h, T, _ptr(x), _ptr(W_router), gu, dn,
                                             _ptr(Ws_gate_up), _ptr(Ws_down), _ptr(out),
                                             _stream_handle(stream)))
@@ -198,8 +250,10 @@ class L4MoE:
         """l4moe_forward_static: the same layer with the library's fixed device
         scratch array instead of an allocated workspace (no device allocation
         in the call; `out` must be supplied)."""
-        T = x.shape[0]
-        gu, dn = self._weights(W_gate_up, W_down)
+        T = self._check_io(x, W_router, out)
+        if out is None:
+            raise ValueError("l4moe: forward_static needs `out`")
+        gu, dn = self._weights(W_gate_up, W_down, Ws_gate_up, Ws_down)
         self._check(self._lib.l4moe_forward_static(self._h, T, _ptr(x), _ptr(W_router), gu, dn,
                                                    _ptr(Ws_gate_up), _ptr(Ws_down), _ptr(out),
                                                    _stream_handle(stream)))
@@ -207,8 +261,10 @@ class L4MoE:
 
     def forward_host(self, x_host, W_router, W_gate_up, W_down, Ws_gate_up, Ws_down, out_host,
                      stream=None):
-        T = x_host.shape[0]
-        gu, dn = self._weights(W_gate_up, W_down)
+        T = self._check_io(x_host, W_router, out_host, host=True)
+        if out_host is None:
+            raise ValueError("l4moe: forward_host needs `out_host`")
+        gu, dn = self._weights(W_gate_up, W_down, Ws_gate_up, Ws_down)
         self._check(self._lib.l4moe_forward_host(self._h, T, _ptr(x_host), _ptr(W_router), gu, dn,
                                                  _ptr(Ws_gate_up), _ptr(Ws_down), _ptr(out_host),
                                                  _stream_handle(stream)))

@@ -1,0 +1,62 @@
+"""Argument checks of the Python binding (no GPU needed): the C ABI takes raw
+pointers, so the binding compares every tensor's shape, dtype and device
+with the layer before a call could make the kernels read past a buffer."""
+import pytest
+import torch
+
+from sparse_moe_transformer_router_b200.binding import L4MoE
+
+
+def _layer(d=64, F=32, Fs=48, E=3, dtype="bf16"):
+    layer = object.__new__(L4MoE)  # no library call: only the host-side checks
+    layer.d_model, layer.expert_ffn, layer.shared_ffn, layer.num_experts, layer.dtype = d, F, Fs, E, dtype
+    return layer
+
+
+def test_io_shapes_dtypes_and_devices_are_checked():
+    layer = _layer()
+    x = torch.zeros(5, 64, dtype=torch.bfloat16)
+    Wr = torch.zeros(64, 3, dtype=torch.bfloat16)
+    with pytest.raises(ValueError, match="shape"):
+        layer._check_io(torch.zeros(5, 32, dtype=torch.bfloat16), Wr, None)
+    with pytest.raises(ValueError, match="dtype"):
+        layer._check_io(torch.zeros(5, 64, dtype=torch.float32), Wr, None)
+    with pytest.raises(ValueError, match="shape"):
+        layer._check_io(x, torch.zeros(64, 4, dtype=torch.bfloat16), None, host=True)
+    with pytest.raises(ValueError, match="out has shape"):
+        layer._check_io(x, Wr, torch.zeros(6, 64, dtype=torch.bfloat16), host=True)
+    with pytest.raises(ValueError, match="x must be a CUDA tensor"):
+        layer._check_io(x, Wr, None)  # right shape and dtype, but on the host
+    # the host-buffer entry point takes host x / out (W_router stays on the device)
+    with pytest.raises(ValueError, match="W_router must be a CUDA tensor"):
+        layer._check_io(x, Wr, torch.zeros(5, 64, dtype=torch.bfloat16), host=True)
+    with pytest.raises(ValueError, match="x must be"):
+        layer._check_io(torch.zeros(64, dtype=torch.bfloat16), Wr, None)
+
+
+def test_layers_without_experts_need_no_router():
+    layer = _layer(E=0, F=0)
+    x = torch.zeros(5, 64, dtype=torch.bfloat16)
+    with pytest.raises(ValueError, match="CUDA tensor"):
+        layer._check_io(x, None, None)   # reaches the device check: W_router is not asked for
+
+
+@pytest.mark.parametrize("dtype,wdt", [("bf16", torch.bfloat16), ("fp8", torch.float8_e4m3fn),
+                                       ("int8", torch.int8), ("f32", torch.float32)])
+def test_weight_shapes_and_dtypes_are_checked(dtype, wdt):
+    layer = _layer(dtype=dtype)
+    d, F, Fs, E = 64, 32, 48, 3
+    gu = [torch.zeros(d, 2 * F, dtype=wdt) for _ in range(E)]
+    dn = [torch.zeros(F, d, dtype=wdt) for _ in range(E)]
+    sgu, sdn = torch.zeros(d, 2 * Fs, dtype=wdt), torch.zeros(Fs, d, dtype=wdt)
+    with pytest.raises(ValueError, match="expected 3 expert weights"):
+        layer._weights(gu[:2], dn, sgu, sdn)
+    with pytest.raises(ValueError, match=r"W_down\[1\] has shape"):
+        layer._weights(gu, [dn[0], torch.zeros(d, F, dtype=wdt), dn[2]], sgu, sdn)
+    other = torch.bfloat16 if wdt != torch.bfloat16 else torch.float32
+    with pytest.raises(ValueError, match=r"W_gate_up\[0\] has dtype"):
+        layer._weights([gu[0].to(other)] + gu[1:], dn, sgu, sdn)
+    with pytest.raises(ValueError, match="Ws_down has shape"):
+        layer._weights(gu, dn, sgu, torch.zeros(d, Fs, dtype=wdt))
+    with pytest.raises(ValueError, match="CUDA tensor"):
+        layer._weights(gu, dn, sgu, sdn)
