@@ -1,5 +1,6 @@
 """The harness's FLOP accounting, pinned to the modelled costs printed on
-llm-architectures-explained 'Llama 4 Maverick' (section 'Modelled costs')."""
+llm-architectures-explained 'Llama 4 Maverick' (section 'Modelled costs'),
+and to the Scout parameter counts of the superteams.ai glossary."""
 import json
 import os
 
@@ -47,3 +48,30 @@ def test_layer_counts():
     # Scout-shaped prefill: 16 experts touched, bf16
     b = layer_bytes(4096, 5120, 16, 8192, 8192, "bf16", 16)
     assert 4.6e9 < b < 4.8e9
+
+
+def _scout_params(d_shared: int):
+    g = json.load(open(os.path.join(os.path.dirname(__file__), "golden", "scout_glossary_params.json")))
+    a = g["architecture"]
+    d, V, L = a["d_model"], a["vocab"], a["layers"]
+    assert a["moe_every"] == 1 and not a["tie_embeddings"]
+    kv = a["kv_heads"] * a["head_dim"]
+    attn_proj = d * (a["heads"] * a["head_dim"] + 2 * kv) + a["heads"] * a["head_dim"] * d
+    moe_active = flops_per_token(d, a["experts"], a["d_expert"], d_shared) // 2
+    moe_total = d * a["experts"] + a["experts"] * 3 * d * a["d_expert"] + 3 * d * d_shared
+    emb = 2 * d * V  # untied embedding and output head
+    return g, (L * (moe_total + attn_proj) + emb) / 1e9, (L * (moe_active + attn_proj) + emb) / 1e9
+
+
+def test_scout_parameter_counts_select_the_8192_shared_width():
+    """The glossary's Scout figures (about 109B stored, 17B active) follow from
+    the KerasFormers Scout defaults with a shared expert of width 8192 (the
+    Maverick table's d_shared), and not with KerasFormers' dense_mlp_dim of
+    16384, which would make about 23B active per token."""
+    g, total, active = _scout_params(8192)
+    tol = g["printed_relative_tolerance"]
+    assert abs(total - g["printed"]["params_total_b"]) <= tol["params_total_b"] * g["printed"]["params_total_b"]
+    assert abs(active - g["printed"]["params_active_b"]) <= tol["params_active_b"] * g["printed"]["params_active_b"]
+    _, total16, active16 = _scout_params(g["shared_width_readings"]["kerasformers_dense_mlp_dim"])
+    assert abs(active16 - g["printed"]["params_active_b"]) > 0.3 * g["printed"]["params_active_b"]
+    assert g["shared_width_readings"]["maverick_table_d_shared"] == 8192
