@@ -20,6 +20,9 @@
  *     Maverick" field table (ffns.moe.* rows: gated experts of width 8192,
  *     one shared expert of width 8192).
  *   SwiGLU_W(u) = (silu(u . Wg) * (u . Wu)) . Wd with silu(z) = z/(1+e^-z).
+ * l4moe_set_top_k selects k > 1 experts per token instead (the k largest
+ * logits, each expert gated by the sigmoid of its own logit, the k routed
+ * outputs added to the shared one).
  * With E = 0 the layer is the dense SwiGLU feed-forward of the layers
  * without experts (the Maverick field table's dense width 16384 as Fs):
  * W_router, W_gate_up and W_down are unused (may be NULL) and F may be 0.
@@ -58,7 +61,10 @@
  *
  * Requirements: d, F, Fs multiples of 64; 0 <= E <= 256 (F > 0 when E > 0); all tensor pointers
  * 16-byte aligned.  One handle serves one stream at a time (the workspace is
- * shared by the calls made with it).
+ * shared by the calls made with it).  The library sees raw pointers, not
+ * buffer sizes: every tensor must hold at least the elements its layout above
+ * states, or the kernels read or write past it (the Python binding checks
+ * shapes and dtypes before it calls in).
  */
 #ifndef L4MOE_H
 #define L4MOE_H
@@ -116,8 +122,10 @@ L4MOE_API l4moe_status l4moe_create(const l4moe_params *params, l4moe_handle **o
 L4MOE_API void l4moe_destroy(l4moe_handle *h);
 
 /* Bytes of device workspace l4moe_forward needs for up to max_tokens tokens
- * (routing vectors, permutation, group tables, gated expert-ordered input,
- * both hidden activations, host-path staging).  0 on a bad argument. */
+ * with the handle's current experts per token (l4moe_set_top_k): routing
+ * vectors, permutation, group tables, gated expert-ordered input, both
+ * hidden activations, fp32 partials, host-path staging.  0 on a bad
+ * argument. */
 L4MOE_API size_t l4moe_workspace_size(const l4moe_handle *h, int max_tokens);
 
 /* Give the handle a caller-owned device workspace of `bytes` bytes (256-byte
