@@ -148,7 +148,8 @@ L4MOE_API l4moe_status l4moe_set_router_bias(l4moe_handle *h, const float *bias_
  * l4moe_get_routing then hold T * k entries (entry t * k + j: token t's j-th
  * expert; margin stays [T]: the k-th logit minus the next one).  Changing k
  * frees a workspace the handle allocated (it synchronises the device) and
- * fails with L4MOE_ERR_WORKSPACE when a caller's workspace is too small. */
+ * fails with L4MOE_ERR_WORKSPACE when a caller's workspace is too small; the
+ * routing arrays then describe the next forward, not the earlier ones. */
 L4MOE_API l4moe_status l4moe_set_top_k(l4moe_handle *h, int k);
 
 /* E4M3 or int8 weights only: per-output-column fp32 scales (device
