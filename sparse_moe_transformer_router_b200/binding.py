@@ -161,6 +161,8 @@ class L4MoE:
         self._h = h
         self._keep = []
         self.last_T = 0
+        # the handle belongs to the device current at creation (as in the C ABI)
+        self.device = torch.device("cuda", torch.cuda.current_device()) if torch.cuda.is_available() else None
 
     def close(self):
         if getattr(self, "_h", None):
@@ -293,7 +295,7 @@ class L4MoE:
                 ("perm", (Tv,), "<i4")]
         out = {}
         for (name, shape, ts), p in zip(spec, ptrs):
-            out[name] = torch.as_tensor(_DevView(p.value, shape, ts), device="cuda")
+            out[name] = torch.as_tensor(_DevView(p.value, shape, ts), device=self.device)
         return out
 
     def check_device_status(self, stream=None):
