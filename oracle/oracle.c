@@ -51,7 +51,12 @@
  * logit gives the sigmoid closed form and pins input (not output) gating;
  * ties resolve to the lowest index like numpy.argmax; the permutation equals
  * numpy's stable argsort; zero input gives exactly zero output; the E4M3 and
- * bf16 decoders agree with torch's for every code.
+ * bf16 decoders agree with torch's for every code; E4M3 and int8 weights
+ * equal the dense layer on dequantised weights, int8 codes with unit scales
+ * the bf16 layer on the same integers, int4 codes the int8 layer on the same
+ * integers; top-k selection equals a lexsort of the logits, and with k = E
+ * the layer equals a library evaluation over every expert; without experts
+ * the layer is one library SwiGLU.
  */
 #include <math.h>
 #include <stdint.h>
