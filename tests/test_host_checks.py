@@ -6,7 +6,11 @@
   logits with ties, NaN and -inf (tests/host/topk_check.cu);
 - the grouped GEMM's tile schedule (tile_at, decode_tile) on random work
   lists: every tile decoded exactly once and inside its group
-  (tests/host/schedule_check.cu).
+  (tests/host/schedule_check.cu);
+- the workspace layout and split-K plan of the library's host code on random
+  shapes, dtypes, k and token budgets: aligned, ordered segments large
+  enough for any smaller batch, partial planes included
+  (tests/host/layout_check.cu).
 """
 import os
 import shutil
@@ -18,8 +22,8 @@ ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
 NVCC = shutil.which("nvcc") or ("/usr/local/cuda/bin/nvcc" if os.path.exists("/usr/local/cuda/bin/nvcc") else None)
 
 
-def _build_and_run(src: str, exe, extra=()):
-    subprocess.run([NVCC, "-std=c++17", "-O2", "-x", "cu", "--expt-relaxed-constexpr",
+def _build_and_run(src: str, exe, extra=("-O2",)):
+    subprocess.run([NVCC, "-std=c++17", "-x", "cu", "--expt-relaxed-constexpr",
                     "-gencode", "arch=compute_100a,code=sm_100a", *extra,
                     "-I", os.path.join(ROOT, "include"),
                     "-I", os.path.join(ROOT, "sparse_moe_transformer_router_b200", "csrc"),
@@ -37,3 +41,8 @@ def test_topk_list_matches_brute_force(tmp_path):
 @pytest.mark.skipif(NVCC is None, reason="nvcc not available")
 def test_gemm_tile_schedule_covers_every_tile_once(tmp_path):
     _build_and_run("schedule_check.cu", tmp_path / "schedule_check")
+
+
+@pytest.mark.skipif(NVCC is None, reason="nvcc not available")
+def test_workspace_layout_holds_every_smaller_batch(tmp_path):
+    _build_and_run("layout_check.cu", tmp_path / "layout_check", extra=("-O1",))
