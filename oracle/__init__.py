@@ -79,8 +79,10 @@ def _load():
             lib.oracle_forward.argtypes = [i32, i32, i32, i32, i32, i32,
                                            vp, i32, vp, i32, f32p,
                                            vp, vp, vp, vp, i32,
-                                           vp, vp, vp, vp,
+                                           vp, vp, vp, vp, i32,
                                            i32, vp, vp, vp, vp]
+            lib.oracle_e4m3_encode.restype = ctypes.c_uint8
+            lib.oracle_e4m3_encode.argtypes = [ctypes.c_float]
             lib.oracle_num_threads.restype = ctypes.c_int
             lib.oracle_num_threads.argtypes = []
             _lib = lib
@@ -116,6 +118,11 @@ def bf16_to_f64(bits: int) -> float:
 
 def e4m3_to_f64(code: int) -> float:
     return float(_load().oracle_e4m3_to_double(int(code)))
+
+
+def e4m3_encode(v: float) -> int:
+    """E4M3 code of an fp32 value (round to nearest even, saturating)."""
+    return int(_load().oracle_e4m3_encode(float(np.float32(v))))
 
 
 def route(x: np.ndarray, Wr: np.ndarray, bias: np.ndarray | None = None):
@@ -173,7 +180,7 @@ def permutation(idx: np.ndarray, E: int):
 
 def forward(x, Wr, W_gate_up, W_down, Ws_gate_up, Ws_down, *, bias=None,
             s_gate_up=None, s_down=None, ss_gate_up=None, ss_down=None,
-            tokens=None, k=1):
+            tokens=None, k=1, act_fp8=False):
     """Layer output in fp64 for ``tokens`` (all tokens when None).
 
     W_gate_up / W_down are length-E lists of [d, 2F] / [F, d] arrays; entries
@@ -183,7 +190,8 @@ def forward(x, Wr, W_gate_up, W_down, Ws_gate_up, Ws_down, *, bias=None,
     k highest-scoring experts, each on the input gated by the sigmoid of its
     own logit, and their outputs add to the shared expert's.  Returns
     (out f64[n_sel, d], idx int32[n_sel], gate f64[n_sel]), or [n_sel, k]
-    index and gate arrays for k > 1.
+    index and gate arrays for k > 1.  act_fp8: the FP8 activation mode (every
+    contraction input row quantised to E4M3 with its own fp32 scale).
     """
     x = np.ascontiguousarray(x)
     Wr = np.ascontiguousarray(Wr)
@@ -242,7 +250,7 @@ def forward(x, Wr, W_gate_up, W_down, Ws_gate_up, Ws_down, *, bias=None,
         w_code,
         None if sgu_ptrs is None else ctypes.cast(sgu_ptrs, ctypes.c_void_p),
         None if sdn_ptrs is None else ctypes.cast(sdn_ptrs, ctypes.c_void_p),
-        _ptr(ss_gate_up), _ptr(ss_down), n_sel, _ptr(sel), _ptr(out),
+        _ptr(ss_gate_up), _ptr(ss_down), 1 if act_fp8 else 0, n_sel, _ptr(sel), _ptr(out),
         _ptr(sel_idx), _ptr(sel_gate))
     del keep
     if rc != 0:

@@ -40,6 +40,14 @@
  *   - int8 weights (KerasFormers "Llama 4" page, "Lower memory": weight-only
  *     int8 loading) are two's-complement integers with one fp32 scale per
  *     output column, symmetric (no zero point); w = q * scale.
+ *   - FP8 activations, an opt-in mode (superteams.ai glossary, "Running
+ *     Llama 4 Yourself": Maverick served with FP8 quantisation): each
+ *     contraction input row -- a token's x, and a token's hidden row of each
+ *     expert it runs -- is quantised to E4M3 with its own scale:
+ *     s = fp32(max|v| / 448) (1 for an all-zero row), code =
+ *     e4m3_rne_satfinite(fp32(v / s)), value = code * s.  The hidden rows
+ *     are rounded to fp32 before they are quantised.  The gate still scales
+ *     the routed expert's (dequantised) input.
  *   - int4 weights (superteams.ai glossary, "The Llama 4 Herd": Scout fits on
  *     one H100 quantized to int4; aibase model card, "Quantization": on-the-fly
  *     int4) are two's-complement 4-bit integers packed two per byte along the
@@ -90,6 +98,46 @@ double oracle_e4m3_to_double(uint8_t q) {
     else
         v = ldexp(1.0 + (double)m / 8.0, e - 7);
     return sign ? -v : v;
+}
+
+/* OCP E4M3 encoding of a float: round to nearest even, values beyond the
+ * largest finite one (448) saturate to +-448, NaN gives 0x7F.  Normal
+ * numbers are 1.f * 2^E with E in [-6, 8] and 3 fraction bits (exponent
+ * field E + 7); below 2^-6 the codes are multiples of 2^-9 (exponent field 0).
+ * Every step below is exact in double except the one rint (round half to
+ * even, the default rounding mode). */
+uint8_t oracle_e4m3_encode(float v) {
+    if (v != v) return 0x7F;
+    const uint8_t sign = signbit(v) ? 0x80 : 0x00;
+    const double a = fabs((double)v);
+    if (a >= 448.0) return sign | 0x7E;
+    if (a < ldexp(1.0, -6)) /* 0..8 multiples of 2^-9; 8 is 2^-6, code 0x08 */
+        return sign | (uint8_t)rint(a * 512.0);
+    int e2;
+    frexp(a, &e2); /* a = m * 2^e2, m in [0.5, 1) */
+    int E = e2 - 1;
+    double f = rint((a / ldexp(1.0, E) - 1.0) * 8.0);
+    if (f == 8.0) {
+        f = 0.0;
+        E += 1;
+    }
+    return sign | (uint8_t)(((E + 7) << 3) | (int)f);
+}
+
+/* FP8 activation mode: v[0..n) (fp64 values, first rounded to fp32) replaced
+ * by their E4M3 quantisation with one scale for the row (see the header). */
+static void quantise_row_e4m3(int n, double *v) {
+    float amax = 0.0f;
+    for (int j = 0; j < n; ++j) {
+        float a = fabsf((float)v[j]);
+        if (a > amax) amax = a;
+    }
+    float s = amax / 448.0f;
+    if (s == 0.0f) s = 1.0f;
+    for (int j = 0; j < n; ++j) {
+        float q = (float)v[j] / s;
+        v[j] = oracle_e4m3_to_double(oracle_e4m3_encode(q)) * (double)s;
+    }
 }
 
 static double load_elem(const void *p, int dtype, size_t i) {
@@ -193,7 +241,7 @@ static void route_token_topk(int d, int E, int k, const void *x_t, int x_dtype,
  *   a = u . Wgu  (2Fw values), h_j = silu(a_j) * a_{Fw+j},  y += h . Wd.  */
 static void swiglu_ffn_accumulate(int d, int Fw, const double *u,
                                   const void *Wgu, const void *Wd, int w_dtype,
-                                  const float *s_gu, const float *s_d,
+                                  const float *s_gu, const float *s_d, int act_fp8,
                                   double *a, double *h, double *y) {
     size_t two_f = 2 * (size_t)Fw;
     for (size_t j = 0; j < two_f; ++j) a[j] = 0.0;
@@ -203,6 +251,7 @@ static void swiglu_ffn_accumulate(int d, int Fw, const double *u,
             a[j] += uk * load_weight(Wgu, w_dtype, s_gu, (size_t)k, two_f, j);
     }
     for (int j = 0; j < Fw; ++j) h[j] = silu(a[j]) * a[Fw + j];
+    if (act_fp8) quantise_row_e4m3(Fw, h);
     for (int j = 0; j < Fw; ++j) {
         double hj = h[j];
         for (int n = 0; n < d; ++n)
@@ -262,7 +311,7 @@ int oracle_forward(int T, int d, int E, int k, int F, int Fs,
                    const void *const *W_gate_up, const void *const *W_down,
                    const void *Ws_gate_up, const void *Ws_down, int w_dtype,
                    const float *const *s_gate_up, const float *const *s_down,
-                   const float *ss_gate_up, const float *ss_down,
+                   const float *ss_gate_up, const float *ss_down, int act_fp8,
                    int n_sel, const int32_t *sel, double *out,
                    int32_t *sel_idx, double *sel_gate) {
     size_t xs = (x_dtype == ORACLE_F32) ? 4 : 2;
@@ -281,12 +330,16 @@ int oracle_forward(int T, int d, int E, int k, int F, int Fs,
         /* shared expert on the ungated input (with E == 0 the whole layer:
          * the dense SwiGLU feed-forward of the layers without experts) */
         for (int k = 0; k < d; ++k) u[k] = load_elem(x_t, x_dtype, (size_t)k);
+        if (act_fp8) quantise_row_e4m3(d, u); /* x_t as the contractions see it */
+        double *xq = (double *)malloc(sizeof(double) * (size_t)d);
+        for (int k = 0; k < d; ++k) xq[k] = u[k];
         swiglu_ffn_accumulate(d, Fs, u, Ws_gate_up, Ws_down, w_dtype,
-                              ss_gate_up, ss_down, a, h, y);
+                              ss_gate_up, ss_down, act_fp8, a, h, y);
         if (E == 0) {
             if (sel_idx) sel_idx[i] = -1;
             if (sel_gate) sel_gate[i] = 0.0;
             free(u);
+            free(xq);
             free(a);
             free(h);
             continue;
@@ -308,12 +361,13 @@ int oracle_forward(int T, int d, int E, int k, int F, int Fs,
                 missing |= 1;
                 continue;
             }
-            for (int kk = 0; kk < d; ++kk) u[kk] = g * load_elem(x_t, x_dtype, (size_t)kk);
+            for (int kk = 0; kk < d; ++kk) u[kk] = g * xq[kk];
             swiglu_ffn_accumulate(d, F, u, W_gate_up[e], W_down[e], w_dtype,
                                   s_gate_up ? s_gate_up[e] : NULL,
-                                  s_down ? s_down[e] : NULL, a, h, y);
+                                  s_down ? s_down[e] : NULL, act_fp8, a, h, y);
         }
         free(u);
+        free(xq);
         free(a);
         free(h);
     }

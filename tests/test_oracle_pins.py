@@ -427,3 +427,95 @@ def test_int4_quantised_weights_equal_their_codes_in_the_int8_layer():
     assert np.all(g4 == 1.0)
     ref = _dense_swiglu(x64, gu[3], dn[3]) + _dense_swiglu(x64, sgu[3], sdn[3])
     assert np.max(np.abs(o4 - ref)) <= 1e-12 * np.sqrt(np.mean(ref ** 2))
+
+
+def test_e4m3_encoder_round_trips_every_code_and_matches_torch():
+    """The FP8 activation mode's encoder: every finite code decodes and
+    re-encodes to itself (both zeros included); on random fp32 values across
+    the whole range (subnormals, ties, the top binade) it agrees with torch's
+    float8_e4m3fn cast (round to nearest even); beyond 448 it saturates."""
+    for c in range(256):
+        if c & 0x7F == 0x7F:
+            continue
+        assert oracle.e4m3_encode(oracle.e4m3_to_f64(c)) == c, hex(c)
+    rng = np.random.default_rng(21)
+    mag = np.exp2(rng.uniform(-12, np.log2(448.0), 20000)).astype(np.float32)
+    v = mag * rng.choice([-1.0, 1.0], mag.size).astype(np.float32)
+    ties = np.array([(a + b) / 2 for a, b in zip(range(0, 8), range(1, 9))], np.float32) * np.float32(2.0 ** -9)
+    v = np.concatenate([v, ties, -ties, np.float32([1.0625, 1.1875, 416.0, 432.0, 440.0])])
+    want = torch.from_numpy(v).to(torch.float8_e4m3fn).view(torch.uint8).numpy()
+    got = np.array([oracle.e4m3_encode(x) for x in v], np.uint8)
+    assert np.array_equal(got, want)
+    for big in (448.0, 449.0, 464.0, 1e6, float("inf")):
+        assert oracle.e4m3_encode(big) == 0x7E and oracle.e4m3_encode(-big) == 0xFE
+
+
+def _e4m3_rows(v64: np.ndarray) -> np.ndarray:
+    """Per-row E4M3 quantisation through torch: s = fp32(max|v| / 448), codes
+    = float8 cast of fp32(v / s), values = codes * s (fp64)."""
+    v = torch.from_numpy(np.ascontiguousarray(v64)).float()
+    s = v.abs().amax(dim=1, keepdim=True) / 448.0
+    s = torch.where(s == 0, torch.ones_like(s), s)
+    q = (v / s).to(torch.float8_e4m3fn)
+    return (q.double() * s.double()).numpy()
+
+
+def test_fp8_activation_mode_is_the_layer_on_e4m3_rows():
+    """FP8 activation mode: the layer equals a library evaluation where x and
+    every hidden row (shared and routed) are quantised per row by torch's
+    float8 cast with the same fp32 scale arithmetic, and the gate scales the
+    routed expert's quantised input."""
+    rng = np.random.default_rng(22)
+    T, d, E, F, Fs = 7, 64, 3, 32, 48
+    L = _layer(rng, T, d, E, F, Fs, "bf16", wstd=0.2)
+    out, idx, gate = oracle.forward(L["x"], L["Wr"], L["Wgu"], L["Wd"], L["Wsgu"], L["Wsd"], act_fp8=True)
+    xq = _e4m3_rows(L["x64"])
+
+    def ffn(u, Wgu, Wd):
+        a = u @ Wgu
+        Fw = Wd.shape[0]
+        h = torch.nn.functional.silu(torch.from_numpy(a[:, :Fw])).numpy() * a[:, Fw:]
+        return _e4m3_rows(h) @ Wd
+
+    ref = ffn(xq, L["Wsgu64"], L["Wsd64"])
+    for t in range(T):
+        e = int(idx[t])
+        ref[t] += ffn(gate[t] * xq[t:t + 1], L["Wgu64"][e], L["Wd64"][e])[0]
+    scale = np.sqrt(np.mean(ref ** 2))
+    assert np.max(np.abs(out - ref)) <= 1e-12 * scale
+    # and it is a different layer from the bf16-activation one
+    plain, _, _ = oracle.forward(L["x"], L["Wr"], L["Wgu"], L["Wd"], L["Wsgu"], L["Wsd"])
+    rel = np.sqrt(np.mean((out - plain) ** 2)) / scale
+    assert 1e-3 < rel < 0.2
+
+
+def test_fp8_activation_mode_keeps_rows_already_in_e4m3():
+    """Input rows that are E4M3 values times a power of two, with the row
+    maximum at 448 times it, quantise to themselves: with one expert and a
+    saturated gate the mode then equals the library evaluation that
+    quantises only the hidden rows (a slip in the scale, say max / 447, or
+    in the rounding would move some of the inputs)."""
+    codes = np.array([oracle.e4m3_to_f64(c) for c in range(0x00, 0x7F)], np.float64)
+    rng = np.random.default_rng(23)
+    T, d, F, Fs = 4, 64, 32, 48
+    x = rng.choice(np.concatenate([codes, -codes]), size=(T, d)) * 2.0 ** -6
+    x[:, 0] = 448.0 * 2.0 ** -6
+    xb = _bf16_bits(x)
+    assert np.array_equal(_bf16_f64(xb), x)          # exact in bf16
+    Wr, _ = _store(rng.standard_normal((d, 1)), "bf16")
+    Wgu, Wgu64 = _store(rng.standard_normal((d, 2 * F)) * 0.2, "bf16")
+    Wd, Wd64 = _store(rng.standard_normal((F, d)) * 0.2, "bf16")
+    Wsgu, Wsgu64 = _store(rng.standard_normal((d, 2 * Fs)) * 0.2, "bf16")
+    Wsd, Wsd64 = _store(rng.standard_normal((Fs, d)) * 0.2, "bf16")
+    out, _, gate = oracle.forward(xb, Wr, [Wgu], [Wd], Wsgu, Wsd, bias=np.array([100.0], np.float32),
+                                  act_fp8=True)
+    assert np.all(gate == 1.0)
+
+    def ffn(u, A, B):
+        a = u @ A
+        Fw = B.shape[0]
+        h = torch.nn.functional.silu(torch.from_numpy(a[:, :Fw])).numpy() * a[:, Fw:]
+        return _e4m3_rows(h) @ B
+
+    ref = ffn(x, Wsgu64, Wsd64) + ffn(x, Wgu64, Wd64)
+    assert np.max(np.abs(out - ref)) <= 1e-12 * np.sqrt(np.mean(ref ** 2))
