@@ -200,11 +200,17 @@ class L4MoE:
     set_fp8_scales = set_weight_scales
 
     def _weights(self, W_gate_up, W_down, Ws_gate_up, Ws_down):
-        """Pointer arrays of the expert weights; shapes and dtypes are checked
-        whenever the set of weight tensors changes."""
-        key = (tuple(_ptr(w) for w in W_gate_up), tuple(_ptr(w) for w in W_down), _ptr(Ws_gate_up),
-               _ptr(Ws_down))
-        if getattr(self, "_wkey", None) != key:
+        """Pointer arrays of the expert weights; shapes, dtypes, devices and
+        contiguity are checked whenever the weights' addresses change.  The
+        key is the plain address list (the per-call cost with 128 experts is
+        ~20 us of Python, against ~60 us when every call re-checked every
+        tensor)."""
+        try:
+            key = ([w.data_ptr() for w in W_gate_up], [w.data_ptr() for w in W_down],
+                   Ws_gate_up.data_ptr(), Ws_down.data_ptr())
+        except AttributeError:  # a missing weight: the checks below name it
+            key = None
+        if key is None or getattr(self, "_wkey", None) != key:
             d, F, Fs, E = self.d_model, self.expert_ffn, self.shared_ffn, self.num_experts
             wdt = _W_DTYPE[self.dtype]
             if len(W_gate_up) != E or len(W_down) != E:

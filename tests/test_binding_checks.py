@@ -60,3 +60,25 @@ def test_weight_shapes_and_dtypes_are_checked(dtype, wdt):
         layer._weights(gu, dn, sgu, torch.zeros(d, Fs, dtype=wdt))
     with pytest.raises(ValueError, match="CUDA tensor"):
         layer._weights(gu, dn, sgu, sdn)
+
+
+def test_weight_arrays_are_cached_by_address_and_rechecked_on_change(monkeypatch):
+    from sparse_moe_transformer_router_b200 import binding
+    monkeypatch.setattr(binding, "_where", lambda t, name, host=False: None)  # host tensors stand in
+    layer = _layer()
+    d, F, Fs, E = 64, 32, 48, 3
+    gu = [torch.zeros(d, 2 * F, dtype=torch.bfloat16) for _ in range(E)]
+    dn = [torch.zeros(F, d, dtype=torch.bfloat16) for _ in range(E)]
+    sgu, sdn = torch.zeros(d, 2 * Fs, dtype=torch.bfloat16), torch.zeros(Fs, d, dtype=torch.bfloat16)
+    first = layer._weights(gu, dn, sgu, sdn)
+    assert [first[0][i] for i in range(E)] == [w.data_ptr() for w in gu]
+    assert layer._weights(list(gu), list(dn), sgu, sdn) is first      # same addresses: cached
+    gu2 = gu[:2] + [torch.ones(d, 2 * F, dtype=torch.bfloat16)]
+    second = layer._weights(gu2, dn, sgu, sdn)
+    assert second is not first and second[0][2] == gu2[2].data_ptr()
+    with pytest.raises(ValueError, match=r"W_down\[0\] is required"):
+        layer._weights(gu, [None] + dn[1:], sgu, sdn)
+    with pytest.raises(ValueError, match=r"W_gate_up\[1\] has shape"):
+        layer._weights([gu[0], torch.zeros(d, F, dtype=torch.bfloat16), gu[2]], dn, sgu, sdn)
+    with pytest.raises(ValueError, match="contiguous"):
+        layer._weights([gu[0], torch.zeros(2 * F, d, dtype=torch.bfloat16).t(), gu[2]], dn, sgu, sdn)
