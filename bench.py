@@ -285,9 +285,28 @@ def replica_throughput(world: int, tokens_per_rank: int, steps: int, t_ms: float
     return world * tokens_per_rank * steps / (t_ms / 1e3)
 
 
+def free_port() -> int:
+    import socket
+    with socket.socket() as s:
+        s.bind(("127.0.0.1", 0))
+        return s.getsockname()[1]
+
+
+def relaunch_ranks(n: int) -> int:
+    """`--gpus N` without a launcher: start N ranks of this same command
+    line under torch.distributed.run on this node (rendezvous on 127.0.0.1)
+    and return its exit status.  The ranks find WORLD_SIZE set and run."""
+    cmd = [sys.executable, "-m", "torch.distributed.run", "--nnodes=1", f"--nproc-per-node={n}",
+           "--master-addr", "127.0.0.1", "--master-port", str(free_port()),
+           os.path.abspath(__file__), *sys.argv[1:]]
+    return subprocess.call(cmd)
+
+
 def main():
     ap = argparse.ArgumentParser()
-    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--gpus", type=int, default=None,
+                    help="ranks (one per GPU); without torchrun, N > 1 relaunches this command "
+                         "under torch.distributed.run")
     ap.add_argument("--steps", type=int, default=100)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--workload", default=DEFAULT_WORKLOAD, choices=sorted(CONFIGS))
@@ -299,7 +318,11 @@ def main():
     ap.add_argument("--e2e-steps", type=int, default=0)
     args = ap.parse_args()
     args.warmup = max(args.warmup, 3)
+    if args.gpus is not None and args.gpus > 1 and "WORLD_SIZE" not in os.environ:
+        sys.exit(relaunch_ranks(args.gpus))
     rank, world, local = dist_env()
+    if args.gpus is not None and world != args.gpus:
+        raise SystemExit(f"bench.py: --gpus {args.gpus} but the launcher started {world} ranks")
     if world > 1:
         import datetime
         import torch.distributed as dist

@@ -216,7 +216,14 @@ L4MOE_API l4moe_status l4moe_forward_host(l4moe_handle *h, int T, const void *x_
  * handle, shares the one array: calls
  * whose work overlaps on the GPU (other streams, other threads) race and
  * corrupt each other; serialise them.  The array keeps the last call's
- * contents; the call clears the device error word itself.  Per-kernel
+ * contents; the call clears the device error word itself.  Each call copies
+ * the handle's weight descriptors (and, for 8-bit weights, its scale-pointer
+ * table) from host tables the handle owns into the array; those tables sit at
+ * fixed addresses for the handle's life and always describe the weights of
+ * the handle's latest call (and scales of its latest l4moe_set_weight_scales).
+ * Copies recorded under stream capture read them again at every replay, so
+ * such a graph needs its handle alive and still keyed to the graph's weights
+ * and scales.  Per-kernel
  * timing is not recorded for these calls, and l4moe_get_routing /
  * l4moe_check_device_status keep referring to the handle's own workspace. */
 #define L4MOE_STATIC_WORKSPACE_BYTES (32u << 20)

@@ -80,7 +80,9 @@ def _load():
                                            vp, i32, vp, i32, f32p,
                                            vp, vp, vp, vp, i32,
                                            vp, vp, vp, vp, i32,
-                                           i32, vp, vp, vp, vp]
+                                           i32, vp, vp, vp, vp, i32, vp]
+            lib.oracle_round_hidden.restype = ctypes.c_double
+            lib.oracle_round_hidden.argtypes = [ctypes.c_double, i32]
             lib.oracle_e4m3_encode.restype = ctypes.c_uint8
             lib.oracle_e4m3_encode.argtypes = [ctypes.c_float]
             lib.oracle_num_threads.restype = ctypes.c_int
@@ -178,9 +180,18 @@ def permutation(idx: np.ndarray, E: int):
     return counts, offsets, perm
 
 
+HIDDEN_ROUND = {None: 0, "bf16": 1, "f16": 2}
+
+
+def round_hidden(v: float, kind: str) -> float:
+    """The oracle's rounding of one hidden value (fp64 -> fp32 -> bf16 or
+    f16, nearest even)."""
+    return float(_load().oracle_round_hidden(float(v), HIDDEN_ROUND[kind]))
+
+
 def forward(x, Wr, W_gate_up, W_down, Ws_gate_up, Ws_down, *, bias=None,
             s_gate_up=None, s_down=None, ss_gate_up=None, ss_down=None,
-            tokens=None, k=1, act_fp8=False):
+            tokens=None, k=1, act_fp8=False, hidden_round=None):
     """Layer output in fp64 for ``tokens`` (all tokens when None).
 
     W_gate_up / W_down are length-E lists of [d, 2F] / [F, d] arrays; entries
@@ -192,6 +203,10 @@ def forward(x, Wr, W_gate_up, W_down, Ws_gate_up, Ws_down, *, bias=None,
     (out f64[n_sel, d], idx int32[n_sel], gate f64[n_sel]), or [n_sel, k]
     index and gate arrays for k > 1.  act_fp8: the FP8 activation mode (every
     contraction input row quantised to E4M3 with its own fp32 scale).
+    hidden_round ("bf16" or "f16"): also return, as a fourth element, the
+    same outputs with every hidden value rounded to that type (through fp32)
+    before the down projection -- the roundings a GPU that keeps the hidden
+    rows in that type makes, with everything else exact.
     """
     x = np.ascontiguousarray(x)
     Wr = np.ascontiguousarray(Wr)
@@ -243,6 +258,7 @@ def forward(x, Wr, W_gate_up, W_down, Ws_gate_up, Ws_down, *, bias=None,
     out = np.zeros((n_sel, d), np.float64)
     sel_idx = np.empty(n_sel * k, np.int32)
     sel_gate = np.empty(n_sel * k, np.float64)
+    out_h = np.zeros((n_sel, d), np.float64) if hidden_round else None
     rc = _load().oracle_forward(
         T, d, E, k, F, Fs, _ptr(x), _dtype_code(x), _ptr(Wr), _dtype_code(Wr),
         _ptr(bias), ctypes.cast(gu_ptrs, ctypes.c_void_p),
@@ -251,7 +267,7 @@ def forward(x, Wr, W_gate_up, W_down, Ws_gate_up, Ws_down, *, bias=None,
         None if sgu_ptrs is None else ctypes.cast(sgu_ptrs, ctypes.c_void_p),
         None if sdn_ptrs is None else ctypes.cast(sdn_ptrs, ctypes.c_void_p),
         _ptr(ss_gate_up), _ptr(ss_down), 1 if act_fp8 else 0, n_sel, _ptr(sel), _ptr(out),
-        _ptr(sel_idx), _ptr(sel_gate))
+        _ptr(sel_idx), _ptr(sel_gate), HIDDEN_ROUND[hidden_round], _ptr(out_h))
     del keep
     if rc != 0:
         raise ValueError("oracle.forward: a selected token routes to an expert "
@@ -259,4 +275,6 @@ def forward(x, Wr, W_gate_up, W_down, Ws_gate_up, Ws_down, *, bias=None,
     if k > 1:
         sel_idx = sel_idx.reshape(n_sel, k)
         sel_gate = sel_gate.reshape(n_sel, k)
+    if hidden_round:
+        return out, sel_idx, sel_gate, out_h
     return out, sel_idx, sel_gate

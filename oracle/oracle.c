@@ -166,6 +166,48 @@ static double load_weight(const void *W, int dtype, const float *col_scale,
     return w;
 }
 
+/* Hidden-row rounding of the reading where the GPU keeps the hidden rows in
+ * a 16-bit type: the fp64 value is first rounded to fp32 (the GPU forms h in
+ * fp32), then to bf16 or IEEE binary16 by round-to-nearest-even. */
+enum { HROUND_NONE = 0, HROUND_BF16 = 1, HROUND_F16 = 2 };
+
+/* fp32 -> bf16 (8-bit significand), round to nearest even: add half of the
+ * dropped 16 bits' weight plus the kept lsb, then truncate (the carry moves
+ * into the exponent when the significand overflows, as it should). */
+static double round_bf16(double v) {
+    float f = (float)v;
+    uint32_t u;
+    memcpy(&u, &f, sizeof u);
+    if ((u & 0x7F800000u) == 0x7F800000u) return (double)f; /* inf / NaN */
+    u += 0x7FFFu + ((u >> 16) & 1u);
+    u &= 0xFFFF0000u;
+    memcpy(&f, &u, sizeof f);
+    return (double)f;
+}
+
+/* fp32 -> binary16 (11-bit significand, exponents -14..15, subnormals in
+ * steps of 2^-24, largest finite 65504), round to nearest even; values that
+ * round beyond 65504 become infinite. */
+static double round_f16(double v) {
+    double a = fabs((double)(float)v), q;
+    if (a != a || a == INFINITY) return (double)(float)v;
+    if (a < ldexp(1.0, -14)) {
+        q = ldexp(rint(ldexp(a, 24)), -24);           /* subnormal grid */
+    } else {
+        int e2;
+        frexp(a, &e2);                                /* a in [2^(e2-1), 2^e2) */
+        q = ldexp(rint(ldexp(a, 11 - e2)), e2 - 11);  /* 11 significant bits */
+        if (q > 65504.0) q = INFINITY;
+    }
+    return v < 0 ? -q : q;
+}
+
+static double round_hidden(double v, int h_round) {
+    return h_round == HROUND_BF16 ? round_bf16(v) : h_round == HROUND_F16 ? round_f16(v) : v;
+}
+
+double oracle_round_hidden(double v, int h_round) { return round_hidden(v, h_round); }
+
 static double sigmoid(double z) { return 1.0 / (1.0 + exp(-z)); }
 static double silu(double z) { return z / (1.0 + exp(-z)); }
 
@@ -238,11 +280,14 @@ static void route_token_topk(int d, int E, int k, const void *x_t, int x_dtype,
 }
 
 /* One SwiGLU FFN on one input row u[d]:
- *   a = u . Wgu  (2Fw values), h_j = silu(a_j) * a_{Fw+j},  y += h . Wd.  */
+ *   a = u . Wgu  (2Fw values), h_j = silu(a_j) * a_{Fw+j},  y += h . Wd.
+ * yh (optional): the same down projection with each h_j rounded as h_round
+ * says, added into yh. */
 static void swiglu_ffn_accumulate(int d, int Fw, const double *u,
                                   const void *Wgu, const void *Wd, int w_dtype,
                                   const float *s_gu, const float *s_d, int act_fp8,
-                                  double *a, double *h, double *y) {
+                                  double *a, double *h, double *y,
+                                  int h_round, double *yh) {
     size_t two_f = 2 * (size_t)Fw;
     for (size_t j = 0; j < two_f; ++j) a[j] = 0.0;
     for (int k = 0; k < d; ++k) {
@@ -256,6 +301,12 @@ static void swiglu_ffn_accumulate(int d, int Fw, const double *u,
         double hj = h[j];
         for (int n = 0; n < d; ++n)
             y[n] += hj * load_weight(Wd, w_dtype, s_d, (size_t)j, (size_t)d, (size_t)n);
+    }
+    if (!yh) return;
+    for (int j = 0; j < Fw; ++j) {
+        double hj = round_hidden(h[j], h_round);
+        for (int n = 0; n < d; ++n)
+            yh[n] += hj * load_weight(Wd, w_dtype, s_d, (size_t)j, (size_t)d, (size_t)n);
     }
 }
 
@@ -313,7 +364,7 @@ int oracle_forward(int T, int d, int E, int k, int F, int Fs,
                    const float *const *s_gate_up, const float *const *s_down,
                    const float *ss_gate_up, const float *ss_down, int act_fp8,
                    int n_sel, const int32_t *sel, double *out,
-                   int32_t *sel_idx, double *sel_gate) {
+                   int32_t *sel_idx, double *sel_gate, int h_round, double *out_h) {
     size_t xs = (x_dtype == ORACLE_F32) ? 4 : 2;
     int missing = 0;
     (void)T;
@@ -326,7 +377,9 @@ int oracle_forward(int T, int d, int E, int k, int F, int Fs,
         double *a = (double *)malloc(sizeof(double) * 2 * (size_t)Fmax);
         double *h = (double *)malloc(sizeof(double) * (size_t)Fmax);
         double *y = out + (size_t)i * (size_t)d;
+        double *yh = out_h ? out_h + (size_t)i * (size_t)d : NULL;
         for (int n = 0; n < d; ++n) y[n] = 0.0;
+        for (int n = 0; yh && n < d; ++n) yh[n] = 0.0;
         /* shared expert on the ungated input (with E == 0 the whole layer:
          * the dense SwiGLU feed-forward of the layers without experts) */
         for (int k = 0; k < d; ++k) u[k] = load_elem(x_t, x_dtype, (size_t)k);
@@ -334,7 +387,7 @@ int oracle_forward(int T, int d, int E, int k, int F, int Fs,
         double *xq = (double *)malloc(sizeof(double) * (size_t)d);
         for (int k = 0; k < d; ++k) xq[k] = u[k];
         swiglu_ffn_accumulate(d, Fs, u, Ws_gate_up, Ws_down, w_dtype,
-                              ss_gate_up, ss_down, act_fp8, a, h, y);
+                              ss_gate_up, ss_down, act_fp8, a, h, y, h_round, yh);
         if (E == 0) {
             if (sel_idx) sel_idx[i] = -1;
             if (sel_gate) sel_gate[i] = 0.0;
@@ -364,7 +417,7 @@ int oracle_forward(int T, int d, int E, int k, int F, int Fs,
             for (int kk = 0; kk < d; ++kk) u[kk] = g * xq[kk];
             swiglu_ffn_accumulate(d, F, u, W_gate_up[e], W_down[e], w_dtype,
                                   s_gate_up ? s_gate_up[e] : NULL,
-                                  s_down ? s_down[e] : NULL, act_fp8, a, h, y);
+                                  s_down ? s_down[e] : NULL, act_fp8, a, h, y, h_round, yh);
         }
         free(u);
         free(xq);

@@ -201,13 +201,17 @@ class L4MoE:
 
     def _weights(self, W_gate_up, W_down, Ws_gate_up, Ws_down):
         """Pointer arrays of the expert weights; shapes, dtypes, devices and
-        contiguity are checked whenever the weights' addresses change.  The
-        key is the plain address list (the per-call cost with 128 experts is
-        ~20 us of Python, against ~60 us when every call re-checked every
-        tensor)."""
+        contiguity are checked whenever the weight tensors change.  The key is
+        each tensor's identity and address: a view of a checked weight (a
+        transpose, a slice, a reinterpreting .view) is another tensor object,
+        so it is checked again even at the same address, and the checked
+        tensors are held (self._wkeep) so that their identities cannot be
+        reused by new tensors while the key stands.  (The per-call cost with
+        128 experts is ~20 us of Python, against ~60 us when every call
+        re-checked every tensor.)"""
         try:
-            key = ([w.data_ptr() for w in W_gate_up], [w.data_ptr() for w in W_down],
-                   Ws_gate_up.data_ptr(), Ws_down.data_ptr())
+            ws = list(W_gate_up) + list(W_down) + [Ws_gate_up, Ws_down]
+            key = (tuple(id(w) for w in ws), tuple(w.data_ptr() for w in ws))
         except AttributeError:  # a missing weight: the checks below name it
             key = None
         if key is None or getattr(self, "_wkey", None) != key:
@@ -222,8 +226,10 @@ class L4MoE:
                 _expect(t, name, shape, wdt)
             for t, name, _ in named:
                 _where(t, name)
-            self._wkey = key
+            self._wkey = None
             self._warr = (_ptr_array(W_gate_up), _ptr_array(W_down))
+            self._wkeep = ws
+            self._wkey = key
         return self._warr
 
     def _check_io(self, x, W_router, out, host=False):

@@ -200,11 +200,17 @@ struct l4moe_handle {
     const float* ss_dn = nullptr;
     const float** d_scales = nullptr;  // device [2][E+1] scale pointers (gate/up, down)
     bool scales_dirty = false;
+    // host copy of that table, the source of every upload: sized once at
+    // creation and rewritten in place by l4moe_set_weight_scales, so its
+    // address stays fixed for the handle's life (a copy recorded under stream
+    // capture reads it again at every replay)
+    std::vector<const float*> scale_tab;
     // TMA descriptors of the weights, keyed by pointer value
     std::vector<const void*> key_gu, key_dn;
     const void* key_sgu = nullptr;
     const void* key_sdn = nullptr;
-    std::vector<CUtensorMap> h_maps;  // [2][E+1]: gate/up set then down set
+    std::vector<CUtensorMap> h_maps;  // [2][E+1]: gate/up set then down set; capacity
+                                      // reserved at creation, so its address is fixed
     std::vector<const void*> hkey_gu, hkey_dn;  // weights h_maps was encoded for
     const void* hkey_sgu = nullptr;
     const void* hkey_sdn = nullptr;
@@ -690,20 +696,17 @@ l4moe_status run_layer(l4moe_handle* h, int T, const void* x, const void* Wr, co
     return L4MOE_OK;
 }
 
-// Device table of the per-column scale vectors of the 8-bit weights:
-// [gate/up of experts 0..E-1, shared gate/up, down of experts 0..E-1, shared down].
-// The column-scale pointers of 8-bit weights in the kernels' order: gate/up of experts
-// 0..E-1, the shared gate/up, then the same for down.
-std::vector<const float*> scale_table(const l4moe_handle* h) {
+// The column-scale pointers of 8-bit weights in the kernels' order: gate/up of
+// experts 0..E-1, the shared gate/up, then the same for down.  Rewritten in
+// place (the table never moves).
+void fill_scale_table(l4moe_handle* h) {
     const int E = h->p.num_experts;
-    std::vector<const float*> tab(2 * (E + 1));
     for (int e = 0; e < E; ++e) {
-        tab[e] = h->s_gu[e];
-        tab[E + 1 + e] = h->s_dn[e];
+        h->scale_tab[e] = h->s_gu[e];
+        h->scale_tab[E + 1 + e] = h->s_dn[e];
     }
-    tab[E] = h->ss_gu;
-    tab[2 * E + 1] = h->ss_dn;
-    return tab;
+    h->scale_tab[E] = h->ss_gu;
+    h->scale_tab[2 * E + 1] = h->ss_dn;
 }
 
 l4moe_status ensure_scales(l4moe_handle* h, cudaStream_t st) {
@@ -714,9 +717,7 @@ l4moe_status ensure_scales(l4moe_handle* h, cudaStream_t st) {
         h->scales_dirty = true;
     }
     if (!h->scales_dirty) return L4MOE_OK;
-    const std::vector<const float*> tab = scale_table(h);
-    // pageable source: staged before the call returns
-    cudaError_t e = cudaMemcpyAsync(h->d_scales, tab.data(), sizeof(float*) * tab.size(),
+    cudaError_t e = cudaMemcpyAsync(h->d_scales, h->scale_tab.data(), sizeof(float*) * h->scale_tab.size(),
                                     cudaMemcpyHostToDevice, st);
     if (e != cudaSuccess) return cuda_fail(h, e, "scale table upload");
     h->scales_dirty = false;
@@ -832,9 +833,8 @@ l4moe_status l4moe_forward_static(l4moe_handle* h, int T, const void* x, const v
     if (e != cudaSuccess) return cuda_fail(h, e, "static error word clear");
     const float* const* scales = nullptr;
     if (fp8) {  // the scale-pointer table of 8-bit weights follows the descriptors
-        const std::vector<const float*> tab = scale_table(h);
         scales = reinterpret_cast<const float* const*>(base + ws_bytes + maps_bytes);
-        e = cudaMemcpyAsync(const_cast<const float**>(scales), tab.data(), scales_bytes,
+        e = cudaMemcpyAsync(const_cast<const float**>(scales), h->scale_tab.data(), scales_bytes,
                             cudaMemcpyHostToDevice, st);
         if (e != cudaSuccess) return cuda_fail(h, e, "static scale table upload");
     }
@@ -896,6 +896,8 @@ l4moe_status l4moe_create(const l4moe_params* params, l4moe_handle** out) {
     h->p = p;
     h->device = dev;
     h->sms = sms;
+    h->h_maps.reserve(2 * (size_t)(p.num_experts + 1));
+    h->scale_tab.assign(2 * (size_t)(p.num_experts + 1), nullptr);
     *out = h;
     return L4MOE_OK;
 }
@@ -985,6 +987,7 @@ l4moe_status l4moe_set_weight_scales(l4moe_handle* h, const float* const* s_gate
     h->s_dn.assign(s_down, s_down + (E > 0 ? E : 0));
     h->ss_gu = ss_gate_up;
     h->ss_dn = ss_down;
+    fill_scale_table(h);
     h->scales_dirty = true;
     return L4MOE_OK;
 }

@@ -82,3 +82,28 @@ def test_weight_arrays_are_cached_by_address_and_rechecked_on_change(monkeypatch
         layer._weights([gu[0], torch.zeros(d, F, dtype=torch.bfloat16), gu[2]], dn, sgu, sdn)
     with pytest.raises(ValueError, match="contiguous"):
         layer._weights([gu[0], torch.zeros(2 * F, d, dtype=torch.bfloat16).t(), gu[2]], dn, sgu, sdn)
+
+
+def test_a_view_at_a_checked_address_is_checked_again(monkeypatch):
+    """A transpose, a slice or a reinterpreting view of a checked weight
+    shares its address but is another tensor: the cache must not let it
+    through unchecked."""
+    from sparse_moe_transformer_router_b200 import binding
+    monkeypatch.setattr(binding, "_where", lambda t, name, host=False: None)  # host tensors stand in
+    layer = _layer(d=64, F=48, Fs=32)
+    d, F, Fs, E = 64, 48, 32, 3
+    gu = [torch.zeros(d, 2 * F, dtype=torch.bfloat16) for _ in range(E)]
+    dn = [torch.zeros(F, d, dtype=torch.bfloat16) for _ in range(E)]
+    sgu, sdn = torch.zeros(d, 2 * Fs, dtype=torch.bfloat16), torch.zeros(Fs, d, dtype=torch.bfloat16)
+    layer._weights(gu, dn, sgu, sdn)
+    with pytest.raises(ValueError, match=r"W_gate_up\[0\] has shape"):
+        layer._weights([gu[0].t()] + gu[1:], dn, sgu, sdn)          # same address, transposed
+    with pytest.raises(ValueError, match=r"W_down\[0\] has shape"):
+        layer._weights(gu, [dn[0][: F // 2]] + dn[1:], sgu, sdn)      # same address, fewer rows
+    with pytest.raises(ValueError, match=r"W_gate_up\[1\] has dtype"):
+        layer._weights([gu[0], gu[1].view(torch.float16)] + gu[2:], dn, sgu, sdn)
+    with pytest.raises(ValueError, match="Ws_down has shape"):
+        layer._weights(gu, dn, sgu, sdn.view(d, Fs))                  # same bytes, reshaped
+    # the original tensors are accepted again (and held by the layer)
+    layer._weights(gu, dn, sgu, sdn)
+    assert layer._wkeep[0] is gu[0]

@@ -63,3 +63,19 @@ def test_reference_arm_under_torchrun_prints_one_line_from_rank_zero():
     assert line["impl"] == "reference" and line["n_gpus"] == 2
     assert line["cpu_baseline"]["kind"] == "oracle" and line["value"] > 0
     assert line["e2e"]["h2d_bytes_per_step"] == 0
+
+
+def test_gpus_flag_without_a_launcher_starts_that_many_ranks():
+    """`bench.py --gpus 2` run directly (no torchrun) relaunches itself as two
+    ranks; the reference arm's line then reports both."""
+    cmd = [sys.executable, os.path.join(ROOT, "bench.py"), "--gpus", "2", "--impl", "reference",
+           "--workload", "tiny_f32", "--steps", "1", "--warmup", "3"]
+    env = {k: v for k, v in os.environ.items() if k not in ("WORLD_SIZE", "RANK", "LOCAL_RANK")}
+    env["OMP_NUM_THREADS"] = "2"
+    p = subprocess.run(cmd, capture_output=True, text=True, timeout=300, cwd=ROOT, env=env)
+    assert p.returncode == 0, p.stderr[-2000:]
+    lines = [l for l in p.stdout.splitlines() if l.startswith("{")]
+    assert len(lines) == 1
+    line = json.loads(lines[0])
+    assert line["n_gpus"] == 2 and line["impl"] == "reference"
+    assert line["config"]["parallelism"] == "replicas2"

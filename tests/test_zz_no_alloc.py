@@ -7,24 +7,22 @@ reserved up front).  It runs the same kernels as l4moe_forward but keeps its
 workspace in the library's fixed device array.  This file runs last so that a
 run stopping at the first failure has already run every other test.
 """
-import numpy as np
 import pytest
 import torch
 
-from parity_util import OUT_UNIT_ROUNDOFF, TOL, make_layer
+from parity_util import make_layer
 from sparse_moe_transformer_router_b200.binding import ERR_WORKSPACE, L4MoEError
 from sparse_moe_transformer_router_b200.workloads import LayerConfig, generate
 
 pytestmark = pytest.mark.gpu
 
 
-def _assert_close(out: torch.Tensor, ref: torch.Tensor, dtype: str):
-    o = out.double().cpu().numpy()
-    r = ref.double().cpu().numpy()
-    assert np.all(np.isfinite(o))
-    rms = float(np.sqrt(np.mean(r ** 2)))
-    bound = TOL[dtype] * rms + OUT_UNIT_ROUNDOFF[dtype] * np.abs(r)
-    assert np.all(np.abs(o - r) <= bound)
+def _assert_same(out: torch.Tensor, ref: torch.Tensor):
+    """The two entry points run the same deterministic kernels on the same
+    inputs (only the workspace's address differs), so the outputs are equal
+    bit for bit."""
+    assert torch.isfinite(out.float()).all()
+    assert torch.equal(out, ref)
 
 
 @pytest.mark.parametrize("dtype", ["bf16", "f32", "fp8", "int8"])
@@ -39,7 +37,7 @@ def test_static_forward_matches_allocating_forward_on_two_calls(dtype):
         out = torch.full_like(ref, float("nan"))
         layer.forward_static(*args, out)
         torch.cuda.synchronize()
-        _assert_close(out, ref, dtype)
+        _assert_same(out, ref)
 
 
 def test_static_forward_rejects_batches_beyond_its_array():
@@ -55,10 +53,12 @@ def test_static_forward_rejects_batches_beyond_its_array():
     assert "static" in str(ei.value)
 
 
-def test_static_forward_replays_inside_a_cuda_graph():
+@pytest.mark.parametrize("dtype", ["bf16", "fp8", "int8"])
+def test_static_forward_replays_inside_a_cuda_graph(dtype):
     """The use it exists for: record the layer once under stream capture,
-    replay it, including after the input values change in place."""
-    cfg = LayerConfig("noalloc_graph", 200, 256, 8, 384, 256, "bf16", wr_std=0.1)
+    replay it, including after the input values change in place.  The 8-bit
+    layers' replays also re-read the handle's scale-pointer table."""
+    cfg = LayerConfig(f"noalloc_graph_{dtype}", 200, 256, 8, 384, 256, dtype, wr_std=0.1)
     inp = generate(cfg, seed=13, device="cuda")
     layer = make_layer(inp)
     args = (inp.x, inp.W_router, inp.W_gate_up, inp.W_down, inp.Ws_gate_up, inp.Ws_down)
@@ -74,4 +74,5 @@ def test_static_forward_replays_inside_a_cuda_graph():
         out.fill_(float("nan"))
         graph.replay()
         torch.cuda.synchronize()
-        _assert_close(out, ref, "bf16")
+        _assert_same(out, ref)
+    del graph
