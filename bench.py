@@ -315,6 +315,8 @@ def main():
                     help="override E (smaller profiling captures)")
     ap.add_argument("--impl", default="b200", choices=["b200", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-workloads", action="store_true",
+                    help="measure only --workload (skip the other shapes measured after it)")
     ap.add_argument("--e2e-steps", type=int, default=0)
     args = ap.parse_args()
     args.warmup = max(args.warmup, 3)
@@ -346,35 +348,72 @@ def main():
     run_b200(args, rank, world, local)
 
 
-def run_b200(args, rank, world, local):
+# Datasheet figures (NVIDIA B200: dense bf16 tensor throughput, HBM3e
+# bandwidth), reported next to the fractions of the measured peaks.
+DATASHEET = {"bf16_tflops": 2250.0, "hbm_gbs": 8000.0}
+
+# Workloads measured after the headline in the same run, each with its own
+# timed region, roofline and clocks: the other shapes the layer is quoted on.
+EXTRA_WORKLOADS = ("maverick_prefill_bf16", "maverick_decode_bf16@T1", "maverick_decode_bf16@T8",
+                   "maverick_decode_bf16@T32", "maverick_decode_bf16@T128", "maverick_fp8",
+                   "maverick_int8", "maverick_dense_bf16", "tiny_f32")
+
+
+def workload_config(name: str):
+    base, _, t = name.partition("@T")
+    cfg = CONFIGS[base]
+    return cfg.with_tokens(int(t)) if t else cfg
+
+
+def make_layer(cfg, rank):
     from sparse_moe_transformer_router_b200.binding import L4MoE
-    torch.cuda.set_device(local)
-    cfg = CONFIGS[args.workload]
     inp = generate(cfg, seed=rank, device="cuda")
     layer = L4MoE(cfg.d_model, cfg.expert_ffn, cfg.shared_ffn, cfg.num_experts, cfg.dtype)
     if inp.bias is not None:
         layer.set_router_bias(inp.bias)
     if cfg.dtype in ("fp8", "int8"):
         layer.set_weight_scales(inp.s_gate_up, inp.s_down, inp.ss_gate_up, inp.ss_down)
+    return inp, layer
+
+
+def roofline_of(flops: float, nbytes: float, seconds: float, tensor_peak: float, hbm: float,
+                tensor_sheet: float, hbm_sheet: float) -> dict:
+    """The binding roof of work (flops, bytes) done in `seconds`: achieved
+    rate and fraction of the measured peak and of the datasheet figure."""
+    t_tensor = flops / (tensor_peak * 1e12) if flops else 0.0
+    t_hbm = nbytes / (hbm * 1e9)
+    if t_tensor >= t_hbm:
+        achieved = flops / seconds / 1e12
+        return {"bound": "tensor", "achieved": achieved, "peak": tensor_peak, "unit": "TFLOP/s",
+                "frac": achieved / tensor_peak, "datasheet_peak": tensor_sheet,
+                "frac_of_datasheet": achieved / tensor_sheet}
+    achieved = nbytes / seconds / 1e9
+    return {"bound": "hbm", "achieved": achieved, "peak": hbm, "unit": "GB/s", "frac": achieved / hbm,
+            "datasheet_peak": hbm_sheet, "frac_of_datasheet": achieved / hbm_sheet}
+
+
+def measure(cfg, inp, layer, steps: int, warmup: int, world: int, local: int) -> dict:
+    """Device-timed forwards of one workload: warm-up, a per-kernel
+    breakdown pass, then `steps` forwards between two events on the
+    launching stream (barrier + synchronize on both sides, max over ranks),
+    with the dominant kernel's own events inside that region and nvidia-smi
+    clock samples during it.  Returns the measurement and roofline fields."""
     out = torch.empty((cfg.T, cfg.d_model), dtype=inp.x.dtype, device="cuda")
     fwd = lambda: layer.forward(inp.x, inp.W_router, inp.W_gate_up, inp.W_down,  # noqa: E731
                                 inp.Ws_gate_up, inp.Ws_down, out=out)
     stream = torch.cuda.current_stream()
-    barrier = lambda: rank_barrier(world)  # noqa: E731
-    max_over_ranks = lambda v: rank_max(v, world, "cuda")  # noqa: E731
-
-    for _ in range(args.warmup):
+    for _ in range(warmup):
         fwd()
     torch.cuda.synchronize()
     layer.check_device_status()
-    counts = layer.routing()["counts"].cpu().numpy()
+    counts = layer.routing()["counts"].cpu().numpy() if cfg.num_experts > 0 else np.zeros(0)
     layer.read_timing()  # drop anything recorded so far
 
-    # per-kernel breakdown (a short pass of its own, every kernel timed):
-    # it names the dominant kernel, the only one timed inside the timed
-    # region, where every event pair would add to the step
+    # per-kernel breakdown (a short pass of its own, every kernel timed): it
+    # names the dominant kernel, the only one timed inside the timed region,
+    # where every event pair would add to the step
     layer.set_timing(True)
-    n_break = max(3, min(20, args.steps // 5))
+    n_break = max(3, min(20, steps // 5))
     for _ in range(n_break):
         fwd()
     torch.cuda.synchronize()
@@ -382,67 +421,31 @@ def run_b200(args, rank, world, local):
     breakdown = layer.read_timing()
     dom = max((k for k in breakdown if breakdown[k][1]), key=lambda k: breakdown[k][0])
 
-    # ---------------------------------------------------------------- timed
     sampler = ClockSampler(local)
     sampler.start()
     layer.set_timing([dom])
     launches0 = layer.launch_count
-    barrier()
+    rank_barrier(world)
     torch.cuda.synchronize()
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     e0.record(stream)
-    for _ in range(args.steps):
+    for _ in range(steps):
         fwd()
     e1.record(stream)
     torch.cuda.synchronize()
-    barrier()
+    rank_barrier(world)
+    clocks = sampler.stop()
     layer.set_timing(False)
     launches = layer.launch_count - launches0
-    t_ms = max_over_ranks(e0.elapsed_time(e1))
+    t_ms = rank_max(e0.elapsed_time(e1), world, "cuda")
     ktimes = layer.read_timing()
     layer.check_device_status()
+    ms_step = t_ms / steps
 
-    ms_step = t_ms / args.steps
-    value = replica_throughput(world, cfg.T, args.steps, t_ms)
-
-    # ------------------------------------------------------------- e2e (host buffers)
-    x_host = inp.x.cpu().pin_memory()
-    out_host = torch.empty_like(x_host).pin_memory()
-    e2e_steps = args.e2e_steps or args.steps  # same length as the device-timed region
-    fwd_h = lambda: layer.forward_host(x_host, inp.W_router, inp.W_gate_up, inp.W_down,  # noqa: E731
-                                       inp.Ws_gate_up, inp.Ws_down, out_host)
-    for _ in range(2):
-        fwd_h()
-    torch.cuda.synchronize()
-    barrier()
-    h0, h1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    h0.record(stream)
-    for _ in range(e2e_steps):
-        fwd_h()
-    layer.join_host(stream)  # the end event waits for the last output copy
-    h1.record(stream)
-    torch.cuda.synchronize()
-    barrier()
-    th_ms = max_over_ranks(h0.elapsed_time(h1))
-    clocks = sampler.stop()  # samples span the device-timed and the end-to-end regions
-    layer.check_device_status()
-    io_bytes = cfg.T * cfg.d_model * inp.x.element_size()
-    e2e = {"value": replica_throughput(world, cfg.T, e2e_steps, th_ms), "unit": "tokens/s",
-           "h2d_bytes_per_step": io_bytes, "d2h_bytes_per_step": io_bytes,
-           "ms_per_step": th_ms / e2e_steps,
-           "path": "l4moe_forward_host per step: pinned host x -> device (copy-in stream), layer "
-                   "(caller stream), device -> pinned host out (copy-out stream); consecutive "
-                   "steps overlap their copies with each other's compute; the timed region "
-                   "ends after the last output copy"}
-
-    if rank != 0:
-        if world > 1:
-            import torch.distributed as dist
-            dist.destroy_process_group()
-        return
-
-    # ---------------------------------------------------------------- roofline
     peaks, peak_src = load_peaks()
+    long_region = t_ms > 1000.0
+    tensor_peak = peaks.get("bf16_tflops_sustained" if long_region else "bf16_tflops")
+    hbm = peaks["hbm_gbs"]
     kfb = kernel_flops_bytes(cfg, counts)
     per_kernel = {}
     for name, (ms, n) in breakdown.items():
@@ -455,51 +458,137 @@ def run_b200(args, rank, world, local):
     for v in per_kernel.values():
         v["share"] = v["avg_us"] / tot if tot else None
     dom_ms, dom_n = ktimes[dom]
-    long_region = t_ms > 1000.0
-    tensor_peak = peaks.get("bf16_tflops_sustained" if long_region else "bf16_tflops")
-    hbm = peaks["hbm_gbs"]
     f, b = kfb[dom]["flops"], kfb[dom]["bytes"]
-    t_tensor = f / (tensor_peak * 1e12) if f else 0.0
-    t_hbm = b / (hbm * 1e9)
-    bound = "tensor" if t_tensor >= t_hbm else "hbm"
     avg_s = dom_ms / dom_n / 1e3  # the dominant kernel's events inside the timed region
-    if bound == "tensor":
-        achieved, peak, unit = f / avg_s / 1e12, tensor_peak, "TFLOP/s"
-    else:
-        achieved, peak, unit = b / avg_s / 1e9, hbm, "GB/s"
-    traffic = profile_traffic(dom, cfg.name)
-    roofline = {"kernel": dom, "bound": bound, "achieved": achieved, "peak": peak, "unit": unit,
-                "frac": achieved / peak, "traffic": traffic,
-                "peak_source": f"{peak_src} ({'sustained' if (bound == 'tensor' and long_region) else 'burst'})"
-                if bound == "tensor" else f"{peak_src} hbm_gbs",
-                "algorithmic_per_launch": {"flops": f, "bytes": b},
-                "avg_us_timed_region": avg_s * 1e6, "launches_timed": dom_n}
+    roof = roofline_of(f, b, avg_s, tensor_peak, hbm, DATASHEET["bf16_tflops"], DATASHEET["hbm_gbs"])
+    roof = {"kernel": dom, **roof, "traffic": profile_traffic(dom, cfg.name),
+            "peak_source": (f"{peak_src} ({'sustained' if long_region else 'burst'})"
+                            if roof["bound"] == "tensor" else f"{peak_src} hbm_gbs"),
+            "algorithmic_per_launch": {"flops": f, "bytes": b},
+            "avg_us_timed_region": avg_s * 1e6, "launches_timed": dom_n}
     # whole layer against its own roof
+    touched = accounting.experts_touched(counts)
     flops = accounting.layer_flops(cfg.T, cfg.d_model, cfg.num_experts, cfg.expert_ffn, cfg.shared_ffn)
     lbytes = accounting.layer_bytes(cfg.T, cfg.d_model, cfg.num_experts, cfg.expert_ffn, cfg.shared_ffn,
-                                    cfg.dtype, accounting.experts_touched(counts))
-    t_roof = max(flops / (tensor_peak * 1e12), lbytes / (hbm * 1e9))
-    layer_roof = {"bound": "tensor" if flops / (tensor_peak * 1e12) >= lbytes / (hbm * 1e9) else "hbm",
-                  "frac": t_roof / (ms_step / 1e3), "tflops_active": flops / (ms_step / 1e3) / 1e12,
+                                    cfg.dtype, touched)
+    lr = roofline_of(flops, lbytes, ms_step / 1e3, tensor_peak, hbm, DATASHEET["bf16_tflops"],
+                     DATASHEET["hbm_gbs"])
+    layer_roof = {"bound": lr["bound"], "frac": lr["frac"], "frac_of_datasheet": lr["frac_of_datasheet"],
+                  "tflops_active": flops / (ms_step / 1e3) / 1e12,
                   "gbs_algorithmic": lbytes / (ms_step / 1e3) / 1e9,
                   "flops_per_step": flops, "bytes_per_step": lbytes}
+    return {"ms_per_step": ms_step, "t_ms": t_ms, "steps": steps, "roofline": roof,
+            "layer_roofline": layer_roof, "kernels": per_kernel, "n_break": n_break, "dom": dom,
+            "gpu_launches": launches, "clocks": clocks, "experts_touched": touched}
+
+
+def run_extra_workloads(args, rank, world, local) -> dict:
+    """The other workloads, one after another (each one's inputs freed before
+    the next): tokens/s, ms/step, both rooflines and clocks for each."""
+    res = {}
+    for name in EXTRA_WORKLOADS:
+        cfg = workload_config(name)
+        inp, layer = make_layer(cfg, rank)
+        # a timed region of at least ~200 ms (and at least --steps forwards)
+        out = torch.empty((cfg.T, cfg.d_model), dtype=inp.x.dtype, device="cuda")
+        layer.forward(inp.x, inp.W_router, inp.W_gate_up, inp.W_down, inp.Ws_gate_up, inp.Ws_down, out=out)
+        torch.cuda.synchronize()
+        t0 = time.perf_counter()
+        layer.forward(inp.x, inp.W_router, inp.W_gate_up, inp.W_down, inp.Ws_gate_up, inp.Ws_down, out=out)
+        torch.cuda.synchronize()
+        est_ms = (time.perf_counter() - t0) * 1e3
+        steps = int(max(args.steps, min(400, 200.0 / max(est_ms, 1e-3))))
+        m = measure(cfg, inp, layer, steps, args.warmup, world, local)
+        res[name] = {"tokens_per_s": replica_throughput(world, cfg.T, steps, m["t_ms"]),
+                     "ms_per_step": m["ms_per_step"], "steps": steps, "T": cfg.T,
+                     "experts": cfg.num_experts, "dtype": cfg.dtype, "router": cfg.router,
+                     "layer_roofline": m["layer_roofline"], "roofline": m["roofline"],
+                     "kernels": {k: round(v["avg_us"], 2) for k, v in m["kernels"].items()},
+                     "gpu_launches": m["gpu_launches"], "clocks": m["clocks"],
+                     "experts_touched": m["experts_touched"]}
+        layer.close()
+        del inp, layer, out
+        torch.cuda.empty_cache()
+    return res
+
+
+def run_b200(args, rank, world, local):
+    torch.cuda.set_device(local)
+    cfg = CONFIGS[args.workload]
+    inp, layer = make_layer(cfg, rank)
+    m = measure(cfg, inp, layer, args.steps, args.warmup, world, local)
+    value = replica_throughput(world, cfg.T, args.steps, m["t_ms"])
+
+    # ------------------------------------------------------------- e2e (host buffers)
+    stream = torch.cuda.current_stream()
+    x_host = inp.x.cpu().pin_memory()
+    out_host = torch.empty_like(x_host).pin_memory()
+    e2e_steps = args.e2e_steps or args.steps  # same length as the device-timed region
+    fwd_h = lambda: layer.forward_host(x_host, inp.W_router, inp.W_gate_up, inp.W_down,  # noqa: E731
+                                       inp.Ws_gate_up, inp.Ws_down, out_host)
+    for _ in range(2):
+        fwd_h()
+    torch.cuda.synchronize()
+    rank_barrier(world)
+    sampler = ClockSampler(local)
+    sampler.start()
+    h0, h1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    h0.record(stream)
+    for _ in range(e2e_steps):
+        fwd_h()
+    layer.join_host(stream)  # the end event waits for the last output copy
+    h1.record(stream)
+    torch.cuda.synchronize()
+    rank_barrier(world)
+    e2e_clocks = sampler.stop()
+    th_ms = rank_max(h0.elapsed_time(h1), world, "cuda")
+    layer.check_device_status()
+    io_bytes = cfg.T * cfg.d_model * inp.x.element_size()
+    e2e = {"value": replica_throughput(world, cfg.T, e2e_steps, th_ms), "unit": "tokens/s",
+           "h2d_bytes_per_step": io_bytes, "d2h_bytes_per_step": io_bytes,
+           "ms_per_step": th_ms / e2e_steps, "clocks": e2e_clocks,
+           "path": "l4moe_forward_host per step: pinned host x -> device (copy-in stream), layer "
+                   "(caller stream), device -> pinned host out (copy-out stream); consecutive "
+                   "steps overlap their copies with each other's compute; the timed region "
+                   "ends after the last output copy"}
+
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        cpu = cpu_baseline(inp)
+    layer.close()
+    del inp, layer
+    torch.cuda.empty_cache()
+    extra = {} if args.no_workloads else run_extra_workloads(args, rank, world, local)
+
+    if rank != 0:
+        if world > 1:
+            import torch.distributed as dist
+            dist.destroy_process_group()
+        return
 
     line = {"metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world, "steps": args.steps,
-            "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True, "scaling": "weak",
-            "vs_baseline": None, "dtype": "bf16" if cfg.dtype != "f32" else "f32",
+            "warmup": args.warmup, "ms_per_step": m["ms_per_step"], "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "bf16" if cfg.dtype != "f32" else "f32",
             "data": "synthetic (seeded N(0,1) inputs, N(0,0.02) weights, random-init)",
-            "config": config_dict(cfg, world), "roofline": roofline, "layer_roofline": layer_roof,
-            "kernels": per_kernel,
-            "kernels_note": f"every kernel event-timed over {n_break} steps after the warm-up; only "
-                            f"the dominant kernel ({dom}) is timed inside the timed region",
-            "e2e": e2e, "gpu_launches": launches, "clocks": clocks,
-            "experts_touched": accounting.experts_touched(counts)}
+            "config": config_dict(cfg, world), "roofline": m["roofline"],
+            "layer_roofline": m["layer_roofline"], "kernels": m["kernels"],
+            "kernels_note": f"every kernel event-timed over {m['n_break']} steps after the warm-up; only "
+                            f"the dominant kernel ({m['dom']}) is timed inside the timed region",
+            "e2e": e2e, "gpu_launches": m["gpu_launches"], "clocks": m["clocks"],
+            "experts_touched": m["experts_touched"],
+            "peaks_note": "frac: of the measured peak (peak_source); frac_of_datasheet: of NVIDIA's "
+                          "dense bf16 2250 TFLOP/s or HBM3e 8000 GB/s"}
     if cfg.dtype in ("fp8", "int8"):
         wname = "E4M3" if cfg.dtype == "fp8" else "int8"
         line["dtype"] = f"f16 ({wname} weights widened exactly to f16, fp32 accumulate; bf16 in and out)"
-    if world == 1 and not args.no_cpu_baseline:
-        line["cpu_baseline"] = cpu_baseline(inp)
+    if cpu is not None:
+        line["cpu_baseline"] = cpu
+    if extra:
+        line["workloads"] = extra
     print(json.dumps(line), flush=True)
+    if world > 1:
+        import torch.distributed as dist
+        dist.destroy_process_group()
 
 
 if __name__ == "__main__":

@@ -199,7 +199,7 @@ __global__ void __launch_bounds__(1024) permute_kernel(const float* __restrict__
             running[x] = acc;
         }
         __syncthreads();
-        if (e >= 0) inv[t] = wcnt[warp * E + e] + lane_rank;  // rank inside expert
+        if (t < Tv) inv[t] = e >= 0 ? wcnt[warp * E + e] + lane_rank : -1;  // rank inside expert
         __syncthreads();
     }
     // exclusive scan of the counts (warp 0, up to 8 experts per lane)
@@ -289,6 +289,7 @@ __global__ void __launch_bounds__(256) permute_rows_kernel(const IT* __restrict_
     for (int n = (blockIdx.x * blockDim.x + threadIdx.x) >> 5; n < T * k; n += warps) {
         const int t = n / k;
         const int slot = inv ? inv[n] : n;
+        if (slot < 0 || slot >= T * k) continue;  // an entry the permutation rejected (bad expert index)
         if (lane == 0 && gate_slot) gate_slot[slot] = gate[n];
         const uint4* s = reinterpret_cast<const uint4*>(x + (size_t)t * d);
         uint4* o = reinterpret_cast<uint4*>(xp + (size_t)slot * d);

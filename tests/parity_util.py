@@ -6,14 +6,23 @@ Acceptance (the layer's stated tolerances):
     margin is >= 1e-4 (closer tokens are excluded and counted);
   * per-expert counts equal the histogram of the indices, offsets/perm equal
     the oracle's stable permutation of the CUDA indices (exact);
-  * outputs: per element |out - oracle| <= tol * rms(oracle) + u * |oracle|
-    with tol = 2e-2 (f32 / bf16 weights) or 6e-2 (E4M3 weights) and u the
-    unit roundoff of the output type (2^-8 for bf16, 2^-24 for f32).  The
-    u * |oracle| term is the rounding of the exact result to the output type
-    itself: a correctly rounded bf16 copy of the fp64 oracle already reaches
-    1-2% of rms(oracle) at the tails of these layers, so a bound of
-    tol * rms alone would fail even for exact arithmetic.  The plain
-    max|err| / rms(oracle) is reported alongside.
+  * outputs, two assertions (check_outputs):
+    - the reading check: every output equals the oracle's exact evaluation
+      of the stated roundings (hidden rows rounded to the activation type,
+      bf16 -- f16 for 8-bit weight layers -- everything else exact) to
+      within the output's own rounding and a small allowance for fp32
+      accumulation order: |out - ref_h| <= halfulp(out) + READING_SLACK *
+      rms(oracle).  (fp32 layers multiply in TF32, which the oracle does not
+      model: they take the plain bound below only.)
+    - the stated bound max|out - oracle| <= tol * rms(oracle), tol = 2e-2
+      (fp32, bf16) or 6e-2 (E4M3, int8 weights), asserted wherever every
+      exact implementation of those roundings meets it: where the largest
+      error such an implementation can make,
+          max over elements of (halfulp(ref_h) + |ref_h - oracle|) / rms,
+      plus READING_SLACK, is within tol.  Elsewhere the bound is out of
+      reach of exact arithmetic itself (the bf16 rounding of the output
+      alone can exceed 2e-2 * rms at the tails of small layers) and only the
+      reading check applies; the plain max|err| / rms is reported either way.
 """
 from __future__ import annotations
 
@@ -26,7 +35,29 @@ from sparse_moe_transformer_router_b200.workloads import LayerInputs, to_storage
 
 MARGIN_EXCLUDE = 1e-4
 TOL = {"f32": 2e-2, "bf16": 2e-2, "fp8": 6e-2, "int8": 6e-2}
-OUT_UNIT_ROUNDOFF = {"f32": 2.0 ** -24, "bf16": 2.0 ** -8, "fp8": 2.0 ** -8, "int8": 2.0 ** -8}
+# the type the GPU holds the hidden rows in (None: fp32 layers, TF32 products)
+HIDDEN = {"f32": None, "bf16": "bf16", "fp8": "f16", "int8": "f16"}
+# allowance, in units of rms(oracle), for fp32 accumulation order and for the
+# rare hidden values whose fp32 value sits at a 16-bit rounding midpoint
+READING_SLACK = 2e-3
+
+
+def halfulp_bf16(v: np.ndarray) -> np.ndarray:
+    """Half the spacing of bf16 numbers (8-bit significand) in the binade of
+    each |v|: the largest rounding error a value that rounds to v can have
+    had (for v a power of two, the larger spacing above it).  Zero for 0."""
+    a = np.abs(np.asarray(v, dtype=np.float64))
+    e = np.floor(np.log2(np.where(a > 0, a, 1.0)))
+    return np.where(a > 0, np.exp2(e - 8), 0.0)
+
+
+def round_out(v: np.ndarray, dtype: str) -> np.ndarray:
+    """v rounded to the layer's output type (through fp32, as the GPU forms
+    the output in fp32): a library conversion, not the oracle's."""
+    f = torch.from_numpy(np.asarray(v, dtype=np.float64).astype(np.float32))
+    if dtype == "f32":
+        return f.double().numpy()
+    return f.to(torch.bfloat16).double().numpy()
 
 
 def make_layer(inp: LayerInputs) -> L4MoE:
@@ -117,64 +148,132 @@ def check_routing_topk(inp: LayerInputs, r: dict, k: int) -> dict:
             "counts": counts, "same": same, "o_idx": o_idx}
 
 
+def oracle_outputs(inp: LayerInputs, tokens: np.ndarray, o_idx=None, k: int = 1,
+                   chunk_experts: int = 16):
+    """The oracle's exact outputs and its evaluation of the stated roundings
+    (None for fp32 layers) for `tokens`, in that order.  With the oracle's
+    routing `o_idx` (top-1 layers), the tokens are evaluated in groups of at
+    most `chunk_experts` experts, so that only those experts' weights are
+    held on the host at a time (a full-size sample can touch all of them)."""
+    c = inp.cfg
+    hidden = HIDDEN[c.dtype]
+    x = to_storage_numpy(inp.x)
+    Wr = to_storage_numpy(inp.W_router)
+    b = None if inp.bias is None else inp.bias.detach().cpu().numpy()
+    Ws_gu, Ws_dn = to_storage_numpy(inp.Ws_gate_up), to_storage_numpy(inp.Ws_down)
+    E = c.num_experts
+    if o_idx is None or k > 1 or E == 0:
+        groups = [(tokens, set(range(E)) if o_idx is None else
+                   set(int(e) for e in np.asarray(o_idx)[tokens].ravel()))]
+    else:
+        te = np.asarray(o_idx)[tokens]
+        experts = sorted(set(int(e) for e in te))
+        groups = []
+        for i in range(0, len(experts), chunk_experts):
+            chunk = set(experts[i:i + chunk_experts])
+            groups.append((tokens[np.isin(te, list(chunk))], chunk))
+    ref = np.zeros((tokens.size, c.d_model))
+    ref_h = np.zeros_like(ref) if hidden else None
+    pos = {int(t): i for i, t in enumerate(tokens)}
+    for toks, need in groups:
+        Wgu = [to_storage_numpy(inp.W_gate_up[e]) if e in need else None for e in range(E)]
+        Wdn = [to_storage_numpy(inp.W_down[e]) if e in need else None for e in range(E)]
+        kw = {}
+        if c.dtype in ("fp8", "int8"):
+            kw = dict(s_gate_up=[inp.s_gate_up[e].cpu().numpy() if e in need else None for e in range(E)],
+                      s_down=[inp.s_down[e].cpu().numpy() if e in need else None for e in range(E)],
+                      ss_gate_up=inp.ss_gate_up.cpu().numpy(), ss_down=inp.ss_down.cpu().numpy())
+        res = oracle.forward(x, Wr, Wgu, Wdn, Ws_gu, Ws_dn, bias=b, tokens=toks, k=k,
+                             hidden_round=hidden, **kw)
+        rows = np.array([pos[int(t)] for t in toks], dtype=np.int64)
+        ref[rows] = res[0]
+        if hidden:
+            ref_h[rows] = res[3]
+        del Wgu, Wdn, kw, res
+    return ref, ref_h
+
+
+def judge_outputs(got: np.ndarray, ref: np.ndarray, ref_h, dtype: str, tol: float | None = None) -> dict:
+    """The two output assertions (module docstring) on aligned arrays."""
+    assert np.all(np.isfinite(got)), "non-finite outputs"
+    rms = float(np.sqrt(np.mean(ref ** 2)))
+    err = np.abs(got - ref)
+    tol = TOL[dtype] if tol is None else tol
+    plain = float(np.max(err)) / rms if rms > 0 else float(np.max(err))
+    rep = {"plain": plain, "n_tokens": int(got.shape[0])}
+    if ref_h is None:
+        rep.update(reading=None, floor=None, stated_bound_asserted=True)
+        assert plain <= tol, f"max|err|/rms = {plain:.4g} exceeds tol {tol}"
+        return rep
+    dev = np.abs(got - ref_h) - halfulp_bf16(got)
+    reading = float(np.max(dev)) / rms
+    floor = float(np.max(halfulp_bf16(ref_h) + np.abs(ref_h - ref))) / rms
+    asserted = floor + READING_SLACK <= tol
+    rep.update(reading=reading, floor=floor, stated_bound_asserted=bool(asserted))
+    assert reading <= READING_SLACK, (
+        f"output off the oracle's evaluation of the stated roundings by {reading:.3g} * rms beyond "
+        f"its own rounding (allowed {READING_SLACK}); max|err|/rms = {plain:.4g}")
+    if asserted:
+        assert plain <= tol, f"max|err|/rms = {plain:.4g} exceeds tol {tol} (floor {floor:.4g})"
+    return rep
+
+
 def check_outputs(inp: LayerInputs, out: torch.Tensor, tokens, same_mask=None, o_idx=None,
-                  tol: float | None = None, k: int = 1) -> float:
+                  tol: float | None = None, k: int = 1) -> dict:
     """Oracle outputs for `tokens` (None = all) against the CUDA output rows.
     Tokens whose routing flipped on a near-tie are skipped.  Asserts the
-    per-element bound (tol defaults to the dtype's); returns
-    max|err| / rms(oracle)."""
-    c = inp.cfg
-    T = c.T
+    reading check and, where every exact implementation of the stated
+    roundings meets it, the stated bound (see the module docstring).
+    Returns {"plain": max|err| / rms, "reading": max over elements of
+    (|out - ref_h| - halfulp(out)) / rms, "floor": the largest error an exact
+    implementation could make / rms, "stated_bound_asserted": bool,
+    "n_tokens": tokens compared}."""
+    T = inp.cfg.T
     if tokens is None:
         tokens = np.arange(T, dtype=np.int32)
     tokens = np.asarray(tokens, dtype=np.int32)
     if same_mask is not None:
         tokens = tokens[same_mask[tokens]]
-    need = set(range(c.num_experts)) if o_idx is None else set(int(e) for e in np.asarray(o_idx)[tokens].ravel())
-    x = to_storage_numpy(inp.x)
-    Wr = to_storage_numpy(inp.W_router)
-    b = None if inp.bias is None else inp.bias.detach().cpu().numpy()
-    Wgu = [to_storage_numpy(inp.W_gate_up[e]) if e in need else None for e in range(c.num_experts)]
-    Wdn = [to_storage_numpy(inp.W_down[e]) if e in need else None for e in range(c.num_experts)]
-    kw = {}
-    if c.dtype in ("fp8", "int8"):
-        kw = dict(s_gate_up=[inp.s_gate_up[e].cpu().numpy() if e in need else None for e in range(c.num_experts)],
-                  s_down=[inp.s_down[e].cpu().numpy() if e in need else None for e in range(c.num_experts)],
-                  ss_gate_up=inp.ss_gate_up.cpu().numpy(), ss_down=inp.ss_down.cpu().numpy())
-    ref, _, _ = oracle.forward(x, Wr, Wgu, Wdn, to_storage_numpy(inp.Ws_gate_up),
-                               to_storage_numpy(inp.Ws_down), bias=b, tokens=tokens, k=k, **kw)
+    ref, ref_h = oracle_outputs(inp, tokens, o_idx, k)
     got = out[torch.as_tensor(tokens, device=out.device, dtype=torch.long)].float().cpu().numpy().astype(np.float64)
-    rms = float(np.sqrt(np.mean(ref ** 2)))
-    err = np.abs(got - ref)
-    tol = TOL[c.dtype] if tol is None else tol
-    bound = tol * rms + OUT_UNIT_ROUNDOFF[c.dtype] * np.abs(ref)
-    worst = float(np.max(err / bound))
-    ratio = float(np.max(err)) / rms if rms > 0 else float(np.max(err))
-    assert worst <= 1.0, (f"|err| exceeds tol*rms + u*|ref| by {worst:.3f}x "
-                          f"(max|err|/rms = {ratio:.4g}, tol {tol})")
-    return ratio
+    return judge_outputs(got, ref, ref_h, inp.cfg.dtype, tol)
 
 
-def sample_tokens(r: dict, rep: dict, T: int, seed: int = 0, per_expert: int = 4, n_experts: int = 5):
-    """Tokens to check at full size: from the most and least loaded non-empty
-    experts plus random ones, the first and last slot of each (the ragged tail
-    of its last token tile), a slot at a 256-token tile boundary and a random
-    slot; plus tokens 0 and T-1."""
+def describe(rep: dict) -> str:
+    """One line of a check_outputs report for the test log."""
+    s = f"max|err|/rms = {rep['plain']:.3e} over {rep['n_tokens']} tokens"
+    if rep.get("reading") is not None:
+        s += (f", beyond own rounding {rep['reading']:.2e}, floor {rep['floor']:.3e}, stated bound "
+              f"{'asserted' if rep['stated_bound_asserted'] else 'out of reach (floor + slack > tol)'}")
+    return s
+
+
+def sample_tokens(r: dict, rep: dict, T: int, seed: int = 0, n_min: int = 1024, tile: int = 256):
+    """A stratified sample of at least `n_min` tokens (all of them when T is
+    not larger): for every non-empty expert the first and last slot of its
+    rows, the two slots on each side of every `tile`-row token-tile boundary
+    inside them, and random slots in proportion to its rows; for the shared
+    expert (token order) the same at every token-tile boundary; then evenly
+    spaced tokens until `n_min` are reached.  Every GEMM token tile, every
+    band of tiles and every expert is hit."""
+    if T <= n_min:
+        return np.arange(T, dtype=np.int32)
     rng = np.random.default_rng(seed)
-    counts = rep["counts"]
+    counts = np.asarray(rep["counts"])
     offs = np.concatenate([[0], np.cumsum(counts)])
     perm = r["perm"].cpu().numpy()
-    nonempty = np.nonzero(counts)[0]
-    order = nonempty[np.argsort(-counts[nonempty], kind="stable")]
-    chosen = list(dict.fromkeys([int(order[0]), int(order[-1])] +
-                                [int(e) for e in rng.choice(nonempty, size=min(len(nonempty), n_experts), replace=False)]))
-    chosen = chosen[:n_experts]
     toks = {0, T - 1}
-    for e in chosen:
+    for j in range(tile, T, tile):            # shared expert's tile boundaries
+        toks.update((j - 1, j))
+    slots = set()
+    for e in np.nonzero(counts)[0]:
         lo, hi = int(offs[e]), int(offs[e + 1])
-        slots = {lo, hi - 1, int(rng.integers(lo, hi))}
-        if hi - lo > 256:
-            slots.add(lo + 256)
-        for s in list(slots)[:per_expert]:
-            toks.add(int(perm[s]))
+        slots.update((lo, hi - 1))
+        for j in range(lo + tile, hi, tile):
+            slots.update((j - 1, j))
+        n_rand = max(1, (n_min // 2) * (hi - lo) // max(1, int(counts.sum())))
+        slots.update(int(v) for v in rng.integers(lo, hi, size=n_rand))
+    toks.update(int(perm[s_]) for s_ in slots)
+    if len(toks) < n_min:
+        toks.update(int(v) for v in np.linspace(0, T - 1, n_min - len(toks) + 2).astype(np.int64))
     return np.array(sorted(toks), dtype=np.int32)

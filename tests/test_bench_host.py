@@ -78,3 +78,24 @@ def test_cpu_baseline_times_the_oracle_on_a_bounded_sample():
     cb = bench.cpu_baseline(inp, budget_s=0.5)
     assert cb["kind"] == "oracle" and cb["unit"] == "tokens/s" and cb["value"] > 0
     assert cb["cores"] >= 1 and "of the 64 tokens" in cb["sample"]
+
+
+def test_roofline_reports_measured_and_datasheet_fractions():
+    # 1 TFLOP and 1 GB in 1 ms: tensor-bound at 1000 TFLOP/s against a 1600
+    # measured / 2250 datasheet peak; HBM-bound when the bytes dominate
+    r = bench.roofline_of(1e12, 1e9, 1e-3, 1600.0, 6500.0, 2250.0, 8000.0)
+    assert r["bound"] == "tensor" and r["achieved"] == pytest.approx(1000.0)
+    assert r["frac"] == pytest.approx(1000.0 / 1600.0)
+    assert r["frac_of_datasheet"] == pytest.approx(1000.0 / 2250.0)
+    r = bench.roofline_of(1e9, 5e9, 1e-3, 1600.0, 6500.0, 2250.0, 8000.0)
+    assert r["bound"] == "hbm" and r["achieved"] == pytest.approx(5000.0)
+    assert r["frac"] == pytest.approx(5000.0 / 6500.0)
+    assert r["frac_of_datasheet"] == pytest.approx(5000.0 / 8000.0)
+
+
+def test_extra_workloads_name_known_shapes():
+    for name in bench.EXTRA_WORKLOADS:
+        cfg = bench.workload_config(name)
+        assert cfg.T > 0 and cfg.d_model > 0
+    assert bench.workload_config("maverick_decode_bf16@T8").T == 8
+    assert bench.DEFAULT_WORKLOAD not in bench.EXTRA_WORKLOADS
