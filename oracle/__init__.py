@@ -11,9 +11,10 @@ Inputs are numpy arrays in their storage dtype: float32, bf16 as uint16 bit
 patterns, E4M3 as uint8 codes, int8 weights as int8, int4 weights as packed
 bytes viewed with ``INT4X2``.
 
-Every function is pinned by ``tests/test_oracle_pins.py`` to something other
-than itself (library matmuls on reductions of the layer, closed forms,
-invariants, numpy's argmax / stable argsort, torch's bf16 and float8 decoders).
+Every function is pinned by ``tests/test_oracle_pins.py`` and
+``tests/test_tolerance_floor.py`` to something other than itself (library
+matmuls on reductions of the layer, closed forms, invariants, numpy's argmax /
+stable argsort, torch's bf16 and float8 decoders and conversions).
 """
 from __future__ import annotations
 
@@ -81,6 +82,8 @@ def _load():
                                            vp, vp, vp, vp, i32,
                                            vp, vp, vp, vp, i32,
                                            i32, vp, vp, vp, vp, i32, vp]
+            lib.oracle_expert_rows.restype = None
+            lib.oracle_expert_rows.argtypes = [i32, i32, i32, vp, i32, vp, vp, vp, i32, vp, vp, vp]
             lib.oracle_round_hidden.restype = ctypes.c_double
             lib.oracle_round_hidden.argtypes = [ctypes.c_double, i32]
             lib.oracle_e4m3_encode.restype = ctypes.c_uint8
@@ -178,6 +181,29 @@ def permutation(idx: np.ndarray, E: int):
     _load().oracle_permutation(T, E, _ptr(idx), _ptr(counts), _ptr(offsets),
                                _ptr(perm))
     return counts, offsets, perm
+
+
+def expert_rows(x_rows, gates, W_gate_up, W_down, *, s_gate_up=None, s_down=None):
+    """One expert's SwiGLU on given rows: out[i] = SwiGLU(g[i] * x[i]) in
+    fp64 ([n, d]), the routed part of the layer for each (token, expert)
+    entry that expert receives."""
+    x_rows = np.ascontiguousarray(x_rows)
+    n, d = x_rows.shape
+    g = np.ascontiguousarray(gates, dtype=np.float64)
+    assert g.shape == (n,)
+    Wgu = np.ascontiguousarray(W_gate_up)
+    Wdn = np.ascontiguousarray(W_down)
+    F = Wdn.shape[0]
+    w_code = _dtype_code(Wgu)
+    sgu = sdn = None
+    if w_code in (E4M3, INT8, INT4):
+        sgu = np.ascontiguousarray(s_gate_up, dtype=np.float32)
+        sdn = np.ascontiguousarray(s_down, dtype=np.float32)
+    out = np.zeros((n, d), np.float64)
+    if n:
+        _load().oracle_expert_rows(n, d, F, _ptr(x_rows), _dtype_code(x_rows), _ptr(g), _ptr(Wgu), _ptr(Wdn),
+                                   w_code, _ptr(sgu), _ptr(sdn), _ptr(out))
+    return out
 
 
 HIDDEN_ROUND = {None: 0, "bf16": 1, "f16": 2}

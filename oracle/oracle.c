@@ -64,7 +64,10 @@
  * the bf16 layer on the same integers, int4 codes the int8 layer on the same
  * integers; top-k selection equals a lexsort of the logits, and with k = E
  * the layer equals a library evaluation over every expert; without experts
- * the layer is one library SwiGLU.
+ * the layer is one library SwiGLU; the hidden-rounding output equals a
+ * library evaluation that rounds the hidden values with torch's own
+ * conversions; one expert's rows (oracle_expert_rows) equal a library
+ * SwiGLU of the gated rows.
  */
 #include <math.h>
 #include <stdint.h>
@@ -425,6 +428,32 @@ int oracle_forward(int T, int d, int E, int k, int F, int Fs,
         free(h);
     }
     return missing ? -1 : 0;
+}
+
+/* One expert's SwiGLU on n given rows: out[i] = SwiGLU_W(g[i] * x[i]) for
+ * rows x[i] of width d (storage dtype x_dtype) with their gates g[i] -- the
+ * routed part of the layer for each (token, expert) entry, as an expert
+ * holding W_gate_up [d, 2F] / W_down [F, d] (and, for 8-bit or int4
+ * weights, their column scales) computes it.  out is [n, d] fp64. */
+void oracle_expert_rows(int n, int d, int F, const void *x, int x_dtype, const double *g,
+                        const void *W_gate_up, const void *W_down, int w_dtype,
+                        const float *s_gate_up, const float *s_down, double *out) {
+    size_t xs = (x_dtype == ORACLE_F32) ? 4 : 2;
+#pragma omp parallel for schedule(dynamic, 1)
+    for (int i = 0; i < n; ++i) {
+        const char *x_i = (const char *)x + (size_t)i * (size_t)d * xs;
+        double *u = (double *)malloc(sizeof(double) * (size_t)d);
+        double *a = (double *)malloc(sizeof(double) * 2 * (size_t)F);
+        double *h = (double *)malloc(sizeof(double) * (size_t)F);
+        double *y = out + (size_t)i * (size_t)d;
+        for (int k = 0; k < d; ++k) u[k] = g[i] * load_elem(x_i, x_dtype, (size_t)k);
+        for (int k = 0; k < d; ++k) y[k] = 0.0;
+        swiglu_ffn_accumulate(d, F, u, W_gate_up, W_down, w_dtype, s_gate_up, s_down, 0, a, h, y,
+                              HROUND_NONE, NULL);
+        free(u);
+        free(a);
+        free(h);
+    }
 }
 
 int oracle_num_threads(void) {

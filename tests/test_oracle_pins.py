@@ -519,3 +519,31 @@ def test_fp8_activation_mode_keeps_rows_already_in_e4m3():
 
     ref = ffn(x, Wsgu64, Wsd64) + ffn(x, Wgu64, Wd64)
     assert np.max(np.abs(out - ref)) <= 1e-12 * np.sqrt(np.mean(ref ** 2))
+
+
+def test_expert_rows_equals_a_library_swiglu_on_gated_rows():
+    """oracle.expert_rows (one expert on given rows, the routed part of each
+    (token, expert) entry) against torch fp64: SwiGLU(g * x), bf16 and E4M3
+    weights (the latter dequantised per output column)."""
+    import torch
+    rng = np.random.default_rng(11)
+    n, d, F = 7, 64, 48
+    x = torch.from_numpy(rng.standard_normal((n, d)).astype(np.float32)).bfloat16()
+    g = rng.uniform(0.1, 1.0, size=n)
+    Wgu = torch.from_numpy((rng.standard_normal((d, 2 * F)) * 0.1).astype(np.float32)).bfloat16()
+    Wd = torch.from_numpy((rng.standard_normal((F, d)) * 0.1).astype(np.float32)).bfloat16()
+    bits = lambda t: t.view(torch.int16).numpy().view(np.uint16)  # noqa: E731
+    y = oracle.expert_rows(bits(x), g, bits(Wgu), bits(Wd))
+    a = (x.double() * torch.from_numpy(g)[:, None]) @ Wgu.double()
+    lib = (torch.nn.functional.silu(a[:, :F]) * a[:, F:]) @ Wd.double()
+    np.testing.assert_allclose(y, lib.numpy(), rtol=1e-12, atol=1e-13)
+    # E4M3 weights with column scales
+    q_gu = torch.from_numpy(rng.integers(0, 0x7F, size=(d, 2 * F), dtype=np.uint8)).view(torch.float8_e4m3fn)
+    q_d = torch.from_numpy(rng.integers(0, 0x7F, size=(F, d), dtype=np.uint8)).view(torch.float8_e4m3fn)
+    s_gu = rng.uniform(0.001, 0.01, size=2 * F).astype(np.float32)
+    s_d = rng.uniform(0.001, 0.01, size=d).astype(np.float32)
+    y8 = oracle.expert_rows(bits(x), g, q_gu.view(torch.uint8).numpy(), q_d.view(torch.uint8).numpy(),
+                            s_gate_up=s_gu, s_down=s_d)
+    a8 = (x.double() * torch.from_numpy(g)[:, None]) @ (q_gu.double() * torch.from_numpy(s_gu).double())
+    lib8 = (torch.nn.functional.silu(a8[:, :F]) * a8[:, F:]) @ (q_d.double() * torch.from_numpy(s_d).double())
+    np.testing.assert_allclose(y8, lib8.numpy(), rtol=1e-12, atol=1e-13)
