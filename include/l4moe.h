@@ -40,8 +40,13 @@
  *                   output column (l4moe_set_weight_scales); x, W_router, out bf16.
  *                   The expert contractions run in f16 (kind::f16 MMA, fp32
  *                   accumulate): weights widened exactly, x and the hidden
- *                   rows held in f16 (exact for bf16 values of magnitude in
- *                   [2^-14, 65504]), the column scale applied in fp32.
+ *                   rows held in f16, the column scale applied in fp32.  Each
+ *                   token row of x is divided by a power of two that brings
+ *                   its largest value within f16's 65504 (1 for rows already
+ *                   inside), which the fp32 accumulators get back, so every
+ *                   bf16 value of magnitude >= 2^-14 times that scale is
+ *                   exact; a hidden value that f16 cannot hold (|h| >= 65520)
+ *                   sets L4MOE_ERR_RANGE in the device status.
  *   L4MOE_INT8      expert and shared weights int8 (two's complement, symmetric:
  *                   no zero point) with one fp32 scale per output column, the
  *                   weight-only int8 of KerasFormers "Llama 4", "Lower memory";
@@ -90,7 +95,8 @@ typedef enum {
     L4MOE_ERR_CUDA = 4,         /* a CUDA runtime or driver call failed        */
     L4MOE_ERR_WORKSPACE = 5,    /* workspace too small / allocation failed     */
     L4MOE_ERR_TIMEOUT = 6,      /* a kernel's bounded wait ran out             */
-    L4MOE_ERR_UNSUPPORTED = 7   /* device is not sm_100 or feature unavailable */
+    L4MOE_ERR_UNSUPPORTED = 7,  /* device is not sm_100 or feature unavailable */
+    L4MOE_ERR_RANGE = 8         /* E4M3 / int8 layers: a hidden value left f16's range */
 } l4moe_status;
 
 typedef enum {
@@ -251,8 +257,21 @@ L4MOE_API l4moe_status l4moe_get_routing(const l4moe_handle *h, const int32_t **
 
 /* Synchronise `stream` (and the handle's copy-out stream) and read the device
  * error word of the handle's workspace: L4MOE_OK, L4MOE_ERR_TIMEOUT (a
- * bounded wait ran out) or L4MOE_ERR_CUDA.  Clears the word. */
+ * bounded wait ran out), L4MOE_ERR_RANGE (an E4M3 / int8 layer met a hidden
+ * value beyond f16's range: that forward's output is not valid), L4MOE_ERR_ARG
+ * (an expert index out of range reached the permutation) or L4MOE_ERR_CUDA.
+ * Clears the word. */
 L4MOE_API l4moe_status l4moe_check_device_status(l4moe_handle *h, void *stream);
+
+/* Self-test of the device failure path (no counterpart in the pages): enqueue
+ * on `stream` one small kernel that waits, with a limit of limit_ms
+ * milliseconds (0 < limit_ms <= 1000), for an mbarrier phase that nothing
+ * completes.  The wait gives up as every bounded wait of the layer's kernels
+ * does -- it records a timeout bit in the handle's device error word and the
+ * kernel returns -- so the next l4moe_check_device_status returns
+ * L4MOE_ERR_TIMEOUT and clears the word.  Nothing faults or hangs; the
+ * context stays usable.  Allocates the handle's workspace if it has none. */
+L4MOE_API l4moe_status l4moe_selftest_wait(l4moe_handle *h, double limit_ms, void *stream);
 
 /* Per-kernel timing.  `mask` selects kernel slots (bit i = slot i; 0 turns
  * timing off; L4MOE_TIME_ALL every slot; anything else: L4MOE_ERR_ARG).

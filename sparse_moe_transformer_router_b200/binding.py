@@ -14,7 +14,7 @@ import torch
 _PKG = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(_PKG, "libl4moe.so")
 
-OK, ERR_ARG, ERR_DTYPE, ERR_ALIGN, ERR_CUDA, ERR_WORKSPACE, ERR_TIMEOUT, ERR_UNSUPPORTED = range(8)
+OK, ERR_ARG, ERR_DTYPE, ERR_ALIGN, ERR_CUDA, ERR_WORKSPACE, ERR_TIMEOUT, ERR_UNSUPPORTED, ERR_RANGE = range(9)
 DTYPES = {"f32": 0, "bf16": 1, "fp8": 2, "int8": 3}
 EXPORTED = ("l4moe_create", "l4moe_destroy", "l4moe_workspace_size", "l4moe_set_workspace",
             "l4moe_set_router_bias", "l4moe_set_fp8_scales", "l4moe_forward",
@@ -22,7 +22,7 @@ EXPORTED = ("l4moe_create", "l4moe_destroy", "l4moe_workspace_size", "l4moe_set_
             "l4moe_launch_count", "l4moe_last_error", "l4moe_status_string", "l4moe_version",
             "l4moe_set_timing", "l4moe_read_timing", "l4moe_kernel_name",
             "l4moe_forward_static", "l4moe_join_host", "l4moe_set_top_k",
-            "l4moe_set_weight_scales")
+            "l4moe_set_weight_scales", "l4moe_selftest_wait")
 STATIC_WORKSPACE_BYTES = 32 << 20
 NUM_KERNELS = 5
 
@@ -77,6 +77,7 @@ def load_library():
     lib.l4moe_version.argtypes = []
     lib.l4moe_set_timing.argtypes = [vp, i32]
     lib.l4moe_set_top_k.argtypes = [vp, i32]
+    lib.l4moe_selftest_wait.argtypes = [vp, ctypes.c_double, vp]
     lib.l4moe_read_timing.argtypes = [vp, ctypes.POINTER(ctypes.c_double),
                                       ctypes.POINTER(ctypes.c_uint64)]
     lib.l4moe_kernel_name.argtypes = [i32]
@@ -85,7 +86,7 @@ def load_library():
                  "l4moe_set_fp8_scales", "l4moe_forward", "l4moe_forward_host",
                  "l4moe_get_routing", "l4moe_check_device_status", "l4moe_version",
                  "l4moe_set_timing", "l4moe_read_timing", "l4moe_forward_static",
-                 "l4moe_join_host", "l4moe_set_top_k", "l4moe_set_weight_scales"):
+                 "l4moe_join_host", "l4moe_set_top_k", "l4moe_set_weight_scales", "l4moe_selftest_wait"):
         getattr(lib, name).restype = ctypes.c_int
     _lib = lib
     return lib
@@ -309,6 +310,11 @@ class L4MoE:
         for (name, shape, ts), p in zip(spec, ptrs):
             out[name] = torch.as_tensor(_DevView(p.value, shape, ts), device=self.device)
         return out
+
+    def selftest_wait(self, limit_ms: float = 5.0, stream=None):
+        """l4moe_selftest_wait: a device wait that runs out after limit_ms; the
+        next check_device_status raises with ERR_TIMEOUT."""
+        self._check(self._lib.l4moe_selftest_wait(self._h, float(limit_ms), _stream_handle(stream)))
 
     def check_device_status(self, stream=None):
         self._check(self._lib.l4moe_check_device_status(self._h, _stream_handle(stream)))

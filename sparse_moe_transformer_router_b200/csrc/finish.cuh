@@ -5,6 +5,7 @@
 #include <cuda_bf16.h>
 #include <cuda_fp16.h>
 #include <cstdint>
+#include <type_traits>
 
 #include "moe_gemm.cuh"
 #include "ptx.cuh"
@@ -13,12 +14,15 @@ namespace l4moe {
 
 // Split-K finish of the gate/up contraction: h = silu(g * sum_s a_gate) *
 // (g * sum_s a_up) over the splits in order, for the routed slots (g = the
-// slot's sigmoid gate) and the shared rows (g = 1).  One thread per output.
+// slot's sigmoid gate, times its row's power-of-two scale for 8-bit weight
+// layers) and the shared rows (g = 1, or the token's row scale: tokscale).
+// One thread per output.
 template <typename ET>
 __global__ void __launch_bounds__(256) gateup_finish_kernel(
     const float* __restrict__ part_r, long long ld_r, long long stride_r, const float* __restrict__ part_s,
     long long ld_s, long long stride_s, int ksplit, int Tr, int T, int F, int Fs,
-    const float* __restrict__ gslot, ET* __restrict__ hr, ET* __restrict__ hs) {
+    const float* __restrict__ gslot, const float* __restrict__ tokscale, ET* __restrict__ hr,
+    ET* __restrict__ hs, unsigned* err) {
     pdl_enter();
     // Tr routed rows (token entries), T shared rows
     const long long n_r = (long long)Tr * F, n = n_r + (long long)T * Fs;
@@ -35,8 +39,11 @@ __global__ void __launch_bounds__(256) gateup_finish_kernel(
             ag += p[st * s + (long long)row * ld + f];
             au += p[st * s + (long long)row * ld + w + f];
         }
-        const float g = shared ? 1.0f : gslot[row];
-        store_elem((shared ? hs : hr) + (long long)row * w + f, silu_f(g * ag) * (g * au));
+        const float g = shared ? (tokscale ? tokscale[row] : 1.0f) : gslot[row];
+        const float hv = silu_f(g * ag) * (g * au);
+        if (sizeof(ET) == 2 && !std::is_same<ET, __nv_bfloat16>::value && !(fabsf(hv) < 65520.0f))
+            atomicOr(err, DEV_ERR_F16_RANGE);  // f16 hidden rows (8-bit weights): out of range
+        store_elem((shared ? hs : hr) + (long long)row * w + f, hv);
     }
 }
 

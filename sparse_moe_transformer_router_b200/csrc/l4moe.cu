@@ -25,6 +25,7 @@
 #include "finish.cuh"
 #include "moe_gemm.cuh"
 #include "permute.cuh"
+#include "route_small.cuh"
 #include "router.cuh"
 
 using namespace l4moe;
@@ -74,8 +75,8 @@ constexpr int kMaxSplit = 16;
 constexpr int kRouterKSplit = 8;
 
 struct WsLayout {
-    size_t err, idx, gate, lmax, margin, inv, perm, gslot, counts, offsets, tab_gu, tab_dn, xg, hr,
-        hs, x16, part, logits, xin, xout;
+    size_t err, idx, gate, lmax, margin, inv, perm, gslot, counts, offsets, chunk, tab_gu, tab_dn, xg, hr,
+        hs, x16, xsc, part, logits, xin, xout;
     size_t device_total;  // everything l4moe_forward uses
     size_t total;         // plus the host-path staging slots (last)
 };
@@ -155,7 +156,7 @@ WsLayout ws_layout(const l4moe_params& p, int T, int sms, int k) {
     };
     const size_t t = (size_t)std::max(T, 1), E = (size_t)p.num_experts, es = act_bytes(p.dtype);
     const size_t tv = t * (size_t)k;
-    L.err = take(256);
+    L.err = take(256);  // device error word, then the routing kernels' ticket (zeroed once)
     L.idx = take(4 * tv);
     L.gate = take(4 * tv);
     L.lmax = take(4 * tv);
@@ -165,6 +166,7 @@ WsLayout ws_layout(const l4moe_params& p, int T, int sms, int k) {
     L.gslot = take(4 * tv);
     L.counts = take(4 * E);
     L.offsets = take(4 * (E + 1));
+    L.chunk = take(4 * ((tv + kDispatchChunk - 1) / kDispatchChunk) * E);  // dispatch chunk bases
     L.tab_gu = take(sizeof(GroupTable));
     L.tab_dn = take(sizeof(GroupTable));
     L.xg = take(tv * p.d_model * es);
@@ -172,8 +174,13 @@ WsLayout ws_layout(const l4moe_params& p, int T, int sms, int k) {
     L.hs = take(t * p.shared_ffn * es);
     // 8-bit weight layers: x in f16, token order (the shared expert's operand)
     L.x16 = take(coded8(p.dtype) ? t * p.d_model * 2 : 0);
+    L.xsc = take(coded8(p.dtype) ? 4 * t : 0);  // and each token row's power-of-two scale
     L.part = take(sizeof(float) * part_floats(p, (int)t, sms, k));
-    L.logits = take(sizeof(float) * std::min<size_t>(t, 128) * E);  // expert-split router
+    // expert-split router logits [min(T, 128)][E]; for batches the one-launch
+    // routing takes, its partial logits [slices][T][E]
+    const size_t small_part = (size_t)((p.d_model + kSmallSliceK - 1) / kSmallSliceK) *
+                              std::min<size_t>(t, kSmallMaxTokens) * E;
+    L.logits = take(sizeof(float) * std::max(std::min<size_t>(t, 128) * E, small_part));
     L.device_total = off;
     L.xin = take(2 * t * p.d_model * es);   // host path: two input staging slots
     L.xout = take(2 * t * p.d_model * es);  // and two output staging slots
@@ -484,6 +491,7 @@ l4moe_status run_layer(l4moe_handle* h, int T, const void* x, const void* Wr, co
     GT* hr = reinterpret_cast<GT*>(w + L.hr);
     GT* hs = reinterpret_cast<GT*>(w + L.hs);
     GT* x16 = reinterpret_cast<GT*>(w + L.x16);
+    float* tokscale = FP8W ? reinterpret_cast<float*>(w + L.xsc) : nullptr;
 
     // per-call activation descriptors (K-major rows of 128 B): the router's
     // x (64-row boxes) and the GEMMs' token operands (full- and small-tile
@@ -540,7 +548,19 @@ l4moe_status run_layer(l4moe_handle* h, int T, const void* x, const void* Wr, co
     // split-K k-ranges when a small batch leaves too few tiles
     const SplitPlan plan = split_plan(p, T, h->sms, h->top_k);
     const int s_gu = plan.s_gu, s_dn = plan.s_dn;
-    if (E > 0) {
+    if (E > 0 && T <= kSmallMaxTokens) {
+        // a few tokens: router, top-k, permutation and row copy in one launch
+        const int slices = (d + kSmallSliceK - 1) / kSmallSliceK;
+        float* part_logits = reinterpret_cast<float*>(w + L.logits);
+        unsigned* ticket = err + 1;  // zero between launches (each last CTA resets it)
+        LaunchTimer t_router(h, 0, st);
+        launch_k(route_small_kernel<ET, GT>, dim3(slices), dim3(kSmallThreads), route_small_smem_bytes(T, E), st,
+                 static_cast<const ET*>(x), static_cast<const ET*>(Wr), (const float*)h->bias, T, d, E, k,
+                 part_logits, ticket, idx, gate, lmax, margin, counts, offsets, perm, inv, gslot, tab_gu, tab_dn,
+                 fb_gu_r * s_gu, fb_gu_s * s_gu, fb_dn * s_dn, xg, FP8W ? x16 : (GT*)nullptr, tokscale);
+        t_router.stop();
+        L4MOE_CHECK_LAUNCH("small-batch routing launch");
+    } else if (E > 0) {
         LaunchTimer t_router(h, 0, st);
         // one token tile and many experts: split the router over 16-expert chunks
         const bool split_router = sizeof(ET) == 2 && E % 16 == 0 && E >= 32 && T <= 128;
@@ -572,17 +592,27 @@ l4moe_status run_layer(l4moe_handle* h, int T, const void* x, const void* Wr, co
         L4MOE_CHECK_LAUNCH("router launch");
 
         const size_t psmem = sizeof(int) * (34 * (size_t)E + 1);
+        int32_t* chunk_base = nullptr;
         LaunchTimer t_perm(h, 1, st);
-        launch_k(permute_kernel, dim3(1), dim3(1024), psmem, st, (const float*)logits,
-                 gate, lmax, margin, idx, T, k, E, fb_gu_r * s_gu, fb_gu_s * s_gu, fb_dn * s_dn, counts, offsets,
-                 perm, inv, tab_gu, tab_dn, err);
+        if (logits) {
+            // the arg-max of the split logits and the whole permutation in one CTA
+            launch_k(permute_kernel, dim3(1), dim3(1024), psmem, st, (const float*)logits,
+                     gate, lmax, margin, idx, T, k, E, fb_gu_r * s_gu, fb_gu_s * s_gu, fb_dn * s_dn, counts,
+                     offsets, perm, inv, tab_gu, tab_dn, err);
+        } else {
+            chunk_base = reinterpret_cast<int32_t*>(w + L.chunk);
+            launch_k(dispatch_kernel, dim3((Tv + kDispatchChunk - 1) / kDispatchChunk), dim3(kDispatchChunk), psmem,
+                     st, (const int32_t*)idx, T, k, E, fb_gu_r * s_gu, fb_gu_s * s_gu, fb_dn * s_dn, chunk_base,
+                     counts, offsets, inv, tab_gu, tab_dn, err + 1, err);
+        }
         t_perm.stop();
         L4MOE_CHECK_LAUNCH("permute launch");
 
         const int sc_blocks = std::min((Tv + 7) / 8, h->sms * 8);
         LaunchTimer t_rows(h, 2, st);
         launch_k(permute_rows_kernel<ET, GT>, dim3(sc_blocks), dim3(256), 0, st, static_cast<const ET*>(x),
-                 (const float*)gate, (const int32_t*)inv, T, k, d, xg, gslot, FP8W ? x16 : (GT*)nullptr);
+                 (const float*)gate, inv, T, k, d, xg, gslot, FP8W ? x16 : (GT*)nullptr, (const int32_t*)idx,
+                 (const int32_t*)chunk_base, E, perm, tokscale);
         t_rows.stop();
         L4MOE_CHECK_LAUNCH("row permutation launch");
     } else {
@@ -596,7 +626,8 @@ l4moe_status run_layer(l4moe_handle* h, int T, const void* x, const void* Wr, co
             const int sc_blocks = std::min((T + 7) / 8, h->sms * 8);
             LaunchTimer t_rows(h, 2, st);
             launch_k(permute_rows_kernel<ET, GT>, dim3(sc_blocks), dim3(256), 0, st, static_cast<const ET*>(x),
-                     (const float*)nullptr, (const int32_t*)nullptr, T, 1, d, x16, (float*)nullptr, (GT*)nullptr);
+                     (const float*)nullptr, (int32_t*)nullptr, T, 1, d, x16, (float*)nullptr, (GT*)nullptr,
+                     (const int32_t*)nullptr, (const int32_t*)nullptr, 0, (int32_t*)nullptr, tokscale);
             t_rows.stop();
             L4MOE_CHECK_LAUNCH("row conversion launch");
         }
@@ -625,7 +656,8 @@ l4moe_status run_layer(l4moe_handle* h, int T, const void* x, const void* Wr, co
     gu.ld_shared = Fs;
     gu.rowmap_routed = nullptr;
     gu.rowmap_shared = nullptr;  // shared hidden rows in token order
-    gu.colscale_routed = gslot;  // sigmoid gate of each routed slot
+    gu.colscale_routed = gslot;      // sigmoid gate of each routed slot (times its row scale)
+    gu.colscale_shared = tokscale;   // 8-bit weights: each token row's scale, else null
     gu.wscale = FP8W ? scales : nullptr;
     float* part = reinterpret_cast<float*>(w + L.part);
     gu.ksplit = s_gu;
@@ -646,7 +678,7 @@ l4moe_status run_layer(l4moe_handle* h, int T, const void* x, const void* Wr, co
         launch_k(gateup_finish_kernel<GT>, dim3((int)std::min<long long>((n + 255) / 256, 4LL * h->sms)),
                  dim3(256), 0, st, (const float*)gu.part_routed, gu.ld_part_routed, gu.part_stride_routed,
                  (const float*)gu.part_shared, gu.ld_part_shared, gu.part_stride_shared, s_gu, Tv, T, F, Fs,
-                 (const float*)gslot, hr, hs);
+                 (const float*)gslot, (const float*)tokscale, hr, hs, err);
         ++h->launches;
     }
     t_gu.stop();
@@ -667,6 +699,7 @@ l4moe_status run_layer(l4moe_handle* h, int T, const void* x, const void* Wr, co
     dn.rowmap_routed = perm;     // slot -> token: un-permute on store
     dn.rowmap_shared = nullptr;  // shared rows are tokens
     dn.colscale_routed = nullptr;
+    dn.colscale_shared = nullptr;
     dn.wscale = FP8W ? scales + (E + 1) : nullptr;
     dn.ksplit = s_dn;
     dn.partial_out = 1;
@@ -826,10 +859,11 @@ l4moe_status l4moe_forward_static(l4moe_handle* h, int T, const void* x, const v
     cudaStream_t st = static_cast<cudaStream_t>(stream);
     CUtensorMap* maps = reinterpret_cast<CUtensorMap*>(base + ws_bytes);
     // every call shares the array: upload this call's descriptors and clear
-    // the error word (the only state a forward expects to start at zero)
+    // the state a forward expects to start at zero
     cudaError_t e = cudaMemcpyAsync(maps, h->h_maps.data(), maps_bytes, cudaMemcpyHostToDevice, st);
     if (e != cudaSuccess) return cuda_fail(h, e, "static descriptor upload");
-    e = cudaMemsetAsync(base + ws_layout(h->p, T, h->sms, h->top_k).err, 0, sizeof(unsigned), st);
+    // the error word and the routing kernels' ticket that follows it
+    e = cudaMemsetAsync(base + ws_layout(h->p, T, h->sms, h->top_k).err, 0, 2 * sizeof(unsigned), st);
     if (e != cudaSuccess) return cuda_fail(h, e, "static error word clear");
     const float* const* scales = nullptr;
     if (fp8) {  // the scale-pointer table of 8-bit weights follows the descriptors
@@ -866,6 +900,7 @@ const char* l4moe_status_string(l4moe_status s) {
     case L4MOE_ERR_WORKSPACE: return "L4MOE_ERR_WORKSPACE";
     case L4MOE_ERR_TIMEOUT: return "L4MOE_ERR_TIMEOUT";
     case L4MOE_ERR_UNSUPPORTED: return "L4MOE_ERR_UNSUPPORTED";
+    case L4MOE_ERR_RANGE: return "L4MOE_ERR_RANGE";
     }
     return "L4MOE_ERR_UNKNOWN";
 }
@@ -1097,8 +1132,24 @@ l4moe_status l4moe_check_device_status(l4moe_handle* h, void* stream) {
     if (word == 0) return L4MOE_OK;
     cudaMemset(h->ws + ws_layout(h->p, h->ws_tokens, h->sms, h->top_k).err, 0, sizeof(word));
     char msg[160];
-    snprintf(msg, sizeof msg, "device error word 0x%x (1: producer wait, 2: MMA wait, 4: epilogue wait, 8: bad expert index)", word);
-    return fail(h, (word & 7u) ? L4MOE_ERR_TIMEOUT : L4MOE_ERR_ARG, msg);
+    snprintf(msg, sizeof msg,
+             "device error word 0x%x (1: producer wait, 2: MMA wait, 4: epilogue wait, 8: bad expert index, "
+             "16: hidden value beyond f16)", word);
+    return fail(h, (word & 7u) ? L4MOE_ERR_TIMEOUT : (word & 16u) ? L4MOE_ERR_RANGE : L4MOE_ERR_ARG, msg);
+}
+
+l4moe_status l4moe_selftest_wait(l4moe_handle* h, double limit_ms, void* stream) {
+    if (!h) return L4MOE_ERR_ARG;
+    if (!(limit_ms > 0.0 && limit_ms <= 1000.0)) return fail(h, L4MOE_ERR_ARG, "limit_ms must be in (0, 1000]");
+    l4moe_status s;
+    if ((s = ensure_workspace(h, 1)) != L4MOE_OK) return s;
+    const WsLayout L = ws_layout(h->p, h->ws_tokens, h->sms, h->top_k);
+    unsigned* err = reinterpret_cast<unsigned*>(h->ws + L.err);
+    wait_selftest_kernel<<<1, 32, 0, static_cast<cudaStream_t>(stream)>>>(err, (uint64_t)(limit_ms * 1e6));
+    ++h->launches;
+    cudaError_t e = cudaGetLastError();
+    if (e != cudaSuccess) return cuda_fail(h, e, "self-test launch");
+    return L4MOE_OK;
 }
 
 l4moe_status l4moe_set_timing(l4moe_handle* h, int mask) {

@@ -108,7 +108,8 @@ struct GemmArgs {
     long long ld_shared;
     const int32_t* rowmap_routed;  // down: output row (token) of a slot (perm), else null
     const int32_t* rowmap_shared;  // gate/up: slot of a token (inv); down: perm
-    const float* colscale_routed;  // gate/up: sigmoid gate of each slot, else null
+    const float* colscale_routed;  // gate/up: sigmoid gate of each slot (times its row's scale), else null
+    const float* colscale_shared;  // gate/up, 8-bit weights: power-of-two scale of each token's f16 row, else null
     const float* const* wscale;    // E4M3 weights: per-column scale vector of each of the
                                    // E + 1 weight matrices of this launch, else null
     // fp32 partial output (always for down; for gate/up when split): each
@@ -557,7 +558,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(GemmCfg<MODE, ET, WQ
             OT* outp = reinterpret_cast<OT*>(ti.shared ? args.out_shared : args.out_routed);
             const long long ld = ti.shared ? args.ld_shared : args.ld_routed;
             const int32_t* rowmap = ti.shared ? args.rowmap_shared : args.rowmap_routed;
-            const float* colscale = ti.shared ? nullptr : args.colscale_routed;
+            const float* colscale = ti.shared ? args.colscale_shared : args.colscale_routed;
             // E4M3 weights: the scale of this TMEM lane's weight column (lane =
             // row of the A tile: gate/up [gate 64 | up 64] features, down 128)
             float wsc = 1.0f;
@@ -648,8 +649,13 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(GemmCfg<MODE, ET, WQ
                         const float g = __shfl_sync(0xffffffffu, my_scale, col);
                         const float gv = gate_warp ? v[i] : xg[lane * Cfg::XLD + i];
                         const float uv = gate_warp ? xu[lane * Cfg::XLD + i] : v[16 + i];
+                        const float hv = silu_f(g * gv) * (g * uv);
+                        if constexpr (FP8W) {  // hidden rows held in f16: report values beyond its range
+                            if (fvalid && c + col < ti.n_valid && !(fabsf(hv) < 65520.0f))  // rounds to inf
+                                atomicOr(args.err, DEV_ERR_F16_RANGE);
+                        }
                         if (fvalid && c + col < ti.n_valid)
-                            store_elem(outp + (size_t)orow * ld + f, silu_f(g * gv) * (g * uv));
+                            store_elem(outp + (size_t)orow * ld + f, hv);
                     }
                     named_bar_sync(1, 128);  // exchange buffer free for the next chunk
                 } else {

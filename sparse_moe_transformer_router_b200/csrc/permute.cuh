@@ -10,6 +10,7 @@
 #include <cuda_bf16.h>
 #include <cuda_fp16.h>
 #include <cstdint>
+#include <type_traits>
 
 #include "ptx.cuh"
 #include "schedule.cuh"
@@ -252,6 +253,119 @@ __global__ void __launch_bounds__(1024) permute_kernel(const float* __restrict__
     }
 }
 
+// Multi-CTA dispatch of a batch whose routing is already in idx[T * k]: CTA
+// c ranks the kDispatchChunk entries [c * kDispatchChunk, ...) -- a warp's
+// __match_any_sync groups its entries by expert, a prefix over the 32 warps
+// orders the groups -- and writes each entry's rank inside its expert and
+// chunk to inv[n] and the chunk's per-expert counts to chunk_base[c][E].  The
+// last CTA to finish (atomic ticket after a memory fence, no waiting) turns
+// the counts into chunk bases (offsets[e] + entries of e in earlier chunks),
+// writes counts[E], offsets[E + 1] and the two work lists, and resets the
+// ticket.  A slot is then chunk_base[c][e] + inv[n] (permute_rows_kernel):
+// the stable expert order, as the single-CTA permute_kernel gives it.
+// smem: wcnt[32][E] + tot[E] + soff[E + 1] ints.
+constexpr int kDispatchChunk = 1024;
+
+__global__ void __launch_bounds__(kDispatchChunk) dispatch_kernel(
+    const int32_t* __restrict__ idx, int T, int k, int E, int fb_gu_routed, int fb_gu_shared, int fb_down,
+    int32_t* __restrict__ chunk_base, int32_t* __restrict__ counts, int32_t* __restrict__ offsets,
+    int32_t* __restrict__ inv, GroupTable* tab_gu, GroupTable* tab_dn, unsigned* ticket, unsigned* err) {
+    pdl_enter();
+    extern __shared__ int dsm[];
+    int* wcnt = dsm;           // [32][E]
+    int* tot = dsm + 32 * E;   // [E]
+    int* soff = tot + E;       // [E + 1]
+    __shared__ unsigned s_last;
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    const int Tv = T * k;
+    const int chunks = gridDim.x;
+    for (int i = tid; i < 32 * E; i += kDispatchChunk) wcnt[i] = 0;
+    __syncthreads();
+    const int n = blockIdx.x * kDispatchChunk + tid;
+    int e = -1;
+    if (n < Tv) {
+        e = idx[n];
+        if (e < 0 || e >= E) {
+            atomicOr(err, DEV_ERR_BAD_INDEX);
+            e = -1;
+        }
+    }
+    const unsigned same = __match_any_sync(0xffffffffu, e);
+    const int lane_rank = __popc(same & ((1u << lane) - 1u));
+    if (e >= 0 && lane_rank == 0) wcnt[warp * E + e] = __popc(same);
+    __syncthreads();
+    for (int x = tid; x < E; x += kDispatchChunk) {  // prefix over warps, per expert
+        int acc = 0;
+        for (int w = 0; w < 32; ++w) {
+            const int v = wcnt[w * E + x];
+            wcnt[w * E + x] = acc;
+            acc += v;
+        }
+        chunk_base[(size_t)blockIdx.x * E + x] = acc;  // this chunk's count for now
+    }
+    __syncthreads();
+    if (n < Tv) inv[n] = e >= 0 ? wcnt[warp * E + e] + lane_rank : -1;
+
+    __threadfence();
+    __syncthreads();
+    if (tid == 0) s_last = (atomicAdd(ticket, 1u) == (unsigned)chunks - 1u) ? 1u : 0u;
+    __syncthreads();
+    if (!s_last) return;
+    __threadfence();
+    // last CTA: per expert, the entries of earlier chunks, then the totals
+    for (int x = tid; x < E; x += kDispatchChunk) {
+        int acc = 0;
+#pragma unroll 8
+        for (int c = 0; c < chunks; ++c) {
+            const int v = __ldcg(chunk_base + (size_t)c * E + x);
+            chunk_base[(size_t)c * E + x] = acc;
+            acc += v;
+        }
+        tot[x] = acc;
+    }
+    __syncthreads();
+    if (tid == 0) *ticket = 0u;
+    if (warp == 0) {  // exclusive scan of the counts (up to 8 experts per lane)
+        int local[8];
+        int sum = 0;
+#pragma unroll
+        for (int j = 0; j < 8; ++j) {
+            const int x = lane * 8 + j;
+            local[j] = (x < E) ? tot[x] : 0;
+            sum += local[j];
+        }
+        const int incl = warp_incl_scan(sum);
+        int acc = incl - sum;
+#pragma unroll
+        for (int j = 0; j < 8; ++j) {
+            const int x = lane * 8 + j;
+            if (x < E) {
+                soff[x] = acc;
+                offsets[x] = acc;
+                counts[x] = local[j];
+            }
+            acc += local[j];
+        }
+        if (lane == 31) {
+            soff[E] = incl;
+            offsets[E] = incl;
+        }
+    }
+    __syncthreads();
+    for (int i = tid; i < chunks * E; i += kDispatchChunk) chunk_base[i] += soff[i % E];
+    if (warp == 0) {
+        // gate/up: candidate 0 is the shared expert, 1..E the routed experts
+        build_table(
+            tab_gu, E + 1, [&](int g) { return g == 0 ? T : tot[g - 1]; },
+            [&](int g) { return g == 0 ? 0 : soff[g - 1]; }, [&](int g) { return g == 0 ? E : g - 1; },
+            [&](int g) { return g == 0 ? fb_gu_shared : fb_gu_routed; });
+        build_table(
+            tab_dn, E + 1, [&](int g) { return g == 0 ? T : tot[g - 1]; },
+            [&](int g) { return g == 0 ? 0 : soff[g - 1]; }, [&](int g) { return g == 0 ? E : g - 1; },
+            [&](int) { return fb_down; });
+    }
+}
+
 // Expert-ordered copy of the input rows, xp[inv[n]] = x[n / k] for each
 // entry n, and the gate of each slot, gate_slot[inv[n]] = gate[n].  The sigmoid gate scales the
 // routed expert's input, which is linear in the gate/up contraction, so it
@@ -261,26 +375,60 @@ __global__ void __launch_bounds__(1024) permute_kernel(const float* __restrict__
 // x_tok (if not null) also receives the f16 rows in token order.  inv ==
 // null keeps token order (and gate / gate_slot are then unused).
 // One warp per token row, 16-byte vectors; d % 8 == 0.
-__device__ __forceinline__ uint4 cvt_row_vec(uint4 v, __nv_bfloat16, __half) {
+// inv_s: the reciprocal of the row's power-of-two scale (f16_row_scale).
+__device__ __forceinline__ uint4 cvt_row_vec(uint4 v, __nv_bfloat16, __half, float inv_s = 1.0f) {
     uint32_t w[4] = {v.x, v.y, v.z, v.w};
 #pragma unroll
     for (int i = 0; i < 4; ++i) {
         const float2 f = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&w[i]));
-        const __half2 hv = __floats2half2_rn(f.x, f.y);
+        const __half2 hv = __floats2half2_rn(f.x * inv_s, f.y * inv_s);
         w[i] = *reinterpret_cast<const uint32_t*>(&hv);
     }
     return make_uint4(w[0], w[1], w[2], w[3]);
 }
 template <typename T>
-__device__ __forceinline__ uint4 cvt_row_vec(uint4 v, T, T) { return v; }
+__device__ __forceinline__ uint4 cvt_row_vec(uint4 v, T, T, float = 1.0f) { return v; }
 
+// Layers with 8-bit weights hold x in f16 for their contractions.  A row
+// whose largest |x| is beyond f16's largest finite value (65504) is divided
+// by a power of two that brings it inside -- exact, only the exponents
+// change -- and the row's fp32 accumulators are multiplied back by it in the
+// gate/up epilogue (with the sigmoid gate for routed rows).  Rows in range,
+// and rows holding inf or NaN, keep the scale 1.
+__device__ __forceinline__ float f16_row_scale(float amax) {
+    if (!(amax > 65504.0f) || !(amax < INFINITY)) return 1.0f;
+    int e;
+    frexpf(amax / 65504.0f, &e);  // amax / 65504 < 2^e
+    return ldexpf(1.0f, e);
+}
+
+// Largest |x| of 8 bf16 values.
+__device__ __forceinline__ float absmax_vec(uint4 v, float m) {
+    const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+        const float2 f = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&w[i]));
+        m = fmaxf(m, fmaxf(fabsf(f.x), fabsf(f.y)));
+    }
+    return m;
+}
+
+// chunk_base (not null, after dispatch_kernel): inv[n] holds the entry's
+// rank inside its expert and chunk; its slot is chunk_base[chunk][idx[n]] +
+// inv[n], which this kernel writes back to inv[n] and records in perm.
+// tokscale (8-bit weight layers; not null): each token's power-of-two row
+// scale, written once per token; gate_slot then carries gate * scale.
 template <typename IT, typename OT>
 __global__ void __launch_bounds__(256) permute_rows_kernel(const IT* __restrict__ x,
                                                            const float* __restrict__ gate,
-                                                           const int32_t* __restrict__ inv,
+                                                           int32_t* __restrict__ inv,
                                                            int T, int k, int d, OT* __restrict__ xp,
                                                            float* __restrict__ gate_slot,
-                                                           OT* __restrict__ x_tok) {
+                                                           OT* __restrict__ x_tok,
+                                                           const int32_t* __restrict__ idx,
+                                                           const int32_t* __restrict__ chunk_base, int E,
+                                                           int32_t* __restrict__ perm,
+                                                           float* __restrict__ tokscale) {
     pdl_enter();
     static_assert(sizeof(IT) == sizeof(OT), "row copy keeps the element size");
     const int lane = threadIdx.x & 31;
@@ -288,15 +436,36 @@ __global__ void __launch_bounds__(256) permute_rows_kernel(const IT* __restrict_
     // one warp per entry n = t * k + j (token t's j-th expert)
     for (int n = (blockIdx.x * blockDim.x + threadIdx.x) >> 5; n < T * k; n += warps) {
         const int t = n / k;
-        const int slot = inv ? inv[n] : n;
+        int slot = inv ? inv[n] : n;
+        if (chunk_base) {
+            if (lane == 0) {
+                const int e = idx[n];
+                slot = (slot >= 0 && e >= 0 && e < E) ? chunk_base[(size_t)(n / kDispatchChunk) * E + e] + slot : -1;
+                if (slot >= 0 && slot < T * k) {
+                    inv[n] = slot;
+                    perm[slot] = n;
+                }
+            }
+            slot = __shfl_sync(0xffffffffu, slot, 0);
+        }
         if (slot < 0 || slot >= T * k) continue;  // an entry the permutation rejected (bad expert index)
-        if (lane == 0 && gate_slot) gate_slot[slot] = gate[n];
         const uint4* s = reinterpret_cast<const uint4*>(x + (size_t)t * d);
         uint4* o = reinterpret_cast<uint4*>(xp + (size_t)slot * d);
         uint4* ot = (x_tok && n % k == 0) ? reinterpret_cast<uint4*>(x_tok + (size_t)t * d) : nullptr;
         const int nv = d * (int)sizeof(IT) / 16;
+        float sc = 1.0f;  // the row's power-of-two scale (f16 rows of 8-bit weight layers)
+        if constexpr (!std::is_same<IT, OT>::value) {
+            float m = 0.0f;
+            for (int i = lane; i < nv; i += 32) m = absmax_vec(s[i], m);
+#pragma unroll
+            for (int off = 16; off > 0; off >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, off));
+            sc = f16_row_scale(m);
+            if (lane == 0 && tokscale && n % k == 0) tokscale[t] = sc;
+        }
+        if (lane == 0 && gate_slot) gate_slot[slot] = gate[n] * sc;
+        const float inv_s = 1.0f / sc;
         for (int i = lane; i < nv; i += 32) {
-            const uint4 v = cvt_row_vec(s[i], IT{}, OT{});
+            const uint4 v = cvt_row_vec(s[i], IT{}, OT{}, inv_s);
             o[i] = v;
             if (ot) ot[i] = v;
         }

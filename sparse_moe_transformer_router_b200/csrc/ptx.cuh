@@ -13,6 +13,7 @@ enum : unsigned {
     DEV_ERR_TIMEOUT_MMA = 1u << 1,
     DEV_ERR_TIMEOUT_EPILOGUE = 1u << 2,
     DEV_ERR_BAD_INDEX = 1u << 3,
+    DEV_ERR_F16_RANGE = 1u << 4,  // a hidden value of an 8-bit-weight layer beyond f16's range
 };
 
 // Every spin on an mbarrier gives up after this many nanoseconds, records a
@@ -60,18 +61,31 @@ __device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
 }
 
 // Wait for the phase with the given parity to complete.  Returns false (and
-// sets `code` in *err) if it has not completed within kWaitLimitNs.
+// sets `code` in *err) if it has not completed within limit_ns.
 __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, unsigned* err,
-                                          unsigned code) {
+                                          unsigned code, uint64_t limit_ns = kWaitLimitNs) {
     if (mbar_try_wait(bar, parity)) return true;
     const uint64_t t0 = global_timer_ns();
     while (!mbar_try_wait(bar, parity)) {
-        if (global_timer_ns() - t0 > kWaitLimitNs) {
+        if (global_timer_ns() - t0 > limit_ns) {
             atomicOr(err, code);
             return false;
         }
     }
     return true;
+}
+
+// Self-test of the failure path above: one thread initialises an mbarrier
+// that expects one arrival, which never comes, and waits for its first
+// phase with a limit of limit_ns.  The wait gives up, records
+// DEV_ERR_TIMEOUT_PRODUCER in the error word and the kernel returns.
+__global__ void wait_selftest_kernel(unsigned* err, uint64_t limit_ns) {
+    __shared__ __align__(8) uint64_t bar;
+    if (threadIdx.x != 0) return;
+    const uint32_t b = smem_u32(&bar);
+    mbar_init(b, 1);
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+    mbar_wait(b, 0, err, DEV_ERR_TIMEOUT_PRODUCER, limit_ns);
 }
 
 // Cluster-scope wait: used where the arrivals come from the peer CTA.

@@ -21,7 +21,8 @@ bool fail_case(const char* what, const l4moe_params& p, int T, int k, int sms) {
 bool check(const l4moe_params& p, int Tmax, int k, int sms) {
     const WsLayout L = ws_layout(p, Tmax, sms, k);
     const size_t seg[] = {L.err, L.idx, L.gate, L.lmax, L.margin, L.inv, L.perm, L.gslot, L.counts, L.offsets,
-                          L.tab_gu, L.tab_dn, L.xg, L.hr, L.hs, L.x16, L.part, L.logits, L.device_total,
+                          L.chunk, L.tab_gu, L.tab_dn, L.xg, L.hr, L.hs, L.x16, L.xsc, L.part, L.logits,
+                          L.device_total,
                           L.xin, L.xout, L.total};
     const int nseg = sizeof(seg) / sizeof(seg[0]);
     for (int i = 0; i < nseg; ++i) {
@@ -50,8 +51,16 @@ bool check(const l4moe_params& p, int Tmax, int k, int sms) {
     if ((E && size_of(L.xg) < tv * d * a) || (E && size_of(L.hr) < tv * F * a) || size_of(L.hs) < t * Fs * a)
         return fail_case("activation rows too small", p, Tmax, k, sms);
     if (coded8(p.dtype) && size_of(L.x16) < t * d * 2) return fail_case("f16 x too small", p, Tmax, k, sms);
+    if (coded8(p.dtype) && size_of(L.xsc) < 4 * t) return fail_case("row scales too small", p, Tmax, k, sms);
     if (E && size_of(L.logits) < 4 * std::min<size_t>(t, 128) * E)
         return fail_case("router logits too small", p, Tmax, k, sms);
+    // the small-batch routing's partial logits [slices][T][E] for T <= kSmallMaxTokens
+    const size_t slices = (d + kSmallSliceK - 1) / kSmallSliceK;
+    if (E && size_of(L.logits) < 4 * slices * std::min<size_t>(t, kSmallMaxTokens) * E)
+        return fail_case("small-batch partial logits too small", p, Tmax, k, sms);
+    // the dispatch's chunk bases [chunks][E]
+    if (E && size_of(L.chunk) < 4 * ((tv + kDispatchChunk - 1) / kDispatchChunk) * E)
+        return fail_case("dispatch chunk bases too small", p, Tmax, k, sms);
     if (L.xout + 2 * t * d * a > L.total || L.xin + 2 * t * d * a > L.xout)
         return fail_case("host staging too small", p, Tmax, k, sms);
     const int kblk = (int)(128 / a);

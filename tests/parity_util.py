@@ -12,8 +12,10 @@ Acceptance (the layer's stated tolerances):
       bf16 -- f16 for 8-bit weight layers -- everything else exact) to
       within the output's own rounding and a small allowance for fp32
       accumulation order: |out - ref_h| <= halfulp(out) + READING_SLACK *
-      rms(oracle).  (fp32 layers multiply in TF32, which the oracle does not
-      model: they take the plain bound below only.)
+      rms(oracle), the slack covering hidden values whose fp32 value rounds
+      to the neighbour of the exact value's rounding (see READING_SLACK).
+      (fp32 layers multiply in TF32, which the oracle does not model: they
+      take the plain bound below only.)
     - the stated bound max|out - oracle| <= tol * rms(oracle), tol = 2e-2
       (fp32, bf16) or 6e-2 (E4M3, int8 weights), asserted wherever every
       exact implementation of those roundings meets it: where the largest
@@ -37,9 +39,18 @@ MARGIN_EXCLUDE = 1e-4
 TOL = {"f32": 2e-2, "bf16": 2e-2, "fp8": 6e-2, "int8": 6e-2}
 # the type the GPU holds the hidden rows in (None: fp32 layers, TF32 products)
 HIDDEN = {"f32": None, "bf16": "bf16", "fp8": "f16", "int8": "f16"}
-# allowance, in units of rms(oracle), for fp32 accumulation order and for the
-# rare hidden values whose fp32 value sits at a 16-bit rounding midpoint
-READING_SLACK = 2e-3
+# Allowance, in units of rms(oracle), beyond the output's own rounding.  The
+# GPU forms each hidden value in fp32 (tensor-core accumulation, fast exp)
+# before rounding it to the hidden type; where that fp32 value and the exact
+# one fall on either side of a rounding midpoint, the two round to adjacent
+# values, and that one-spacing difference moves every output of the token
+# by the spacing times the down-projection weights.  A relative 1e-6 to 1e-5
+# error in the hidden values -- fp32 accumulation order -- is enough for a
+# few such flips per token, and one flip of a large hidden value dominates:
+# the CPU reproduction (tests/test_tolerance_floor.py) moves outputs by up to
+# about 6e-3 * rms with bf16 hidden rows; f16 rows have an 8 times finer
+# spacing.
+READING_SLACK = {"bf16": 8e-3, "f16": 1.5e-3}
 
 
 def halfulp_bf16(v: np.ndarray) -> np.ndarray:
@@ -205,14 +216,15 @@ def judge_outputs(got: np.ndarray, ref: np.ndarray, ref_h, dtype: str, tol: floa
         rep.update(reading=None, floor=None, stated_bound_asserted=True)
         assert plain <= tol, f"max|err|/rms = {plain:.4g} exceeds tol {tol}"
         return rep
+    slack = READING_SLACK[HIDDEN[dtype]]
     dev = np.abs(got - ref_h) - halfulp_bf16(got)
     reading = float(np.max(dev)) / rms
     floor = float(np.max(halfulp_bf16(ref_h) + np.abs(ref_h - ref))) / rms
-    asserted = floor + READING_SLACK <= tol
+    asserted = floor + slack <= tol
     rep.update(reading=reading, floor=floor, stated_bound_asserted=bool(asserted))
-    assert reading <= READING_SLACK, (
+    assert reading <= slack, (
         f"output off the oracle's evaluation of the stated roundings by {reading:.3g} * rms beyond "
-        f"its own rounding (allowed {READING_SLACK}); max|err|/rms = {plain:.4g}")
+        f"its own rounding (allowed {slack}); max|err|/rms = {plain:.4g}")
     if asserted:
         assert plain <= tol, f"max|err|/rms = {plain:.4g} exceeds tol {tol} (floor {floor:.4g})"
     return rep

@@ -36,6 +36,7 @@ def test_status_strings_and_version(lib):
     assert lib.l4moe_version() == 100
     assert lib.l4moe_status_string(0) == b"L4MOE_OK"
     assert lib.l4moe_status_string(6) == b"L4MOE_ERR_TIMEOUT"
+    assert lib.l4moe_status_string(8) == b"L4MOE_ERR_RANGE"
 
 
 def _create(lib, d, F, Fs, E, dtype):

@@ -46,6 +46,12 @@ SMALL = {
     "fp8_splitk": LayerConfig("fp8_splitk", 2, 1024, 8, 1024, 1024, "fp8", wr_std=0.03),
     "int8_splitk": LayerConfig("int8_splitk", 2, 1024, 8, 1024, 1024, "int8", wr_std=0.03),
     "bf16_router_split": LayerConfig("bf16_router_split", 1, 1024, 64, 512, 512, "bf16", wr_std=0.03),
+    # the largest batch of the one-launch small-batch routing; fp32 with an
+    # expert count that is not a multiple of 8
+    "bf16_T16_E128": LayerConfig("bf16_T16_E128", 16, 512, 128, 256, 256, "bf16", wr_std=0.05),
+    "f32_T16_E6": LayerConfig("f32_T16_E6", 16, 320, 6, 128, 192, "f32", wr_std=0.1),
+    "fp8_T9_zipf": LayerConfig("fp8_T9_zipf", 9, 256, 16, 128, 128, "fp8", router="zipf", n_dead=4,
+                               wr_std=0.05),
     "bf16_T40_E32": LayerConfig("bf16_T40_E32", 40, 512, 32, 512, 768, "bf16", wr_std=0.05),
     # few token tiles and E < 32: the router splits K into 4 slices per token
     # tile and reduces them inside a cluster (ragged last tile)
@@ -96,6 +102,8 @@ TOPK = {
     # one token tile with E >= 32: expert-split router, top-k in the permutation
     "bf16_k3_split_router": (LayerConfig("bf16_k3_sr", 40, 512, 32, 256, 384, "bf16", wr_std=0.05), 3),
     "bf16_k2_T1": (LayerConfig("bf16_k2_T1", 1, 1024, 64, 512, 512, "bf16", wr_std=0.03), 2),
+    # small-batch routing at its limits: 16 tokens x 4 experts of 256
+    "bf16_k4_T16_E256": (LayerConfig("bf16_k4_T16_E256", 16, 512, 256, 64, 128, "bf16", wr_std=0.05), 4),
 }
 
 
@@ -284,3 +292,56 @@ def test_full_size_maverick_fp8_zipf():
 
 def test_full_size_maverick_int8_zipf():
     _full_size(CONFIGS["maverick_int8"])
+
+
+@pytest.mark.parametrize("dtype,T,E", [("fp8", 300, 8), ("int8", 5, 8), ("fp8", 3, 0), ("int8", 40, 0)],
+                         ids=["fp8_T300", "int8_T5_small_batch", "fp8_dense_T3", "int8_dense_T40"])
+def test_8bit_layers_take_inputs_beyond_f16_range(dtype, T, E):
+    """E4M3 / int8 layers hold x in f16 for their contractions.  With bf16
+    inputs around 1e5 (beyond f16's 65504) each token row is divided by a
+    power of two on the way to f16 and the accumulators get it back: the
+    outputs still match the oracle, which sees the inputs as they are.  The
+    weights are small so that the hidden values stay in range."""
+    cfg = LayerConfig(f"{dtype}_big_x", T, 256, E, 128 if E else 0, 192, dtype, x_std=1e5, w_std=1e-6,
+                      wr_std=1e-6)
+    inp = generate(cfg, seed=5, device="cuda")
+    assert float(inp.x.float().abs().max()) > 65504.0
+    layer = make_layer(inp)
+    if E:
+        out, r = run_gpu(layer, inp)
+        rep = check_routing(inp, r)
+        res = check_outputs(inp, out, None, rep["same"])
+    else:
+        res = check_outputs(inp, _dense_forward(inp), None)
+    print(f"{cfg.name} T={T}: {describe(res)}")
+
+
+def test_hidden_values_beyond_f16_range_are_reported():
+    """A hidden value of an 8-bit-weight layer that f16 cannot hold is not
+    stored silently as infinity: the device status says so."""
+    from sparse_moe_transformer_router_b200.binding import ERR_RANGE, L4MoEError
+    cfg = LayerConfig("fp8_big_hidden", 64, 256, 4, 128, 128, "fp8", x_std=1e3, wr_std=1e-4)
+    inp = generate(cfg, seed=6, device="cuda")
+    layer = make_layer(inp)
+    layer.forward(inp.x, inp.W_router, inp.W_gate_up, inp.W_down, inp.Ws_gate_up, inp.Ws_down)
+    with pytest.raises(L4MoEError) as ei:
+        layer.check_device_status()
+    assert ei.value.status == ERR_RANGE
+    layer.check_device_status()  # the word was cleared
+
+
+def test_a_bounded_wait_that_runs_out_is_reported_and_the_context_survives():
+    """The failure path of every mbarrier wait in the kernels: a wait whose
+    phase never completes gives up after its limit (here 5 ms), records a
+    timeout in the device status and returns; the next forward still runs."""
+    from sparse_moe_transformer_router_b200.binding import ERR_TIMEOUT, L4MoEError
+    inp = generate(SMALL["bf16_ragged"], seed=3, device="cuda")
+    layer = make_layer(inp)
+    layer.selftest_wait(5.0)
+    with pytest.raises(L4MoEError) as ei:
+        layer.check_device_status()
+    assert ei.value.status == ERR_TIMEOUT
+    layer.check_device_status()  # cleared
+    out, r = run_gpu(layer, inp)
+    rep = check_routing(inp, r)
+    check_outputs(inp, out, None, rep["same"])

@@ -78,7 +78,7 @@ def test_parity_check_accepts_the_reading_and_rejects_one_spacing_off(dtype):
         judge_outputs(bad, ref, ref_h, dtype)
     # a small extra error everywhere (an approximate contraction) is caught too
     rms = np.sqrt(np.mean(ref ** 2))
-    noisy = round_out(ref_h + 3 * READING_SLACK * rms * np.sign(ref_h), dtype)
+    noisy = round_out(ref_h + 3 * READING_SLACK[HIDDEN[dtype]] * rms * np.sign(ref_h), dtype)
     with pytest.raises(AssertionError):
         judge_outputs(noisy, ref, ref_h, dtype)
 
@@ -115,3 +115,29 @@ def test_oracle_hidden_rounding_matches_a_library_evaluation():
         h2 = torch.nn.functional.silu(a2[:, :Fs]) * a2[:, Fs:]
         lib_h1 = lib_h + h2.float().to(tdt).double() @ W2d.double()
         np.testing.assert_allclose(out_h1, lib_h1.numpy(), rtol=1e-12, atol=1e-12)
+
+
+@pytest.mark.parametrize("hidden,tdt", [("bf16", torch.bfloat16), ("f16", torch.float16)])
+def test_hidden_rounding_flips_stay_within_the_reading_slack(hidden, tdt):
+    """The reading check's slack covers hidden values that fp32 arithmetic
+    rounds to the other neighbour of the exact value's rounding.  Perturbing
+    every hidden value of a layer by a relative 1e-6 (an fp32 accumulation
+    error) flips a small fraction of them and moves outputs by up to a few
+    thousandths of rms with bf16 rows -- more than any allowance for fp32
+    noise alone, within READING_SLACK -- and by 8 times less with f16 rows."""
+    cfg = LayerConfig("flips", 300, 256, 0, 0, 384, "bf16")
+    inp = generate(cfg, seed=0, device="cpu")
+    x, Wgu, Wd = inp.x.double(), inp.Ws_gate_up.double(), inp.Ws_down.double()
+    a = x @ Wgu
+    h = torch.nn.functional.silu(a[:, :384]) * a[:, 384:]
+    rng = np.random.default_rng(1)
+    hn = h * (1 + 1e-6 * torch.from_numpy(rng.standard_normal(tuple(h.shape))))
+    hb, hnb = h.float().to(tdt).double(), hn.float().to(tdt).double()
+    flipped = (hb != hnb).double().mean().item()
+    y = hb @ Wd
+    dy = ((hnb @ Wd) - y).abs().max().item() / y.pow(2).mean().sqrt().item()
+    assert 0 < flipped < 1e-2
+    assert dy <= READING_SLACK[hidden]
+    if hidden == "bf16":
+        assert dy > 1e-3      # far above fp32 noise: the flips themselves
+    print(f"{hidden}: {flipped:.2e} of hidden values flipped, max output change {dy:.2e} * rms")
