@@ -40,7 +40,7 @@ ROOT = os.path.dirname(os.path.abspath(__file__))
 sys.path.insert(0, ROOT)
 
 from sparse_moe_transformer_router_b200 import accounting  # noqa: E402
-from sparse_moe_transformer_router_b200.workloads import CONFIGS, generate, to_storage_numpy  # noqa: E402
+from sparse_moe_transformer_router_b200.workloads import CODED, CONFIGS, generate, to_storage_numpy  # noqa: E402
 
 DEFAULT_WORKLOAD = "scout_prefill_bf16"
 METRIC = "moe_layer_tokens_per_s"
@@ -173,24 +173,33 @@ class HostLayer:
         self.x = to_storage_numpy(inp.x)
         self.Wr = to_storage_numpy(inp.W_router)
         self.bias = None if inp.bias is None else inp.bias.cpu().numpy()
-        self.Ws_gu = to_storage_numpy(inp.Ws_gate_up)
-        self.Ws_dn = to_storage_numpy(inp.Ws_down)
+        self.Ws_gu = self._w(inp.Ws_gate_up)
+        self.Ws_dn = self._w(inp.Ws_down)
         self.idx = None
         self._gu, self._dn, self._sgu, self._sdn = {}, {}, {}, {}
+
+    def _w(self, t):
+        """A weight in the oracle's storage form (packed int4 bytes viewed as
+        the oracle's int4 type)."""
+        a = to_storage_numpy(t)
+        if self.inp.cfg.dtype == "int4":
+            import oracle
+            a = oracle.as_int4x2(a)
+        return a
 
     def expert_args(self, need):
         inp, E = self.inp, self.inp.cfg.num_experts
         for e in need:
             if e not in self._gu:
-                self._gu[e] = to_storage_numpy(inp.W_gate_up[e])
-                self._dn[e] = to_storage_numpy(inp.W_down[e])
-                if inp.cfg.dtype in ("fp8", "int8"):
+                self._gu[e] = self._w(inp.W_gate_up[e])
+                self._dn[e] = self._w(inp.W_down[e])
+                if inp.cfg.dtype in CODED:
                     self._sgu[e] = inp.s_gate_up[e].cpu().numpy()
                     self._sdn[e] = inp.s_down[e].cpu().numpy()
         Wgu = [self._gu.get(e) if e in need else None for e in range(E)]
         Wdn = [self._dn.get(e) if e in need else None for e in range(E)]
         kw = {}
-        if inp.cfg.dtype in ("fp8", "int8"):
+        if inp.cfg.dtype in CODED:
             kw = dict(s_gate_up=[self._sgu.get(e) if e in need else None for e in range(E)],
                       s_down=[self._sdn.get(e) if e in need else None for e in range(E)],
                       ss_gate_up=inp.ss_gate_up.cpu().numpy(), ss_down=inp.ss_down.cpu().numpy())
@@ -356,7 +365,7 @@ DATASHEET = {"bf16_tflops": 2250.0, "hbm_gbs": 8000.0}
 # timed region, roofline and clocks: the other shapes the layer is quoted on.
 EXTRA_WORKLOADS = ("maverick_prefill_bf16", "maverick_decode_bf16@T1", "maverick_decode_bf16@T8",
                    "maverick_decode_bf16@T32", "maverick_decode_bf16@T128", "maverick_fp8",
-                   "maverick_int8", "maverick_dense_bf16", "tiny_f32")
+                   "maverick_int8", "scout_prefill_int4", "maverick_dense_bf16", "tiny_f32")
 
 
 def workload_config(name: str):
@@ -371,7 +380,7 @@ def make_layer(cfg, rank):
     layer = L4MoE(cfg.d_model, cfg.expert_ffn, cfg.shared_ffn, cfg.num_experts, cfg.dtype)
     if inp.bias is not None:
         layer.set_router_bias(inp.bias)
-    if cfg.dtype in ("fp8", "int8"):
+    if cfg.dtype in CODED:
         layer.set_weight_scales(inp.s_gate_up, inp.s_down, inp.ss_gate_up, inp.ss_down)
     return inp, layer
 
@@ -578,8 +587,8 @@ def run_b200(args, rank, world, local):
             "experts_touched": m["experts_touched"],
             "peaks_note": "frac: of the measured peak (peak_source); frac_of_datasheet: of NVIDIA's "
                           "dense bf16 2250 TFLOP/s or HBM3e 8000 GB/s"}
-    if cfg.dtype in ("fp8", "int8"):
-        wname = "E4M3" if cfg.dtype == "fp8" else "int8"
+    if cfg.dtype in CODED:
+        wname = {"fp8": "E4M3", "int8": "int8", "int4": "int4"}[cfg.dtype]
         line["dtype"] = f"f16 ({wname} weights widened exactly to f16, fp32 accumulate; bf16 in and out)"
     if cpu is not None:
         line["cpu_baseline"] = cpu

@@ -51,6 +51,13 @@
  *                   no zero point) with one fp32 scale per output column, the
  *                   weight-only int8 of KerasFormers "Llama 4", "Lower memory";
  *                   otherwise as L4MOE_FP8_E4M3 (every int8 value is exact in f16).
+ *   L4MOE_INT4      expert and shared weights int4 (two's-complement nibbles,
+ *                   symmetric) with one fp32 scale per output column, the
+ *                   int4 the glossary's "The Llama 4 Herd" and the aibase
+ *                   card's "Quantization" name for Scout; packed two per byte
+ *                   along the output columns, the even column in the low
+ *                   nibble: W_gate_up is [d, F] bytes, W_down [F, d/2] (same
+ *                   for the shared expert); otherwise as L4MOE_INT8.
  *
  * Ownership: the caller owns every tensor, the scale vectors, the bias and
  * the stream.  The handle owns only its workspace (unless the caller supplies
@@ -103,7 +110,8 @@ typedef enum {
     L4MOE_F32 = 0,
     L4MOE_BF16 = 1,
     L4MOE_FP8_E4M3 = 2,
-    L4MOE_INT8 = 3
+    L4MOE_INT8 = 3,
+    L4MOE_INT4 = 4
 } l4moe_dtype;
 
 typedef struct {
@@ -149,7 +157,7 @@ L4MOE_API l4moe_status l4moe_set_router_bias(l4moe_handle *h, const float *bias_
  * equal values, NaN never selected), each on the input gated by the sigmoid
  * of its own logit, and their outputs add to the shared expert's (the
  * "experts per token" of a token-choice router, torchtune MoE
- * documentation).  1 <= k <= min(4, E); k > 1 needs bf16, E4M3 or int8 weights and
+ * documentation).  1 <= k <= min(4, E); k > 1 needs bf16, E4M3, int8 or int4 weights and
  * E % 8 == 0 (else L4MOE_ERR_UNSUPPORTED).  The routing arrays of
  * l4moe_get_routing then hold T * k entries (entry t * k + j: token t's j-th
  * expert; margin stays [T]: the k-th logit minus the next one).  Changing k
@@ -158,7 +166,7 @@ L4MOE_API l4moe_status l4moe_set_router_bias(l4moe_handle *h, const float *bias_
  * routing arrays then describe the next forward, not the earlier ones. */
 L4MOE_API l4moe_status l4moe_set_top_k(l4moe_handle *h, int k);
 
-/* E4M3 or int8 weights only: per-output-column fp32 scales (device
+/* E4M3, int8 or int4 weights only: per-output-column fp32 scales (device
  * pointers).  s_gate_up / s_down are HOST arrays of E device pointers to
  * [2F] / [d] vectors; ss_gate_up [2Fs] and ss_down [d] are the shared
  * expert's.  The dequantised weight is e4m3(q) * scale[column] or

@@ -17,8 +17,8 @@ from __future__ import annotations
 
 import numpy as np
 
-ACT_BYTES = {"f32": 4, "bf16": 2, "fp8": 2, "int8": 2}
-W_BYTES = {"f32": 4, "bf16": 2, "fp8": 1, "int8": 1}
+ACT_BYTES = {"f32": 4, "bf16": 2, "fp8": 2, "int8": 2, "int4": 2}
+W_BYTES = {"f32": 4, "bf16": 2, "fp8": 1, "int8": 1, "int4": 0.5}
 
 
 def flops_per_token(d: int, E: int, F: int, Fs: int) -> int:
@@ -32,14 +32,14 @@ def layer_flops(T: int, d: int, E: int, F: int, Fs: int) -> int:
 def layer_bytes(T: int, d: int, E: int, F: int, Fs: int, dtype: str, experts_touched: int) -> int:
     a, w = ACT_BYTES[dtype], W_BYTES[dtype]
     weights = (experts_touched * 3 * d * F + 3 * d * Fs) * w
-    if dtype in ("fp8", "int8"):  # per-output-column fp32 scales
+    if dtype in ("fp8", "int8", "int4"):  # per-output-column fp32 scales
         weights += (experts_touched * (2 * F + d) + (2 * Fs + d)) * 4
     router = d * E * a
     acts = T * d * a * 2                 # x read, out write
     if E > 0:
         acts += T * d * a * 2            # gated expert-ordered input: write + read
     acts += T * (F + Fs) * a * 2         # hidden activations: write + read
-    return weights + router + acts
+    return int(weights + router + acts)
 
 
 def experts_touched(counts) -> int:

@@ -15,7 +15,7 @@ _PKG = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(_PKG, "libl4moe.so")
 
 OK, ERR_ARG, ERR_DTYPE, ERR_ALIGN, ERR_CUDA, ERR_WORKSPACE, ERR_TIMEOUT, ERR_UNSUPPORTED, ERR_RANGE = range(9)
-DTYPES = {"f32": 0, "bf16": 1, "fp8": 2, "int8": 3}
+DTYPES = {"f32": 0, "bf16": 1, "fp8": 2, "int8": 3, "int4": 4}
 EXPORTED = ("l4moe_create", "l4moe_destroy", "l4moe_workspace_size", "l4moe_set_workspace",
             "l4moe_set_router_bias", "l4moe_set_fp8_scales", "l4moe_forward",
             "l4moe_forward_host", "l4moe_get_routing", "l4moe_check_device_status",
@@ -117,8 +117,11 @@ def _stream_handle(stream) -> int | None:
     return stream.cuda_stream
 
 
-_ACT_DTYPE = {"f32": torch.float32, "bf16": torch.bfloat16, "fp8": torch.bfloat16, "int8": torch.bfloat16}
-_W_DTYPE = {"f32": torch.float32, "bf16": torch.bfloat16, "fp8": torch.float8_e4m3fn, "int8": torch.int8}
+_ACT_DTYPE = {"f32": torch.float32, "bf16": torch.bfloat16, "fp8": torch.bfloat16, "int8": torch.bfloat16,
+              "int4": torch.bfloat16}
+# int4 weights are packed two per byte along the output columns
+_W_DTYPE = {"f32": torch.float32, "bf16": torch.bfloat16, "fp8": torch.float8_e4m3fn, "int8": torch.int8,
+            "int4": torch.uint8}
 
 
 def _expect(t, name, shape, dtype):
@@ -193,7 +196,7 @@ class L4MoE:
         self._bias = bias
 
     def set_weight_scales(self, s_gate_up, s_down, ss_gate_up, ss_down):
-        """Per-output-column fp32 scales of E4M3 or int8 weights (device tensors)."""
+        """Per-output-column fp32 scales of E4M3, int8 or int4 weights (device tensors)."""
         a, b = _ptr_array(s_gate_up), _ptr_array(s_down)
         self._check(self._lib.l4moe_set_weight_scales(self._h, a, b, _ptr(ss_gate_up), _ptr(ss_down)))
         self._scales = (list(s_gate_up), list(s_down), ss_gate_up, ss_down)
@@ -220,9 +223,10 @@ class L4MoE:
             wdt = _W_DTYPE[self.dtype]
             if len(W_gate_up) != E or len(W_down) != E:
                 raise ValueError(f"l4moe: expected {E} expert weights, got {len(W_gate_up)} / {len(W_down)}")
-            named = [(W_gate_up[e], f"W_gate_up[{e}]", (d, 2 * F)) for e in range(E)]
-            named += [(W_down[e], f"W_down[{e}]", (F, d)) for e in range(E)]
-            named += [(Ws_gate_up, "Ws_gate_up", (d, 2 * Fs)), (Ws_down, "Ws_down", (Fs, d))]
+            cols = (lambda n: n // 2) if self.dtype == "int4" else (lambda n: n)  # noqa: E731 (packed bytes)
+            named = [(W_gate_up[e], f"W_gate_up[{e}]", (d, cols(2 * F))) for e in range(E)]
+            named += [(W_down[e], f"W_down[{e}]", (F, cols(d))) for e in range(E)]
+            named += [(Ws_gate_up, "Ws_gate_up", (d, cols(2 * Fs))), (Ws_down, "Ws_down", (Fs, cols(d)))]
             for t, name, shape in named:
                 _expect(t, name, shape, wdt)
             for t, name, _ in named:

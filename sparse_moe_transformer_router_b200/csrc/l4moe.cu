@@ -82,9 +82,13 @@ struct WsLayout {
 };
 
 size_t act_bytes(l4moe_dtype dt) { return dt == L4MOE_F32 ? 4 : 2; }
-size_t w_bytes(l4moe_dtype dt) { return dt == L4MOE_F32 ? 4 : (dt == L4MOE_BF16 ? 2 : 1); }
-// 8-bit weight codes (E4M3 or int8) with per-output-column scales
-bool coded8(l4moe_dtype dt) { return dt == L4MOE_FP8_E4M3 || dt == L4MOE_INT8; }
+// Bytes of a row of n weights (int4: two per byte).
+uint64_t w_row_bytes(l4moe_dtype dt, uint64_t n) {
+    return dt == L4MOE_F32 ? 4 * n : dt == L4MOE_BF16 ? 2 * n : dt == L4MOE_INT4 ? n / 2 : n;
+}
+// coded weights (E4M3, int8 or int4) with per-output-column scales, widened
+// to f16 in the GEMMs (the activations of these layers are f16 there)
+bool coded8(l4moe_dtype dt) { return dt == L4MOE_FP8_E4M3 || dt == L4MOE_INT8 || dt == L4MOE_INT4; }
 
 // Split-K plan of one forward of T tokens: how many k-ranges the gate/up and
 // the down launches use.  Only batches of at most kSplitMaxTokens split, into
@@ -345,15 +349,17 @@ l4moe_status encode_weight_maps(l4moe_handle* h, const void* const* Wgu, const v
     for (int e = 0; same && e < E; ++e) same = h->hkey_gu[e] == Wgu[e] && h->hkey_dn[e] == Wdn[e];
     if (same) return L4MOE_OK;
     const int d = h->p.d_model, F = h->p.expert_ffn, Fs = h->p.shared_ffn;
-    const size_t wb = w_bytes(h->p.dtype);
-    CUtensorMapDataType dt = h->p.dtype == L4MOE_F32 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT32
-                             : h->p.dtype == L4MOE_BF16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16
-                                                        : CU_TENSOR_MAP_DATA_TYPE_UINT8;
-    const bool fp8 = coded8(h->p.dtype);
-    const uint32_t bk = h->p.dtype == L4MOE_F32 ? 32 : 64;  // K rows per box
-    // features per box: one 128-byte swizzled slab; 8-bit weights are staged
-    // raw (64-feature boxes, unswizzled) and widened in shared memory
-    const uint32_t bw = fp8 ? 64u : (uint32_t)(128 / wb);
+    const l4moe_dtype wdt = h->p.dtype;
+    CUtensorMapDataType dt = wdt == L4MOE_F32 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT32
+                             : wdt == L4MOE_BF16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16
+                                                 : CU_TENSOR_MAP_DATA_TYPE_UINT8;
+    const bool fp8 = coded8(wdt);
+    const uint32_t bk = wdt == L4MOE_F32 ? 32 : 64;  // K rows per box
+    // box width in elements of the map: one 128-byte swizzled slab of
+    // features; coded weights are staged raw (64-feature boxes, unswizzled;
+    // int4 maps count bytes, 32 of them per 64 features) and widened in
+    // shared memory
+    const uint32_t bw = wdt == L4MOE_INT4 ? 32u : fp8 ? 64u : (uint32_t)(128 / w_row_bytes(wdt, 1));
     // MN-major 32-bit operands need the 32-byte swizzle unit
     const CUtensorMapSwizzle swz = fp8 ? CU_TENSOR_MAP_SWIZZLE_NONE
                                    : h->p.dtype == L4MOE_F32 ? CU_TENSOR_MAP_SWIZZLE_128B_ATOM_32B
@@ -365,8 +371,11 @@ l4moe_status encode_weight_maps(l4moe_handle* h, const void* const* Wgu, const v
         const void* gu = sh ? Wsgu : Wgu[e];
         const void* dn = sh ? Wsdn : Wdn[e];
         const int f = sh ? Fs : F;
-        if (!encode_2d(&h->h_maps[e], dt, gu, 2ull * f, (uint64_t)d, 2ull * f * wb, bw, bk, swz) ||
-            !encode_2d(&h->h_maps[E + 1 + e], dt, dn, (uint64_t)d, (uint64_t)f, (uint64_t)d * wb, bw,
+        // map elements per row: features, or bytes for int4
+        const uint64_t gu_w = wdt == L4MOE_INT4 ? (uint64_t)f : 2ull * f;
+        const uint64_t dn_w = wdt == L4MOE_INT4 ? (uint64_t)d / 2 : (uint64_t)d;
+        if (!encode_2d(&h->h_maps[e], dt, gu, gu_w, (uint64_t)d, w_row_bytes(wdt, 2ull * f), bw, bk, swz) ||
+            !encode_2d(&h->h_maps[E + 1 + e], dt, dn, dn_w, (uint64_t)f, w_row_bytes(wdt, (uint64_t)d), bw,
                        bk, swz)) {
             h->h_maps.clear();
             return fail(h, L4MOE_ERR_CUDA, "cuTensorMapEncodeTiled failed for a weight");
@@ -453,7 +462,7 @@ void launch_router(const void* x, const void* Wr, const float* bias, int T, int 
 
 template <int MODE, typename ET, int WQ>
 void launch_gemm(int grid, const BMaps& bm, const GemmArgs& a, cudaStream_t st) {
-    using Cfg = GemmCfg<MODE, ET, WQ != kWqNone>;
+    using Cfg = GemmCfg<MODE, ET, WQ>;
     static std::atomic<uint64_t> attr_done{0};
     ensure_smem_attr(attr_done, moe_gemm_kernel<MODE, ET, WQ>, Cfg::SMEM_BYTES);
     launch_k(moe_gemm_kernel<MODE, ET, WQ>, dim3(grid), dim3(Cfg::THREADS), Cfg::SMEM_BYTES, st, bm, a);
@@ -503,7 +512,7 @@ l4moe_status run_layer(l4moe_handle* h, int T, const void* x, const void* Wr, co
     const CUtensorMapDataType adt = tmap_type(sizeof(ET), false);
     const CUtensorMapDataType gdt = tmap_type(sizeof(GT), FP8W);
     const uint32_t bk = (uint32_t)(128 / sizeof(ET));
-    using GCfg = GemmCfg<MODE_GATEUP, ET, FP8W>;
+    using GCfg = GemmCfg<MODE_GATEUP, ET, WQ>;
     constexpr uint32_t rb = GCfg::B_BOX_ROWS, rs = GCfg::B_SMALL_ROWS;
     CUtensorMap m_x;
     BMaps bm_gu, bm_dn;
@@ -800,6 +809,9 @@ l4moe_status forward_impl(l4moe_handle* h, int T, const void* x, const void* Wr,
     case L4MOE_INT8:
         return run_layer<__nv_bfloat16, kWqInt8>(h, T, x, Wr, Wsgu, Wsdn, out, st, h->ws, h->ws_tokens,
                                                  h->d_maps, h->d_scales);
+    case L4MOE_INT4:
+        return run_layer<__nv_bfloat16, kWqInt4>(h, T, x, Wr, Wsgu, Wsdn, out, st, h->ws, h->ws_tokens,
+                                                 h->d_maps, h->d_scales);
     }
     return fail(h, L4MOE_ERR_DTYPE, "unknown dtype");
 }
@@ -882,6 +894,9 @@ l4moe_status l4moe_forward_static(l4moe_handle* h, int T, const void* x, const v
     else if (h->p.dtype == L4MOE_INT8)
         s = run_layer<__nv_bfloat16, kWqInt8>(h, T, x, W_router, Ws_gate_up, Ws_down, out, st, base, T, maps,
                                               scales);
+    else if (h->p.dtype == L4MOE_INT4)
+        s = run_layer<__nv_bfloat16, kWqInt4>(h, T, x, W_router, Ws_gate_up, Ws_down, out, st, base, T, maps,
+                                              scales);
     else
         s = run_layer<__nv_bfloat16>(h, T, x, W_router, Ws_gate_up, Ws_down, out, st, base, T, maps);
     h->timing = timing;
@@ -909,7 +924,8 @@ l4moe_status l4moe_create(const l4moe_params* params, l4moe_handle** out) {
     if (!params || !out) return fail(nullptr, L4MOE_ERR_ARG, "null params or out");
     *out = nullptr;
     const l4moe_params& p = *params;
-    if (p.dtype != L4MOE_F32 && p.dtype != L4MOE_BF16 && p.dtype != L4MOE_FP8_E4M3 && p.dtype != L4MOE_INT8)
+    if (p.dtype != L4MOE_F32 && p.dtype != L4MOE_BF16 && p.dtype != L4MOE_FP8_E4M3 && p.dtype != L4MOE_INT8 &&
+        p.dtype != L4MOE_INT4)
         return fail(nullptr, L4MOE_ERR_DTYPE, "unknown dtype");
     if (p.d_model <= 0 || p.shared_ffn <= 0 || p.num_experts < 0 || p.num_experts > 256 ||
         p.expert_ffn < 0 || (p.num_experts > 0 && p.expert_ffn == 0))
@@ -1012,7 +1028,7 @@ l4moe_status l4moe_set_weight_scales(l4moe_handle* h, const float* const* s_gate
                                      const float* const* s_down, const float* ss_gate_up,
                                      const float* ss_down) {
     if (!h) return L4MOE_ERR_ARG;
-    if (!coded8(h->p.dtype)) return fail(h, L4MOE_ERR_DTYPE, "scales apply to E4M3 or int8 weights only");
+    if (!coded8(h->p.dtype)) return fail(h, L4MOE_ERR_DTYPE, "scales apply to E4M3, int8 or int4 weights only");
     const int E = h->p.num_experts;
     if (!ss_gate_up || !ss_down || (E > 0 && (!s_gate_up || !s_down)))
         return fail(h, L4MOE_ERR_ARG, "null scale pointer");

@@ -130,8 +130,14 @@ struct GemmArgs {
 template <int MODE>
 __host__ __device__ constexpr int pair_features() { return MODE == MODE_GATEUP ? 128 : 256; }
 
-template <int MODE, typename ET, bool FP8W>
+// Weight storage of a GEMM: the layer's own type, or 8-bit or 4-bit codes
+// widened in shared memory (E4M3 floats, int8 or int4 integers, per-column
+// scales).
+enum : int { kWqNone = 0, kWqE4M3 = 1, kWqInt8 = 2, kWqInt4 = 3 };
+
+template <int MODE, typename ET, int WQ>
 struct GemmCfg {
+    static constexpr bool FP8W = WQ != kWqNone;  // coded weights, converter warps
     using C = ElemCfg<ET>;
     static constexpr int A_BYTES = 128 * 128;                // 128 A rows x 128 B of K
     static constexpr int A_BOX_FEATS = 128 / C::BYTES;       // features per A box (one 128 B slab)
@@ -140,7 +146,10 @@ struct GemmCfg {
     static constexpr int B_BOX_ROWS = 128;                   // token rows per full-tile box
     static constexpr int B_SMALL_ROWS = 32;                  // token rows per small-tile box
     static constexpr int B_BYTES = (kTokTile / 2) * 128;     // this CTA's half of the tokens
-    static constexpr int RAW_BYTES = FP8W ? 2 * 64 * 64 : 0; // 2 slabs x 64 K rows x 64 features
+    // raw coded weights: 2 slabs x 64 K rows x 64 features, one byte per code
+    // (half a byte for int4: two codes per byte along the features)
+    static constexpr int RAW_SLAB_BYTES = WQ == kWqInt4 ? 64 * 32 : 64 * 64;
+    static constexpr int RAW_BYTES = FP8W ? 2 * RAW_SLAB_BYTES : 0;
     static constexpr int STAGE_BYTES = A_BYTES + B_BYTES + RAW_BYTES;
     static constexpr int STAGES = FP8W ? 5 : 6;
     static constexpr int ACC_BUFS = 2;
@@ -245,9 +254,28 @@ __device__ __forceinline__ uint4 int8x8_to_f16(uint2 raw) {
                       i8x2_to_f16x2(hi, 0x4140u), i8x2_to_f16x2(hi, 0x4342u));
 }
 
-// Weight storage of a GEMM: the layer's own type, or 8-bit codes widened in
-// shared memory (E4M3 floats or int8 integers, per-column scales).
-enum : int { kWqNone = 0, kWqE4M3 = 1, kWqInt8 = 2 };
+// 8 int4 codes (two's complement nibbles, the lower-numbered code in the low
+// nibble of each byte, bytes little-endian in a uint32) -> 8 f16 values,
+// exactly.  As for int8: flipping each nibble's sign bit gives u = q + 8 in
+// [0, 15]; the f16 with high byte 0x64 and low bits u has the value 1024 + u,
+// and subtracting 1032 = 1024 + 8 leaves q (every value an integer below
+// 2^11, so every step is exact).  Byte i of the biased word holds the pair
+// (code 2i, code 2i+1): its low nibble goes to the low f16 of the pair, its
+// high nibble to the high f16.
+__device__ __forceinline__ uint32_t i4pair_to_f16x2(uint32_t biased, int byte) {
+    const uint32_t t = biased >> (8 * byte);
+    const uint32_t h = (t & 0x0Fu) | ((t & 0xF0u) << 12) | 0x64006400u;
+    uint32_t r;
+    asm("sub.rn.f16x2 %0, %1, %2;" : "=r"(r) : "r"(h), "r"(0x64086408u));
+    return r;
+}
+
+__device__ __forceinline__ uint4 int4x8_to_f16(uint32_t raw) {
+    const uint32_t b = raw ^ 0x88888888u;
+    return make_uint4(i4pair_to_f16x2(b, 0), i4pair_to_f16x2(b, 1), i4pair_to_f16x2(b, 2),
+                      i4pair_to_f16x2(b, 3));
+}
+
 
 // The contractions' activation (token operand and hidden) type: the layer's
 // own, or f16 for E4M3 weights (kind::f16 takes both operands in one type).
@@ -278,11 +306,11 @@ struct BMaps {
 };
 
 template <int MODE, typename ET, int WQ>
-__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(GemmCfg<MODE, ET, WQ != kWqNone>::THREADS, 1)
+__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(GemmCfg<MODE, ET, WQ>::THREADS, 1)
     moe_gemm_kernel(const __grid_constant__ BMaps bm, const GemmArgs args) {
     pdl_enter();
-    constexpr bool FP8W = WQ != kWqNone;  // 8-bit weight codes with converter warps
-    using Cfg = GemmCfg<MODE, ET, FP8W>;
+    constexpr bool FP8W = WQ != kWqNone;  // coded (8- or 4-bit) weights with converter warps
+    using Cfg = GemmCfg<MODE, ET, WQ>;
     using C = ElemCfg<ET>;
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>(
@@ -387,7 +415,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(GemmCfg<MODE, ET, WQ
                     const uint32_t sb = stage0 + (uint32_t)stage * Cfg::STAGE_BYTES;
                     const int k = kb * C::BK;
                     if constexpr (FP8W) {
-                        // raw 8-bit weights: two 64-feature slabs, signalled locally
+                        // raw coded weights: two 64-feature slabs, signalled locally
+                        // (int4: the tensor map counts bytes, two features each)
                         const uint32_t rb = sb + Cfg::A_BYTES + Cfg::B_BYTES;
                         mbar_arrive_expect_tx(rawfull_bar(stage), Cfg::RAW_BYTES);
 #pragma unroll
@@ -395,7 +424,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(GemmCfg<MODE, ET, WQ
                             const int col = (MODE == MODE_GATEUP)
                                                 ? (j == 0 ? acol0 : ti.up_off + acol0)
                                                 : acol0 + 64 * j;
-                            tma_load_2d(rb + j * 4096, amap, rawfull_bar(stage), col, k);
+                            tma_load_2d(rb + j * Cfg::RAW_SLAB_BYTES, amap, rawfull_bar(stage),
+                                        WQ == kWqInt4 ? col / 2 : col, k);
                         }
                     } else {
 #pragma unroll
@@ -496,7 +526,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(GemmCfg<MODE, ET, WQ
             mbar_wait(drain_bar, 0, args.err, DEV_ERR_TIMEOUT_MMA);
         }
     } else if (FP8W && warp >= 6) {
-        // --------------------------------------- weight-code converters (E4M3, int8)
+        // --------------------------------------- weight-code converters (E4M3, int8, int4)
         constexpr int NCT = 32 * (Cfg::CONV_WARPS > 0 ? Cfg::CONV_WARPS : 8);  // converter threads
         static_assert(NCT == 256, "each converter thread owns 4 units: slab i / 2");
         const int ct = threadIdx.x - 192;           // 0 .. NCT-1
@@ -520,10 +550,16 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(GemmCfg<MODE, ET, WQ
                     // unit u = ct + NCT i (of 2 slabs x 64 K rows x 8 chunks):
                     // slab u / 512, K row (u / 8) % 64, chunk c8
                     const int j = (i * NCT) >> 9, kr = ((ct >> 3) + (NCT / 8) * i) & 63;
-                    const uint2 q8 = *reinterpret_cast<const uint2*>(raw + j * 4096 + kr * 64 + c8 * 8);
                     uint4 h8;
-                    if constexpr (WQ == kWqInt8) h8 = int8x8_to_f16(q8);
-                    else h8 = e4m3x8_to_f16(q8);
+                    if constexpr (WQ == kWqInt4) {
+                        h8 = int4x8_to_f16(*reinterpret_cast<const uint32_t*>(raw + j * Cfg::RAW_SLAB_BYTES +
+                                                                              kr * 32 + c8 * 4));
+                    } else {
+                        const uint2 q8 = *reinterpret_cast<const uint2*>(raw + j * Cfg::RAW_SLAB_BYTES + kr * 64 +
+                                                                         c8 * 8);
+                        if constexpr (WQ == kWqInt8) h8 = int8x8_to_f16(q8);
+                        else h8 = e4m3x8_to_f16(q8);
+                    }
                     *reinterpret_cast<uint4*>(a + j * 8192 + kr * 128 + ((c8 ^ (kr & 7)) << 4)) = h8;
                 }
                 fence_proxy_async_smem();  // generic-proxy writes -> tensor-core reads

@@ -26,6 +26,8 @@ import torch
 E4M3_MAX = 448.0
 INT8_MAX = 127.0
 INT4_MAX = 7.0
+# layer dtypes whose weights are codes with per-output-column fp32 scales
+CODED = ("fp8", "int8", "int4")
 
 
 @dataclass(frozen=True)
@@ -36,7 +38,7 @@ class LayerConfig:
     num_experts: int
     expert_ffn: int
     shared_ffn: int
-    dtype: str            # "f32" | "bf16" | "fp8" / "int8" (E4M3 / int8 weights, bf16 activations)
+    dtype: str            # "f32" | "bf16" | "fp8" / "int8" / "int4" (coded weights, bf16 activations)
     router: str = "plain"  # "plain": no bias; "zipf": per-expert bias for Zipf loads
     x_std: float = 1.0
     w_std: float = 0.02
@@ -66,6 +68,8 @@ CONFIGS = {
     # weight-only int8 experts (per-output-column scales), Maverick-shaped
     "maverick_int8": LayerConfig("maverick_int8", 16384, 5120, 128, 8192, 8192, "int8",
                                  router="zipf", n_dead=10),
+    # weight-only int4 experts, Scout-shaped (the glossary's Scout on one GPU in int4)
+    "scout_prefill_int4": LayerConfig("scout_prefill_int4", 4096, 5120, 16, 8192, 8192, "int4"),
 }
 DECODE_TOKENS = (1, 8, 32, 128)
 
@@ -209,6 +213,8 @@ def generate(cfg: LayerConfig, seed: int = 0, device="cpu", experts=None) -> Lay
             return quantize_e4m3_columns(w)
         if cfg.dtype == "int8":
             return quantize_int8_columns(w)
+        if cfg.dtype == "int4":
+            return quantize_int4_columns(w)
         return w.to(act), None
 
     W_gu, W_dn, s_gu, s_dn = [], [], [], []
@@ -224,7 +230,7 @@ def generate(cfg: LayerConfig, seed: int = 0, device="cpu", experts=None) -> Lay
         s_dn.append(sb)
     Ws_gu, ss_gu = weight((d, 2 * Fs), "Ws_gate_up", -1)
     Ws_dn, ss_dn = weight((Fs, d), "Ws_down", -1)
-    scaled = cfg.dtype in ("fp8", "int8")
+    scaled = cfg.dtype in CODED
     return LayerInputs(cfg, x, Wr, bias, W_gu, W_dn, Ws_gu, Ws_dn,
                        s_gu if scaled else None, s_dn if scaled else None,
                        ss_gu if scaled else None, ss_dn if scaled else None)
@@ -240,20 +246,26 @@ E4M3_SUBNORMAL_CODES = tuple(range(0x00, 0x08)) + tuple(range(0x80, 0x88))
 INT8_CODES = tuple(range(-128, 128))
 
 
+INT4_CODES = tuple(range(-8, 8))
+
+
 def with_weight_codes(inp: LayerInputs, codes, scale: float, seed: int) -> LayerInputs:
-    """Replace an E4M3 (or int8) layer's expert and shared weights by codes
-    drawn uniformly (seeded) from ``codes`` and set every column scale to
-    ``scale``."""
-    assert inp.cfg.dtype in ("fp8", "int8")
-    int8 = inp.cfg.dtype == "int8"
-    table = torch.tensor(codes, dtype=torch.int8 if int8 else torch.uint8)
+    """Replace an E4M3, int8 or int4 layer's expert and shared weights by
+    codes drawn uniformly (seeded) from ``codes`` and set every column scale
+    to ``scale``."""
+    assert inp.cfg.dtype in CODED
+    ints = inp.cfg.dtype in ("int8", "int4")
+    table = torch.tensor(codes, dtype=torch.int8 if ints else torch.uint8)
 
     def draw(w, name, e):
         if w is None:
             return None
         g = torch.Generator().manual_seed(_seed(seed, "codes:" + name, e))
+        if inp.cfg.dtype == "int4":  # packed [K, N / 2] bytes: draw [K, N] codes, pack them
+            i = torch.randint(0, table.numel(), (w.shape[0], 2 * w.shape[1]), generator=g)
+            return pack_int4(table[i]).to(w.device)
         i = torch.randint(0, table.numel(), tuple(w.shape), generator=g)
-        return (table[i] if int8 else table[i].view(torch.float8_e4m3fn)).to(w.device)
+        return (table[i] if ints else table[i].view(torch.float8_e4m3fn)).to(w.device)
 
     def full(s):
         return None if s is None else torch.full_like(s, scale)
@@ -271,7 +283,8 @@ def with_weight_codes(inp: LayerInputs, codes, scale: float, seed: int) -> Layer
 
 def to_storage_numpy(t: torch.Tensor | None) -> np.ndarray | None:
     """Host copy in storage form: float32 as is, bf16 as uint16 bit patterns,
-    float8_e4m3fn as uint8 codes, int8 as int8 (marshalling only, no arithmetic)."""
+    float8_e4m3fn as uint8 codes, int8 as int8, packed int4 bytes as uint8
+    (marshalling only, no arithmetic)."""
     if t is None:
         return None
     t = t.detach().contiguous().cpu()
@@ -281,6 +294,6 @@ def to_storage_numpy(t: torch.Tensor | None) -> np.ndarray | None:
         return t.view(torch.int16).numpy().view(np.uint16)
     if t.dtype == torch.float8_e4m3fn:
         return t.view(torch.uint8).numpy()
-    if t.dtype in (torch.int8, torch.int32, torch.int64):
+    if t.dtype in (torch.int8, torch.uint8, torch.int32, torch.int64):
         return t.numpy()
     raise TypeError(f"no storage mapping for {t.dtype}")

@@ -33,12 +33,12 @@ import torch
 
 import oracle
 from sparse_moe_transformer_router_b200.binding import L4MoE
-from sparse_moe_transformer_router_b200.workloads import LayerInputs, to_storage_numpy
+from sparse_moe_transformer_router_b200.workloads import CODED, LayerInputs, to_storage_numpy
 
 MARGIN_EXCLUDE = 1e-4
-TOL = {"f32": 2e-2, "bf16": 2e-2, "fp8": 6e-2, "int8": 6e-2}
+TOL = {"f32": 2e-2, "bf16": 2e-2, "fp8": 6e-2, "int8": 6e-2, "int4": 6e-2}
 # the type the GPU holds the hidden rows in (None: fp32 layers, TF32 products)
-HIDDEN = {"f32": None, "bf16": "bf16", "fp8": "f16", "int8": "f16"}
+HIDDEN = {"f32": None, "bf16": "bf16", "fp8": "f16", "int8": "f16", "int4": "f16"}
 # Allowance, in units of rms(oracle), beyond the output's own rounding.  The
 # GPU forms each hidden value in fp32 (tensor-core accumulation, fast exp)
 # before rounding it to the hidden type; where that fp32 value and the exact
@@ -76,7 +76,7 @@ def make_layer(inp: LayerInputs) -> L4MoE:
     layer = L4MoE(c.d_model, c.expert_ffn, c.shared_ffn, c.num_experts, c.dtype)
     if inp.bias is not None:
         layer.set_router_bias(inp.bias)
-    if c.dtype in ("fp8", "int8"):
+    if c.dtype in CODED:
         layer.set_weight_scales(inp.s_gate_up, inp.s_down, inp.ss_gate_up, inp.ss_down)
     return layer
 
@@ -159,6 +159,13 @@ def check_routing_topk(inp: LayerInputs, r: dict, k: int) -> dict:
             "counts": counts, "same": same, "o_idx": o_idx}
 
 
+def w_storage(t, dtype: str):
+    """A weight in the oracle's storage form: packed int4 bytes are viewed as
+    the oracle's int4 type, everything else as to_storage_numpy gives it."""
+    a = to_storage_numpy(t)
+    return oracle.as_int4x2(a) if dtype == "int4" and a is not None else a
+
+
 def oracle_outputs(inp: LayerInputs, tokens: np.ndarray, o_idx=None, k: int = 1,
                    chunk_experts: int = 16):
     """The oracle's exact outputs and its evaluation of the stated roundings
@@ -171,7 +178,7 @@ def oracle_outputs(inp: LayerInputs, tokens: np.ndarray, o_idx=None, k: int = 1,
     x = to_storage_numpy(inp.x)
     Wr = to_storage_numpy(inp.W_router)
     b = None if inp.bias is None else inp.bias.detach().cpu().numpy()
-    Ws_gu, Ws_dn = to_storage_numpy(inp.Ws_gate_up), to_storage_numpy(inp.Ws_down)
+    Ws_gu, Ws_dn = w_storage(inp.Ws_gate_up, c.dtype), w_storage(inp.Ws_down, c.dtype)
     E = c.num_experts
     if o_idx is None or k > 1 or E == 0:
         groups = [(tokens, set(range(E)) if o_idx is None else
@@ -187,10 +194,10 @@ def oracle_outputs(inp: LayerInputs, tokens: np.ndarray, o_idx=None, k: int = 1,
     ref_h = np.zeros_like(ref) if hidden else None
     pos = {int(t): i for i, t in enumerate(tokens)}
     for toks, need in groups:
-        Wgu = [to_storage_numpy(inp.W_gate_up[e]) if e in need else None for e in range(E)]
-        Wdn = [to_storage_numpy(inp.W_down[e]) if e in need else None for e in range(E)]
+        Wgu = [w_storage(inp.W_gate_up[e], c.dtype) if e in need else None for e in range(E)]
+        Wdn = [w_storage(inp.W_down[e], c.dtype) if e in need else None for e in range(E)]
         kw = {}
-        if c.dtype in ("fp8", "int8"):
+        if c.dtype in CODED:
             kw = dict(s_gate_up=[inp.s_gate_up[e].cpu().numpy() if e in need else None for e in range(E)],
                       s_down=[inp.s_down[e].cpu().numpy() if e in need else None for e in range(E)],
                       ss_gate_up=inp.ss_gate_up.cpu().numpy(), ss_down=inp.ss_down.cpu().numpy())

@@ -107,3 +107,20 @@ def test_a_view_at_a_checked_address_is_checked_again(monkeypatch):
     # the original tensors are accepted again (and held by the layer)
     layer._weights(gu, dn, sgu, sdn)
     assert layer._wkeep[0] is gu[0]
+
+
+def test_int4_weights_are_packed_two_per_byte(monkeypatch):
+    """int4 layers take uint8 weights packed along the output columns:
+    W_gate_up [d, F] bytes (2F codes), W_down [F, d / 2]."""
+    from sparse_moe_transformer_router_b200 import binding
+    monkeypatch.setattr(binding, "_where", lambda t, name, host=False: None)
+    layer = _layer(dtype="int4")
+    d, F, Fs, E = 64, 32, 48, 3
+    gu = [torch.zeros(d, F, dtype=torch.uint8) for _ in range(E)]
+    dn = [torch.zeros(F, d // 2, dtype=torch.uint8) for _ in range(E)]
+    sgu, sdn = torch.zeros(d, Fs, dtype=torch.uint8), torch.zeros(Fs, d // 2, dtype=torch.uint8)
+    layer._weights(gu, dn, sgu, sdn)
+    with pytest.raises(ValueError, match=r"W_gate_up\[0\] has shape"):
+        layer._weights([torch.zeros(d, 2 * F, dtype=torch.uint8)] + gu[1:], dn, sgu, sdn)  # unpacked
+    with pytest.raises(ValueError, match=r"W_down\[2\] has dtype"):
+        layer._weights(gu, dn[:2] + [dn[2].view(torch.int8)], sgu, sdn)

@@ -10,7 +10,7 @@ from parity_util import (check_outputs, check_routing, check_routing_topk, descr
                          oracle_routing, run_gpu, sample_tokens)
 from sparse_moe_transformer_router_b200.workloads import (CONFIGS, DECODE_TOKENS,
                                                           E4M3_FINITE_CODES, E4M3_SUBNORMAL_CODES,
-                                                          INT8_CODES, LayerConfig, generate,
+                                                          INT4_CODES, INT8_CODES, LayerConfig, generate,
                                                           with_weight_codes)
 
 pytestmark = pytest.mark.gpu
@@ -39,6 +39,12 @@ SMALL = {
     "int8_zipf": LayerConfig("int8_zipf", 700, 192, 16, 128, 320, "int8", router="zipf", n_dead=4,
                              wr_std=0.05),
     "int8_T1": LayerConfig("int8_T1", 1, 256, 8, 256, 256, "int8", wr_std=0.1),
+    # int4 weights (two per byte) with per-output-column scales
+    "int4_ragged": LayerConfig("int4_ragged", 300, 256, 8, 384, 256, "int4", wr_std=0.1),
+    "int4_zipf": LayerConfig("int4_zipf", 700, 192, 16, 128, 320, "int4", router="zipf", n_dead=4,
+                             wr_std=0.05),
+    "int4_T1": LayerConfig("int4_T1", 1, 256, 8, 256, 256, "int4", wr_std=0.1),
+    "int4_splitk": LayerConfig("int4_splitk", 2, 1024, 8, 1024, 1024, "int4", wr_std=0.03),
     # few tiles: split-K partials + finish kernels; T <= 128 with E % 16 == 0:
     # expert-split router with the arg-max in the permutation kernel
     "bf16_splitk": LayerConfig("bf16_splitk", 2, 1024, 8, 1024, 1024, "bf16", wr_std=0.03),
@@ -73,8 +79,10 @@ def test_small_layer_matches_oracle(name):
 
 @pytest.mark.parametrize("dtype,codes,scale", [("fp8", E4M3_FINITE_CODES, 4e-4),
                                                ("fp8", E4M3_SUBNORMAL_CODES, 20.0),
-                                               ("int8", INT8_CODES, 1.5e-3)],
-                         ids=["e4m3_all_finite_codes", "e4m3_subnormal_codes", "int8_all_codes"])
+                                               ("int8", INT8_CODES, 1.5e-3),
+                                               ("int4", INT4_CODES, 2.5e-2)],
+                         ids=["e4m3_all_finite_codes", "e4m3_subnormal_codes", "int8_all_codes",
+                              "int4_all_codes"])
 def test_weight_widening_is_exact_for_every_code(dtype, codes, scale):
     """Weights drawn from every finite E4M3 code (or from the zero and
     subnormal codes alone), or from every int8 code, with one column scale:
@@ -97,6 +105,7 @@ TOPK = {
                                  wr_std=0.05), 4),
     "fp8_k2": (LayerConfig("fp8_k2", 300, 256, 8, 384, 256, "fp8", wr_std=0.1), 2),
     "int8_k2": (LayerConfig("int8_k2", 300, 256, 8, 384, 256, "int8", wr_std=0.1), 2),
+    "int4_k2": (LayerConfig("int4_k2", 300, 256, 8, 384, 256, "int4", wr_std=0.1), 2),
     # K slices reduced in a cluster before the top-k epilogue
     "bf16_k2_kslices": (LayerConfig("bf16_k2_kslices", 700, 1024, 16, 256, 256, "bf16", wr_std=0.03), 2),
     # one token tile with E >= 32: expert-split router, top-k in the permutation
@@ -147,6 +156,7 @@ DENSE = {
     "dense_f32": LayerConfig("dense_f32", 130, 128, 0, 0, 192, "f32"),
     "dense_fp8": LayerConfig("dense_fp8", 300, 256, 0, 0, 320, "fp8"),
     "dense_int8": LayerConfig("dense_int8", 300, 256, 0, 0, 320, "int8"),
+    "dense_int4": LayerConfig("dense_int4", 300, 256, 0, 0, 320, "int4"),
     "dense_T1": LayerConfig("dense_T1", 1, 1024, 0, 0, 1024, "bf16"),
 }
 
@@ -255,7 +265,7 @@ def test_weight_pointer_change_rebuilds_descriptors():
     assert not torch.equal(out_a, out_b)
 
 
-def _full_size(cfg, seed=0):
+def _full_size(cfg, seed=0, all_tokens_up_to=4096):
     """Full-size workload: routing of every token against the oracle; outputs
     of every token when T <= 1024 (decode) or T = 4096 (Scout), else of a
     stratified sample of >= 1024 tokens covering every non-empty expert, every
@@ -265,7 +275,7 @@ def _full_size(cfg, seed=0):
     out, r = run_gpu(layer, inp)
     ora = oracle_routing(inp)
     rep = check_routing(inp, r, ora)
-    toks = np.arange(cfg.T, dtype=np.int32) if cfg.T <= 4096 else sample_tokens(r, rep, cfg.T, seed=seed)
+    toks = np.arange(cfg.T, dtype=np.int32) if cfg.T <= all_tokens_up_to else sample_tokens(r, rep, cfg.T, seed=seed)
     res = check_outputs(inp, out, toks, rep["same"], rep["o_idx"])
     print(f"{cfg.name}: {describe(res)}, excluded {rep['excluded']}, flipped {rep['flipped']}, "
           f"experts with tokens {int(np.count_nonzero(rep['counts']))}")
@@ -294,8 +304,13 @@ def test_full_size_maverick_int8_zipf():
     _full_size(CONFIGS["maverick_int8"])
 
 
-@pytest.mark.parametrize("dtype,T,E", [("fp8", 300, 8), ("int8", 5, 8), ("fp8", 3, 0), ("int8", 40, 0)],
-                         ids=["fp8_T300", "int8_T5_small_batch", "fp8_dense_T3", "int8_dense_T40"])
+def test_full_size_scout_int4():
+    _full_size(CONFIGS["scout_prefill_int4"], all_tokens_up_to=1024)
+
+
+@pytest.mark.parametrize("dtype,T,E", [("fp8", 300, 8), ("int8", 5, 8), ("fp8", 3, 0), ("int8", 40, 0),
+                                       ("int4", 64, 8)],
+                         ids=["fp8_T300", "int8_T5_small_batch", "fp8_dense_T3", "int8_dense_T40", "int4_T64"])
 def test_8bit_layers_take_inputs_beyond_f16_range(dtype, T, E):
     """E4M3 / int8 layers hold x in f16 for their contractions.  With bf16
     inputs around 1e5 (beyond f16's 65504) each token row is divided by a

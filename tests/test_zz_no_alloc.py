@@ -25,7 +25,7 @@ def _assert_same(out: torch.Tensor, ref: torch.Tensor):
     assert torch.equal(out, ref)
 
 
-@pytest.mark.parametrize("dtype", ["bf16", "f32", "fp8", "int8"])
+@pytest.mark.parametrize("dtype", ["bf16", "f32", "fp8", "int8", "int4"])
 def test_static_forward_matches_allocating_forward_on_two_calls(dtype):
     cfg = LayerConfig(f"noalloc_{dtype}", 300, 256, 8, 384, 256, dtype, wr_std=0.1)
     inp = generate(cfg, seed=11, device="cuda")
