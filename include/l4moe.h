@@ -157,9 +157,8 @@ L4MOE_API l4moe_status l4moe_set_router_bias(l4moe_handle *h, const float *bias_
  * equal values, NaN never selected), each on the input gated by the sigmoid
  * of its own logit, and their outputs add to the shared expert's (the
  * "experts per token" of a token-choice router, torchtune MoE
- * documentation).  1 <= k <= min(4, E); k > 1 needs bf16, E4M3, int8 or int4 weights and
- * E % 8 == 0 (else L4MOE_ERR_UNSUPPORTED).  The routing arrays of
- * l4moe_get_routing then hold T * k entries (entry t * k + j: token t's j-th
+ * documentation).  1 <= k <= min(4, E), any dtype and expert count.  The
+ * routing arrays of l4moe_get_routing then hold T * k entries (entry t * k + j: token t's j-th
  * expert; margin stays [T]: the k-th logit minus the next one).  Changing k
  * frees a workspace the handle allocated (it synchronises the device) and
  * fails with L4MOE_ERR_WORKSPACE when a caller's workspace is too small; the

@@ -436,7 +436,7 @@ void ensure_smem_attr(std::atomic<uint64_t>& done, K kernel, size_t bytes) {
 
 template <typename ET, int NT, int TPT, int NG>
 void launch_router_t(const void* x, const void* Wr, const float* bias, int T, int d, int E,
-                     int32_t* idx, float* gate, float* lmax, float* margin, cudaStream_t st) {
+                     int32_t* idx, float* gate, float* lmax, float* margin, int k, cudaStream_t st) {
     constexpr size_t smem = router_smem_bytes<NT, TPT, NG>();
     static std::atomic<uint64_t> attr_done{0};
     ensure_smem_attr(attr_done, router_kernel<ET, NT, TPT, NG>, smem);
@@ -444,20 +444,20 @@ void launch_router_t(const void* x, const void* Wr, const float* bias, int T, in
     const int wr_vec = (E % Vec16<ET>::N) == 0 ? 1 : 0;
     launch_k(router_kernel<ET, NT, TPT, NG>, dim3((T + TT - 1) / TT), dim3(NT), smem, st,
              static_cast<const ET*>(x), static_cast<const ET*>(Wr), bias, T, d, E, wr_vec, idx, gate,
-             lmax, margin);
+             lmax, margin, k);
 }
 
 template <typename ET>
 void launch_router(const void* x, const void* Wr, const float* bias, int T, int d, int E,
-                   int32_t* idx, float* gate, float* lmax, float* margin, cudaStream_t st) {
+                   int32_t* idx, float* gate, float* lmax, float* margin, int k, cudaStream_t st) {
     const int EG = (E + 3) / 4;
-    if (EG <= 1) launch_router_t<ET, 128, 1, 1>(x, Wr, bias, T, d, E, idx, gate, lmax, margin, st);
-    else if (EG <= 2) launch_router_t<ET, 128, 2, 1>(x, Wr, bias, T, d, E, idx, gate, lmax, margin, st);
-    else if (EG <= 4) launch_router_t<ET, 128, 4, 1>(x, Wr, bias, T, d, E, idx, gate, lmax, margin, st);
-    else if (EG <= 8) launch_router_t<ET, 128, 8, 1>(x, Wr, bias, T, d, E, idx, gate, lmax, margin, st);
-    else if (EG <= 16) launch_router_t<ET, 256, 8, 2>(x, Wr, bias, T, d, E, idx, gate, lmax, margin, st);
-    else if (EG <= 32) launch_router_t<ET, 256, 8, 4>(x, Wr, bias, T, d, E, idx, gate, lmax, margin, st);
-    else launch_router_t<ET, 256, 8, 8>(x, Wr, bias, T, d, E, idx, gate, lmax, margin, st);
+    if (EG <= 1) launch_router_t<ET, 128, 1, 1>(x, Wr, bias, T, d, E, idx, gate, lmax, margin, k, st);
+    else if (EG <= 2) launch_router_t<ET, 128, 2, 1>(x, Wr, bias, T, d, E, idx, gate, lmax, margin, k, st);
+    else if (EG <= 4) launch_router_t<ET, 128, 4, 1>(x, Wr, bias, T, d, E, idx, gate, lmax, margin, k, st);
+    else if (EG <= 8) launch_router_t<ET, 128, 8, 1>(x, Wr, bias, T, d, E, idx, gate, lmax, margin, k, st);
+    else if (EG <= 16) launch_router_t<ET, 256, 8, 2>(x, Wr, bias, T, d, E, idx, gate, lmax, margin, k, st);
+    else if (EG <= 32) launch_router_t<ET, 256, 8, 4>(x, Wr, bias, T, d, E, idx, gate, lmax, margin, k, st);
+    else launch_router_t<ET, 256, 8, 8>(x, Wr, bias, T, d, E, idx, gate, lmax, margin, k, st);
 }
 
 template <int MODE, typename ET, int WQ>
@@ -595,7 +595,7 @@ l4moe_status run_layer(l4moe_handle* h, int T, const void* x, const void* Wr, co
                       kslices == 1 ? 0u : (unsigned)kslices, m_x, m_wr, (const float*)h->bias,
                       T, d, E, n_chunk, logits, idx, gate, lmax, margin, err, k);
         } else {
-            launch_router<ET>(x, Wr, h->bias, T, d, E, idx, gate, lmax, margin, st);
+            launch_router<ET>(x, Wr, h->bias, T, d, E, idx, gate, lmax, margin, k, st);
         }
         t_router.stop();
         L4MOE_CHECK_LAUNCH("router launch");
@@ -983,9 +983,6 @@ l4moe_status l4moe_set_top_k(l4moe_handle* h, int k) {
     const int E = h->p.num_experts;
     if (k < 1 || k > kMaxTopK || (E > 0 && k > E) || (E == 0 && k != 1))
         return fail(h, L4MOE_ERR_ARG, "top_k must be in [1, min(4, E)]");
-    if (k > 1 && (h->p.dtype == L4MOE_F32 || E % 8 != 0))
-        return fail(h, L4MOE_ERR_UNSUPPORTED,
-                    "top_k > 1 takes the tensor-core router: bf16, E4M3 or int8 weights and E % 8 == 0");
     if (k == h->top_k) return L4MOE_OK;
     if (h->ws && !h->ws_owned && h->ws_bytes < ws_layout(h->p, h->ws_tokens, h->sms, k).total)
         return fail(h, L4MOE_ERR_WORKSPACE, "the caller's workspace is too small for this top_k");

@@ -12,10 +12,12 @@
 // One CTA handles TT = NT / TPT tokens; TPT threads share a token and each
 // owns NG groups of 4 consecutive experts.  x and W_router are staged through
 // shared memory in K chunks of 64 and converted to fp32; each thread keeps
-// 4 * NG fp32 accumulators (sequential fma over k).  The per-token arg-max
-// uses a strict ">" in ascending expert order inside a thread and "larger
-// value, then lower index" across threads, which is the sequential rule
-// "lowest index among the maxima; NaN never wins".
+// 4 * NG fp32 accumulators (sequential fma over k).  Each thread offers its
+// experts, in ascending order, to its own top-k list (a strict ">" keeps the
+// lower index first among equal values; NaN is never taken); the token's TPT
+// threads then take k + 1 heads in (value, then index) order with butterfly
+// shuffles -- the sequential rule "the k largest, lowest index first among
+// equal values", whose k = 1 case is the arg-max.
 #pragma once
 #include <cuda_bf16.h>
 #include <cstdint>
@@ -70,7 +72,7 @@ __global__ void __launch_bounds__(NT) router_kernel(const ET* __restrict__ x,
                                                     int E, int wr_vec, int32_t* __restrict__ idx,
                                                     float* __restrict__ gate,
                                                     float* __restrict__ lmax,
-                                                    float* __restrict__ margin) {
+                                                    float* __restrict__ margin, int topk) {
     pdl_enter();
     constexpr int TT = NT / TPT;
     constexpr int EPAD = 4 * TPT * NG;
@@ -140,46 +142,53 @@ __global__ void __launch_bounds__(NT) router_kernel(const ET* __restrict__ x,
         __syncthreads();
     }
 
-    // thread-local best / runner-up in ascending expert order
-    float best = -INFINITY, second = -INFINITY;
-    int bi = (4 * r < E) ? 4 * r : 0x7fffffff;
+    // this thread's list (its experts in ascending order)
+    TopK tk;
+    tk.init();
 #pragma unroll
     for (int j = 0; j < NG; ++j) {
 #pragma unroll
         for (int c = 0; c < 4; ++c) {
             const int e = 4 * (r + TPT * j) + c;
-            if (e < E) {
-                const float l = acc[j][c] + (bias ? bias[e] : 0.f);
-                if (l > best) {
-                    second = best;
-                    best = l;
-                    bi = e;
-                } else if (l > second) {
-                    second = l;
-                }
-            }
+            if (e < E) tk.offer(acc[j][c] + (bias ? bias[e] : 0.f), e);
         }
     }
-    // combine the TPT threads of this token (consecutive lanes)
+    // the token's TPT lists (consecutive lanes): k + 1 heads in selection order
+    TopK sel;
+    sel.init();
+    int pos = 0;  // entries of this thread's list already taken
 #pragma unroll
-    for (int off = TPT / 2; off > 0; off /= 2) {
-        const float ob = __shfl_xor_sync(0xffffffffu, best, off);
-        const float os = __shfl_xor_sync(0xffffffffu, second, off);
-        const int oi = __shfl_xor_sync(0xffffffffu, bi, off);
-        if (ob > best || (ob == best && oi < bi)) {
-            second = fmaxf(os, best);
-            best = ob;
-            bi = oi;
-        } else {
-            second = fmaxf(second, ob);
+    for (int j = 0; j <= kMaxTopK; ++j) {
+        float hv = tk.value(pos);
+        int hi = pos <= kMaxTopK ? tk.index(pos) : -1;
+        int hl = r;
+#pragma unroll
+        for (int off = TPT / 2; off > 0; off /= 2) {
+            const float ov = __shfl_xor_sync(0xffffffffu, hv, off);
+            const int oi = __shfl_xor_sync(0xffffffffu, hi, off);
+            const int ol = __shfl_xor_sync(0xffffffffu, hl, off);
+            if (topk_before(ov, oi, hv, hi)) {
+                hv = ov;
+                hi = oi;
+                hl = ol;
+            }
         }
+        sel.set(j, hv, hi);
+        if (hl == r && hi >= 0) ++pos;
     }
     const int t = t0 + tl;
     if (r == 0 && t < T) {
-        idx[t] = bi;
-        lmax[t] = best;
-        margin[t] = best - second;
-        gate[t] = 1.0f / (1.0f + expf(-best));
+        sel.fill_empty(topk);
+#pragma unroll
+        for (int j = 0; j < kMaxTopK; ++j) {
+            if (j < topk) {
+                const size_t n = (size_t)t * topk + j;
+                idx[n] = sel.index(j);
+                lmax[n] = sel.value(j);
+                gate[n] = 1.0f / (1.0f + expf(-sel.value(j)));
+            }
+        }
+        margin[t] = sel.value(topk - 1) - sel.value(topk);  // k-th against the next one
     }
 }
 

@@ -111,6 +111,13 @@ TOPK = {
     # one token tile with E >= 32: expert-split router, top-k in the permutation
     "bf16_k3_split_router": (LayerConfig("bf16_k3_sr", 40, 512, 32, 256, 384, "bf16", wr_std=0.05), 3),
     "bf16_k2_T1": (LayerConfig("bf16_k2_T1", 1, 1024, 64, 512, 512, "bf16", wr_std=0.03), 2),
+    # the CUDA-core router's top-k: fp32 layers, and expert counts that are
+    # not a multiple of 8 (one and several threads per token)
+    "f32_k2": (LayerConfig("f32_k2", 300, 256, 8, 384, 256, "f32", wr_std=0.1), 2),
+    "bf16_k3_E12": (LayerConfig("bf16_k3_E12", 300, 256, 12, 128, 256, "bf16", wr_std=0.1), 3),
+    "f32_k4_E6_zipf": (LayerConfig("f32_k4_E6_zipf", 200, 128, 6, 128, 128, "f32", router="zipf", n_dead=1,
+                                   wr_std=0.1), 4),
+    "f32_k2_E40": (LayerConfig("f32_k2_E40", 100, 128, 40, 64, 64, "f32", wr_std=0.1), 2),
     # small-batch routing at its limits: 16 tokens x 4 experts of 256
     "bf16_k4_T16_E256": (LayerConfig("bf16_k4_T16_E256", 16, 512, 256, 64, 128, "bf16", wr_std=0.05), 4),
 }
@@ -129,17 +136,13 @@ def test_topk_layer_matches_oracle(name):
 
 
 def test_top_k_bounds():
-    from sparse_moe_transformer_router_b200.binding import ERR_ARG, ERR_UNSUPPORTED, L4MoEError
+    from sparse_moe_transformer_router_b200.binding import ERR_ARG, L4MoEError
     inp = generate(TOPK["bf16_k2"][0], seed=0, device="cuda")
     layer = make_layer(inp)
     for bad in (0, 5, 9):
         with pytest.raises(L4MoEError) as ei:
             layer.set_top_k(bad)
         assert ei.value.status == ERR_ARG
-    f32 = make_layer(generate(SMALL["f32_ragged"], seed=0, device="cuda"))
-    with pytest.raises(L4MoEError) as ei:
-        f32.set_top_k(2)
-    assert ei.value.status == ERR_UNSUPPORTED
     # back to one expert per token after a top-2 forward
     layer.set_top_k(2)
     run_gpu(layer, inp)
