@@ -103,10 +103,7 @@ SplitPlan split_plan(const l4moe_params& p, int T, int sms, int k = 1) {
     const int fb_gu_r = (F + 127) / 128, fb_gu_s = (Fs + 127) / 128, fb_dn = (d + 255) / 256;
     // Tiles are striped over the CTA pairs, so the launch lasts ceil(units /
     // pairs) tile times: take the split count that fills the last wave best
-    // (fewer splits unless more fill it clearly better).  On decode batches of
-    // a Maverick-shaped layer a split gate/up launch (partials plus a finish
-    // kernel) was slower than the unsplit one whenever at least half of the
-    // pairs had a tile, so gate/up splits only below that.
+    // (fewer splits unless more fill it clearly better).
     const long long pairs = std::max(1, sms / 2);
     auto pick = [&](long long tiles, int nkb) {
         if ((size_t)T > kSplitMaxTokens || tiles <= 0) return 1;
@@ -127,7 +124,7 @@ SplitPlan split_plan(const l4moe_params& p, int T, int sms, int k = 1) {
     const long long eg = std::min<long long>(E, (long long)T * k);  // non-empty routed experts
     SplitPlan sp;
     const long long gu_tiles = (long long)fb_gu_s + fb_gu_r * eg;
-    sp.s_gu = 2 * gu_tiles < pairs ? pick(gu_tiles, d / kblk) : 1;
+    sp.s_gu = pick(gu_tiles, d / kblk);
     sp.s_dn = pick((long long)fb_dn * (eg + 1), std::min(F, Fs) / kblk);
     return sp;
 }
@@ -562,8 +559,10 @@ l4moe_status run_layer(l4moe_handle* h, int T, const void* x, const void* Wr, co
         const int slices = (d + kSmallSliceK - 1) / kSmallSliceK;
         float* part_logits = reinterpret_cast<float*>(w + L.logits);
         unsigned* ticket = err + 1;  // zero between launches (each last CTA resets it)
+        static std::atomic<uint64_t> attr_done{0};
+        ensure_smem_attr(attr_done, route_small_kernel<ET, GT>, route_small_smem_bytes<ET>(kSmallMaxTokens, 256));
         LaunchTimer t_router(h, 0, st);
-        launch_k(route_small_kernel<ET, GT>, dim3(slices), dim3(kSmallThreads), route_small_smem_bytes(T, E), st,
+        launch_k(route_small_kernel<ET, GT>, dim3(slices), dim3(kSmallThreads), route_small_smem_bytes<ET>(T, E), st,
                  static_cast<const ET*>(x), static_cast<const ET*>(Wr), (const float*)h->bias, T, d, E, k,
                  part_logits, ticket, idx, gate, lmax, margin, counts, offsets, perm, inv, gslot, tab_gu, tab_dn,
                  fb_gu_r * s_gu, fb_gu_s * s_gu, fb_dn * s_dn, xg, FP8W ? x16 : (GT*)nullptr, tokscale);

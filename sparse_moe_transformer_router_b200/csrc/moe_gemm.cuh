@@ -200,8 +200,13 @@ __host__ __device__ __forceinline__ TileInfo decode_tile(const GroupTable& tab, 
     const int rem = local - b * band * fbk;
     const int tb = b * band + rem % nb;
     const int rest = rem / nb;
-    const int split = rest % a.ksplit;
-    const int fb = rest / a.ksplit;
+    // split-K units go split-major: the units that run side by side cover
+    // different feature blocks (column bands of the weight) instead of
+    // different K rows of one band, spreading their weight stream over the
+    // memory channels
+    const int nfb = fbk / a.ksplit;  // feature blocks
+    const int fb = rest % nfb;
+    const int split = rest / nfb;
     ti.split = split;
     ti.row0 = tab.row0[g] + tb * kTokTile;
     ti.n_valid = min(kTokTile, rows - tb * kTokTile);

@@ -38,10 +38,13 @@ constexpr int kSmallSliceK = 128;    // W_router rows per CTA
 constexpr int kSmallThreads = 256;
 constexpr int kSmallMaxEntries = kSmallMaxTokens * kMaxTopK;
 
-// Dynamic shared memory: x slice [T][kSmallSliceK] fp32, then the logits
-// [T][E] fp32 (last CTA only, aliasing the x slice).
+// Dynamic shared memory: the x slice [T][kSmallSliceK] fp32 and the
+// W_router slice [kSmallSliceK][E] in its storage type (both loaded with
+// 16-byte vectors by every thread at once: one memory round trip), then the
+// logits [T][E] fp32 (last CTA only, aliasing them).
+template <typename ET>
 __host__ __device__ constexpr size_t route_small_smem_bytes(int T, int E) {
-    const size_t a = sizeof(float) * (size_t)T * kSmallSliceK;
+    const size_t a = sizeof(float) * (size_t)T * kSmallSliceK + sizeof(ET) * (size_t)kSmallSliceK * E;
     const size_t b = sizeof(float) * (size_t)T * (size_t)E;
     return a > b ? a : b;
 }
@@ -75,10 +78,29 @@ __global__ void __launch_bounds__(kSmallThreads) route_small_kernel(
     {
         const int k0 = blockIdx.x * kSmallSliceK;
         const int kn = min(kSmallSliceK, d - k0);
-        float* xs = rs_smem;  // [T][kSmallSliceK]
-        for (int i = tid; i < T * kn; i += kSmallThreads) {
-            const int t = i / kn, kk = i - t * kn;
-            xs[t * kSmallSliceK + kk] = to_f32(x[(size_t)t * d + k0 + kk]);
+        float* xs = rs_smem;                                                   // [T][kSmallSliceK]
+        ET* ws = reinterpret_cast<ET*>(rs_smem + (size_t)T * kSmallSliceK);  // [kn][E]
+        // the slice's rows of W_router are contiguous (kn * E elements): 16-byte
+        // vectors, every thread at once, then the x slice (16-byte vectors too)
+        {
+            const int V = 16 / (int)sizeof(ET);
+            const int nw = kn * E;  // E * sizeof(ET) need not be a multiple of 16: copy the flat range
+            const ET* src = Wr + (size_t)k0 * E;
+            const bool vec = ((reinterpret_cast<uintptr_t>(src) & 15u) == 0) && (nw % V == 0);
+            if (vec) {
+                for (int i = tid; i < nw / V; i += kSmallThreads)
+                    reinterpret_cast<uint4*>(ws)[i] = reinterpret_cast<const uint4*>(src)[i];
+            } else {
+                for (int i = tid; i < nw; i += kSmallThreads) ws[i] = src[i];
+            }
+            const int xv = kn / V;  // x rows: kn elements from k0 (k0, kn multiples of 64)
+            for (int i = tid; i < T * xv; i += kSmallThreads) {
+                const int t = i / xv, c = i - t * xv;
+                ET tmp[16 / sizeof(ET)];
+                *reinterpret_cast<uint4*>(tmp) = reinterpret_cast<const uint4*>(x + (size_t)t * d + k0)[c];
+#pragma unroll
+                for (int u = 0; u < V; ++u) xs[t * kSmallSliceK + c * V + u] = to_f32(tmp[u]);
+            }
         }
         __syncthreads();
         // thread -> (expert e, token group g); a group takes tokens g, g + G, ...
@@ -88,10 +110,10 @@ __global__ void __launch_bounds__(kSmallThreads) route_small_kernel(
             float acc[kSmallMaxTokens];
 #pragma unroll
             for (int j = 0; j < kSmallMaxTokens; ++j) acc[j] = 0.f;
-            const ET* wcol = Wr + (size_t)k0 * E + e;
+            const ET* wcol = ws + e;
 #pragma unroll 4
             for (int kk = 0; kk < kn; ++kk) {
-                const float w = to_f32(wcol[(size_t)kk * E]);
+                const float w = to_f32(wcol[kk * E]);
 #pragma unroll
                 for (int j = 0; j < kSmallMaxTokens; ++j) {
                     const int t = g + j * G;
@@ -115,12 +137,31 @@ __global__ void __launch_bounds__(kSmallThreads) route_small_kernel(
     __threadfence();
 
     // ---------------------------------------------- logits: slices in order, + bias
+    // each thread owns outputs i = tid + 256 q; every slice's loads are issued
+    // for all of them before they are added (independent, in flight together),
+    // and the slices are added in order
     float* lg = rs_smem;  // [T][E]
-    for (int i = tid; i < T * E; i += kSmallThreads) {
-        float v = 0.f;
-#pragma unroll 8
-        for (unsigned s = 0; s < gridDim.x; ++s) v += __ldcg(partial + (size_t)s * T * E + i);
-        lg[i] = v + (bias ? bias[i % E] : 0.f);
+    {
+        constexpr int Q = (kSmallMaxTokens * kMaxGroups + kSmallThreads - 1) / kSmallThreads;
+        const int n = T * E;
+        float v[Q];
+#pragma unroll
+        for (int q = 0; q < Q; ++q) v[q] = 0.f;
+        for (unsigned s = 0; s < gridDim.x; ++s) {
+            float ld[Q];
+#pragma unroll
+            for (int q = 0; q < Q; ++q) {
+                const int i = tid + kSmallThreads * q;
+                ld[q] = i < n ? __ldcg(partial + (size_t)s * n + i) : 0.f;
+            }
+#pragma unroll
+            for (int q = 0; q < Q; ++q) v[q] += ld[q];
+        }
+#pragma unroll
+        for (int q = 0; q < Q; ++q) {
+            const int i = tid + kSmallThreads * q;
+            if (i < n) lg[i] = v[q] + (bias ? bias[i % E] : 0.f);
+        }
     }
     __syncthreads();
     if (tid == 0) *ticket = 0u;  // every CTA has taken its ticket: ready for the next launch

@@ -217,8 +217,9 @@ constexpr size_t SMEM_BYTES = 1024 + (size_t)STAGES * STAGE_BYTES + (2 * STAGES 
 // after a cluster barrier rank 0 adds ranks 1..S-1's partials to its own in
 // slice order (deterministic) and runs the arg-max epilogue.  This spreads
 // the x stream of a batch of few token tiles over S times more SMs.
-// Each CTA's partial (fp32, column-major [n_pad][128], at most 128 KB for
-// E = 256) reuses its own operand stages.
+// Each CTA's partial (fp32, row-major [128 tokens][n_pad + 4], at most
+// 130 KB for E = 256) reuses its own operand stages; rank 0 reads a token's
+// row from each other rank with 16-byte loads issued before any is used.
 //
 // Expert-split mode (logits != null, for batches of one token tile): CTA
 // (y, z) computes experts [y*n_chunk, (y+1)*n_chunk) over K slice z of
@@ -321,74 +322,110 @@ __global__ void __launch_bounds__(128, 1)
     const bool ok = mbar_wait(done_bar, 0, err, DEV_ERR_TIMEOUT_EPILOGUE);
     const bool kreduce = gridDim.z > 1;  // K slices: always launched as clusters along z
     const uint32_t crank = kreduce ? cluster_ctarank() : 0u;
-    float* red = reinterpret_cast<float*>(smem);  // this CTA's partial, [n_pad][128] (column-major)
+    float* red = reinterpret_cast<float*>(smem);  // this CTA's partial, [128][n_pad + 4] (row-major)
+    // K-slice partials of ranks 1..S-1: row-major [128 tokens][rld] fp32 in
+    // each CTA's own (now idle) stage memory, one row per thread, so rank 0
+    // reads a row with 16-byte cluster loads, all issued before they are used
+    const int rld = n_pad + 4;
     if (kreduce) {
         // every CTA reaches both cluster barriers, whatever its waits gave
         if (crank != 0 && __all_sync(0xffffffffu, ok)) {
             tc_fence_after();
+            float* row = red + (size_t)(32 * warp + lane) * rld;
             for (int c = 0; c < n_pad; c += 32) {
                 float v[32];
                 tmem_ld_32x32(tmem_base + ((uint32_t)(32 * warp) << 16) + (uint32_t)c, v);
                 tmem_wait_ld();
 #pragma unroll
-                for (int i = 0; i < 32; ++i)
-                    if (c + i < n_pad) red[(c + i) * 128 + 32 * warp + lane] = v[i];
+                for (int i = 0; i < 32; i += 4)
+                    if (c + i < n_pad)
+                        *reinterpret_cast<float4*>(row + c + i) = make_float4(v[i], v[i + 1], v[i + 2], v[i + 3]);
             }
         }
         cluster_sync();  // partials of ranks 1..S-1 complete in their shared memory
     }
+    // the logits of this thread's token, 32 experts at a time: own partial,
+    // then slices 1..S-1 in order (a fixed order: deterministic)
+    auto logits_chunk = [&](int c, float (&v)[32]) {
+        tmem_ld_32x32(tmem_base + ((uint32_t)(32 * warp) << 16) + (uint32_t)c, v);
+        tmem_wait_ld();
+        for (uint32_t z = 1; kreduce && z < gridDim.z; ++z) {
+            const uint32_t base = mapa_shared(smem_u32(red + (size_t)(32 * warp + lane) * rld + c), z);
+            float4 r[8];
+#pragma unroll
+            for (int q = 0; q < 8; ++q)
+                r[q] = (c + 4 * q < n_pad) ? ld_shared_cluster_v4(base + 16u * q) : make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll
+            for (int q = 0; q < 8; ++q) {
+                v[4 * q] += r[q].x;
+                v[4 * q + 1] += r[q].y;
+                v[4 * q + 2] += r[q].z;
+                v[4 * q + 3] += r[q].w;
+            }
+        }
+    };
     if ((!kreduce || crank == 0) && __all_sync(0xffffffffu, ok)) {
         tc_fence_after();
         const int t = t0 + 32 * warp + lane;
         if (logits) {
             for (int c = 0; c < n_pad; c += 32) {
                 float v[32];
-                tmem_ld_32x32(tmem_base + ((uint32_t)(32 * warp) << 16) + (uint32_t)c, v);
-                tmem_wait_ld();
-                for (uint32_t z = 1; kreduce && z < gridDim.z; ++z) {  // slices in order
-                    const uint32_t base = mapa_shared(smem_u32(red + c * 128 + 32 * warp + lane), z);
-#pragma unroll
-                    for (int i = 0; i < 32; ++i)
-                        if (c + i < n_pad) v[i] += ld_shared_cluster_f32(base + 512u * i);
-                }
+                logits_chunk(c, v);
 #pragma unroll
                 for (int i = 0; i < 32; ++i) {
                     const int e = c + i;
                     if (e < ne && t < T) logits[(size_t)t * E + e0 + e] = v[i] + (bias ? bias[e0 + e] : 0.f);
                 }
             }
-        }
-        TopK tk;
-        tk.init();
-        for (int c = 0; !logits && c < n_pad; c += 32) {
-            float v[32];
-            tmem_ld_32x32(tmem_base + ((uint32_t)(32 * warp) << 16) + (uint32_t)c, v);
-            tmem_wait_ld();
-            for (uint32_t z = 1; kreduce && z < gridDim.z; ++z) {  // slices in order
-                // a warp reads 32 consecutive rows of a column: 128 B per load
-                const uint32_t base = mapa_shared(smem_u32(red + c * 128 + 32 * warp + lane), z);
+        } else if (topk == 1) {
+            // the arg-max (strict ">" in ascending order: the lowest index
+            // among the maxima; NaN never wins) and the runner-up, branch-free
+            float best = -INFINITY, second = -INFINITY;
+            int bi = 0;
+            for (int c = 0; c < n_pad; c += 32) {
+                float v[32];
+                logits_chunk(c, v);
 #pragma unroll
-                for (int i = 0; i < 32; ++i)
-                    if (c + i < n_pad) v[i] += ld_shared_cluster_f32(base + 512u * i);
-            }
-#pragma unroll
-            for (int i = 0; i < 32; ++i) {
-                const int e = c + i;
-                if (e < E) tk.offer(v[i] + (bias ? bias[e] : 0.f), e);
-            }
-        }
-        if (!logits && t < T) {
-            tk.fill_empty(topk);
-#pragma unroll
-            for (int j = 0; j < kMaxTopK; ++j) {
-                if (j < topk) {
-                    const size_t n = (size_t)t * topk + j;
-                    idx[n] = tk.index(j);
-                    lmax[n] = tk.value(j);
-                    gate[n] = 1.0f / (1.0f + expf(-tk.value(j)));
+                for (int i = 0; i < 32; ++i) {
+                    const int e = c + i;
+                    const float l = e < E ? v[i] + (bias ? bias[e] : 0.f) : -INFINITY;
+                    const bool gt = l > best;
+                    second = gt ? best : fmaxf(second, l);
+                    bi = gt ? e : bi;
+                    best = gt ? l : best;
                 }
             }
-            margin[t] = tk.value(topk - 1) - tk.value(topk);  // k-th against the next one
+            if (t < T) {
+                idx[t] = bi;
+                lmax[t] = best;
+                gate[t] = 1.0f / (1.0f + expf(-best));
+                margin[t] = best - second;
+            }
+        } else {
+            TopK tk;
+            tk.init();
+            for (int c = 0; c < n_pad; c += 32) {
+                float v[32];
+                logits_chunk(c, v);
+#pragma unroll
+                for (int i = 0; i < 32; ++i) {
+                    const int e = c + i;
+                    if (e < E) tk.offer(v[i] + (bias ? bias[e] : 0.f), e);
+                }
+            }
+            if (t < T) {
+                tk.fill_empty(topk);
+#pragma unroll
+                for (int j = 0; j < kMaxTopK; ++j) {
+                    if (j < topk) {
+                        const size_t n = (size_t)t * topk + j;
+                        idx[n] = tk.index(j);
+                        lmax[n] = tk.value(j);
+                        gate[n] = 1.0f / (1.0f + expf(-tk.value(j)));
+                    }
+                }
+                margin[t] = tk.value(topk - 1) - tk.value(topk);  // k-th against the next one
+            }
         }
     }
     if (kreduce) cluster_sync();  // rank 0 done reading the others' shared memory
