@@ -66,11 +66,6 @@ bool encode_2d(CUtensorMap* m, CUtensorMapDataType dt, const void* base, uint64_
                CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-// The small-batch routing kernel's shared memory must fit one CTA (it grows
-// with d: the x rows of a cluster rank's share of W_router); wider layers
-// take the separate router, permutation and row copy.
-constexpr size_t kMaxSmallSmem = 220u << 10;
-
 // Split-K is used for batches of at most this many tokens, into at most
 // kMaxSplit k-ranges (tiles too few to fill the GPU, e.g. decode).
 constexpr size_t kSplitMaxTokens = 64;
@@ -166,7 +161,7 @@ WsLayout ws_layout(const l4moe_params& p, int T, int sms, int k) {
     };
     const size_t t = (size_t)std::max(T, 1), E = (size_t)p.num_experts, es = act_bytes(p.dtype);
     const size_t tv = t * (size_t)k;
-    L.err = take(256);  // device error word, then the dispatch kernel's ticket (zeroed once)
+    L.err = take(256);  // device error word, then the routing kernels' ticket (zeroed once)
     L.idx = take(4 * tv);
     L.gate = take(4 * tv);
     L.lmax = take(4 * tv);
@@ -186,7 +181,11 @@ WsLayout ws_layout(const l4moe_params& p, int T, int sms, int k) {
     L.x16 = take(coded8(p.dtype) ? t * p.d_model * 2 : 0);
     L.xsc = take(coded8(p.dtype) ? 4 * t : 0);  // and each token row's power-of-two scale
     L.part = take(sizeof(float) * part_floats(p, (int)t, sms, k));
-    L.logits = take(sizeof(float) * std::min<size_t>(t, 128) * E);  // expert-split router
+    // expert-split router logits [min(T, 128)][E]; for batches the one-launch
+    // routing takes, its partial logits [slices][T][E]
+    const size_t small_part = (size_t)((p.d_model + kSmallSliceK - 1) / kSmallSliceK) *
+                              std::min<size_t>(t, kSmallMaxTokens) * E;
+    L.logits = take(sizeof(float) * std::max(std::min<size_t>(t, 128) * E, small_part));
     L.device_total = off;
     L.xin = take(2 * t * p.d_model * es);   // host path: two input staging slots
     L.xout = take(2 * t * p.d_model * es);  // and two output staging slots
@@ -559,16 +558,18 @@ l4moe_status run_layer(l4moe_handle* h, int T, const void* x, const void* Wr, co
     // split-K k-ranges when a small batch leaves too few tiles
     const SplitPlan plan = split_plan(p, T, h->sms, h->top_k);
     const int s_gu = plan.s_gu, s_dn = plan.s_dn;
-    if (E > 0 && T <= kSmallMaxTokens && route_small_smem_bytes<ET>(kSmallMaxTokens, 256, d) <= kMaxSmallSmem) {
+    if (E > 0 && T <= kSmallMaxTokens) {
         // a few tokens: router, top-k, permutation and row copy in one launch
+        const int slices = (d + kSmallSliceK - 1) / kSmallSliceK;
+        float* part_logits = reinterpret_cast<float*>(w + L.logits);
+        unsigned* ticket = err + 1;  // zero between launches (each last CTA resets it)
         static std::atomic<uint64_t> attr_done{0};
-        ensure_smem_attr(attr_done, route_small_kernel<ET, GT>, route_small_smem_bytes<ET>(kSmallMaxTokens, 256, d));
+        ensure_smem_attr(attr_done, route_small_kernel<ET, GT>, route_small_smem_bytes<ET>(kSmallMaxTokens, 256));
         LaunchTimer t_router(h, 0, st);
-        launch_kc(route_small_kernel<ET, GT>, dim3(1, 1, kSmallCluster), dim3(kSmallThreads),
-                  route_small_smem_bytes<ET>(T, E, d), st, (unsigned)kSmallCluster, static_cast<const ET*>(x),
-                  static_cast<const ET*>(Wr), (const float*)h->bias, T, d, E, k, idx, gate, lmax, margin, counts,
-                  offsets, perm, inv, gslot, tab_gu, tab_dn, fb_gu_r * s_gu, fb_gu_s * s_gu, fb_dn * s_dn, xg,
-                  FP8W ? x16 : (GT*)nullptr, tokscale);
+        launch_k(route_small_kernel<ET, GT>, dim3(slices), dim3(kSmallThreads), route_small_smem_bytes<ET>(T, E), st,
+                 static_cast<const ET*>(x), static_cast<const ET*>(Wr), (const float*)h->bias, T, d, E, k,
+                 part_logits, ticket, idx, gate, lmax, margin, counts, offsets, perm, inv, gslot, tab_gu, tab_dn,
+                 fb_gu_r * s_gu, fb_gu_s * s_gu, fb_dn * s_dn, xg, FP8W ? x16 : (GT*)nullptr, tokscale);
         t_router.stop();
         L4MOE_CHECK_LAUNCH("small-batch routing launch");
     } else if (E > 0) {
@@ -876,7 +877,7 @@ l4moe_status l4moe_forward_static(l4moe_handle* h, int T, const void* x, const v
     // the state a forward expects to start at zero
     cudaError_t e = cudaMemcpyAsync(maps, h->h_maps.data(), maps_bytes, cudaMemcpyHostToDevice, st);
     if (e != cudaSuccess) return cuda_fail(h, e, "static descriptor upload");
-    // the error word and the dispatch kernel's ticket that follows it
+    // the error word and the routing kernels' ticket that follows it
     e = cudaMemsetAsync(base + ws_layout(h->p, T, h->sms, h->top_k).err, 0, 2 * sizeof(unsigned), st);
     if (e != cudaSuccess) return cuda_fail(h, e, "static error word clear");
     const float* const* scales = nullptr;

@@ -145,14 +145,13 @@ struct GemmCfg {
     static constexpr int A_BOX_BYTES = C::BK * 128;          // BK rows x 128 B
     static constexpr int B_BOX_ROWS = 128;                   // token rows per full-tile box
     static constexpr int B_SMALL_ROWS = 32;                  // token rows per small-tile box
-    static constexpr int B_ACC_BYTES = (kAccTokens / 2) * 128;  // this CTA's half of one accumulator's tokens
-    static constexpr int B_BYTES = 2 * B_ACC_BYTES;                // both accumulators
+    static constexpr int B_BYTES = (kTokTile / 2) * 128;     // this CTA's half of the tokens
     // raw coded weights: 2 slabs x 64 K rows x 64 features, one byte per code
     // (half a byte for int4: two codes per byte along the features)
     static constexpr int RAW_SLAB_BYTES = WQ == kWqInt4 ? 64 * 32 : 64 * 64;
     static constexpr int RAW_BYTES = FP8W ? 2 * RAW_SLAB_BYTES : 0;
     static constexpr int STAGE_BYTES = A_BYTES + B_BYTES + RAW_BYTES;
-    static constexpr int STAGES = (WQ == kWqE4M3 || WQ == kWqInt8) ? 3 : 4;
+    static constexpr int STAGES = FP8W ? 5 : 6;
     static constexpr int ACC_BUFS = 2;
     static constexpr int TMEM_COLS = 512;
     static constexpr int CONV_WARPS = FP8W ? 8 : 0;         // E4M3 widening warps (6..13)
@@ -164,10 +163,8 @@ struct GemmCfg {
                                          XCH_BYTES + NUM_BARS * 8 + 16 + sizeof(GroupTable);
 };
 
-// A tile's tokens: [0, 256) go to the first accumulator (N = n_mma), the
-// rest, if any, to the second (N = n_mma1; 0 when the tile has <= 256 tokens).
 struct TileInfo {
-    int expert, row0, n_valid, n_mma, n_mma1, f0, K, M, up_off;
+    int expert, row0, n_valid, n_mma, f0, K, M, up_off;
     int split, kb0, kb1;  // k-block range [kb0, kb1) of this tile's split
     bool shared;
 };
@@ -213,8 +210,7 @@ __host__ __device__ __forceinline__ TileInfo decode_tile(const GroupTable& tab, 
     ti.split = split;
     ti.row0 = tab.row0[g] + tb * kTokTile;
     ti.n_valid = min(kTokTile, rows - tb * kTokTile);
-    ti.n_mma = (min(ti.n_valid, kAccTokens) + 15) & ~15;
-    ti.n_mma1 = ti.n_valid > kAccTokens ? ((ti.n_valid - kAccTokens + 15) & ~15) : 0;
+    ti.n_mma = (ti.n_valid + 15) & ~15;
     ti.f0 = fb * pair_features<MODE>();
     ti.M = ti.shared ? a.m_shared : a.m_routed;
     ti.up_off = ti.shared ? a.up_shared : a.up_routed;
@@ -400,22 +396,15 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(GemmCfg<MODE, ET, WQ
             for (int L = pair; L < total && !aborted; L += npairs) {
                 const TileInfo ti = decode_tile<MODE, C::BK, C::BYTES>(*tab, args, L);
                 const CUtensorMap* amap = args.a_maps + ti.expert;
-                // token operand of each accumulator: this CTA's half of its
-                // tokens, as one 128-row box or 32-row boxes
-                const void* bmap[2];
-                int brows[2], nbb[2], brow[2];
-                uint32_t tx_cta = FP8W ? 0u : (uint32_t)Cfg::A_BYTES;
-#pragma unroll
-                for (int a = 0; a < 2; ++a) {
-                    const int half = (a ? ti.n_mma1 : ti.n_mma) >> 1;  // tokens per CTA
-                    const bool big = half > 2 * Cfg::B_SMALL_ROWS;
-                    bmap[a] = ti.shared ? (big ? (const void*)&bm.shared : (const void*)&bm.shared_small)
-                                        : (big ? (const void*)&bm.routed : (const void*)&bm.routed_small);
-                    brows[a] = big ? Cfg::B_BOX_ROWS : Cfg::B_SMALL_ROWS;
-                    nbb[a] = (half + brows[a] - 1) / brows[a];
-                    brow[a] = ti.row0 + kAccTokens * a + (int)rank * half;
-                    tx_cta += (uint32_t)(nbb[a] * brows[a] * 128);
-                }
+                const int half = ti.n_mma >> 1;  // tokens per CTA
+                const bool big = half > 2 * Cfg::B_SMALL_ROWS;
+                const void* bmap = ti.shared ? (big ? (const void*)&bm.shared : (const void*)&bm.shared_small)
+                                             : (big ? (const void*)&bm.routed : (const void*)&bm.routed_small);
+                const int brows = big ? Cfg::B_BOX_ROWS : Cfg::B_SMALL_ROWS;
+                const int nbb = (half + brows - 1) / brows;
+                const uint32_t tx_cta =
+                    (FP8W ? 0u : (uint32_t)Cfg::A_BYTES) + (uint32_t)(nbb * brows * 128);
+                const int brow = ti.row0 + (int)rank * half;
                 // this CTA's A columns: gate/up -> [gate 64 | up 64] of features
                 // f0 + 64*rank; down -> 128 features f0 + 128*rank
                 const int acol0 =
@@ -457,11 +446,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(GemmCfg<MODE, ET, WQ
                         }
                     }
                     const uint32_t bb = sb + Cfg::A_BYTES;
-#pragma unroll
-                    for (int a = 0; a < 2; ++a)
-                        for (int j = 0; j < nbb[a]; ++j)
-                            tma_load_2d_pair(bb + (uint32_t)(a * Cfg::B_ACC_BYTES + j * brows[a] * 128), bmap[a],
-                                             fb_leader, k, brow[a] + j * brows[a]);
+                    for (int j = 0; j < nbb; ++j)
+                        tma_load_2d_pair(bb + (uint32_t)(j * brows * 128), bmap, fb_leader, k,
+                                         brow + j * brows);
                     used |= 1u << stage;
                     last_par = (last_par & ~(1u << stage)) | (phase << stage);
                     if (++stage == Cfg::STAGES) {
@@ -490,28 +477,16 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(GemmCfg<MODE, ET, WQ
             // ------------------------------------------------ MMA issuer (leader)
             int stage = 0;
             uint32_t phase = 0;
-            // TMEM: two 256-column accumulator buffers.  A tile of <= 256
-            // tokens takes the next buffer in turn (its epilogue overlaps the
-            // next tile's MMAs); a wider tile takes both (columns = its tokens).
-            int nb = 0;
-            uint32_t use_par = 0u;  // bit b: parity of the times buffer b was taken
+            int acc = 0;
+            uint32_t acc_phase = 0;
             for (int L = pair; L < total; L += npairs) {
                 const TileInfo ti = decode_tile<MODE, C::BK, C::BYTES>(*tab, args, L);
-                const bool wide = ti.n_mma1 > 0;
-                const int b0 = wide ? 0 : nb;
-                bool free_ = mbar_wait_cluster(tempty_bar(b0), ((use_par >> b0) & 1u) ^ 1u, args.err,
-                                               DEV_ERR_TIMEOUT_MMA);
-                if (free_ && wide)
-                    free_ = mbar_wait_cluster(tempty_bar(1), ((use_par >> 1) & 1u) ^ 1u, args.err, DEV_ERR_TIMEOUT_MMA);
-                if (!free_) break;
-                use_par ^= wide ? 3u : (1u << b0);
-                nb = wide ? 0 : (nb ^ 1);
+                if (!mbar_wait_cluster(tempty_bar(acc), acc_phase ^ 1u, args.err, DEV_ERR_TIMEOUT_MMA))
+                    break;
                 tc_fence_after();
-                // coded-weight layers: both operands f16 (format 0), else the layer's type
+                // E4M3 layers: both operands f16 (format 0), else the layer's type
                 const uint32_t idesc = make_idesc(FP8W ? 0u : C::FMT, 1u, 0u, (uint32_t)ti.n_mma, 256u);
-                const uint32_t idesc1 = make_idesc(FP8W ? 0u : C::FMT, 1u, 0u, wide ? (uint32_t)ti.n_mma1 : 16u, 256u);
-                const uint32_t d_tmem = tmem_base + (uint32_t)b0 * 256u;
-                const uint32_t d_tmem1 = tmem_base + 256u;
+                const uint32_t d_tmem = tmem_base + (uint32_t)acc * 256u;
                 bool ok = true;
                 for (int kb = ti.kb0; kb < ti.kb1; ++kb) {
                     if (!mbar_wait(full_bar(stage), phase, args.err, DEV_ERR_TIMEOUT_MMA)) {
@@ -537,13 +512,6 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(GemmCfg<MODE, ET, WQ
                             mma_bf16_pair(d_tmem, adesc, bdesc, idesc, accum);
                         else
                             mma_tf32_pair(d_tmem, adesc, bdesc, idesc, accum);
-                        if (wide) {  // the same weight stage against the second block of tokens
-                            const uint64_t bdesc1 = smem_desc(bb + Cfg::B_ACC_BYTES + kk * 32, 16, 1024, 2);
-                            if constexpr (C::FMT == 1)
-                                mma_bf16_pair(d_tmem1, adesc, bdesc1, idesc1, accum);
-                            else
-                                mma_tf32_pair(d_tmem1, adesc, bdesc1, idesc1, accum);
-                        }
                     }
                     mma_commit_pair_mc(empty_bar(stage), 0x3);  // frees the stage in both CTAs
                     if (++stage == Cfg::STAGES) {
@@ -552,7 +520,11 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(GemmCfg<MODE, ET, WQ
                     }
                 }
                 if (!ok) break;
-                mma_commit_pair_mc(tfull_bar(b0), 0x3);  // accumulator(s) ready in both CTAs
+                mma_commit_pair_mc(tfull_bar(acc), 0x3);  // accumulator ready in both CTAs
+                if (++acc == Cfg::ACC_BUFS) {
+                    acc = 0;
+                    acc_phase ^= 1u;
+                }
             }
             // every issued MMA must finish before the pair releases TMEM
             mma_commit_pair(drain_bar);
@@ -607,19 +579,12 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(GemmCfg<MODE, ET, WQ
     } else {
         // ---------------------------------------------------- epilogue
         const int q = warp & 3;  // TMEM lane quarter of this warp
-        // the MMA issuer's buffer sequence (see there): a tile of <= 256
-        // tokens fills the next buffer in turn, a wider one both (signalled
-        // on buffer 0)
-        int nb = 0;
-        uint32_t fill_par = 0u;  // bit b: parity of the times buffer b was filled
+        int acc = 0;
+        uint32_t acc_phase = 0;
         volatile uint32_t* abort_flag = misc + 1;
         for (int L = pair; L < total; L += npairs) {
             const TileInfo ti = decode_tile<MODE, C::BK, C::BYTES>(*tab, args, L);
-            const bool wide = ti.n_mma1 > 0;
-            const int b0 = wide ? 0 : nb;
-            nb = wide ? 0 : (nb ^ 1);
-            const bool ok = mbar_wait(tfull_bar(b0), (fill_par >> b0) & 1u, args.err, DEV_ERR_TIMEOUT_EPILOGUE);
-            fill_par ^= 1u << b0;
+            const bool ok = mbar_wait(tfull_bar(acc), acc_phase, args.err, DEV_ERR_TIMEOUT_EPILOGUE);
             if constexpr (MODE == MODE_GATEUP) {
                 // the 4 warps meet at named barriers below: leave together or not at all
                 if (!__all_sync(0xffffffffu, ok) && lane == 0) *abort_flag = 1u;
@@ -629,8 +594,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(GemmCfg<MODE, ET, WQ
                 if (!__all_sync(0xffffffffu, ok)) break;
             }
             tc_fence_after();
-            // TMEM column = the token's position in the tile (wide tiles from column 0)
-            const uint32_t tb = tmem_base + ((uint32_t)(q * 32) << 16) + (uint32_t)b0 * 256u;
+            const uint32_t tb = tmem_base + ((uint32_t)(q * 32) << 16) + (uint32_t)acc * 256u;
             using OT = typename GemmAct<ET, FP8W>::type;  // hidden rows (gate/up's output)
             OT* outp = reinterpret_cast<OT*>(ti.shared ? args.out_shared : args.out_routed);
             const long long ld = ti.shared ? args.ld_shared : args.ld_routed;
@@ -682,9 +646,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(GemmCfg<MODE, ET, WQ
                 }
                 tc_fence_before();
                 __syncwarp();
-                if (lane == 0) {
-                    mbar_arrive_remote(mapa_shared(tempty_bar(b0), 0));
-                    if (wide) mbar_arrive_remote(mapa_shared(tempty_bar(1), 0));
+                if (lane == 0) mbar_arrive_remote(mapa_shared(tempty_bar(acc), 0));
+                if (++acc == Cfg::ACC_BUFS) {
+                    acc = 0;
+                    acc_phase ^= 1u;
                 }
                 continue;
             }
@@ -747,9 +712,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(GemmCfg<MODE, ET, WQ
             }
             tc_fence_before();
             __syncwarp();
-            if (lane == 0) {  // to the leader
-                mbar_arrive_remote(mapa_shared(tempty_bar(b0), 0));
-                if (wide) mbar_arrive_remote(mapa_shared(tempty_bar(1), 0));
+            if (lane == 0) mbar_arrive_remote(mapa_shared(tempty_bar(acc), 0));  // to the leader
+            if (++acc == Cfg::ACC_BUFS) {
+                acc = 0;
+                acc_phase ^= 1u;
             }
         }
     }

@@ -10,10 +10,7 @@ namespace l4moe {
 // group are (feature block) x (token block); group g holds
 // ceil(rows/kTokTile) * feature_blocks tiles.
 constexpr int kMaxGroups = 257;  // 256 routed experts + the shared expert
-// Tokens per GEMM tile (the MMA's N, swap-AB): up to two accumulators of at
-// most 256 tokens each that share the tile's weight (A) stages.
-constexpr int kTokTile = 512;
-constexpr int kAccTokens = 256;  // tokens per accumulator (largest MMA N)
+constexpr int kTokTile = 256;    // tokens per GEMM tile (MMA N, swap-AB)
 
 // Groups are listed in two runs: first the "heavy" groups (at least
 // kHeavyRows rows: enough tokens per weight tile that the tensor cores, not

@@ -54,6 +54,10 @@ bool check(const l4moe_params& p, int Tmax, int k, int sms) {
     if (coded8(p.dtype) && size_of(L.xsc) < 4 * t) return fail_case("row scales too small", p, Tmax, k, sms);
     if (E && size_of(L.logits) < 4 * std::min<size_t>(t, 128) * E)
         return fail_case("router logits too small", p, Tmax, k, sms);
+    // the small-batch routing's partial logits [slices][T][E] for T <= kSmallMaxTokens
+    const size_t slices = (d + kSmallSliceK - 1) / kSmallSliceK;
+    if (E && size_of(L.logits) < 4 * slices * std::min<size_t>(t, kSmallMaxTokens) * E)
+        return fail_case("small-batch partial logits too small", p, Tmax, k, sms);
     // the dispatch's chunk bases [chunks][E]
     if (E && size_of(L.chunk) < 4 * ((tv + kDispatchChunk - 1) / kDispatchChunk) * E)
         return fail_case("dispatch chunk bases too small", p, Tmax, k, sms);

@@ -84,11 +84,8 @@ static bool run_case(std::mt19937& rng, int c) {
         const int rel = ti.row0 - (g >= 0 ? tab.row0[g] : 0);
         const int nkb = (sh ? K_s : K_r) / BK;
         const bool ok = g >= 0 && ti.shared == sh && rel >= 0 && rel % kTokTile == 0 && rel < tab.rows[g] &&
-                        ti.n_valid == std::min(kTokTile, tab.rows[g] - rel) &&
-                        ti.n_mma + ti.n_mma1 >= ti.n_valid && ti.n_mma % 16 == 0 && ti.n_mma1 % 16 == 0 &&
-                        ti.n_mma <= kAccTokens && ti.n_mma1 <= kAccTokens &&
-                        (ti.n_mma1 > 0) == (ti.n_valid > kAccTokens) &&
-                        (ti.n_mma1 == 0 || ti.n_mma == kAccTokens) && ti.f0 >= 0 && ti.f0 % pair_features<MODE>() == 0 &&
+                        ti.n_valid == std::min(kTokTile, tab.rows[g] - rel) && ti.n_mma >= ti.n_valid &&
+                        ti.n_mma % 16 == 0 && ti.n_mma <= kTokTile && ti.f0 >= 0 && ti.f0 % pair_features<MODE>() == 0 &&
                         ti.f0 < (sh ? M_s : M_r) && ti.split >= 0 && ti.split < ksplit &&
                         ti.kb0 == (int)((long long)nkb * ti.split / ksplit) &&
                         ti.kb1 == (int)((long long)nkb * (ti.split + 1) / ksplit) && ti.K == (sh ? K_s : K_r) &&
