@@ -396,6 +396,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(GemmCfg<MODE, ET, WQ
             for (int L = pair; L < total && !aborted; L += npairs) {
                 const TileInfo ti = decode_tile<MODE, C::BK, C::BYTES>(*tab, args, L);
                 const CUtensorMap* amap = args.a_maps + ti.expert;
+                // the next tile's weight descriptor, fetched while this tile streams
+                // (split-K units and small groups change expert every few k-blocks)
+                if (L + npairs < total)
+                    tma_prefetch_desc(args.a_maps + decode_tile<MODE, C::BK, C::BYTES>(*tab, args, L + npairs).expert);
                 const int half = ti.n_mma >> 1;  // tokens per CTA
                 const bool big = half > 2 * Cfg::B_SMALL_ROWS;
                 const void* bmap = ti.shared ? (big ? (const void*)&bm.shared : (const void*)&bm.shared_small)
