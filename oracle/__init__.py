@@ -228,7 +228,9 @@ def forward(x, Wr, W_gate_up, W_down, Ws_gate_up, Ws_down, *, bias=None,
     own logit, and their outputs add to the shared expert's.  Returns
     (out f64[n_sel, d], idx int32[n_sel], gate f64[n_sel]), or [n_sel, k]
     index and gate arrays for k > 1.  act_fp8: the FP8 activation mode (every
-    contraction input row quantised to E4M3 with its own fp32 scale).
+    contraction input row quantised to E4M3 with its own fp32 scale; a hidden
+    row is first held in the layer's activation type, bf16 for bf16 inputs;
+    the hidden-rounding output then equals the plain one).
     hidden_round ("bf16" or "f16"): also return, as a fourth element, the
     same outputs with every hidden value rounded to that type (through fp32)
     before the down projection -- the roundings a GPU that keeps the hidden

@@ -45,9 +45,11 @@
  *     contraction input row -- a token's x, and a token's hidden row of each
  *     expert it runs -- is quantised to E4M3 with its own scale:
  *     s = fp32(max|v| / 448) (1 for an all-zero row), code =
- *     e4m3_rne_satfinite(fp32(v / s)), value = code * s.  The hidden rows
- *     are rounded to fp32 before they are quantised.  The gate still scales
- *     the routed expert's (dequantised) input.
+ *     e4m3_rne_satfinite(fp32(v / s)), value = code * s.  A hidden row is
+ *     held in the layer's activation type before it is quantised: each
+ *     value is rounded to fp32 and then, in layers with bf16 activations, to
+ *     bf16 (round to nearest even).  The gate still scales the routed
+ *     expert's (dequantised) input.
  *   - int4 weights (superteams.ai glossary, "The Llama 4 Herd": Scout fits on
  *     one H100 quantized to int4; aibase model card, "Quantization": on-the-fly
  *     int4) are two's-complement 4-bit integers packed two per byte along the
@@ -289,7 +291,7 @@ static void route_token_topk(int d, int E, int k, const void *x_t, int x_dtype,
 static void swiglu_ffn_accumulate(int d, int Fw, const double *u,
                                   const void *Wgu, const void *Wd, int w_dtype,
                                   const float *s_gu, const float *s_d, int act_fp8,
-                                  double *a, double *h, double *y,
+                                  int act_bf16, double *a, double *h, double *y,
                                   int h_round, double *yh) {
     size_t two_f = 2 * (size_t)Fw;
     for (size_t j = 0; j < two_f; ++j) a[j] = 0.0;
@@ -299,7 +301,15 @@ static void swiglu_ffn_accumulate(int d, int Fw, const double *u,
             a[j] += uk * load_weight(Wgu, w_dtype, s_gu, (size_t)k, two_f, j);
     }
     for (int j = 0; j < Fw; ++j) h[j] = silu(a[j]) * a[Fw + j];
-    if (act_fp8) quantise_row_e4m3(Fw, h);
+    if (act_fp8) {
+        /* the hidden row in the layer's activation type, then quantised; the
+         * quantised values are what the down contraction reads, so the
+         * hidden-rounding variant below has nothing left to round */
+        if (act_bf16)
+            for (int j = 0; j < Fw; ++j) h[j] = round_bf16(h[j]);
+        quantise_row_e4m3(Fw, h);
+        h_round = HROUND_NONE;
+    }
     for (int j = 0; j < Fw; ++j) {
         double hj = h[j];
         for (int n = 0; n < d; ++n)
@@ -369,6 +379,7 @@ int oracle_forward(int T, int d, int E, int k, int F, int Fs,
                    int n_sel, const int32_t *sel, double *out,
                    int32_t *sel_idx, double *sel_gate, int h_round, double *out_h) {
     size_t xs = (x_dtype == ORACLE_F32) ? 4 : 2;
+    const int act_bf16 = x_dtype == ORACLE_BF16; /* the layer's activations are bf16 */
     int missing = 0;
     (void)T;
 #pragma omp parallel for schedule(dynamic, 1) reduction(| : missing)
@@ -390,7 +401,7 @@ int oracle_forward(int T, int d, int E, int k, int F, int Fs,
         double *xq = (double *)malloc(sizeof(double) * (size_t)d);
         for (int k = 0; k < d; ++k) xq[k] = u[k];
         swiglu_ffn_accumulate(d, Fs, u, Ws_gate_up, Ws_down, w_dtype,
-                              ss_gate_up, ss_down, act_fp8, a, h, y, h_round, yh);
+                              ss_gate_up, ss_down, act_fp8, act_bf16, a, h, y, h_round, yh);
         if (E == 0) {
             if (sel_idx) sel_idx[i] = -1;
             if (sel_gate) sel_gate[i] = 0.0;
@@ -420,7 +431,7 @@ int oracle_forward(int T, int d, int E, int k, int F, int Fs,
             for (int kk = 0; kk < d; ++kk) u[kk] = g * xq[kk];
             swiglu_ffn_accumulate(d, F, u, W_gate_up[e], W_down[e], w_dtype,
                                   s_gate_up ? s_gate_up[e] : NULL,
-                                  s_down ? s_down[e] : NULL, act_fp8, a, h, y, h_round, yh);
+                                  s_down ? s_down[e] : NULL, act_fp8, act_bf16, a, h, y, h_round, yh);
         }
         free(u);
         free(xq);
@@ -448,7 +459,7 @@ void oracle_expert_rows(int n, int d, int F, const void *x, int x_dtype, const d
         double *y = out + (size_t)i * (size_t)d;
         for (int k = 0; k < d; ++k) u[k] = g[i] * load_elem(x_i, x_dtype, (size_t)k);
         for (int k = 0; k < d; ++k) y[k] = 0.0;
-        swiglu_ffn_accumulate(d, F, u, W_gate_up, W_down, w_dtype, s_gate_up, s_down, 0, a, h, y,
+        swiglu_ffn_accumulate(d, F, u, W_gate_up, W_down, w_dtype, s_gate_up, s_down, 0, 0, a, h, y,
                               HROUND_NONE, NULL);
         free(u);
         free(a);

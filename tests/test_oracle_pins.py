@@ -460,22 +460,31 @@ def _e4m3_rows(v64: np.ndarray) -> np.ndarray:
     return (q.double() * s.double()).numpy()
 
 
+def _bf16_rows(v64: np.ndarray) -> np.ndarray:
+    """Values rounded to fp32, then to bf16, by torch's casts (fp64)."""
+    return torch.from_numpy(np.ascontiguousarray(v64)).float().bfloat16().double().numpy()
+
+
 def test_fp8_activation_mode_is_the_layer_on_e4m3_rows():
     """FP8 activation mode: the layer equals a library evaluation where x and
     every hidden row (shared and routed) are quantised per row by torch's
-    float8 cast with the same fp32 scale arithmetic, and the gate scales the
-    routed expert's quantised input."""
+    float8 cast with the same fp32 scale arithmetic, each hidden row first
+    rounded to bf16 (the layer's activation type) by torch's casts, and the
+    gate scales the routed expert's quantised input.  The hidden-rounding
+    output has nothing more to round and equals the plain one."""
     rng = np.random.default_rng(22)
     T, d, E, F, Fs = 7, 64, 3, 32, 48
     L = _layer(rng, T, d, E, F, Fs, "bf16", wstd=0.2)
-    out, idx, gate = oracle.forward(L["x"], L["Wr"], L["Wgu"], L["Wd"], L["Wsgu"], L["Wsd"], act_fp8=True)
+    out, idx, gate, out_h = oracle.forward(L["x"], L["Wr"], L["Wgu"], L["Wd"], L["Wsgu"], L["Wsd"],
+                                           act_fp8=True, hidden_round="bf16")
+    assert np.array_equal(out, out_h)
     xq = _e4m3_rows(L["x64"])
 
     def ffn(u, Wgu, Wd):
         a = u @ Wgu
         Fw = Wd.shape[0]
         h = torch.nn.functional.silu(torch.from_numpy(a[:, :Fw])).numpy() * a[:, Fw:]
-        return _e4m3_rows(h) @ Wd
+        return _e4m3_rows(_bf16_rows(h)) @ Wd
 
     ref = ffn(xq, L["Wsgu64"], L["Wsd64"])
     for t in range(T):
@@ -515,7 +524,7 @@ def test_fp8_activation_mode_keeps_rows_already_in_e4m3():
         a = u @ A
         Fw = B.shape[0]
         h = torch.nn.functional.silu(torch.from_numpy(a[:, :Fw])).numpy() * a[:, Fw:]
-        return _e4m3_rows(h) @ B
+        return _e4m3_rows(_bf16_rows(h)) @ B
 
     ref = ffn(x, Wsgu64, Wsd64) + ffn(x, Wgu64, Wd64)
     assert np.max(np.abs(out - ref)) <= 1e-12 * np.sqrt(np.mean(ref ** 2))
