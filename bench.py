@@ -109,20 +109,24 @@ class ClockSampler:
                 "sm_max_mhz": max(mx) if mx else None, "reasons": reasons, "samples": len(rows)}
 
 
-def kernel_flops_bytes(cfg, counts):
-    """Algorithmic FLOPs / bytes per launch of each kernel."""
+def kernel_flops_bytes(cfg, counts, act8: bool = False):
+    """Algorithmic FLOPs / bytes per launch of each kernel.  act8: the FP8
+    activation mode (the contractions read 1-byte token and hidden rows; the
+    hidden rows are written in bf16 and quantised by their own kernel)."""
     T, d, E, F, Fs = cfg.T, cfg.d_model, cfg.num_experts, cfg.expert_ffn, cfg.shared_ffn
     a = accounting.ACT_BYTES[cfg.dtype]
     w = accounting.W_BYTES[cfg.dtype]
+    q = 1 if act8 else a  # bytes of a contraction's token-row element
     touched = int(np.count_nonzero(counts))
     return {
         "router": {"flops": 2 * T * d * E, "bytes": T * d * a + d * E * a + T * 16},
         "permute": {"flops": 0, "bytes": T * 4 * 4},
-        "row_copy": {"flops": 0, "bytes": 2 * T * d * a + T * 12},
+        "row_copy": {"flops": 0, "bytes": T * d * a + 2 * T * d * q + T * 12},
         "gemm_gate_up": {"flops": 4 * T * d * (F + Fs),
-                         "bytes": (touched * 2 * d * F + 2 * d * Fs) * w + 2 * T * d * a + T * (F + Fs) * a},
+                         "bytes": (touched * 2 * d * F + 2 * d * Fs) * w + 2 * T * d * q + T * (F + Fs) * a},
         "gemm_down": {"flops": 2 * T * d * (F + Fs),
-                      "bytes": (touched * F * d + Fs * d) * w + T * (F + Fs) * a + T * d * a},
+                      "bytes": (touched * F * d + Fs * d) * w + T * (F + Fs) * q + T * d * a},
+        "quant_hidden": {"flops": 0, "bytes": T * (F + Fs) * (a + 1) + 2 * T * 4},
     }
 
 
@@ -323,6 +327,8 @@ def main():
     ap.add_argument("--experts", type=int, default=0,
                     help="override E (smaller profiling captures)")
     ap.add_argument("--impl", default="b200", choices=["b200", "reference"])
+    ap.add_argument("--act-fp8", action="store_true",
+                    help="E4M3-weight workloads: run the FP8 activation mode")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-workloads", action="store_true",
                     help="measure only --workload (skip the other shapes measured after it)")
@@ -360,21 +366,30 @@ def main():
 # Datasheet figures (NVIDIA B200: dense bf16 tensor throughput, HBM3e
 # bandwidth), reported next to the fractions of the measured peaks.
 DATASHEET = {"bf16_tflops": 2250.0, "hbm_gbs": 8000.0}
+# dense E4M3 over dense bf16 tensor throughput, nominal (4.5 / 2.25 PFLOP/s)
+FP8_OVER_BF16 = 2.0
 
 # Workloads measured after the headline in the same run, each with its own
 # timed region, roofline and clocks: the other shapes the layer is quoted on.
 EXTRA_WORKLOADS = ("maverick_prefill_bf16", "maverick_decode_bf16@T1", "maverick_decode_bf16@T8",
                    "maverick_decode_bf16@T32", "maverick_decode_bf16@T128", "maverick_fp8",
-                   "maverick_int8", "scout_prefill_int4", "maverick_dense_bf16", "tiny_f32")
+                   "maverick_fp8+act8", "maverick_int8", "scout_prefill_int4", "maverick_dense_bf16",
+                   "tiny_f32")
 
 
 def workload_config(name: str):
-    base, _, t = name.partition("@T")
+    """A workload name: a config, optionally `@T<n>` (another token count)
+    and `+act8` (the FP8 activation mode; see workload_act8)."""
+    base, _, t = name.replace("+act8", "").partition("@T")
     cfg = CONFIGS[base]
     return cfg.with_tokens(int(t)) if t else cfg
 
 
-def make_layer(cfg, rank):
+def workload_act8(name: str) -> bool:
+    return name.endswith("+act8")
+
+
+def make_layer(cfg, rank, act8: bool = False):
     from sparse_moe_transformer_router_b200.binding import L4MoE
     inp = generate(cfg, seed=rank, device="cuda")
     layer = L4MoE(cfg.d_model, cfg.expert_ffn, cfg.shared_ffn, cfg.num_experts, cfg.dtype)
@@ -382,6 +397,8 @@ def make_layer(cfg, rank):
         layer.set_router_bias(inp.bias)
     if cfg.dtype in CODED:
         layer.set_weight_scales(inp.s_gate_up, inp.s_down, inp.ss_gate_up, inp.ss_down)
+    if act8:
+        layer.set_act_fp8(True)
     return inp, layer
 
 
@@ -401,7 +418,7 @@ def roofline_of(flops: float, nbytes: float, seconds: float, tensor_peak: float,
             "datasheet_peak": hbm_sheet, "frac_of_datasheet": achieved / hbm_sheet}
 
 
-def measure(cfg, inp, layer, steps: int, warmup: int, world: int, local: int) -> dict:
+def measure(cfg, inp, layer, steps: int, warmup: int, world: int, local: int, act8: bool = False) -> dict:
     """Device-timed forwards of one workload: warm-up, a per-kernel
     breakdown pass, then `steps` forwards between two events on the
     launching stream (barrier + synchronize on both sides, max over ranks),
@@ -454,8 +471,12 @@ def measure(cfg, inp, layer, steps: int, warmup: int, world: int, local: int) ->
     peaks, peak_src = load_peaks()
     long_region = t_ms > 1000.0
     tensor_peak = peaks.get("bf16_tflops_sustained" if long_region else "bf16_tflops")
+    tensor_sheet = DATASHEET["bf16_tflops"]
+    if act8:  # E4M3 x E4M3: the measured bf16 peak times the nominal FP8 / bf16 ratio
+        tensor_peak *= FP8_OVER_BF16
+        tensor_sheet *= FP8_OVER_BF16
     hbm = peaks["hbm_gbs"]
-    kfb = kernel_flops_bytes(cfg, counts)
+    kfb = kernel_flops_bytes(cfg, counts, act8)
     per_kernel = {}
     for name, (ms, n) in breakdown.items():
         if n:
@@ -469,9 +490,10 @@ def measure(cfg, inp, layer, steps: int, warmup: int, world: int, local: int) ->
     dom_ms, dom_n = ktimes[dom]
     f, b = kfb[dom]["flops"], kfb[dom]["bytes"]
     avg_s = dom_ms / dom_n / 1e3  # the dominant kernel's events inside the timed region
-    roof = roofline_of(f, b, avg_s, tensor_peak, hbm, DATASHEET["bf16_tflops"], DATASHEET["hbm_gbs"])
-    roof = {"kernel": dom, **roof, "traffic": profile_traffic(dom, cfg.name),
+    roof = roofline_of(f, b, avg_s, tensor_peak, hbm, tensor_sheet, DATASHEET["hbm_gbs"])
+    roof = {"kernel": dom, **roof, "traffic": profile_traffic(dom, cfg.name + ("+act8" if act8 else "")),
             "peak_source": (f"{peak_src} ({'sustained' if long_region else 'burst'})"
+                            + (f" x {FP8_OVER_BF16:g} (nominal E4M3 / bf16 ratio)" if act8 else "")
                             if roof["bound"] == "tensor" else f"{peak_src} hbm_gbs"),
             "algorithmic_per_launch": {"flops": f, "bytes": b},
             "avg_us_timed_region": avg_s * 1e6, "launches_timed": dom_n}
@@ -480,8 +502,7 @@ def measure(cfg, inp, layer, steps: int, warmup: int, world: int, local: int) ->
     flops = accounting.layer_flops(cfg.T, cfg.d_model, cfg.num_experts, cfg.expert_ffn, cfg.shared_ffn)
     lbytes = accounting.layer_bytes(cfg.T, cfg.d_model, cfg.num_experts, cfg.expert_ffn, cfg.shared_ffn,
                                     cfg.dtype, touched)
-    lr = roofline_of(flops, lbytes, ms_step / 1e3, tensor_peak, hbm, DATASHEET["bf16_tflops"],
-                     DATASHEET["hbm_gbs"])
+    lr = roofline_of(flops, lbytes, ms_step / 1e3, tensor_peak, hbm, tensor_sheet, DATASHEET["hbm_gbs"])
     layer_roof = {"bound": lr["bound"], "frac": lr["frac"], "frac_of_datasheet": lr["frac_of_datasheet"],
                   "tflops_active": flops / (ms_step / 1e3) / 1e12,
                   "gbs_algorithmic": lbytes / (ms_step / 1e3) / 1e9,
@@ -497,7 +518,8 @@ def run_extra_workloads(args, rank, world, local) -> dict:
     res = {}
     for name in EXTRA_WORKLOADS:
         cfg = workload_config(name)
-        inp, layer = make_layer(cfg, rank)
+        act8 = workload_act8(name)
+        inp, layer = make_layer(cfg, rank, act8)
         # a timed region of at least ~200 ms (and at least --steps forwards)
         out = torch.empty((cfg.T, cfg.d_model), dtype=inp.x.dtype, device="cuda")
         layer.forward(inp.x, inp.W_router, inp.W_gate_up, inp.W_down, inp.Ws_gate_up, inp.Ws_down, out=out)
@@ -507,7 +529,7 @@ def run_extra_workloads(args, rank, world, local) -> dict:
         torch.cuda.synchronize()
         est_ms = (time.perf_counter() - t0) * 1e3
         steps = int(max(args.steps, min(400, 200.0 / max(est_ms, 1e-3))))
-        m = measure(cfg, inp, layer, steps, args.warmup, world, local)
+        m = measure(cfg, inp, layer, steps, args.warmup, world, local, act8)
         res[name] = {"tokens_per_s": replica_throughput(world, cfg.T, steps, m["t_ms"]),
                      "ms_per_step": m["ms_per_step"], "steps": steps, "T": cfg.T,
                      "experts": cfg.num_experts, "dtype": cfg.dtype, "router": cfg.router,
@@ -524,8 +546,8 @@ def run_extra_workloads(args, rank, world, local) -> dict:
 def run_b200(args, rank, world, local):
     torch.cuda.set_device(local)
     cfg = CONFIGS[args.workload]
-    inp, layer = make_layer(cfg, rank)
-    m = measure(cfg, inp, layer, args.steps, args.warmup, world, local)
+    inp, layer = make_layer(cfg, rank, args.act_fp8)
+    m = measure(cfg, inp, layer, args.steps, args.warmup, world, local, args.act_fp8)
     value = replica_throughput(world, cfg.T, args.steps, m["t_ms"])
 
     # ------------------------------------------------------------- e2e (host buffers)
@@ -590,6 +612,9 @@ def run_b200(args, rank, world, local):
     if cfg.dtype in CODED:
         wname = {"fp8": "E4M3", "int8": "int8", "int4": "int4"}[cfg.dtype]
         line["dtype"] = f"f16 ({wname} weights widened exactly to f16, fp32 accumulate; bf16 in and out)"
+    if args.act_fp8:
+        line["dtype"] = "e4m3 (E4M3 weights and per-row E4M3 token / hidden rows, fp32 accumulate; bf16 in and out)"
+        line["config"]["workload"] += "+act8"
     if cpu is not None:
         line["cpu_baseline"] = cpu
     if extra:

@@ -136,7 +136,8 @@ L4MOE_API l4moe_status l4moe_create(const l4moe_params *params, l4moe_handle **o
 L4MOE_API void l4moe_destroy(l4moe_handle *h);
 
 /* Bytes of device workspace l4moe_forward needs for up to max_tokens tokens
- * with the handle's current experts per token (l4moe_set_top_k): routing
+ * with the handle's current experts per token (l4moe_set_top_k) and FP8
+ * activation mode (l4moe_set_act_fp8): routing
  * vectors, permutation, group tables, gated expert-ordered input, both
  * hidden activations, fp32 partials, host-path staging.  0 on a bad
  * argument. */
@@ -179,6 +180,26 @@ L4MOE_API l4moe_status l4moe_set_weight_scales(l4moe_handle *h, const float *con
 L4MOE_API l4moe_status l4moe_set_fp8_scales(l4moe_handle *h, const float *const *s_gate_up,
                                   const float *const *s_down, const float *ss_gate_up,
                                   const float *ss_down);
+
+/* FP8 activation mode (on = 1; off = 0, the default), E4M3 weights only.
+ * superteams.ai "Llama 4" glossary, "Running Llama 4 Yourself": Maverick is
+ * served with FP8 quantisation; the pages fix no activation scaling, so this
+ * is an opt-in reading.  Every contraction input row is quantised to E4M3
+ * with one fp32 scale for the row: a token's x (before the router's gate,
+ * which still scales the routed expert's dequantised input), and each
+ * hidden row an expert produces, held in bf16 first:
+ *   s = fp32(max|v| / 448) (1 for a row of zeros),
+ *   code = E4M3 round-to-nearest-even, saturating, of fp32(v / s),
+ * and every tensor-core contraction multiplies E4M3 codes by E4M3 codes
+ * (tcgen05 kind::f8f6f4), the weight column scale and the row scale applied
+ * to the fp32 accumulator.  The router still reads the bf16 x.  The layer
+ * then differs from the bf16-activation one by the quantisation (a few
+ * percent of rms(out)).  Changing the mode frees a workspace the handle
+ * allocated (it synchronises the device; the mode needs room for the hidden
+ * rows' codes) and fails with L4MOE_ERR_WORKSPACE when a caller's workspace
+ * is too small.  L4MOE_ERR_DTYPE for other weight types, L4MOE_ERR_ARG for
+ * `on` other than 0 or 1. */
+L4MOE_API l4moe_status l4moe_set_act_fp8(l4moe_handle *h, int on);
 
 /* Enqueue one forward pass of the layer for T tokens on `stream` (a
  * cudaStream_t, NULL = legacy default stream).  x, W_router, Ws_gate_up,
@@ -287,11 +308,12 @@ L4MOE_API l4moe_status l4moe_selftest_wait(l4moe_handle *h, double limit_ms, voi
  * are those of the real launches in place (every event pair adds a little
  * to the step, so time only what is needed).  Kernel slots: 0 router,
  * 1 permute, 2 row copy, 3 gate/up GEMM (+ its split-K finish), 4 down GEMM
- * + finish (L4MOE_NUM_KERNELS).  l4moe_read_timing synchronises on the last recorded
+ * + finish, 5 hidden-row quantisation of the FP8 activation mode
+ * (L4MOE_NUM_KERNELS).  l4moe_read_timing synchronises on the last recorded
  * event, adds every recorded pair to ms[slot] and launches[slot] (arrays of
  * at least L4MOE_NUM_KERNELS entries, accumulated into), and recycles the
  * events.  Returns L4MOE_ERR_CUDA if an event call fails. */
-#define L4MOE_NUM_KERNELS 5
+#define L4MOE_NUM_KERNELS 6
 #define L4MOE_TIME_ALL ((1 << L4MOE_NUM_KERNELS) - 1)
 L4MOE_API l4moe_status l4moe_set_timing(l4moe_handle *h, int mask);
 L4MOE_API l4moe_status l4moe_read_timing(l4moe_handle *h, double *ms, uint64_t *launches);

@@ -81,7 +81,7 @@ def _load():
                                            vp, i32, vp, i32, f32p,
                                            vp, vp, vp, vp, i32,
                                            vp, vp, vp, vp, i32,
-                                           i32, vp, vp, vp, vp, i32, vp]
+                                           i32, vp, vp, vp, vp, i32, vp, vp]
             lib.oracle_expert_rows.restype = None
             lib.oracle_expert_rows.argtypes = [i32, i32, i32, vp, i32, vp, vp, vp, i32, vp, vp, vp]
             lib.oracle_round_hidden.restype = ctypes.c_double
@@ -217,7 +217,7 @@ def round_hidden(v: float, kind: str) -> float:
 
 def forward(x, Wr, W_gate_up, W_down, Ws_gate_up, Ws_down, *, bias=None,
             s_gate_up=None, s_down=None, ss_gate_up=None, ss_down=None,
-            tokens=None, k=1, act_fp8=False, hidden_round=None):
+            tokens=None, k=1, act_fp8=False, hidden_round=None, scale_margin=False):
     """Layer output in fp64 for ``tokens`` (all tokens when None).
 
     W_gate_up / W_down are length-E lists of [d, 2F] / [F, d] arrays; entries
@@ -235,6 +235,10 @@ def forward(x, Wr, W_gate_up, W_down, Ws_gate_up, Ws_down, *, bias=None,
     same outputs with every hidden value rounded to that type (through fp32)
     before the down projection -- the roundings a GPU that keeps the hidden
     rows in that type makes, with everything else exact.
+    scale_margin (FP8 activation mode, bf16 activations): also return, last,
+    each token's smallest distance (relative to the row's largest value) of a
+    near-largest hidden value to a bf16 rounding midpoint over its hidden
+    rows -- where an fp32 evaluation may give the row another scale.
     """
     x = np.ascontiguousarray(x)
     Wr = np.ascontiguousarray(Wr)
@@ -287,6 +291,7 @@ def forward(x, Wr, W_gate_up, W_down, Ws_gate_up, Ws_down, *, bias=None,
     sel_idx = np.empty(n_sel * k, np.int32)
     sel_gate = np.empty(n_sel * k, np.float64)
     out_h = np.zeros((n_sel, d), np.float64) if hidden_round else None
+    margin = np.full(n_sel, np.inf) if scale_margin else None
     rc = _load().oracle_forward(
         T, d, E, k, F, Fs, _ptr(x), _dtype_code(x), _ptr(Wr), _dtype_code(Wr),
         _ptr(bias), ctypes.cast(gu_ptrs, ctypes.c_void_p),
@@ -295,7 +300,7 @@ def forward(x, Wr, W_gate_up, W_down, Ws_gate_up, Ws_down, *, bias=None,
         None if sgu_ptrs is None else ctypes.cast(sgu_ptrs, ctypes.c_void_p),
         None if sdn_ptrs is None else ctypes.cast(sdn_ptrs, ctypes.c_void_p),
         _ptr(ss_gate_up), _ptr(ss_down), 1 if act_fp8 else 0, n_sel, _ptr(sel), _ptr(out),
-        _ptr(sel_idx), _ptr(sel_gate), HIDDEN_ROUND[hidden_round], _ptr(out_h))
+        _ptr(sel_idx), _ptr(sel_gate), HIDDEN_ROUND[hidden_round], _ptr(out_h), _ptr(margin))
     del keep
     if rc != 0:
         raise ValueError("oracle.forward: a selected token routes to an expert "
@@ -303,6 +308,5 @@ def forward(x, Wr, W_gate_up, W_down, Ws_gate_up, Ws_down, *, bias=None,
     if k > 1:
         sel_idx = sel_idx.reshape(n_sel, k)
         sel_gate = sel_gate.reshape(n_sel, k)
-    if hidden_round:
-        return out, sel_idx, sel_gate, out_h
-    return out, sel_idx, sel_gate
+    res = (out, sel_idx, sel_gate) + ((out_h,) if hidden_round else ()) + ((margin,) if scale_margin else ())
+    return res

@@ -213,6 +213,41 @@ static double round_hidden(double v, int h_round) {
 
 double oracle_round_hidden(double v, int h_round) { return round_hidden(v, h_round); }
 
+/* FP8 activation mode, bf16 activations: how near a hidden row's scale is
+ * to changing.  The scale comes from the largest |value| after the bf16
+ * rounding; an implementation that forms the values in fp32 with a slightly
+ * different rounding error rounds an element to the other bf16 neighbour
+ * when the element lies near a rounding midpoint, and if that element is
+ * (or becomes) the largest, the whole row gets another scale.  Returns the
+ * smallest distance, relative to the row's largest |fp32 value|, from an
+ * element within one bf16 spacing of that largest value to its nearest bf16
+ * rounding midpoint (bf16 keeps 8 significant bits: spacing 2^(e-8) in the
+ * binade [2^(e-1), 2^e), half that just below it); +inf for a zero row. */
+static double hidden_scale_margin(int n, const double *h) {
+    double m = 0.0;
+    for (int j = 0; j < n; ++j) {
+        double a = fabs((double)(float)h[j]);
+        if (a > m) m = a;
+    }
+    if (m == 0.0) return INFINITY;
+    double best = INFINITY;
+    for (int j = 0; j < n; ++j) {
+        double a = fabs((double)(float)h[j]);
+        if (a < m * (1.0 - ldexp(1.0, -7)) || a == 0.0) continue;
+        int e2;
+        frexp(a, &e2); /* a in [2^(e2-1), 2^e2) */
+        double ulp = ldexp(1.0, e2 - 8);
+        double lo = floor(a / ulp) * ulp;
+        double dist = fabs(a - (lo + 0.5 * ulp));
+        if (lo == ldexp(1.0, e2 - 1)) { /* the midpoint below the binade is finer */
+            double below = a - (lo - 0.25 * ulp);
+            if (below < dist) dist = below;
+        }
+        if (dist / m < best) best = dist / m;
+    }
+    return best;
+}
+
 static double sigmoid(double z) { return 1.0 / (1.0 + exp(-z)); }
 static double silu(double z) { return z / (1.0 + exp(-z)); }
 
@@ -292,7 +327,7 @@ static void swiglu_ffn_accumulate(int d, int Fw, const double *u,
                                   const void *Wgu, const void *Wd, int w_dtype,
                                   const float *s_gu, const float *s_d, int act_fp8,
                                   int act_bf16, double *a, double *h, double *y,
-                                  int h_round, double *yh) {
+                                  int h_round, double *yh, double *scale_margin) {
     size_t two_f = 2 * (size_t)Fw;
     for (size_t j = 0; j < two_f; ++j) a[j] = 0.0;
     for (int k = 0; k < d; ++k) {
@@ -305,8 +340,13 @@ static void swiglu_ffn_accumulate(int d, int Fw, const double *u,
         /* the hidden row in the layer's activation type, then quantised; the
          * quantised values are what the down contraction reads, so the
          * hidden-rounding variant below has nothing left to round */
-        if (act_bf16)
+        if (act_bf16) {
+            if (scale_margin) {
+                double mg = hidden_scale_margin(Fw, h);
+                if (mg < *scale_margin) *scale_margin = mg;
+            }
             for (int j = 0; j < Fw; ++j) h[j] = round_bf16(h[j]);
+        }
         quantise_row_e4m3(Fw, h);
         h_round = HROUND_NONE;
     }
@@ -368,7 +408,9 @@ void oracle_permutation(int T, int E, const int32_t *idx, int32_t *counts,
  * W_down[e] may be NULL for experts that none of the selected tokens
  * reaches; returns -1 if a needed expert is missing, 0 on success.
  * sel_idx / sel_gate (optional) receive each selected token's expert and
- * gate. */
+ * gate.  scale_margin (optional, [n_sel]): in the FP8 activation mode with
+ * bf16 activations, the smallest hidden_scale_margin over the token's hidden
+ * rows (shared and routed), else +inf. */
 int oracle_forward(int T, int d, int E, int k, int F, int Fs,
                    const void *x, int x_dtype,
                    const void *Wr, int wr_dtype, const float *bias,
@@ -377,7 +419,8 @@ int oracle_forward(int T, int d, int E, int k, int F, int Fs,
                    const float *const *s_gate_up, const float *const *s_down,
                    const float *ss_gate_up, const float *ss_down, int act_fp8,
                    int n_sel, const int32_t *sel, double *out,
-                   int32_t *sel_idx, double *sel_gate, int h_round, double *out_h) {
+                   int32_t *sel_idx, double *sel_gate, int h_round, double *out_h,
+                   double *scale_margin) {
     size_t xs = (x_dtype == ORACLE_F32) ? 4 : 2;
     const int act_bf16 = x_dtype == ORACLE_BF16; /* the layer's activations are bf16 */
     int missing = 0;
@@ -394,6 +437,7 @@ int oracle_forward(int T, int d, int E, int k, int F, int Fs,
         double *yh = out_h ? out_h + (size_t)i * (size_t)d : NULL;
         for (int n = 0; n < d; ++n) y[n] = 0.0;
         for (int n = 0; yh && n < d; ++n) yh[n] = 0.0;
+        if (scale_margin) scale_margin[i] = INFINITY;
         /* shared expert on the ungated input (with E == 0 the whole layer:
          * the dense SwiGLU feed-forward of the layers without experts) */
         for (int k = 0; k < d; ++k) u[k] = load_elem(x_t, x_dtype, (size_t)k);
@@ -401,7 +445,8 @@ int oracle_forward(int T, int d, int E, int k, int F, int Fs,
         double *xq = (double *)malloc(sizeof(double) * (size_t)d);
         for (int k = 0; k < d; ++k) xq[k] = u[k];
         swiglu_ffn_accumulate(d, Fs, u, Ws_gate_up, Ws_down, w_dtype,
-                              ss_gate_up, ss_down, act_fp8, act_bf16, a, h, y, h_round, yh);
+                              ss_gate_up, ss_down, act_fp8, act_bf16, a, h, y, h_round, yh,
+                              scale_margin ? &scale_margin[i] : NULL);
         if (E == 0) {
             if (sel_idx) sel_idx[i] = -1;
             if (sel_gate) sel_gate[i] = 0.0;
@@ -431,7 +476,8 @@ int oracle_forward(int T, int d, int E, int k, int F, int Fs,
             for (int kk = 0; kk < d; ++kk) u[kk] = g * xq[kk];
             swiglu_ffn_accumulate(d, F, u, W_gate_up[e], W_down[e], w_dtype,
                                   s_gate_up ? s_gate_up[e] : NULL,
-                                  s_down ? s_down[e] : NULL, act_fp8, act_bf16, a, h, y, h_round, yh);
+                                  s_down ? s_down[e] : NULL, act_fp8, act_bf16, a, h, y, h_round, yh,
+                                  scale_margin ? &scale_margin[i] : NULL);
         }
         free(u);
         free(xq);
@@ -460,7 +506,7 @@ void oracle_expert_rows(int n, int d, int F, const void *x, int x_dtype, const d
         for (int k = 0; k < d; ++k) u[k] = g[i] * load_elem(x_i, x_dtype, (size_t)k);
         for (int k = 0; k < d; ++k) y[k] = 0.0;
         swiglu_ffn_accumulate(d, F, u, W_gate_up, W_down, w_dtype, s_gate_up, s_down, 0, 0, a, h, y,
-                              HROUND_NONE, NULL);
+                              HROUND_NONE, NULL, NULL);
         free(u);
         free(a);
         free(h);

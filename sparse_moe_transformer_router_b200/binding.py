@@ -22,9 +22,9 @@ EXPORTED = ("l4moe_create", "l4moe_destroy", "l4moe_workspace_size", "l4moe_set_
             "l4moe_launch_count", "l4moe_last_error", "l4moe_status_string", "l4moe_version",
             "l4moe_set_timing", "l4moe_read_timing", "l4moe_kernel_name",
             "l4moe_forward_static", "l4moe_join_host", "l4moe_set_top_k",
-            "l4moe_set_weight_scales", "l4moe_selftest_wait")
+            "l4moe_set_weight_scales", "l4moe_selftest_wait", "l4moe_set_act_fp8")
 STATIC_WORKSPACE_BYTES = 32 << 20
-NUM_KERNELS = 5
+NUM_KERNELS = 6
 
 _lib = None
 
@@ -77,6 +77,7 @@ def load_library():
     lib.l4moe_version.argtypes = []
     lib.l4moe_set_timing.argtypes = [vp, i32]
     lib.l4moe_set_top_k.argtypes = [vp, i32]
+    lib.l4moe_set_act_fp8.argtypes = [vp, i32]
     lib.l4moe_selftest_wait.argtypes = [vp, ctypes.c_double, vp]
     lib.l4moe_read_timing.argtypes = [vp, ctypes.POINTER(ctypes.c_double),
                                       ctypes.POINTER(ctypes.c_uint64)]
@@ -86,7 +87,8 @@ def load_library():
                  "l4moe_set_fp8_scales", "l4moe_forward", "l4moe_forward_host",
                  "l4moe_get_routing", "l4moe_check_device_status", "l4moe_version",
                  "l4moe_set_timing", "l4moe_read_timing", "l4moe_forward_static",
-                 "l4moe_join_host", "l4moe_set_top_k", "l4moe_set_weight_scales", "l4moe_selftest_wait"):
+                 "l4moe_join_host", "l4moe_set_top_k", "l4moe_set_weight_scales", "l4moe_selftest_wait",
+                 "l4moe_set_act_fp8"):
         getattr(lib, name).restype = ctypes.c_int
     _lib = lib
     return lib
@@ -298,6 +300,11 @@ class L4MoE:
         """Experts per token (l4moe_set_top_k)."""
         self._check(self._lib.l4moe_set_top_k(self._h, int(k)))
         self.top_k = int(k)
+
+    def set_act_fp8(self, on: bool = True):
+        """FP8 activation mode (l4moe_set_act_fp8): E4M3 token and hidden rows."""
+        self._check(self._lib.l4moe_set_act_fp8(self._h, 1 if on else 0))
+        self.act_fp8 = bool(on)
 
     def routing(self):
         """Zero-copy device views of the last forward's routing (valid until

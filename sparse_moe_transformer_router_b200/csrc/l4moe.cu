@@ -25,6 +25,7 @@
 #include "finish.cuh"
 #include "moe_gemm.cuh"
 #include "permute.cuh"
+#include "quant.cuh"
 #include "route_small.cuh"
 #include "router.cuh"
 
@@ -76,7 +77,7 @@ constexpr int kRouterKSplit = 8;
 
 struct WsLayout {
     size_t err, idx, gate, lmax, margin, inv, perm, gslot, counts, offsets, chunk, tab_gu, tab_dn, xg, hr,
-        hs, x16, xsc, part, logits, xin, xout;
+        hs, x16, xsc, hq, hsc, part, logits, xin, xout;
     size_t device_total;  // everything l4moe_forward uses
     size_t total;         // plus the host-path staging slots (last)
 };
@@ -97,9 +98,10 @@ struct SplitPlan {
     int s_gu, s_dn;
 };
 
-SplitPlan split_plan(const l4moe_params& p, int T, int sms, int k = 1) {
+SplitPlan split_plan(const l4moe_params& p, int T, int sms, int k = 1, bool act8 = false) {
     const int d = p.d_model, F = p.expert_ffn, Fs = p.shared_ffn, E = p.num_experts;
-    const int kblk = (int)(128 / act_bytes(p.dtype));  // K elements per k-block
+    // K elements per k-block (one 128-byte token row; E4M3 rows in the FP8 activation mode)
+    const int kblk = act8 ? 128 : (int)(128 / act_bytes(p.dtype));
     const int fb_gu_r = (F + 127) / 128, fb_gu_s = (Fs + 127) / 128, fb_dn = (d + 255) / 256;
     // Tiles are striped over the CTA pairs, so the launch lasts ceil(units /
     // pairs) tile times: take the split count that fills the last wave best
@@ -135,10 +137,10 @@ SplitPlan split_plan(const l4moe_params& p, int T, int sms, int k = 1) {
 
 // fp32 partial floats any forward of at most T tokens needs: split gate/up
 // results, and the down's shared + routed results (times its splits).
-size_t part_floats(const l4moe_params& p, int T, int sms, int k) {
+size_t part_floats(const l4moe_params& p, int T, int sms, int k, bool act8) {
     size_t need = 0;
     auto add = [&](int t) {  // t tokens: t * k routed entries, t shared rows
-        const SplitPlan sp = split_plan(p, t, sms, k);
+        const SplitPlan sp = split_plan(p, t, sms, k, act8);
         const size_t tv = (size_t)t * k;
         if (sp.s_gu > 1)
             need = std::max<size_t>(need, (size_t)sp.s_gu * (tv * 2ull * p.expert_ffn + (size_t)t * 2ull * p.shared_ffn));
@@ -150,8 +152,9 @@ size_t part_floats(const l4moe_params& p, int T, int sms, int k) {
 }
 
 // k: selected experts per token (l4moe_set_top_k); the routed rows are the
-// T * k token entries.
-WsLayout ws_layout(const l4moe_params& p, int T, int sms, int k) {
+// T * k token entries.  act8: the FP8 activation mode (E4M3 hidden rows and
+// their scales).
+WsLayout ws_layout(const l4moe_params& p, int T, int sms, int k, bool act8 = false) {
     WsLayout L{};
     size_t off = 0;
     auto take = [&](size_t bytes) {
@@ -179,8 +182,12 @@ WsLayout ws_layout(const l4moe_params& p, int T, int sms, int k) {
     L.hs = take(t * p.shared_ffn * es);
     // 8-bit weight layers: x in f16, token order (the shared expert's operand)
     L.x16 = take(coded8(p.dtype) ? t * p.d_model * 2 : 0);
-    L.xsc = take(coded8(p.dtype) ? 4 * t : 0);  // and each token row's power-of-two scale
-    L.part = take(sizeof(float) * part_floats(p, (int)t, sms, k));
+    L.xsc = take(coded8(p.dtype) ? 4 * t : 0);  // and each token row's scale
+    // FP8 activation mode: the hidden rows' E4M3 codes (routed [T k][F], then
+    // shared [T][Fs]) and their row scales ([T k] then [T])
+    L.hq = take(act8 ? tv * p.expert_ffn + t * p.shared_ffn : 0);
+    L.hsc = take(act8 ? 4 * (tv + t) : 0);
+    L.part = take(sizeof(float) * part_floats(p, (int)t, sms, k, act8));
     // expert-split router logits [min(T, 128)][E]; for batches the one-launch
     // routing takes, its partial logits [slices][T][E]
     const size_t small_part = (size_t)((p.d_model + kSmallSliceK - 1) / kSmallSliceK) *
@@ -205,6 +212,7 @@ struct l4moe_handle {
     size_t ws_bytes = 0;
     int ws_tokens = 0;
     int top_k = 1;  // selected experts per token (l4moe_set_top_k)
+    bool act8 = false;  // FP8 activation mode (l4moe_set_act_fp8)
     bool ws_owned = false;
     const float* bias = nullptr;
     std::vector<const float*> s_gu, s_dn;
@@ -328,7 +336,7 @@ l4moe_status ensure_workspace(l4moe_handle* h, int T) {
         h->ws = nullptr;
     }
     const int cap = std::max(T, 256);
-    const WsLayout L = ws_layout(h->p, cap, h->sms, h->top_k);
+    const WsLayout L = ws_layout(h->p, cap, h->sms, h->top_k, h->act8);
     void* p = nullptr;
     cudaError_t e = cudaMalloc(&p, L.total);
     if (e != cudaSuccess) return cuda_fail(h, e, "workspace cudaMalloc");
@@ -354,15 +362,18 @@ l4moe_status encode_weight_maps(l4moe_handle* h, const void* const* Wgu, const v
     CUtensorMapDataType dt = wdt == L4MOE_F32 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT32
                              : wdt == L4MOE_BF16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16
                                                  : CU_TENSOR_MAP_DATA_TYPE_UINT8;
-    const bool fp8 = coded8(wdt);
-    const uint32_t bk = wdt == L4MOE_F32 ? 32 : 64;  // K rows per box
+    const bool act8 = h->act8;               // E4M3 codes read raw by the MMA
+    const bool fp8 = coded8(wdt) && !act8;  // codes widened in shared memory
+    const uint32_t bk = wdt == L4MOE_F32 ? 32 : act8 ? 128 : 64;  // K rows per box
     // box width in elements of the map: one 128-byte swizzled slab of
     // features; coded weights are staged raw (64-feature boxes, unswizzled;
     // int4 maps count bytes, 32 of them per 64 features) and widened in
-    // shared memory
-    const uint32_t bw = wdt == L4MOE_INT4 ? 32u : fp8 ? 64u : (uint32_t)(128 / w_row_bytes(wdt, 1));
+    // shared memory; in the FP8 activation mode the codes land as the MMA
+    // reads them: 64-feature slabs in the 64-byte swizzle
+    const uint32_t bw = wdt == L4MOE_INT4 ? 32u : (fp8 || act8) ? 64u : (uint32_t)(128 / w_row_bytes(wdt, 1));
     // MN-major 32-bit operands need the 32-byte swizzle unit
-    const CUtensorMapSwizzle swz = fp8 ? CU_TENSOR_MAP_SWIZZLE_NONE
+    const CUtensorMapSwizzle swz = act8 ? CU_TENSOR_MAP_SWIZZLE_64B
+                                   : fp8 ? CU_TENSOR_MAP_SWIZZLE_NONE
                                    : h->p.dtype == L4MOE_F32 ? CU_TENSOR_MAP_SWIZZLE_128B_ATOM_32B
                                                              : CU_TENSOR_MAP_SWIZZLE_128B;
     h->h_maps.assign(2 * (E + 1), CUtensorMap{});
@@ -472,16 +483,19 @@ void launch_gemm(int grid, const BMaps& bm, const GemmArgs& a, cudaStream_t st) 
 // The launch sequence of one forward.  w / ws_tokens: the workspace and the
 // token count its layout was made for; maps: device array of the 2(E+1)
 // weight descriptors.
-// WQ: the weights' storage (kWqNone: the layer's type; kWqE4M3 / kWqInt8:
-// 8-bit codes with per-column scales, widened to f16 in the GEMMs).
+// WQ: the weights' storage (kWqNone: the layer's type; kWqE4M3 / kWqInt8 /
+// kWqInt4: codes with per-column scales, widened to f16 in the GEMMs;
+// kWqAct8: E4M3 codes multiplied raw with E4M3 token rows, the FP8
+// activation mode).
 template <typename ET, int WQ = kWqNone>
 l4moe_status run_layer(l4moe_handle* h, int T, const void* x, const void* Wr, const void* Wsgu,
                        const void* Wsdn, void* out, cudaStream_t st, uint8_t* w, int ws_tokens,
                        const CUtensorMap* maps, const float* const* scales = nullptr) {
-    constexpr bool FP8W = WQ != kWqNone;  // 8-bit weight codes (E4M3 or int8)
+    constexpr bool FP8W = WQ != kWqNone;  // coded weights with per-column scales
+    constexpr bool ACT8 = WQ == kWqAct8;  // and E4M3 token rows (FP8 activation mode)
     const l4moe_params& p = h->p;
     const int d = p.d_model, F = p.expert_ffn, Fs = p.shared_ffn, E = p.num_experts;
-    const WsLayout L = ws_layout(p, ws_tokens, h->sms, h->top_k);
+    const WsLayout L = ws_layout(p, ws_tokens, h->sms, h->top_k, h->act8);
     unsigned* err = reinterpret_cast<unsigned*>(w + L.err);
     int32_t* idx = reinterpret_cast<int32_t*>(w + L.idx);
     float* gate = reinterpret_cast<float*>(w + L.gate);
@@ -494,25 +508,33 @@ l4moe_status run_layer(l4moe_handle* h, int T, const void* x, const void* Wr, co
     int32_t* offsets = reinterpret_cast<int32_t*>(w + L.offsets);
     GroupTable* tab_gu = reinterpret_cast<GroupTable*>(w + L.tab_gu);
     GroupTable* tab_dn = reinterpret_cast<GroupTable*>(w + L.tab_dn);
-    // the GEMMs' activation type: the layer's, or f16 for 8-bit weights
-    // (widened exactly to f16; kind::f16 wants both operands of one type)
-    using GT = typename GemmAct<ET, FP8W>::type;
+    // the hidden rows' type: the layer's, or f16 for widened coded weights
+    // (kind::f16 wants both operands of one type); the token operand's type:
+    // the same, or E4M3 codes in the FP8 activation mode (hidden rows then
+    // stay bf16 until their own quantisation)
+    using HT = typename GemmAct<ET, FP8W && !ACT8>::type;
+    using GT = typename std::conditional<ACT8, uint8_t, HT>::type;
     GT* xg = reinterpret_cast<GT*>(w + L.xg);
-    GT* hr = reinterpret_cast<GT*>(w + L.hr);
-    GT* hs = reinterpret_cast<GT*>(w + L.hs);
+    HT* hr = reinterpret_cast<HT*>(w + L.hr);
+    HT* hs = reinterpret_cast<HT*>(w + L.hs);
     GT* x16 = reinterpret_cast<GT*>(w + L.x16);
     float* tokscale = FP8W ? reinterpret_cast<float*>(w + L.xsc) : nullptr;
+    // FP8 activation mode: hidden-row codes and scales (routed, then shared)
+    uint8_t* hq_r = ACT8 ? w + L.hq : nullptr;
+    float* hsc_r = ACT8 ? reinterpret_cast<float*>(w + L.hsc) : nullptr;
 
     // per-call activation descriptors (K-major rows of 128 B): the router's
     // x (64-row boxes) and the GEMMs' token operands (full- and small-tile
     // boxes: gate/up reads x in expert order and x, down reads H_r and H_s)
     auto tmap_type = [](size_t bytes, bool f16) {
         return bytes == 4 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT32
-                          : f16 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT16 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16;
+               : bytes == 1 ? CU_TENSOR_MAP_DATA_TYPE_UINT8
+               : f16 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT16 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16;
     };
     const CUtensorMapDataType adt = tmap_type(sizeof(ET), false);
-    const CUtensorMapDataType gdt = tmap_type(sizeof(GT), FP8W);
-    const uint32_t bk = (uint32_t)(128 / sizeof(ET));
+    const CUtensorMapDataType gdt = tmap_type(sizeof(GT), FP8W);  // gate/up token operand
+    const CUtensorMapDataType ddt = ACT8 ? CU_TENSOR_MAP_DATA_TYPE_UINT8 : gdt;  // down's: hidden rows
+    const size_t dsz = ACT8 ? 1 : sizeof(HT);
     using GCfg = GemmCfg<MODE_GATEUP, ET, WQ>;
     constexpr uint32_t rb = GCfg::B_BOX_ROWS, rs = GCfg::B_SMALL_ROWS;
     CUtensorMap m_x;
@@ -521,26 +543,31 @@ l4moe_status run_layer(l4moe_handle* h, int T, const void* x, const void* Wr, co
     // the routed rows (x in expert order, the routed hidden rows)
     const int k = h->top_k;
     const int Tv = T * k;
+    // K-major rows, boxes of 128 bytes of K by `rows` rows; esz: element bytes
     auto act_n = [&](CUtensorMap* m, CUtensorMapDataType dt, const void* base, int width, int nrows,
-                     uint32_t rows) {
-        return encode_2d(m, dt, base, (uint64_t)width, (uint64_t)nrows, (uint64_t)width * sizeof(ET), bk, rows);
+                     uint32_t rows, size_t esz) {
+        return encode_2d(m, dt, base, (uint64_t)width, (uint64_t)nrows, (uint64_t)width * esz,
+                         (uint32_t)(128 / esz), rows);
     };
-    auto act = [&](CUtensorMap* m, CUtensorMapDataType dt, const void* base, int width, uint32_t rows) {
-        return act_n(m, dt, base, width, T, rows);
-    };
-    auto act_r = [&](CUtensorMap* m, CUtensorMapDataType dt, const void* base, int width, uint32_t rows) {
-        return act_n(m, dt, base, width, Tv, rows);
-    };
+    auto act = [&](CUtensorMap* m, CUtensorMapDataType dt, const void* base, int width, uint32_t rows,
+                   size_t esz) { return act_n(m, dt, base, width, T, rows, esz); };
+    auto act_r = [&](CUtensorMap* m, CUtensorMapDataType dt, const void* base, int width, uint32_t rows,
+                     size_t esz) { return act_n(m, dt, base, width, Tv, rows, esz); };
     const void* xs = FP8W ? (const void*)x16 : x;  // the shared expert's operand
+    // the down's token operand: the hidden rows, or their codes in the FP8
+    // activation mode (routed [Tv][F] then shared [T][Fs])
+    const void* hdr = ACT8 ? (const void*)hq_r : (const void*)hr;
+    const void* hds = ACT8 ? (const void*)(hq_r + (size_t)Tv * F) : (const void*)hs;
     // without experts (F may be 0) the routed hidden descriptors are never
     // read: give them the shared hidden rows to describe
-    const void* hrm = F > 0 ? (const void*)hr : (const void*)hs;
+    const void* hrm = F > 0 ? hdr : hds;
     const int Fr = F > 0 ? F : Fs;
-    if (!act(&m_x, adt, x, d, 64) || !act_r(&bm_gu.routed, gdt, xg, d, rb) ||
-        !act_r(&bm_gu.routed_small, gdt, xg, d, rs) || !act(&bm_gu.shared, gdt, xs, d, rb) ||
-        !act(&bm_gu.shared_small, gdt, xs, d, rs) || !act_r(&bm_dn.routed, gdt, hrm, Fr, rb) ||
-        !act_r(&bm_dn.routed_small, gdt, hrm, Fr, rs) || !act(&bm_dn.shared, gdt, hs, Fs, rb) ||
-        !act(&bm_dn.shared_small, gdt, hs, Fs, rs))
+    const size_t gsz = sizeof(GT);
+    if (!act(&m_x, adt, x, d, 64, sizeof(ET)) || !act_r(&bm_gu.routed, gdt, xg, d, rb, gsz) ||
+        !act_r(&bm_gu.routed_small, gdt, xg, d, rs, gsz) || !act(&bm_gu.shared, gdt, xs, d, rb, gsz) ||
+        !act(&bm_gu.shared_small, gdt, xs, d, rs, gsz) || !act_r(&bm_dn.routed, ddt, hrm, Fr, rb, dsz) ||
+        !act_r(&bm_dn.routed_small, ddt, hrm, Fr, rs, dsz) || !act(&bm_dn.shared, ddt, hds, Fs, rb, dsz) ||
+        !act(&bm_dn.shared_small, ddt, hds, Fs, rs, dsz))
         return fail(h, L4MOE_ERR_CUDA, "cuTensorMapEncodeTiled failed for an activation");
 
     cudaError_t e;
@@ -556,7 +583,7 @@ l4moe_status run_layer(l4moe_handle* h, int T, const void* x, const void* Wr, co
     const int fb_gu_s = (Fs + fpg - 1) / fpg;
     const int fb_dn = (d + fpd - 1) / fpd;
     // split-K k-ranges when a small batch leaves too few tiles
-    const SplitPlan plan = split_plan(p, T, h->sms, h->top_k);
+    const SplitPlan plan = split_plan(p, T, h->sms, h->top_k, ACT8);
     const int s_gu = plan.s_gu, s_dn = plan.s_dn;
     if (E > 0 && T <= kSmallMaxTokens) {
         // a few tokens: router, top-k, permutation and row copy in one launch
@@ -687,7 +714,7 @@ l4moe_status run_layer(l4moe_handle* h, int T, const void* x, const void* Wr, co
         bm_gu, gu, st);
     if (s_gu > 1) {
         const long long n = (long long)Tv * F + (long long)T * Fs;
-        launch_k(gateup_finish_kernel<GT>, dim3((int)std::min<long long>((n + 255) / 256, 4LL * h->sms)),
+        launch_k(gateup_finish_kernel<HT>, dim3((int)std::min<long long>((n + 255) / 256, 4LL * h->sms)),
                  dim3(256), 0, st, (const float*)gu.part_routed, gu.ld_part_routed, gu.part_stride_routed,
                  (const float*)gu.part_shared, gu.ld_part_shared, gu.part_stride_shared, s_gu, Tv, T, F, Fs,
                  (const float*)gslot, (const float*)tokscale, hr, hs, err);
@@ -695,6 +722,17 @@ l4moe_status run_layer(l4moe_handle* h, int T, const void* x, const void* Wr, co
     }
     t_gu.stop();
     L4MOE_CHECK_LAUNCH("gate/up launch");
+    if constexpr (ACT8) {
+        // the hidden rows' E4M3 codes and row scales, one warp per row
+        const int Tr = E > 0 ? Tv : 0;
+        const int rows = Tr + T;
+        LaunchTimer t_q(h, 5, st);
+        launch_k(quant_hidden_kernel, dim3(std::min((rows + 7) / 8, h->sms * 8)), dim3(256), 0, st,
+                 (const __nv_bfloat16*)hr, (const __nv_bfloat16*)hs, Tr, T, F, Fs, hq_r,
+                 hq_r + (size_t)Tv * F, hsc_r, hsc_r + Tv);
+        t_q.stop();
+        L4MOE_CHECK_LAUNCH("hidden quantisation launch");
+    }
 
     GemmArgs dn{};
     dn.table = tab_dn;
@@ -710,8 +748,8 @@ l4moe_status run_layer(l4moe_handle* h, int T, const void* x, const void* Wr, co
     dn.ld_shared = d;
     dn.rowmap_routed = perm;     // slot -> token: un-permute on store
     dn.rowmap_shared = nullptr;  // shared rows are tokens
-    dn.colscale_routed = nullptr;
-    dn.colscale_shared = nullptr;
+    dn.colscale_routed = hsc_r;                       // FP8 activation mode: hidden row scales
+    dn.colscale_shared = ACT8 ? hsc_r + Tv : nullptr;
     dn.wscale = FP8W ? scales + (E + 1) : nullptr;
     dn.ksplit = s_dn;
     dn.partial_out = 1;
@@ -807,6 +845,9 @@ l4moe_status forward_impl(l4moe_handle* h, int T, const void* x, const void* Wr,
         return run_layer<__nv_bfloat16>(h, T, x, Wr, Wsgu, Wsdn, out, st, h->ws, h->ws_tokens,
                                         h->d_maps);
     case L4MOE_FP8_E4M3:
+        if (h->act8)
+            return run_layer<__nv_bfloat16, kWqAct8>(h, T, x, Wr, Wsgu, Wsdn, out, st, h->ws, h->ws_tokens,
+                                                     h->d_maps, h->d_scales);
         return run_layer<__nv_bfloat16, kWqE4M3>(h, T, x, Wr, Wsgu, Wsdn, out, st, h->ws, h->ws_tokens,
                                                  h->d_maps, h->d_scales);
     case L4MOE_INT8:
@@ -858,7 +899,7 @@ l4moe_status l4moe_forward_static(l4moe_handle* h, int T, const void* x, const v
     if (s != L4MOE_OK || T == 0) return s;
     const int E = h->p.num_experts;
     const bool fp8 = coded8(h->p.dtype);
-    const size_t ws_bytes = (ws_layout(h->p, T, h->sms, h->top_k).device_total + 255) & ~size_t(255);
+    const size_t ws_bytes = (ws_layout(h->p, T, h->sms, h->top_k, h->act8).device_total + 255) & ~size_t(255);
     const size_t maps_bytes = sizeof(CUtensorMap) * 2 * (E + 1);
     const size_t scales_bytes = fp8 ? sizeof(float*) * 2 * (E + 1) : 0;
     if (ws_bytes + maps_bytes + scales_bytes > L4MOE_STATIC_WORKSPACE_BYTES) {
@@ -878,7 +919,7 @@ l4moe_status l4moe_forward_static(l4moe_handle* h, int T, const void* x, const v
     cudaError_t e = cudaMemcpyAsync(maps, h->h_maps.data(), maps_bytes, cudaMemcpyHostToDevice, st);
     if (e != cudaSuccess) return cuda_fail(h, e, "static descriptor upload");
     // the error word and the routing kernels' ticket that follows it
-    e = cudaMemsetAsync(base + ws_layout(h->p, T, h->sms, h->top_k).err, 0, 2 * sizeof(unsigned), st);
+    e = cudaMemsetAsync(base + ws_layout(h->p, T, h->sms, h->top_k, h->act8).err, 0, 2 * sizeof(unsigned), st);
     if (e != cudaSuccess) return cuda_fail(h, e, "static error word clear");
     const float* const* scales = nullptr;
     if (fp8) {  // the scale-pointer table of 8-bit weights follows the descriptors
@@ -891,6 +932,9 @@ l4moe_status l4moe_forward_static(l4moe_handle* h, int T, const void* x, const v
     h->timing = 0;
     if (h->p.dtype == L4MOE_F32)
         s = run_layer<float>(h, T, x, W_router, Ws_gate_up, Ws_down, out, st, base, T, maps);
+    else if (h->p.dtype == L4MOE_FP8_E4M3 && h->act8)
+        s = run_layer<__nv_bfloat16, kWqAct8>(h, T, x, W_router, Ws_gate_up, Ws_down, out, st, base, T, maps,
+                                              scales);
     else if (h->p.dtype == L4MOE_FP8_E4M3)
         s = run_layer<__nv_bfloat16, kWqE4M3>(h, T, x, W_router, Ws_gate_up, Ws_down, out, st, base, T, maps,
                                               scales);
@@ -978,7 +1022,7 @@ void l4moe_destroy(l4moe_handle* h) {
 
 size_t l4moe_workspace_size(const l4moe_handle* h, int max_tokens) {
     if (!h || max_tokens < 0) return 0;
-    return ws_layout(h->p, max_tokens, h->sms, h->top_k).total;
+    return ws_layout(h->p, max_tokens, h->sms, h->top_k, h->act8).total;
 }
 
 l4moe_status l4moe_set_top_k(l4moe_handle* h, int k) {
@@ -987,7 +1031,7 @@ l4moe_status l4moe_set_top_k(l4moe_handle* h, int k) {
     if (k < 1 || k > kMaxTopK || (E > 0 && k > E) || (E == 0 && k != 1))
         return fail(h, L4MOE_ERR_ARG, "top_k must be in [1, min(4, E)]");
     if (k == h->top_k) return L4MOE_OK;
-    if (h->ws && !h->ws_owned && h->ws_bytes < ws_layout(h->p, h->ws_tokens, h->sms, k).total)
+    if (h->ws && !h->ws_owned && h->ws_bytes < ws_layout(h->p, h->ws_tokens, h->sms, k, h->act8).total)
         return fail(h, L4MOE_ERR_WORKSPACE, "the caller's workspace is too small for this top_k");
     if (h->ws && h->ws_owned) {  // re-laid out (and re-sized) by the next forward
         cudaError_t e = cudaFree(h->ws);  // synchronises: work in flight is done
@@ -999,12 +1043,35 @@ l4moe_status l4moe_set_top_k(l4moe_handle* h, int k) {
     return L4MOE_OK;
 }
 
+l4moe_status l4moe_set_act_fp8(l4moe_handle* h, int on) {
+    if (!h) return L4MOE_ERR_ARG;
+    if (on != 0 && on != 1) return fail(h, L4MOE_ERR_ARG, "act_fp8 must be 0 or 1");
+    if (on && h->p.dtype != L4MOE_FP8_E4M3)
+        return fail(h, L4MOE_ERR_DTYPE, "the FP8 activation mode needs E4M3 weights");
+    const bool a = on != 0;
+    if (a == h->act8) return L4MOE_OK;
+    if (h->ws && !h->ws_owned && h->ws_bytes < ws_layout(h->p, h->ws_tokens, h->sms, h->top_k, a).total)
+        return fail(h, L4MOE_ERR_WORKSPACE, "the caller's workspace is too small for the FP8 activation mode");
+    if (h->ws && h->ws_owned) {  // re-laid out (and re-sized) by the next forward
+        cudaError_t e = cudaFree(h->ws);  // synchronises: work in flight is done
+        h->ws = nullptr;
+        h->ws_tokens = 0;
+        if (e != cudaSuccess) return cuda_fail(h, e, "workspace cudaFree");
+    }
+    // the weight descriptors' boxes differ: encode them again at the next forward
+    h->h_maps.clear();
+    h->hkey_sgu = h->hkey_sdn = nullptr;
+    h->key_sgu = h->key_sdn = nullptr;
+    h->act8 = a;
+    return L4MOE_OK;
+}
+
 l4moe_status l4moe_set_workspace(l4moe_handle* h, void* dev_ptr, size_t bytes, int max_tokens) {
     if (!h) return L4MOE_ERR_ARG;
     if (!dev_ptr || max_tokens < 1) return fail(h, L4MOE_ERR_ARG, "null workspace or max_tokens < 1");
     if (reinterpret_cast<uintptr_t>(dev_ptr) & 255u)
         return fail(h, L4MOE_ERR_ALIGN, "workspace must be 256-byte aligned");
-    if (bytes < ws_layout(h->p, max_tokens, h->sms, h->top_k).total)
+    if (bytes < ws_layout(h->p, max_tokens, h->sms, h->top_k, h->act8).total)
         return fail(h, L4MOE_ERR_WORKSPACE, "workspace smaller than l4moe_workspace_size");
     if (h->ws_owned && h->ws) cudaFree(h->ws);
     h->ws = static_cast<uint8_t*>(dev_ptr);
@@ -1078,7 +1145,7 @@ l4moe_status l4moe_forward_host(l4moe_handle* h, int T, const void* x_host, cons
                 return cuda_fail(h, e, "copy event creation");
     }
     cudaStream_t st = static_cast<cudaStream_t>(stream);
-    const WsLayout L = ws_layout(h->p, h->ws_tokens, h->sms, h->top_k);
+    const WsLayout L = ws_layout(h->p, h->ws_tokens, h->sms, h->top_k, h->act8);
     const size_t slab = (size_t)h->ws_tokens * h->p.d_model * act_bytes(h->p.dtype);
     const int b = h->host_slot;
     h->host_slot ^= 1;
@@ -1124,7 +1191,7 @@ l4moe_status l4moe_get_routing(const l4moe_handle* h, const int32_t** idx, const
                                const float** lmax, const float** margin, const int32_t** counts,
                                const int32_t** offsets, const int32_t** perm) {
     if (!h || !h->ws) return L4MOE_ERR_ARG;
-    const WsLayout L = ws_layout(h->p, h->ws_tokens, h->sms, h->top_k);
+    const WsLayout L = ws_layout(h->p, h->ws_tokens, h->sms, h->top_k, h->act8);
     if (idx) *idx = reinterpret_cast<const int32_t*>(h->ws + L.idx);
     if (gate) *gate = reinterpret_cast<const float*>(h->ws + L.gate);
     if (lmax) *lmax = reinterpret_cast<const float*>(h->ws + L.lmax);
@@ -1143,10 +1210,10 @@ l4moe_status l4moe_check_device_status(l4moe_handle* h, void* stream) {
     if (e != cudaSuccess) return cuda_fail(h, e, "stream synchronize");
     if (!h->ws) return L4MOE_OK;
     unsigned word = 0;
-    e = cudaMemcpy(&word, h->ws + ws_layout(h->p, h->ws_tokens, h->sms, h->top_k).err, sizeof(word), cudaMemcpyDeviceToHost);
+    e = cudaMemcpy(&word, h->ws + ws_layout(h->p, h->ws_tokens, h->sms, h->top_k, h->act8).err, sizeof(word), cudaMemcpyDeviceToHost);
     if (e != cudaSuccess) return cuda_fail(h, e, "error word read");
     if (word == 0) return L4MOE_OK;
-    cudaMemset(h->ws + ws_layout(h->p, h->ws_tokens, h->sms, h->top_k).err, 0, sizeof(word));
+    cudaMemset(h->ws + ws_layout(h->p, h->ws_tokens, h->sms, h->top_k, h->act8).err, 0, sizeof(word));
     char msg[160];
     snprintf(msg, sizeof msg,
              "device error word 0x%x (1: producer wait, 2: MMA wait, 4: epilogue wait, 8: bad expert index, "
@@ -1159,7 +1226,7 @@ l4moe_status l4moe_selftest_wait(l4moe_handle* h, double limit_ms, void* stream)
     if (!(limit_ms > 0.0 && limit_ms <= 1000.0)) return fail(h, L4MOE_ERR_ARG, "limit_ms must be in (0, 1000]");
     l4moe_status s;
     if ((s = ensure_workspace(h, 1)) != L4MOE_OK) return s;
-    const WsLayout L = ws_layout(h->p, h->ws_tokens, h->sms, h->top_k);
+    const WsLayout L = ws_layout(h->p, h->ws_tokens, h->sms, h->top_k, h->act8);
     unsigned* err = reinterpret_cast<unsigned*>(h->ws + L.err);
     wait_selftest_kernel<<<1, 32, 0, static_cast<cudaStream_t>(stream)>>>(err, (uint64_t)(limit_ms * 1e6));
     ++h->launches;
@@ -1194,7 +1261,7 @@ l4moe_status l4moe_read_timing(l4moe_handle* h, double* ms, uint64_t* launches) 
 
 const char* l4moe_kernel_name(int slot) {
     static const char* names[L4MOE_NUM_KERNELS] = {"router", "permute", "row_copy", "gemm_gate_up",
-                                                   "gemm_down"};
+                                                   "gemm_down", "quant_hidden"};
     return (slot >= 0 && slot < L4MOE_NUM_KERNELS) ? names[slot] : "";
 }
 

@@ -45,6 +45,16 @@
 // token tile and for both CTAs' converted weights, and the epilogue
 // multiplies each accumulator row by its weight column's fp32 scale.
 //
+// FP8 activation mode (WQ = kWqAct8): the weights are E4M3 codes and so
+// are the token rows (x quantised per row while it is permuted, the hidden
+// rows quantised per row by their own kernel), and the MMA takes both raw:
+// kind::f8f6f4, 128 K per stage (one 128-byte token row), the weight tile as
+// two 64-feature slabs in the 64-byte swizzle (a slab row is 64 features of
+// one K row), no converter warps.  The epilogue multiplies each accumulator
+// row by its weight column's scale and each column by its token row's scale
+// (gate/up: the sigmoid gate times the x row's scale, through the same
+// column-scale path as the gate; down: the hidden row's scale).
+//
 // Tiles: a group's tiles are (feature block) x (token tile) x (k range), the
 // token tiles of one feature block adjacent so that they share the weight
 // tile through L2, in bands whose token rows stay in L2 while the band
@@ -74,6 +84,9 @@ namespace l4moe {
 
 enum GemmMode : int { MODE_GATEUP = 0, MODE_DOWN = 1 };
 
+// The MMA operand type's tiling: K per stage (one 128-byte token row), K per
+// MMA, the instruction's format code, and the MN-major weight tile's slabs
+// (A_BOX_FEATS features per slab row, one TMA box per slab) and swizzle.
 template <typename ET>
 struct ElemCfg;
 template <>
@@ -82,6 +95,7 @@ struct ElemCfg<__nv_bfloat16> {
     static constexpr int BK = 64;     // K elements per stage (one 128-byte row)
     static constexpr int MMA_K = 16;  // K per tcgen05.mma (kind::f16)
     static constexpr uint32_t FMT = 1;
+    static constexpr int A_BOX_FEATS = 64;    // one 128-byte slab row
     static constexpr uint32_t A_LAYOUT = 2;   // MN-major weights: 128B swizzle, 16B unit
     static constexpr uint32_t A_SBO = 1024;   // 8 K rows per atom
 };
@@ -91,8 +105,21 @@ struct ElemCfg<float> {
     static constexpr int BK = 32;
     static constexpr int MMA_K = 8;   // kind::tf32
     static constexpr uint32_t FMT = 2;
+    static constexpr int A_BOX_FEATS = 32;
     static constexpr uint32_t A_LAYOUT = 1;   // MN-major 32-bit: 128B swizzle, 32B unit
     static constexpr uint32_t A_SBO = 512;    // 4 K rows per atom
+};
+// E4M3 codes on both sides (the FP8 activation mode)
+struct E4M3Op {};
+template <>
+struct ElemCfg<E4M3Op> {
+    static constexpr int BYTES = 1;
+    static constexpr int BK = 128;
+    static constexpr int MMA_K = 32;  // kind::f8f6f4
+    static constexpr uint32_t FMT = 0;        // E4M3
+    static constexpr int A_BOX_FEATS = 64;    // [gate 64 | up 64] stays two slabs
+    static constexpr uint32_t A_LAYOUT = 4;   // MN-major: 64B swizzle, slab rows of 64 bytes
+    static constexpr uint32_t A_SBO = 512;    // 8 K rows per atom
 };
 
 struct GemmArgs {
@@ -133,16 +160,30 @@ __host__ __device__ constexpr int pair_features() { return MODE == MODE_GATEUP ?
 // Weight storage of a GEMM: the layer's own type, or 8-bit or 4-bit codes
 // widened in shared memory (E4M3 floats, int8 or int4 integers, per-column
 // scales).
-enum : int { kWqNone = 0, kWqE4M3 = 1, kWqInt8 = 2, kWqInt4 = 3 };
+// kWqAct8: E4M3 weights read raw by an MMA on E4M3 token rows (the FP8
+// activation mode).
+enum : int { kWqNone = 0, kWqE4M3 = 1, kWqInt8 = 2, kWqInt4 = 3, kWqAct8 = 4 };
+
+// The MMA operand type of a GEMM: the layer's type, or E4M3 codes.
+template <typename ET, int WQ>
+struct OperandOf {
+    using type = ET;
+};
+template <typename ET>
+struct OperandOf<ET, kWqAct8> {
+    using type = E4M3Op;
+};
 
 template <int MODE, typename ET, int WQ>
 struct GemmCfg {
-    static constexpr bool FP8W = WQ != kWqNone;  // coded weights, converter warps
-    using C = ElemCfg<ET>;
+    static constexpr bool ACT8 = WQ == kWqAct8;               // E4M3 x E4M3, raw operands
+    static constexpr bool FP8W = WQ != kWqNone && !ACT8;      // coded weights, converter warps
+    using C = ElemCfg<typename OperandOf<ET, WQ>::type>;
     static constexpr int A_BYTES = 128 * 128;                // 128 A rows x 128 B of K
-    static constexpr int A_BOX_FEATS = 128 / C::BYTES;       // features per A box (one 128 B slab)
+    static constexpr int A_BOX_FEATS = C::A_BOX_FEATS;       // features per A box (one slab)
     static constexpr int A_BOXES = 128 / A_BOX_FEATS;        // boxes per CTA A tile
-    static constexpr int A_BOX_BYTES = C::BK * 128;          // BK rows x 128 B
+    static constexpr int A_ROW_BYTES = A_BOX_FEATS * C::BYTES;  // bytes of one K row of a slab
+    static constexpr int A_BOX_BYTES = C::BK * A_ROW_BYTES;  // BK rows of a slab
     static constexpr int B_BOX_ROWS = 128;                   // token rows per full-tile box
     static constexpr int B_SMALL_ROWS = 32;                  // token rows per small-tile box
     static constexpr int B_BYTES = (kTokTile / 2) * 128;     // this CTA's half of the tokens
@@ -214,7 +255,7 @@ __host__ __device__ __forceinline__ TileInfo decode_tile(const GroupTable& tab, 
     ti.f0 = fb * pair_features<MODE>();
     ti.M = ti.shared ? a.m_shared : a.m_routed;
     ti.up_off = ti.shared ? a.up_shared : a.up_routed;
-    const int nkb = ti.K / ElemCfgBK;
+    const int nkb = (ti.K + ElemCfgBK - 1) / ElemCfgBK;  // a ragged last block reads zeros
     ti.kb0 = (int)(((long long)nkb * split) / a.ksplit);
     ti.kb1 = (int)(((long long)nkb * (split + 1)) / a.ksplit);
     return ti;
@@ -314,9 +355,11 @@ template <int MODE, typename ET, int WQ>
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(GemmCfg<MODE, ET, WQ>::THREADS, 1)
     moe_gemm_kernel(const __grid_constant__ BMaps bm, const GemmArgs args) {
     pdl_enter();
-    constexpr bool FP8W = WQ != kWqNone;  // coded (8- or 4-bit) weights with converter warps
     using Cfg = GemmCfg<MODE, ET, WQ>;
-    using C = ElemCfg<ET>;
+    constexpr bool FP8W = Cfg::FP8W;      // coded (8- or 4-bit) weights with converter warps
+    constexpr bool ACT8 = Cfg::ACT8;      // E4M3 weights and token rows, read raw
+    constexpr bool WSC = WQ != kWqNone;   // per-column weight scales in the epilogue
+    using C = typename Cfg::C;
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>(
         (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
@@ -488,7 +531,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(GemmCfg<MODE, ET, WQ
                 if (!mbar_wait_cluster(tempty_bar(acc), acc_phase ^ 1u, args.err, DEV_ERR_TIMEOUT_MMA))
                     break;
                 tc_fence_after();
-                // E4M3 layers: both operands f16 (format 0), else the layer's type
+                // 8-bit weight layers: both operands f16 (format 0), else the operand type
                 const uint32_t idesc = make_idesc(FP8W ? 0u : C::FMT, 1u, 0u, (uint32_t)ti.n_mma, 256u);
                 const uint32_t d_tmem = tmem_base + (uint32_t)acc * 256u;
                 bool ok = true;
@@ -509,10 +552,12 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(GemmCfg<MODE, ET, WQ
 #pragma unroll
                     for (int kk = 0; kk < C::BK / C::MMA_K; ++kk) {
                         const uint64_t bdesc = smem_desc(bb + kk * 32, 16, 1024, 2);
-                        const uint64_t adesc = smem_desc(sb + kk * C::MMA_K * 128, Cfg::A_BOX_BYTES,
-                                                         C::A_SBO, C::A_LAYOUT);
+                        const uint64_t adesc = smem_desc(sb + kk * C::MMA_K * Cfg::A_ROW_BYTES,
+                                                         Cfg::A_BOX_BYTES, C::A_SBO, C::A_LAYOUT);
                         const uint32_t accum = (kb != ti.kb0 || kk != 0) ? 1u : 0u;
-                        if constexpr (C::FMT == 1)
+                        if constexpr (ACT8)
+                            mma_f8_pair(d_tmem, adesc, bdesc, idesc, accum);
+                        else if constexpr (FP8W || C::FMT == 1)
                             mma_bf16_pair(d_tmem, adesc, bdesc, idesc, accum);
                         else
                             mma_tf32_pair(d_tmem, adesc, bdesc, idesc, accum);
@@ -604,10 +649,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(GemmCfg<MODE, ET, WQ
             const long long ld = ti.shared ? args.ld_shared : args.ld_routed;
             const int32_t* rowmap = ti.shared ? args.rowmap_shared : args.rowmap_routed;
             const float* colscale = ti.shared ? args.colscale_shared : args.colscale_routed;
-            // E4M3 weights: the scale of this TMEM lane's weight column (lane =
+            // coded weights: the scale of this TMEM lane's weight column (lane =
             // row of the A tile: gate/up [gate 64 | up 64] features, down 128)
             float wsc = 1.0f;
-            if constexpr (FP8W) {
+            if constexpr (WSC) {
                 const int r = q * 32 + lane;
                 const int f = (MODE == MODE_GATEUP) ? ti.f0 + 64 * (int)rank + (r & 63)
                                                     : ti.f0 + 128 * (int)rank + r;
@@ -631,16 +676,25 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(GemmCfg<MODE, ET, WQ
                     col = fcheck;
                 }
                 const bool fvalid = fcheck < ti.M;
+                // down: a token row's scale (the FP8 activation mode's hidden
+                // row scale) applies here; gate/up partials take theirs in the finish
+                const float* tscale = MODE == MODE_DOWN ? (ti.shared ? args.colscale_shared : args.colscale_routed)
+                                                        : nullptr;
                 for (int c = 0; c < ti.n_valid; c += 32) {
                     const bool cval = c + lane < ti.n_valid;
                     const int my_row =
                         cval ? (rowmap ? rowmap[ti.row0 + c + lane] : ti.row0 + c + lane) : 0;
+                    const float my_ts = (cval && tscale) ? tscale[ti.row0 + c + lane] : 1.0f;
                     float v[32];
                     tmem_ld_32x32(tb + (uint32_t)c, v);
                     tmem_wait_ld();
-                    if constexpr (FP8W) {
+                    if constexpr (WSC) {
 #pragma unroll
                         for (int i = 0; i < 32; ++i) v[i] *= wsc;
+                    }
+                    if constexpr (ACT8) {
+#pragma unroll
+                        for (int i = 0; i < 32; ++i) v[i] *= __shfl_sync(0xffffffffu, my_ts, i);
                     }
 #pragma unroll
                     for (int i = 0; i < 32; ++i) {
@@ -666,7 +720,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(GemmCfg<MODE, ET, WQ
                 float v[32];
                 tmem_ld_32x32(tb + (uint32_t)c, v);
                 tmem_wait_ld();
-                if constexpr (FP8W) {
+                if constexpr (WSC) {
 #pragma unroll
                     for (int i = 0; i < 32; ++i) v[i] *= wsc;
                 }

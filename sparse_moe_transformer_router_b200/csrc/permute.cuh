@@ -13,6 +13,7 @@
 #include <type_traits>
 
 #include "ptx.cuh"
+#include "quant.cuh"
 #include "schedule.cuh"
 #include "topk.cuh"
 
@@ -402,22 +403,32 @@ __device__ __forceinline__ float f16_row_scale(float amax) {
     return ldexpf(1.0f, e);
 }
 
-// Largest |x| of 8 bf16 values.
-__device__ __forceinline__ float absmax_vec(uint4 v, float m) {
-    const uint32_t w[4] = {v.x, v.y, v.z, v.w};
-#pragma unroll
-    for (int i = 0; i < 4; ++i) {
-        const float2 f = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&w[i]));
-        m = fmaxf(m, fmaxf(fabsf(f.x), fabsf(f.y)));
-    }
-    return m;
+// The scale of a token row converted from IT to OT: the power-of-two f16
+// range scale (8-bit weight layers), or the E4M3 row scale (FP8 activation
+// mode, OT = uint8_t codes).
+template <typename IT, typename OT>
+__device__ __forceinline__ float row_scale_of(float amax) {
+    if constexpr (std::is_same<OT, uint8_t>::value) return e4m3_row_scale(amax);
+    else return f16_row_scale(amax);
+}
+
+// 16 bytes of an input row (vector c) -> the same elements of the output
+// row: copied, divided by the power-of-two scale s into f16, or quantised
+// to E4M3 codes with the row scale s (8 bytes).
+template <typename IT, typename OT>
+__device__ __forceinline__ void put_row_vec(OT* orow, int c, uint4 v, float s) {
+    if constexpr (std::is_same<OT, uint8_t>::value)
+        reinterpret_cast<uint2*>(orow)[c] = bf16x8_to_e4m3(v, s);
+    else
+        reinterpret_cast<uint4*>(orow)[c] = cvt_row_vec(v, IT{}, OT{}, 1.0f / s);
 }
 
 // chunk_base (not null, after dispatch_kernel): inv[n] holds the entry's
 // rank inside its expert and chunk; its slot is chunk_base[chunk][idx[n]] +
 // inv[n], which this kernel writes back to inv[n] and records in perm.
-// tokscale (8-bit weight layers; not null): each token's power-of-two row
-// scale, written once per token; gate_slot then carries gate * scale.
+// tokscale (8-bit weight layers; not null): each token's row scale (the
+// power-of-two f16 range scale, or the E4M3 scale when OT is uint8_t codes),
+// written once per token; gate_slot then carries gate * scale.
 template <typename IT, typename OT>
 __global__ void __launch_bounds__(256) permute_rows_kernel(const IT* __restrict__ x,
                                                            const float* __restrict__ gate,
@@ -430,7 +441,8 @@ __global__ void __launch_bounds__(256) permute_rows_kernel(const IT* __restrict_
                                                            int32_t* __restrict__ perm,
                                                            float* __restrict__ tokscale) {
     pdl_enter();
-    static_assert(sizeof(IT) == sizeof(OT), "row copy keeps the element size");
+    static_assert(sizeof(IT) == sizeof(OT) || std::is_same<OT, uint8_t>::value,
+                  "row copy keeps the element size unless it quantises");
     const int lane = threadIdx.x & 31;
     const int warps = (gridDim.x * blockDim.x) >> 5;
     // one warp per entry n = t * k + j (token t's j-th expert)
@@ -450,24 +462,23 @@ __global__ void __launch_bounds__(256) permute_rows_kernel(const IT* __restrict_
         }
         if (slot < 0 || slot >= T * k) continue;  // an entry the permutation rejected (bad expert index)
         const uint4* s = reinterpret_cast<const uint4*>(x + (size_t)t * d);
-        uint4* o = reinterpret_cast<uint4*>(xp + (size_t)slot * d);
-        uint4* ot = (x_tok && n % k == 0) ? reinterpret_cast<uint4*>(x_tok + (size_t)t * d) : nullptr;
+        OT* o = xp + (size_t)slot * d;
+        OT* ot = (x_tok && n % k == 0) ? x_tok + (size_t)t * d : nullptr;
         const int nv = d * (int)sizeof(IT) / 16;
-        float sc = 1.0f;  // the row's power-of-two scale (f16 rows of 8-bit weight layers)
+        float sc = 1.0f;  // the row's scale (converted rows of 8-bit weight layers)
         if constexpr (!std::is_same<IT, OT>::value) {
             float m = 0.0f;
             for (int i = lane; i < nv; i += 32) m = absmax_vec(s[i], m);
 #pragma unroll
             for (int off = 16; off > 0; off >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, off));
-            sc = f16_row_scale(m);
+            sc = row_scale_of<IT, OT>(m);
             if (lane == 0 && tokscale && n % k == 0) tokscale[t] = sc;
         }
         if (lane == 0 && gate_slot) gate_slot[slot] = gate[n] * sc;
-        const float inv_s = 1.0f / sc;
         for (int i = lane; i < nv; i += 32) {
-            const uint4 v = cvt_row_vec(s[i], IT{}, OT{}, inv_s);
-            o[i] = v;
-            if (ot) ot[i] = v;
+            const uint4 v = s[i];
+            put_row_vec<IT, OT>(o, i, v, sc);
+            if (ot) put_row_vec<IT, OT>(ot, i, v, sc);
         }
     }
 }

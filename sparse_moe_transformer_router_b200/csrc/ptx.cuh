@@ -237,6 +237,16 @@ __device__ __forceinline__ void mma_tf32_pair(uint32_t d_tmem, uint64_t adesc, u
         "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate)
         : "memory");
 }
+// E4M3 (or other 8-bit float) operands on both sides, fp32 accumulator.
+__device__ __forceinline__ void mma_f8_pair(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc,
+                                            uint32_t idesc, uint32_t accumulate) {
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "setp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::2.kind::f8f6f4 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
+        "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate)
+        : "memory");
+}
 // Arrive once on `bar` in every CTA of `cta_mask` when all MMAs this thread
 // issued so far have completed.
 __device__ __forceinline__ void mma_commit_pair_mc(uint32_t bar, uint16_t cta_mask) {
@@ -322,16 +332,19 @@ __device__ __forceinline__ void tmem_ld_32x32(uint32_t taddr, float (&v)[32]) {
     for (int i = 0; i < 32; ++i) v[i] = __uint_as_float(r[i]);
 }
 
-// Shared-memory matrix descriptor for a 128-byte-swizzled operand tile.
+// Shared-memory matrix descriptor for a swizzled operand tile.
 //   K-major tiles: rows of 128 bytes (one MN index per row), 8-row atoms
 //     1024 bytes apart (stride byte offset); leading byte offset unused.
-//   MN-major tiles: each 128-byte row holds consecutive MN elements of one
-//     K index; K-row atoms `sbo` bytes apart (8 rows = 1024 B for the 16-byte
-//     swizzle unit, 4 rows = 512 B for the 32-byte unit that 32-bit MN-major
-//     operands require); the next 128-byte MN slab is `lbo` bytes further.
+//   MN-major tiles: each slab row (128 bytes, or 64 with the 64-byte
+//     swizzle) holds consecutive MN elements of one K index; K-row atoms
+//     `sbo` bytes apart (8 rows = 1024 B for the 16-byte swizzle unit, 4 rows
+//     = 512 B for the 32-byte unit that 32-bit MN-major operands require,
+//     8 rows of 64 B = 512 B for the 64-byte swizzle); the next MN slab is
+//     `lbo` bytes further.
 // layout: 2 = 128-byte swizzle (16-byte unit), 1 = 128-byte swizzle with a
-// 32-byte unit.  The tile base must be aligned to its atom except for the
-// sub-atom K offsets (32/64/96 bytes) used to step a K-major operand.
+// 32-byte unit, 4 = 64-byte swizzle.  The tile base must be aligned to its
+// atom except for the sub-atom K offsets (32/64/96 bytes) used to step a
+// K-major operand.
 __device__ __forceinline__ uint64_t smem_desc(uint32_t saddr, uint32_t lbo, uint32_t sbo,
                                               uint32_t layout) {
     uint64_t d = 0;
@@ -344,7 +357,8 @@ __device__ __forceinline__ uint64_t smem_desc(uint32_t saddr, uint32_t lbo, uint
 }
 
 // Instruction descriptor: fp32 accumulator, A/B element format (1 = bf16,
-// 2 = tf32 under their kinds), A MN-major flag, B MN-major flag, N, M.
+// 2 = tf32 under their kinds; 0 = f16 under kind::f16, E4M3 under
+// kind::f8f6f4), A MN-major flag, B MN-major flag, N, M.
 __host__ __device__ constexpr uint32_t make_idesc(uint32_t ab_fmt, uint32_t a_mn_major,
                                                   uint32_t b_mn_major, uint32_t n, uint32_t m) {
     return (1u << 4) | (ab_fmt << 7) | (ab_fmt << 10) | (a_mn_major << 15) | (b_mn_major << 16) |

@@ -51,9 +51,11 @@ __host__ __device__ constexpr size_t route_small_smem_bytes(int T, int E) {
 
 // Grid: ceil(d / kSmallSliceK) CTAs of kSmallThreads.  partial: [grid][T][E]
 // fp32.  ticket: a word that is 0 when the launch starts (the finishing CTA
-// leaves it at 0).  GT: the GEMMs' activation type (the layer's, or f16 for
-// 8-bit weights; x16 then receives x in f16, token order, each row divided
-// by its power-of-two scale, recorded in tokscale and folded into gslot).
+// leaves it at 0).  GT: the GEMMs' activation type (the layer's, f16 for
+// 8-bit weights, or uint8_t E4M3 codes in the FP8 activation mode; x16 then
+// receives x converted, token order, each row divided by its scale -- the
+// power-of-two f16 range scale or the E4M3 row scale -- recorded in
+// tokscale and folded into gslot).
 template <typename ET, typename GT>
 __global__ void __launch_bounds__(kSmallThreads) route_small_kernel(
     const ET* __restrict__ x, const ET* __restrict__ Wr, const float* __restrict__ bias, int T, int d,
@@ -70,7 +72,7 @@ __global__ void __launch_bounds__(kSmallThreads) route_small_kernel(
     __shared__ float s_gate[kSmallMaxEntries];
     __shared__ int32_t s_rows[kMaxGroups];        // entries per expert
     __shared__ int32_t s_off[kMaxGroups + 1];     // exclusive prefix of s_rows
-    __shared__ float s_scale[kSmallMaxTokens];    // power-of-two row scale (f16 rows; else 1)
+    __shared__ float s_scale[kSmallMaxTokens];    // row scale (converted rows; else 1)
     __shared__ unsigned s_last;
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
 
@@ -228,7 +230,7 @@ __global__ void __launch_bounds__(kSmallThreads) route_small_kernel(
             for (int i = lane; i < nv; i += 32) m = absmax_vec(reinterpret_cast<const uint4*>(x + (size_t)t * d)[i], m);
 #pragma unroll
             for (int off = 16; off > 0; off >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, off));
-            sc = f16_row_scale(m);
+            sc = row_scale_of<ET, GT>(m);
             if (lane == 0 && tokscale) tokscale[t] = sc;
         }
         if (lane == 0) s_scale[t] = sc;
@@ -301,9 +303,8 @@ __global__ void __launch_bounds__(kSmallThreads) route_small_kernel(
         const bool tok = r >= Tv;
         const int t = tok ? r - Tv : r / k;
         const int orow = tok ? t : s_off[s_ent[r]] + s_rank[r];
-        const uint4 v = cvt_row_vec(reinterpret_cast<const uint4*>(x + (size_t)t * d)[c], ET{}, GT{},
-                                    1.0f / s_scale[t]);
-        reinterpret_cast<uint4*>((tok ? x16 : xg) + (size_t)orow * d)[c] = v;
+        put_row_vec<ET, GT>((tok ? x16 : xg) + (size_t)orow * d, c,
+                            reinterpret_cast<const uint4*>(x + (size_t)t * d)[c], s_scale[t]);
     }
 }
 

@@ -1,6 +1,7 @@
 // Host-side check of the library's workspace layout and split-K plan
 // (csrc/l4moe.cu, compiled into this program): for random layer shapes,
-// dtypes, experts per token, SM counts and token budgets, every workspace
+// dtypes (E4M3 with and without the FP8 activation mode), experts per
+// token, SM counts and token budgets, every workspace
 // segment is 256-byte aligned, in order and large enough for any batch of at
 // most the budgeted tokens -- in particular the fp32 partial planes of the
 // split-K plan a batch of T tokens gets -- and every k-range of a split keeps
@@ -12,17 +13,20 @@
 
 namespace {
 
+bool g_act8 = false;  // the case being checked is in the FP8 activation mode
+
 bool fail_case(const char* what, const l4moe_params& p, int T, int k, int sms) {
-    printf("BAD %s: d %d F %d Fs %d E %d dtype %d T %d k %d sms %d\n", what, p.d_model, p.expert_ffn,
-           p.shared_ffn, p.num_experts, (int)p.dtype, T, k, sms);
+    printf("BAD %s: d %d F %d Fs %d E %d dtype %d act8 %d T %d k %d sms %d\n", what, p.d_model, p.expert_ffn,
+           p.shared_ffn, p.num_experts, (int)p.dtype, (int)g_act8, T, k, sms);
     return false;
 }
 
-bool check(const l4moe_params& p, int Tmax, int k, int sms) {
-    const WsLayout L = ws_layout(p, Tmax, sms, k);
+bool check(const l4moe_params& p, int Tmax, int k, int sms, bool act8 = false) {
+    g_act8 = act8;
+    const WsLayout L = ws_layout(p, Tmax, sms, k, act8);
     const size_t seg[] = {L.err, L.idx, L.gate, L.lmax, L.margin, L.inv, L.perm, L.gslot, L.counts, L.offsets,
-                          L.chunk, L.tab_gu, L.tab_dn, L.xg, L.hr, L.hs, L.x16, L.xsc, L.part, L.logits,
-                          L.device_total,
+                          L.chunk, L.tab_gu, L.tab_dn, L.xg, L.hr, L.hs, L.x16, L.xsc, L.hq, L.hsc, L.part,
+                          L.logits, L.device_total,
                           L.xin, L.xout, L.total};
     const int nseg = sizeof(seg) / sizeof(seg[0]);
     for (int i = 0; i < nseg; ++i) {
@@ -52,6 +56,9 @@ bool check(const l4moe_params& p, int Tmax, int k, int sms) {
         return fail_case("activation rows too small", p, Tmax, k, sms);
     if (coded8(p.dtype) && size_of(L.x16) < t * d * 2) return fail_case("f16 x too small", p, Tmax, k, sms);
     if (coded8(p.dtype) && size_of(L.xsc) < 4 * t) return fail_case("row scales too small", p, Tmax, k, sms);
+    // FP8 activation mode: hidden codes (routed [T k][F] then shared [T][Fs]) and row scales
+    if (act8 && (size_of(L.hq) < tv * F + t * Fs || size_of(L.hsc) < 4 * (tv + t)))
+        return fail_case("hidden codes / scales too small", p, Tmax, k, sms);
     if (E && size_of(L.logits) < 4 * std::min<size_t>(t, 128) * E)
         return fail_case("router logits too small", p, Tmax, k, sms);
     // the small-batch routing's partial logits [slices][T][E] for T <= kSmallMaxTokens
@@ -63,9 +70,9 @@ bool check(const l4moe_params& p, int Tmax, int k, int sms) {
         return fail_case("dispatch chunk bases too small", p, Tmax, k, sms);
     if (L.xout + 2 * t * d * a > L.total || L.xin + 2 * t * d * a > L.xout)
         return fail_case("host staging too small", p, Tmax, k, sms);
-    const int kblk = (int)(128 / a);
+    const int kblk = act8 ? 128 : (int)(128 / a);
     for (int T = 1; T <= Tmax; T = (T < 80 ? T + 1 : T * 2 + 1)) {
-        const SplitPlan sp = split_plan(p, T, sms, k);
+        const SplitPlan sp = split_plan(p, T, sms, k, act8);
         if (sp.s_gu < 1 || sp.s_gu > kMaxSplit || sp.s_dn < 1 || sp.s_dn > kMaxSplit)
             return fail_case("split count out of range", p, T, k, sms);
         if (sp.s_gu > 1 && (int)(d / kblk) / sp.s_gu < 8) return fail_case("gate/up range < 8 k-blocks", p, T, k, sms);
@@ -97,7 +104,8 @@ int main() {
         const int kmax = p.num_experts ? std::min(kMaxTopK, p.num_experts) : 1;
         const int k = 1 + (int)(rng() % kmax);
         const int Tmax = (c % 3 == 0) ? 1 + (int)(rng() % 100) : 1 + (int)(rng() % 20000);
-        if (!check(p, Tmax, k, smss[rng() % 4])) return 1;
+        const bool act8 = p.dtype == L4MOE_FP8_E4M3 && (rng() & 1);
+        if (!check(p, Tmax, k, smss[rng() % 4], act8)) return 1;
         ++cases;
     }
     // the workloads' own shapes at their token counts
@@ -108,6 +116,10 @@ int main() {
                 l4moe_params p{s[0], s[2], s[3], s[1], dt};
                 if (!check(p, Tmax, 1, 148)) return 1;
                 ++cases;
+                if (dt == L4MOE_FP8_E4M3) {
+                    if (!check(p, Tmax, 1, 148, true)) return 1;
+                    ++cases;
+                }
             }
     printf("OK %d\n", cases);
     return 0;

@@ -6,8 +6,8 @@ import numpy as np
 import pytest
 import torch
 
-from parity_util import (check_outputs, check_routing, check_routing_topk, describe, make_layer,
-                         oracle_routing, run_gpu, sample_tokens)
+from parity_util import (check_outputs, check_outputs_act8, check_routing, check_routing_topk, describe,
+                         make_layer, oracle_routing, run_gpu, sample_tokens)
 from sparse_moe_transformer_router_b200.workloads import (CONFIGS, DECODE_TOKENS,
                                                           E4M3_FINITE_CODES, E4M3_SUBNORMAL_CODES,
                                                           INT4_CODES, INT8_CODES, LayerConfig, generate,
@@ -165,7 +165,10 @@ DENSE = {
 
 
 def _dense_forward(inp):
-    layer = make_layer(inp)
+    return _dense_forward_on(make_layer(inp), inp)
+
+
+def _dense_forward_on(layer, inp):
     out = layer.forward(inp.x, None, [], [], inp.Ws_gate_up, inp.Ws_down)
     torch.cuda.synchronize()
     layer.check_device_status()
@@ -177,6 +180,84 @@ def test_dense_layer_matches_oracle(name):
     inp = generate(DENSE[name], seed=0, device="cuda")
     res = check_outputs(inp, _dense_forward(inp), None)
     print(f"{name}: {describe(res)}")
+
+
+ACT8 = {
+    # FP8 activation mode: E4M3 x E4M3 tensor-core contractions with per-row
+    # token scales (ragged token and feature tiles, idle experts)
+    "act8_ragged": (LayerConfig("act8_ragged", 300, 256, 8, 384, 256, "fp8", wr_std=0.1), 1),
+    # d = 192: the second 128-deep k-block is half past the rows (zero-filled)
+    "act8_zipf_d192": (LayerConfig("act8_zipf_d192", 700, 192, 16, 128, 320, "fp8", router="zipf", n_dead=4,
+                                   wr_std=0.05), 1),
+    "act8_T1": (LayerConfig("act8_T1", 1, 256, 8, 256, 256, "fp8", wr_std=0.1), 1),
+    # the one-launch small-batch routing writes the codes
+    "act8_T9_zipf": (LayerConfig("act8_T9_zipf", 9, 256, 16, 128, 128, "fp8", router="zipf", n_dead=4,
+                                 wr_std=0.05), 1),
+    # split-K: gate/up partials finished in bf16 before the quantisation;
+    # down partials take the hidden row scales
+    "act8_splitk": (LayerConfig("act8_splitk", 2, 1024, 8, 1024, 1024, "fp8", wr_std=0.03), 1),
+    "act8_k2": (LayerConfig("act8_k2", 300, 256, 8, 384, 256, "fp8", wr_std=0.1), 2),
+    "act8_dense": (LayerConfig("act8_dense", 300, 256, 0, 0, 320, "fp8"), 1),
+    "act8_T40_E32": (LayerConfig("act8_T40_E32", 40, 512, 32, 512, 768, "fp8", wr_std=0.05), 1),
+}
+
+
+def _act8_run(inp, k=1):
+    layer = make_layer(inp)
+    layer.set_act_fp8(True)
+    if k > 1:
+        layer.set_top_k(k)
+    if inp.cfg.num_experts == 0:
+        return layer, _dense_forward_on(layer, inp), None
+    out, r = run_gpu(layer, inp)
+    return layer, out, r
+
+
+@pytest.mark.parametrize("name", list(ACT8))
+def test_act8_layer_matches_oracle(name):
+    cfg, k = ACT8[name]
+    inp = generate(cfg, seed=0, device="cuda")
+    _, out, r = _act8_run(inp, k)
+    if r is None:
+        res = check_outputs_act8(inp, out, None)
+        print(f"{name}: {describe(res)}, scale-excluded {res['scale_excluded']}")
+        return
+    rep = check_routing(inp, r) if k == 1 else check_routing_topk(inp, r, k)
+    res = check_outputs_act8(inp, out, None, rep["same"], rep["o_idx"], k=k)
+    print(f"{name}: {describe(res)}, excluded {rep['excluded']}, flipped {rep['flipped']}, "
+          f"scale-excluded {res['scale_excluded']}")
+
+
+def test_act8_mode_is_opt_in_and_for_e4m3_weights_only():
+    from sparse_moe_transformer_router_b200.binding import ERR_DTYPE, L4MoEError
+    inp = generate(ACT8["act8_ragged"][0], seed=0, device="cuda")
+    layer = make_layer(inp)
+    plain, _ = run_gpu(layer, inp)
+    layer.set_act_fp8(True)
+    q, _ = run_gpu(layer, inp)
+    layer.set_act_fp8(False)
+    back, _ = run_gpu(layer, inp)
+    assert torch.equal(plain, back) and not torch.equal(plain, q)
+    bf = generate(SMALL["bf16_ragged"], seed=0, device="cuda")
+    with pytest.raises(L4MoEError) as ei:
+        make_layer(bf).set_act_fp8(True)
+    assert ei.value.status == ERR_DTYPE
+
+
+def test_full_size_maverick_fp8_act8():
+    """Maverick-shaped E4M3 layer (T 16384, Zipf loads) in the FP8 activation
+    mode: routing of every token, outputs of a stratified sample."""
+    cfg = CONFIGS["maverick_fp8"]
+    inp = generate(cfg, seed=0, device="cuda")
+    layer, out, r = _act8_run(inp)
+    ora = oracle_routing(inp)
+    rep = check_routing(inp, r, ora)
+    toks = sample_tokens(r, rep, cfg.T, seed=0)
+    res = check_outputs_act8(inp, out, toks, rep["same"], rep["o_idx"])
+    print(f"{cfg.name} act8: {describe(res)}, excluded {rep['excluded']}, flipped {rep['flipped']}, "
+          f"scale-excluded {res['scale_excluded']}")
+    del inp, layer
+    torch.cuda.empty_cache()
 
 
 def test_full_size_maverick_dense_layer():

@@ -141,3 +141,99 @@ def test_hidden_rounding_flips_stay_within_the_reading_slack(hidden, tdt):
     if hidden == "bf16":
         assert dy > 1e-3      # far above fp32 noise: the flips themselves
     print(f"{hidden}: {flipped:.2e} of hidden values flipped, max output change {dy:.2e} * rms")
+
+
+def _e4m3_rows_lib(v: torch.Tensor):
+    """Per-row E4M3 quantisation with torch's casts (fp64 values out) and
+    the row scales: s = fp32(max|v| / 448), 1 for a zero row."""
+    s = v.float().abs().amax(dim=1, keepdim=True) / 448.0
+    s = torch.where(s == 0, torch.ones_like(s), s)
+    q = (v.float() / s).to(torch.float8_e4m3fn)
+    return q.double() * s.double(), s
+
+
+def _bf16_margin_lib(h: torch.Tensor) -> np.ndarray:
+    """The hidden-scale margin of each row by torch's bf16 arithmetic: for
+    every element within one bf16 spacing of the row's largest |fp32 value|,
+    its distance to the midpoints between its bf16 neighbours (found with
+    nextafter in bf16), relative to that largest value; the row minimum."""
+    a = h.float().abs()
+    m = a.amax(dim=1, keepdim=True)
+    lo = torch.from_numpy((a.numpy().view(np.uint32) & np.uint32(0xFFFF0000)).view(np.float32))
+    lo_b = lo.bfloat16()
+    hi_b = torch.nextafter(lo_b, torch.full_like(lo_b, float("inf")))
+    below_b = torch.nextafter(lo_b, torch.zeros_like(lo_b))
+    a64, lo64 = a.double(), lo_b.double()
+    d_up = (a64 - (lo64 + hi_b.double()) / 2).abs()
+    d_dn = (a64 - (lo64 + below_b.double()) / 2).abs()
+    dist = torch.minimum(d_up, d_dn) / m.double()
+    near = (a64 >= m.double() * (1 - 2.0 ** -7)) & (a64 > 0)
+    return torch.where(near, dist, torch.full_like(dist, float("inf"))).amin(dim=1).numpy()
+
+
+def test_act8_scale_margin_matches_a_library_evaluation():
+    """The oracle's hidden-scale margin (FP8 activation mode) equals a torch
+    evaluation on the same hidden rows, on a dense layer (one hidden row per
+    token); and rows whose margin is large keep their scale under a relative
+    perturbation well below it, while perturbing a row's largest element
+    across its nearest midpoint changes the scale."""
+    cfg = LayerConfig("margin", 200, 128, 0, 0, 512, "bf16")
+    inp = generate(cfg, seed=4, device="cpu")
+    from parity_util import w_storage
+    x = inp.x.double()
+    xq, _ = _e4m3_rows_lib(x)
+    a = xq @ inp.Ws_gate_up.double()
+    h = torch.nn.functional.silu(a[:, :512]) * a[:, 512:]
+    want = _bf16_margin_lib(h)
+    res = oracle.forward(w_storage(inp.x, "bf16"), np.zeros((128, 0), np.uint16), [], [],
+                         w_storage(inp.Ws_gate_up, "bf16"), w_storage(inp.Ws_down, "bf16"),
+                         act_fp8=True, scale_margin=True)
+    got = res[-1]
+    np.testing.assert_allclose(got, want, rtol=1e-9, atol=1e-15)
+    assert np.all(np.isfinite(got)) and got.min() < 1e-3 < got.max()
+    _, s0 = _e4m3_rows_lib(h.float().bfloat16().double())
+    wide = got > 1e-4
+    hp = h * (1 + 3e-5 * torch.from_numpy(np.random.default_rng(5).standard_normal(tuple(h.shape))))
+    _, s1 = _e4m3_rows_lib(hp.float().bfloat16().double())
+    assert torch.equal(s0[wide], s1[wide])
+    # the row with the smallest margin: push its largest element across the midpoint
+    r = int(np.argmin(got))
+    j = int(h[r].abs().argmax())
+    hq = h.clone()
+    step = 4 * got[r] * float(h[r].abs().max())
+    for sgn in (1.0, -1.0):
+        hq[r, j] = h[r, j] + sgn * step * np.sign(float(h[r, j]))
+        _, s2 = _e4m3_rows_lib(hq.float().bfloat16().double())
+        if not torch.equal(s2[r], s0[r]):
+            break
+    assert not torch.equal(s2[r], s0[r])
+
+
+def test_act8_hidden_flips_stay_within_the_reading_slack():
+    """The FP8 activation mode's reading slack: with every hidden value of a
+    layer (hidden width 2048) perturbed by a relative 1e-6 (fp32 accumulation
+    error) before its bf16 rounding and E4M3 quantisation, the tokens whose
+    scale margin is at least SCALE_MARGIN_EXCLUDE keep their scales, and
+    their outputs move by at most READING_SLACK["act8"] * rms -- by more than
+    the bf16 slack: a flipped code moves its element by a whole E4M3 step."""
+    from parity_util import SCALE_MARGIN_EXCLUDE
+    F = 2048
+    cfg = LayerConfig("act8_flips", 300, 512, 0, 0, F, "bf16")
+    inp = generate(cfg, seed=0, device="cpu")
+    xq, _ = _e4m3_rows_lib(inp.x.double())
+    a = xq @ inp.Ws_gate_up.double()
+    h = torch.nn.functional.silu(a[:, :F]) * a[:, F:]
+    Wd = inp.Ws_down.double()
+    margin = _bf16_margin_lib(h)
+    keep = margin >= SCALE_MARGIN_EXCLUDE
+    worst = 0.0
+    for seed in (1, 2, 3):
+        hn = h * (1 + 1e-6 * torch.from_numpy(np.random.default_rng(seed).standard_normal(tuple(h.shape))))
+        q, s = _e4m3_rows_lib(h.float().bfloat16().double())
+        qn, sn = _e4m3_rows_lib(hn.float().bfloat16().double())
+        assert torch.equal(s[torch.from_numpy(keep)], sn[torch.from_numpy(keep)])
+        y, yn = q @ Wd, qn @ Wd
+        rms = y.pow(2).mean().sqrt().item()
+        worst = max(worst, ((yn - y).abs().amax(dim=1).numpy()[keep]).max() / rms)
+    assert 5e-3 < worst <= READING_SLACK["act8"]
+    print(f"act8: {np.count_nonzero(~keep)} of {keep.size} tokens excluded, worst output change {worst:.3e} * rms")
