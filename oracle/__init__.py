@@ -88,6 +88,8 @@ def _load():
             lib.oracle_round_hidden.argtypes = [ctypes.c_double, i32]
             lib.oracle_e4m3_encode.restype = ctypes.c_uint8
             lib.oracle_e4m3_encode.argtypes = [ctypes.c_float]
+            lib.oracle_e4m3_row.restype = ctypes.c_float
+            lib.oracle_e4m3_row.argtypes = [i32, vp, vp]
             lib.oracle_num_threads.restype = ctypes.c_int
             lib.oracle_num_threads.argtypes = []
             _lib = lib
@@ -128,6 +130,19 @@ def e4m3_to_f64(code: int) -> float:
 def e4m3_encode(v: float) -> int:
     """E4M3 code of an fp32 value (round to nearest even, saturating)."""
     return int(_load().oracle_e4m3_encode(float(np.float32(v))))
+
+
+def e4m3_rows(v: np.ndarray):
+    """The FP8 activation mode's quantisation of each row of v (fp32 values):
+    (codes uint8 [rows, n], scales float32 [rows])."""
+    v = np.ascontiguousarray(v, dtype=np.float32)
+    rows, n = v.shape
+    codes = np.empty((rows, n), np.uint8)
+    scales = np.empty(rows, np.float32)
+    lib = _load()
+    for i in range(rows):
+        scales[i] = lib.oracle_e4m3_row(n, v[i].ctypes.data, codes[i].ctypes.data)
+    return codes, scales
 
 
 def route(x: np.ndarray, Wr: np.ndarray, bias: np.ndarray | None = None):
@@ -228,7 +243,8 @@ def forward(x, Wr, W_gate_up, W_down, Ws_gate_up, Ws_down, *, bias=None,
     own logit, and their outputs add to the shared expert's.  Returns
     (out f64[n_sel, d], idx int32[n_sel], gate f64[n_sel]), or [n_sel, k]
     index and gate arrays for k > 1.  act_fp8: the FP8 activation mode (every
-    contraction input row quantised to E4M3 with its own fp32 scale; a hidden
+    contraction input row quantised to E4M3 with its own fp32 scale, the
+    row multiplied by the scale's reciprocal; a hidden
     row is first held in the layer's activation type, bf16 for bf16 inputs;
     the hidden-rounding output then equals the plain one).
     hidden_round ("bf16" or "f16"): also return, as a fourth element, the

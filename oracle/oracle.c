@@ -44,8 +44,8 @@
  *     Llama 4 Yourself": Maverick served with FP8 quantisation): each
  *     contraction input row -- a token's x, and a token's hidden row of each
  *     expert it runs -- is quantised to E4M3 with its own scale:
- *     s = fp32(max|v| / 448) (1 for an all-zero row), code =
- *     e4m3_rne_satfinite(fp32(v / s)), value = code * s.  A hidden row is
+ *     s = fp32(max|v| / 448) (at least 2^-126; 1 for an all-zero row), code =
+ *     e4m3_rne_satfinite(fp32(v * fp32(1 / s))), value = code * s.  A hidden row is
  *     held in the layer's activation type before it is quantised: each
  *     value is rounded to fp32 and then, in layers with bf16 activations, to
  *     bf16 (round to nearest even).  The gate still scales the routed
@@ -129,20 +129,34 @@ uint8_t oracle_e4m3_encode(float v) {
     return sign | (uint8_t)(((E + 7) << 3) | (int)f);
 }
 
-/* FP8 activation mode: v[0..n) (fp64 values, first rounded to fp32) replaced
- * by their E4M3 quantisation with one scale for the row (see the header). */
-static void quantise_row_e4m3(int n, double *v) {
+/* FP8 activation mode, one row of fp32 values v[0..n): its scale
+ * s = fp32(max|v| / 448), at least 2^-126 (the smallest normal fp32, so that
+ * 1 / s is finite), and 1 for an all-zero row, is returned; codes[j] =
+ * e4m3_rne_satfinite(fp32(v[j] * fp32(1 / s))) (see the header). */
+float oracle_e4m3_row(int n, const float *v, uint8_t *codes) {
     float amax = 0.0f;
     for (int j = 0; j < n; ++j) {
-        float a = fabsf((float)v[j]);
+        float a = fabsf(v[j]);
         if (a > amax) amax = a;
     }
     float s = amax / 448.0f;
-    if (s == 0.0f) s = 1.0f;
-    for (int j = 0; j < n; ++j) {
-        float q = (float)v[j] / s;
-        v[j] = oracle_e4m3_to_double(oracle_e4m3_encode(q)) * (double)s;
-    }
+    if (s < 0x1p-126f) s = 0x1p-126f;
+    if (amax == 0.0f) s = 1.0f;
+    const float rcp = 1.0f / s;
+    for (int j = 0; j < n; ++j) codes[j] = oracle_e4m3_encode(v[j] * rcp);
+    return s;
+}
+
+/* FP8 activation mode: v[0..n) (fp64 values, first rounded to fp32) replaced
+ * by their E4M3 quantisation with one scale for the row: code * s. */
+static void quantise_row_e4m3(int n, double *v) {
+    float *f = (float *)calloc((size_t)(n > 0 ? n : 1), sizeof(float));
+    uint8_t *c = (uint8_t *)malloc((size_t)(n > 0 ? n : 1));
+    for (int j = 0; j < n; ++j) f[j] = (float)v[j];
+    const float s = oracle_e4m3_row(n, f, c);
+    for (int j = 0; j < n; ++j) v[j] = oracle_e4m3_to_double(c[j]) * (double)s;
+    free(f);
+    free(c);
 }
 
 static double load_elem(const void *p, int dtype, size_t i) {

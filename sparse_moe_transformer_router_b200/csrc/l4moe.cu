@@ -723,11 +723,11 @@ l4moe_status run_layer(l4moe_handle* h, int T, const void* x, const void* Wr, co
     t_gu.stop();
     L4MOE_CHECK_LAUNCH("gate/up launch");
     if constexpr (ACT8) {
-        // the hidden rows' E4M3 codes and row scales, one warp per row
+        // the hidden rows' E4M3 codes and row scales, one CTA per row at a time
         const int Tr = E > 0 ? Tv : 0;
         const int rows = Tr + T;
         LaunchTimer t_q(h, 5, st);
-        launch_k(quant_hidden_kernel, dim3(std::min((rows + 7) / 8, h->sms * 8)), dim3(256), 0, st,
+        launch_k(quant_hidden_kernel, dim3(std::min(rows, h->sms * 8)), dim3(kQuantThreads), 0, st,
                  (const __nv_bfloat16*)hr, (const __nv_bfloat16*)hs, Tr, T, F, Fs, hq_r,
                  hq_r + (size_t)Tv * F, hsc_r, hsc_r + Tv);
         t_q.stop();

@@ -64,12 +64,14 @@
 // per CTA (measured: a box's issue cost dominated with 64-row boxes), else
 // as 32-row boxes.
 //
-// Roles (192 threads per CTA, 448 with E4M3 weights): warp 0 lane 0 issues TMA loads into a
-// STAGES-deep ring (both CTAs; completion counted on the leader's barrier);
-// warp 1 allocates TMEM (both CTAs) and, in the leader CTA only, lane 0
-// issues the MMAs and commits to both CTAs' barriers; warps 2..5 are the
-// epilogue (warp w reads TMEM lanes 32*(w%4) .. +31) and release the
-// accumulator to the leader.  Every mbarrier wait is bounded: on a timeout a
+// Roles (320 threads per CTA; 448 with widened coded weights): warp 0 lane 0
+// issues TMA loads into a STAGES-deep ring (both CTAs; completion counted on
+// the leader's barrier); warp 1 allocates TMEM (both CTAs) and, in the
+// leader CTA only, lane 0 issues the MMAs and commits to both CTAs'
+// barriers; warps 2..9 are the epilogue (warp w reads TMEM lanes
+// 32*(w%4) .. +31, the two warps of a lane quarter alternate 32-column
+// chunks; with widened coded weights warps 2..5 alone, one per quarter,
+// then the converter warps) and release the accumulator to the leader.  Every mbarrier wait is bounded: on a timeout a
 // role records a bit in the error word and returns; the leader drains the
 // copies and MMAs in flight before the pair synchronises and frees TMEM.
 #pragma once
@@ -195,10 +197,18 @@ struct GemmCfg {
     static constexpr int STAGES = FP8W ? 5 : 6;
     static constexpr int ACC_BUFS = 2;
     static constexpr int TMEM_COLS = 512;
-    static constexpr int CONV_WARPS = FP8W ? 8 : 0;         // E4M3 widening warps (6..13)
-    static constexpr int THREADS = 192 + 32 * CONV_WARPS;
+    // epilogue warps: one per TMEM lane quarter, or two (each taking every
+    // other 32-column chunk) where a tile's mainloop is short enough that
+    // one warp per quarter cannot keep up (the E4M3 x E4M3 tiles: half the
+    // k-blocks of a bf16 tile for the same epilogue work)
+    static constexpr int EPI_WARPS = FP8W ? 4 : 8;
+    static constexpr int EPI_HALVES = EPI_WARPS / 4;
+    static constexpr int CONV_WARPS = FP8W ? 8 : 0;         // widening warps (after the epilogue's)
+    static constexpr int CONV_WARP0 = 2 + EPI_WARPS;
+    static constexpr int THREADS = 64 + 32 * EPI_WARPS + 32 * CONV_WARPS;
     static constexpr int XLD = 17;                           // exchange row stride (floats)
-    static constexpr int XCH_BYTES = (MODE == MODE_GATEUP) ? 2 * 2 * 32 * XLD * 4 : 0;
+    static constexpr int XCH_FLOATS = 2 * 2 * 32 * XLD;      // one half's exchange buffers
+    static constexpr int XCH_BYTES = (MODE == MODE_GATEUP) ? EPI_HALVES * XCH_FLOATS * 4 : 0;
     static constexpr int NUM_BARS = 2 * STAGES + 2 * ACC_BUFS + 1 + (FP8W ? 2 * STAGES : 0);
     static constexpr size_t SMEM_BYTES = 1024 /*alignment slack*/ + (size_t)STAGES * STAGE_BYTES +
                                          XCH_BYTES + NUM_BARS * 8 + 16 + sizeof(GroupTable);
@@ -398,7 +408,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(GemmCfg<MODE, ET, WQ
         }
         for (int b = 0; b < Cfg::ACC_BUFS; ++b) {
             mbar_init(tfull_bar(b), 1);
-            mbar_init(tempty_bar(b), 8);  // leader: 4 epilogue warps of each CTA
+            mbar_init(tempty_bar(b), 2 * Cfg::EPI_WARPS);  // leader: the epilogue warps of each CTA
         }
         mbar_init(drain_bar, 1);
         if constexpr (FP8W) {
@@ -579,11 +589,11 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(GemmCfg<MODE, ET, WQ
             mma_commit_pair(drain_bar);
             mbar_wait(drain_bar, 0, args.err, DEV_ERR_TIMEOUT_MMA);
         }
-    } else if (FP8W && warp >= 6) {
+    } else if (FP8W && warp >= Cfg::CONV_WARP0) {
         // --------------------------------------- weight-code converters (E4M3, int8, int4)
         constexpr int NCT = 32 * (Cfg::CONV_WARPS > 0 ? Cfg::CONV_WARPS : 8);  // converter threads
         static_assert(NCT == 256, "each converter thread owns 4 units: slab i / 2");
-        const int ct = threadIdx.x - 192;           // 0 .. NCT-1
+        const int ct = threadIdx.x - 32 * Cfg::CONV_WARP0;  // 0 .. NCT-1
         const int c8 = ct & 7;                      // 8-feature chunk of each slab this thread owns
         int stage = 0;
         uint32_t phase = 0;
@@ -628,6 +638,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(GemmCfg<MODE, ET, WQ
     } else {
         // ---------------------------------------------------- epilogue
         const int q = warp & 3;  // TMEM lane quarter of this warp
+        const int half = (warp - 2) >> 2;  // which 32-column chunks: half, half + halves, ...
+        constexpr int CSTEP = 32 * Cfg::EPI_HALVES;
+        float* xch_h = xch + half * Cfg::XCH_FLOATS;  // this half's exchange buffers
+        const uint32_t bar_id = 1u + (uint32_t)half;  // this half's named barrier
         int acc = 0;
         uint32_t acc_phase = 0;
         volatile uint32_t* abort_flag = misc + 1;
@@ -635,9 +649,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(GemmCfg<MODE, ET, WQ
             const TileInfo ti = decode_tile<MODE, C::BK, C::BYTES>(*tab, args, L);
             const bool ok = mbar_wait(tfull_bar(acc), acc_phase, args.err, DEV_ERR_TIMEOUT_EPILOGUE);
             if constexpr (MODE == MODE_GATEUP) {
-                // the 4 warps meet at named barriers below: leave together or not at all
+                // the 4 warps of a half meet at named barriers below: leave together or not at all
                 if (!__all_sync(0xffffffffu, ok) && lane == 0) *abort_flag = 1u;
-                named_bar_sync(1, 128);
+                named_bar_sync(bar_id, 128);
                 if (*abort_flag) break;
             } else {
                 if (!__all_sync(0xffffffffu, ok)) break;
@@ -680,7 +694,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(GemmCfg<MODE, ET, WQ
                 // row scale) applies here; gate/up partials take theirs in the finish
                 const float* tscale = MODE == MODE_DOWN ? (ti.shared ? args.colscale_shared : args.colscale_routed)
                                                         : nullptr;
-                for (int c = 0; c < ti.n_valid; c += 32) {
+                for (int c = 32 * half; c < ti.n_valid; c += CSTEP) {
                     const bool cval = c + lane < ti.n_valid;
                     const int my_row =
                         cval ? (rowmap ? rowmap[ti.row0 + c + lane] : ti.row0 + c + lane) : 0;
@@ -711,7 +725,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(GemmCfg<MODE, ET, WQ
                 }
                 continue;
             }
-            for (int c = 0; c < ti.n_valid; c += 32) {
+            for (int c = 32 * half; c < ti.n_valid; c += CSTEP) {
                 // output row (token or slot) and scale of each of the 32 columns, one per lane
                 const bool cval = c + lane < ti.n_valid;
                 const int my_row =
@@ -730,14 +744,14 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(GemmCfg<MODE, ET, WQ
                     // columns c+16..c+31; each hands the other half over.
                     const bool gate_warp = q < 2;
                     const int pq = q & 1;  // feature quarter of the pair
-                    float* xg = xch + (0 * 2 + pq) * 32 * Cfg::XLD;  // gate values, cols 16..31
-                    float* xu = xch + (1 * 2 + pq) * 32 * Cfg::XLD;  // up values, cols 0..15
+                    float* xg = xch_h + (0 * 2 + pq) * 32 * Cfg::XLD;  // gate values, cols 16..31
+                    float* xu = xch_h + (1 * 2 + pq) * 32 * Cfg::XLD;  // up values, cols 0..15
 #pragma unroll
                     for (int i = 0; i < 16; ++i) {
                         if (gate_warp) xg[lane * Cfg::XLD + i] = v[16 + i];
                         else xu[lane * Cfg::XLD + i] = v[i];
                     }
-                    named_bar_sync(1, 128);
+                    named_bar_sync(bar_id, 128);
                     const int f = ti.f0 + 64 * (int)rank + 32 * pq + lane;
                     const bool fvalid = f < ti.M;
                     const int cb = gate_warp ? 0 : 16;
@@ -756,7 +770,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(GemmCfg<MODE, ET, WQ
                         if (fvalid && c + col < ti.n_valid)
                             store_elem(outp + (size_t)orow * ld + f, hv);
                     }
-                    named_bar_sync(1, 128);  // exchange buffer free for the next chunk
+                    named_bar_sync(bar_id, 128);  // exchange buffer free for the next chunk
                 } else {
                     const int f = ti.f0 + 128 * (int)rank + 32 * q + lane;
                     const bool fvalid = f < ti.M;

@@ -413,14 +413,15 @@ __device__ __forceinline__ float row_scale_of(float amax) {
 }
 
 // 16 bytes of an input row (vector c) -> the same elements of the output
-// row: copied, divided by the power-of-two scale s into f16, or quantised
-// to E4M3 codes with the row scale s (8 bytes).
+// row: copied, divided by the power-of-two scale q.s into f16 (times its
+// reciprocal, exact for a power of two), or quantised to E4M3 codes with the
+// row scale q.s (8 bytes).
 template <typename IT, typename OT>
-__device__ __forceinline__ void put_row_vec(OT* orow, int c, uint4 v, float s) {
+__device__ __forceinline__ void put_row_vec(OT* orow, int c, uint4 v, const RowScale& q) {
     if constexpr (std::is_same<OT, uint8_t>::value)
-        reinterpret_cast<uint2*>(orow)[c] = bf16x8_to_e4m3(v, s);
+        reinterpret_cast<uint2*>(orow)[c] = bf16x8_to_e4m3(v, q);
     else
-        reinterpret_cast<uint4*>(orow)[c] = cvt_row_vec(v, IT{}, OT{}, 1.0f / s);
+        reinterpret_cast<uint4*>(orow)[c] = cvt_row_vec(v, IT{}, OT{}, q.r);
 }
 
 // chunk_base (not null, after dispatch_kernel): inv[n] holds the entry's
@@ -475,10 +476,11 @@ __global__ void __launch_bounds__(256) permute_rows_kernel(const IT* __restrict_
             if (lane == 0 && tokscale && n % k == 0) tokscale[t] = sc;
         }
         if (lane == 0 && gate_slot) gate_slot[slot] = gate[n] * sc;
+        const RowScale q = row_scale(sc);
         for (int i = lane; i < nv; i += 32) {
             const uint4 v = s[i];
-            put_row_vec<IT, OT>(o, i, v, sc);
-            if (ot) put_row_vec<IT, OT>(ot, i, v, sc);
+            put_row_vec<IT, OT>(o, i, v, q);
+            if (ot) put_row_vec<IT, OT>(ot, i, v, q);
         }
     }
 }

@@ -304,7 +304,7 @@ __global__ void __launch_bounds__(kSmallThreads) route_small_kernel(
         const int t = tok ? r - Tv : r / k;
         const int orow = tok ? t : s_off[s_ent[r]] + s_rank[r];
         put_row_vec<ET, GT>((tok ? x16 : xg) + (size_t)orow * d, c,
-                            reinterpret_cast<const uint4*>(x + (size_t)t * d)[c], s_scale[t]);
+                            reinterpret_cast<const uint4*>(x + (size_t)t * d)[c], row_scale(s_scale[t]));
     }
 }
 

@@ -450,13 +450,20 @@ def test_e4m3_encoder_round_trips_every_code_and_matches_torch():
         assert oracle.e4m3_encode(big) == 0x7E and oracle.e4m3_encode(-big) == 0xFE
 
 
+def _e4m3_scale_lib(v: torch.Tensor) -> torch.Tensor:
+    """Row scales by torch's fp32 arithmetic: max|v| / 448, at least 2^-126,
+    1 for a zero row."""
+    m = v.abs().amax(dim=1, keepdim=True)
+    s = torch.clamp_min(m / 448.0, 2.0 ** -126)
+    return torch.where(m == 0, torch.ones_like(s), s)
+
+
 def _e4m3_rows(v64: np.ndarray) -> np.ndarray:
-    """Per-row E4M3 quantisation through torch: s = fp32(max|v| / 448), codes
-    = float8 cast of fp32(v / s), values = codes * s (fp64)."""
+    """Per-row E4M3 quantisation through torch: s as _e4m3_scale_lib, codes
+    = float8 cast of fp32(v * fp32(1 / s)), values = codes * s (fp64)."""
     v = torch.from_numpy(np.ascontiguousarray(v64)).float()
-    s = v.abs().amax(dim=1, keepdim=True) / 448.0
-    s = torch.where(s == 0, torch.ones_like(s), s)
-    q = (v / s).to(torch.float8_e4m3fn)
+    s = _e4m3_scale_lib(v)
+    q = (v * (1.0 / s)).to(torch.float8_e4m3fn)
     return (q.double() * s.double()).numpy()
 
 
@@ -556,3 +563,42 @@ def test_expert_rows_equals_a_library_swiglu_on_gated_rows():
     a8 = (x.double() * torch.from_numpy(g)[:, None]) @ (q_gu.double() * torch.from_numpy(s_gu).double())
     lib8 = (torch.nn.functional.silu(a8[:, :F]) * a8[:, F:]) @ (q_d.double() * torch.from_numpy(s_d).double())
     np.testing.assert_allclose(y8, lib8.numpy(), rtol=1e-12, atol=1e-13)
+
+
+def test_e4m3_row_quantisation_matches_torch_and_handles_ties_and_zero_rows():
+    """oracle.e4m3_rows (the FP8 activation mode's per-row step): the scale
+    is fp32(max|v| / 448) (at least 2^-126, 1 for a zero row) and the codes
+    equal torch's float8_e4m3fn cast of fp32(v * fp32(1 / s)), including rows
+    whose values scale to exact midpoints between two codes (ties to even),
+    rows too small for 1 / s to be finite without the 2^-126 floor, and rows
+    where dividing by s instead would give other codes."""
+    rng = np.random.default_rng(31)
+    v = (rng.standard_normal((50, 96)) * np.exp2(rng.uniform(-30, 30, size=(50, 1)))).astype(np.float32)
+    vals = np.array([oracle.e4m3_to_f64(c) for c in range(0x00, 0x7F)])
+    mids = ((vals[:-1] + vals[1:]) / 2).astype(np.float32)
+    tie = rng.choice(np.concatenate([mids, -mids]), size=96).astype(np.float32) * np.float32(2.0 ** -5)
+    tie[0] = 448.0 * 2.0 ** -5
+    tiny = (rng.standard_normal(96) * 1e-39).astype(np.float32)   # max / 448 below 2^-126
+    # rows (bf16 values, as the layer's) where the reciprocal and the division disagree
+    differ = []
+    while len(differ) < 3:
+        r = torch.from_numpy((rng.standard_normal(96) * np.exp2(rng.uniform(-10, 10))).astype(np.float32))
+        r = r.bfloat16().float()
+        sr = _e4m3_scale_lib(r[None])
+        if not torch.equal((r * (1.0 / sr)).to(torch.float8_e4m3fn).view(torch.uint8),
+                           (r / sr).to(torch.float8_e4m3fn).view(torch.uint8)):
+            differ.append(r.numpy())
+    v = np.vstack([v, np.array(differ), tiny[None], tie[None], np.zeros((1, 96), np.float32)])
+    codes, scales = oracle.e4m3_rows(v)
+    t = torch.from_numpy(v)
+    s = _e4m3_scale_lib(t)
+    want = (t * (1.0 / s)).to(torch.float8_e4m3fn).view(torch.uint8).numpy()
+    assert np.array_equal(scales, s.numpy().ravel())
+    assert np.array_equal(codes, want)
+    assert scales[-1] == 1.0 and np.all(codes[-1] == 0)
+    assert scales[-3] == np.float32(2.0 ** -126)
+    # the tie row: every value is an exact midpoint times 2^-5 (but the
+    # maximum), and half of the ties went up, half down (to the even code)
+    q = t[-2] / s[-2]
+    up = (torch.from_numpy(codes[-2]).view(torch.float8_e4m3fn).float().abs() > q.abs())[1:]
+    assert 0 < int(up.sum()) < up.numel()

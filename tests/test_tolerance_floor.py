@@ -145,10 +145,12 @@ def test_hidden_rounding_flips_stay_within_the_reading_slack(hidden, tdt):
 
 def _e4m3_rows_lib(v: torch.Tensor):
     """Per-row E4M3 quantisation with torch's casts (fp64 values out) and
-    the row scales: s = fp32(max|v| / 448), 1 for a zero row."""
-    s = v.float().abs().amax(dim=1, keepdim=True) / 448.0
-    s = torch.where(s == 0, torch.ones_like(s), s)
-    q = (v.float() / s).to(torch.float8_e4m3fn)
+    the row scales: s = fp32(max|v| / 448) (at least 2^-126, 1 for a zero
+    row), codes from fp32(v * fp32(1 / s))."""
+    m = v.float().abs().amax(dim=1, keepdim=True)
+    s = torch.clamp_min(m / 448.0, 2.0 ** -126)
+    s = torch.where(m == 0, torch.ones_like(s), s)
+    q = (v.float() * (1.0 / s)).to(torch.float8_e4m3fn)
     return q.double() * s.double(), s
 
 
