@@ -51,22 +51,32 @@ __global__ void __launch_bounds__(256) gateup_finish_kernel(
 // routed partial of entry t * k + j, then sum over s of the shared partial)
 // -- one rounding, a fixed order.  Partials: routed [splits_r][T * k][d],
 // shared [splits_s][T][d] (fp32, rows un-permuted to entries / tokens).
-// Four outputs per thread; d % 4 == 0.
+// Four outputs per thread; d % 4 == 0.  done (fused launches, else null):
+// the fused GEMM's two tile counters, reset here for the next forward (the
+// GEMM has finished: this kernel's entry waits for it).
 template <typename ET>
 __global__ void __launch_bounds__(256) down_finish_kernel(const float* __restrict__ part_r, long long stride_r,
                                                           int splits_r, const float* __restrict__ part_s,
                                                           long long stride_s, int splits_s, int k, int d,
-                                                          long long n, ET* __restrict__ out) {
+                                                          long long n, ET* __restrict__ out, unsigned* done) {
     pdl_enter();
+    if (done && blockIdx.x == 0 && threadIdx.x < 2) done[threadIdx.x] = 0u;
     const long long n4 = n >> 2;
     const int d4 = d >> 2;
     for (long long i = blockIdx.x * (long long)blockDim.x + threadIdx.x; i < n4;
          i += (long long)gridDim.x * blockDim.x) {
         float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
         if (k == 1) {  // routed row t is entry t: the same index as the output
-            for (int s = 0; s < splits_r; ++s) {
-                const float4 v = reinterpret_cast<const float4*>(part_r + stride_r * s)[i];
-                acc.x += v.x, acc.y += v.y, acc.z += v.z, acc.w += v.w;
+            // the partials of up to 8 splits are loaded before any is added
+            // (a small batch is latency-bound here: one round trip per 8)
+            for (int s0 = 0; s0 < splits_r; s0 += 8) {
+                float4 v[8];
+#pragma unroll
+                for (int j = 0; j < 8; ++j)
+                    v[j] = s0 + j < splits_r ? reinterpret_cast<const float4*>(part_r + stride_r * (s0 + j))[i]
+                                             : make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll
+                for (int j = 0; j < 8; ++j) acc.x += v[j].x, acc.y += v[j].y, acc.z += v[j].z, acc.w += v[j].w;
             }
         } else {
             const long long t = i / d4, c4 = i - t * d4;
@@ -77,9 +87,14 @@ __global__ void __launch_bounds__(256) down_finish_kernel(const float* __restric
                     acc.x += v.x, acc.y += v.y, acc.z += v.z, acc.w += v.w;
                 }
         }
-        for (int s = 0; s < splits_s; ++s) {
-            const float4 v = reinterpret_cast<const float4*>(part_s + stride_s * s)[i];
-            acc.x += v.x, acc.y += v.y, acc.z += v.z, acc.w += v.w;
+        for (int s0 = 0; s0 < splits_s; s0 += 8) {
+            float4 v[8];
+#pragma unroll
+            for (int j = 0; j < 8; ++j)
+                v[j] = s0 + j < splits_s ? reinterpret_cast<const float4*>(part_s + stride_s * (s0 + j))[i]
+                                         : make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll
+            for (int j = 0; j < 8; ++j) acc.x += v[j].x, acc.y += v[j].y, acc.z += v[j].z, acc.w += v[j].w;
         }
         if constexpr (sizeof(ET) == 2) {
             const __nv_bfloat162 lo = __floats2bfloat162_rn(acc.x, acc.y);

@@ -164,7 +164,8 @@ WsLayout ws_layout(const l4moe_params& p, int T, int sms, int k, bool act8 = fal
     };
     const size_t t = (size_t)std::max(T, 1), E = (size_t)p.num_experts, es = act_bytes(p.dtype);
     const size_t tv = t * (size_t)k;
-    L.err = take(256);  // device error word, then the routing kernels' ticket (zeroed once)
+    L.err = take(256);  // device error word, the routing kernels' ticket, the fused GEMM's two
+                        // tile counters (zeroed once; each user leaves them at zero)
     L.idx = take(4 * tv);
     L.gate = take(4 * tv);
     L.lmax = take(4 * tv);
@@ -472,12 +473,29 @@ void launch_router(const void* x, const void* Wr, const float* bias, int T, int 
     else launch_router_t<ET, 256, 8, 8>(x, Wr, bias, T, d, E, idx, gate, lmax, margin, k, st);
 }
 
-template <int MODE, typename ET, int WQ>
-void launch_gemm(int grid, const BMaps& bm, const GemmArgs& a, cudaStream_t st) {
-    using Cfg = GemmCfg<MODE, ET, WQ>;
+// bm / a: the GEMM (a fused launch's gate/up); bm2 / a2: a fused launch's down
+template <int MODE, typename ET, int WQ, bool SMALLN>
+void launch_gemm_cfg(int grid, const BMaps& bm, const GemmArgs& a, const BMaps& bm2, const GemmArgs& a2,
+                     cudaStream_t st) {
+    using Cfg = GemmCfg<MODE, ET, WQ, SMALLN>;
     static std::atomic<uint64_t> attr_done{0};
-    ensure_smem_attr(attr_done, moe_gemm_kernel<MODE, ET, WQ>, Cfg::SMEM_BYTES);
-    launch_k(moe_gemm_kernel<MODE, ET, WQ>, dim3(grid), dim3(Cfg::THREADS), Cfg::SMEM_BYTES, st, bm, a);
+    ensure_smem_attr(attr_done, moe_gemm_kernel<MODE, ET, WQ, SMALLN>, Cfg::SMEM_BYTES);
+    launch_k(moe_gemm_kernel<MODE, ET, WQ, SMALLN>, dim3(grid), dim3(Cfg::THREADS), Cfg::SMEM_BYTES, st, bm, a,
+             bm2, a2);
+}
+
+// small: every group of the launch has at most 64 rows (the small-batch
+// configuration with the deeper weight ring)
+template <int MODE, typename ET, int WQ>
+void launch_gemm_pair(int grid, const BMaps& bm, const GemmArgs& a, const BMaps& bm2, const GemmArgs& a2,
+                      cudaStream_t st, bool small) {
+    if (small) launch_gemm_cfg<MODE, ET, WQ, true>(grid, bm, a, bm2, a2, st);
+    else launch_gemm_cfg<MODE, ET, WQ, false>(grid, bm, a, bm2, a2, st);
+}
+
+template <int MODE, typename ET, int WQ>
+void launch_gemm(int grid, const BMaps& bm, const GemmArgs& a, cudaStream_t st, bool small) {
+    launch_gemm_pair<MODE, ET, WQ>(grid, bm, a, bm, a, st, small);
 }
 
 // The launch sequence of one forward.  w / ws_tokens: the workspace and the
@@ -708,31 +726,16 @@ l4moe_status run_layer(l4moe_handle* h, int T, const void* x, const void* Wr, co
     gu.ld_part_shared = 2LL * Fs;
     gu.part_stride_shared = (long long)T * 2 * Fs;
     gu.err = err;
-    LaunchTimer t_gu(h, 3, st);
-    launch_gemm<MODE_GATEUP, ET, WQ>(
-        grid_for(s_gu * ((long long)fb_gu_s * tb + (long long)fb_gu_r * (tbv + std::min(E, Tv)))),
-        bm_gu, gu, st);
-    if (s_gu > 1) {
-        const long long n = (long long)Tv * F + (long long)T * Fs;
-        launch_k(gateup_finish_kernel<HT>, dim3((int)std::min<long long>((n + 255) / 256, 4LL * h->sms)),
-                 dim3(256), 0, st, (const float*)gu.part_routed, gu.ld_part_routed, gu.part_stride_routed,
-                 (const float*)gu.part_shared, gu.ld_part_shared, gu.part_stride_shared, s_gu, Tv, T, F, Fs,
-                 (const float*)gslot, (const float*)tokscale, hr, hs, err);
-        ++h->launches;
-    }
-    t_gu.stop();
-    L4MOE_CHECK_LAUNCH("gate/up launch");
-    if constexpr (ACT8) {
-        // the hidden rows' E4M3 codes and row scales, one CTA per row at a time
-        const int Tr = E > 0 ? Tv : 0;
-        const int rows = Tr + T;
-        LaunchTimer t_q(h, 5, st);
-        launch_k(quant_hidden_kernel, dim3(std::min(rows, h->sms * 8)), dim3(kQuantThreads), 0, st,
-                 (const __nv_bfloat16*)hr, (const __nv_bfloat16*)hs, Tr, T, F, Fs, hq_r,
-                 hq_r + (size_t)Tv * F, hsc_r, hsc_r + Tv);
-        t_q.stop();
-        L4MOE_CHECK_LAUNCH("hidden quantisation launch");
-    }
+    // after the one-launch routing of a small batch, the shared expert's tiles
+    // (operand x itself, which the routing does not write) go first in the
+    // work list and may run while the routing finishes: the GEMM waits for it
+    // only at its first routed tile (8- and 4-bit weight layers read the f16
+    // copy of x that the routing writes, so they wait at entry)
+    const bool early = E > 0 && T <= kSmallMaxTokens && !FP8W;
+    gu.early_tiles = early ? fb_gu_s * s_gu * tb : 0;
+    gu.early_rows = T;
+    // no group can have more than 64 rows: the small-batch GEMM configuration
+    const bool small_tiles = T <= 2 * GCfg::B_SMALL_ROWS && Tv <= 2 * GCfg::B_SMALL_ROWS;
 
     GemmArgs dn{};
     dn.table = tab_dn;
@@ -761,15 +764,58 @@ l4moe_status run_layer(l4moe_handle* h, int T, const void* x, const void* Wr, co
     dn.ld_part_shared = d;
     dn.part_stride_shared = (long long)T * d;
     dn.err = err;
+    // A small batch whose gate/up starts early and needs no split-K finish
+    // runs both contractions as one launch: its pairs take the gate/up tiles
+    // and then the down tiles, each down tile waiting (on device counters of
+    // finished gate/up tiles) only for the hidden rows of its own class, so
+    // the pairs that finish their gate/up tiles stream down weights while the
+    // others still stream gate/up weights
+    const bool fused = early && s_gu == 1;
+    unsigned* done = fused ? err + 2 : nullptr;  // zero here; the down finish resets them
+    gu.done = done;
+    dn.done = done;
+    const long long gu_units = s_gu * ((long long)fb_gu_s * tb + (long long)fb_gu_r * (tbv + std::min(E, Tv)));
+    const long long dn_units = s_dn * (long long)fb_dn * (tb + tbv + std::min(E, Tv));
+    if (fused) {
+        LaunchTimer t_gu(h, 3, st);
+        launch_gemm_pair<MODE_FUSED, ET, WQ>(grid_for(gu_units + dn_units), bm_gu, gu, bm_dn, dn, st, small_tiles);
+        t_gu.stop();
+        L4MOE_CHECK_LAUNCH("fused gate/up and down launch");
+    } else {
+        LaunchTimer t_gu(h, 3, st);
+        launch_gemm<MODE_GATEUP, ET, WQ>(grid_for(gu_units), bm_gu, gu, st, small_tiles);
+        if (s_gu > 1) {
+            const long long n = (long long)Tv * F + (long long)T * Fs;
+            launch_k(gateup_finish_kernel<HT>, dim3((int)std::min<long long>((n + 255) / 256, 4LL * h->sms)),
+                     dim3(256), 0, st, (const float*)gu.part_routed, gu.ld_part_routed, gu.part_stride_routed,
+                     (const float*)gu.part_shared, gu.ld_part_shared, gu.part_stride_shared, s_gu, Tv, T, F, Fs,
+                     (const float*)gslot, (const float*)tokscale, hr, hs, err);
+            ++h->launches;
+        }
+        t_gu.stop();
+        L4MOE_CHECK_LAUNCH("gate/up launch");
+        if constexpr (ACT8) {
+            // the hidden rows' E4M3 codes and row scales, one CTA per row at a time
+            const int Tr = E > 0 ? Tv : 0;
+            const int rows = Tr + T;
+            LaunchTimer t_q(h, 5, st);
+            launch_k(quant_hidden_kernel, dim3(std::min(rows, h->sms * 8)), dim3(kQuantThreads), 0, st,
+                     (const __nv_bfloat16*)hr, (const __nv_bfloat16*)hs, Tr, T, F, Fs, hq_r,
+                     hq_r + (size_t)Tv * F, hsc_r, hsc_r + Tv);
+            t_q.stop();
+            L4MOE_CHECK_LAUNCH("hidden quantisation launch");
+        }
+    }
+
     LaunchTimer t_dn(h, 4, st);
-    launch_gemm<MODE_DOWN, ET, WQ>(grid_for(s_dn * (long long)fb_dn * (tb + tbv + std::min(E, Tv))),
-                                     bm_dn, dn, st);
+    if (!fused) launch_gemm<MODE_DOWN, ET, WQ>(grid_for(dn_units), bm_dn, dn, st, small_tiles);
     {
         const long long n = (long long)T * d;
         // the routed planes then the shared ones; without experts only the shared
         launch_k(down_finish_kernel<ET>, dim3((int)std::min<long long>((n / 4 + 255) / 256, 4LL * h->sms)),
                  dim3(256), 0, st, (const float*)part, dn.part_stride_routed, E > 0 ? s_dn : 0,
-                 (const float*)dn.part_shared, dn.part_stride_shared, s_dn, k, d, n, static_cast<ET*>(out));
+                 (const float*)dn.part_shared, dn.part_stride_shared, s_dn, k, d, n, static_cast<ET*>(out),
+                 done);
         ++h->launches;
     }
     t_dn.stop();
@@ -918,8 +964,9 @@ l4moe_status l4moe_forward_static(l4moe_handle* h, int T, const void* x, const v
     // the state a forward expects to start at zero
     cudaError_t e = cudaMemcpyAsync(maps, h->h_maps.data(), maps_bytes, cudaMemcpyHostToDevice, st);
     if (e != cudaSuccess) return cuda_fail(h, e, "static descriptor upload");
-    // the error word and the routing kernels' ticket that follows it
-    e = cudaMemsetAsync(base + ws_layout(h->p, T, h->sms, h->top_k, h->act8).err, 0, 2 * sizeof(unsigned), st);
+    // the error word, the routing kernels' ticket and the fused GEMM's two
+    // tile counters that follow it
+    e = cudaMemsetAsync(base + ws_layout(h->p, T, h->sms, h->top_k, h->act8).err, 0, 4 * sizeof(unsigned), st);
     if (e != cudaSuccess) return cuda_fail(h, e, "static error word clear");
     const float* const* scales = nullptr;
     if (fp8) {  // the scale-pointer table of 8-bit weights follows the descriptors

@@ -84,7 +84,9 @@
 
 namespace l4moe {
 
-enum GemmMode : int { MODE_GATEUP = 0, MODE_DOWN = 1 };
+// MODE_FUSED: one launch takes the gate/up tiles and then the down tiles of
+// a small batch (see TileCursor and the down tiles' wait in the producer).
+enum GemmMode : int { MODE_GATEUP = 0, MODE_DOWN = 1, MODE_FUSED = 2 };
 
 // The MMA operand type's tiling: K per stage (one 128-byte token row), K per
 // MMA, the instruction's format code, and the MN-major weight tile's slabs
@@ -153,6 +155,15 @@ struct GemmArgs {
     long long part_stride_routed;  // elements between splits
     long long part_stride_shared;
     unsigned* err;
+    // early start (gate/up after the small-batch routing, shared operand x):
+    // the leading early_tiles positions are the shared expert's tiles over
+    // early_rows tokens, run before the routing has finished; 0 = none
+    int early_tiles;
+    int early_rows;
+    // fused launches: [0] shared, [1] routed gate/up epilogue warps done
+    // (each warp of both CTAs counts once per tile; zero when the launch
+    // starts, reset by the down finish kernel)
+    unsigned* done;
 };
 
 // Output features covered by one pair tile.
@@ -176,7 +187,12 @@ struct OperandOf<ET, kWqAct8> {
     using type = E4M3Op;
 };
 
-template <int MODE, typename ET, int WQ>
+// SMALLN: every tile of the launch has at most 2 * B_SMALL_ROWS token rows
+// (small batches: decode).  The token operand then needs one 32-row box per
+// CTA and stage, so a stage shrinks to the weight tile plus 4 KB and the ring
+// holds more stages: these launches stream weights, and the bytes in flight
+// per SM set how much of the HBM bandwidth they reach.
+template <int MODE, typename ET, int WQ, bool SMALLN = false>
 struct GemmCfg {
     static constexpr bool ACT8 = WQ == kWqAct8;               // E4M3 x E4M3, raw operands
     static constexpr bool FP8W = WQ != kWqNone && !ACT8;      // coded weights, converter warps
@@ -188,13 +204,13 @@ struct GemmCfg {
     static constexpr int A_BOX_BYTES = C::BK * A_ROW_BYTES;  // BK rows of a slab
     static constexpr int B_BOX_ROWS = 128;                   // token rows per full-tile box
     static constexpr int B_SMALL_ROWS = 32;                  // token rows per small-tile box
-    static constexpr int B_BYTES = (kTokTile / 2) * 128;     // this CTA's half of the tokens
+    static constexpr int B_BYTES = (SMALLN ? B_SMALL_ROWS : kTokTile / 2) * 128;  // this CTA's token rows
     // raw coded weights: 2 slabs x 64 K rows x 64 features, one byte per code
     // (half a byte for int4: two codes per byte along the features)
     static constexpr int RAW_SLAB_BYTES = WQ == kWqInt4 ? 64 * 32 : 64 * 64;
     static constexpr int RAW_BYTES = FP8W ? 2 * RAW_SLAB_BYTES : 0;
     static constexpr int STAGE_BYTES = A_BYTES + B_BYTES + RAW_BYTES;
-    static constexpr int STAGES = FP8W ? 5 : 6;
+    static constexpr int STAGES = SMALLN ? (FP8W ? 7 : 10) : (FP8W ? 5 : 6);
     static constexpr int ACC_BUFS = 2;
     static constexpr int TMEM_COLS = 512;
     // epilogue warps: one per TMEM lane quarter, or two (each taking every
@@ -208,13 +224,15 @@ struct GemmCfg {
     static constexpr int THREADS = 64 + 32 * EPI_WARPS + 32 * CONV_WARPS;
     static constexpr int XLD = 17;                           // exchange row stride (floats)
     static constexpr int XCH_FLOATS = 2 * 2 * 32 * XLD;      // one half's exchange buffers
-    static constexpr int XCH_BYTES = (MODE == MODE_GATEUP) ? EPI_HALVES * XCH_FLOATS * 4 : 0;
+    static constexpr int XCH_BYTES = (MODE != MODE_DOWN) ? EPI_HALVES * XCH_FLOATS * 4 : 0;
     static constexpr int NUM_BARS = 2 * STAGES + 2 * ACC_BUFS + 1 + (FP8W ? 2 * STAGES : 0);
     static constexpr size_t SMEM_BYTES = 1024 /*alignment slack*/ + (size_t)STAGES * STAGE_BYTES +
                                          XCH_BYTES + NUM_BARS * 8 + 16 + sizeof(GroupTable);
+    static_assert(SMEM_BYTES <= 227 * 1024, "shared memory of one CTA");
 };
 
 struct TileInfo {
+    int mode;  // 0: a gate/up tile, 1: a down tile
     int expert, row0, n_valid, n_mma, f0, K, M, up_off;
     int split, kb0, kb1;  // k-block range [kb0, kb1) of this tile's split
     bool shared;
@@ -224,20 +242,15 @@ struct TileInfo {
 // dies caches what its SMs read, so this stays well under half of L2).
 constexpr long long kBandBytes = 24ll << 20;
 
+// Tile `local` of a group: `rows` activation rows from `row0`, weights of
+// `expert`, `group_tiles` tiles in all.
 template <int MODE, int ElemCfgBK, int ElemBytes>
-__host__ __device__ __forceinline__ TileInfo decode_tile(const GroupTable& tab, const GemmArgs& a, int pos) {
-    const int L = tile_at(pos, tab.heavy_tiles, tab.total_tiles);
-    int lo = 0, hi = tab.num_groups - 1;
-    while (lo < hi) {
-        const int mid = (lo + hi + 1) >> 1;
-        if (tab.tile_start[mid] <= L) lo = mid; else hi = mid - 1;
-    }
-    const int g = lo;
-    const int local = L - tab.tile_start[g];
-    const int rows = tab.rows[g];
+__host__ __device__ __forceinline__ TileInfo decode_in_group(const GemmArgs& a, int rows, int row0, int expert,
+                                                             int group_tiles, int local) {
     const int ntb = (rows + kTokTile - 1) / kTokTile;
     TileInfo ti;
-    ti.expert = tab.expert[g];
+    ti.mode = MODE == MODE_DOWN ? 1 : 0;
+    ti.expert = expert;
     ti.shared = (ti.expert == a.num_experts);
     ti.K = ti.shared ? a.k_shared : a.k_routed;
     // Token tiles go in bands of `band` tiles whose activation rows (the B
@@ -245,7 +258,7 @@ __host__ __device__ __forceinline__ TileInfo decode_tile(const GroupTable& tab, 
     // feature block; inside a band the token tile varies fastest, so the
     // tiles that share a weight tile run side by side.
     const int band = max(1, (int)(kBandBytes / ((long long)kTokTile * ti.K * ElemBytes)));
-    const int fbk = (tab.tile_start[g + 1] - tab.tile_start[g]) / ntb;  // feature blocks x splits
+    const int fbk = group_tiles / ntb;  // feature blocks x splits
     const int b = local / (band * fbk);
     const int nb = min(band, ntb - b * band);  // token tiles in this band (the last may be short)
     const int rem = local - b * band * fbk;
@@ -259,7 +272,7 @@ __host__ __device__ __forceinline__ TileInfo decode_tile(const GroupTable& tab, 
     const int fb = rest % nfb;
     const int split = rest / nfb;
     ti.split = split;
-    ti.row0 = tab.row0[g] + tb * kTokTile;
+    ti.row0 = row0 + tb * kTokTile;
     ti.n_valid = min(kTokTile, rows - tb * kTokTile);
     ti.n_mma = (ti.n_valid + 15) & ~15;
     ti.f0 = fb * pair_features<MODE>();
@@ -269,6 +282,94 @@ __host__ __device__ __forceinline__ TileInfo decode_tile(const GroupTable& tab, 
     ti.kb0 = (int)(((long long)nkb * split) / a.ksplit);
     ti.kb1 = (int)(((long long)nkb * (split + 1)) / a.ksplit);
     return ti;
+}
+
+// Launch position `pos` -> its tile, through the work list.
+template <int MODE, int ElemCfgBK, int ElemBytes>
+__host__ __device__ __forceinline__ TileInfo decode_tile(const GroupTable& tab, const GemmArgs& a, int pos) {
+    const int L = tile_at(pos, tab.heavy_tiles, tab.total_tiles);
+    int lo = 0, hi = tab.num_groups - 1;
+    while (lo < hi) {
+        const int mid = (lo + hi + 1) >> 1;
+        if (tab.tile_start[mid] <= L) lo = mid; else hi = mid - 1;
+    }
+    const int g = lo;
+    return decode_in_group<MODE, ElemCfgBK, ElemBytes>(a, tab.rows[g], tab.row0[g], tab.expert[g],
+                                                       tab.tile_start[g + 1] - tab.tile_start[g],
+                                                       L - tab.tile_start[g]);
+}
+
+// The tiles of one launch as a role walks them.  Normally every tile comes
+// from the work list, copied to shared memory once the kernel that writes it
+// has finished (the wait at kernel entry).  With early_tiles > 0 the launch
+// starts before that kernel has finished: its first early_tiles positions
+// are the shared expert's tiles (rows 0 .. early_rows of the shared operand,
+// which that kernel does not write), decoded without the work list; the
+// first position past them waits for the preceding kernel (griddepcontrol)
+// and from there on decodes through the work list in global memory.  A
+// fused launch (always early) continues past the gate/up work list's tiles
+// with the down work list's.
+template <int MODE, int ElemCfgBK, int ElemBytes>
+struct TileCursor {
+    static constexpr int GU = MODE == MODE_FUSED ? MODE_GATEUP : MODE;  // mode of the first work list
+    const GroupTable* tab;  // shared-memory copy (not early)
+    int total;              // tiles of the launch
+    int n_first;            // tiles of the first (gate/up, or the only) work list
+    bool waited;
+
+    __device__ __forceinline__ TileCursor(const GroupTable* smem_tab, const GemmArgs& a)
+        : tab(smem_tab),
+          total(a.early_tiles > 0 ? 0x7FFFFFFF : smem_tab->total_tiles),
+          n_first(a.early_tiles > 0 ? 0x7FFFFFFF : smem_tab->total_tiles),
+          waited(a.early_tiles == 0) {}
+
+    __device__ __forceinline__ TileInfo tile(const GemmArgs& a, const GemmArgs& dn, int L) const {
+        if (L < a.early_tiles)
+            return decode_in_group<GU, ElemCfgBK, ElemBytes>(a, a.early_rows, 0, a.num_experts, a.early_tiles, L);
+        if (L < n_first) return decode_tile<GU, ElemCfgBK, ElemBytes>(a.early_tiles > 0 ? *a.table : *tab, a, L);
+        return decode_tile<MODE_DOWN, ElemCfgBK, ElemBytes>(*dn.table, dn, L - n_first);
+    }
+
+    // Tile at position L, or false past the last one.
+    __device__ __forceinline__ bool at(const GemmArgs& a, const GemmArgs& dn, int L, TileInfo& ti) {
+        if (!waited && L >= a.early_tiles) {
+            asm volatile("griddepcontrol.wait;" ::: "memory");
+            waited = true;
+            n_first = a.table->total_tiles;
+            total = n_first + (MODE == MODE_FUSED ? dn.table->total_tiles : 0);
+        }
+        if (L >= total) return false;
+        ti = tile(a, dn, L);
+        return true;
+    }
+    // The weight descriptor of the tile at L when it can be known now (else null).
+    __device__ __forceinline__ const CUtensorMap* map_if_known(const GemmArgs& a, const GemmArgs& dn, int L) const {
+        if (L < a.early_tiles) return a.a_maps + a.num_experts;
+        if (!waited || L >= total) return nullptr;
+        const TileInfo t = tile(a, dn, L);
+        return (t.mode ? dn.a_maps : a.a_maps) + t.expert;
+    }
+};
+
+// Bounded wait until *count >= target (acquire), for a fused launch's down
+// tiles; on a timeout the producer's bit is set in the error word.
+__device__ __forceinline__ uint32_t ld_acquire_gpu(const unsigned* p) {
+    uint32_t v;
+    asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
+    return v;
+}
+
+__device__ __forceinline__ bool wait_count(const unsigned* count, unsigned target, unsigned* err) {
+    if (ld_acquire_gpu(count) >= target) return true;
+    const uint64_t t0 = global_timer_ns();
+    while (ld_acquire_gpu(count) < target) {
+        if (global_timer_ns() - t0 > kWaitLimitNs) {
+            atomicOr(err, DEV_ERR_TIMEOUT_PRODUCER);
+            return false;
+        }
+        __nanosleep(64);
+    }
+    return true;
 }
 
 __device__ __forceinline__ float silu_f(float z) { return __fdividef(z, 1.0f + __expf(-z)); }
@@ -361,11 +462,16 @@ struct BMaps {
     CUtensorMap routed, shared, routed_small, shared_small;
 };
 
-template <int MODE, typename ET, int WQ>
-__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(GemmCfg<MODE, ET, WQ>::THREADS, 1)
-    moe_gemm_kernel(const __grid_constant__ BMaps bm, const GemmArgs args) {
-    pdl_enter();
-    using Cfg = GemmCfg<MODE, ET, WQ>;
+template <int MODE, typename ET, int WQ, bool SMALLN>
+__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(GemmCfg<MODE, ET, WQ, SMALLN>::THREADS, 1)
+    moe_gemm_kernel(const __grid_constant__ BMaps bm, const __grid_constant__ GemmArgs args,
+                    const __grid_constant__ BMaps bm_dn, const __grid_constant__ GemmArgs args_dn) {
+    // bm / args: the launch's GEMM, or a fused launch's gate/up; bm_dn /
+    // args_dn: a fused launch's down (unused otherwise)
+    // early start: the work list is read after the first wait (TileCursor)
+    if (args.early_tiles > 0) asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+    else pdl_enter();
+    using Cfg = GemmCfg<MODE, ET, WQ, SMALLN>;
     constexpr bool FP8W = Cfg::FP8W;      // coded (8- or 4-bit) weights with converter warps
     constexpr bool ACT8 = Cfg::ACT8;      // E4M3 weights and token rows, read raw
     constexpr bool WSC = WQ != kWqNone;   // per-column weight scales in the epilogue
@@ -396,7 +502,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(GemmCfg<MODE, ET, WQ
         return bar0 + 8u * (3 * Cfg::STAGES + 2 * Cfg::ACC_BUFS + 1 + s);
     };
 
-    {   // work list -> shared memory
+    if (args.early_tiles == 0) {  // work list -> shared memory
         const int* src = reinterpret_cast<const int*>(args.table);
         int* dst = reinterpret_cast<int*>(tab);
         for (int i = threadIdx.x; i < (int)(sizeof(GroupTable) / 4); i += blockDim.x) dst[i] = src[i];
@@ -425,6 +531,12 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(GemmCfg<MODE, ET, WQ
         tma_prefetch_desc(&bm.shared);
         tma_prefetch_desc(&bm.routed_small);
         tma_prefetch_desc(&bm.shared_small);
+        if constexpr (MODE == MODE_FUSED) {
+            tma_prefetch_desc(&bm_dn.routed);
+            tma_prefetch_desc(&bm_dn.shared);
+            tma_prefetch_desc(&bm_dn.routed_small);
+            tma_prefetch_desc(&bm_dn.shared_small);
+        }
     }
     cluster_sync();  // barriers of both CTAs initialised before any remote use
     if (warp == 1) {
@@ -435,7 +547,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(GemmCfg<MODE, ET, WQ
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem_base = misc[0];
-    const int total = tab->total_tiles;
+    using Cursor = TileCursor<MODE, C::BK, C::BYTES>;
     const int pair = blockIdx.x >> 1;
     const int npairs = gridDim.x >> 1;
 
@@ -446,26 +558,58 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(GemmCfg<MODE, ET, WQ
             uint32_t phase = 0;
             uint32_t used = 0, last_par = 0;  // per stage: issued at least once / its parity
             bool aborted = false;
-            for (int L = pair; L < total && !aborted; L += npairs) {
-                const TileInfo ti = decode_tile<MODE, C::BK, C::BYTES>(*tab, args, L);
-                const CUtensorMap* amap = args.a_maps + ti.expert;
+            uint32_t dep_ready = 0;  // fused: bit c set once class c's hidden rows are complete
+            Cursor cur(tab, args);
+            TileInfo ti;
+            for (int L = pair; !aborted && cur.at(args, args_dn, L, ti); L += npairs) {
+                const bool dn_tile = MODE == MODE_FUSED && ti.mode == 1;
+                const GemmArgs& A = dn_tile ? args_dn : args;
+                const BMaps& BM = dn_tile ? bm_dn : bm;
+                const bool gu = MODE == MODE_GATEUP || (MODE == MODE_FUSED && ti.mode == 0);
+                const CUtensorMap* amap = A.a_maps + ti.expert;
                 // the next tile's weight descriptor, fetched while this tile streams
                 // (split-K units and small groups change expert every few k-blocks)
-                if (L + npairs < total)
-                    tma_prefetch_desc(args.a_maps + decode_tile<MODE, C::BK, C::BYTES>(*tab, args, L + npairs).expert);
+                const CUtensorMap* next_map = cur.map_if_known(args, args_dn, L + npairs);
+                if (next_map) tma_prefetch_desc(next_map);
+                if constexpr (MODE == MODE_FUSED) {
+                    // a down tile reads hidden rows the gate/up tiles of its class
+                    // (shared or routed) write, on any CTA: wait until all of them
+                    // are counted, then order this CTA's tensor-copy reads after
+                    if (dn_tile) {
+                        const int cls = ti.shared ? 0 : 1;
+                        if (!(dep_ready >> cls & 1u)) {
+                            const int tiles = cls == 0 ? args.early_tiles : cur.n_first - args.early_tiles;
+                            if (!wait_count(args.done + cls, (unsigned)tiles * 2u * Cfg::EPI_WARPS, args.err)) {
+                                aborted = true;
+                                break;
+                            }
+                            asm volatile("fence.proxy.async.global;" ::: "memory");
+                            dep_ready |= 1u << cls;
+                        }
+                    }
+                }
                 const int half = ti.n_mma >> 1;  // tokens per CTA
                 const bool big = half > 2 * Cfg::B_SMALL_ROWS;
-                const void* bmap = ti.shared ? (big ? (const void*)&bm.shared : (const void*)&bm.shared_small)
-                                             : (big ? (const void*)&bm.routed : (const void*)&bm.routed_small);
+                const void* bmap = ti.shared ? (big ? (const void*)&BM.shared : (const void*)&BM.shared_small)
+                                             : (big ? (const void*)&BM.routed : (const void*)&BM.routed_small);
                 const int brows = big ? Cfg::B_BOX_ROWS : Cfg::B_SMALL_ROWS;
                 const int nbb = (half + brows - 1) / brows;
+                if constexpr (SMALLN) {
+                    // the host launches this configuration only for tiles of at
+                    // most 2 * B_SMALL_ROWS rows; anything larger would overrun the
+                    // stage: report it (bad argument) and stop issuing
+                    if (nbb * brows > Cfg::B_SMALL_ROWS) {
+                        atomicOr(args.err, DEV_ERR_BAD_INDEX);
+                        aborted = true;
+                        break;
+                    }
+                }
                 const uint32_t tx_cta =
                     (FP8W ? 0u : (uint32_t)Cfg::A_BYTES) + (uint32_t)(nbb * brows * 128);
                 const int brow = ti.row0 + (int)rank * half;
                 // this CTA's A columns: gate/up -> [gate 64 | up 64] of features
                 // f0 + 64*rank; down -> 128 features f0 + 128*rank
-                const int acol0 =
-                    (MODE == MODE_GATEUP) ? ti.f0 + 64 * (int)rank : ti.f0 + 128 * (int)rank;
+                const int acol0 = gu ? ti.f0 + 64 * (int)rank : ti.f0 + 128 * (int)rank;
                 for (int kb = ti.kb0; kb < ti.kb1; ++kb) {
                     if (!mbar_wait(empty_bar(stage), phase ^ 1u, args.err, DEV_ERR_TIMEOUT_PRODUCER)) {
                         aborted = true;
@@ -483,9 +627,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(GemmCfg<MODE, ET, WQ
                         mbar_arrive_expect_tx(rawfull_bar(stage), Cfg::RAW_BYTES);
 #pragma unroll
                         for (int j = 0; j < 2; ++j) {
-                            const int col = (MODE == MODE_GATEUP)
-                                                ? (j == 0 ? acol0 : ti.up_off + acol0)
-                                                : acol0 + 64 * j;
+                            const int col = gu ? (j == 0 ? acol0 : ti.up_off + acol0) : acol0 + 64 * j;
                             tma_load_2d(rb + j * Cfg::RAW_SLAB_BYTES, amap, rawfull_bar(stage),
                                         WQ == kWqInt4 ? col / 2 : col, k);
                         }
@@ -493,7 +635,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(GemmCfg<MODE, ET, WQ
 #pragma unroll
                         for (int bx = 0; bx < Cfg::A_BOXES; ++bx) {
                             int col;
-                            if constexpr (MODE == MODE_GATEUP) {
+                            if (gu) {
                                 const int j = bx * Cfg::A_BOX_FEATS;  // 0..127 within [gate 64 | up 64]
                                 col = (j < 64 ? 0 : ti.up_off - 64) + acol0 + j;
                             } else {
@@ -536,8 +678,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(GemmCfg<MODE, ET, WQ
             uint32_t phase = 0;
             int acc = 0;
             uint32_t acc_phase = 0;
-            for (int L = pair; L < total; L += npairs) {
-                const TileInfo ti = decode_tile<MODE, C::BK, C::BYTES>(*tab, args, L);
+            Cursor cur(tab, args);
+            TileInfo ti;
+            for (int L = pair; cur.at(args, args_dn, L, ti); L += npairs) {
                 if (!mbar_wait_cluster(tempty_bar(acc), acc_phase ^ 1u, args.err, DEV_ERR_TIMEOUT_MMA))
                     break;
                 tc_fence_after();
@@ -598,8 +741,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(GemmCfg<MODE, ET, WQ
         int stage = 0;
         uint32_t phase = 0;
         bool ok = true;
-        for (int L = pair; L < total && ok; L += npairs) {
-            const TileInfo ti = decode_tile<MODE, C::BK, C::BYTES>(*tab, args, L);
+        Cursor cur(tab, args);
+        TileInfo ti;
+        for (int L = pair; ok && cur.at(args, args_dn, L, ti); L += npairs) {
             for (int kb = ti.kb0; kb < ti.kb1; ++kb) {
                 const bool got = mbar_wait(rawfull_bar(stage), phase, args.err, DEV_ERR_TIMEOUT_PRODUCER);
                 if (!__all_sync(0xffffffffu, got)) {
@@ -645,10 +789,13 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(GemmCfg<MODE, ET, WQ
         int acc = 0;
         uint32_t acc_phase = 0;
         volatile uint32_t* abort_flag = misc + 1;
-        for (int L = pair; L < total; L += npairs) {
-            const TileInfo ti = decode_tile<MODE, C::BK, C::BYTES>(*tab, args, L);
+        Cursor cur(tab, args);
+        TileInfo ti;
+        for (int L = pair; cur.at(args, args_dn, L, ti); L += npairs) {
+            const bool gu = MODE == MODE_GATEUP || (MODE == MODE_FUSED && ti.mode == 0);
+            const GemmArgs& A = (MODE == MODE_FUSED && ti.mode == 1) ? args_dn : args;
             const bool ok = mbar_wait(tfull_bar(acc), acc_phase, args.err, DEV_ERR_TIMEOUT_EPILOGUE);
-            if constexpr (MODE == MODE_GATEUP) {
+            if (gu) {
                 // the 4 warps of a half meet at named barriers below: leave together or not at all
                 if (!__all_sync(0xffffffffu, ok) && lane == 0) *abort_flag = 1u;
                 named_bar_sync(bar_id, 128);
@@ -659,29 +806,28 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(GemmCfg<MODE, ET, WQ
             tc_fence_after();
             const uint32_t tb = tmem_base + ((uint32_t)(q * 32) << 16) + (uint32_t)acc * 256u;
             using OT = typename GemmAct<ET, FP8W>::type;  // hidden rows (gate/up's output)
-            OT* outp = reinterpret_cast<OT*>(ti.shared ? args.out_shared : args.out_routed);
-            const long long ld = ti.shared ? args.ld_shared : args.ld_routed;
-            const int32_t* rowmap = ti.shared ? args.rowmap_shared : args.rowmap_routed;
-            const float* colscale = ti.shared ? args.colscale_shared : args.colscale_routed;
+            OT* outp = reinterpret_cast<OT*>(ti.shared ? A.out_shared : A.out_routed);
+            const long long ld = ti.shared ? A.ld_shared : A.ld_routed;
+            const int32_t* rowmap = ti.shared ? A.rowmap_shared : A.rowmap_routed;
+            const float* colscale = ti.shared ? A.colscale_shared : A.colscale_routed;
             // coded weights: the scale of this TMEM lane's weight column (lane =
             // row of the A tile: gate/up [gate 64 | up 64] features, down 128)
             float wsc = 1.0f;
             if constexpr (WSC) {
                 const int r = q * 32 + lane;
-                const int f = (MODE == MODE_GATEUP) ? ti.f0 + 64 * (int)rank + (r & 63)
-                                                    : ti.f0 + 128 * (int)rank + r;
-                const int wcol = (MODE == MODE_GATEUP && r >= 64) ? ti.up_off + f : f;
-                wsc = f < ti.M ? args.wscale[ti.expert][wcol] : 0.0f;
+                const int f = gu ? ti.f0 + 64 * (int)rank + (r & 63) : ti.f0 + 128 * (int)rank + r;
+                const int wcol = (gu && r >= 64) ? ti.up_off + f : f;
+                wsc = f < ti.M ? A.wscale[ti.expert][wcol] : 0.0f;
             }
-            if (args.partial_out) {
+            if (A.partial_out) {
                 // split-K: store this split's fp32 partial; row = slot (gate/up) or
                 // token (down), column = the weight column of this TMEM lane
-                float* pbase = ti.shared ? args.part_shared : args.part_routed;
-                const long long pld = ti.shared ? args.ld_part_shared : args.ld_part_routed;
-                const long long pst = ti.shared ? args.part_stride_shared : args.part_stride_routed;
+                float* pbase = ti.shared ? A.part_shared : A.part_routed;
+                const long long pld = ti.shared ? A.ld_part_shared : A.ld_part_routed;
+                const long long pst = ti.shared ? A.part_stride_shared : A.part_stride_routed;
                 float* pp = pbase + pst * ti.split;
                 int col, fcheck;
-                if constexpr (MODE == MODE_GATEUP) {
+                if (gu) {
                     const int r = q * 32 + lane;                      // 0..127: [gate 64 | up 64]
                     fcheck = ti.f0 + 64 * (int)rank + (r & 63);       // feature
                     col = (r < 64 ? 0 : ti.up_off) + fcheck;
@@ -692,7 +838,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(GemmCfg<MODE, ET, WQ
                 const bool fvalid = fcheck < ti.M;
                 // down: a token row's scale (the FP8 activation mode's hidden
                 // row scale) applies here; gate/up partials take theirs in the finish
-                const float* tscale = MODE == MODE_DOWN ? (ti.shared ? args.colscale_shared : args.colscale_routed)
+                const float* tscale = !gu ? (ti.shared ? A.colscale_shared : A.colscale_routed)
                                                         : nullptr;
                 for (int c = 32 * half; c < ti.n_valid; c += CSTEP) {
                     const bool cval = c + lane < ti.n_valid;
@@ -738,7 +884,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(GemmCfg<MODE, ET, WQ
 #pragma unroll
                     for (int i = 0; i < 32; ++i) v[i] *= wsc;
                 }
-                if constexpr (MODE == MODE_GATEUP) {
+                if (gu) {
                     // lanes 0-63: gate rows, 64-127: up rows of the same 64 features.
                     // Gate warps (q 0,1) finish columns c..c+15, up warps (q 2,3)
                     // columns c+16..c+31; each hands the other half over.
@@ -765,7 +911,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(GemmCfg<MODE, ET, WQ
                         const float hv = silu_f(g * gv) * (g * uv);
                         if constexpr (FP8W) {  // hidden rows held in f16: report values beyond its range
                             if (fvalid && c + col < ti.n_valid && !(fabsf(hv) < 65520.0f))  // rounds to inf
-                                atomicOr(args.err, DEV_ERR_F16_RANGE);
+                                atomicOr(A.err, DEV_ERR_F16_RANGE);
                         }
                         if (fvalid && c + col < ti.n_valid)
                             store_elem(outp + (size_t)orow * ld + f, hv);
@@ -780,6 +926,13 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(GemmCfg<MODE, ET, WQ
                         if (fvalid && c + i < ti.n_valid)
                             store_elem(outp + (size_t)orow * ld + f, v[i]);
                     }
+                }
+            }
+            if constexpr (MODE == MODE_FUSED) {
+                if (gu) {  // this warp's hidden values of the tile are stored: count them
+                    __threadfence();
+                    __syncwarp();
+                    if (lane == 0) atomicAdd(args.done + (ti.shared ? 0 : 1), 1u);
                 }
             }
             tc_fence_before();

@@ -4,7 +4,11 @@
 // several widths) every launch position decodes to a distinct
 // (group, token tile, feature block, k range), together they cover every
 // tile exactly once, and each tile's rows, features and k-blocks stay inside
-// its group.  Prints "OK <cases>" or the first violation.
+// its group.  For the work lists of small batches (the shared expert listed
+// first, every group light), the leading tiles a launch decodes without the
+// work list (decode_in_group over the shared rows: the early start of the
+// gate/up launch) equal the work list's own.  Prints "OK <cases>" or the
+// first violation.
 #include <cstdio>
 #include <random>
 #include <set>
@@ -108,9 +112,55 @@ static bool run_case(std::mt19937& rng, int c) {
     return true;
 }
 
+// A small batch's table (shared expert first, then the routed experts in
+// index order, every group light): the shared expert's tiles decoded without
+// the table equal the table's first tiles.
+template <int MODE>
+static bool early_case(std::mt19937& rng, int c) {
+    const int E = 1 + (int)(rng() % 256);
+    const int T = 1 + (int)(rng() % 16), k = 1 + (int)(rng() % 4);
+    const int ksplit = 1 + (int)(rng() % 16);
+    const int K_r = 64 * (1 + (int)(rng() % 130)), K_s = 64 * (1 + (int)(rng() % 130));
+    const int M_r = 64 * (1 + (int)(rng() % 160)), M_s = 64 * (1 + (int)(rng() % 160));
+    std::vector<Group> cand;
+    cand.push_back({T, E});
+    for (int e = 0; e < E; ++e) cand.push_back({(rng() % 8 == 0) ? (int)(rng() % (T * k + 1)) : 0, e});
+    const int fb_r = (M_r + pair_features<MODE>() - 1) / pair_features<MODE>();
+    const int fb_s = (M_s + pair_features<MODE>() - 1) / pair_features<MODE>();
+    GroupTable tab{};
+    make_table(tab, cand, fb_r, fb_s, ksplit, E);
+    GemmArgs a{};
+    a.num_experts = E;
+    a.k_routed = K_r;
+    a.k_shared = K_s;
+    a.m_routed = M_r;
+    a.m_shared = M_s;
+    a.ksplit = ksplit;
+    const int early = ((T + kTokTile - 1) / kTokTile) * fb_s * ksplit;
+    if (tab.heavy_tiles != 0 || tab.expert[0] != E || tab.tile_start[1] != early) {
+        printf("BAD early case %d: table does not lead with the shared expert\n", c);
+        return false;
+    }
+    for (int L = 0; L < early; ++L) {
+        const TileInfo x = decode_in_group<MODE, 64, 2>(a, T, 0, E, early, L);
+        const TileInfo y = decode_tile<MODE, 64, 2>(tab, a, L);
+        if (x.expert != y.expert || x.row0 != y.row0 || x.n_valid != y.n_valid || x.n_mma != y.n_mma ||
+            x.f0 != y.f0 || x.K != y.K || x.M != y.M || x.up_off != y.up_off || x.split != y.split ||
+            x.kb0 != y.kb0 || x.kb1 != y.kb1 || x.shared != y.shared) {
+            printf("BAD early case %d L %d\n", c, L);
+            return false;
+        }
+    }
+    return true;
+}
+
 int main() {
     std::mt19937 rng(2024);
     int cases = 0;
+    for (int c = 0; c < 2000; ++c) {
+        if (!early_case<MODE_GATEUP>(rng, c) || !early_case<MODE_DOWN>(rng, c)) return 1;
+        cases += 2;
+    }
     // tile_at alone: a permutation of [0, total) that keeps each run's order
     for (int total = 1; total <= 300; ++total)
         for (int heavy = 0; heavy <= total; ++heavy) {

@@ -319,7 +319,7 @@ def test_repeatable_and_host_path_identical():
 
 
 def test_kernel_timing_records_only_the_selected_kernels():
-    from sparse_moe_transformer_router_b200.binding import ERR_ARG, L4MoEError
+    from sparse_moe_transformer_router_b200.binding import ERR_ARG, NUM_KERNELS, L4MoEError
     cfg = SMALL["bf16_ragged"]
     inp = generate(cfg, seed=3, device="cuda")
     layer = make_layer(inp)
@@ -332,7 +332,7 @@ def test_kernel_timing_records_only_the_selected_kernels():
     assert t["gemm_gate_up"][1] == 1 and t["gemm_gate_up"][0] > 0
     assert all(n == 0 for k, (ms, n) in t.items() if k != "gemm_gate_up")
     with pytest.raises(L4MoEError) as ei:
-        layer._check(layer._lib.l4moe_set_timing(layer._h, 1 << 5))  # no such kernel slot
+        layer._check(layer._lib.l4moe_set_timing(layer._h, 1 << NUM_KERNELS))  # no such kernel slot
     assert ei.value.status == ERR_ARG
 
 
