@@ -109,16 +109,19 @@ class ClockSampler:
                 "sm_max_mhz": max(mx) if mx else None, "reasons": reasons, "samples": len(rows)}
 
 
-def kernel_flops_bytes(cfg, counts, act8: bool = False):
+def kernel_flops_bytes(cfg, counts, act8: bool = False, plan: dict | None = None):
     """Algorithmic FLOPs / bytes per launch of each kernel.  act8: the FP8
     activation mode (the contractions read 1-byte token and hidden rows; the
-    hidden rows are written in bf16 and quantised by their own kernel)."""
+    hidden rows are written in bf16 and quantised by their own kernel).
+    plan (the layer's launch plan): with a fused launch the gate/up timing
+    slot covers both contractions and the down slot only the finish kernel
+    (which reads the down's fp32 partials and writes the output)."""
     T, d, E, F, Fs = cfg.T, cfg.d_model, cfg.num_experts, cfg.expert_ffn, cfg.shared_ffn
     a = accounting.ACT_BYTES[cfg.dtype]
     w = accounting.W_BYTES[cfg.dtype]
     q = 1 if act8 else a  # bytes of a contraction's token-row element
     touched = int(np.count_nonzero(counts))
-    return {
+    out = {
         "router": {"flops": 2 * T * d * E, "bytes": T * d * a + d * E * a + T * 16},
         "permute": {"flops": 0, "bytes": T * 4 * 4},
         "row_copy": {"flops": 0, "bytes": T * d * a + 2 * T * d * q + T * 12},
@@ -128,6 +131,11 @@ def kernel_flops_bytes(cfg, counts, act8: bool = False):
                       "bytes": (touched * F * d + Fs * d) * w + T * (F + Fs) * q + T * d * a},
         "quant_hidden": {"flops": 0, "bytes": T * (F + Fs) * (a + 1) + 2 * T * 4},
     }
+    if plan and plan.get("fused"):
+        gu, dn = out["gemm_gate_up"], out["gemm_down"]
+        out["gemm_gate_up"] = {"flops": gu["flops"] + dn["flops"], "bytes": gu["bytes"] + dn["bytes"]}
+        out["gemm_down"] = {"flops": 0, "bytes": plan["split_down"] * 2 * T * d * 4 + T * d * a}
+    return out
 
 
 def profile_traffic(kernel: str, workload: str):
@@ -488,7 +496,8 @@ def measure(cfg, inp, layer, steps: int, warmup: int, world: int, local: int, ac
         tensor_peak *= FP8_OVER_BF16
         tensor_sheet *= FP8_OVER_BF16
     hbm = peaks["hbm_gbs"]
-    kfb = kernel_flops_bytes(cfg, counts, act8)
+    plan = layer.plan()
+    kfb = kernel_flops_bytes(cfg, counts, act8, plan)
     per_kernel = {}
     for name, (ms, n) in breakdown.items():
         if n:
@@ -521,7 +530,7 @@ def measure(cfg, inp, layer, steps: int, warmup: int, world: int, local: int, ac
                   "tflops_active": flops / (ms_step / 1e3) / 1e12,
                   "gbs_algorithmic": lbytes / (ms_step / 1e3) / 1e9,
                   "flops_per_step": flops, "bytes_per_step": lbytes}
-    return {"ms_per_step": ms_step, "t_ms": t_ms, "steps": steps, "roofline": roof,
+    return {"ms_per_step": ms_step, "t_ms": t_ms, "steps": steps, "roofline": roof, "plan": plan,
             "layer_roofline": layer_roof, "kernels": per_kernel, "n_break": n_break, "dom": dom,
             "gpu_launches": launches, "clocks": clocks, "experts_touched": touched}
 
@@ -549,7 +558,7 @@ def run_extra_workloads(args, rank, world, local) -> dict:
                      "experts": cfg.num_experts, "dtype": cfg.dtype, "router": cfg.router,
                      "layer_roofline": m["layer_roofline"], "roofline": m["roofline"],
                      "kernels": {k: round(v["avg_us"], 2) for k, v in m["kernels"].items()},
-                     "gpu_launches": m["gpu_launches"], "clocks": m["clocks"],
+                     "gpu_launches": m["gpu_launches"], "clocks": m["clocks"], "plan": m["plan"],
                      "experts_touched": m["experts_touched"]}
         layer.close()
         del inp, layer, out
@@ -620,7 +629,7 @@ def run_b200(args, rank, world, local):
             "kernels_note": f"every kernel event-timed over {m['n_break']} steps after the warm-up; the "
                             f"dominant kernel ({m['dom']}) again over a region of the timed steps; the "
                             f"step time itself is taken without per-kernel events",
-            "e2e": e2e, "gpu_launches": m["gpu_launches"], "clocks": m["clocks"],
+            "e2e": e2e, "gpu_launches": m["gpu_launches"], "clocks": m["clocks"], "plan": m["plan"],
             "experts_touched": m["experts_touched"],
             "peaks_note": "frac: of the measured peak (peak_source); frac_of_datasheet: of NVIDIA's "
                           "dense bf16 2250 TFLOP/s or HBM3e 8000 GB/s"}

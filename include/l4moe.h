@@ -301,6 +301,20 @@ L4MOE_API l4moe_status l4moe_check_device_status(l4moe_handle *h, void *stream);
  * context stays usable.  Allocates the handle's workspace if it has none. */
 L4MOE_API l4moe_status l4moe_selftest_wait(l4moe_handle *h, double limit_ms, void *stream);
 
+/* How the last forward on this handle was launched (all zero before the
+ * first): split_gate_up / split_down, the split-K ranges of the two GEMMs
+ * (1 = none); small_routing, routing, top-k, permutation and row copy in one
+ * launch (batches of up to 16 tokens with experts); early_shared, the
+ * gate/up launch began with the shared expert's tiles while that routing
+ * launch was still running; fused, gate/up and down ran as one launch (the
+ * kernel-timing slot of gate/up then covers both, the down slot only its
+ * finish); small_tiles, the GEMMs used the configuration for groups of at
+ * most 64 rows.  L4MOE_ERR_ARG for a null pointer. */
+typedef struct {
+    int split_gate_up, split_down, small_routing, early_shared, fused, small_tiles;
+} l4moe_plan;
+L4MOE_API l4moe_status l4moe_get_plan(const l4moe_handle *h, l4moe_plan *plan);
+
 /* Per-kernel timing.  `mask` selects kernel slots (bit i = slot i; 0 turns
  * timing off; L4MOE_TIME_ALL every slot; anything else: L4MOE_ERR_ARG).
  * For each selected slot l4moe_forward records a CUDA event before and

@@ -22,7 +22,7 @@ EXPORTED = ("l4moe_create", "l4moe_destroy", "l4moe_workspace_size", "l4moe_set_
             "l4moe_launch_count", "l4moe_last_error", "l4moe_status_string", "l4moe_version",
             "l4moe_set_timing", "l4moe_read_timing", "l4moe_kernel_name",
             "l4moe_forward_static", "l4moe_join_host", "l4moe_set_top_k",
-            "l4moe_set_weight_scales", "l4moe_selftest_wait", "l4moe_set_act_fp8")
+            "l4moe_set_weight_scales", "l4moe_selftest_wait", "l4moe_set_act_fp8", "l4moe_get_plan")
 STATIC_WORKSPACE_BYTES = 32 << 20
 NUM_KERNELS = 6
 
@@ -33,6 +33,12 @@ class L4MoEError(RuntimeError):
     def __init__(self, status: int, message: str):
         super().__init__(f"{message} (status {status})")
         self.status = status
+
+
+class Plan(ctypes.Structure):
+    _fields_ = [("split_gate_up", ctypes.c_int), ("split_down", ctypes.c_int),
+                ("small_routing", ctypes.c_int), ("early_shared", ctypes.c_int),
+                ("fused", ctypes.c_int), ("small_tiles", ctypes.c_int)]
 
 
 class Params(ctypes.Structure):
@@ -78,6 +84,7 @@ def load_library():
     lib.l4moe_set_timing.argtypes = [vp, i32]
     lib.l4moe_set_top_k.argtypes = [vp, i32]
     lib.l4moe_set_act_fp8.argtypes = [vp, i32]
+    lib.l4moe_get_plan.argtypes = [vp, ctypes.POINTER(Plan)]
     lib.l4moe_selftest_wait.argtypes = [vp, ctypes.c_double, vp]
     lib.l4moe_read_timing.argtypes = [vp, ctypes.POINTER(ctypes.c_double),
                                       ctypes.POINTER(ctypes.c_uint64)]
@@ -88,7 +95,7 @@ def load_library():
                  "l4moe_get_routing", "l4moe_check_device_status", "l4moe_version",
                  "l4moe_set_timing", "l4moe_read_timing", "l4moe_forward_static",
                  "l4moe_join_host", "l4moe_set_top_k", "l4moe_set_weight_scales", "l4moe_selftest_wait",
-                 "l4moe_set_act_fp8"):
+                 "l4moe_set_act_fp8", "l4moe_get_plan"):
         getattr(lib, name).restype = ctypes.c_int
     _lib = lib
     return lib
@@ -300,6 +307,12 @@ class L4MoE:
         """Experts per token (l4moe_set_top_k)."""
         self._check(self._lib.l4moe_set_top_k(self._h, int(k)))
         self.top_k = int(k)
+
+    def plan(self) -> dict:
+        """How the last forward was launched (l4moe_get_plan)."""
+        p = Plan()
+        self._check(self._lib.l4moe_get_plan(self._h, ctypes.byref(p)))
+        return {name: int(getattr(p, name)) for name, _ in Plan._fields_}
 
     def set_act_fp8(self, on: bool = True):
         """FP8 activation mode (l4moe_set_act_fp8): E4M3 token and hidden rows."""

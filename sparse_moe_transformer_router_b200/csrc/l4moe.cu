@@ -239,6 +239,7 @@ struct l4moe_handle {
     uint64_t launches = 0;
     std::string err;
     int last_T = 0;
+    l4moe_plan last_plan{};  // launch plan of the last forward
     // host path (l4moe_forward_host): copy streams and per-slot events so
     // consecutive calls overlap their copies with each other's compute
     cudaStream_t s_in = nullptr, s_out = nullptr;
@@ -774,6 +775,12 @@ l4moe_status run_layer(l4moe_handle* h, int T, const void* x, const void* Wr, co
     unsigned* done = fused ? err + 2 : nullptr;  // zero here; the down finish resets them
     gu.done = done;
     dn.done = done;
+    h->last_plan.split_gate_up = s_gu;
+    h->last_plan.split_down = s_dn;
+    h->last_plan.early_shared = early ? 1 : 0;
+    h->last_plan.fused = fused ? 1 : 0;
+    h->last_plan.small_tiles = small_tiles ? 1 : 0;
+    h->last_plan.small_routing = (E > 0 && T <= kSmallMaxTokens) ? 1 : 0;
     const long long gu_units = s_gu * ((long long)fb_gu_s * tb + (long long)fb_gu_r * (tbv + std::min(E, Tv)));
     const long long dn_units = s_dn * (long long)fb_dn * (tb + tbv + std::min(E, Tv));
     if (fused) {
@@ -1313,6 +1320,12 @@ const char* l4moe_kernel_name(int slot) {
 }
 
 uint64_t l4moe_launch_count(const l4moe_handle* h) { return h ? h->launches : 0; }
+
+l4moe_status l4moe_get_plan(const l4moe_handle* h, l4moe_plan* plan) {
+    if (!h || !plan) return L4MOE_ERR_ARG;
+    *plan = h->last_plan;
+    return L4MOE_OK;
+}
 
 const char* l4moe_last_error(const l4moe_handle* h) {
     return h ? h->err.c_str() : g_create_error.c_str();

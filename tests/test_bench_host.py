@@ -26,6 +26,11 @@ def test_kernel_flops_add_up_to_the_layer(name):
     # the weights each GEMM streams: touched routed experts plus the shared one
     w = accounting.W_BYTES[cfg.dtype]
     assert k["gemm_down"]["bytes"] >= (cfg.num_experts * cfg.expert_ffn + cfg.shared_ffn) * cfg.d_model * w
+    # a fused launch: the gate/up slot carries both contractions, the down slot the finish
+    f = bench.kernel_flops_bytes(cfg, counts, plan={"fused": 1, "split_down": 3})
+    assert f["gemm_gate_up"]["flops"] == k["gemm_gate_up"]["flops"] + k["gemm_down"]["flops"]
+    assert f["gemm_gate_up"]["bytes"] == k["gemm_gate_up"]["bytes"] + k["gemm_down"]["bytes"]
+    assert f["gemm_down"]["flops"] == 0 and sum(v["flops"] for v in f.values()) == total
 
 
 def test_profile_traffic_needs_the_current_kernel_hash(tmp_path, monkeypatch):

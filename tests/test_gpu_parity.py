@@ -135,6 +135,23 @@ def test_topk_layer_matches_oracle(name):
     print(f"{name}: k={k} {describe(res)}, excluded {rep['excluded']}, flipped {rep['flipped']}")
 
 
+def test_launch_plan_of_small_and_large_batches():
+    """Batches of up to 16 tokens route in one launch; with bf16 or fp32
+    activations their gate/up starts with the shared expert's tiles while the
+    routing runs and the two contractions go out as one fused launch (layers
+    with coded weights read the routing's f16 copy of x and do not start
+    early); larger batches take the separate launches."""
+    for name, small, early in (("bf16_T1", 1, 1), ("bf16_T16_E128", 1, 1), ("f32_T16_E6", 1, 1),
+                               ("fp8_T1", 1, 0), ("bf16_ragged", 0, 0)):
+        inp = generate(SMALL[name], seed=0, device="cuda")
+        layer = make_layer(inp)
+        run_gpu(layer, inp)
+        p = layer.plan()
+        assert p["small_routing"] == small and p["early_shared"] == early, (name, p)
+        assert p["fused"] == (early and p["split_gate_up"] == 1), (name, p)
+        assert p["small_tiles"] == (SMALL[name].T <= 64), (name, p)
+
+
 def test_top_k_bounds():
     from sparse_moe_transformer_router_b200.binding import ERR_ARG, L4MoEError
     inp = generate(TOPK["bf16_k2"][0], seed=0, device="cuda")
