@@ -96,6 +96,7 @@ bool coded8(l4moe_dtype dt) { return dt == L4MOE_FP8_E4M3 || dt == L4MOE_INT8 ||
 // ranges of at least 8 k-blocks.
 struct SplitPlan {
     int s_gu, s_dn;
+    bool fused;  // gate/up and down in one launch (small batches, see run_layer)
 };
 
 SplitPlan split_plan(const l4moe_params& p, int T, int sms, int k = 1, bool act8 = false) {
@@ -132,6 +133,18 @@ SplitPlan split_plan(const l4moe_params& p, int T, int sms, int k = 1, bool act8
     // gate/up splits only below that.
     sp.s_gu = 2 * gu_tiles < pairs ? pick(gu_tiles, d / kblk) : 1;
     sp.s_dn = pick((long long)fb_dn * (eg + 1), std::min(F, Fs) / kblk);
+    // small batches of layers whose shared operand is x run both GEMMs as one
+    // launch (when gate/up needs no split); there the down units share the
+    // pairs with the gate/up tiles, and units about as long as a gate/up tile
+    // (a K split of about min(F, Fs) / d, ranges of at least 8 k-blocks)
+    // packed best (Maverick decode, T = 1: 2 splits 0.109 ms, 4 0.113, 11
+    // -- the fill-the-wave count of a down launch alone -- 0.121, 16 0.133)
+    sp.fused = E > 0 && T <= kSmallMaxTokens && !coded8(p.dtype) && sp.s_gu == 1;
+    if (sp.fused) {
+        const int nkb = std::min(F, Fs) / kblk;
+        sp.s_dn = std::max(1, std::min({kMaxSplit, std::max(1, nkb / 8),
+                                        (int)((std::min(F, Fs) + d / 2) / d)}));
+    }
     return sp;
 }
 
@@ -771,7 +784,7 @@ l4moe_status run_layer(l4moe_handle* h, int T, const void* x, const void* Wr, co
     // finished gate/up tiles) only for the hidden rows of its own class, so
     // the pairs that finish their gate/up tiles stream down weights while the
     // others still stream gate/up weights
-    const bool fused = early && s_gu == 1;
+    const bool fused = plan.fused;
     unsigned* done = fused ? err + 2 : nullptr;  // zero here; the down finish resets them
     gu.done = done;
     dn.done = done;
