@@ -47,6 +47,21 @@ __global__ void __launch_bounds__(256) gateup_finish_kernel(
     }
 }
 
+// Four fp32 sums -> outputs 4i .. 4i+3, rounded once to the output type.
+template <typename ET>
+__device__ __forceinline__ void store_out4(ET* out, long long i, float4 acc) {
+    if constexpr (sizeof(ET) == 2) {
+        const __nv_bfloat162 lo = __floats2bfloat162_rn(acc.x, acc.y);
+        const __nv_bfloat162 hi = __floats2bfloat162_rn(acc.z, acc.w);
+        uint2 pk;
+        pk.x = *reinterpret_cast<const uint32_t*>(&lo);
+        pk.y = *reinterpret_cast<const uint32_t*>(&hi);
+        reinterpret_cast<uint2*>(out)[i] = pk;
+    } else {
+        reinterpret_cast<float4*>(out)[i] = acc;
+    }
+}
+
 // Down finish: out[t] = rn(sum over splits s and selected experts j of the
 // routed partial of entry t * k + j, then sum over s of the shared partial)
 // -- one rounding, a fixed order.  Partials: routed [splits_r][T * k][d],
@@ -63,8 +78,28 @@ __global__ void __launch_bounds__(256) down_finish_kernel(const float* __restric
     if (done && blockIdx.x == 0 && threadIdx.x < 2) done[threadIdx.x] = 0u;
     const long long n4 = n >> 2;
     const int d4 = d >> 2;
-    for (long long i = blockIdx.x * (long long)blockDim.x + threadIdx.x; i < n4;
-         i += (long long)gridDim.x * blockDim.x) {
+    const long long stride = (long long)gridDim.x * blockDim.x;
+    long long i0 = blockIdx.x * (long long)blockDim.x + threadIdx.x;
+    if (k == 1 && splits_r == 1 && splits_s == 1) {
+        // one routed and one shared partial per output (prefill): two outputs
+        // per thread and pass, their four loads issued before any is used,
+        // so that enough bytes are in flight to keep HBM busy
+        for (; i0 < n4; i0 += 2 * stride) {
+            const long long i1 = i0 + stride;
+            const bool two = i1 < n4;
+            const float4 r0 = reinterpret_cast<const float4*>(part_r)[i0];
+            const float4 s0 = reinterpret_cast<const float4*>(part_s)[i0];
+            float4 r1 = make_float4(0.f, 0.f, 0.f, 0.f), s1 = r1;
+            if (two) {
+                r1 = reinterpret_cast<const float4*>(part_r)[i1];
+                s1 = reinterpret_cast<const float4*>(part_s)[i1];
+            }
+            store_out4(out, i0, make_float4(r0.x + s0.x, r0.y + s0.y, r0.z + s0.z, r0.w + s0.w));
+            if (two) store_out4(out, i1, make_float4(r1.x + s1.x, r1.y + s1.y, r1.z + s1.z, r1.w + s1.w));
+        }
+        return;
+    }
+    for (long long i = i0; i < n4; i += stride) {
         float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
         if (k == 1) {  // routed row t is entry t: the same index as the output
             // the partials of up to 8 splits are loaded before any is added
@@ -96,16 +131,7 @@ __global__ void __launch_bounds__(256) down_finish_kernel(const float* __restric
 #pragma unroll
             for (int j = 0; j < 8; ++j) acc.x += v[j].x, acc.y += v[j].y, acc.z += v[j].z, acc.w += v[j].w;
         }
-        if constexpr (sizeof(ET) == 2) {
-            const __nv_bfloat162 lo = __floats2bfloat162_rn(acc.x, acc.y);
-            const __nv_bfloat162 hi = __floats2bfloat162_rn(acc.z, acc.w);
-            uint2 pk;
-            pk.x = *reinterpret_cast<const uint32_t*>(&lo);
-            pk.y = *reinterpret_cast<const uint32_t*>(&hi);
-            reinterpret_cast<uint2*>(out)[i] = pk;
-        } else {
-            reinterpret_cast<float4*>(out)[i] = acc;
-        }
+        store_out4(out, i, acc);
     }
 }
 

@@ -645,15 +645,19 @@ l4moe_status run_layer(l4moe_handle* h, int T, const void* x, const void* Wr, co
             ensure_smem_attr(attr_done, router_mma_kernel, rmma::SMEM_BYTES);
             const int n_chunk = split_router ? 16 : E;
             const int tiles = (T + 127) / 128;
+            // stages sized for this launch's experts; two CTAs share an SM
+            // when that leaves each at most half of its shared memory
+            const size_t rsmem = rmma::smem_bytes(n_chunk);
+            const int per_sm = rsmem <= 112 * 1024 ? 2 : 1;
             int kslices;
             if (split_router) {
                 kslices = std::min(kRouterKSplit, std::max(1, d / 256));
             } else {
-                // few token tiles: K slices per tile (at most 4 and the SMs'
-                // worth), reduced inside a cluster of the slices
-                kslices = std::max(1, std::min({4, h->sms / tiles, d / 256}));
+                // few token tiles: K slices per tile (a cluster of at most 8,
+                // at most the resident CTAs' worth), reduced inside the cluster
+                kslices = std::max(1, std::min({4 * per_sm, per_sm * h->sms / tiles, d / 256}));
             }
-            launch_kc(router_mma_kernel, dim3(tiles, E / n_chunk, kslices), dim3(128), rmma::SMEM_BYTES, st,
+            launch_kc(router_mma_kernel, dim3(tiles, E / n_chunk, kslices), dim3(128), rsmem, st,
                       kslices == 1 ? 0u : (unsigned)kslices, m_x, m_wr, (const float*)h->bias,
                       T, d, E, n_chunk, logits, idx, gate, lmax, margin, err, k);
         } else {
@@ -832,7 +836,7 @@ l4moe_status run_layer(l4moe_handle* h, int T, const void* x, const void* Wr, co
     {
         const long long n = (long long)T * d;
         // the routed planes then the shared ones; without experts only the shared
-        launch_k(down_finish_kernel<ET>, dim3((int)std::min<long long>((n / 4 + 255) / 256, 4LL * h->sms)),
+        launch_k(down_finish_kernel<ET>, dim3((int)std::min<long long>((n / 4 + 255) / 256, 8LL * h->sms)),
                  dim3(256), 0, st, (const float*)part, dn.part_stride_routed, E > 0 ? s_dn : 0,
                  (const float*)dn.part_shared, dn.part_stride_shared, s_dn, k, d, n, static_cast<ET*>(out),
                  done);

@@ -209,6 +209,15 @@ constexpr int B_BOX_BYTES = 64 * 128;  // 64 K rows x 64 experts (bf16)
 constexpr int MAX_B_BOXES = 4;         // E <= 256
 constexpr int STAGE_BYTES = A_BYTES + MAX_B_BOXES * B_BOX_BYTES;
 constexpr size_t SMEM_BYTES = 1024 + (size_t)STAGES * STAGE_BYTES + (2 * STAGES + 1) * 8 + 16;
+// A launch whose CTAs each take n_chunk experts needs stages of the token
+// tile plus ceil(n_chunk / 64) weight boxes only: fewer bytes, so that two
+// CTAs fit on an SM when the experts are few.
+__host__ __device__ constexpr int stage_bytes(int n_chunk) {
+    return A_BYTES + ((n_chunk + 63) / 64) * B_BOX_BYTES;
+}
+__host__ __device__ constexpr size_t smem_bytes(int n_chunk) {
+    return 1024 + (size_t)STAGES * stage_bytes(n_chunk) + (2 * STAGES + 1) * 8 + 16;
+}
 }  // namespace rmma
 
 // Cluster K-split (gridDim.z = S > 1, launched as clusters of (1, 1, S)):
@@ -227,7 +236,7 @@ constexpr size_t SMEM_BYTES = 1024 + (size_t)STAGES * STAGE_BYTES + (2 * STAGES 
 // stores the biased fp32 logits to logits[T][E]; the arg-max then runs in
 // the permutation kernel.  This spreads the router weight stream over
 // (E / n_chunk) x slices SMs instead of one.
-__global__ void __launch_bounds__(128, 1)
+__global__ void __launch_bounds__(128, 2)
     router_mma_kernel(const __grid_constant__ CUtensorMap x_map, const __grid_constant__ CUtensorMap wr_map,
                       const float* __restrict__ bias, int T, int d, int E, int n_chunk,
                       float* __restrict__ logits, int32_t* __restrict__ idx,
@@ -237,7 +246,8 @@ __global__ void __launch_bounds__(128, 1)
     extern __shared__ uint8_t rsmem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>(
         (reinterpret_cast<uintptr_t>(rsmem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
-    uint64_t* bars = reinterpret_cast<uint64_t*>(smem + (size_t)rmma::STAGES * rmma::STAGE_BYTES);
+    const int stage_bytes = rmma::stage_bytes(n_chunk);  // this launch's stage stride
+    uint64_t* bars = reinterpret_cast<uint64_t*>(smem + (size_t)rmma::STAGES * stage_bytes);
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 2 * rmma::STAGES + 1);
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const uint32_t stage0 = smem_u32(smem), bar0 = smem_u32(bars);
@@ -279,7 +289,7 @@ __global__ void __launch_bounds__(128, 1)
         for (int kb = 0; kb < nkb; ++kb) {
             if (!mbar_wait(empty_bar(stage), phase ^ 1u, err, DEV_ERR_TIMEOUT_PRODUCER)) break;
             mbar_arrive_expect_tx(full_bar(stage), rmma::A_BYTES + nbb * rmma::B_BOX_BYTES);
-            const uint32_t sb = stage0 + (uint32_t)stage * rmma::STAGE_BYTES;
+            const uint32_t sb = stage0 + (uint32_t)stage * stage_bytes;
             const int kg = (kb_begin + kb) * 64;
             tma_load_2d(sb, &x_map, full_bar(stage), kg, t0);
             tma_load_2d(sb + 64 * 128, &x_map, full_bar(stage), kg, t0 + 64);
@@ -302,7 +312,7 @@ __global__ void __launch_bounds__(128, 1)
         for (int kb = 0; kb < nkb; ++kb) {
             if (!mbar_wait(full_bar(stage), phase, err, DEV_ERR_TIMEOUT_MMA)) break;
             tc_fence_after();
-            const uint32_t sb = stage0 + (uint32_t)stage * rmma::STAGE_BYTES;
+            const uint32_t sb = stage0 + (uint32_t)stage * stage_bytes;
 #pragma unroll
             for (int kk = 0; kk < 4; ++kk) {
                 const uint64_t adesc = smem_desc(sb + kk * 32, 16, 1024, 2);
