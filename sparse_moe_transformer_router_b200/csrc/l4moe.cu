@@ -188,7 +188,7 @@ WsLayout ws_layout(const l4moe_params& p, int T, int sms, int k, bool act8 = fal
     L.gslot = take(4 * tv);
     L.counts = take(4 * E);
     L.offsets = take(4 * (E + 1));
-    L.chunk = take(4 * ((tv + kDispatchChunk - 1) / kDispatchChunk) * E);  // dispatch chunk bases
+    L.chunk = take(4 * router_max_chunks(tv) * E);  // dispatch chunk bases (either dispatch)
     L.tab_gu = take(sizeof(GroupTable));
     L.tab_dn = take(sizeof(GroupTable));
     L.xg = take(tv * p.d_model * es);
@@ -636,6 +636,11 @@ l4moe_status run_layer(l4moe_handle* h, int T, const void* x, const void* Wr, co
         // one token tile and many experts: split the router over 16-expert chunks
         const bool split_router = sizeof(ET) == 2 && E % 16 == 0 && E >= 32 && T <= 128;
         float* logits = split_router ? reinterpret_cast<float*>(w + L.logits) : nullptr;
+        int32_t* chunk_base = logits ? nullptr : reinterpret_cast<int32_t*>(w + L.chunk);
+        // the tensor-core top-1 router finishes the dispatch itself (a chunk per CTA)
+        const bool router_dispatch = sizeof(ET) == 2 && E % 8 == 0 && !split_router && k == 1 &&
+                                     router_max_chunks(T) <= (size_t)router_stage_cap(E);
+        int router_slices = 1;  // K slices of the tensor-core router launch
         if (sizeof(ET) == 2 && E % 8 == 0) {
             // tensor-core router: W_router [d, E] as the MN-major operand
             CUtensorMap m_wr;
@@ -647,7 +652,8 @@ l4moe_status run_layer(l4moe_handle* h, int T, const void* x, const void* Wr, co
             const int tiles = (T + 127) / 128;
             // stages sized for this launch's experts; two CTAs share an SM
             // when that leaves each at most half of its shared memory
-            const size_t rsmem = rmma::smem_bytes(n_chunk);
+            const int nst = rmma::stages(n_chunk);
+            const size_t rsmem = rmma::smem_bytes(n_chunk, nst);
             const int per_sm = rsmem <= 112 * 1024 ? 2 : 1;
             int kslices;
             if (split_router) {
@@ -657,37 +663,57 @@ l4moe_status run_layer(l4moe_handle* h, int T, const void* x, const void* Wr, co
                 // at most the resident CTAs' worth), reduced inside the cluster
                 kslices = std::max(1, std::min({4 * per_sm, per_sm * h->sms / tiles, d / 256}));
             }
+            while (kslices & (kslices - 1)) kslices &= kslices - 1;  // a power of two: it divides the tile
+            router_slices = kslices;
+            RouterDispatch dsp{};
+            if (router_dispatch) {
+                dsp.chunk_base = chunk_base;
+                dsp.counts = counts;
+                dsp.offsets = offsets;
+                dsp.inv = inv;
+                dsp.tab_gu = tab_gu;
+                dsp.tab_dn = tab_dn;
+                dsp.ticket = err + 1;  // zero between launches (the last CTA resets it)
+                dsp.fb_gu_routed = fb_gu_r * s_gu;
+                dsp.fb_gu_shared = fb_gu_s * s_gu;
+                dsp.fb_down = fb_dn * s_dn;
+            }
             launch_kc(router_mma_kernel, dim3(tiles, E / n_chunk, kslices), dim3(128), rsmem, st,
                       kslices == 1 ? 0u : (unsigned)kslices, m_x, m_wr, (const float*)h->bias,
-                      T, d, E, n_chunk, logits, idx, gate, lmax, margin, err, k);
+                      T, d, E, n_chunk, logits, idx, gate, lmax, margin, err, k, nst, dsp);
         } else {
             launch_router<ET>(x, Wr, h->bias, T, d, E, idx, gate, lmax, margin, k, st);
         }
         t_router.stop();
         L4MOE_CHECK_LAUNCH("router launch");
 
-        const size_t psmem = sizeof(int) * (34 * (size_t)E + 1);
-        int32_t* chunk_base = nullptr;
-        LaunchTimer t_perm(h, 1, st);
-        if (logits) {
-            // the arg-max of the split logits and the whole permutation in one CTA
-            launch_k(permute_kernel, dim3(1), dim3(1024), psmem, st, (const float*)logits,
-                     gate, lmax, margin, idx, T, k, E, fb_gu_r * s_gu, fb_gu_s * s_gu, fb_dn * s_dn, counts,
-                     offsets, perm, inv, tab_gu, tab_dn, err);
-        } else {
-            chunk_base = reinterpret_cast<int32_t*>(w + L.chunk);
-            launch_k(dispatch_kernel, dim3((Tv + kDispatchChunk - 1) / kDispatchChunk), dim3(kDispatchChunk), psmem,
-                     st, (const int32_t*)idx, T, k, E, fb_gu_r * s_gu, fb_gu_s * s_gu, fb_dn * s_dn, chunk_base,
-                     counts, offsets, inv, tab_gu, tab_dn, err + 1, err);
+        // dispatch_kernel: wcnt[32][E] (also the staging of its last CTA's
+        // scan, which needs a row per chunk), tot[E], soff[E + 1]
+        const size_t dchunks = (Tv + kDispatchChunk - 1) / kDispatchChunk;
+        const size_t psmem = sizeof(int) * (std::max<size_t>(32 * (size_t)E, dchunks) + 2 * (size_t)E + 1);
+        if (!router_dispatch) {
+            LaunchTimer t_perm(h, 1, st);
+            if (logits) {
+                // the arg-max of the split logits and the whole permutation in one CTA
+                launch_k(permute_kernel, dim3(1), dim3(1024), psmem, st, (const float*)logits,
+                         gate, lmax, margin, idx, T, k, E, fb_gu_r * s_gu, fb_gu_s * s_gu, fb_dn * s_dn, counts,
+                         offsets, perm, inv, tab_gu, tab_dn, err);
+            } else {
+                launch_k(dispatch_kernel, dim3((Tv + kDispatchChunk - 1) / kDispatchChunk), dim3(kDispatchChunk),
+                         psmem, st, (const int32_t*)idx, T, k, E, fb_gu_r * s_gu, fb_gu_s * s_gu, fb_dn * s_dn,
+                         chunk_base, counts, offsets, inv, tab_gu, tab_dn, err + 1, err);
+            }
+            t_perm.stop();
+            L4MOE_CHECK_LAUNCH("permute launch");
         }
-        t_perm.stop();
-        L4MOE_CHECK_LAUNCH("permute launch");
+        // entries per dispatch chunk: the router's tokens per CTA, or dispatch_kernel's
+        const int chunk = router_dispatch ? router_tokens_per_cta(router_slices) : kDispatchChunk;
 
         const int sc_blocks = std::min((Tv + 7) / 8, h->sms * 8);
         LaunchTimer t_rows(h, 2, st);
         launch_k(permute_rows_kernel<ET, GT>, dim3(sc_blocks), dim3(256), 0, st, static_cast<const ET*>(x),
                  (const float*)gate, inv, T, k, d, xg, gslot, FP8W ? x16 : (GT*)nullptr, (const int32_t*)idx,
-                 (const int32_t*)chunk_base, E, perm, tokscale);
+                 (const int32_t*)chunk_base, chunk, E, perm, tokscale);
         t_rows.stop();
         L4MOE_CHECK_LAUNCH("row permutation launch");
     } else {
@@ -702,7 +728,7 @@ l4moe_status run_layer(l4moe_handle* h, int T, const void* x, const void* Wr, co
             LaunchTimer t_rows(h, 2, st);
             launch_k(permute_rows_kernel<ET, GT>, dim3(sc_blocks), dim3(256), 0, st, static_cast<const ET*>(x),
                      (const float*)nullptr, (int32_t*)nullptr, T, 1, d, x16, (float*)nullptr, (GT*)nullptr,
-                     (const int32_t*)nullptr, (const int32_t*)nullptr, 0, (int32_t*)nullptr, tokscale);
+                     (const int32_t*)nullptr, (const int32_t*)nullptr, 1, 0, (int32_t*)nullptr, tokscale);
             t_rows.stop();
             L4MOE_CHECK_LAUNCH("row conversion launch");
         }

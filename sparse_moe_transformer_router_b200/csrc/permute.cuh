@@ -68,6 +68,196 @@ __device__ void build_table(GroupTable* tab, int G, RowsF rows_of, Row0F row0_of
     }
 }
 
+// Stable ranks inside one chunk of entries, thread i of the CTA holding the
+// chunk's entry i with expert e (-1: none).  Returns the entry's rank among
+// the chunk's entries of its expert held by lower threads (-1 for none) and
+// writes the chunk's per-expert counts to chunk_row[E].  A warp's
+// __match_any_sync groups its entries by expert; a prefix over the warps,
+// per expert, orders the groups.  smem: wcnt[warps][E] ints.
+__device__ int chunk_rank(int e, int E, int* wcnt, int32_t* __restrict__ chunk_row) {
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5, nwarps = blockDim.x >> 5;
+    for (int i = tid; i < nwarps * E; i += blockDim.x) wcnt[i] = 0;
+    __syncthreads();
+    const unsigned same = __match_any_sync(0xffffffffu, e);
+    const int lane_rank = __popc(same & ((1u << lane) - 1u));
+    if (e >= 0 && lane_rank == 0) wcnt[warp * E + e] = __popc(same);
+    __syncthreads();
+    for (int x = tid; x < E; x += blockDim.x) {  // prefix over warps, per expert
+        int acc = 0;
+        for (int w = 0; w < nwarps; ++w) {
+            const int v = wcnt[w * E + x];
+            wcnt[w * E + x] = acc;
+            acc += v;
+        }
+        chunk_row[x] = acc;
+    }
+    __syncthreads();
+    return e >= 0 ? wcnt[warp * E + e] + lane_rank : -1;
+}
+
+// The final step of a chunked dispatch, run by one CTA once every chunk's
+// per-expert counts are in chunk_base[chunks][E] and visible to it: each
+// count becomes its chunk's first slot for the expert (offsets[e] plus the
+// expert's entries in earlier chunks), and counts[E], offsets[E + 1] and the
+// two work lists are written.  Any CTA size that is a multiple of 32.
+// The counts are staged in shared memory a block of experts at a time, each
+// thread's loads of a pass issued before any is stored (one L2 round trip
+// per pass, not per element); tpe consecutive threads scan one expert, each
+// a run of consecutive chunks, joined by a segmented shuffle scan; warp 0
+// then scans over the experts and writes the lists.
+// smem: tot[E], soff[E + 1] and stage[cap] ints, cap >= chunks, stage and
+// chunk_base 16-byte aligned.  U: 4-byte loads in flight per thread (2U
+// 16-byte ones): more for a small CTA, fewer where registers are scarce.
+template <int U>
+__device__ void dispatch_finish(int32_t* chunk_base, int chunks, int T, int E, int fb_gu_routed,
+                                int fb_gu_shared, int fb_down, int32_t* __restrict__ counts,
+                                int32_t* __restrict__ offsets, GroupTable* tab_gu, GroupTable* tab_dn,
+                                int* tot, int* soff, int* stage, int cap) {
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5, nt = blockDim.x;
+    // threads per expert: a power of two, at most a warp
+    int tpe = 1;
+    while (tpe < 32 && 2 * tpe * E <= nt) tpe *= 2;
+    const int xblk = max(1, min(E, cap / chunks));  // experts per staged block
+    const int per = (chunks + tpe - 1) / tpe;        // chunks per thread
+    const int seg = lane & ~(tpe - 1);               // first lane of this thread's segment
+    const bool whole = xblk >= E;                    // every expert staged at once: no write-back pass
+    for (int x0 = 0; x0 < E; x0 += xblk) {
+        const int xe = min(xblk, E - x0);
+        const int n = chunks * xe;
+        if (whole && (E & 3) == 0) {  // [chunks][E] as it lies in memory: 16-byte loads, 2U in flight
+            const int n4 = n >> 2;
+            const int4* src = reinterpret_cast<const int4*>(chunk_base);
+            int4* dst = reinterpret_cast<int4*>(stage);
+            for (int i0 = 0; i0 < n4; i0 += 2 * U * nt) {
+                int4 v[2 * U];
+#pragma unroll
+                for (int j = 0; j < 2 * U; ++j) {
+                    const int i = i0 + j * nt + tid;
+                    if (i < n4) v[j] = __ldcg(src + i);
+                }
+#pragma unroll
+                for (int j = 0; j < 2 * U; ++j) {
+                    const int i = i0 + j * nt + tid;
+                    if (i < n4) dst[i] = v[j];
+                }
+            }
+        } else {
+            for (int i0 = 0; i0 < n; i0 += U * nt) {
+                int v[U];
+#pragma unroll
+                for (int j = 0; j < U; ++j) {
+                    const int i = i0 + j * nt + tid;
+                    const int c = i / xe;
+                    v[j] = i < n ? __ldcg(chunk_base + (size_t)c * E + x0 + (i - c * xe)) : 0;
+                }
+#pragma unroll
+                for (int j = 0; j < U; ++j) {
+                    const int i = i0 + j * nt + tid;
+                    if (i < n) stage[i] = v[j];
+                }
+            }
+        }
+        __syncthreads();
+        for (int xx0 = 0; xx0 < xe; xx0 += nt / tpe) {
+            const int xx = xx0 + tid / tpe;  // this thread's expert (block-relative)
+            const int part = tid & (tpe - 1);
+            const int c0 = min(chunks, part * per), c1 = min(chunks, c0 + per);
+            int s = 0;
+            if (xx < xe) {
+#pragma unroll 8
+                for (int c = c0; c < c1; ++c) s += stage[c * xe + xx];
+            }
+            int incl = s;  // inclusive scan over the expert's tpe threads
+            for (int off = 1; off < tpe; off <<= 1) {
+                const int o = __shfl_up_sync(0xffffffffu, incl, off, tpe);
+                if ((lane - seg) >= off) incl += o;
+            }
+            int acc = incl - s;
+            if (xx < xe) {
+#pragma unroll 8
+                for (int c = c0; c < c1; ++c) {
+                    const int v = stage[c * xe + xx];
+                    stage[c * xe + xx] = acc;
+                    acc += v;
+                }
+                if (part == tpe - 1) tot[x0 + xx] = incl;
+            }
+        }
+        __syncthreads();
+        if (!whole) {  // the block's prefixes back to the chunk bases (the offsets follow)
+            for (int i = tid; i < n; i += nt) {
+                const int c = i / xe, x = i - c * xe;
+                chunk_base[(size_t)c * E + x0 + x] = stage[i];
+            }
+            __syncthreads();
+        }
+    }
+    __syncthreads();
+    if (warp == 0) {  // exclusive scan of the counts (up to 8 experts per lane)
+        int local[8];
+        int sum = 0;
+#pragma unroll
+        for (int j = 0; j < 8; ++j) {
+            const int x = lane * 8 + j;
+            local[j] = (x < E) ? tot[x] : 0;
+            sum += local[j];
+        }
+        const int incl = warp_incl_scan(sum);
+        int acc = incl - sum;
+#pragma unroll
+        for (int j = 0; j < 8; ++j) {
+            const int x = lane * 8 + j;
+            if (x < E) {
+                soff[x] = acc;
+                offsets[x] = acc;
+                counts[x] = local[j];
+            }
+            acc += local[j];
+        }
+        if (lane == 31) {
+            soff[E] = incl;
+            offsets[E] = incl;
+        }
+    }
+    __syncthreads();
+    if (whole && (E & 3) == 0) {  // stage is [chunks][E]: 16-byte stores
+        const int4* src = reinterpret_cast<const int4*>(stage);
+        int4* dst = reinterpret_cast<int4*>(chunk_base);
+        for (int i = tid; i < (chunks * E) >> 2; i += nt) {
+            const int x = (4 * i) % E;
+            const int4 v = src[i];
+            dst[i] = make_int4(v.x + soff[x], v.y + soff[x + 1], v.z + soff[x + 2], v.w + soff[x + 3]);
+        }
+    } else if (whole) {
+        for (int i = tid; i < chunks * E; i += nt) chunk_base[i] = stage[i] + soff[i % E];
+    } else {
+        for (int i0 = 0; i0 < chunks * E; i0 += U * nt) {
+            int v[U];
+#pragma unroll
+            for (int j = 0; j < U; ++j) {
+                const int i = i0 + j * nt + tid;
+                v[j] = i < chunks * E ? chunk_base[i] : 0;
+            }
+#pragma unroll
+            for (int j = 0; j < U; ++j) {
+                const int i = i0 + j * nt + tid;
+                if (i < chunks * E) chunk_base[i] = v[j] + soff[i % E];
+            }
+        }
+    }
+    if (warp == 0) {
+        // gate/up: candidate 0 is the shared expert, 1..E the routed experts
+        build_table(
+            tab_gu, E + 1, [&](int g) { return g == 0 ? T : tot[g - 1]; },
+            [&](int g) { return g == 0 ? 0 : soff[g - 1]; }, [&](int g) { return g == 0 ? E : g - 1; },
+            [&](int g) { return g == 0 ? fb_gu_shared : fb_gu_routed; });
+        build_table(
+            tab_dn, E + 1, [&](int g) { return g == 0 ? T : tot[g - 1]; },
+            [&](int g) { return g == 0 ? 0 : soff[g - 1]; }, [&](int g) { return g == 0 ? E : g - 1; },
+            [&](int) { return fb_down; });
+    }
+}
+
 // Work lists of a layer without experts: one group (the shared SwiGLU, as
 // expert 0 == num_experts) over the T tokens in order.  One warp.
 __global__ void dense_table_kernel(GroupTable* tab_gu, GroupTable* tab_dn, int T, int fb_gu, int fb_dn) {
@@ -264,24 +454,30 @@ __global__ void __launch_bounds__(1024) permute_kernel(const float* __restrict__
 // writes counts[E], offsets[E + 1] and the two work lists, and resets the
 // ticket.  A slot is then chunk_base[c][e] + inv[n] (permute_rows_kernel):
 // the stable expert order, as the single-CTA permute_kernel gives it.
-// smem: wcnt[32][E] + tot[E] + soff[E + 1] ints.
+// smem: wcnt[max(32 * E, chunks)] + tot[E] + soff[E + 1] ints.
 constexpr int kDispatchChunk = 1024;
+// Chunks of either dispatch of n entries: dispatch_kernel's of kDispatchChunk
+// entries, or a dispatching router's of 128 / S tokens (S <= 8 K slices,
+// 128-token tiles, the last one ragged), whichever are more.
+__host__ __device__ constexpr size_t router_max_chunks(size_t n) {
+    return 8 * ((n + 127) / 128) > (n + kDispatchChunk - 1) / kDispatchChunk ? 8 * ((n + 127) / 128)
+                                                                              : (n + kDispatchChunk - 1) / kDispatchChunk;
+}
 
 __global__ void __launch_bounds__(kDispatchChunk) dispatch_kernel(
     const int32_t* __restrict__ idx, int T, int k, int E, int fb_gu_routed, int fb_gu_shared, int fb_down,
     int32_t* __restrict__ chunk_base, int32_t* __restrict__ counts, int32_t* __restrict__ offsets,
     int32_t* __restrict__ inv, GroupTable* tab_gu, GroupTable* tab_dn, unsigned* ticket, unsigned* err) {
     pdl_enter();
-    extern __shared__ int dsm[];
+    extern __shared__ __align__(16) int dsm[];
+    const int stage_n = max(32 * E, (int)gridDim.x);  // wcnt, then the last CTA's staging (a row per chunk)
     int* wcnt = dsm;           // [32][E]
-    int* tot = dsm + 32 * E;   // [E]
+    int* tot = dsm + stage_n;  // [E]
     int* soff = tot + E;       // [E + 1]
     __shared__ unsigned s_last;
-    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    const int tid = threadIdx.x;
     const int Tv = T * k;
     const int chunks = gridDim.x;
-    for (int i = tid; i < 32 * E; i += kDispatchChunk) wcnt[i] = 0;
-    __syncthreads();
     const int n = blockIdx.x * kDispatchChunk + tid;
     int e = -1;
     if (n < Tv) {
@@ -291,21 +487,8 @@ __global__ void __launch_bounds__(kDispatchChunk) dispatch_kernel(
             e = -1;
         }
     }
-    const unsigned same = __match_any_sync(0xffffffffu, e);
-    const int lane_rank = __popc(same & ((1u << lane) - 1u));
-    if (e >= 0 && lane_rank == 0) wcnt[warp * E + e] = __popc(same);
-    __syncthreads();
-    for (int x = tid; x < E; x += kDispatchChunk) {  // prefix over warps, per expert
-        int acc = 0;
-        for (int w = 0; w < 32; ++w) {
-            const int v = wcnt[w * E + x];
-            wcnt[w * E + x] = acc;
-            acc += v;
-        }
-        chunk_base[(size_t)blockIdx.x * E + x] = acc;  // this chunk's count for now
-    }
-    __syncthreads();
-    if (n < Tv) inv[n] = e >= 0 ? wcnt[warp * E + e] + lane_rank : -1;
+    const int r = chunk_rank(e, E, wcnt, chunk_base + (size_t)blockIdx.x * E);
+    if (n < Tv) inv[n] = r;
 
     __threadfence();
     __syncthreads();
@@ -313,58 +496,11 @@ __global__ void __launch_bounds__(kDispatchChunk) dispatch_kernel(
     __syncthreads();
     if (!s_last) return;
     __threadfence();
-    // last CTA: per expert, the entries of earlier chunks, then the totals
-    for (int x = tid; x < E; x += kDispatchChunk) {
-        int acc = 0;
-#pragma unroll 8
-        for (int c = 0; c < chunks; ++c) {
-            const int v = __ldcg(chunk_base + (size_t)c * E + x);
-            chunk_base[(size_t)c * E + x] = acc;
-            acc += v;
-        }
-        tot[x] = acc;
-    }
-    __syncthreads();
+    // last CTA: the chunk bases, counts, offsets and work lists (the warps'
+    // count rows are free now and stage the chunks' counts)
+    dispatch_finish<2>(chunk_base, chunks, T, E, fb_gu_routed, fb_gu_shared, fb_down, counts, offsets, tab_gu,
+                       tab_dn, tot, soff, wcnt, stage_n);
     if (tid == 0) *ticket = 0u;
-    if (warp == 0) {  // exclusive scan of the counts (up to 8 experts per lane)
-        int local[8];
-        int sum = 0;
-#pragma unroll
-        for (int j = 0; j < 8; ++j) {
-            const int x = lane * 8 + j;
-            local[j] = (x < E) ? tot[x] : 0;
-            sum += local[j];
-        }
-        const int incl = warp_incl_scan(sum);
-        int acc = incl - sum;
-#pragma unroll
-        for (int j = 0; j < 8; ++j) {
-            const int x = lane * 8 + j;
-            if (x < E) {
-                soff[x] = acc;
-                offsets[x] = acc;
-                counts[x] = local[j];
-            }
-            acc += local[j];
-        }
-        if (lane == 31) {
-            soff[E] = incl;
-            offsets[E] = incl;
-        }
-    }
-    __syncthreads();
-    for (int i = tid; i < chunks * E; i += kDispatchChunk) chunk_base[i] += soff[i % E];
-    if (warp == 0) {
-        // gate/up: candidate 0 is the shared expert, 1..E the routed experts
-        build_table(
-            tab_gu, E + 1, [&](int g) { return g == 0 ? T : tot[g - 1]; },
-            [&](int g) { return g == 0 ? 0 : soff[g - 1]; }, [&](int g) { return g == 0 ? E : g - 1; },
-            [&](int g) { return g == 0 ? fb_gu_shared : fb_gu_routed; });
-        build_table(
-            tab_dn, E + 1, [&](int g) { return g == 0 ? T : tot[g - 1]; },
-            [&](int g) { return g == 0 ? 0 : soff[g - 1]; }, [&](int g) { return g == 0 ? E : g - 1; },
-            [&](int) { return fb_down; });
-    }
 }
 
 // Expert-ordered copy of the input rows, xp[inv[n]] = x[n / k] for each
@@ -424,9 +560,10 @@ __device__ __forceinline__ void put_row_vec(OT* orow, int c, uint4 v, const RowS
         reinterpret_cast<uint4*>(orow)[c] = cvt_row_vec(v, IT{}, OT{}, q.r);
 }
 
-// chunk_base (not null, after dispatch_kernel): inv[n] holds the entry's
-// rank inside its expert and chunk; its slot is chunk_base[chunk][idx[n]] +
-// inv[n], which this kernel writes back to inv[n] and records in perm.
+// chunk_base (not null, after dispatch_kernel or a dispatching router):
+// inv[n] holds the entry's rank inside its expert and chunk (chunk entries
+// per chunk); its slot is chunk_base[n / chunk][idx[n]] + inv[n], which this
+// kernel writes back to inv[n] and records in perm.
 // tokscale (8-bit weight layers; not null): each token's row scale (the
 // power-of-two f16 range scale, or the E4M3 scale when OT is uint8_t codes),
 // written once per token; gate_slot then carries gate * scale.
@@ -438,7 +575,8 @@ __global__ void __launch_bounds__(256) permute_rows_kernel(const IT* __restrict_
                                                            float* __restrict__ gate_slot,
                                                            OT* __restrict__ x_tok,
                                                            const int32_t* __restrict__ idx,
-                                                           const int32_t* __restrict__ chunk_base, int E,
+                                                           const int32_t* __restrict__ chunk_base, int chunk,
+                                                           int E,
                                                            int32_t* __restrict__ perm,
                                                            float* __restrict__ tokscale) {
     pdl_enter();
@@ -453,7 +591,7 @@ __global__ void __launch_bounds__(256) permute_rows_kernel(const IT* __restrict_
         if (chunk_base) {
             if (lane == 0) {
                 const int e = idx[n];
-                slot = (slot >= 0 && e >= 0 && e < E) ? chunk_base[(size_t)(n / kDispatchChunk) * E + e] + slot : -1;
+                slot = (slot >= 0 && e >= 0 && e < E) ? chunk_base[(size_t)(n / chunk) * E + e] + slot : -1;
                 if (slot >= 0 && slot < T * k) {
                     inv[n] = slot;
                     perm[slot] = n;
@@ -477,10 +615,18 @@ __global__ void __launch_bounds__(256) permute_rows_kernel(const IT* __restrict_
         }
         if (lane == 0 && gate_slot) gate_slot[slot] = gate[n] * sc;
         const RowScale q = row_scale(sc);
-        for (int i = lane; i < nv; i += 32) {
-            const uint4 v = s[i];
-            put_row_vec<IT, OT>(o, i, v, q);
-            if (ot) put_row_vec<IT, OT>(ot, i, v, q);
+        // four 16-byte loads per lane in flight before any store
+        for (int i0 = lane; i0 < nv; i0 += 4 * 32) {
+            uint4 v[4];
+#pragma unroll
+            for (int j = 0; j < 4; ++j)
+                if (i0 + 32 * j < nv) v[j] = s[i0 + 32 * j];
+#pragma unroll
+            for (int j = 0; j < 4; ++j) {
+                if (i0 + 32 * j >= nv) continue;
+                put_row_vec<IT, OT>(o, i0 + 32 * j, v[j], q);
+                if (ot) put_row_vec<IT, OT>(ot, i0 + 32 * j, v[j], q);
+            }
         }
     }
 }

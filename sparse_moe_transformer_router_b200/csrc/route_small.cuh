@@ -105,29 +105,32 @@ __global__ void __launch_bounds__(kSmallThreads) route_small_kernel(
             }
         }
         __syncthreads();
-        // thread -> (expert e, token group g); a group takes tokens g, g + G, ...
-        const int G = max(1, kSmallThreads / E);
-        const int e = tid % E, g = tid / E;
-        if (g < G && tid < G * E) {
+        // thread -> (expert e, token group g); a group takes tokens g, g + G,
+        // ... (jn of them).  The loop bounds are held in registers (in_reg):
+        // a kernel parameter read in the loop costs a constant-bank access
+        // per use.
+        const int nT = in_reg(T), nE = in_reg(E), nkn = in_reg(kn);
+        const int G = max(1, kSmallThreads / nE);
+        const int e = tid % nE, g = tid / nE;
+        if (g < G && tid < G * nE) {
+            const int jn = g < nT ? (nT - g + G - 1) / G : 0;  // tokens g + j * G < T
             float acc[kSmallMaxTokens];
 #pragma unroll
             for (int j = 0; j < kSmallMaxTokens; ++j) acc[j] = 0.f;
             const ET* wcol = ws + e;
+            const float* xg0 = xs + (size_t)g * kSmallSliceK;
+            const int xstep = G * kSmallSliceK;
 #pragma unroll 4
-            for (int kk = 0; kk < kn; ++kk) {
-                const float w = to_f32(wcol[kk * E]);
+            for (int kk = 0; kk < nkn; ++kk) {
+                const float w = to_f32(wcol[kk * nE]);
 #pragma unroll
-                for (int j = 0; j < kSmallMaxTokens; ++j) {
-                    const int t = g + j * G;
-                    if (t < T) acc[j] = fmaf(xs[t * kSmallSliceK + kk], w, acc[j]);
-                }
+                for (int j = 0; j < kSmallMaxTokens; ++j)
+                    if (j < jn) acc[j] = fmaf(xg0[j * xstep + kk], w, acc[j]);
             }
-            float* p = partial + (size_t)blockIdx.x * T * E;
+            float* p = partial + (size_t)blockIdx.x * nT * nE;
 #pragma unroll
-            for (int j = 0; j < kSmallMaxTokens; ++j) {
-                const int t = g + j * G;
-                if (t < T) p[(size_t)t * E + e] = acc[j];
-            }
+            for (int j = 0; j < kSmallMaxTokens; ++j)
+                if (j < jn) p[(size_t)(g + j * G) * nE + e] = acc[j];
         }
     }
     // the last CTA to get here finishes the routing
@@ -143,9 +146,10 @@ __global__ void __launch_bounds__(kSmallThreads) route_small_kernel(
     // of 8 slices for all of them are issued before any is added (one memory
     // round trip per 8 slices), and each output adds its slices in order
     float* lg = rs_smem;  // [T][E]
+    const int nT = in_reg(T), nE = in_reg(E), nk = in_reg(k);
     {
-        const int n = T * E;
-        const int S = (int)gridDim.x;
+        const int n = nT * nE;
+        const int S = in_reg((int)gridDim.x);
         for (int i0 = tid; i0 < n; i0 += 4 * kSmallThreads) {
             float v[4] = {0.f, 0.f, 0.f, 0.f};
             for (int s0 = 0; s0 < S; s0 += 8) {
@@ -165,7 +169,7 @@ __global__ void __launch_bounds__(kSmallThreads) route_small_kernel(
 #pragma unroll
             for (int q = 0; q < 4; ++q) {
                 const int i = i0 + kSmallThreads * q;
-                if (i < n) lg[i] = v[q] + (bias ? bias[i % E] : 0.f);
+                if (i < n) lg[i] = v[q] + (bias ? bias[i % nE] : 0.f);
             }
         }
     }
@@ -176,10 +180,10 @@ __global__ void __launch_bounds__(kSmallThreads) route_small_kernel(
     // each lane keeps the list of its experts (lane, lane + 32, ...: ascending,
     // so ties keep the lower index), then k + 1 butterfly rounds each take
     // the first head in (value, index) order
-    for (int t = warp; t < T; t += kSmallThreads / 32) {
+    for (int t = warp; t < nT; t += kSmallThreads / 32) {
         TopK tk;
         tk.init();
-        for (int e = lane; e < E; e += 32) tk.offer(lg[t * E + e], e);
+        for (int e = lane; e < nE; e += 32) tk.offer(lg[t * nE + e], e);
         TopK sel;
         sel.init();
         int pos = 0;
@@ -203,11 +207,11 @@ __global__ void __launch_bounds__(kSmallThreads) route_small_kernel(
             if (hl == lane && hi >= 0) ++pos;
         }
         if (lane == 0) {
-            sel.fill_empty(k);
+            sel.fill_empty(nk);
 #pragma unroll
             for (int j = 0; j < kMaxTopK; ++j) {
-                if (j < k) {
-                    const int n = t * k + j;
+                if (j < nk) {
+                    const int n = t * nk + j;
                     const float g = 1.0f / (1.0f + expf(-sel.value(j)));
                     idx[n] = sel.index(j);
                     lmax[n] = sel.value(j);
@@ -216,14 +220,14 @@ __global__ void __launch_bounds__(kSmallThreads) route_small_kernel(
                     s_gate[n] = g;
                 }
             }
-            margin[t] = sel.value(k - 1) - sel.value(k);
+            margin[t] = sel.value(nk - 1) - sel.value(nk);
         }
     }
-    for (int e = tid; e < E; e += kSmallThreads) s_rows[e] = 0;
+    for (int e = tid; e < nE; e += kSmallThreads) s_rows[e] = 0;
     // each token row's power-of-two scale into f16's range (8-bit weight
     // layers, f16_row_scale), one warp per token
-    const int nv = d * (int)sizeof(ET) / 16;
-    for (int t = warp; t < T; t += kSmallThreads / 32) {
+    const int nv = in_reg(d * (int)sizeof(ET) / 16);
+    for (int t = warp; t < nT; t += kSmallThreads / 32) {
         float sc = 1.0f;
         if constexpr (!std::is_same<ET, GT>::value) {
             float m = 0.0f;
@@ -238,7 +242,7 @@ __global__ void __launch_bounds__(kSmallThreads) route_small_kernel(
     __syncthreads();
 
     // ---------------------------------------------- ranks, counts, offsets (warp 0)
-    const int Tv = T * k;
+    const int Tv = nT * nk;
     if (warp == 0) {
         for (int c0 = 0; c0 < Tv; c0 += 32) {
             const int n = c0 + lane;
@@ -255,7 +259,7 @@ __global__ void __launch_bounds__(kSmallThreads) route_small_kernel(
 #pragma unroll
         for (int j = 0; j < 8; ++j) {
             const int e = lane * 8 + j;
-            local[j] = e < E ? s_rows[e] : 0;
+            local[j] = e < nE ? s_rows[e] : 0;
             sum += local[j];
         }
         const int incl = warp_incl_scan(sum);
@@ -263,7 +267,7 @@ __global__ void __launch_bounds__(kSmallThreads) route_small_kernel(
 #pragma unroll
         for (int j = 0; j < 8; ++j) {
             const int e = lane * 8 + j;
-            if (e < E) {
+            if (e < nE) {
                 s_off[e] = acc;
                 offsets[e] = acc;
                 counts[e] = local[j];
@@ -271,8 +275,8 @@ __global__ void __launch_bounds__(kSmallThreads) route_small_kernel(
             acc += local[j];
         }
         if (lane == 31) {
-            s_off[E] = incl;
-            offsets[E] = incl;
+            s_off[nE] = incl;
+            offsets[nE] = incl;
         }
     }
     __syncthreads();
@@ -280,28 +284,28 @@ __global__ void __launch_bounds__(kSmallThreads) route_small_kernel(
         const int slot = s_off[s_ent[n]] + s_rank[n];
         inv[n] = slot;
         perm[slot] = n;
-        gslot[slot] = s_gate[n] * s_scale[n / k];
+        gslot[slot] = s_gate[n] * s_scale[n / nk];
     }
     if (warp == 0) {
         // gate/up: candidate 0 is the shared expert, 1..E the routed experts
         build_table(
-            tab_gu, E + 1, [&](int g) { return g == 0 ? T : s_rows[g - 1]; },
-            [&](int g) { return g == 0 ? 0 : s_off[g - 1]; }, [&](int g) { return g == 0 ? E : g - 1; },
+            tab_gu, nE + 1, [&](int g) { return g == 0 ? nT : s_rows[g - 1]; },
+            [&](int g) { return g == 0 ? 0 : s_off[g - 1]; }, [&](int g) { return g == 0 ? nE : g - 1; },
             [&](int g) { return g == 0 ? fb_gu_shared : fb_gu_routed; });
         build_table(
-            tab_dn, E + 1, [&](int g) { return g == 0 ? T : s_rows[g - 1]; },
-            [&](int g) { return g == 0 ? 0 : s_off[g - 1]; }, [&](int g) { return g == 0 ? E : g - 1; },
+            tab_dn, nE + 1, [&](int g) { return g == 0 ? nT : s_rows[g - 1]; },
+            [&](int g) { return g == 0 ? 0 : s_off[g - 1]; }, [&](int g) { return g == 0 ? nE : g - 1; },
             [&](int) { return fb_down; });
     }
 
     // ---------------------------------------------- rows in expert order
     // xg[slot of n] = x[n / k] (16-byte vectors, converted for 8-bit weight
     // layers), and x16[t] = x[t] in token order when it is given
-    const int rows = Tv + (x16 ? T : 0);
+    const int rows = Tv + (x16 ? nT : 0);
     for (int i = tid; i < rows * nv; i += kSmallThreads) {
         const int r = i / nv, c = i - r * nv;
         const bool tok = r >= Tv;
-        const int t = tok ? r - Tv : r / k;
+        const int t = tok ? r - Tv : r / nk;
         const int orow = tok ? t : s_off[s_ent[r]] + s_rank[r];
         put_row_vec<ET, GT>((tok ? x16 : xg) + (size_t)orow * d, c,
                             reinterpret_cast<const uint4*>(x + (size_t)t * d)[c], row_scale(s_scale[t]));

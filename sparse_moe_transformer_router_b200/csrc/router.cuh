@@ -22,6 +22,7 @@
 #include <cuda_bf16.h>
 #include <cstdint>
 
+#include "permute.cuh"
 #include "ptx.cuh"
 #include "topk.cuh"
 
@@ -203,57 +204,127 @@ __global__ void __launch_bounds__(NT) router_kernel(const ET* __restrict__ x,
 // sigmoid rule as the CUDA-core router above.  Warp 0 lane 0 issues the TMA
 // loads, warp 1 lane 0 the MMAs; all four warps run the epilogue.
 namespace rmma {
-constexpr int STAGES = 4;
 constexpr int A_BYTES = 128 * 128;     // 128 tokens x 64 K (bf16)
 constexpr int B_BOX_BYTES = 64 * 128;  // 64 K rows x 64 experts (bf16)
 constexpr int MAX_B_BOXES = 4;         // E <= 256
-constexpr int STAGE_BYTES = A_BYTES + MAX_B_BOXES * B_BOX_BYTES;
-constexpr size_t SMEM_BYTES = 1024 + (size_t)STAGES * STAGE_BYTES + (2 * STAGES + 1) * 8 + 16;
+constexpr int MAX_STAGES = 6;
+// The largest dynamic shared memory a launch asks for (stages, barriers, slack).
+constexpr size_t SMEM_BYTES = 226 * 1024;
 // A launch whose CTAs each take n_chunk experts needs stages of the token
 // tile plus ceil(n_chunk / 64) weight boxes only: fewer bytes, so that two
 // CTAs fit on an SM when the experts are few.
 __host__ __device__ constexpr int stage_bytes(int n_chunk) {
     return A_BYTES + ((n_chunk + 63) / 64) * B_BOX_BYTES;
 }
-__host__ __device__ constexpr size_t smem_bytes(int n_chunk) {
-    return 1024 + (size_t)STAGES * stage_bytes(n_chunk) + (2 * STAGES + 1) * 8 + 16;
+__host__ __device__ constexpr size_t smem_bytes(int n_chunk, int nst) {
+    return 1024 + (size_t)nst * stage_bytes(n_chunk) + (2 * nst + 1) * 8 + 16;
+}
+// Stages of a launch: 4 when two CTAs then share an SM (each at most half of
+// its shared memory), else as many as one CTA's shared memory holds, up to
+// MAX_STAGES -- the bytes in flight per SM are what keep the x stream at the
+// HBM rate.
+__host__ __device__ constexpr int stages(int n_chunk) {
+    return smem_bytes(n_chunk, 4) <= 112 * 1024 ? 4
+           : (int)((SMEM_BYTES - 1024 - 16 - 8) / (stage_bytes(n_chunk) + 16)) < MAX_STAGES
+               ? (int)((SMEM_BYTES - 1024 - 16 - 8) / (stage_bytes(n_chunk) + 16))
+               : MAX_STAGES;
 }
 }  // namespace rmma
 
-// Cluster K-split (gridDim.z = S > 1, launched as clusters of (1, 1, S)):
-// CTA z of a cluster computes the partial logits of
-// the same 128 tokens over K slice z and keeps them in its shared memory;
-// after a cluster barrier rank 0 adds ranks 1..S-1's partials to its own in
-// slice order (deterministic) and runs the arg-max epilogue.  This spreads
-// the x stream of a batch of few token tiles over S times more SMs.
-// Each CTA's partial (fp32, row-major [128 tokens][n_pad + 4], at most
-// 130 KB for E = 256) reuses its own operand stages; rank 0 reads a token's
-// row from each other rank with 16-byte loads issued before any is used.
+// The dispatch a top-1 router launch may finish itself (chunk_base not
+// null): the tokens each CTA finishes (tokens_per_cta of one 128-token tile,
+// below) form a dispatch chunk whose stable ranks go to inv[t] and whose
+// per-expert counts go to chunk_base[chunk][E]; the last CTA to finish
+// (atomic ticket after a memory fence, no waiting) writes the chunk bases,
+// counts, offsets and the two work lists (dispatch_finish) and resets the
+// ticket.  The outputs are those of dispatch_kernel with chunks of
+// tokens_per_cta entries.
+struct RouterDispatch {
+    int32_t* chunk_base;  // [chunks][E]
+    int32_t* counts;      // [E]
+    int32_t* offsets;     // [E + 1]
+    int32_t* inv;         // [T]: rank inside (chunk, expert)
+    GroupTable* tab_gu;
+    GroupTable* tab_dn;
+    unsigned* ticket;     // zero between launches
+    int fb_gu_routed, fb_gu_shared, fb_down;
+};
+
+// Tokens of a tile that each CTA of a K-split launch (S slices) finishes.
+__host__ __device__ constexpr int router_tokens_per_cta(int S) { return 128 / S; }
+
+// Ints of a dispatching router CTA's stage memory left for the staging of
+// the last CTA's scan (after tot and soff); the launch dispatches only when
+// its chunks fit (a row of E per chunk, or at least one column).
+__host__ __device__ constexpr int router_stage_cap(int E) {
+    return (int)((size_t)rmma::stages(E) * rmma::stage_bytes(E) / 4) - ((2 * E + 1 + 3) & ~3);
+}
+
+// A kernel parameter copied into a register the compiler cannot re-derive:
+// the epilogue's loops otherwise re-read such scalars from the constant
+// bank on every element, which costs tens of cycles each.
+__device__ __forceinline__ int in_reg(int v) {
+    int r;
+    asm volatile("mov.b32 %0, %1;" : "=r"(r) : "r"(v));
+    return r;
+}
+
+__device__ __forceinline__ void cluster_arrive_release() {
+    asm volatile("barrier.cluster.arrive.release;" ::: "memory");
+}
+__device__ __forceinline__ void cluster_wait_acquire() {
+    asm volatile("barrier.cluster.wait.acquire;" ::: "memory");
+}
+// 16 bytes to a shared::cluster address (this or another CTA of the cluster).
+__device__ __forceinline__ void st_shared_cluster_v4(uint32_t addr, float a, float b, float c, float d) {
+    asm volatile("st.shared::cluster.v4.f32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "f"(a), "f"(b), "f"(c),
+                 "f"(d)
+                 : "memory");
+}
+// 16 bytes to this CTA's shared memory.
+__device__ __forceinline__ void st_shared_v4(uint32_t addr, float a, float b, float c, float d) {
+    asm volatile("st.shared.v4.f32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "f"(a), "f"(b), "f"(c), "f"(d)
+                 : "memory");
+}
+
+// K split (gridDim.z = S slices, S a power of two <= 8, launched as clusters
+// of (1, 1, S) when S > 1): CTA z of a cluster computes the partial logits
+// of the same 128 tokens over K slice z.  The slices then meet in the CTA
+// that finishes each token: CTA z owns the tile's tokens [z * 128 / S,
+// (z + 1) * 128 / S).  After a cluster barrier (every CTA's operand stages
+// are idle), each thread stores its token row's partial (TMEM lane = token)
+// into the owner's shared memory, slot z: recv[S][128 / S][n_pad + 4] fp32;
+// a second barrier (release / acquire) makes the rows visible.  The owner's
+// S consecutive lanes per token each sum a 1/S share of the experts over the
+// slices in order 0 .. S-1 (deterministic), then merge their arg-max (or
+// top-k) with shuffles.  With S = 1 the same exchange runs inside the CTA.
+// This spreads the x stream of a batch of few token tiles over S times more
+// SMs and keeps the reduction parallel: no CTA waits on remote loads.
 //
 // Expert-split mode (logits != null, for batches of one token tile): CTA
 // (y, z) computes experts [y*n_chunk, (y+1)*n_chunk) over K slice z of
-// gridDim.z; the slices meet in rank 0 of their cluster as above, which
-// stores the biased fp32 logits to logits[T][E]; the arg-max then runs in
-// the permutation kernel.  This spreads the router weight stream over
-// (E / n_chunk) x slices SMs instead of one.
+// gridDim.z; the slices meet as above and the owners store the biased fp32
+// logits to logits[T][E]; the arg-max then runs in the permutation kernel.
+// This spreads the router weight stream over (E / n_chunk) x slices SMs
+// instead of one.
 __global__ void __launch_bounds__(128, 2)
     router_mma_kernel(const __grid_constant__ CUtensorMap x_map, const __grid_constant__ CUtensorMap wr_map,
                       const float* __restrict__ bias, int T, int d, int E, int n_chunk,
                       float* __restrict__ logits, int32_t* __restrict__ idx,
                       float* __restrict__ gate, float* __restrict__ lmax,
-                      float* __restrict__ margin, unsigned* err, int topk) {
-    pdl_enter();
+                      float* __restrict__ margin, unsigned* err, int topk, int nst, const RouterDispatch dsp) {
     extern __shared__ uint8_t rsmem_raw[];
+    __shared__ unsigned s_last;
     uint8_t* smem = reinterpret_cast<uint8_t*>(
         (reinterpret_cast<uintptr_t>(rsmem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
     const int stage_bytes = rmma::stage_bytes(n_chunk);  // this launch's stage stride
-    uint64_t* bars = reinterpret_cast<uint64_t*>(smem + (size_t)rmma::STAGES * stage_bytes);
-    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 2 * rmma::STAGES + 1);
+    uint64_t* bars = reinterpret_cast<uint64_t*>(smem + (size_t)nst * stage_bytes);  // nst stages
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 2 * nst + 1);
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const uint32_t stage0 = smem_u32(smem), bar0 = smem_u32(bars);
     auto full_bar = [&](int s) { return bar0 + 8u * s; };
-    auto empty_bar = [&](int s) { return bar0 + 8u * (rmma::STAGES + s); };
-    const uint32_t done_bar = bar0 + 8u * (2 * rmma::STAGES);
+    auto empty_bar = [&](int s) { return bar0 + 8u * (nst + s); };
+    const uint32_t done_bar = bar0 + 8u * (2 * nst);
     const int e0 = blockIdx.y * n_chunk;        // first expert of this CTA
     const int ne = min(n_chunk, E - e0);         // experts of this CTA
     const int n_pad = (ne + 15) & ~15;
@@ -261,14 +332,18 @@ __global__ void __launch_bounds__(128, 2)
     uint32_t ncols = 32;
     while ((int)ncols < n_pad) ncols <<= 1;
 
+    // set-up that touches no input: before the wait on the preceding kernel
     if (threadIdx.x == 0) {
-        for (int s = 0; s < rmma::STAGES; ++s) {
+        for (int s = 0; s < nst; ++s) {
             mbar_init(full_bar(s), 1);
             mbar_init(empty_bar(s), 1);
         }
         mbar_init(done_bar, 1);
         fence_barrier_init();
+        tma_prefetch_desc(&x_map);
+        tma_prefetch_desc(&wr_map);
     }
+    pdl_enter();
     if (warp == 1) {
         tmem_alloc(smem_u32(tmem_slot), ncols);
         tmem_relinquish();
@@ -298,12 +373,12 @@ __global__ void __launch_bounds__(128, 2)
                             kg);
             used |= 1u << stage;
             last_par = (last_par & ~(1u << stage)) | (phase << stage);
-            if (++stage == rmma::STAGES) {
+            if (++stage == nst) {
                 stage = 0;
                 phase ^= 1u;
             }
         }
-        for (int s = 0; s < rmma::STAGES; ++s)  // drain copies in flight
+        for (int s = 0; s < nst; ++s)  // drain copies in flight
             if (used & (1u << s)) mbar_wait(full_bar(s), (last_par >> s) & 1u, err, DEV_ERR_TIMEOUT_PRODUCER);
     } else if (warp == 1 && lane == 0) {
         int stage = 0;
@@ -320,7 +395,7 @@ __global__ void __launch_bounds__(128, 2)
                 mma_bf16(tmem_base, adesc, bdesc, idesc, (kb | kk) != 0 ? 1u : 0u);
             }
             mma_commit(empty_bar(stage));
-            if (++stage == rmma::STAGES) {
+            if (++stage == nst) {
                 stage = 0;
                 phase ^= 1u;
             }
@@ -328,117 +403,194 @@ __global__ void __launch_bounds__(128, 2)
         mma_commit(done_bar);  // logits complete (or every issued MMA finished)
     }
     __syncwarp();
-    // epilogue: thread = token row (TMEM lane 32*warp + lane)
     const bool ok = mbar_wait(done_bar, 0, err, DEV_ERR_TIMEOUT_EPILOGUE);
-    const bool kreduce = gridDim.z > 1;  // K slices: always launched as clusters along z
-    const uint32_t crank = kreduce ? cluster_ctarank() : 0u;
-    float* red = reinterpret_cast<float*>(smem);  // this CTA's partial, [128][n_pad + 4] (row-major)
-    // K-slice partials of ranks 1..S-1: row-major [128 tokens][rld] fp32 in
-    // each CTA's own (now idle) stage memory, one row per thread, so rank 0
-    // reads a row with 16-byte cluster loads, all issued before they are used
-    const int rld = n_pad + 4;
-    if (kreduce) {
-        // every CTA reaches both cluster barriers, whatever its waits gave
-        if (crank != 0 && __all_sync(0xffffffffu, ok)) {
-            tc_fence_after();
-            float* row = red + (size_t)(32 * warp + lane) * rld;
-            for (int c = 0; c < n_pad; c += 32) {
-                float v[32];
-                tmem_ld_32x32(tmem_base + ((uint32_t)(32 * warp) << 16) + (uint32_t)c, v);
-                tmem_wait_ld();
-#pragma unroll
-                for (int i = 0; i < 32; i += 4)
-                    if (c + i < n_pad)
-                        *reinterpret_cast<float4*>(row + c + i) = make_float4(v[i], v[i + 1], v[i + 2], v[i + 3]);
-            }
-        }
-        cluster_sync();  // partials of ranks 1..S-1 complete in their shared memory
-    }
-    // the logits of this thread's token, 32 experts at a time: own partial,
-    // then slices 1..S-1 in order (a fixed order: deterministic)
-    auto logits_chunk = [&](int c, float (&v)[32]) {
-        tmem_ld_32x32(tmem_base + ((uint32_t)(32 * warp) << 16) + (uint32_t)c, v);
-        tmem_wait_ld();
-        for (uint32_t z = 1; kreduce && z < gridDim.z; ++z) {
-            const uint32_t base = mapa_shared(smem_u32(red + (size_t)(32 * warp + lane) * rld + c), z);
-            float4 r[8];
-#pragma unroll
-            for (int q = 0; q < 8; ++q)
-                r[q] = (c + 4 * q < n_pad) ? ld_shared_cluster_v4(base + 16u * q) : make_float4(0.f, 0.f, 0.f, 0.f);
+    const bool all_ok = __syncthreads_and(ok) != 0;  // CTA-uniform from here on
+
+    // ---- the slices meet in the CTA that owns each token (see above)
+    const int S = in_reg((int)gridDim.z);
+    const uint32_t z = S > 1 ? cluster_ctarank() : 0u;
+    const int tpc = router_tokens_per_cta(S);
+    const int rld = n_pad + 4;                           // recv row stride (floats)
+    float* recv = reinterpret_cast<float*>(smem);        // [S][tpc][rld] in the idle stages
+    const int row = 32 * warp + lane;                    // this thread's token row (TMEM lane)
+    const uint32_t dst_local = smem_u32(recv + ((size_t)z * tpc + row % tpc) * rld);
+    if (S > 1) cluster_arrive_release();  // this CTA's stages are idle: the others may write them
+    const uint32_t dst = S > 1 ? mapa_shared(dst_local, (uint32_t)(row / tpc)) : dst_local;
+    if (S > 1) cluster_wait_acquire();
+    if (all_ok) {
+        tc_fence_after();
+        for (int c = 0; c < n_pad; c += 32) {
+            float v[32];
+            tmem_ld_32x32(tmem_base + ((uint32_t)(32 * warp) << 16) + (uint32_t)c, v);
+            tmem_wait_ld();
 #pragma unroll
             for (int q = 0; q < 8; ++q) {
-                v[4 * q] += r[q].x;
-                v[4 * q + 1] += r[q].y;
-                v[4 * q + 2] += r[q].z;
-                v[4 * q + 3] += r[q].w;
+                if (c + 4 * q >= n_pad) continue;
+                const uint32_t a = dst + 4u * (uint32_t)(c + 4 * q);
+                if (S > 1) st_shared_cluster_v4(a, v[4 * q], v[4 * q + 1], v[4 * q + 2], v[4 * q + 3]);
+                else st_shared_v4(a, v[4 * q], v[4 * q + 1], v[4 * q + 2], v[4 * q + 3]);
             }
         }
+    }
+    if (S > 1) {
+        cluster_arrive_release();  // every row stored ...
+        cluster_wait_acquire();    // ... and visible to its owner
+    } else {
+        __syncthreads();
+    }
+
+    // ---- this CTA's tokens: S consecutive lanes per token, lane `sub` takes
+    // experts [sub * ne / S, (sub + 1) * ne / S) of the CTA's ne (S divides ne)
+    const int nE = in_reg(E), nT = in_reg(T), nK = in_reg(topk);
+    const bool has_bias = bias != nullptr;
+    const int rl = threadIdx.x / S, sub = threadIdx.x - rl * S;
+    const int t = t0 + (int)z * tpc + rl;
+    const int per = in_reg(ne / S);
+    const int eb = sub * per;
+    const int rld_r = in_reg(rld);
+    const float* rrow = recv + (size_t)rl * rld_r;           // slot 0 of this token's rows
+    const size_t slot_stride = (size_t)tpc * rld_r;
+    auto logit = [&](int e) {  // sum over the slices in order, then the bias
+        float p[8];
+#pragma unroll
+        for (int s = 0; s < 8; ++s) p[s] = s < S ? rrow[s * slot_stride + e] : 0.f;  // loads first
+        float l = 0.f;
+#pragma unroll
+        for (int s = 0; s < 8; ++s)
+            if (s < S) l += p[s];
+        return has_bias ? l + bias[e0 + e] : l;
     };
-    if ((!kreduce || crank == 0) && __all_sync(0xffffffffu, ok)) {
-        tc_fence_after();
-        const int t = t0 + 32 * warp + lane;
+    int e_tok = -1;  // top-1: the token's expert in its lane sub == 0 (-1 past T or on failure)
+    if (all_ok) {
         if (logits) {
-            for (int c = 0; c < n_pad; c += 32) {
-                float v[32];
-                logits_chunk(c, v);
-#pragma unroll
-                for (int i = 0; i < 32; ++i) {
-                    const int e = c + i;
-                    if (e < ne && t < T) logits[(size_t)t * E + e0 + e] = v[i] + (bias ? bias[e0 + e] : 0.f);
-                }
-            }
-        } else if (topk == 1) {
-            // the arg-max (strict ">" in ascending order: the lowest index
-            // among the maxima; NaN never wins) and the runner-up, branch-free
+            for (int e = eb; e < eb + per; ++e)
+                if (t < nT) logits[(size_t)t * nE + e0 + e] = logit(e);
+        } else if (nK == 1) {
+            // this lane's share: the arg-max (strict ">" in ascending order:
+            // the lowest index among the maxima; NaN never wins) and the
+            // runner-up, branch-free
             float best = -INFINITY, second = -INFINITY;
-            int bi = 0;
-            for (int c = 0; c < n_pad; c += 32) {
-                float v[32];
-                logits_chunk(c, v);
+            int bi = eb;
+            auto offer = [&](float l, int e) {
+                const bool gt = l > best;
+                second = gt ? best : fmaxf(second, l);
+                bi = gt ? e : bi;
+                best = gt ? l : best;
+            };
+            if ((per & 3) == 0) {  // four experts per step: 16-byte loads of every slice first
+                for (int e = eb; e < eb + per; e += 4) {
+                    float4 p[8];
 #pragma unroll
-                for (int i = 0; i < 32; ++i) {
-                    const int e = c + i;
-                    const float l = e < E ? v[i] + (bias ? bias[e] : 0.f) : -INFINITY;
-                    const bool gt = l > best;
-                    second = gt ? best : fmaxf(second, l);
-                    bi = gt ? e : bi;
-                    best = gt ? l : best;
+                    for (int s = 0; s < 8; ++s)
+                        p[s] = s < S ? *reinterpret_cast<const float4*>(rrow + s * slot_stride + e)
+                                     : make_float4(0.f, 0.f, 0.f, 0.f);
+                    float4 l = make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll
+                    for (int s = 0; s < 8; ++s) {
+                        if (s >= S) continue;
+                        l.x += p[s].x;
+                        l.y += p[s].y;
+                        l.z += p[s].z;
+                        l.w += p[s].w;
+                    }
+                    if (has_bias) {
+                        l.x += bias[e0 + e];
+                        l.y += bias[e0 + e + 1];
+                        l.z += bias[e0 + e + 2];
+                        l.w += bias[e0 + e + 3];
+                    }
+                    offer(l.x, e);
+                    offer(l.y, e + 1);
+                    offer(l.z, e + 2);
+                    offer(l.w, e + 3);
                 }
+            } else {
+#pragma unroll 4
+                for (int e = eb; e < eb + per; ++e) offer(logit(e), e);
             }
-            if (t < T) {
+            // merge the token's S shares: larger value first, then lower index
+            for (int off = S >> 1; off > 0; off >>= 1) {
+                const float ob = __shfl_xor_sync(0xffffffffu, best, off);
+                const float os = __shfl_xor_sync(0xffffffffu, second, off);
+                const int oi = __shfl_xor_sync(0xffffffffu, bi, off);
+                const bool take = ob > best || (ob == best && oi < bi);
+                second = fmaxf(fmaxf(second, os), take ? best : ob);
+                bi = take ? oi : bi;
+                best = take ? ob : best;
+            }
+            if (sub == 0 && t < nT) {
                 idx[t] = bi;
                 lmax[t] = best;
                 gate[t] = 1.0f / (1.0f + expf(-best));
                 margin[t] = best - second;
+                e_tok = bi;
             }
         } else {
             TopK tk;
             tk.init();
-            for (int c = 0; c < n_pad; c += 32) {
-                float v[32];
-                logits_chunk(c, v);
+            for (int e = eb; e < eb + per; ++e) tk.offer(logit(e), e);
+            // the token's S lists (consecutive lanes): k + 1 heads in selection order
+            TopK sel;
+            sel.init();
+            int pos = 0;  // entries of this lane's list already taken
 #pragma unroll
-                for (int i = 0; i < 32; ++i) {
-                    const int e = c + i;
-                    if (e < E) tk.offer(v[i] + (bias ? bias[e] : 0.f), e);
-                }
-            }
-            if (t < T) {
-                tk.fill_empty(topk);
-#pragma unroll
-                for (int j = 0; j < kMaxTopK; ++j) {
-                    if (j < topk) {
-                        const size_t n = (size_t)t * topk + j;
-                        idx[n] = tk.index(j);
-                        lmax[n] = tk.value(j);
-                        gate[n] = 1.0f / (1.0f + expf(-tk.value(j)));
+            for (int j = 0; j <= kMaxTopK; ++j) {
+                float hv = tk.value(pos);
+                int hi = pos <= kMaxTopK ? tk.index(pos) : -1;
+                int hl = sub;
+                for (int off = S >> 1; off > 0; off >>= 1) {
+                    const float ov = __shfl_xor_sync(0xffffffffu, hv, off);
+                    const int oi = __shfl_xor_sync(0xffffffffu, hi, off);
+                    const int ol = __shfl_xor_sync(0xffffffffu, hl, off);
+                    if (topk_before(ov, oi, hv, hi)) {
+                        hv = ov;
+                        hi = oi;
+                        hl = ol;
                     }
                 }
-                margin[t] = tk.value(topk - 1) - tk.value(topk);  // k-th against the next one
+                sel.set(j, hv, hi);
+                if (hl == sub && hi >= 0) ++pos;
+            }
+            if (sub == 0 && t < nT) {
+                sel.fill_empty(nK);
+#pragma unroll
+                for (int j = 0; j < kMaxTopK; ++j) {
+                    if (j < nK) {
+                        const size_t n = (size_t)t * nK + j;
+                        idx[n] = sel.index(j);
+                        lmax[n] = sel.value(j);
+                        gate[n] = 1.0f / (1.0f + expf(-sel.value(j)));
+                    }
+                }
+                margin[t] = sel.value(nK - 1) - sel.value(nK);  // k-th against the next one
             }
         }
     }
-    if (kreduce) cluster_sync();  // rank 0 done reading the others' shared memory
+
+    if (dsp.chunk_base) {
+        // this CTA's tokens are one dispatch chunk; the ranks' counts follow
+        // recv, and the last CTA's scan reuses the whole stage memory (recv
+        // and wcnt are idle by then)
+        int* wcnt = reinterpret_cast<int*>(recv + (size_t)S * slot_stride);  // [4][E]
+        int* tot = reinterpret_cast<int*>(smem);
+        int* soff = tot + nE;
+        int* stage = tot + ((2 * nE + 1 + 3) & ~3);  // 16-byte aligned
+        const int chunk = blockIdx.x * S + (int)z;
+        const int r = chunk_rank(e_tok, nE, wcnt, dsp.chunk_base + (size_t)chunk * nE);
+        if (sub == 0 && t < nT) dsp.inv[t] = r;
+        __threadfence();
+        __syncthreads();
+        const unsigned ctas = gridDim.x * (unsigned)S;
+        if (threadIdx.x == 0) s_last = (atomicAdd(dsp.ticket, 1u) == ctas - 1u) ? 1u : 0u;
+        __syncthreads();
+        if (s_last) {
+            __threadfence();
+            const int cap = router_stage_cap(nE);  // >= the chunks (the host dispatches here only then)
+            dispatch_finish<8>(dsp.chunk_base, (int)ctas, nT, nE, dsp.fb_gu_routed, dsp.fb_gu_shared, dsp.fb_down,
+                               dsp.counts, dsp.offsets, dsp.tab_gu, dsp.tab_dn, tot, soff, stage, cap);
+            if (threadIdx.x == 0) *dsp.ticket = 0u;
+        }
+    }
     tc_fence_before();
     __syncthreads();
     if (warp == 1) {

@@ -65,8 +65,8 @@ bool check(const l4moe_params& p, int Tmax, int k, int sms, bool act8 = false) {
     const size_t slices = (d + kSmallSliceK - 1) / kSmallSliceK;
     if (E && size_of(L.logits) < 4 * slices * std::min<size_t>(t, kSmallMaxTokens) * E)
         return fail_case("small-batch partial logits too small", p, Tmax, k, sms);
-    // the dispatch's chunk bases [chunks][E]
-    if (E && size_of(L.chunk) < 4 * ((tv + kDispatchChunk - 1) / kDispatchChunk) * E)
+    // the dispatch chunk bases [chunks][E]: up to 8 chunks per 128-token tile (the router's)
+    if (E && size_of(L.chunk) < 4 * 8 * ((tv + 127) / 128) * E)
         return fail_case("dispatch chunk bases too small", p, Tmax, k, sms);
     if (L.xout + 2 * t * d * a > L.total || L.xin + 2 * t * d * a > L.xout)
         return fail_case("host staging too small", p, Tmax, k, sms);
