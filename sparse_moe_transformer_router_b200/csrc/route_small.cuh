@@ -89,19 +89,45 @@ __global__ void __launch_bounds__(kSmallThreads) route_small_kernel(
             const int nw = kn * E;  // E * sizeof(ET) need not be a multiple of 16: copy the flat range
             const ET* src = Wr + (size_t)k0 * E;
             const bool vec = ((reinterpret_cast<uintptr_t>(src) & 15u) == 0) && (nw % V == 0);
+            // each thread's loads of a pass are issued before any store (one
+            // memory round trip per pass, not per vector)
             if (vec) {
-                for (int i = tid; i < nw / V; i += kSmallThreads)
-                    reinterpret_cast<uint4*>(ws)[i] = reinterpret_cast<const uint4*>(src)[i];
+                const int nv16 = nw / V;
+                for (int i0 = tid; i0 < nv16; i0 += 8 * kSmallThreads) {
+                    uint4 v[8];
+#pragma unroll
+                    for (int j = 0; j < 8; ++j)
+                        if (i0 + j * kSmallThreads < nv16)
+                            v[j] = reinterpret_cast<const uint4*>(src)[i0 + j * kSmallThreads];
+#pragma unroll
+                    for (int j = 0; j < 8; ++j)
+                        if (i0 + j * kSmallThreads < nv16) reinterpret_cast<uint4*>(ws)[i0 + j * kSmallThreads] = v[j];
+                }
             } else {
                 for (int i = tid; i < nw; i += kSmallThreads) ws[i] = src[i];
             }
             const int xv = kn / V;  // x rows: kn elements from k0 (k0, kn multiples of 64)
-            for (int i = tid; i < T * xv; i += kSmallThreads) {
-                const int t = i / xv, c = i - t * xv;
-                ET tmp[16 / sizeof(ET)];
-                *reinterpret_cast<uint4*>(tmp) = reinterpret_cast<const uint4*>(x + (size_t)t * d + k0)[c];
+            const int nxv = T * xv;
+            for (int i0 = tid; i0 < nxv; i0 += 4 * kSmallThreads) {
+                uint4 raw[4];
 #pragma unroll
-                for (int u = 0; u < V; ++u) xs[t * kSmallSliceK + c * V + u] = to_f32(tmp[u]);
+                for (int j = 0; j < 4; ++j) {
+                    const int i = i0 + j * kSmallThreads;
+                    if (i < nxv) {
+                        const int t = i / xv, c = i - t * xv;
+                        raw[j] = reinterpret_cast<const uint4*>(x + (size_t)t * d + k0)[c];
+                    }
+                }
+#pragma unroll
+                for (int j = 0; j < 4; ++j) {
+                    const int i = i0 + j * kSmallThreads;
+                    if (i >= nxv) continue;
+                    const int t = i / xv, c = i - t * xv;
+                    ET tmp[16 / sizeof(ET)];
+                    *reinterpret_cast<uint4*>(tmp) = raw[j];
+#pragma unroll
+                    for (int u = 0; u < V; ++u) xs[t * kSmallSliceK + c * V + u] = to_f32(tmp[u]);
+                }
             }
         }
         __syncthreads();
@@ -144,13 +170,29 @@ __global__ void __launch_bounds__(kSmallThreads) route_small_kernel(
     // ---------------------------------------------- logits: slices in order, + bias
     // each pass covers up to 4 outputs per thread (i = i0 + 256 q); the loads
     // of 8 slices for all of them are issued before any is added (one memory
-    // round trip per 8 slices), and each output adds its slices in order
+    // round trip per 8 slices; 16 when a thread has one output), and each
+    // output adds its slices in order
     float* lg = rs_smem;  // [T][E]
     const int nT = in_reg(T), nE = in_reg(E), nk = in_reg(k);
     {
         const int n = nT * nE;
         const int S = in_reg((int)gridDim.x);
-        for (int i0 = tid; i0 < n; i0 += 4 * kSmallThreads) {
+        if (n <= kSmallThreads) {  // one output per thread: 16 slices per round trip
+            if (tid < n) {
+                float v = 0.f;
+                for (int s0 = 0; s0 < S; s0 += 16) {
+                    float ld[16];
+#pragma unroll
+                    for (int u = 0; u < 16; ++u)
+                        ld[u] = s0 + u < S ? __ldcg(partial + (size_t)(s0 + u) * n + tid) : 0.f;
+#pragma unroll
+                    for (int u = 0; u < 16; ++u)
+                        if (s0 + u < S) v += ld[u];
+                }
+                lg[tid] = v + (bias ? bias[tid % nE] : 0.f);
+            }
+        }
+        for (int i0 = tid; n > kSmallThreads && i0 < n; i0 += 4 * kSmallThreads) {
             float v[4] = {0.f, 0.f, 0.f, 0.f};
             for (int s0 = 0; s0 < S; s0 += 8) {
                 float ld[8][4];
@@ -302,13 +344,27 @@ __global__ void __launch_bounds__(kSmallThreads) route_small_kernel(
     // xg[slot of n] = x[n / k] (16-byte vectors, converted for 8-bit weight
     // layers), and x16[t] = x[t] in token order when it is given
     const int rows = Tv + (x16 ? nT : 0);
-    for (int i = tid; i < rows * nv; i += kSmallThreads) {
-        const int r = i / nv, c = i - r * nv;
-        const bool tok = r >= Tv;
-        const int t = tok ? r - Tv : r / nk;
-        const int orow = tok ? t : s_off[s_ent[r]] + s_rank[r];
-        put_row_vec<ET, GT>((tok ? x16 : xg) + (size_t)orow * d, c,
-                            reinterpret_cast<const uint4*>(x + (size_t)t * d)[c], row_scale(s_scale[t]));
+    for (int i0 = tid; i0 < rows * nv; i0 += 4 * kSmallThreads) {
+        uint4 raw[4];  // four 16-byte loads in flight before the stores
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+            const int i = i0 + j * kSmallThreads;
+            if (i < rows * nv) {
+                const int r = i / nv, c = i - r * nv;
+                const int t = r >= Tv ? r - Tv : r / nk;
+                raw[j] = reinterpret_cast<const uint4*>(x + (size_t)t * d)[c];
+            }
+        }
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+            const int i = i0 + j * kSmallThreads;
+            if (i >= rows * nv) continue;
+            const int r = i / nv, c = i - r * nv;
+            const bool tok = r >= Tv;
+            const int t = tok ? r - Tv : r / nk;
+            const int orow = tok ? t : s_off[s_ent[r]] + s_rank[r];
+            put_row_vec<ET, GT>((tok ? x16 : xg) + (size_t)orow * d, c, raw[j], row_scale(s_scale[t]));
+        }
     }
 }
 
