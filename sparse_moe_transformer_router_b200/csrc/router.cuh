@@ -196,13 +196,13 @@ __global__ void __launch_bounds__(NT) router_kernel(const ET* __restrict__ x,
 // ---------------------------------------------------------------------------
 // Tensor-core router for bf16 layers with E % 8 == 0 (E <= 256), top-k
 // (k = topk <= kMaxTopK; idx, gate, lmax hold [T][k], margin [T] is the k-th
-// selected logit minus the next one): one CTA per
-// 128-token tile computes the fp32 logits of all E experts with tcgen05 (M =
-// 128 tokens, N = E rounded up to 16, K = d; x rows are the K-major A
-// operand, W_router [d, E] the MN-major B operand), then each of 128 threads
-// owns one token's logits in TMEM and applies the same arg-max / runner-up /
-// sigmoid rule as the CUDA-core router above.  Warp 0 lane 0 issues the TMA
-// loads, warp 1 lane 0 the MMAs; all four warps run the epilogue.
+// selected logit minus the next one): the CTAs of a 128-token tile compute
+// the fp32 logits of all E experts with tcgen05 (M = 128 tokens, N = E
+// rounded up to 16, K = d or a slice of it; x rows are the K-major A operand,
+// W_router [d, E] the MN-major B operand), then the lanes that finish a
+// token apply the same arg-max / runner-up / sigmoid rule as the CUDA-core
+// router above (details at the kernel).  Warp 0 lane 0 issues the TMA loads,
+// warp 1 lane 0 the MMAs; all four warps run the epilogue.
 namespace rmma {
 constexpr int A_BYTES = 128 * 128;     // 128 tokens x 64 K (bf16)
 constexpr int B_BOX_BYTES = 64 * 128;  // 64 K rows x 64 experts (bf16)
