@@ -29,42 +29,110 @@ __device__ __forceinline__ int warp_incl_scan(int v) {
     return v;
 }
 
-// Warp 0 writes one table from candidate groups [0, G): candidate g has
-// rows(g), row0(g), expert(g), feature blocks fb(g).  Empty groups are left
-// out; heavy groups come first, each run in candidate order.
-template <typename RowsF, typename Row0F, typename ExpF, typename FbF>
-__device__ void build_table(GroupTable* tab, int G, RowsF rows_of, Row0F row0_of, ExpF exp_of,
-                            FbF fb_of) {
-    const int lane = threadIdx.x & 31;
-    int n_base = 0, t_base = 0;
-    for (int run = 0; run < 2; ++run) {  // 0: heavy groups, 1: light groups
-        for (int base = 0; base < G; base += 32) {
-            const int g = base + lane;
-            int rows = 0, tiles = 0;
-            if (g < G) {
-                rows = rows_of(g);
-                const bool in_run = (rows >= kHeavyRows) == (run == 0);
-                tiles = (rows > 0 && in_run) ? ((rows + kTokTile - 1) / kTokTile) * fb_of(g) : 0;
-            }
-            const int flag = tiles > 0 ? 1 : 0;
-            const int fi = warp_incl_scan(flag);
-            const int ti = warp_incl_scan(tiles);
-            if (flag) {
-                const int pos = n_base + fi - 1;
-                tab->rows[pos] = rows;
-                tab->row0[pos] = row0_of(g);
-                tab->expert[pos] = exp_of(g);
-                tab->tile_start[pos] = t_base + ti - tiles;
-            }
-            n_base += __shfl_sync(0xffffffffu, fi, 31);
-            t_base += __shfl_sync(0xffffffffu, ti, 31);
+// CTA-wide inclusive scan of N ints per thread, in thread order, and the
+// CTA's totals.  Every thread of the CTA calls it (it synchronises).
+template <int N>
+__device__ void cta_incl_scan(int (&v)[N], int (&total)[N]) {
+    __shared__ int sc[33 * N];  // warps' totals, their exclusive prefix, the CTA total
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, nw = blockDim.x >> 5;
+#pragma unroll
+    for (int j = 0; j < N; ++j) v[j] = warp_incl_scan(v[j]);
+    if (lane == 31)
+#pragma unroll
+        for (int j = 0; j < N; ++j) sc[warp * N + j] = v[j];
+    __syncthreads();
+    if (warp == 0) {
+#pragma unroll
+        for (int j = 0; j < N; ++j) {
+            const int t = lane < nw ? sc[lane * N + j] : 0;
+            const int it = warp_incl_scan(t);
+            if (lane < nw) sc[lane * N + j] = it - t;
+            if (lane == 31) sc[32 * N + j] = it;
         }
-        if (run == 0 && lane == 0) tab->heavy_tiles = t_base;
     }
-    if (lane == 0) {
-        tab->num_groups = n_base;
-        tab->total_tiles = t_base;
-        tab->tile_start[n_base] = t_base;
+    __syncthreads();
+#pragma unroll
+    for (int j = 0; j < N; ++j) {
+        v[j] += sc[warp * N + j];
+        total[j] = sc[32 * N + j];
+    }
+    __syncthreads();  // sc free for the next call
+}
+
+// Both work lists (gate/up and down) from candidate groups [0, G), by every
+// thread of the CTA: candidate g has rows(g), row0(g), expert(g), and
+// ceil(rows / kTokTile) * fb_gu(g) gate/up tiles, ceil(rows / kTokTile) *
+// fb_down down tiles (every fb >= 1).  Empty groups are left out; heavy
+// groups (rows >= kHeavyRows) come first, each run in candidate order, so
+// both lists hold the same groups at the same positions.  A pass of
+// CTA-wide scans counts the heavy run; a second places every group.
+template <typename RowsF, typename Row0F, typename ExpF, typename FbF>
+__device__ void build_tables(GroupTable* tab_gu, GroupTable* tab_dn, int G, RowsF rows_of, Row0F row0_of,
+                             ExpF exp_of, FbF fb_gu_of, int fb_down) {
+    const int nt = blockDim.x;
+    int heavy[3] = {0, 0, 0};  // the heavy run's groups, gate/up tiles, down tiles
+    for (int base = 0; base < G; base += nt) {
+        const int g = base + threadIdx.x;
+        int v[3] = {0, 0, 0}, t[3];
+        if (g < G) {
+            const int rows = rows_of(g);
+            if (rows >= kHeavyRows) {
+                const int ntb = (rows + kTokTile - 1) / kTokTile;
+                v[0] = 1;
+                v[1] = ntb * fb_gu_of(g);
+                v[2] = ntb * fb_down;
+            }
+        }
+        cta_incl_scan<3>(v, t);
+#pragma unroll
+        for (int j = 0; j < 3; ++j) heavy[j] += t[j];
+    }
+    int carry[6] = {0, 0, 0, 0, 0, 0};  // groups, gate/up tiles, down tiles: heavy run, then light run
+    for (int base = 0; base < G; base += nt) {
+        const int g = base + threadIdx.x;
+        int rows = 0, tg = 0, td = 0;
+        bool hv = false;
+        if (g < G) {
+            rows = rows_of(g);
+            if (rows > 0) {
+                const int ntb = (rows + kTokTile - 1) / kTokTile;
+                tg = ntb * fb_gu_of(g);
+                td = ntb * fb_down;
+                hv = rows >= kHeavyRows;
+            }
+        }
+        const bool in = rows > 0;
+        int v[6] = {in && hv ? 1 : 0, in && hv ? tg : 0, in && hv ? td : 0,
+                    in && !hv ? 1 : 0, in && !hv ? tg : 0, in && !hv ? td : 0};
+        int t[6];
+        cta_incl_scan<6>(v, t);
+        if (in) {  // this group's run: selects, not an index (keeps the arrays in registers)
+            const int pos = (hv ? carry[0] + v[0] : heavy[0] + carry[3] + v[3]) - 1;
+            const int sg = (hv ? carry[1] + v[1] : heavy[1] + carry[4] + v[4]) - tg;
+            const int sd = (hv ? carry[2] + v[2] : heavy[2] + carry[5] + v[5]) - td;
+            const int r0 = row0_of(g), ex = exp_of(g);
+            tab_gu->rows[pos] = rows;
+            tab_gu->row0[pos] = r0;
+            tab_gu->expert[pos] = ex;
+            tab_gu->tile_start[pos] = sg;
+            tab_dn->rows[pos] = rows;
+            tab_dn->row0[pos] = r0;
+            tab_dn->expert[pos] = ex;
+            tab_dn->tile_start[pos] = sd;
+        }
+#pragma unroll
+        for (int j = 0; j < 6; ++j) carry[j] += t[j];
+    }
+    if (threadIdx.x == 0) {
+        const int n = carry[0] + carry[3];
+        tab_gu->num_groups = n;
+        tab_gu->heavy_tiles = carry[1];
+        tab_gu->total_tiles = carry[1] + carry[4];
+        tab_gu->tile_start[n] = carry[1] + carry[4];
+        tab_dn->num_groups = n;
+        tab_dn->heavy_tiles = carry[2];
+        tab_dn->total_tiles = carry[2] + carry[5];
+        tab_dn->tile_start[n] = carry[2] + carry[5];
     }
 }
 
@@ -245,17 +313,11 @@ __device__ void dispatch_finish(int32_t* chunk_base, int chunks, int T, int E, i
             }
         }
     }
-    if (warp == 0) {
-        // gate/up: candidate 0 is the shared expert, 1..E the routed experts
-        build_table(
-            tab_gu, E + 1, [&](int g) { return g == 0 ? T : tot[g - 1]; },
-            [&](int g) { return g == 0 ? 0 : soff[g - 1]; }, [&](int g) { return g == 0 ? E : g - 1; },
-            [&](int g) { return g == 0 ? fb_gu_shared : fb_gu_routed; });
-        build_table(
-            tab_dn, E + 1, [&](int g) { return g == 0 ? T : tot[g - 1]; },
-            [&](int g) { return g == 0 ? 0 : soff[g - 1]; }, [&](int g) { return g == 0 ? E : g - 1; },
-            [&](int) { return fb_down; });
-    }
+    // candidate 0 is the shared expert, 1..E the routed experts
+    build_tables(
+        tab_gu, tab_dn, E + 1, [&](int g) { return g == 0 ? T : tot[g - 1]; },
+        [&](int g) { return g == 0 ? 0 : soff[g - 1]; }, [&](int g) { return g == 0 ? E : g - 1; },
+        [&](int g) { return g == 0 ? fb_gu_shared : fb_gu_routed; }, fb_down);
 }
 
 // Work lists of a layer without experts: one group (the shared SwiGLU, as
@@ -430,18 +492,11 @@ __global__ void __launch_bounds__(1024) permute_kernel(const float* __restrict__
             perm[slot] = t;
         }
     }
-    if (warp == 0) {
-        // gate/up: candidate 0 is the shared expert, 1..E the routed experts
-        build_table(
-            tab_gu, E + 1, [&](int g) { return g == 0 ? T : running[g - 1]; },
-            [&](int g) { return g == 0 ? 0 : soff[g - 1]; },
-            [&](int g) { return g == 0 ? E : g - 1; },
-            [&](int g) { return g == 0 ? fb_gu_shared : fb_gu_routed; });
-        build_table(
-            tab_dn, E + 1, [&](int g) { return g == 0 ? T : running[g - 1]; },
-            [&](int g) { return g == 0 ? 0 : soff[g - 1]; },
-            [&](int g) { return g == 0 ? E : g - 1; }, [&](int) { return fb_down; });
-    }
+    // candidate 0 is the shared expert, 1..E the routed experts
+    build_tables(
+        tab_gu, tab_dn, E + 1, [&](int g) { return g == 0 ? T : running[g - 1]; },
+        [&](int g) { return g == 0 ? 0 : soff[g - 1]; }, [&](int g) { return g == 0 ? E : g - 1; },
+        [&](int g) { return g == 0 ? fb_gu_shared : fb_gu_routed; }, fb_down);
 }
 
 // Multi-CTA dispatch of a batch whose routing is already in idx[T * k]: CTA

@@ -328,17 +328,11 @@ __global__ void __launch_bounds__(kSmallThreads) route_small_kernel(
         perm[slot] = n;
         gslot[slot] = s_gate[n] * s_scale[n / nk];
     }
-    if (warp == 0) {
-        // gate/up: candidate 0 is the shared expert, 1..E the routed experts
-        build_table(
-            tab_gu, nE + 1, [&](int g) { return g == 0 ? nT : s_rows[g - 1]; },
-            [&](int g) { return g == 0 ? 0 : s_off[g - 1]; }, [&](int g) { return g == 0 ? nE : g - 1; },
-            [&](int g) { return g == 0 ? fb_gu_shared : fb_gu_routed; });
-        build_table(
-            tab_dn, nE + 1, [&](int g) { return g == 0 ? nT : s_rows[g - 1]; },
-            [&](int g) { return g == 0 ? 0 : s_off[g - 1]; }, [&](int g) { return g == 0 ? nE : g - 1; },
-            [&](int) { return fb_down; });
-    }
+    // candidate 0 is the shared expert, 1..E the routed experts
+    build_tables(
+        tab_gu, tab_dn, nE + 1, [&](int g) { return g == 0 ? nT : s_rows[g - 1]; },
+        [&](int g) { return g == 0 ? 0 : s_off[g - 1]; }, [&](int g) { return g == 0 ? nE : g - 1; },
+        [&](int g) { return g == 0 ? fb_gu_shared : fb_gu_routed; }, fb_down);
 
     // ---------------------------------------------- rows in expert order
     // xg[slot of n] = x[n / k] (16-byte vectors, converted for 8-bit weight

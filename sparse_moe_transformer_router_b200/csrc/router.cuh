@@ -208,8 +208,9 @@ constexpr int A_BYTES = 128 * 128;     // 128 tokens x 64 K (bf16)
 constexpr int B_BOX_BYTES = 64 * 128;  // 64 K rows x 64 experts (bf16)
 constexpr int MAX_B_BOXES = 4;         // E <= 256
 constexpr int MAX_STAGES = 6;
-// The largest dynamic shared memory a launch asks for (stages, barriers, slack).
-constexpr size_t SMEM_BYTES = 226 * 1024;
+// The largest dynamic shared memory a launch asks for (stages, barriers,
+// slack), leaving room for the kernel's static shared memory.
+constexpr size_t SMEM_BYTES = 224 * 1024;
 // A launch whose CTAs each take n_chunk experts needs stages of the token
 // tile plus ceil(n_chunk / 64) weight boxes only: fewer bytes, so that two
 // CTAs fit on an SM when the experts are few.
