@@ -320,10 +320,13 @@ L4MOE_API l4moe_status l4moe_get_plan(const l4moe_handle *h, l4moe_plan *plan);
  * For each selected slot l4moe_forward records a CUDA event before and
  * after the kernel(s) of that slot, on the caller's stream, so the durations
  * are those of the real launches in place (every event pair adds a little
- * to the step, so time only what is needed).  Kernel slots: 0 router,
- * 1 permute, 2 row copy, 3 gate/up GEMM (+ its split-K finish), 4 down GEMM
- * + finish, 5 hidden-row quantisation of the FP8 activation mode
- * (L4MOE_NUM_KERNELS).  l4moe_read_timing synchronises on the last recorded
+ * to the step, so time only what is needed).  Kernel slots: 0 router
+ * (with the dispatch when a top-1 tensor-core router finishes it; the
+ * whole routing for batches of up to 16 tokens), 1 permute (a separate
+ * dispatch launch, when there is one), 2 row copy, 3 gate/up GEMM (+ its
+ * split-K finish), 4 down GEMM + finish, 5 hidden-row quantisation of the
+ * FP8 activation mode (L4MOE_NUM_KERNELS); a slot with no launch in a
+ * forward records nothing.  l4moe_read_timing synchronises on the last recorded
  * event, adds every recorded pair to ms[slot] and launches[slot] (arrays of
  * at least L4MOE_NUM_KERNELS entries, accumulated into), and recycles the
  * events.  Returns L4MOE_ERR_CUDA if an event call fails. */
