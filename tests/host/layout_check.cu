@@ -5,7 +5,9 @@
 // segment is 256-byte aligned, in order and large enough for any batch of at
 // most the budgeted tokens -- in particular the fp32 partial planes of the
 // split-K plan a batch of T tokens gets -- and every k-range of a split keeps
-// at least 8 k-blocks.  Prints "OK <cases>" or the first violation.
+// at least 8 k-blocks; the tensor-core router's stages, slice exchange and
+// dispatch staging fit its shared memory.  Prints "OK <cases>" or the first
+// violation.
 #include <cstdio>
 #include <random>
 
@@ -120,6 +122,31 @@ int main() {
                     if (!check(p, Tmax, 1, 148, true)) return 1;
                     ++cases;
                 }
+            }
+    // the tensor-core router's shared memory, for every E it takes (E % 8 == 0,
+    // up to 256; a launch's CTA takes all E experts, or 16 in the expert-split
+    // form): its stages fit the limit it asks for, and the slice exchange
+    // (128 token rows of n_pad + 4 floats) and the ranks' counts (4 rows of E
+    // ints) fit its stage memory
+    for (int E = 8; E <= 256; E += 8) {
+        const int nst = rmma::stages(E);
+        const size_t stage_mem = (size_t)nst * rmma::stage_bytes(E);
+        const size_t recv = 4 * 128 * (size_t)(((E + 15) & ~15) + 4);
+        if (nst < 4 || nst > rmma::MAX_STAGES || rmma::smem_bytes(E, nst) > rmma::SMEM_BYTES ||
+            recv + 16 * (size_t)E > stage_mem || router_stage_cap(E) < 1) {
+            printf("BAD router shared memory: E %d stages %d\n", E, nst);
+            return 1;
+        }
+        ++cases;
+    }
+    // the workloads' top-1 bf16 routers at large batches finish the dispatch
+    // themselves: every chunk's counts fit the last CTA's staging
+    for (int E : {16, 128})
+        for (int T : {17, 4096, 8192, 16384, 65536})
+            if (router_max_chunks(T) > (size_t)router_stage_cap(E)) {
+                printf("BAD router dispatch staging: E %d T %d chunks %zu cap %d\n", E, T, router_max_chunks(T),
+                       router_stage_cap(E));
+                return 1;
             }
     printf("OK %d\n", cases);
     return 0;
