@@ -172,7 +172,8 @@ __device__ int chunk_rank(int e, int E, int* wcnt, int32_t* __restrict__ chunk_r
 // thread's loads of a pass issued before any is stored (one L2 round trip
 // per pass, not per element); tpe consecutive threads scan one expert, each
 // a run of consecutive chunks, joined by a segmented shuffle scan; warp 0
-// then scans over the experts and writes the lists.
+// then scans over the experts, and the whole CTA writes the lists
+// (build_tables).
 // smem: tot[E], soff[E + 1] and stage[cap] ints, cap >= chunks, stage and
 // chunk_base 16-byte aligned.  U: 4-byte loads in flight per thread (2U
 // 16-byte ones): more for a small CTA, fewer where registers are scarce.
