@@ -206,7 +206,6 @@ __global__ void __launch_bounds__(NT) router_kernel(const ET* __restrict__ x,
 namespace rmma {
 constexpr int A_BYTES = 128 * 128;     // 128 tokens x 64 K (bf16)
 constexpr int B_BOX_BYTES = 64 * 128;  // 64 K rows x 64 experts (bf16)
-constexpr int MAX_B_BOXES = 4;         // E <= 256
 constexpr int MAX_STAGES = 6;
 // The largest dynamic shared memory a launch asks for (stages, barriers,
 // slack), leaving room for the kernel's static shared memory.
